@@ -1,0 +1,228 @@
+"""CPU oracle for the MoE top-k gate / layout / dispatch / combine path.
+
+TEST INFRASTRUCTURE ONLY.  The tests, the package's ``smoke()`` check and the
+benchmark's CPU-baseline leg are the only callers.  The product library never
+imports this package and this package never imports the product: the two share
+no code.  The arithmetic lives in ``moe_oracle.c`` (plain single-threaded C,
+built with ``-O2 -ffp-contract=off``); this module only marshals numpy arrays.
+
+Arrays: bf16 data is carried as ``numpy.uint16`` bit patterns, FP8 e4m3 as
+``numpy.uint8`` codes, indices as ``int32``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+GATE_SOFTMAX = 0
+GATE_SOFTMAX_RENORM = 1
+GATE_SIGMOID_GROUP = 2
+DT_BF16 = 0
+DT_FP8_E4M3 = 1
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_BAD_INDEX = 4
+
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+          "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source (gcc, plain C)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The oracle library.  ``MOE_ORACLE_LIB`` may name another build of the same
+    source (the mutation test loads deliberately broken copies this way)."""
+    global _lib
+    if _lib is None:
+        path = os.environ.get("MOE_ORACLE_LIB") or build()
+        _lib = ctypes.CDLL(path)
+        _declare(_lib)
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SZ = ctypes.c_size_t
+
+
+def _declare(L):
+    L.oracle_dexp.argtypes = [ctypes.c_float]
+    L.oracle_dexp.restype = ctypes.c_float
+    L.oracle_sigmoid.argtypes = [ctypes.c_float]
+    L.oracle_sigmoid.restype = ctypes.c_float
+    L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+    L.oracle_e4m3_encode.restype = ctypes.c_uint8
+    L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e4m3_decode.restype = ctypes.c_float
+    L.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
+    L.oracle_bf16_from_f32.restype = ctypes.c_uint16
+    L.oracle_f32_from_bf16.argtypes = [ctypes.c_uint16]
+    L.oracle_f32_from_bf16.restype = ctypes.c_float
+    for name in ("oracle_e4m3_encode_array", "oracle_dexp_array", "oracle_sigmoid_array"):
+        getattr(L, name).argtypes = [_P, _P, _SZ]
+        getattr(L, name).restype = None
+    L.oracle_topk_gate.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
+    L.oracle_topk_gate.restype = _I
+    L.oracle_get_layout.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
+    L.oracle_get_layout.restype = _I
+    L.oracle_dispatch.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
+    L.oracle_dispatch.restype = _I
+    L.oracle_combine.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+    L.oracle_combine.restype = _I
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---------------------------------------------------------------- scalars
+def dexp(y: float) -> float:
+    return lib().oracle_dexp(y)
+
+
+def sigmoid(x: float) -> float:
+    return lib().oracle_sigmoid(x)
+
+
+def e4m3_encode(f: float) -> int:
+    return lib().oracle_e4m3_encode(f)
+
+
+def e4m3_decode(c: int) -> float:
+    return lib().oracle_e4m3_decode(c)
+
+
+def bf16_from_f32(f: float) -> int:
+    return lib().oracle_bf16_from_f32(f)
+
+
+def f32_from_bf16(h: int) -> float:
+    return lib().oracle_f32_from_bf16(h)
+
+
+# ---------------------------------------------------------------- arrays
+def e4m3_encode_array(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    lib().oracle_e4m3_encode_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def dexp_array(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.float32)
+    lib().oracle_dexp_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def sigmoid_array(x: np.ndarray) -> np.ndarray:
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.float32)
+    lib().oracle_sigmoid_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def bf16_to_f32(h: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns (uint16) to float32."""
+    h = np.asarray(h, np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+# ---------------------------------------------------------------- steps
+def topk_gate(logits: np.ndarray, k: int, kind: int, n_groups: int = 1,
+              topk_groups: int = 1, group_topn: int = 1):
+    logits = _c(logits, np.float32)
+    N, E = logits.shape
+    idx = np.empty((N, k), np.int32)
+    w = np.empty((N, k), np.float32)
+    st = lib().oracle_topk_gate(_ptr(logits), N, E, k, kind, n_groups, topk_groups,
+                                group_topn, _ptr(idx), _ptr(w))
+    if st != OK:
+        raise ValueError(f"oracle_topk_gate status {st}")
+    return idx, w
+
+
+@dataclass
+class Layout:
+    expert_count: np.ndarray
+    expert_offset: np.ndarray
+    rank_count: np.ndarray
+    rank_offset: np.ndarray
+    rank_tokens: np.ndarray
+    token_slot: np.ndarray
+    slot_token: np.ndarray
+    status: int
+
+
+def get_layout(topk_idx: np.ndarray, E: int, R: int) -> Layout:
+    topk_idx = _c(topk_idx, np.int32)
+    N, k = topk_idx.shape
+    L = Layout(np.empty(E, np.int32), np.empty(E + 1, np.int32), np.empty(R, np.int32),
+               np.empty(R + 1, np.int32), np.empty(R, np.int32), np.empty((N, k), np.int32),
+               np.empty(N * k, np.int32), OK)
+    st = lib().oracle_get_layout(_ptr(topk_idx), N, k, E, R, _ptr(L.expert_count),
+                                 _ptr(L.expert_offset), _ptr(L.rank_count), _ptr(L.rank_offset),
+                                 _ptr(L.rank_tokens), _ptr(L.token_slot), _ptr(L.slot_token))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_get_layout: invalid argument")
+    L.status = st
+    return L
+
+
+def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
+             recv_rows: int | None = None):
+    """Returns (recv_x, recv_scale or None, status).  Rows no slot names stay 0."""
+    x_bf16 = _c(x_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    N, H = x_bf16.shape
+    k = token_slot.shape[1]
+    S = N * k if recv_rows is None else recv_rows
+    if dtype == DT_BF16:
+        recv = np.zeros((S, H), np.uint16)
+        scale = None
+        sp = None
+    else:
+        recv = np.zeros((S, H), np.uint8)
+        scale = np.zeros((S, H // 128), np.float32)
+        sp = _ptr(scale)
+    st = lib().oracle_dispatch(_ptr(x_bf16), N, H, k, _ptr(token_slot), dtype, _ptr(recv), sp)
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_dispatch: invalid argument")
+    return recv, scale, st
+
+
+def combine(y_bf16: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray):
+    """Returns (out bf16 bits [N,H], status)."""
+    y_bf16 = _c(y_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    N, k = token_slot.shape
+    H = y_bf16.shape[1]
+    out = np.empty((N, H), np.uint16)
+    st = lib().oracle_combine(_ptr(y_bf16), N, H, k, _ptr(token_slot), _ptr(topk_w), _ptr(out))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_combine: invalid argument")
+    return out, st

@@ -1,0 +1,473 @@
+/*
+ * moe_oracle.c -- plain, slow, single-threaded CPU oracle for the MoE
+ * routing hot path: top-k gate -> layout -> dispatch -> combine.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the checker the CUDA library is
+ * compared against.  Only the tests, the package's smoke check and the
+ * benchmark's CPU-baseline leg may load it.  It shares no source, header,
+ * table or constant generator with the CUDA library, and the CUDA library
+ * never calls it.
+ *
+ * Every routine states the definition it follows.  The pages cited are:
+ *   [pplx]   "Efficient and portable mixture-of-experts communication"
+ *            (Perplexity Research blog), sections Introduction, Dispatch,
+ *            Combine.
+ *   [EPv2]   "DeepSeek releases the open-source DeepEP library for MoE
+ *            training and inference" (hi.news.hada.io summary of DeepEP V2),
+ *            section "training / prefill / decoding usage patterns".
+ *   [EPv1]   "DeepSeek, DeepEP 오픈소스 공개" (GeekNews), sections
+ *            "Topic Body" and "성능 / 일반 커널" (normal kernels).
+ *   [TK]     "DeepSeek Tile-Kernels / DeepEP V2" (deepinsightai.io), list
+ *            "Funktionen der DeepSeek-Tile-Kernel".
+ * Where the pages leave a rule open, the reading taken is written beside it.
+ *
+ * Arithmetic: fp32 with explicit rounding steps (compile with
+ * -ffp-contract=off so no multiply-add is fused behind our back).  The pages
+ * fix fp32 accumulation for combine and BF16 storage; gate selections and
+ * FP8 codes are integers decided by floating point, so they are decided in
+ * the kernels' precision (fp32) with one exp written out from its
+ * definition below.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_OK 0
+#define ORC_ERR_INVALID_ARG 1
+#define ORC_ERR_BAD_INDEX 4
+
+#define GATE_SOFTMAX 0
+#define GATE_SOFTMAX_RENORM 1
+#define GATE_SIGMOID_GROUP 2
+
+#define DT_BF16 0
+#define DT_FP8_E4M3 1
+
+/* ------------------------------------------------------------------ */
+/* bit helpers                                                         */
+/* ------------------------------------------------------------------ */
+static uint32_t f32_bits(float f) { uint32_t u; memcpy(&u, &f, 4); return u; }
+static float bits_f32(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+
+/* bfloat16 -> fp32 is exact: the bf16 pattern is the top half of the fp32. */
+float oracle_f32_from_bf16(uint16_t h) { return bits_f32(((uint32_t)h) << 16); }
+
+/* fp32 -> bfloat16, round to nearest, ties to even (IEEE 754 default
+ * rounding applied to an 8-bit significand).  NaN stays a quiet NaN. */
+uint16_t oracle_bf16_from_f32(float f)
+{
+    uint32_t u = f32_bits(f);
+    if (isnan(f)) return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t lower = u & 0xFFFFu;
+    uint32_t upper = u >> 16;
+    /* exactly representable, below half, half (tie), above half */
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+/* ------------------------------------------------------------------ */
+/* exp written out from its definition (Cody & Waite argument reduction,
+ * Taylor series).  e^y = 2^n * e^r with n = nearest integer to y/ln2 and
+ * r = y - n*ln2, |r| <= ln2/2; e^r = sum_{i=0..7} r^i / i! by Horner.
+ * ln2 is split into a head with 16 significant bits (so n*head is exact for
+ * |n| < 256) and a tail; both terms are removed with one fused multiply-add
+ * each.  The input is clamped to [-87, 88] so that 2^n stays a normal
+ * float: below -87 the result saturates at about e^-87.
+ * The constants are the mathematical ones rounded to fp32:
+ *   log2(e), ln2 head = floor(ln2 * 2^16) / 2^16, ln2 tail = ln2 - head,
+ *   1/i! for i = 2..7.                                                  */
+/* ------------------------------------------------------------------ */
+float oracle_dexp(float y)
+{
+    const float log2e = 1.44269504088896340736f;
+    const float ln2_head = 45426.0f / 65536.0f; /* 0.693145751953125 */
+    const float ln2_tail = 1.42860682030941723212e-6f;
+    const float c2 = 1.0f / 2.0f, c3 = 1.0f / 6.0f, c4 = 1.0f / 24.0f;
+    const float c5 = 1.0f / 120.0f, c6 = 1.0f / 720.0f, c7 = 1.0f / 5040.0f;
+
+    if (y < -87.0f) y = -87.0f;
+    if (y > 88.0f) y = 88.0f;
+    float t = y * log2e;        /* one fp32 rounding */
+    float n = rintf(t);         /* nearest integer, ties to even */
+    float r = fmaf(-n, ln2_head, y);
+    r = fmaf(-n, ln2_tail, r);
+    float p = c7;
+    p = fmaf(p, r, c6);
+    p = fmaf(p, r, c5);
+    p = fmaf(p, r, c4);
+    p = fmaf(p, r, c3);
+    p = fmaf(p, r, c2);
+    p = fmaf(p, r, 1.0f);
+    p = fmaf(p, r, 1.0f);
+    int ni = (int)n;            /* in [-126, 127] */
+    float two_n = bits_f32((uint32_t)(ni + 127) << 23);
+    return p * two_n;           /* one fp32 rounding */
+}
+
+/* logistic sigmoid 1 / (1 + e^-x), each operation rounded once in fp32 */
+float oracle_sigmoid(float x)
+{
+    float e = oracle_dexp(-x);
+    float d = 1.0f + e;
+    return 1.0f / d;
+}
+
+/* ------------------------------------------------------------------ */
+/* FP8 E4M3 (OCP 8-bit floating point, "E4M3": 1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits; exponent field 0 holds the subnormals
+ * m * 2^-9; S.1111.111 is NaN; no infinities; largest finite 448 =
+ * S.1111.110).  Encoding rounds to nearest, ties to even mantissa, and
+ * saturates every finite value (and infinity) beyond 448 to +-448.       */
+/* ------------------------------------------------------------------ */
+float oracle_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return (float)(s ? -v : v);
+}
+
+uint8_t oracle_e4m3_encode(float f)
+{
+    uint8_t sign = (f32_bits(f) >> 31) ? 0x80 : 0x00;
+    if (isnan(f)) return sign | 0x7F;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;          /* saturate */
+    if (a < ldexp(1.0, -6)) {                    /* subnormal range */
+        double q = a * 512.0;                    /* in units of 2^-9, exact */
+        double m = nearbyint(q);                 /* ties to even */
+        return sign | (uint8_t)m;                /* m == 8 is the code of 2^-6 */
+    }
+    int ex;
+    frexp(a, &ex);                               /* a = fr * 2^ex, fr in [0.5,1) */
+    int unb = ex - 1;                            /* a in [2^unb, 2^(unb+1)) */
+    double q = (ldexp(a, -unb) - 1.0) * 8.0;     /* mantissa in eighths, exact */
+    double m = nearbyint(q);                     /* ties to even */
+    int biased = unb + 7;
+    if (m == 8.0) { m = 0.0; biased += 1; }
+    if (biased > 15 || (biased == 15 && m == 7.0)) return sign | 0x7E;
+    return sign | (uint8_t)((biased << 3) | (int)m);
+}
+
+void oracle_e4m3_encode_array(const float* in, uint8_t* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(in[i]);
+}
+
+void oracle_dexp_array(const float* in, float* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_dexp(in[i]);
+}
+
+void oracle_sigmoid_array(const float* in, float* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = oracle_sigmoid(in[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* top-k selection: k passes of arg-max over the candidates.  Order is by
+ * key descending; equal keys go to the lower index (the reading taken for
+ * ties).  -0.0 and +0.0 compare equal.  Output is in selection order.    */
+/* ------------------------------------------------------------------ */
+static int better(float va, int ia, float vb, int ib)
+{
+    return va > vb || (va == vb && ia < ib);
+}
+
+static void select_topk(const float* key, const unsigned char* cand, int n,
+                        int k, int* sel)
+{
+    unsigned char* taken = (unsigned char*)calloc((size_t)n, 1);
+    for (int j = 0; j < k; ++j) {
+        int best = -1;
+        for (int i = 0; i < n; ++i) {
+            if (!cand[i] || taken[i]) continue;
+            if (best < 0 || better(key[i], i, key[best], best)) best = i;
+        }
+        sel[j] = best;
+        if (best >= 0) taken[best] = 1;
+    }
+    free(taken);
+}
+
+/* ------------------------------------------------------------------ */
+/* Gate.  [pplx] Introduction: the router turns the logits into a
+ * probability distribution, the top-K experts are picked and the output is
+ * the average of their outputs weighted by the router's probabilities.
+ * [TK] list, "Gating" and "MoE-Routing ... Gewichtsnormalisierung": top-k
+ * selection and scoring, with weight normalisation.
+ *
+ *  GATE_SOFTMAX:         p = softmax(logits); w_j = p_{sel j}.
+ *  GATE_SOFTMAX_RENORM:  w_j = p_{sel j} / sum_{j'} p_{sel j'}.
+ *  GATE_SIGMOID_GROUP:   DeepSeek-V3 group-limited gating, which [EPv1]
+ *     Topic Body names and whose run uses top-4 groups and top-8 experts
+ *     ([EPv1] normal kernels).  Reading taken: s = sigmoid(logit); the
+ *     experts split into n_groups consecutive groups; a group's score is
+ *     the sum of its group_topn largest s (added in descending order);
+ *     the topk_groups best groups are kept; the top-k experts by s among
+ *     the kept groups are chosen; w_j = s_{sel j} / sum_{j'} s_{sel j'}.
+ *
+ *  softmax: m = max logit; e_i = exp(l_i - m); Z = sum of e_i in ascending
+ *  expert order; p_i = e_i / Z.  Softmax is strictly increasing, so the
+ *  top-k of p is the top-k of the logits: selection uses the logits.
+ *  Every sum over selected experts runs in slot order (selection order).
+ */
+/* ------------------------------------------------------------------ */
+int oracle_topk_gate(const float* logits, int N, int E, int k, int kind,
+                     int n_groups, int topk_groups, int group_topn,
+                     int32_t* topk_idx, float* topk_w)
+{
+    if (N < 0 || E < 1 || k < 1 || k > E) return ORC_ERR_INVALID_ARG;
+    if (kind == GATE_SIGMOID_GROUP) {
+        if (n_groups < 1 || E % n_groups != 0) return ORC_ERR_INVALID_ARG;
+        int eg = E / n_groups;
+        if (topk_groups < 1 || topk_groups > n_groups) return ORC_ERR_INVALID_ARG;
+        if (group_topn < 1 || group_topn > eg) return ORC_ERR_INVALID_ARG;
+        if (topk_groups * eg < k) return ORC_ERR_INVALID_ARG;
+    } else if (kind != GATE_SOFTMAX && kind != GATE_SOFTMAX_RENORM) {
+        return ORC_ERR_INVALID_ARG;
+    }
+    float* key = (float*)malloc(sizeof(float) * (size_t)E);
+    float* val = (float*)malloc(sizeof(float) * (size_t)E);
+    unsigned char* cand = (unsigned char*)malloc((size_t)E);
+    int* sel = (int*)malloc(sizeof(int) * (size_t)E);
+    float* gscore = (float*)malloc(sizeof(float) * (size_t)(n_groups > 0 ? n_groups : 1));
+    unsigned char* gcand = (unsigned char*)malloc((size_t)(n_groups > 0 ? n_groups : 1));
+    int* gsel = (int*)malloc(sizeof(int) * (size_t)(n_groups > 0 ? n_groups : 1));
+
+    for (int t = 0; t < N; ++t) {
+        const float* l = logits + (size_t)t * E;
+        int32_t* oi = topk_idx + (size_t)t * k;
+        float* ow = topk_w + (size_t)t * k;
+        if (kind == GATE_SOFTMAX || kind == GATE_SOFTMAX_RENORM) {
+            float m = l[0];
+            for (int i = 1; i < E; ++i) if (l[i] > m) m = l[i];
+            float z = 0.0f;
+            for (int i = 0; i < E; ++i) {
+                val[i] = oracle_dexp(l[i] - m);
+                z = z + val[i];
+            }
+            for (int i = 0; i < E; ++i) { key[i] = l[i]; cand[i] = 1; }
+            select_topk(key, cand, E, k, sel);
+            float ps = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                float p = val[sel[j]] / z;
+                oi[j] = sel[j];
+                ow[j] = p;
+                ps = (j == 0) ? p : ps + p;
+            }
+            if (kind == GATE_SOFTMAX_RENORM)
+                for (int j = 0; j < k; ++j) ow[j] = ow[j] / ps;
+        } else {
+            int eg = E / n_groups;
+            for (int i = 0; i < E; ++i) val[i] = oracle_sigmoid(l[i]);
+            for (int g = 0; g < n_groups; ++g) {
+                const float* gv = val + (size_t)g * eg;
+                for (int i = 0; i < eg; ++i) cand[i] = 1;
+                select_topk(gv, cand, eg, group_topn, gsel);
+                float sum = gv[gsel[0]];
+                for (int j = 1; j < group_topn; ++j) sum = sum + gv[gsel[j]];
+                gscore[g] = sum;
+                gcand[g] = 1;
+            }
+            select_topk(gscore, gcand, n_groups, topk_groups, gsel);
+            for (int i = 0; i < E; ++i) cand[i] = 0;
+            for (int j = 0; j < topk_groups; ++j)
+                for (int i = 0; i < eg; ++i) cand[(size_t)gsel[j] * eg + i] = 1;
+            select_topk(val, cand, E, k, sel);
+            float ss = val[sel[0]];
+            for (int j = 1; j < k; ++j) ss = ss + val[sel[j]];
+            for (int j = 0; j < k; ++j) {
+                oi[j] = sel[j];
+                ow[j] = val[sel[j]] / ss;
+            }
+        }
+    }
+    free(key); free(val); free(cand); free(sel);
+    free(gscore); free(gcand); free(gsel);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Layout.  [EPv2] usage patterns: the handle carries the routing metadata
+ * combine needs and the per-expert received-token counts that size the
+ * grouped GEMM.  [pplx] Dispatch: the receiver packs tokens into one
+ * contiguous per-expert buffer and keeps, per received row, the source
+ * token so that combine knows where each row goes back; the order on the
+ * pages is not fixed -- the reading taken is ascending token id (then
+ * top-k slot) inside each expert.  [pplx] Sharding: experts are sharded
+ * over EP ranks; rank r owns experts [r*E/R, (r+1)*E/R).
+ *
+ * Entries equal to -1 are masked slots (no expert); any other id outside
+ * [0, E) is skipped and reported as ORC_ERR_BAD_INDEX.  Skipped entries get
+ * token_slot = -1 and fill the tail rows [expert_offset[E], N*k) of the
+ * receive buffer, whose slot_token is -1.
+ *
+ * expert_count[e]   = #{(t,j) : idx[t,j] = e}
+ * expert_offset[e]  = sum_{e' < e} expert_count[e'],  e = 0..E
+ * token_slot[t,j]   = expert_offset[e] + #{(t',j') before (t,j) in
+ *                     row-major order with idx[t',j'] = e}
+ * slot_token[s]     = t for s = token_slot[t,j]; -1 for the tail rows
+ * rank_count[r]     = sum of expert_count over rank r's experts
+ * rank_offset[r]    = expert_offset[r*E/R], rank_offset[R] = expert_offset[E]
+ * rank_tokens[r]    = #{t : some j has idx[t,j] in rank r}            */
+/* ------------------------------------------------------------------ */
+int oracle_get_layout(const int32_t* topk_idx, int N, int k, int E, int R,
+                      int32_t* expert_count, int32_t* expert_offset,
+                      int32_t* rank_count, int32_t* rank_offset,
+                      int32_t* rank_tokens, int32_t* token_slot,
+                      int32_t* slot_token)
+{
+    if (N < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int epr = E / R;
+    int64_t S = (int64_t)N * k;
+    for (int e = 0; e < E; ++e) expert_count[e] = 0;
+    for (int64_t i = 0; i < S; ++i) {
+        int32_t e = topk_idx[i];
+        if (e >= 0 && e < E) expert_count[e] += 1;
+        else if (e != -1) status = ORC_ERR_BAD_INDEX;
+    }
+    expert_offset[0] = 0;
+    for (int e = 0; e < E; ++e) expert_offset[e + 1] = expert_offset[e] + expert_count[e];
+
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    for (int e = 0; e < E; ++e) cursor[e] = expert_offset[e];
+    int64_t tail = expert_offset[E];
+    for (int t = 0; t < N; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t i = (int64_t)t * k + j;
+            int32_t e = topk_idx[i];
+            if (e >= 0 && e < E) {
+                int32_t s = cursor[e]++;
+                token_slot[i] = s;
+                slot_token[s] = t;
+            } else {
+                token_slot[i] = -1;
+                slot_token[tail++] = -1;
+            }
+        }
+    }
+    free(cursor);
+
+    for (int r = 0; r < R; ++r) {
+        int32_t c = 0;
+        for (int e = r * epr; e < (r + 1) * epr; ++e) c += expert_count[e];
+        rank_count[r] = c;
+        rank_offset[r] = expert_offset[r * epr];
+        rank_tokens[r] = 0;
+    }
+    rank_offset[R] = expert_offset[E];
+    for (int t = 0; t < N; ++t) {
+        for (int r = 0; r < R; ++r) {
+            int hit = 0;
+            for (int j = 0; j < k; ++j) {
+                int32_t e = topk_idx[(int64_t)t * k + j];
+                if (e >= 0 && e < E && e / epr == r) hit = 1;
+            }
+            rank_tokens[r] += hit;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Dispatch.  [pplx] Dispatch: each token's activations (with block scaling
+ * factors when quantised) are sent to every expert it was routed to and
+ * unpacked into one contiguous buffer per expert.  [EPv2] usage patterns:
+ * BF16 and FP8 inputs.  [TK] list, "Quantisierung ... pro Block".
+ *
+ * BF16: recv_x[token_slot[t,j], :] = x[t, :] for every valid slot.
+ * FP8, per token t and block b of 128 channels (reading taken for the
+ * block size and format: e4m3 with one fp32 scale per 128 channels):
+ *   amax  = max_c |x[t,c]|                       (exact)
+ *   inv   = 448 / amax,  scale = amax / 448      (IEEE fp32 divisions)
+ *   q_c   = e4m3(x[t,c] * inv)  (fp32 product, RNE, saturating);
+ *           an element equal to zero encodes as zero with its sign, which
+ *           is what the product gives whenever inv is finite and defines
+ *           the all-zero block (amax = 0, scale = 0).
+ * The same codes and scale go to every slot of the token.
+ * A slot outside [-1, N*k) is skipped and reported.                    */
+/* ------------------------------------------------------------------ */
+int oracle_dispatch(const uint16_t* x, int N, int H, int k,
+                    const int32_t* token_slot, int dtype, void* recv_x,
+                    float* recv_scale)
+{
+    if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_FP8_E4M3 && H % 128 != 0) return ORC_ERR_INVALID_ARG;
+    if (dtype != DT_BF16 && dtype != DT_FP8_E4M3) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int64_t S = (int64_t)N * k;
+    int nb = H / 128;
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* sc = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));
+    for (int t = 0; t < N; ++t) {
+        const uint16_t* xr = x + (size_t)t * H;
+        if (dtype == DT_FP8_E4M3) {
+            for (int b = 0; b < nb; ++b) {
+                float amax = 0.0f;
+                for (int c = b * 128; c < (b + 1) * 128; ++c) {
+                    float v = fabsf(oracle_f32_from_bf16(xr[c]));
+                    if (v > amax) amax = v;
+                }
+                float inv = 448.0f / amax;
+                sc[b] = amax / 448.0f;
+                for (int c = b * 128; c < (b + 1) * 128; ++c) {
+                    float v = oracle_f32_from_bf16(xr[c]);
+                    float p = (v == 0.0f) ? v : v * inv;
+                    q[c] = oracle_e4m3_encode(p);
+                }
+            }
+        }
+        for (int j = 0; j < k; ++j) {
+            int32_t s = token_slot[(int64_t)t * k + j];
+            if (s == -1) continue;
+            if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }
+            if (dtype == DT_BF16) {
+                uint16_t* dst = (uint16_t*)recv_x + (size_t)s * H;
+                for (int c = 0; c < H; ++c) dst[c] = xr[c];
+            } else {
+                uint8_t* dst = (uint8_t*)recv_x + (size_t)s * H;
+                for (int c = 0; c < H; ++c) dst[c] = q[c];
+                for (int b = 0; b < nb; ++b) recv_scale[(size_t)s * nb + b] = sc[b];
+            }
+        }
+    }
+    free(q); free(sc);
+    return status;
+}
+
+/* ------------------------------------------------------------------ */
+/* Combine.  [pplx] Introduction and Combine: the token's output is the
+ * average of its experts' outputs weighted by the router weights; [EPv2]
+ * usage patterns: combine reduces the expert outputs back to the token.
+ *   out[t,c] = bf16_rne( acc ),  acc = +0.0f, then for j = 0..k-1 in slot
+ *   order: acc = fma(w[t,j], y[token_slot[t,j], c], acc)   (fp32)
+ * Masked slots (-1) contribute nothing; other out-of-range slots are
+ * skipped and reported.                                                */
+/* ------------------------------------------------------------------ */
+int oracle_combine(const uint16_t* y, int N, int H, int k,
+                   const int32_t* token_slot, const float* topk_w,
+                   uint16_t* out)
+{
+    if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int64_t S = (int64_t)N * k;
+    for (int t = 0; t < N; ++t) {
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int32_t s = token_slot[(int64_t)t * k + j];
+                if (s == -1) continue;
+                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }
+                float v = oracle_f32_from_bf16(y[(size_t)s * H + c]);
+                acc = fmaf(topk_w[(int64_t)t * k + j], v, acc);
+            }
+            out[(size_t)t * H + c] = oracle_bf16_from_f32(acc);
+        }
+    }
+    return status;
+}

@@ -1,0 +1,54 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of ``oracle/moe_oracle.c`` (a dropped
+term, a wrong sign or index, transposed operands, another tie rule), builds it
+under a temporary directory and runs the pin suite against it; the suite must
+fail.  Everything runs on the CPU; the real oracle is untouched.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
+
+MUTANTS = {
+    "exp_drop_7th_taylor_term": ("float p = c7;", "float p = 0.0f;"),
+    "exp_drop_ln2_tail": ("r = fmaf(-n, ln2_tail, r);", "r = r + 0.0f;"),
+    "sigmoid_wrong_sign": ("float e = oracle_dexp(-x);", "float e = oracle_dexp(x);"),
+    "tie_to_higher_index": ("(va == vb && ia < ib)", "(va == vb && ia > ib)"),
+    "softmax_renorm_dropped": ("for (int j = 0; j < k; ++j) ow[j] = ow[j] / ps;", "(void)ps;"),
+    "group_score_drops_second": ("for (int j = 1; j < group_topn; ++j) sum = sum + gv[gsel[j]];", "(void)0;"),
+    "group_candidates_wrong_index": ("cand[(size_t)gsel[j] * eg + i] = 1;", "cand[(size_t)j * eg + i] = 1;"),
+    "layout_slot_token_stores_slot_index": ("slot_token[s] = t;", "slot_token[s] = j;"),
+    "layout_rank_offset_wrong_index": ("rank_offset[r] = expert_offset[r * epr];", "rank_offset[r] = expert_offset[r];"),
+    "layout_rank_tokens_modulo": ("if (e >= 0 && e < E && e / epr == r) hit = 1;", "if (e >= 0 && e < E && e % epr == r) hit = 1;"),
+    "fp8_scale_transposed": ("sc[b] = amax / 448.0f;", "sc[b] = 448.0f / amax;"),
+    "e4m3_ties_away": ("double m = nearbyint(q);                     /* ties to even */",
+                       "double m = floor(q + 0.5);"),
+    "e4m3_subnormal_step": ("double q = a * 512.0;", "double q = a * 256.0;"),
+    "bf16_ties_up": ("(lower == 0x8000u && (upper & 1u))", "(lower == 0x8000u)"),
+    "combine_weight_index_dropped": ("acc = fmaf(topk_w[(int64_t)t * k + j], v, acc);",
+                                     "acc = fmaf(topk_w[(int64_t)t * k], v, acc);"),
+    "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
+                                        "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    src = open(SRC).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    mut = tmp_path / "moe_oracle_mut.c"
+    mut.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mut.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
+                           "-shared", "-w", "-o", str(lib), str(mut), "-lm"])
+    env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"

@@ -1,0 +1,482 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test ties one oracle routine to a closed form, a library routine
+(torch's bf16 / float8 conversions, float64 exp, stable sorts), a brute-force
+search on tiny inputs, a hand-worked example under ``tests/golden/``, or an
+invariant of the definition.  No expected value here comes from the CUDA path.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _ulp_err(got, ref64):
+    ulp = np.spacing(np.abs(ref64).astype(np.float32)).astype(np.float64)
+    return np.abs(got.astype(np.float64) - ref64) / ulp
+
+
+# ----------------------------------------------------------------- exp
+def test_dexp_closed_forms():
+    assert O.dexp(0.0) == 1.0
+    for n in range(-20, 21):
+        # e^(n ln2) = 2^n: within one ulp of e^y for the fp32-rounded y = n ln2
+        y = np.float32(n * math.log(2))
+        ref = 2.0 ** n * math.exp(float(y) - n * math.log(2))
+        got = O.dexp(y)
+        assert abs(got - ref) <= np.spacing(np.float32(ref))
+        assert abs(got - 2.0 ** n) <= 2.0 ** n * 2e-6
+    assert abs(O.dexp(1.0) - math.e) <= np.spacing(np.float32(math.e))
+
+
+def test_dexp_vs_float64_exp_dense():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.uniform(-87, 88, 1_000_000).astype(np.float32),
+                        np.linspace(-1, 1, 200_001, dtype=np.float32),
+                        np.linspace(-87, -80, 50_001, dtype=np.float32)])
+    got = O.dexp_array(x)
+    err = _ulp_err(got, np.exp(x.astype(np.float64)))
+    assert err.max() <= 1.0, err.max()          # measured 0.90 ulp
+    assert err.mean() < 0.3
+
+
+def test_dexp_saturation_and_monotone():
+    assert O.dexp(-100.0) == O.dexp(-87.0)
+    assert O.dexp(100.0) == O.dexp(88.0)
+    x = np.sort(np.random.default_rng(2).uniform(-90, 90, 500_000).astype(np.float32))
+    assert (np.diff(O.dexp_array(x)) >= 0).all()
+
+
+def test_sigmoid_vs_float64():
+    assert O.sigmoid(0.0) == 0.5
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.normal(0, 3, 500_000), rng.uniform(-80, 80, 200_000)]).astype(np.float32)
+    got = O.sigmoid_array(x)
+    ref = 1.0 / (1.0 + np.exp(-x.astype(np.float64)))
+    assert _ulp_err(got, ref).max() <= 3.0
+    # s(x) + s(-x) = 1 to within rounding
+    assert np.abs(got + O.sigmoid_array(-x) - 1.0).max() < 2.5e-7
+
+
+# ----------------------------------------------------------------- bf16
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(4)
+    bits = rng.integers(0, 2**32, 400_000, dtype=np.uint64).astype(np.uint32)
+    # force exact ties and near-ties in the low half
+    bits[:1000] = (bits[:1000] & 0xFFFF0000) | 0x8000
+    bits[1000:2000] = (bits[1000:2000] & 0xFFFF0000) | 0x7FFF
+    bits[2000:3000] = (bits[2000:3000] & 0xFFFF0000) | 0x8001
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    lib = O.lib()
+    got = np.array([lib.oracle_bf16_from_f32(float(v)) for v in f[:60_000]], np.uint16)
+    ref = torch.from_numpy(f[:60_000].copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    # overflow rounds to infinity
+    assert O.bf16_from_f32(3.4028235e38) == 0x7F80
+    assert O.f32_from_bf16(0x3F80) == 1.0
+
+
+# ----------------------------------------------------------------- e4m3
+def test_e4m3_spec_points():
+    g = _gold("e4m3_ocp_points.json")
+    for p in g["points"]:
+        code = int(p["code"], 16)
+        v = O.e4m3_decode(code)
+        assert v == p["value"] and math.copysign(1, v) == math.copysign(1, p["value"]), p
+        assert O.e4m3_encode(p["value"]) == code, p
+    for c in g["nan_codes"]:
+        assert math.isnan(O.e4m3_decode(int(c, 16)))
+
+
+def _torch_e4m3_decode_table():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    return codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_decode_matches_torch_table():
+    table = _torch_e4m3_decode_table()
+    for c in range(256):
+        v = O.e4m3_decode(c)
+        if math.isnan(table[c]):
+            assert math.isnan(v)
+        else:
+            assert v == table[c], c
+
+
+def test_e4m3_encode_brute_force_nearest():
+    """Nearest code by exhaustive search over the 127 non-negative finite codes,
+    ties to the even code (even mantissa), saturation above 448."""
+    table = _torch_e4m3_decode_table()[:127]    # codes 0x00..0x7e, increasing
+    rng = np.random.default_rng(5)
+    mids = (table[:-1] + table[1:]) / 2.0
+    xs = np.concatenate([
+        table, mids, np.nextafter(mids.astype(np.float32), np.float32(0)),
+        np.nextafter(mids.astype(np.float32), np.float32(1e9)),
+        rng.uniform(0, 470, 20_000), np.exp2(rng.uniform(-14, 9, 20_000)),
+        [448.0, 463.9, 464.0, 464.1, 500.0, 1e30, np.inf, 2.0**-10, 2.0**-10 * 1.0001, 1e-30],
+    ]).astype(np.float32)
+    for sign in (1.0, -1.0):
+        x = (sign * xs).astype(np.float32)
+        got = O.e4m3_encode_array(x)
+        a = np.abs(x.astype(np.float64))
+        d = np.abs(a[:, None] - table[None, :])
+        best = d.min(axis=1, keepdims=True)
+        cand = d == best
+        codes = np.arange(127)
+        # tie -> even code
+        pick = np.where(cand.sum(1) > 1,
+                        np.array([codes[r][(codes[r] % 2) == 0][0] if r.sum() > 1 else -1 for r in cand]),
+                        cand.argmax(1))
+        pick = np.where(a >= 448.0, 0x7E, pick)
+        expect = pick.astype(np.uint8) | (np.uint8(0x80) if sign < 0 else np.uint8(0))
+        assert np.array_equal(got, expect), np.nonzero(got != expect)[0][:10]
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    rng = np.random.default_rng(6)
+    x = np.concatenate([rng.normal(0, 100, 300_000), rng.uniform(-448, 448, 100_000),
+                        np.exp2(rng.uniform(-12, 8.8, 100_000)) * rng.choice([-1, 1], 100_000)])
+    x = np.clip(x, -448, 448).astype(np.float32)
+    got = O.e4m3_encode_array(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+# ----------------------------------------------------------------- gate
+@pytest.mark.parametrize("case", _gold("gate_worked_examples.json")["cases"], ids=lambda c: c["name"])
+def test_gate_worked_examples(case):
+    logits = np.array(case["logits"], np.float32)
+    idx, w = O.topk_gate(logits, case["k"], case["kind"], case["n_groups"],
+                         case["topk_groups"], case["group_topn"])
+    assert idx.tolist() == case["idx"]
+    assert np.abs(w - np.array(case["w"])).max() <= case["tol"]
+
+
+def test_gate_softmax_vs_torch_float64():
+    rng = np.random.default_rng(7)
+    for E, k in [(8, 2), (16, 4), (64, 6), (256, 8)]:
+        logits = rng.normal(0, 2, (300, E)).astype(np.float32)
+        idx, w = O.topk_gate(logits, k, O.GATE_SOFTMAX)
+        ref = torch.softmax(torch.from_numpy(logits).double(), dim=1)
+        rv, ri = torch.topk(ref, k, dim=1)
+        assert np.array_equal(idx, ri.numpy())
+        assert np.abs(w - rv.numpy()).max() <= 4 * np.spacing(np.float32(1.0))
+        idx2, w2 = O.topk_gate(logits, k, O.GATE_SOFTMAX_RENORM)
+        assert np.array_equal(idx2, idx)
+        rn = (rv / rv.sum(1, keepdim=True)).numpy()
+        assert np.abs(w2 - rn).max() <= 4 * np.spacing(np.float32(1.0))
+        assert np.abs(w2.astype(np.float64).sum(1) - 1).max() <= k * 2.0**-23
+
+
+def test_gate_softmax_closed_form_two_experts():
+    rng = np.random.default_rng(8)
+    l = rng.normal(0, 3, (2000, 2)).astype(np.float32)
+    idx, w = O.topk_gate(l, 1, O.GATE_SOFTMAX)
+    d = np.abs(l[:, 0].astype(np.float64) - l[:, 1])
+    expect = 1.0 / (1.0 + np.exp(-d))
+    assert np.array_equal(idx[:, 0], np.where(l[:, 1] > l[:, 0], 1, 0))
+    assert np.abs(w[:, 0] - expect).max() < 4e-7
+
+
+def _group_limited_brute(s, G, TG, n, k):
+    """Exhaustive reference: every subset of TG groups; the kept set is the one
+    with the largest sum of group scores (float64), ties to the subset whose
+    sorted group ids are lexicographically smallest; experts by stable sort."""
+    E = s.shape[0]
+    eg = E // G
+    gs = []
+    for g in range(G):
+        v = np.sort(s[g * eg:(g + 1) * eg])[::-1][:n]
+        acc = np.float32(v[0])
+        for t in v[1:]:
+            acc = np.float32(acc + np.float32(t))
+        gs.append(float(acc))
+    best, best_key = None, None
+    for sub in itertools.combinations(range(G), TG):
+        key = (sum(gs[g] for g in sub), [-g for g in sub])
+        if best is None or key > best_key:
+            best, best_key = sub, key
+    cand = [e for g in best for e in range(g * eg, (g + 1) * eg)]
+    order = sorted(cand, key=lambda e: (-float(s[e]), e))
+    return order[:k], best
+
+
+def test_gate_group_limited_vs_brute_force():
+    rng = np.random.default_rng(9)
+    for (E, G, TG, n, k) in [(256, 8, 4, 2, 8), (64, 8, 3, 2, 6), (32, 4, 2, 1, 3), (48, 6, 2, 3, 5)]:
+        logits = rng.normal(0, 1, (120, E)).astype(np.float32)
+        idx, w = O.topk_gate(logits, k, O.GATE_SIGMOID_GROUP, G, TG, n)
+        s = O.sigmoid_array(logits)
+        for t in range(logits.shape[0]):
+            ref, groups = _group_limited_brute(s[t], G, TG, n, k)
+            assert idx[t].tolist() == ref, (E, t)
+            assert set(int(e) // (E // G) for e in idx[t]) <= set(groups)
+            sel = s[t][idx[t]].astype(np.float64)
+            assert np.abs(w[t] - sel / sel.sum()).max() <= 4 * 2.0**-24
+            assert (w[t] > 0).all()
+
+
+def test_gate_single_group_equals_plain_sigmoid_topk():
+    rng = np.random.default_rng(10)
+    logits = rng.normal(0, 1, (200, 64)).astype(np.float32)
+    idx, _ = O.topk_gate(logits, 8, O.GATE_SIGMOID_GROUP, 1, 1, 1)
+    s = torch.sigmoid(torch.from_numpy(logits).double())
+    _, ri = torch.topk(s, 8, dim=1)
+    assert np.array_equal(idx, ri.numpy())
+
+
+def test_gate_ties_go_to_lower_index():
+    logits = np.zeros((3, 16), np.float32)
+    logits[1, 5] = 1.0
+    logits[2] = -0.0
+    logits[2, ::2] = 0.0
+    idx, _ = O.topk_gate(logits, 4, O.GATE_SOFTMAX)
+    assert idx.tolist() == [[0, 1, 2, 3], [5, 0, 1, 2], [0, 1, 2, 3]]
+    idx, _ = O.topk_gate(logits, 4, O.GATE_SIGMOID_GROUP, 4, 2, 2)
+    assert idx.tolist()[0] == [0, 1, 2, 3]
+    # group 1 (holding expert 5) scores s(1)+s(0); groups 0, 2, 3 tie at 2 s(0) and the
+    # lower index (group 0) is kept: experts 5, then 0, 1, 2 by the index tie rule
+    assert idx.tolist()[1] == [5, 0, 1, 2]
+
+
+# ----------------------------------------------------------------- layout
+def test_layout_worked_example():
+    g = _gold("layout_worked_example.json")
+    L = O.get_layout(np.array(g["topk_idx"], np.int32), g["E"], g["R"])
+    for key in ("expert_count", "expert_offset", "rank_count", "rank_offset", "rank_tokens",
+                "token_slot", "slot_token"):
+        assert getattr(L, key).tolist() == g[key], key
+    assert L.status == O.OK
+
+
+def _layout_naive(idx, E, R):
+    N, k = idx.shape
+    flat = idx.reshape(-1)
+    counts = np.array([(flat == e).sum() for e in range(E)], np.int64)
+    off = np.concatenate([[0], np.cumsum(counts)])
+    token_slot = np.full(N * k, -1, np.int64)
+    slot_token = np.full(N * k, -1, np.int64)
+    for e in range(E):
+        pos = np.nonzero(flat == e)[0]          # ascending (token, slot)
+        token_slot[pos] = off[e] + np.arange(len(pos))
+        slot_token[off[e] + np.arange(len(pos))] = pos // k
+    epr = E // R
+    rank_of = np.where((flat >= 0) & (flat < E), flat // epr, -1).reshape(N, k)
+    rank_tokens = np.array([(rank_of == r).any(1).sum() for r in range(R)])
+    rank_count = counts.reshape(R, epr).sum(1)
+    return counts, off, token_slot.reshape(N, k), slot_token, rank_count, rank_tokens
+
+
+@pytest.mark.parametrize("N,k,E,R,mask", [(1, 1, 1, 1, 0.0), (37, 3, 16, 4, 0.0), (200, 8, 256, 32, 0.0),
+                                          (333, 2, 8, 8, 0.1), (64, 6, 12, 3, 0.3)])
+def test_layout_vs_naive(N, k, E, R, mask):
+    rng = np.random.default_rng(N * 7 + k)
+    idx = rng.integers(0, E, (N, k)).astype(np.int32)
+    idx[rng.random((N, k)) < mask] = -1
+    L = O.get_layout(idx, E, R)
+    counts, off, ts, st, rc, rt = _layout_naive(idx, E, R)
+    assert np.array_equal(L.expert_count, counts)
+    assert np.array_equal(L.expert_offset, off)
+    assert np.array_equal(L.token_slot, ts)
+    assert np.array_equal(L.slot_token, st)
+    assert np.array_equal(L.rank_count, rc)
+    assert np.array_equal(L.rank_tokens, rt)
+    assert np.array_equal(L.rank_offset, off[::E // R])
+    # invariants
+    valid = idx >= 0
+    assert L.expert_count.sum() == valid.sum() == L.expert_offset[E]
+    slots = L.token_slot[valid]
+    assert len(np.unique(slots)) == len(slots)                 # each (t,j) exactly once
+    assert (L.slot_token[slots] == np.nonzero(valid)[0]).all()  # inverse map
+    for e in range(E):                                          # ascending tokens per expert
+        seg = L.slot_token[L.expert_offset[e]:L.expert_offset[e + 1]]
+        assert (np.diff(seg) >= 0).all()
+    assert (L.rank_tokens <= np.minimum(N, L.rank_count)).all()
+    assert L.status == O.OK
+
+
+def test_layout_bad_index_is_skipped_and_reported():
+    idx = np.array([[0, 5], [-3, 1], [1, -1]], np.int32)
+    L = O.get_layout(idx, 4, 2)
+    assert L.status == O.ERR_BAD_INDEX
+    assert L.token_slot.tolist() == [[0, -1], [-1, 1], [2, -1]]
+    assert L.expert_count.tolist() == [1, 2, 0, 0]
+    assert L.slot_token.tolist() == [0, 1, 2, -1, -1, -1]
+
+
+# ----------------------------------------------------------------- dispatch
+def _bf16_bits(a):
+    return torch.from_numpy(np.asarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_dispatch_bf16_is_row_copy():
+    rng = np.random.default_rng(11)
+    N, H, E, k = 50, 136, 8, 3
+    x = _bf16_bits(rng.normal(size=(N, H)))
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(N)]).astype(np.int32)
+    L = O.get_layout(idx, E, 2)
+    recv, sc, st = O.dispatch(x, L.token_slot, O.DT_BF16)
+    assert st == O.OK and sc is None
+    assert np.array_equal(recv[L.token_slot.reshape(-1)], np.repeat(x, k, axis=0))
+    assert np.array_equal(recv[L.slot_token >= 0], x[L.slot_token[L.slot_token >= 0]])
+
+
+def test_dispatch_fp8_worked_example():
+    g = _gold("fp8_block_worked_example.json")
+    row = np.zeros(128, np.float32)
+    for c, v in g["nonzero"].items():
+        row[int(c)] = v
+    x = _bf16_bits(row[None, :])
+    recv, sc, st = O.dispatch(x, np.array([[0]], np.int32), O.DT_FP8_E4M3)
+    assert sc[0, 0] == np.float32(g["scale"])
+    for c, code in g["codes"].items():
+        assert recv[0, int(c)] == int(code, 16), c
+
+
+def test_dispatch_fp8_properties():
+    rng = np.random.default_rng(12)
+    N, H, k = 40, 512, 4
+    xf = rng.normal(size=(N, H)).astype(np.float32)
+    xf[3, 128:256] = 0.0                          # all-zero block
+    xf[4, :128] = -0.0
+    xf[5, 256:384] *= 1e-3
+    x = _bf16_bits(xf)
+    ts = np.arange(N * k, dtype=np.int32).reshape(N, k)
+    recv, sc, st = O.dispatch(x, ts, O.DT_FP8_E4M3)
+    xv = O.bf16_to_f32(x).astype(np.float32)
+    blocks = xv.reshape(N, H // 128, 128)
+    amax = np.abs(blocks).max(2)
+    # scale is the fp32 division amax/448
+    expect_scale = (amax.astype(np.float32) / np.float32(448)).astype(np.float32)
+    for j in range(k):
+        assert np.array_equal(sc[ts[:, j]], expect_scale)
+        assert np.array_equal(recv[ts[:, j]], recv[ts[:, 0]])    # same payload in every slot
+    q = recv[ts[:, 0]].reshape(N, H // 128, 128)
+    # codes match torch's RNE float8 conversion of x * (448/amax) (fp32 product)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        inv = (np.float32(448) / amax.astype(np.float32)).astype(np.float32)
+        prod = (blocks * inv[:, :, None]).astype(np.float32)
+    prod = np.where(blocks == 0, blocks, prod)
+    ref = torch.from_numpy(np.clip(prod, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(q, ref)
+    # the element at amax maps to +-448
+    am = np.abs(blocks).argmax(2)
+    top = np.take_along_axis(q, am[:, :, None], 2)[:, :, 0]
+    nz = amax > 0
+    assert ((top[nz] & 0x7F) == 0x7E).all()
+    # round trip within the e4m3 bound: half a mantissa step (2^-4 relative) or half the
+    # subnormal step (2^-10 * scale) in the scaled domain
+    deq = _torch_e4m3_decode_table()[q] * sc[ts[:, 0]].astype(np.float64)[:, :, None]
+    bound = np.maximum(2.0**-4 * np.abs(blocks), 2.0**-10 * sc[ts[:, 0]][:, :, None]) * (1 + 2.0**-20)
+    assert (np.abs(deq - blocks) <= bound).all()
+    # zero blocks: scale 0, signed-zero codes
+    assert sc[ts[3, 0], 1] == 0.0 and (q[3, 1] == 0).all()
+    assert (q[4, 0] == 0x80).all()
+
+
+def test_dispatch_fp8_tiny_amax_block():
+    """448/amax overflows fp32 for amax below ~1.3e-36: non-zero elements saturate,
+    zeros keep their sign, the scale is still amax/448."""
+    xf = np.zeros((1, 128), np.float32)
+    xf[0, 0] = 1e-37
+    xf[0, 1] = -5e-38
+    xf[0, 2] = -0.0
+    x = _bf16_bits(xf)
+    recv, sc, st = O.dispatch(x, np.array([[0]], np.int32), O.DT_FP8_E4M3)
+    amax = O.bf16_to_f32(x)[0, 0]
+    assert sc[0, 0] == np.float32(amax) / np.float32(448)
+    assert recv[0, 0] == 0x7E and recv[0, 1] == 0xFE and recv[0, 2] == 0x80 and recv[0, 3] == 0
+
+
+# ----------------------------------------------------------------- combine
+def test_combine_identity_experts_return_x():
+    rng = np.random.default_rng(13)
+    N, H, E, k = 300, 64, 8, 2
+    logits = rng.normal(size=(N, E)).astype(np.float32)
+    logits[:, 0] += 2.0
+    idx, w = O.topk_gate(logits, k, O.GATE_SOFTMAX_RENORM)
+    L = O.get_layout(idx, E, 8)
+    x = _bf16_bits(rng.normal(size=(N, H)))
+    recv, _, _ = O.dispatch(x, L.token_slot, O.DT_BF16)
+    out, st = O.combine(recv, L.token_slot, w)
+    assert np.array_equal(out, x)
+
+
+def test_combine_k1_unit_weight_is_gather():
+    rng = np.random.default_rng(14)
+    N, H = 64, 40
+    y = _bf16_bits(rng.normal(size=(N, H)))
+    slot = rng.permutation(N).astype(np.int32).reshape(N, 1)
+    out, _ = O.combine(y, slot, np.ones((N, 1), np.float32))
+    assert np.array_equal(out, y[slot[:, 0]])
+
+
+def test_combine_vs_float64_within_one_bf16_ulp():
+    rng = np.random.default_rng(15)
+    N, H, k = 120, 96, 8
+    y = _bf16_bits(rng.normal(size=(N * k, H)))
+    slot = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    w = rng.random((N, k)).astype(np.float32)
+    w /= w.sum(1, keepdims=True)
+    out, _ = O.combine(y, slot, w)
+    yv = O.bf16_to_f32(y).astype(np.float64)
+    ref = np.einsum("tk,tkh->th", w.astype(np.float64), yv[slot])
+    got = O.bf16_to_f32(out).astype(np.float64)
+    # |got - ref| <= half a bf16 ulp of ref + the fp32 chain error
+    tol = np.abs(ref) * 2.0**-8 + k * 2.0**-24 * np.abs(yv[slot]).max(1) + 1e-30
+    assert (np.abs(got - ref) <= tol).all()
+
+
+def test_combine_linear_in_weights_and_masked_slots():
+    rng = np.random.default_rng(16)
+    N, H, k = 30, 32, 4
+    y = _bf16_bits(rng.integers(-8, 8, size=(N * k, H)))      # small integers: exact sums
+    slot = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    w = rng.integers(0, 4, (N, k)).astype(np.float32)
+    out, _ = O.combine(y, slot, w)
+    yv = O.bf16_to_f32(y)
+    ref = np.einsum("tk,tkh->th", w, yv[slot])
+    assert np.array_equal(O.bf16_to_f32(out), ref.astype(np.float32))
+    slot2 = slot.copy()
+    slot2[:, 1] = -1
+    out2, st = O.combine(y, slot2, w)
+    w2 = w.copy()
+    w2[:, 1] = 0
+    assert np.array_equal(O.bf16_to_f32(out2), np.einsum("tk,tkh->th", w2, yv[slot]).astype(np.float32))
+    assert st == O.OK
+    slot2[0, 0] = N * k                                   # out of range: skipped, reported
+    _, st = O.combine(y, slot2, w)
+    assert st == O.ERR_BAD_INDEX
+
+
+def test_dispatch_combine_adjoint():
+    """<combine(y), g> = <y, w * dispatch(g)> (dispatch and combine are each
+    other's backward: DeepEP V2 summary, usage patterns)."""
+    rng = np.random.default_rng(17)
+    N, H, E, k = 80, 48, 16, 4
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(N)]).astype(np.int32)
+    w = rng.random((N, k)).astype(np.float32)
+    L = O.get_layout(idx, E, 4)
+    y = _bf16_bits(rng.normal(size=(N * k, H)))
+    g = _bf16_bits(rng.normal(size=(N, H)))
+    out, _ = O.combine(y, L.token_slot, w)
+    lhs = (O.bf16_to_f32(out).astype(np.float64) * O.bf16_to_f32(g)).sum()
+    dg, _, _ = O.dispatch(g, L.token_slot, O.DT_BF16)
+    wslot = np.zeros(N * k)
+    wslot[L.token_slot.reshape(-1)] = w.reshape(-1)
+    rhs = (O.bf16_to_f32(y).astype(np.float64) * O.bf16_to_f32(dg) * wslot[:, None]).sum()
+    assert abs(lhs - rhs) <= 2.0**-8 * np.abs(O.bf16_to_f32(out).astype(np.float64) * O.bf16_to_f32(g)).sum()
