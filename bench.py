@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE routing hot path (gate -> layout -> dispatch -> combine).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill] [--impl ours|reference]
+
+One step = one pass of the four steps over one batch of the workload, with
+inputs resident in HBM.  L2 is flushed (a write of twice its size) before every
+step, outside the timed events.  Each op is bracketed by CUDA events on the
+stream it runs on; ``value`` is whole-job tokens/s (all ranks' tokens over the
+slowest rank's summed step time).  ``e2e`` repeats the measurement through the
+same public API with pinned HOST inputs: the host->device copies of the step's
+inputs and the device->host copy of its output are inside the timed region.
+
+For N > 1 (torchrun, one process per GPU) every rank routes its own batch:
+the work shards by tokens with no data-path collective ("weak" scaling); NCCL
+is only used for the barrier and the max over ranks of the timed interval.
+
+``--impl reference`` times the plain single-threaded CPU oracle on a bounded
+sample of the same workload (rank 0 only), the comparison arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from combine_moe_topk_gate_b200.workloads import WORKLOADS, algorithmic_bytes, make_inputs  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and effective HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = {
+    "combine": "combine_moe_topk_gate_b200/csrc/combine.cu",
+    "dispatch": "combine_moe_topk_gate_b200/csrc/dispatch.cu",
+}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="prefill", choices=sorted(WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    return p.parse_args()
+
+
+def describe(w) -> str:
+    gate = {"softmax": "softmax", "softmax_renorm": "softmax renormalised",
+            "sigmoid_group": f"sigmoid group-limited ({w.n_groups} groups, top-{w.topk_groups} groups, "
+                             f"group score = top-{w.group_topn} sum)"}[w.gate]
+    return (f"{w.name}: N={w.N} tokens, H={w.H}, E={w.E} experts, top-{w.k}, {gate}, "
+            f"R={w.R} logical ranks, {w.dtype.upper()} dispatch, BF16 combine, "
+            f"expert outputs {'= dispatched rows' if w.expert_out == 'identity' else 'seeded bf16 N(0,1)'}")
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_hash(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(op: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel source changed since the capture (or there is none)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload][op]
+        if e.get("source_sha256_16") != source_hash(KERNEL_SOURCES[op]):
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of every rank's ``x`` (all ranks call this in the same order)."""
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(tokens_per_rank: int, world: int, steps: int, max_total_ms: float) -> float:
+    """Tokens of all ranks over the slowest rank's timed interval, per second."""
+    return tokens_per_rank * world * steps / (max_total_ms * 1e-3)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML (read-only) for SM clock and clock-event reasons while running."""
+    REASONS = {
+        "gpu_idle": "nvmlClocksEventReasonGpuIdle",
+        "applications_clocks_setting": "nvmlClocksEventReasonApplicationsClocksSetting",
+        "sw_power_cap": "nvmlClocksEventReasonSwPowerCap",
+        "hw_slowdown": "nvmlClocksEventReasonHwSlowdown",
+        "sync_boost": "nvmlClocksEventReasonSyncBoost",
+        "sw_thermal_slowdown": "nvmlClocksEventReasonSwThermalSlowdown",
+        "hw_thermal_slowdown": "nvmlClocksEventReasonHwThermalSlowdown",
+        "hw_power_brake_slowdown": "nvmlClocksEventReasonHwPowerBrakeSlowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self.ok = period_s, False
+        self._stop = threading.Event()
+        try:
+            import pynvml as N
+            self.N = N
+            N.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.h = None
+            for i in range(N.nvmlDeviceGetCount()):
+                h = N.nvmlDeviceGetHandleByIndex(i)
+                u = N.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self.h = h
+            if self.h is None:
+                self.h = N.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = N.nvmlDeviceGetMaxClockInfo(self.h, N.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        N = self.N
+        while not self._stop.is_set():
+            try:
+                self.samples.append(N.nvmlDeviceGetClockInfo(self.h, N.NVML_CLOCK_SM))
+                mask = N.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS.items():
+                    if mask & getattr(N, attr, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "")}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- reference arm
+def oracle_step(w, inp, n):
+    """One pass of the oracle over the first n tokens of the batch."""
+    import numpy as np
+    import oracle as O
+    logits = inp.logits[:n].numpy()
+    x = inp.x[:n].contiguous().view(torch.int16).numpy().view(np.uint16)
+    idx, wts = O.topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn)
+    L = O.get_layout(idx, w.E, w.R)
+    recv, _, _ = O.dispatch(x, L.token_slot, w.dtype_code)
+    if w.expert_out == "identity":
+        y = recv
+    else:
+        y = inp.y[: n * w.k].contiguous().view(torch.int16).numpy().view(np.uint16)
+    O.combine(y, L.token_slot, wts)
+
+
+def oracle_sample_size(w, inp, budget_s):
+    n0 = min(w.N, 32)
+    t = time.perf_counter()
+    oracle_step(w, inp, n0)
+    per_tok = (time.perf_counter() - t) / n0
+    return max(1, min(w.N, int(budget_s / per_tok))), per_tok
+
+
+def cpu_baseline(w, inp, budget_s):
+    n, _ = oracle_sample_size(w, inp, budget_s)
+    t = time.perf_counter()
+    oracle_step(w, inp, n)
+    dt = time.perf_counter() - t
+    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of the {w.N} tokens of the {w.name} batch (seed 0), gate+layout+"
+                      f"dispatch+combine, single-threaded C, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    w = WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    inp = make_inputs(w, 0)
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    n, per_tok = oracle_sample_size(w, inp, budget)
+    for _ in range(args.warmup):
+        oracle_step(w, inp, n)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, inp, n)
+    dt = time.perf_counter() - t
+    v = n * args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": {"workload": describe(w), "tokens_per_step": n},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"first {n} of {w.N} tokens per step, single-threaded C oracle"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args, rank, world, device):
+    from combine_moe_topk_gate_b200 import api
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, rank)
+    stream = torch.cuda.current_stream(device)
+    logits = inp.logits.to(device)
+    x = inp.x.to(device)
+    y_in = inp.y.to(device) if inp.y is not None else None
+    idx = torch.empty((w.N, w.k), dtype=torch.int32, device=device)
+    wts = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
+    L = api.Layout.empty(w.N, w.k, w.E, w.R, device)
+    if w.dtype == "fp8":
+        recv = torch.empty((w.S, w.H), dtype=torch.uint8, device=device)
+        scale = torch.empty((w.S, w.H // 128), dtype=torch.float32, device=device)
+    else:
+        recv = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
+        scale = None
+    out = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
+    y = recv if w.expert_out == "identity" else y_in
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        api.moe_topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn,
+                          topk_idx=idx, topk_w=wts, stream=stream)
+        if ev: ev[1].record(stream)
+        api.moe_get_layout(idx, w.E, w.R, out=L, stream=stream)
+        if ev: ev[2].record(stream)
+        api.moe_dispatch(x, L.token_slot, w.dtype_code, recv_x=recv, recv_scale=scale,
+                         d_status=L.status, stream=stream)
+        if ev: ev[3].record(stream)
+        api.moe_combine(y, L.token_slot, wts, out=out, d_status=L.status, stream=stream)
+        if ev: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    if int(L.status.item()) != 0:
+        raise RuntimeError(f"device status {int(L.status.item())} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    with ClockSampler(device.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    per_op = {n: [] for n in ("gate", "layout", "dispatch", "combine")}
+    step_ms = []
+    for ev in evs:
+        for j, n in enumerate(per_op):
+            per_op[n].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[4]))
+    max_total_ms = max_over_ranks(sum(step_ms), world, device)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world)
+
+    if rank != 0:
+        return
+    ab = algorithmic_bytes(w)
+    peak, peak_kind = measured_peak()
+    avg = {n: sum(v) / len(v) for n, v in per_op.items()}
+    gbs = {n: ab[n] / (avg[n] * 1e-3) / 1e9 for n in avg}
+    dominant = max(("dispatch", "combine"), key=lambda n: avg[n])
+    other = "dispatch" if dominant == "combine" else "combine"
+
+    def roof(n):
+        return {"kernel": n, "bound": "hbm", "achieved": gbs[n], "peak": peak, "unit": "GB/s",
+                "frac": gbs[n] / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                "traffic": ncu_traffic(n, w.name), "algorithmic_bytes": ab[n],
+                "avg_launch_us": 1e3 * avg[n]}
+
+    line = {
+        "impl": "ours", "metric": METRIC,
+        "value": whole_job_rate(w.N, world, args.steps, max_total_ms), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": max_total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": describe(w), "tokens_per_gpu": w.N, "hidden": w.H, "experts": w.E,
+                   "topk": w.k, "logical_ranks": w.R, "payload": f"x bf16, dispatch {w.dtype}, out bf16",
+                   "l2": "flushed before every step (write of 2x L2 size, outside the events)",
+                   "parallelism": f"replicas x{world} (tokens sharded, no collective)"},
+        "per_op_us": {n: 1e3 * v for n, v in avg.items()},
+        "per_op_gbs": gbs,
+        "dispatch_combine_tokens_per_s": w.N * world / ((avg["dispatch"] + avg["combine"]) * 1e-3),
+        "roofline": roof(dominant),
+        "roofline_other": roof(other),
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(),
+        "e2e": e2e,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, make_inputs(w, 0), args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world):
+    """Same step through the public API with the inputs in pinned host memory."""
+    h_logits = inp.logits.pin_memory()
+    h_x = inp.x.pin_memory()
+    h_y = inp.y.pin_memory() if inp.y is not None else None
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = h_logits.numel() * 4 + h_x.numel() * 2 + (h_y.numel() * 2 if h_y is not None else 0)
+    d2h = h_out.numel() * 2
+
+    def e2e_step():
+        logits.copy_(h_logits, non_blocking=True)
+        x.copy_(h_x, non_blocking=True)
+        if h_y is not None:
+            y_in.copy_(h_y, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(3):
+        flush.zero_()
+        e2e_step()
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    total = 0.0
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        b.synchronize()
+        total += a.elapsed_time(b)
+    return {"value": whole_job_rate(w.N, world, steps, max_over_ranks(total, world, device)),
+            "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    try:
+        run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,235 @@
+"""Thin ctypes binding of ``libmoe.so`` (C ABI in ``include/moe.h``).
+
+The functions carry the C entry points' names.  They only marshal: check that
+tensors are CUDA, contiguous and of the right dtype, allocate outputs the
+caller did not pass (``torch.empty`` on the input's device), and pass raw
+pointers, sizes and the current CUDA stream.  Every step of the routing path
+runs in the library's kernels; there is no other implementation behind these
+names.  Importing this module fails if the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX = range(5)
+MOE_GATE_SOFTMAX, MOE_GATE_SOFTMAX_RENORM, MOE_GATE_SIGMOID_GROUP = range(3)
+MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3 = range(2)
+MOE_MAX_EXPERTS = 1024
+MOE_MAX_TOPK = 32
+MOE_FP8_BLOCK = 128
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m combine_moe_topk_gate_b200.build` "
+            "(nvcc, sm_100a).  There is no fallback implementation.")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    L.moe_topk_gate.argtypes = [P, I, I, I, I, I, I, I, P, P, P]
+    L.moe_topk_gate.restype = I
+    L.moe_layout_workspace_bytes.argtypes = [I, I, I, I]
+    L.moe_layout_workspace_bytes.restype = SZ
+    L.moe_get_layout.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P, P]
+    L.moe_get_layout.restype = I
+    L.moe_recv_bytes.argtypes = [I, I, I, I]
+    L.moe_recv_bytes.restype = SZ
+    L.moe_scale_bytes.argtypes = [I, I, I]
+    L.moe_scale_bytes.restype = SZ
+    L.moe_dispatch.argtypes = [P, I, I, I, P, I, P, P, P, P]
+    L.moe_dispatch.restype = I
+    L.moe_combine.argtypes = [P, I, I, I, P, P, P, P, P]
+    L.moe_combine.restype = I
+    L.moe_e4m3_encode.argtypes = [P, SZ, P, P]
+    L.moe_e4m3_encode.restype = I
+    L.moe_status_string.argtypes = [I]
+    L.moe_status_string.restype = ctypes.c_char_p
+    L.moe_abi_version.argtypes = []
+    L.moe_abi_version.restype = I
+    return L
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+# ---------------------------------------------------------------- gate
+def moe_topk_gate(logits: torch.Tensor, k: int, kind: int, n_groups: int = 1,
+                  topk_groups: int = 1, group_topn: int = 1, *, topk_idx=None, topk_w=None,
+                  stream=None):
+    """Top-k router selection and weights; returns ``(topk_idx int32 [N,k], topk_w fp32 [N,k])``."""
+    _need(logits, "logits", torch.float32)
+    N, E = logits.shape
+    if topk_idx is None:
+        topk_idx = torch.empty((N, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((N, k), dtype=torch.float32, device=logits.device)
+    _need(topk_idx, "topk_idx", torch.int32, (N, k))
+    _need(topk_w, "topk_w", torch.float32, (N, k))
+    st = _lib.moe_topk_gate(_ptr(logits), N, E, k, kind, n_groups, topk_groups, group_topn,
+                            _ptr(topk_idx), _ptr(topk_w), _stream(stream, logits.device))
+    _check(st, "moe_topk_gate")
+    return topk_idx, topk_w
+
+
+# ---------------------------------------------------------------- layout
+@dataclass
+class Layout:
+    """Routing metadata of one batch (the reusable handle)."""
+    expert_count: torch.Tensor   # int32 [E]
+    expert_offset: torch.Tensor  # int32 [E+1]
+    rank_count: torch.Tensor     # int32 [R]
+    rank_offset: torch.Tensor    # int32 [R+1]
+    rank_tokens: torch.Tensor    # int32 [R]
+    token_slot: torch.Tensor     # int32 [N, k]
+    slot_token: torch.Tensor     # int32 [N*k]
+    workspace: torch.Tensor      # uint8 scratch
+    status: torch.Tensor         # int32 [1] device status word
+
+    @staticmethod
+    def empty(N: int, k: int, E: int, R: int, device) -> "Layout":
+        i32 = dict(dtype=torch.int32, device=device)
+        ws = moe_layout_workspace_bytes(N, k, E, R)
+        return Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32),
+                      torch.empty(R + 1, **i32), torch.empty(R, **i32), torch.empty((N, k), **i32),
+                      torch.empty(N * k, **i32), torch.empty(ws, dtype=torch.uint8, device=device),
+                      torch.zeros(1, **i32))
+
+
+def moe_layout_workspace_bytes(num_tokens: int, k: int, num_experts: int, num_ranks: int) -> int:
+    return int(_lib.moe_layout_workspace_bytes(num_tokens, k, num_experts, num_ranks))
+
+
+def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, out: Layout | None = None,
+                   stream=None) -> Layout:
+    """Counts, offsets and token<->slot maps; fills (and returns) ``out``.  The
+    device status word ``out.status`` is not cleared here: zero it to start a
+    fresh error record."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    N, k = topk_idx.shape
+    E, R = num_experts, num_ranks
+    if out is None:
+        out = Layout.empty(N, k, E, R, topk_idx.device)
+    st = _lib.moe_get_layout(_ptr(topk_idx), N, k, E, R, _ptr(out.expert_count),
+                             _ptr(out.expert_offset), _ptr(out.rank_count), _ptr(out.rank_offset),
+                             _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token),
+                             _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
+                             _stream(stream, topk_idx.device))
+    _check(st, "moe_get_layout")
+    return out
+
+
+# ---------------------------------------------------------------- dispatch / combine
+def moe_recv_bytes(num_tokens: int, hidden: int, k: int, dtype: int) -> int:
+    return int(_lib.moe_recv_bytes(num_tokens, hidden, k, dtype))
+
+
+def moe_scale_bytes(num_tokens: int, hidden: int, k: int) -> int:
+    return int(_lib.moe_scale_bytes(num_tokens, hidden, k))
+
+
+def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_x=None,
+                 recv_scale=None, d_status=None, stream=None):
+    """Scatter rows of ``x`` (bf16 [N,H]) to their receive rows.  Returns
+    ``(recv_x, recv_scale)``: bf16 [N*k,H] and None, or uint8 e4m3 codes
+    [N*k,H] and fp32 [N*k,H/128]."""
+    _need(x, "x", torch.bfloat16)
+    N, H = x.shape
+    _need(token_slot, "token_slot", torch.int32)
+    k = token_slot.shape[1]
+    S = N * k
+    if dtype == MOE_DTYPE_BF16:
+        if recv_x is None:
+            recv_x = torch.empty((S, H), dtype=torch.bfloat16, device=x.device)
+        _need(recv_x, "recv_x", torch.bfloat16, (S, H))
+        recv_scale = None
+    else:
+        if recv_x is None:
+            recv_x = torch.empty((S, H), dtype=torch.uint8, device=x.device)
+        if recv_scale is None:
+            recv_scale = torch.empty((S, H // MOE_FP8_BLOCK), dtype=torch.float32, device=x.device)
+        _need(recv_x, "recv_x", torch.uint8, (S, H))
+        _need(recv_scale, "recv_scale", torch.float32, (S, H // MOE_FP8_BLOCK))
+    st = _lib.moe_dispatch(_ptr(x), N, H, k, _ptr(token_slot), dtype, _ptr(recv_x),
+                           _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
+    _check(st, "moe_dispatch")
+    return recv_x, recv_scale
+
+
+def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor, *, out=None,
+                d_status=None, stream=None) -> torch.Tensor:
+    """Weighted gather-reduce of expert outputs ``y`` (bf16 [N*k,H]) -> bf16 [N,H]."""
+    _need(y, "y", torch.bfloat16)
+    _need(token_slot, "token_slot", torch.int32)
+    N, k = token_slot.shape
+    H = y.shape[1]
+    _need(topk_w, "topk_w", torch.float32, (N, k))
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=y.device)
+    _need(out, "out", torch.bfloat16, (N, H))
+    st = _lib.moe_combine(_ptr(y), N, H, k, _ptr(token_slot), _ptr(topk_w), _ptr(out),
+                          _ptr(d_status), _stream(stream, y.device))
+    _check(st, "moe_combine")
+    return out
+
+
+def moe_e4m3_encode(x: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
+    """Element-wise e4m3 codes (uint8) of an fp32 tensor, as dispatch encodes them."""
+    _need(x, "x", torch.float32)
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _need(out, "out", torch.uint8, x.shape)
+    st = _lib.moe_e4m3_encode(_ptr(x), x.numel(), _ptr(out), _stream(stream, x.device))
+    _check(st, "moe_e4m3_encode")
+    return out
+
+
+def moe_abi_version() -> int:
+    return int(_lib.moe_abi_version())

@@ -1,0 +1,161 @@
+// dispatch.cu -- scatter each token's hidden row to its k receive rows,
+// optionally quantising it to FP8 e4m3 with one fp32 scale per 128 channels.
+//
+// [pplx] "Efficient and portable mixture-of-experts communication",
+// Dispatch: a token's activations, with block scaling factors when quantised,
+// go to every expert it was routed to, unpacked into a contiguous buffer per
+// expert.  DeepEP V2 summary, usage patterns: BF16 and FP8 dispatch.
+// DeepSeek Tile-Kernels news: per-block FP8 quantisation.
+//
+// Work item = (token, segment).  One warp per item reads the segment of the
+// row once (16-byte streaming loads), converts it in registers and stores it
+// k times (16-byte stores, 512 contiguous bytes per warp and slot).  The
+// segments of one token sit in neighbouring warps of one CTA, so a CTA writes
+// long contiguous runs of every destination row.
+#include "moe_device.cuh"
+#include "moe_launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+
+// FP8: lane owns 16 channels (two 16-byte loads), 8 lanes = one 128-block,
+// a warp covers 512 channels.
+__global__ void __launch_bounds__(kWarps * 32)
+    dispatch_fp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                        const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
+                        float* __restrict__ recv_scale, int32_t* d_status) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (H + 511) / 512;
+  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (item >= static_cast<long long>(N) * segs) return;
+  const int t = static_cast<int>(item / segs);
+  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
+  const int c0 = s * 512 + lane * 16;
+  const bool active = c0 < H;  // H % 128 == 0: whole 8-lane blocks are in or out
+  const long long S = static_cast<long long>(N) * k;
+  const int nblk = H / 128;
+
+  const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (active) {
+    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
+    a = ld_stream(src);
+    b = ld_stream(src + 8);
+  }
+  float f[16];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16_lo(w[i]);
+    f[2 * i + 1] = bf16_hi(w[i]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+  const float inv = __fdiv_rn(448.0f, amax);
+  const float scale = __fdiv_rn(amax, 448.0f);
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float p[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float v = f[4 * i + u];
+      p[u] = (v == 0.0f) ? v : __fmul_rn(v, inv);  // zero keeps its sign
+    }
+    q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+  }
+  const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+  for (int j = 0; j < k; ++j) {
+    const int slot = __shfl_sync(kFullMask, my_slot, j);
+    if (slot == -1) continue;
+    if (slot < -1 || slot >= S) {
+      if (lane == 0) report_bad_index(d_status);
+      continue;
+    }
+    if (active) {
+      st_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
+      if ((lane & 7) == 0) recv_scale[static_cast<size_t>(slot) * nblk + (c0 >> 7)] = scale;
+    }
+  }
+}
+
+// BF16: lane owns 8 channels (one 16-byte vector), a warp covers 256 channels.
+__global__ void __launch_bounds__(kWarps * 32)
+    dispatch_bf16_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                         const int32_t* __restrict__ token_slot, uint16_t* __restrict__ recv_x,
+                         int32_t* d_status) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (H + 255) / 256;
+  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (item >= static_cast<long long>(N) * segs) return;
+  const int t = static_cast<int>(item / segs);
+  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
+  const int c0 = s * 256 + lane * 8;
+  const bool active = c0 < H;  // H % 8 == 0
+  const long long S = static_cast<long long>(N) * k;
+  const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
+  uint4 v = make_uint4(0, 0, 0, 0);
+  if (active) v = ld_stream(x + static_cast<size_t>(t) * H + c0);
+  for (int j = 0; j < k; ++j) {
+    const int slot = __shfl_sync(kFullMask, my_slot, j);
+    if (slot == -1) continue;
+    if (slot < -1 || slot >= S) {
+      if (lane == 0) report_bad_index(d_status);
+      continue;
+    }
+    if (active) st_v4(recv_x + static_cast<size_t>(slot) * H + c0, v);
+  }
+}
+
+__global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
+                                   uint8_t* __restrict__ out) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; 2 * i < n;
+       i += stride) {
+    const float lo = in[2 * i];
+    const float hi = 2 * i + 1 < n ? in[2 * i + 1] : 0.0f;
+    const uint32_t v = e4m3x2(lo, hi);
+    out[2 * i] = static_cast<uint8_t>(v & 0xff);
+    if (2 * i + 1 < n) out[2 * i + 1] = static_cast<uint8_t>(v >> 8);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
+                            int dtype, void* recv_x, float* recv_scale, int32_t* d_status,
+                            cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  if (dtype == MOE_DTYPE_FP8_E4M3) {
+    const long long items = static_cast<long long>(N) * ((H + 511) / 512);
+    const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+    dispatch_fp8_kernel<<<blocks, kWarps * 32, 0, stream>>>(
+        static_cast<const uint16_t*>(x), N, H, k, token_slot, static_cast<uint8_t*>(recv_x),
+        recv_scale, d_status);
+  } else {
+    const long long items = static_cast<long long>(N) * ((H + 255) / 256);
+    const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+    dispatch_bf16_kernel<<<blocks, kWarps * 32, 0, stream>>>(static_cast<const uint16_t*>(x), N,
+                                                            H, k, token_slot,
+                                                            static_cast<uint16_t*>(recv_x),
+                                                            d_status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const size_t pairs = (n + 1) / 2;
+  size_t blocks = (pairs + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  e4m3_encode_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(in, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

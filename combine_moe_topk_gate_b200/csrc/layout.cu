@@ -1,0 +1,257 @@
+// layout.cu -- per-expert / per-rank counts, offsets and token<->slot maps.
+//
+// DeepEP V2 summary, "training / prefill / decoding usage patterns": the
+// handle carries per-expert received-token counts for the grouped GEMM and
+// the routing metadata combine needs.  [pplx] "Efficient and portable
+// mixture-of-experts communication", Dispatch: one contiguous buffer per
+// expert and the source token of every row; Portable kernels: one warp per
+// block counts the tokens bound for each destination; Sharding: experts split
+// over EP ranks (here partitions of one buffer).
+//
+// Two launches, no atomics on the order and no spin waits:
+//   count:  one CTA per chunk of whole tokens (<= 1024 entries); per-chunk
+//           histogram over E+1 buckets (bucket E = masked/invalid entries,
+//           which fill the tail rows) and per-chunk per-rank token counts.
+//   assign: one CTA per chunk again; every CTA sums the histograms of the
+//           chunks before it and of all chunks (column sums, from L2), scans
+//           the totals into expert offsets, ranks its entries inside the
+//           chunk (warp __match_any_sync + popc, then a prefix over the 32
+//           warps) and writes token_slot / slot_token.  CTA 0 writes the
+//           counts and offsets.  The row of entry (t, j) in expert e is the
+//           number of entries routed to e before it in (t, j) order, so the
+//           result is deterministic.
+#include "moe_device.cuh"
+#include "moe_launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int kLayoutThreads = 1024;
+constexpr int kLayoutWarps = kLayoutThreads / 32;
+
+__host__ __device__ __forceinline__ int tokens_per_chunk(int k) { return kLayoutThreads / k; }
+
+__host__ __device__ __forceinline__ int num_chunks(int N, int k) {
+  const int tc = tokens_per_chunk(k);
+  const int c = (N + tc - 1) / tc;
+  return c > 0 ? c : 1;
+}
+
+// bucket of an entry: its expert, E for masked (-1) and invalid ids
+__device__ __forceinline__ int bucket_of(int e, int E) {
+  return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : E;
+}
+
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_count_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R,
+                        int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_rtok,
+                        int32_t* d_status) {
+  extern __shared__ int32_t sm[];
+  int32_t* hist = sm;           // E + 1
+  int32_t* rtok = hist + E + 1;  // R
+  int32_t* sidx = rtok + R;      // kLayoutThreads
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int c = blockIdx.x;
+  const int tc = tokens_per_chunk(k);
+  const long long t0 = static_cast<long long>(c) * tc;
+  const int nt = static_cast<int>(min(static_cast<long long>(tc), N - t0));
+  const int ne = nt > 0 ? nt * k : 0;
+  for (int i = tid; i <= E; i += kLayoutThreads) hist[i] = 0;
+  for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  int e = -1;
+  if (tid < ne) {
+    e = topk_idx[t0 * k + tid];
+    sidx[tid] = e;
+  }
+  __syncthreads();
+  const int b = tid < ne ? bucket_of(e, E) : -1;
+  if (tid < ne && b == E && e != -1) report_bad_index(d_status);
+  // one shared-memory add per distinct bucket in the warp
+  const unsigned same = __match_any_sync(kFullMask, b);
+  if (b >= 0 && (same & lanemask_lt()) == 0) atomicAdd(&hist[b], __popc(same));
+  if (b >= 0 && b < E) {
+    // the token's first slot landing on this rank counts the token once
+    const int epr = E / R;
+    const int r = e / epr;
+    const int j = tid % k;
+    bool first = true;
+    for (int jj = 0; jj < j; ++jj) {
+      const int e2 = sidx[tid - j + jj];
+      if (static_cast<unsigned>(e2) < static_cast<unsigned>(E) && e2 / epr == r) {
+        first = false;
+        break;
+      }
+    }
+    if (first) atomicAdd(&rtok[r], 1);
+  }
+  (void)lane;
+  __syncthreads();
+  for (int i = tid; i <= E; i += kLayoutThreads)
+    chunk_counts[static_cast<size_t>(c) * (E + 1) + i] = hist[i];
+  for (int i = tid; i < R; i += kLayoutThreads) chunk_rtok[static_cast<size_t>(c) * R + i] = rtok[i];
+}
+
+// Exclusive scan of a[0..n) in shared memory, n <= 2 * kLayoutThreads.
+__device__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = 2 * tid, i1 = 2 * tid + 1;
+  const int x0 = i0 < n ? a[i0] : 0;
+  const int x1 = i1 < n ? a[i1] : 0;
+  const int s = x0 + x1;
+  int incl = s;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(kFullMask, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    const int v = warp_sums[lane];
+    int wi = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(kFullMask, wi, off);
+      if (lane >= off) wi += y;
+    }
+    warp_sums[lane] = wi - v;
+  }
+  __syncthreads();
+  const int excl = warp_sums[warp] + incl - s;
+  if (i0 < n) a[i0] = excl;
+  if (i1 < n) a[i1] = excl + x0;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_assign_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R, int C,
+                         const int32_t* __restrict__ chunk_counts,
+                         const int32_t* __restrict__ chunk_rtok, int32_t* __restrict__ expert_count,
+                         int32_t* __restrict__ expert_offset, int32_t* __restrict__ rank_count,
+                         int32_t* __restrict__ rank_offset, int32_t* __restrict__ rank_tokens,
+                         int32_t* __restrict__ token_slot, int32_t* __restrict__ slot_token,
+                         int32_t* d_status) {
+  extern __shared__ int32_t sm[];
+  const int nb = E + 1;
+  int32_t* off = sm;                 // nb: totals, then their exclusive scan
+  int32_t* base = off + nb;          // nb: first row of this chunk per bucket
+  int32_t* wcnt = base + nb;         // kLayoutWarps * nb
+  int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c = blockIdx.x;
+
+  // 1. column sums over chunks: all chunks (totals) and chunks before c
+  for (int b = tid; b < nb; b += kLayoutThreads) {
+    int before = 0, total = 0;
+    for (int cc = 0; cc < C; ++cc) {
+      const int v = chunk_counts[static_cast<size_t>(cc) * nb + b];
+      total += v;
+      before += cc < c ? v : 0;
+    }
+    off[b] = total;
+    base[b] = before;
+  }
+  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
+  __syncthreads();
+  if (c == 0)
+    for (int e = tid; e < E; e += kLayoutThreads) expert_count[e] = off[e];
+  // 2. bucket offsets
+  block_exclusive_scan(off, nb, warp_sums);
+  for (int b = tid; b < nb; b += kLayoutThreads) base[b] += off[b];
+  if (c == 0) {
+    const int epr = E / R;
+    for (int e = tid; e <= E; e += kLayoutThreads) expert_offset[e] = off[e];
+    for (int r = tid; r < R; r += kLayoutThreads) {
+      rank_offset[r] = off[r * epr];
+      rank_count[r] = off[(r + 1) * epr] - off[r * epr];
+      int rt = 0;
+      for (int cc = 0; cc < C; ++cc) rt += chunk_rtok[static_cast<size_t>(cc) * R + r];
+      rank_tokens[r] = rt;
+    }
+    if (tid == 0) rank_offset[R] = off[E];
+  }
+  // 3. ranks inside the chunk
+  const int tc = tokens_per_chunk(k);
+  const long long t0 = static_cast<long long>(c) * tc;
+  const int nt = static_cast<int>(min(static_cast<long long>(tc), N - t0));
+  const int ne = nt > 0 ? nt * k : 0;
+  int e = -1, b = -1;
+  if (tid < ne) {
+    e = topk_idx[t0 * k + tid];
+    b = bucket_of(e, E);
+  }
+  const unsigned same = __match_any_sync(kFullMask, b);
+  const int in_warp = __popc(same & lanemask_lt());
+  if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
+  __syncthreads();
+  for (int bb = tid; bb < nb; bb += kLayoutThreads) {
+    int run = 0;
+    for (int w = 0; w < kLayoutWarps; ++w) {
+      const int v = wcnt[w * nb + bb];
+      wcnt[w * nb + bb] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  if (tid < ne) {
+    const int slot = base[b] + wcnt[warp * nb + b] + in_warp;
+    const long long flat = t0 * k + tid;
+    // counts and ranks come from the same entries, so slot < N*k; the check
+    // only guards against topk_idx changing between the two launches
+    if (slot < 0 || static_cast<long long>(slot) >= static_cast<long long>(N) * k) {
+      token_slot[flat] = -1;
+      report_bad_index(d_status);
+    } else if (b < E) {
+      token_slot[flat] = slot;
+      slot_token[slot] = static_cast<int32_t>(t0 + tid / k);
+    } else {
+      token_slot[flat] = -1;
+      slot_token[slot] = -1;
+    }
+  }
+  (void)lane;
+}
+
+}  // namespace
+
+size_t layout_workspace_bytes(int N, int k, int E, int R) {
+  const size_t C = static_cast<size_t>(num_chunks(N, k));
+  size_t bytes = C * static_cast<size_t>(E + 1 + R) * sizeof(int32_t);
+  bytes = (bytes + 255) / 256 * 256;
+  return bytes < 256 ? 256 : bytes;
+}
+
+cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
+                          int32_t* expert_count, int32_t* expert_offset, int32_t* rank_count,
+                          int32_t* rank_offset, int32_t* rank_tokens, int32_t* token_slot,
+                          int32_t* slot_token, void* workspace, int32_t* d_status,
+                          cudaStream_t stream) {
+  const int C = num_chunks(N, k);
+  int32_t* chunk_counts = static_cast<int32_t*>(workspace);
+  int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
+  const size_t smem_count = (static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
+  const size_t smem_assign =
+      (2 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32) *
+      sizeof(int32_t);
+  cudaError_t err;
+  if (smem_count > 48 * 1024) {
+    err = cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_count));
+    if (err != cudaSuccess) return err;
+  }
+  if (smem_assign > 48 * 1024) {
+    err = cudaFuncSetAttribute(layout_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem_assign));
+    if (err != cudaSuccess) return err;
+  }
+  layout_count_kernel<<<C, kLayoutThreads, smem_count, stream>>>(topk_idx, N, k, E, R, chunk_counts,
+                                                                 chunk_rtok, d_status);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  layout_assign_kernel<<<C, kLayoutThreads, smem_assign, stream>>>(
+      topk_idx, N, k, E, R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
+      rank_offset, rank_tokens, token_slot, slot_token, d_status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

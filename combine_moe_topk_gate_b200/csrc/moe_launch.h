@@ -1,0 +1,33 @@
+// moe_launch.h -- internal launchers behind the C ABI (api.cu validates the
+// arguments, these only pick a launch shape and enqueue the kernels).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+cudaError_t launch_topk_gate(const float* logits, int N, int E, int k, int kind, int n_groups,
+                             int topk_groups, int group_topn, int32_t* topk_idx, float* topk_w,
+                             cudaStream_t stream);
+
+size_t layout_workspace_bytes(int N, int k, int E, int R);
+
+cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
+                          int32_t* expert_count, int32_t* expert_offset, int32_t* rank_count,
+                          int32_t* rank_offset, int32_t* rank_tokens, int32_t* token_slot,
+                          int32_t* slot_token, void* workspace, int32_t* d_status,
+                          cudaStream_t stream);
+
+cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
+                            int dtype, void* recv_x, float* recv_scale, int32_t* d_status,
+                            cudaStream_t stream);
+
+cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
+                           const float* topk_w, void* out, int32_t* d_status,
+                           cudaStream_t stream);
+
+cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream);
+
+}  // namespace moe

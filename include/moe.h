@@ -1,0 +1,210 @@
+/*
+ * moe.h -- C ABI of libmoe.so: the single-GPU MoE routing hot path on B200
+ * (sm_100a): top-k gate -> layout -> dispatch -> combine.
+ *
+ * Pages cited (title, then section):
+ *   [pplx]  "Efficient and portable mixture-of-experts communication"
+ *           (Perplexity Research): Introduction; Sharding and parallelism;
+ *           Portable kernels; Dispatch; Combine.
+ *   [EPv2]  DeepEP V2 release summary (hi.news.hada.io, "DeepSeek ने MoE
+ *           training और inference के लिए open source DeepEP लाइब्रेरी जारी
+ *           की"): "ElasticBuffer interface"; "training / prefill / decoding
+ *           usage patterns".
+ *   [EPv1]  "DeepSeek, DeepEP 오픈소스 공개" (GeekNews): Topic Body;
+ *           성능 / 일반 커널 (normal kernels).
+ *   [TK]    DeepSeek Tile-Kernels / DeepEP V2 news (deepinsightai.io):
+ *           "Funktionen der DeepSeek-Tile-Kernel".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Ownership: every array argument is DEVICE memory owned by the caller.
+ *    The library allocates nothing, frees nothing and keeps no state between
+ *    calls, so the layout outputs can be kept and reused as the "cached
+ *    handle" of [EPv2] usage patterns (routing metadata reused while the
+ *    gating does not change).
+ *  - Streams: `stream` is a cudaStream_t passed as an opaque pointer (NULL is
+ *    the legacy default stream).  Calls only enqueue work on it: they never
+ *    synchronise with the host and return before the GPU work finishes.
+ *  - Host-side errors: arguments are checked before anything is launched; a
+ *    failed check returns MOE_ERR_INVALID_ARG (bad value, NULL pointer,
+ *    misalignment) or MOE_ERR_UNSUPPORTED (beyond a documented limit) and
+ *    enqueues nothing.  A launch the CUDA runtime rejects returns
+ *    MOE_ERR_CUDA.
+ *  - Device-side errors: an index found out of range by a kernel is skipped
+ *    and, when `d_status` is not NULL, MOE_ERR_BAD_INDEX is stored to
+ *    *d_status (one int32 in device memory that the caller zeroes and reads
+ *    after the stream work finished).  No kernel traps or asserts.
+ *  - Sizes: N = num_tokens, H = hidden, E = num_experts, k = experts per
+ *    token, R = logical EP ranks, S = N*k receive rows.  Row-major layouts.
+ *    Byte offsets are 64-bit; S must stay below 2^31 (int32 slot ids).
+ *  - Index -1 in topk_idx / token_slot marks a masked slot: it is skipped
+ *    without an error.  Any other id outside range is MOE_ERR_BAD_INDEX.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_CUDA = 3,
+    MOE_ERR_BAD_INDEX = 4
+} moe_status_t;
+
+typedef enum {
+    MOE_GATE_SOFTMAX = 0,        /* w_j = softmax(logits)[sel_j]                     */
+    MOE_GATE_SOFTMAX_RENORM = 1, /* w_j = p_sel_j / sum_j' p_sel_j'                  */
+    MOE_GATE_SIGMOID_GROUP = 2   /* DeepSeek-V3 group-limited sigmoid gating         */
+} moe_gate_kind_t;
+
+typedef enum {
+    MOE_DTYPE_BF16 = 0,          /* payload copied as bf16                            */
+    MOE_DTYPE_FP8_E4M3 = 1       /* payload quantised to e4m3, one fp32 scale / 128ch */
+} moe_dtype_t;
+
+typedef void* moe_stream_t;      /* a cudaStream_t */
+
+#define MOE_MAX_EXPERTS 1024
+#define MOE_MAX_TOPK 32
+#define MOE_FP8_BLOCK 128
+
+/*
+ * moe_topk_gate -- router top-k selection and weights.
+ *   [pplx] Introduction: the router turns the token's logits into a
+ *   probability distribution, the top-K experts are taken and their outputs
+ *   are averaged with the router's weights.  [TK]: top-k selection, scoring
+ *   and weight normalisation.  [EPv1] Topic Body / normal kernels: DeepSeek-V3
+ *   group-limited gating with top-4 groups and top-8 experts.
+ *
+ *   logits   fp32 [N, E] row-major (read only).
+ *   kind     MOE_GATE_SOFTMAX / _RENORM: p = softmax(logits) with
+ *            e_i = exp(l_i - max l) and Z summed in ascending expert order;
+ *            selection on the logits (softmax is increasing).
+ *            MOE_GATE_SIGMOID_GROUP: s = sigmoid(logit); E experts in
+ *            n_groups consecutive groups; group score = sum of the
+ *            group_topn largest s of the group (added largest first);
+ *            the topk_groups best groups are kept; the k best s among the
+ *            kept experts are selected; w_j = s_j / sum of the selected s
+ *            (summed in slot order).  n_groups/topk_groups/group_topn are
+ *            ignored by the softmax kinds.
+ *   topk_idx int32 [N, k] out: expert ids, best first.  Ties go to the
+ *            lower expert (or group) index.
+ *   topk_w   fp32  [N, k] out: weights in the same order.
+ *   exp is one fixed fp32 routine (Cody-Waite reduction + degree-7 Taylor,
+ *   input clamped to [-87, 88]), so results are reproducible bit for bit.
+ *   Limits: 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= min(E, MOE_MAX_TOPK);
+ *   group kind: E % n_groups == 0, 1 <= topk_groups <= n_groups,
+ *   1 <= group_topn <= E/n_groups, topk_groups*(E/n_groups) >= k.
+ *   Pointers 4-byte aligned.  N == 0 enqueues nothing.
+ */
+moe_status_t moe_topk_gate(const float* logits, int num_tokens, int num_experts, int k,
+                           moe_gate_kind_t kind, int n_groups, int topk_groups,
+                           int group_topn, int32_t* topk_idx, float* topk_w,
+                           moe_stream_t stream);
+
+/* Bytes of device scratch moe_get_layout needs for these sizes (>= 256). */
+size_t moe_layout_workspace_bytes(int num_tokens, int k, int num_experts, int num_ranks);
+
+/*
+ * moe_get_layout -- per-expert / per-rank counts, offsets and the
+ * token<->slot maps of the expert-contiguous receive buffer.
+ *   [EPv2] usage patterns: the dispatch handle carries the routing metadata
+ *   for combine and the per-expert received-token counts for the grouped
+ *   GEMM.  [pplx] Dispatch: tokens land in one contiguous per-expert buffer
+ *   and the source token of every row is kept for combine.  [pplx] Sharding:
+ *   experts are sharded over EP ranks, rank r owning experts
+ *   [r*E/R, (r+1)*E/R); here ranks are partitions of one buffer.
+ *
+ *   topk_idx      int32 [N, k] in (from moe_topk_gate or the caller).
+ *   expert_count  int32 [E]    rows per expert.
+ *   expert_offset int32 [E+1]  exclusive prefix sum; expert_offset[E] = valid rows.
+ *   rank_count    int32 [R]    rows per logical rank.
+ *   rank_offset   int32 [R+1]  = expert_offset[r*E/R]; rank_offset[R] = valid rows.
+ *   rank_tokens   int32 [R]    tokens with at least one expert on rank r.
+ *   token_slot    int32 [N, k] receive row of (token, j); -1 if masked/invalid.
+ *   slot_token    int32 [S]    source token of every receive row; the tail rows
+ *                              [expert_offset[E], S) (masked entries) hold -1.
+ *   Order inside an expert is ascending token id, then slot j: the result is
+ *   deterministic (the pages leave the receive order open).
+ *   workspace     device scratch of moe_layout_workspace_bytes() bytes, 16-byte
+ *                 aligned; contents need no initialisation and are not kept.
+ *   Limits: 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= MOE_MAX_TOPK, E % R == 0.
+ */
+moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k,
+                            int num_experts, int num_ranks, int32_t* expert_count,
+                            int32_t* expert_offset, int32_t* rank_count,
+                            int32_t* rank_offset, int32_t* rank_tokens,
+                            int32_t* token_slot, int32_t* slot_token, void* workspace,
+                            size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
+
+/* Receive-buffer payload bytes: N*k rows of H bf16 (2 B) or e4m3 (1 B). */
+size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
+/* FP8 scale bytes: N*k rows of H/128 fp32. */
+size_t moe_scale_bytes(int num_tokens, int hidden, int k);
+
+/*
+ * moe_dispatch -- scatter each token's row to all of its receive rows.
+ *   [pplx] Dispatch: a token's activations (plus block scaling factors when
+ *   quantised) go to every expert it was routed to.  [EPv2] usage patterns:
+ *   BF16 and FP8 dispatch.  [TK]: per-block FP8 quantisation.
+ *
+ *   x           bf16 [N, H] in.
+ *   token_slot  int32 [N, k] from moe_get_layout.
+ *   BF16:  recv_x bf16 [S, H]: recv_x[token_slot[t,j]] = x[t]; recv_scale unused.
+ *          H % 8 == 0; x and recv_x 16-byte aligned.
+ *   FP8:   recv_x e4m3 [S, H], recv_scale fp32 [S, H/128].  Per token and
+ *          128-channel block: amax = max|x|, scale = amax/448,
+ *          code = e4m3_rne_satfinite(x * (448/amax)) (fp32 divisions and
+ *          product, IEEE rounding); zeros keep their sign (so an all-zero
+ *          block gives scale 0 and zero codes).  H % 128 == 0; x, recv_x
+ *          16-byte aligned, recv_scale 4-byte aligned.
+ *   Rows no slot names are not written.  A slot outside [-1, S) is skipped
+ *   and reported through d_status.
+ */
+moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
+                          const int32_t* token_slot, moe_dtype_t dtype, void* recv_x,
+                          float* recv_scale, int32_t* d_status, moe_stream_t stream);
+
+/*
+ * moe_combine -- weighted gather-reduce of each token's k expert outputs.
+ *   [pplx] Introduction and Combine: the output is the average of the
+ *   selected experts' outputs weighted by the router weights; [EPv2] usage
+ *   patterns: combine reduces expert outputs back to the token.
+ *
+ *   y          bf16 [S, H] expert outputs, one row per receive slot.
+ *   token_slot int32 [N, k], topk_w fp32 [N, k].
+ *   out        bf16 [N, H]:  acc = +0.0f; for j = 0..k-1 (slot order):
+ *              acc = fmaf(topk_w[t,j], y[token_slot[t,j], c], acc);
+ *              out = bf16 round-to-nearest-even(acc).  Masked slots add
+ *              nothing.  H % 8 == 0; y and out 16-byte aligned.
+ */
+moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
+                         const int32_t* token_slot, const float* topk_w, void* out,
+                         int32_t* d_status, moe_stream_t stream);
+
+/*
+ * moe_e4m3_encode -- the element encoder moe_dispatch uses, exposed on its
+ * own: out[i] = e4m3 code of in[i], round to nearest even, finite values and
+ * infinities beyond 448 saturated to +-448, zero keeps its sign, NaN -> NaN
+ * code.  (OCP 8-bit floating point, E4M3.)  n may be 0.
+ */
+moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t status);
+
+/* ABI version: bumped when a signature or a documented behaviour changes. */
+int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,110 @@
+"""CPU checks of the C ABI: the library loads, exports every entry point that
+``include/*.h`` declares, answers size queries, and rejects invalid arguments
+on the host before anything is launched (no compute call needs a GPU here)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def api():
+    from combine_moe_topk_gate_b200 import build
+    build.build()
+    from combine_moe_topk_gate_b200 import api as A
+    return A
+
+
+def test_every_declared_symbol_is_exported(api):
+    names = _declared()
+    assert {"moe_topk_gate", "moe_get_layout", "moe_dispatch", "moe_combine"} <= set(names)
+    L = api.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_size_queries(api):
+    assert api.moe_recv_bytes(4096, 7168, 8, api.MOE_DTYPE_FP8_E4M3) == 4096 * 8 * 7168
+    assert api.moe_recv_bytes(16384, 4096, 2, api.MOE_DTYPE_BF16) == 16384 * 2 * 4096 * 2
+    assert api.moe_scale_bytes(4096, 7168, 8) == 4096 * 8 * 56 * 4
+    ws = api.moe_layout_workspace_bytes(4096, 8, 256, 32)
+    assert ws >= 256 and ws % 256 == 0
+    assert api.moe_layout_workspace_bytes(0, 8, 256, 32) >= 256
+    assert api.moe_layout_workspace_bytes(-1, 8, 256, 32) == 0
+    assert api.moe_abi_version() >= 1
+    assert api.status_string(api.MOE_ERR_BAD_INDEX)
+
+
+def _P(v=0x1000):
+    return ctypes.c_void_p(v)
+
+
+def test_gate_rejects_bad_arguments(api):
+    L = api.lib()
+    ok = dict(N=10, E=8, k=2, kind=0, G=1, TG=1, n=1)
+
+    def call(**kw):
+        a = {**ok, **kw}
+        return L.moe_topk_gate(_P(), a["N"], a["E"], a["k"], a["kind"], a["G"], a["TG"], a["n"],
+                               _P(), _P(), None)
+    assert call(k=9) == api.MOE_ERR_INVALID_ARG             # k > E
+    assert call(k=0) == api.MOE_ERR_INVALID_ARG
+    assert call(N=-1) == api.MOE_ERR_INVALID_ARG
+    assert call(kind=7) == api.MOE_ERR_INVALID_ARG
+    assert call(E=2048, k=4) == api.MOE_ERR_UNSUPPORTED      # beyond MOE_MAX_EXPERTS
+    assert call(E=64, k=33) == api.MOE_ERR_UNSUPPORTED       # beyond MOE_MAX_TOPK
+    assert call(kind=2, E=256, G=7, TG=4, n=2, k=8) == api.MOE_ERR_INVALID_ARG   # E % G
+    assert call(kind=2, E=256, G=8, TG=9, n=2, k=8) == api.MOE_ERR_INVALID_ARG   # TG > G
+    assert call(kind=2, E=256, G=8, TG=4, n=33, k=8) == api.MOE_ERR_INVALID_ARG  # n > E/G
+    assert call(kind=2, E=256, G=64, TG=1, n=2, k=8) == api.MOE_ERR_INVALID_ARG  # TG*E/G < k
+    assert L.moe_topk_gate(None, 10, 8, 2, 0, 1, 1, 1, _P(), _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_topk_gate(_P(0x1001), 10, 8, 2, 0, 1, 1, 1, _P(), _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert call(N=0) == api.MOE_OK                            # empty: nothing enqueued
+
+
+def test_layout_rejects_bad_arguments(api):
+    L = api.lib()
+    ws = api.moe_layout_workspace_bytes(100, 4, 16, 4)
+
+    def call(N=100, k=4, E=16, R=4, wsb=ws, idx=_P(), work=_P()):
+        return L.moe_get_layout(idx, N, k, E, R, _P(), _P(), _P(), _P(), _P(), _P(), _P(), work, wsb,
+                                None, None)
+    assert call(R=3) == api.MOE_ERR_INVALID_ARG       # E % R
+    assert call(R=0) == api.MOE_ERR_INVALID_ARG
+    assert call(wsb=ws - 1) == api.MOE_ERR_INVALID_ARG
+    assert call(idx=None) == api.MOE_ERR_INVALID_ARG
+    assert call(work=_P(0x1008)) == api.MOE_ERR_INVALID_ARG   # workspace not 16-byte aligned
+    assert call(k=40) == api.MOE_ERR_UNSUPPORTED
+    assert call(E=2048, R=4) == api.MOE_ERR_UNSUPPORTED
+    assert call(N=1 << 29, k=8, wsb=1 << 40) == api.MOE_ERR_UNSUPPORTED   # N*k >= 2^31
+
+
+def test_dispatch_combine_reject_bad_arguments(api):
+    L = api.lib()
+    FP8, BF16 = api.MOE_DTYPE_FP8_E4M3, api.MOE_DTYPE_BF16
+    assert L.moe_dispatch(_P(), 10, 200, 2, _P(), FP8, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(_P(), 10, 100, 2, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), FP8, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(_P(0x1008), 10, 256, 2, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), 5, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(_P(), 10, 256, 40, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_UNSUPPORTED
+    assert L.moe_dispatch(None, 0, 256, 2, None, BF16, None, None, None, None) == api.MOE_OK
+    assert L.moe_combine(_P(), 10, 100, 2, _P(), _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(_P(), 10, 256, 2, _P(), _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(_P(), 10, 256, 2, _P(), _P(), _P(0x1004), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(None, 0, 256, 2, None, None, None, None, None) == api.MOE_OK
+    assert L.moe_e4m3_encode(None, 0, None, None) == api.MOE_OK
+    assert L.moe_e4m3_encode(None, 5, _P(), None) == api.MOE_ERR_INVALID_ARG
