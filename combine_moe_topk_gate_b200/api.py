@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     L.moe_layout_workspace_bytes.restype = SZ
     L.moe_get_layout.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P, P]
     L.moe_get_layout.restype = I
+    L.moe_get_layout_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, P]
+    L.moe_get_layout_noalloc.restype = I
     L.moe_recv_bytes.argtypes = [I, I, I, I]
     L.moe_recv_bytes.restype = SZ
     L.moe_scale_bytes.argtypes = [I, I, I]
@@ -163,6 +165,31 @@ def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, 
                              _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
                              _stream(stream, topk_idx.device))
     _check(st, "moe_get_layout")
+    return out
+
+
+MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 1 << 20
+
+
+def moe_get_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *,
+                           out: Layout | None = None, stream=None) -> Layout:
+    """``moe_get_layout`` for callers that cannot allocate device scratch: the
+    library uses its own fixed array (``MOE_LAYOUT_NOALLOC_SCRATCH_BYTES``)
+    instead of ``out.workspace``.  Calls must not overlap on the GPU (they share
+    the array); the first call on a device should come before any stream
+    capture.  Outputs are still the caller's (allocated here when ``out`` is
+    None, like every other binding)."""
+    _need(topk_idx, "topk_idx", torch.int32)
+    N, k = topk_idx.shape
+    E, R = num_experts, num_ranks
+    if out is None:
+        out = Layout.empty(N, k, E, R, topk_idx.device)
+    st = _lib.moe_get_layout_noalloc(_ptr(topk_idx), N, k, E, R, _ptr(out.expert_count),
+                                     _ptr(out.expert_offset), _ptr(out.rank_count),
+                                     _ptr(out.rank_offset), _ptr(out.rank_tokens),
+                                     _ptr(out.token_slot), _ptr(out.slot_token), _ptr(out.status),
+                                     _stream(stream, topk_idx.device))
+    _check(st, "moe_get_layout_noalloc")
     return out
 
 

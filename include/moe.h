@@ -144,6 +144,33 @@ moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k,
                             int32_t* token_slot, int32_t* slot_token, void* workspace,
                             size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
 
+/*
+ * moe_get_layout_noalloc -- moe_get_layout without a caller-provided
+ * workspace.  The pages have no counterpart: this is an addition for callers
+ * that cannot allocate device memory, such as serving runtimes that reserve
+ * all of the GPU's memory for their own pool at start-up, or deployments
+ * whose memory plan is fixed before the first request; cudaMalloc there
+ * fails or breaks the budget.  The scratch is a fixed array of
+ * MOE_LAYOUT_NOALLOC_SCRATCH_BYTES in the library's device memory, held by
+ * every GPU that loads the library until the process exits.
+ *   Arguments, outputs and results are those of moe_get_layout.  The call
+ *   allocates nothing.  It returns MOE_ERR_UNSUPPORTED, enqueueing nothing,
+ *   when moe_layout_workspace_bytes(N, k, E, R) exceeds the array.
+ *   The first call on a device looks up the array's address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.  All calls share the one array and it keeps the last
+ *   call's contents (nothing in it needs clearing): calls whose GPU work
+ *   overlaps -- other streams, other host threads -- race on it, so
+ *   serialise them.
+ */
+#define MOE_LAYOUT_NOALLOC_SCRATCH_BYTES (1u << 20)
+moe_status_t moe_get_layout_noalloc(const int32_t* topk_idx, int num_tokens, int k,
+                                    int num_experts, int num_ranks, int32_t* expert_count,
+                                    int32_t* expert_offset, int32_t* rank_count,
+                                    int32_t* rank_offset, int32_t* rank_tokens,
+                                    int32_t* token_slot, int32_t* slot_token, int32_t* d_status,
+                                    moe_stream_t stream);
+
 /* Receive-buffer payload bytes: N*k rows of H bf16 (2 B) or e4m3 (1 B). */
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
 /* FP8 scale bytes: N*k rows of H/128 fp32. */
