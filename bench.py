@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    p.add_argument("--tokens", type=int, default=None,
+                   help="override the workload's token count (profiling captures of a smaller case)")
     return p.parse_args()
 
 
@@ -214,8 +216,13 @@ def cpu_baseline(w, inp, budget_s):
                       f"dispatch+combine, single-threaded C, {dt:.1f} s"}
 
 
-def run_reference(args, rank, world):
+def workload(args):
     w = WORKLOADS[args.workload]
+    return w if args.tokens is None else w.scaled(args.tokens)
+
+
+def run_reference(args, rank, world):
+    w = workload(args)
     if rank != 0:
         return
     inp = make_inputs(w, 0)
@@ -243,7 +250,7 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------- our arm
 def run_ours(args, rank, world, device):
     from combine_moe_topk_gate_b200 import api
-    w = WORKLOADS[args.workload]
+    w = workload(args)
     inp = make_inputs(w, rank)
     stream = torch.cuda.current_stream(device)
     logits = inp.logits.to(device)
