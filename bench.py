@@ -271,6 +271,7 @@ def run_ours(args, rank, world, device):
     flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
 
     def step(ev=None):
+        stream = torch.cuda.current_stream(device)  # the capture stream inside torch.cuda.graph
         if ev: ev[0].record(stream)
         api.moe_topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn,
                           topk_idx=idx, topk_w=wts, stream=stream)
@@ -290,23 +291,35 @@ def run_ours(args, rank, world, device):
     if int(L.status.item()) != 0:
         raise RuntimeError(f"device status {int(L.status.item())} after warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # The step is captured once as a CUDA graph (event-record nodes between the
+    # ops) and replayed, so the timed interval is device time of the 5 kernels
+    # back to back, not the Python binding's launch overhead.
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(evs)
+    for _ in range(args.warmup):
+        flush.zero_()
+        graph.replay()
+    torch.cuda.synchronize(device)
+    per_op = {n: [] for n in ("gate", "layout", "dispatch", "combine")}
+    step_ms = []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(device.index) as clk:
         for i in range(args.steps):
             flush.zero_()
-            step(evs[i])
+            graph.replay()
+            evs[4].synchronize()
+            for j, n in enumerate(per_op):
+                per_op[n].append(evs[j].elapsed_time(evs[j + 1]))
+            step_ms.append(evs[0].elapsed_time(evs[4]))
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
-    per_op = {n: [] for n in ("gate", "layout", "dispatch", "combine")}
-    step_ms = []
-    for ev in evs:
-        for j, n in enumerate(per_op):
-            per_op[n].append(ev[j].elapsed_time(ev[j + 1]))
-        step_ms.append(ev[0].elapsed_time(ev[4]))
+    if int(L.status.item()) != 0:
+        raise RuntimeError(f"device status {int(L.status.item())} after the timed steps")
     max_total_ms = max_over_ranks(sum(step_ms), world, device)
 
     e2e = None
@@ -337,6 +350,8 @@ def run_ours(args, rank, world, device):
         "config": {"workload": describe(w), "tokens_per_gpu": w.N, "hidden": w.H, "experts": w.E,
                    "topk": w.k, "logical_ranks": w.R, "payload": f"x bf16, dispatch {w.dtype}, out bf16",
                    "l2": "flushed before every step (write of 2x L2 size, outside the events)",
+                   "timing": "one step captured as a CUDA graph, replayed per step; CUDA events "
+                             "(graph event-record nodes) between the ops",
                    "parallelism": f"replicas x{world} (tokens sharded, no collective)"},
         "per_op_us": {n: 1e3 * v for n, v in avg.items()},
         "per_op_gbs": gbs,

@@ -31,6 +31,7 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_UNSUPPORTED: return "unsupported size or option";
     case MOE_ERR_CUDA: return "CUDA launch error";
     case MOE_ERR_BAD_INDEX: return "index out of range (skipped)";
+    case MOE_ERR_TIMEOUT: return "device wait timed out (output incomplete)";
   }
   return "unknown status";
 }

@@ -5,77 +5,197 @@
 // experts' outputs weighted by the router weights.  DeepEP V2 summary, usage
 // patterns: combine reduces the expert outputs back to the token.
 //
-// Work item = (token, 256-channel segment), one warp each; lane owns 8
-// channels.  Up to 8 slot rows are loaded (16 bytes per lane each) before any
-// of them is used, so every lane keeps 128 bytes in flight; the partial rows
-// live in registers and are folded with fmaf in slot order, then rounded to
-// bf16 once:  acc = +0; acc = fmaf(w_j, y_j, acc) for j = 0..k-1.
+//   out[t, c] = bf16_rne(acc),  acc = +0, then acc = fmaf(w[t,j], y[slot[t,j], c], acc)
+//   for j = 0..k-1 in slot order (masked slots skipped).
+//
+// Persistent, warp-specialised CTAs.  Work item = (token, 1024-channel
+// segment); each CTA walks a contiguous range of items, so consecutive items
+// mostly share a token and its metadata.
+//   producer warp: per item, waits for a free stage of a shared-memory ring,
+//     writes the item's weights and valid-slot mask into the stage header and
+//     issues one 1-D bulk copy (cp.async.bulk, global -> shared, completing on
+//     the stage's "full" mbarrier) per valid slot row -- lane j copies row j.
+//     The next token's slots and weights are loaded one token ahead.
+//   4 consumer warps: per item, wait for "full", each thread folds its 8
+//     channels of the k staged rows in slot order, stores 16 bytes of bf16,
+//     and the warp releases the stage through its "empty" mbarrier.
+// The stages keep k * 2 KB * stages bytes per CTA in flight without any
+// registers holding them; waits are bounded (1 s, then MOE_ERR_TIMEOUT).
+#include <algorithm>
+
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;
-constexpr int kBatch = 8;
+constexpr int kSeg = 1024;              // channels per work item
+constexpr int kSegBytes = kSeg * 2;     // one bf16 row segment
+constexpr int kConsumerWarps = 4;       // 128 threads x 8 channels = kSeg
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kHeaderBytes = 256;       // weights[32] + valid mask, per stage
+constexpr int kStageTarget = 64 * 1024; // shared bytes in flight per CTA
+constexpr int kMaxStages = 8;
 
-__global__ void __launch_bounds__(kWarps * 32)
-    combine_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
-                   const int32_t* __restrict__ token_slot, const float* __restrict__ topk_w,
-                   uint16_t* __restrict__ out, int32_t* d_status) {
-  const int lane = threadIdx.x & 31;
-  const int segs = (H + 255) / 256;
-  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(N) * segs) return;
-  const int t = static_cast<int>(item / segs);
-  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
-  const int c0 = s * 256 + lane * 8;
-  const bool active = c0 < H;
+struct Layout {
+  int nstage;
+  size_t stage_bytes;
+  size_t bars_off, hdr_off, data_off, total;
+};
+
+__host__ __device__ inline Layout smem_layout(int k) {
+  Layout L;
+  L.stage_bytes = static_cast<size_t>(k) * kSegBytes;
+  int ns = static_cast<int>(kStageTarget / L.stage_bytes);
+  L.nstage = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
+  L.bars_off = 0;
+  L.hdr_off = 128;  // 2 * kMaxStages mbarriers of 8 bytes
+  L.data_off = L.hdr_off + static_cast<size_t>(L.nstage) * kHeaderBytes;
+  L.total = L.data_off + static_cast<size_t>(L.nstage) * L.stage_bytes;
+  return L;
+}
+
+__global__ void __launch_bounds__(kThreads)
+    combine_bulk_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
+                        const int32_t* __restrict__ token_slot, const float* __restrict__ topk_w,
+                        uint16_t* __restrict__ out, int32_t* d_status) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const Layout L = smem_layout(k);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t bars = smem_addr(smem + L.bars_off);  // full[s] at bars + 8s, empty[s] at + 64
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 64u + 8u * s; };
+  const uint32_t data = smem_addr(smem + L.data_off);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L.nstage; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kConsumerWarps);
+    }
+    mbar_init_fence();
+  }
+  __syncthreads();
+
+  const int segs = (H + kSeg - 1) / kSeg;
+  const long long items = static_cast<long long>(N) * segs;
+  const long long per = (items + gridDim.x - 1) / gridDim.x;
+  const long long i0 = static_cast<long long>(blockIdx.x) * per;
+  const long long i1 = i0 + per < items ? i0 + per : items;
   const long long S = static_cast<long long>(N) * k;
 
-  int my_slot = -1;
-  float my_w = 0.0f;
-  if (lane < k) {
-    my_slot = token_slot[static_cast<size_t>(t) * k + lane];
-    my_w = topk_w[static_cast<size_t>(t) * k + lane];
-  }
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-
-  for (int j0 = 0; j0 < k; j0 += kBatch) {
-    uint4 v[kBatch];
-    float wj[kBatch];
-    bool use[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int j = j0 + u;
-      const int slot = __shfl_sync(kFullMask, my_slot, j & 31);
-      wj[u] = __shfl_sync(kFullMask, my_w, j & 31);
-      const bool in_range = slot >= 0 && slot < S;
-      if (j < k && (slot < -1 || slot >= S) && lane == 0) report_bad_index(d_status);
-      use[u] = j < k && in_range;
-      v[u] = make_uint4(0, 0, 0, 0);
-      if (use[u] && active) v[u] = ld_stream(y + static_cast<size_t>(slot) * H + c0);
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (!use[u]) continue;
-      const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = __fmaf_rn(wj[u], bf16_lo(w4[i]), acc[2 * i]);
-        acc[2 * i + 1] = __fmaf_rn(wj[u], bf16_hi(w4[i]), acc[2 * i + 1]);
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    int stage = 0;
+    uint32_t phase = 0;
+    long long issued = 0;
+    bool ok = true;
+    int cur_t = -1, my_slot = -1, next_slot = -1;
+    float my_w = 0.0f, next_w = 0.0f;
+    if (i0 < i1) {
+      const int t0 = static_cast<int>(i0 / segs);
+      if (lane < k) {
+        next_slot = token_slot[static_cast<size_t>(t0) * k + lane];
+        next_w = topk_w[static_cast<size_t>(t0) * k + lane];
       }
     }
-  }
-  if (active) {
-    uint4 o;
-    o.x = pack_bf16x2(acc[0], acc[1]);
-    o.y = pack_bf16x2(acc[2], acc[3]);
-    o.z = pack_bf16x2(acc[4], acc[5]);
-    o.w = pack_bf16x2(acc[6], acc[7]);
-    st_v4(out + static_cast<size_t>(t) * H + c0, o);
+    for (long long it = i0; it < i1; ++it) {
+      const int t = static_cast<int>(it / segs);
+      const int s = static_cast<int>(it - static_cast<long long>(t) * segs);
+      if (t != cur_t) {
+        cur_t = t;
+        my_slot = next_slot;
+        my_w = next_w;
+        if (lane < k && t + 1 < N) {  // one token ahead
+          next_slot = token_slot[static_cast<size_t>(t + 1) * k + lane];
+          next_w = topk_w[static_cast<size_t>(t + 1) * k + lane];
+        }
+        if (lane < k && (my_slot < -1 || my_slot >= S)) report_bad_index(d_status);
+      }
+      if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
+        report_timeout(d_status);
+        ok = false;
+        break;
+      }
+      const int seg_ch = H - s * kSeg < kSeg ? H - s * kSeg : kSeg;
+      const uint32_t row_bytes = static_cast<uint32_t>(seg_ch) * 2u;
+      const bool valid = lane < k && my_slot >= 0 && my_slot < S;
+      const uint32_t vmask = __ballot_sync(kFullMask, valid);
+      float* hw = reinterpret_cast<float*>(smem + L.hdr_off + static_cast<size_t>(stage) * kHeaderBytes);
+      if (lane < k) hw[lane] = my_w;
+      if (lane == 0) reinterpret_cast<uint32_t*>(hw)[32] = vmask;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), __popc(vmask) * row_bytes);
+      __syncwarp();
+      if (valid)
+        bulk_g2s(data + static_cast<uint32_t>(stage * L.stage_bytes) + lane * kSegBytes,
+                 y + static_cast<size_t>(my_slot) * H + static_cast<size_t>(s) * kSeg, row_bytes,
+                 full_bar(stage));
+      ++issued;
+      if (++stage == L.nstage) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if (!ok) {
+      // let the copies already issued land before the CTA may exit
+      const long long n = issued < L.nstage ? issued : L.nstage;
+      for (long long q = issued - n; q < issued; ++q)  // q-th issue: stage q % ns, parity (q / ns) & 1
+        mbar_wait(full_bar(static_cast<int>(q % L.nstage)),
+                  static_cast<uint32_t>((q / L.nstage) & 1));
+    }
+  } else {
+    // ------------------------------------------------------------ consumers
+    int stage = 0;
+    uint32_t phase = 0;
+    const int c = threadIdx.x * 8;  // this thread's 8 channels of the segment
+    for (long long it = i0; it < i1; ++it) {
+      const int t = static_cast<int>(it / segs);
+      const int s = static_cast<int>(it - static_cast<long long>(t) * segs);
+      if (!mbar_wait(full_bar(stage), phase)) {
+        report_timeout(d_status);
+        break;
+      }
+      const int seg_ch = H - s * kSeg < kSeg ? H - s * kSeg : kSeg;
+      if (c < seg_ch) {
+        const float* hw =
+            reinterpret_cast<const float*>(smem + L.hdr_off + static_cast<size_t>(stage) * kHeaderBytes);
+        const uint32_t vmask = reinterpret_cast<const uint32_t*>(hw)[32];
+        const uint32_t row0 = data + static_cast<uint32_t>(stage * L.stage_bytes) + c * 2;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int j0 = 0; j0 < k; j0 += 8) {
+          uint4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            if (j0 + u < k) v[u] = ld_shared_v4(row0 + (j0 + u) * kSegBytes);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + u;
+            if (j >= k || !((vmask >> j) & 1u)) continue;
+            const float wj = hw[j];
+            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              acc[2 * i] = __fmaf_rn(wj, bf16_lo(w4[i]), acc[2 * i]);
+              acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(w4[i]), acc[2 * i + 1]);
+            }
+          }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(acc[0], acc[1]);
+        o.y = pack_bf16x2(acc[2], acc[3]);
+        o.z = pack_bf16x2(acc[4], acc[5]);
+        o.w = pack_bf16x2(acc[6], acc[7]);
+        st_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * kSeg + c, o);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty_bar(stage));
+      if (++stage == L.nstage) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
   }
 }
 
@@ -85,11 +205,24 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
                            const float* topk_w, void* out, int32_t* d_status,
                            cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
-  const long long items = static_cast<long long>(N) * ((H + 255) / 256);
-  const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  combine_kernel<<<blocks, kWarps * 32, 0, stream>>>(static_cast<const uint16_t*>(y), N, H, k,
-                                                     token_slot, topk_w,
-                                                     static_cast<uint16_t*>(out), d_status);
+  const Layout L = smem_layout(k);
+  cudaError_t err = cudaFuncSetAttribute(combine_bulk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L.total));
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, kThreads,
+                                                           L.total)) != cudaSuccess)
+    return err;
+  if (per_sm < 1) per_sm = 1;
+  const long long items = static_cast<long long>(N) * ((H + kSeg - 1) / kSeg);
+  const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
+  combine_bulk_kernel<<<static_cast<unsigned>(grid), kThreads, L.total, stream>>>(
+      static_cast<const uint16_t*>(y), N, H, k, token_slot, topk_w, static_cast<uint16_t*>(out),
+      d_status);
   return cudaGetLastError();
 }
 

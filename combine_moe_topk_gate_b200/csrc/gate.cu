@@ -7,45 +7,231 @@
 // normalisation.  "DeepSeek, DeepEP 오픈소스 공개", Topic Body and 일반 커널:
 // DeepSeek-V3 group-limited gating, top-4 groups / top-8 experts.
 //
-// Layout in registers: lane l holds experts l, l+32, l+64, ... (coalesced
-// 128-byte row loads).  A selection round finds, per lane, the best candidate
-// ranked strictly after the previous winner (value descending, lower index on
-// ties) and a 5-step butterfly leaves the warp's winner in every lane, so
-// k rounds produce the slots in order without "taken" flags.
-#include <float.h>
-
+// Selection keys.  A candidate (value v, expert e) is packed into 64 bits as
+// (order-preserving bits of v) << 32 | (0xffffffff - e), so a larger key means
+// a larger value and, on equal values, a lower index -- the tie rule.  -0.0 is
+// turned into +0.0 first so that the two compare equal.  One selection round
+// takes, per lane, the largest key below the previous winner and finds the
+// warp's largest with two redux.sync max operations (high word, then low word
+// among the lanes that hold the high maximum).  k rounds give the slots in
+// order.
+//
+// Two kernels:
+//  * lanes kernel (E = 32*V): lane l holds experts [l*V, (l+1)*V) -- one
+//    vector load per lane.  For group-limited gating whose groups cover whole
+//    lanes (E/G a multiple of V), a group is LPG = E/(G*V) neighbouring lanes:
+//    each lane takes the top-n of its own values and LPG-lane xor-shuffle
+//    merges give every lane its group's top-n, summed largest first.
+//  * generic kernel (any E <= 1024): lane l holds experts l, l+32, ...; group
+//    scores come from a per-warp shared-memory scan.
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
 namespace moe {
 namespace {
 
-constexpr int kGateWarps = 4;
-constexpr int kNone = 0x7fffffff;
+constexpr int kGateWarps = 8;
+constexpr int kMaxTopn = 4;
 
-// (va, ia) is ranked before (vb, ib): larger value first, lower index on ties.
-__device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
+// Order-preserving map of a float onto uint32 (larger float -> larger code).
+__device__ __forceinline__ uint32_t ord32(float v) {
+  const uint32_t b = __float_as_uint(__fadd_rn(v, 0.0f));  // -0 -> +0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float from_ord32(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+__device__ __forceinline__ uint64_t make_key(float v, int e) {
+  return (static_cast<uint64_t>(ord32(v)) << 32) | (0xffffffffu - static_cast<uint32_t>(e));
+}
+__device__ __forceinline__ int key_index(uint64_t key) {
+  return static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));  // sentinel 0 -> -1
+}
+__device__ __forceinline__ float key_value(uint64_t key) {
+  return from_ord32(static_cast<uint32_t>(key >> 32));
 }
 
-__device__ __forceinline__ void warp_best(float& bv, int& bi) {
+// Largest key of the warp (all lanes get it).  Key 0 means "no candidate".
+__device__ __forceinline__ uint64_t warp_max_key(uint64_t key) {
+  const uint32_t hi = __reduce_max_sync(kFullMask, static_cast<uint32_t>(key >> 32));
+  const uint32_t lo =
+      __reduce_max_sync(kFullMask, static_cast<uint32_t>(key >> 32) == hi ? static_cast<uint32_t>(key) : 0u);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_key(uint64_t key, int m) {
+  const uint32_t hi = __shfl_xor_sync(kFullMask, static_cast<uint32_t>(key >> 32), m);
+  const uint32_t lo = __shfl_xor_sync(kFullMask, static_cast<uint32_t>(key), m);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_key(uint64_t key, int src) {
+  const uint32_t hi = __shfl_sync(kFullMask, static_cast<uint32_t>(key >> 32), src);
+  const uint32_t lo = __shfl_sync(kFullMask, static_cast<uint32_t>(key), src);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+// k selection rounds over the lane's keys (key 0 = not a candidate).  Lane j
+// receives slot j; every lane gets the slot-order sum of the winners' values.
+template <int V>
+__device__ __forceinline__ void select_topk(const uint64_t (&key)[V], int k, int lane, int& sel_i,
+                                            float& sel_v, float& sum) {
+  uint64_t prev = ~0ull;
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = 0;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const float ov = __shfl_xor_sync(kFullMask, bv, off);
-    const int oi = __shfl_xor_sync(kFullMask, bi, off);
-    if (oi != kNone && (bi == kNone || ranks_before(ov, oi, bv, bi))) {
-      bv = ov;
-      bi = oi;
+    for (int v = 0; v < V; ++v)
+      if (key[v] < prev && key[v] > best) best = key[v];
+    const uint64_t win = warp_max_key(best);
+    const float wv = key_value(win);
+    sum = (j == 0) ? wv : __fadd_rn(sum, wv);
+    if (lane == j) {
+      sel_i = key_index(win);
+      sel_v = wv;
+    }
+    prev = win;
+  }
+}
+
+// ------------------------------------------------------------------ lanes kernel
+// Softmax needs Z summed in ascending expert order: the exp terms go to shared
+// memory and lane 0 adds them one by one.
+template <int V, int TOPN>
+__global__ void __launch_bounds__(kGateWarps * 32)
+    topk_gate_lanes_kernel(const float* __restrict__ logits, int N, int k, int kind, int LPG_log2,
+                           int TG, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  constexpr int E = 32 * V;
+  constexpr int topn = TOPN;  // group score = sum of the TOPN best scores of a group
+  __shared__ float sh_exp[kGateWarps][E];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int e0 = lane * V;
+
+  for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
+    const float* row = logits + static_cast<size_t>(t) * E + e0;
+    float l[V];
+    if constexpr (V % 4 == 0) {
+#pragma unroll
+      for (int q = 0; q < V / 4; ++q) {
+        const float4 f = reinterpret_cast<const float4*>(row)[q];
+        l[4 * q] = f.x;
+        l[4 * q + 1] = f.y;
+        l[4 * q + 2] = f.z;
+        l[4 * q + 3] = f.w;
+      }
+    } else if constexpr (V == 2) {
+      const float2 f = *reinterpret_cast<const float2*>(row);
+      l[0] = f.x;
+      l[1] = f.y;
+    } else {
+      l[0] = row[0];
+    }
+    uint64_t key[V];
+    int sel_i = -1;
+    float sel_v = 0.0f, sum = 0.0f;
+
+    if (kind == MOE_GATE_SIGMOID_GROUP) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) key[v] = make_key(logistic(l[v]), e0 + v);
+      // this lane's top-n, best first (key 0 pads when n > V)
+      uint64_t top[topn];
+      uint64_t prev = ~0ull;
+#pragma unroll
+      for (int p = 0; p < topn; ++p) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+          if (key[v] < prev && key[v] > best) best = key[v];
+        top[p] = best;
+        prev = best;
+      }
+      // merge with the other lanes of the group: top-n of two sorted lists is
+      // max(a_i, b_{n-1-i}) (a bitonic sequence), then sorted again
+#pragma unroll
+      for (int step = 0; step < 5; ++step) {  // LPG <= 32 lanes: at most 5 merges
+        if (step >= LPG_log2) break;            // warp-uniform
+        const int m = 1 << step;
+        uint64_t other[topn], mrg[topn];
+#pragma unroll
+        for (int p = 0; p < topn; ++p) other[p] = shfl_xor_key(top[p], m);
+#pragma unroll
+        for (int p = 0; p < topn; ++p) mrg[p] = top[p] > other[topn - 1 - p] ? top[p] : other[topn - 1 - p];
+        // sort the merged keys, largest first
+#pragma unroll
+        for (int a = 0; a < topn; ++a)
+#pragma unroll
+          for (int b = topn - 1; b > a; --b)
+            if (mrg[b] > mrg[b - 1]) {
+              const uint64_t tmp = mrg[b];
+              mrg[b] = mrg[b - 1];
+              mrg[b - 1] = tmp;
+            }
+#pragma unroll
+        for (int p = 0; p < topn; ++p) top[p] = mrg[p];
+      }
+      float gscore = key_value(top[0]);
+#pragma unroll
+      for (int p = 1; p < topn; ++p) gscore = __fadd_rn(gscore, key_value(top[p]));
+      // rank of this lane's group among all groups (group h leads lanes h*LPG..)
+      const int g = lane >> LPG_log2;
+      const int G = 32 >> LPG_log2;
+      const uint64_t gkey = make_key(gscore, g);
+      int before = 0;
+      for (int h = 0; h < G; ++h) before += shfl_key(gkey, h << LPG_log2) > gkey ? 1 : 0;
+      if (before >= TG) {
+#pragma unroll
+        for (int v = 0; v < V; ++v) key[v] = 0;
+      }
+      select_topk<V>(key, k, lane, sel_i, sel_v, sum);
+      if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
+    } else {
+      float m = l[0];
+#pragma unroll
+      for (int v = 1; v < V; ++v) m = fmaxf(m, l[v]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
+#pragma unroll
+      for (int v = 0; v < V; ++v) {
+        sh_exp[warp][e0 + v] = fixed_exp(__fsub_rn(l[v], m));
+        key[v] = make_key(l[v], e0 + v);
+      }
+      __syncwarp();
+      float z = 0.0f;
+      if (lane == 0)
+        for (int i = 0; i < E; ++i) z = __fadd_rn(z, sh_exp[warp][i]);
+      z = __shfl_sync(kFullMask, z, 0);
+      uint64_t prev = ~0ull;
+      for (int j = 0; j < k; ++j) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int v = 0; v < V; ++v)
+          if (key[v] < prev && key[v] > best) best = key[v];
+        const uint64_t win = warp_max_key(best);
+        const int wi = key_index(win);
+        const float p = (wi >= 0 && wi < E) ? __fdiv_rn(sh_exp[warp][wi], z) : 0.0f;
+        sum = (j == 0) ? p : __fadd_rn(sum, p);
+        if (lane == j) {
+          sel_i = (wi >= 0 && wi < E) ? wi : -1;
+          sel_v = p;
+        }
+        prev = win;
+      }
+      if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
+      __syncwarp();  // sh_exp is rewritten for the next token
+    }
+    if (lane < k) {
+      topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
+      topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
     }
   }
 }
 
+// ------------------------------------------------------------------ generic kernel
 // Per-warp shared memory: vals[E] (scores or exp terms), gscore[G], gkeep[G].
 template <int V>
 __global__ void __launch_bounds__(kGateWarps * 32)
-    topk_gate_kernel(const float* __restrict__ logits, int N, int E, int k, int kind, int G,
-                     int TG, int topn, int32_t* __restrict__ topk_idx,
-                     float* __restrict__ topk_w) {
+    topk_gate_generic_kernel(const float* __restrict__ logits, int N, int E, int k, int kind,
+                             int G, int TG, int topn, int32_t* __restrict__ topk_idx,
+                             float* __restrict__ topk_w) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -56,133 +242,103 @@ __global__ void __launch_bounds__(kGateWarps * 32)
 
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
     const float* row = logits + static_cast<size_t>(t) * E;
-    float key[V];
+    float l[V];
+    uint64_t key[V];
 #pragma unroll
     for (int v = 0; v < V; ++v) {
       const int e = v * 32 + lane;
-      key[v] = e < E ? row[e] : 0.0f;
+      l[v] = e < E ? row[e] : 0.0f;
     }
     int sel_i = -1;
-    float sel_v = 0.0f;
-    float sum_sel = 0.0f;
+    float sel_v = 0.0f, sum = 0.0f;
 
     if (kind == MOE_GATE_SIGMOID_GROUP) {
 #pragma unroll
       for (int v = 0; v < V; ++v) {
         const int e = v * 32 + lane;
         if (e < E) {
-          key[v] = logistic(key[v]);
-          vals[e] = key[v];
+          const float s = logistic(l[v]);
+          vals[e] = s;
+          key[v] = make_key(s, e);
+        } else {
+          key[v] = 0;
         }
       }
       __syncwarp();
       // group score: the topn best scores of the group, added best first
       for (int g = lane; g < G; g += 32) {
         const float* gv = vals + g * eg;
-        float pv = INFINITY, sum = 0.0f;
-        int pi = -1;
+        uint64_t prev = ~0ull;
+        float gs = 0.0f;
         for (int p = 0; p < topn; ++p) {
-          float bv = 0.0f;
-          int bi = kNone;
+          uint64_t best = 0;
           for (int i = 0; i < eg; ++i) {
-            const float v = gv[i];
-            if (ranks_before(pv, pi, v, i) && (bi == kNone || ranks_before(v, i, bv, bi))) {
-              bv = v;
-              bi = i;
-            }
+            const uint64_t kv = make_key(gv[i], i);
+            if (kv < prev && kv > best) best = kv;
           }
-          sum = (p == 0) ? bv : __fadd_rn(sum, bv);
-          pv = bv;
-          pi = bi;
+          gs = (p == 0) ? key_value(best) : __fadd_rn(gs, key_value(best));
+          prev = best;
         }
-        gscore[g] = sum;
+        gscore[g] = gs;
       }
       __syncwarp();
       // a group is kept when fewer than TG groups rank before it
       for (int g = lane; g < G; g += 32) {
-        const float s = gscore[g];
+        const uint64_t mine = make_key(gscore[g], g);
         int before = 0;
-        for (int h = 0; h < G; ++h) before += ranks_before(gscore[h], h, s, g) ? 1 : 0;
+        for (int h = 0; h < G; ++h) before += make_key(gscore[h], h) > mine ? 1 : 0;
         gkeep[g] = before < TG;
       }
       __syncwarp();
-      bool cand[V];
 #pragma unroll
       for (int v = 0; v < V; ++v) {
         const int e = v * 32 + lane;
-        cand[v] = e < E && gkeep[e / eg] != 0;
+        if (e < E && !gkeep[e / eg]) key[v] = 0;
       }
-      float pv = INFINITY;
-      int pi = -1;
-      for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int bi = kNone;
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-          const int e = v * 32 + lane;
-          if (cand[v] && ranks_before(pv, pi, key[v], e) &&
-              (bi == kNone || ranks_before(key[v], e, bv, bi))) {
-            bv = key[v];
-            bi = e;
-          }
-        }
-        warp_best(bv, bi);
-        sum_sel = (j == 0) ? bv : __fadd_rn(sum_sel, bv);
-        if (lane == j) {
-          sel_i = bi;
-          sel_v = bv;
-        }
-        pv = bv;
-        pi = bi;
-      }
-      if (lane < k) sel_v = __fdiv_rn(sel_v, sum_sel);
+      select_topk<V>(key, k, lane, sel_i, sel_v, sum);
+      if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
     } else {
-      // softmax: m = max logit, e_i = exp(l_i - m), Z summed in expert order
       float m = -INFINITY;
 #pragma unroll
       for (int v = 0; v < V; ++v)
-        if (v * 32 + lane < E) m = fmaxf(m, key[v]);
+        if (v * 32 + lane < E) m = fmaxf(m, l[v]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
 #pragma unroll
       for (int v = 0; v < V; ++v) {
         const int e = v * 32 + lane;
-        if (e < E) vals[e] = fixed_exp(__fsub_rn(key[v], m));
+        if (e < E) {
+          vals[e] = fixed_exp(__fsub_rn(l[v], m));
+          key[v] = make_key(l[v], e);
+        } else {
+          key[v] = 0;
+        }
       }
       __syncwarp();
       float z = 0.0f;
       if (lane == 0)
         for (int i = 0; i < E; ++i) z = __fadd_rn(z, vals[i]);
       z = __shfl_sync(kFullMask, z, 0);
-      float pv = INFINITY;
-      int pi = -1;
+      uint64_t prev = ~0ull;
       for (int j = 0; j < k; ++j) {
-        float bv = 0.0f;
-        int bi = kNone;
+        uint64_t best = 0;
 #pragma unroll
-        for (int v = 0; v < V; ++v) {
-          const int e = v * 32 + lane;
-          if (e < E && ranks_before(pv, pi, key[v], e) &&
-              (bi == kNone || ranks_before(key[v], e, bv, bi))) {
-            bv = key[v];
-            bi = e;
-          }
-        }
-        warp_best(bv, bi);
+        for (int v = 0; v < V; ++v)
+          if (key[v] < prev && key[v] > best) best = key[v];
+        const uint64_t win = warp_max_key(best);
+        const int wi = key_index(win);
         // only NaN logits can leave a round without a candidate
-        const float p = bi == kNone ? 0.0f : __fdiv_rn(vals[bi], z);
-        sum_sel = (j == 0) ? p : __fadd_rn(sum_sel, p);
+        const float p = (wi >= 0 && wi < E) ? __fdiv_rn(vals[wi], z) : 0.0f;
+        sum = (j == 0) ? p : __fadd_rn(sum, p);
         if (lane == j) {
-          sel_i = bi;
+          sel_i = (wi >= 0 && wi < E) ? wi : -1;
           sel_v = p;
         }
-        pv = bv;
-        pi = bi;
+        prev = win;
       }
-      if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum_sel);
+      if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
     }
     if (lane < k) {
-      if (sel_i == kNone) sel_i = -1;
       topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
       topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
     }
@@ -190,21 +346,50 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   }
 }
 
+unsigned grid_for(int N) {
+  int blocks = (N + kGateWarps - 1) / kGateWarps;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  return static_cast<unsigned>(blocks);
+}
+
 template <int V>
-cudaError_t launch_v(const float* logits, int N, int E, int k, int kind, int G, int TG, int topn,
-                     int32_t* idx, float* w, cudaStream_t stream) {
+cudaError_t launch_generic(const float* logits, int N, int E, int k, int kind, int G, int TG,
+                           int topn, int32_t* idx, float* w, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(kGateWarps) * (E + 2 * G) * sizeof(float);
   if (smem > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(topk_gate_kernel<V>,
+    cudaError_t err = cudaFuncSetAttribute(topk_gate_generic_kernel<V>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  int blocks = (N + kGateWarps - 1) / kGateWarps;
-  if (blocks > 148 * 64) blocks = 148 * 64;
-  topk_gate_kernel<V><<<blocks, kGateWarps * 32, smem, stream>>>(logits, N, E, k, kind, G, TG,
-                                                                  topn, idx, w);
+  topk_gate_generic_kernel<V><<<grid_for(N), kGateWarps * 32, smem, stream>>>(
+      logits, N, E, k, kind, G, TG, topn, idx, w);
   return cudaGetLastError();
+}
+
+template <int V, int TOPN>
+cudaError_t launch_lanes_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
+                           int32_t* idx, float* w, cudaStream_t stream) {
+  topk_gate_lanes_kernel<V, TOPN><<<grid_for(N), kGateWarps * 32, 0, stream>>>(
+      logits, N, k, kind, lpg_log2, TG, idx, w);
+  return cudaGetLastError();
+}
+
+template <int V>
+cudaError_t launch_lanes(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
+                         int topn, int32_t* idx, float* w, cudaStream_t stream) {
+  switch (topn) {
+    case 1: return launch_lanes_n<V, 1>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
+    case 2: return launch_lanes_n<V, 2>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
+    case 3: return launch_lanes_n<V, 3>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
+    default: return launch_lanes_n<V, 4>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
+  }
+}
+
+int log2_exact(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return (1 << r) == x ? r : -1;
 }
 
 }  // namespace
@@ -215,13 +400,33 @@ cudaError_t launch_topk_gate(const float* logits, int N, int E, int k, int kind,
   if (N == 0) return cudaSuccess;
   int G = n_groups, TG = topk_groups, topn = group_topn;
   if (kind != MOE_GATE_SIGMOID_GROUP) G = TG = topn = 1;
+
+  // lanes kernel: E = 32*V with V a power of two up to 8, 16-byte aligned rows,
+  // and (group kind) groups made of whole lanes with topn <= 4
+  const int V = E / 32;
+  bool lanes = E % 32 == 0 && log2_exact(V) >= 0 && V <= 8 &&
+               (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+  int lpg_log2 = 0;
+  if (lanes && kind == MOE_GATE_SIGMOID_GROUP) {
+    const int eg = E / G;
+    lpg_log2 = (eg % V == 0) ? log2_exact(eg / V) : -1;
+    lanes = lpg_log2 >= 0 && topn <= kMaxTopn;
+  }
+  if (lanes) {
+    switch (V) {
+      case 1: return launch_lanes<1>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
+      case 2: return launch_lanes<2>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
+      case 4: return launch_lanes<4>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
+      default: return launch_lanes<8>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
+    }
+  }
   const int per_lane = (E + 31) / 32;
-  if (per_lane <= 1) return launch_v<1>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 2) return launch_v<2>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 4) return launch_v<4>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 8) return launch_v<8>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 16) return launch_v<16>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  return launch_v<32>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  if (per_lane <= 1) return launch_generic<1>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  if (per_lane <= 2) return launch_generic<2>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  if (per_lane <= 4) return launch_generic<4>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  if (per_lane <= 8) return launch_generic<8>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  if (per_lane <= 16) return launch_generic<16>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  return launch_generic<32>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
 }
 
 }  // namespace moe

@@ -140,10 +140,22 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x;
 
-  // 1. column sums over chunks: all chunks (totals) and chunks before c
+  // 1. column sums over chunks: all chunks (totals) and chunks before c.
+  //    Loads go out 8 chunks at a time so one L2 round trip covers 8 chunks.
   for (int b = tid; b < nb; b += kLayoutThreads) {
     int before = 0, total = 0;
-    for (int cc = 0; cc < C; ++cc) {
+    int cc = 0;
+    for (; cc + 8 <= C; cc += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[static_cast<size_t>(cc + u) * nb + b];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        total += v[u];
+        before += (cc + u) < c ? v[u] : 0;
+      }
+    }
+    for (; cc < C; ++cc) {
       const int v = chunk_counts[static_cast<size_t>(cc) * nb + b];
       total += v;
       before += cc < c ? v : 0;
@@ -165,6 +177,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
       rank_offset[r] = off[r * epr];
       rank_count[r] = off[(r + 1) * epr] - off[r * epr];
       int rt = 0;
+#pragma unroll 8
       for (int cc = 0; cc < C; ++cc) rt += chunk_rtok[static_cast<size_t>(cc) * R + r];
       rank_tokens[r] = rt;
     }

@@ -33,7 +33,10 @@
  *  - Device-side errors: an index found out of range by a kernel is skipped
  *    and, when `d_status` is not NULL, MOE_ERR_BAD_INDEX is stored to
  *    *d_status (one int32 in device memory that the caller zeroes and reads
- *    after the stream work finished).  No kernel traps or asserts.
+ *    after the stream work finished).  No kernel traps or asserts.  Kernels
+ *    that wait on in-flight copies bound every wait to one second; a wait
+ *    that runs out stores MOE_ERR_TIMEOUT, lets the copies it issued land
+ *    and returns (its output is then incomplete).
  *  - Sizes: N = num_tokens, H = hidden, E = num_experts, k = experts per
  *    token, R = logical EP ranks, S = N*k receive rows.  Row-major layouts.
  *    Byte offsets are 64-bit; S must stay below 2^31 (int32 slot ids).
@@ -55,7 +58,8 @@ typedef enum {
     MOE_ERR_INVALID_ARG = 1,
     MOE_ERR_UNSUPPORTED = 2,
     MOE_ERR_CUDA = 3,
-    MOE_ERR_BAD_INDEX = 4
+    MOE_ERR_BAD_INDEX = 4,
+    MOE_ERR_TIMEOUT = 5          /* a kernel's bounded wait gave up (device status only) */
 } moe_status_t;
 
 typedef enum {
