@@ -268,7 +268,19 @@ def run_ours(args, rank, world, device):
     out = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
     y = recv if w.expert_out == "identity" else y_in
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+    flush_r = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=device)
+
+    class _Flush:
+        # write a buffer of twice the L2 size (evicts every line), then read
+        # another one (so the lines left behind are clean, not dirty lines the
+        # next step would have to write back)
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            flush_r.max()
+
+    flush = _Flush()
 
     def step(ev=None):
         stream = torch.cuda.current_stream(device)  # the capture stream inside torch.cuda.graph
@@ -291,16 +303,26 @@ def run_ours(args, rank, world, device):
     if int(L.status.item()) != 0:
         raise RuntimeError(f"device status {int(L.status.item())} after warm-up")
 
-    # The step is captured once as a CUDA graph (event-record nodes between the
-    # ops) and replayed, so the timed interval is device time of the 5 kernels
-    # back to back, not the Python binding's launch overhead.
+    # The step is captured once as a CUDA graph and replayed, so the timed
+    # interval is device time of the 5 kernels back to back (their launches
+    # overlap through programmatic dependent launch), not the Python binding's
+    # launch overhead.  graph_step has events only at its ends and gives the
+    # step time; graph_ops has an event-record node between the ops (which
+    # also cuts the launch overlap) and gives the per-op breakdown.
+    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+    graph_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_step):
+        ends[0].record(torch.cuda.current_stream(device))
+        step()
+        ends[1].record(torch.cuda.current_stream(device))
     evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
+    graph_ops = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_ops):
         step(evs)
     for _ in range(args.warmup):
-        flush.zero_()
-        graph.replay()
+        for g in (graph_step, graph_ops):
+            flush.zero_()
+            g.replay()
     torch.cuda.synchronize(device)
     per_op = {n: [] for n in ("gate", "layout", "dispatch", "combine")}
     step_ms = []
@@ -310,11 +332,15 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device.index) as clk:
         for i in range(args.steps):
             flush.zero_()
-            graph.replay()
+            graph_step.replay()
+            ends[1].synchronize()
+            step_ms.append(ends[0].elapsed_time(ends[1]))
+        for i in range(args.steps):
+            flush.zero_()
+            graph_ops.replay()
             evs[4].synchronize()
             for j, n in enumerate(per_op):
                 per_op[n].append(evs[j].elapsed_time(evs[j + 1]))
-            step_ms.append(evs[0].elapsed_time(evs[4]))
         torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
@@ -349,16 +375,18 @@ def run_ours(args, rank, world, device):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": describe(w), "tokens_per_gpu": w.N, "hidden": w.H, "experts": w.E,
                    "topk": w.k, "logical_ranks": w.R, "payload": f"x bf16, dispatch {w.dtype}, out bf16",
-                   "l2": "flushed before every step (write of 2x L2 size, outside the events)",
-                   "timing": "one step captured as a CUDA graph, replayed per step; CUDA events "
-                             "(graph event-record nodes) between the ops",
+                   "l2": "flushed before every step, outside the events: a write of 2x the L2 size, "
+                         "then a read of another 2x L2 buffer (the step starts cold and clean)",
+                   "timing": "step captured once as a CUDA graph and replayed; step time from events "
+                             "at the graph's ends, per-op times from a second graph with event nodes "
+                             "between the ops",
                    "parallelism": f"replicas x{world} (tokens sharded, no collective)"},
         "per_op_us": {n: 1e3 * v for n, v in avg.items()},
         "per_op_gbs": gbs,
         "dispatch_combine_tokens_per_s": w.N * world / ((avg["dispatch"] + avg["combine"]) * 1e-3),
         "roofline": roof(dominant),
         "roofline_other": roof(other),
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": 10 * args.steps,  # 5 kernels per replay, two timed loops
         "clocks": clk.summary(),
         "e2e": e2e,
     }

@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kThreads)
     mbar_init_fence();
   }
   __syncthreads();
+  pdl_wait();  // everything above touched shared memory only
+  pdl_trigger();
 
   const int segs = (H + kSeg - 1) / kSeg;
   const long long items = static_cast<long long>(N) * segs;
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kThreads)
         o.y = pack_bf16x2(acc[2], acc[3]);
         o.z = pack_bf16x2(acc[4], acc[5]);
         o.w = pack_bf16x2(acc[6], acc[7]);
-        st_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * kSeg + c, o);
+        st_stream_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * kSeg + c, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(stage));
@@ -220,10 +222,9 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
   if (per_sm < 1) per_sm = 1;
   const long long items = static_cast<long long>(N) * ((H + kSeg - 1) / kSeg);
   const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
-  combine_bulk_kernel<<<static_cast<unsigned>(grid), kThreads, L.total, stream>>>(
-      static_cast<const uint16_t*>(y), N, H, k, token_slot, topk_w, static_cast<uint16_t*>(out),
-      d_status);
-  return cudaGetLastError();
+  return launch_pdl(combine_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total, stream,
+                    static_cast<const uint16_t*>(y), N, H, k, token_slot, topk_w,
+                    static_cast<uint16_t*>(out), d_status);
 }
 
 }  // namespace moe

@@ -36,6 +36,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const bool active = c0 < H;  // H % 128 == 0: whole 8-lane blocks are in or out
   const long long S = static_cast<long long>(N) * k;
   const int nblk = H / 128;
+  pdl_wait();
+  pdl_trigger();
 
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
   uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
@@ -79,7 +81,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       continue;
     }
     if (active) {
-      st_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
+      st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
       if ((lane & 7) == 0) recv_scale[static_cast<size_t>(slot) * nblk + (c0 >> 7)] = scale;
     }
   }
@@ -99,6 +101,8 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int c0 = s * 256 + lane * 8;
   const bool active = c0 < H;  // H % 8 == 0
   const long long S = static_cast<long long>(N) * k;
+  pdl_wait();
+  pdl_trigger();
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
   uint4 v = make_uint4(0, 0, 0, 0);
   if (active) v = ld_stream(x + static_cast<size_t>(t) * H + c0);
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (lane == 0) report_bad_index(d_status);
       continue;
     }
-    if (active) st_v4(recv_x + static_cast<size_t>(slot) * H + c0, v);
+    if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, v);
   }
 }
 
@@ -135,18 +139,16 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   if (dtype == MOE_DTYPE_FP8_E4M3) {
     const long long items = static_cast<long long>(N) * ((H + 511) / 512);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-    dispatch_fp8_kernel<<<blocks, kWarps * 32, 0, stream>>>(
-        static_cast<const uint16_t*>(x), N, H, k, token_slot, static_cast<uint8_t*>(recv_x),
-        recv_scale, d_status);
+    return launch_pdl(dispatch_fp8_kernel, blocks, kWarps * 32, 0, stream,
+                      static_cast<const uint16_t*>(x), N, H, k, token_slot,
+                      static_cast<uint8_t*>(recv_x), recv_scale, d_status);
   } else {
     const long long items = static_cast<long long>(N) * ((H + 255) / 256);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-    dispatch_bf16_kernel<<<blocks, kWarps * 32, 0, stream>>>(static_cast<const uint16_t*>(x), N,
-                                                            H, k, token_slot,
-                                                            static_cast<uint16_t*>(recv_x),
-                                                            d_status);
+    return launch_pdl(dispatch_bf16_kernel, blocks, kWarps * 32, 0, stream,
+                      static_cast<const uint16_t*>(x), N, H, k, token_slot,
+                      static_cast<uint16_t*>(recv_x), d_status);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream) {

@@ -105,6 +105,8 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int e0 = lane * V;
+  pdl_wait();
+  pdl_trigger();
 
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
     const float* row = logits + static_cast<size_t>(t) * E + e0;
@@ -239,6 +241,8 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   float* gscore = vals + E;
   int* gkeep = reinterpret_cast<int*>(gscore + G);
   const int eg = E / G;
+  pdl_wait();
+  pdl_trigger();
 
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
     const float* row = logits + static_cast<size_t>(t) * E;
@@ -362,17 +366,15 @@ cudaError_t launch_generic(const float* logits, int N, int E, int k, int kind, i
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  topk_gate_generic_kernel<V><<<grid_for(N), kGateWarps * 32, smem, stream>>>(
-      logits, N, E, k, kind, G, TG, topn, idx, w);
-  return cudaGetLastError();
+  return launch_pdl(topk_gate_generic_kernel<V>, grid_for(N), kGateWarps * 32, smem, stream, logits,
+                    N, E, k, kind, G, TG, topn, idx, w);
 }
 
 template <int V, int TOPN>
 cudaError_t launch_lanes_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
                            int32_t* idx, float* w, cudaStream_t stream) {
-  topk_gate_lanes_kernel<V, TOPN><<<grid_for(N), kGateWarps * 32, 0, stream>>>(
-      logits, N, k, kind, lpg_log2, TG, idx, w);
-  return cudaGetLastError();
+  return launch_pdl(topk_gate_lanes_kernel<V, TOPN>, grid_for(N), kGateWarps * 32, 0, stream,
+                    logits, N, k, kind, lpg_log2, TG, idx, w);
 }
 
 template <int V>

@@ -8,14 +8,16 @@
 // block counts the tokens bound for each destination; Sharding: experts split
 // over EP ranks (here partitions of one buffer).
 //
-// Two launches, no atomics on the order and no spin waits:
+// Two launches, no atomics on the order and no spin waits.  Entries with the
+// same bucket inside a warp are found with one ballot per bucket bit
+// (warp_match), which on B200 costs far less than __match_any_sync:
 //   count:  one CTA per chunk of whole tokens (<= 1024 entries); per-chunk
 //           histogram over E+1 buckets (bucket E = masked/invalid entries,
 //           which fill the tail rows) and per-chunk per-rank token counts.
 //   assign: one CTA per chunk again; every CTA sums the histograms of the
 //           chunks before it and of all chunks (column sums, from L2), scans
 //           the totals into expert offsets, ranks its entries inside the
-//           chunk (warp __match_any_sync + popc, then a prefix over the 32
+//           chunk (warp_match + popc, then a prefix over the 32
 //           warps) and writes token_slot / slot_token.  CTA 0 writes the
 //           counts and offsets.  The row of entry (t, j) in expert e is the
 //           number of entries routed to e before it in (t, j) order, so the
@@ -56,8 +58,11 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const long long t0 = static_cast<long long>(c) * tc;
   const int nt = static_cast<int>(min(static_cast<long long>(tc), N - t0));
   const int ne = nt > 0 ? nt * k : 0;
+  const int nbits = 32 - __clz(E + 1);  // bucket + 1 lies in [0, E + 1]
   for (int i = tid; i <= E; i += kLayoutThreads) hist[i] = 0;
   for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  pdl_wait();
+  pdl_trigger();
   int e = -1;
   if (tid < ne) {
     e = topk_idx[t0 * k + tid];
@@ -67,7 +72,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int b = tid < ne ? bucket_of(e, E) : -1;
   if (tid < ne && b == E && e != -1) report_bad_index(d_status);
   // one shared-memory add per distinct bucket in the warp
-  const unsigned same = __match_any_sync(kFullMask, b);
+  const unsigned same = warp_match(static_cast<unsigned>(b + 1), nbits);
   if (b >= 0 && (same & lanemask_lt()) == 0) atomicAdd(&hist[b], __popc(same));
   if (b >= 0 && b < E) {
     // the token's first slot landing on this rank counts the token once
@@ -137,53 +142,14 @@ __global__ void __launch_bounds__(kLayoutThreads)
   int32_t* base = off + nb;          // nb: first row of this chunk per bucket
   int32_t* wcnt = base + nb;         // kLayoutWarps * nb
   int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
+  int32_t* rtok = warp_sums + 32;                 // R (CTA 0: tokens per rank)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x;
+  const int nbits = 32 - __clz(E + 1);
+  pdl_wait();
+  pdl_trigger();
 
-  // 1. column sums over chunks: all chunks (totals) and chunks before c.
-  //    Loads go out 8 chunks at a time so one L2 round trip covers 8 chunks.
-  for (int b = tid; b < nb; b += kLayoutThreads) {
-    int before = 0, total = 0;
-    int cc = 0;
-    for (; cc + 8 <= C; cc += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = chunk_counts[static_cast<size_t>(cc + u) * nb + b];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        total += v[u];
-        before += (cc + u) < c ? v[u] : 0;
-      }
-    }
-    for (; cc < C; ++cc) {
-      const int v = chunk_counts[static_cast<size_t>(cc) * nb + b];
-      total += v;
-      before += cc < c ? v : 0;
-    }
-    off[b] = total;
-    base[b] = before;
-  }
-  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
-  __syncthreads();
-  if (c == 0)
-    for (int e = tid; e < E; e += kLayoutThreads) expert_count[e] = off[e];
-  // 2. bucket offsets
-  block_exclusive_scan(off, nb, warp_sums);
-  for (int b = tid; b < nb; b += kLayoutThreads) base[b] += off[b];
-  if (c == 0) {
-    const int epr = E / R;
-    for (int e = tid; e <= E; e += kLayoutThreads) expert_offset[e] = off[e];
-    for (int r = tid; r < R; r += kLayoutThreads) {
-      rank_offset[r] = off[r * epr];
-      rank_count[r] = off[(r + 1) * epr] - off[r * epr];
-      int rt = 0;
-#pragma unroll 8
-      for (int cc = 0; cc < C; ++cc) rt += chunk_rtok[static_cast<size_t>(cc) * R + r];
-      rank_tokens[r] = rt;
-    }
-    if (tid == 0) rank_offset[R] = off[E];
-  }
-  // 3. ranks inside the chunk
+  // this CTA's entries are loaded first so their latency overlaps the sums
   const int tc = tokens_per_chunk(k);
   const long long t0 = static_cast<long long>(c) * tc;
   const int nt = static_cast<int>(min(static_cast<long long>(tc), N - t0));
@@ -193,17 +159,73 @@ __global__ void __launch_bounds__(kLayoutThreads)
     e = topk_idx[t0 * k + tid];
     b = bucket_of(e, E);
   }
-  const unsigned same = __match_any_sync(kFullMask, b);
+  // 1. column sums over chunks: all chunks (totals) and chunks before c.  All
+  //    threads load the C x nb counts in one pass (one L2 round trip) and add
+  //    them into shared memory.
+  for (int i = tid; i < nb; i += kLayoutThreads) off[i] = base[i] = 0;
+  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
+  for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  __syncthreads();
+  if (c == 0) {  // block-uniform: CTA 0 also sums the per-chunk tokens per rank
+    const int total_vals = C * R;
+    for (int i = tid; i < total_vals; i += kLayoutThreads) {
+      const int v = chunk_rtok[i];
+      if (v != 0) atomicAdd(&rtok[i % R], v);
+    }
+  }
+  {
+    const int total_vals = C * nb;
+    constexpr int kBatch = 16;
+    for (int i0 = 0; i0 < total_vals; i0 += kBatch * kLayoutThreads) {
+      int v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kLayoutThreads + tid;
+        v[u] = i < total_vals ? chunk_counts[i] : 0;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kLayoutThreads + tid;
+        if (v[u] != 0) {
+          const int cc = i / nb, bb = i - cc * nb;
+          atomicAdd(&off[bb], v[u]);
+          if (cc < c) atomicAdd(&base[bb], v[u]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (c == 0)
+    for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = off[i];
+  // 2. bucket offsets
+  block_exclusive_scan(off, nb, warp_sums);
+  for (int i = tid; i < nb; i += kLayoutThreads) base[i] += off[i];
+  if (c == 0) {
+    const int epr = E / R;
+    for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
+    for (int r = tid; r < R; r += kLayoutThreads) {
+      rank_offset[r] = off[r * epr];
+      rank_count[r] = off[(r + 1) * epr] - off[r * epr];
+      rank_tokens[r] = rtok[r];
+    }
+    if (tid == 0) rank_offset[R] = off[E];
+  }
+  // 3. ranks inside the chunk
+  const unsigned same = warp_match(static_cast<unsigned>(b + 1), nbits);
   const int in_warp = __popc(same & lanemask_lt());
   if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
   __syncthreads();
-  for (int bb = tid; bb < nb; bb += kLayoutThreads) {
-    int run = 0;
-    for (int w = 0; w < kLayoutWarps; ++w) {
-      const int v = wcnt[w * nb + bb];
-      wcnt[w * nb + bb] = run;
-      run += v;
+  // exclusive prefix over the 32 warps of every bucket: one warp per bucket
+  // at a time, lane w holding warp w's count
+  for (int bb = warp; bb < nb; bb += kLayoutWarps) {
+    const int v = wcnt[lane * nb + bb];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFullMask, incl, o);
+      if (lane >= o) incl += y;
     }
+    wcnt[lane * nb + bb] = incl - v;
   }
   __syncthreads();
   if (tid < ne) {
@@ -244,7 +266,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
   int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
   const size_t smem_count = (static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
   const size_t smem_assign =
-      (2 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32) *
+      (2 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
       sizeof(int32_t);
   cudaError_t err;
   if (smem_count > 48 * 1024) {
@@ -257,14 +279,12 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
                                static_cast<int>(smem_assign));
     if (err != cudaSuccess) return err;
   }
-  layout_count_kernel<<<C, kLayoutThreads, smem_count, stream>>>(topk_idx, N, k, E, R, chunk_counts,
-                                                                 chunk_rtok, d_status);
-  err = cudaGetLastError();
+  err = launch_pdl(layout_count_kernel, C, kLayoutThreads, smem_count, stream, topk_idx, N, k, E, R,
+                   chunk_counts, chunk_rtok, d_status);
   if (err != cudaSuccess) return err;
-  layout_assign_kernel<<<C, kLayoutThreads, smem_assign, stream>>>(
-      topk_idx, N, k, E, R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
-      rank_offset, rank_tokens, token_slot, slot_token, d_status);
-  return cudaGetLastError();
+  return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
+                    R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
+                    rank_offset, rank_tokens, token_slot, slot_token, d_status);
 }
 
 }  // namespace moe

@@ -94,6 +94,38 @@ __device__ __forceinline__ void st_v4(void* p, uint4 v) {
                : "memory");
 }
 
+// Streaming store: evict-first in L2, so written rows drain to DRAM while the
+// kernel still runs instead of piling up as dirty lines for the next kernel.
+__device__ __forceinline__ void st_stream_v4(void* p, uint4 v) {
+  asm volatile("st.global.cs.v4.u32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+// Lanes of the warp holding the same key (the bits of key above nbits must be
+// zero): one ballot per key bit, intersected.  On B200 this is far cheaper
+// than __match_any_sync.
+__device__ __forceinline__ unsigned warp_match(unsigned key, int nbits) {
+  unsigned peers = kFullMask;
+  for (int i = 0; i < nbits; ++i) {
+    const bool bit = (key >> i) & 1u;
+    const unsigned m = __ballot_sync(kFullMask, bit);
+    peers &= bit ? m : ~m;
+  }
+  return peers;
+}
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialisation attribute may start while its predecessor finishes;
+// pdl_wait() blocks until the predecessor's grid has completed and its writes
+// are visible, so it must come before the first global read or write.
+// pdl_trigger() lets the successor start launching.  Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void report_bad_index(int32_t* d_status) {
   if (d_status) *reinterpret_cast<volatile int32_t*>(d_status) = MOE_ERR_BAD_INDEX;
 }
@@ -179,6 +211,23 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
   return m;
+}
+
+// Launch with the programmatic stream-serialisation attribute (see pdl_wait).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
 }  // namespace moe
