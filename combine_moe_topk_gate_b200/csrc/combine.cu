@@ -8,19 +8,23 @@
 //   out[t, c] = bf16_rne(acc),  acc = +0, then acc = fmaf(w[t,j], y[slot[t,j], c], acc)
 //   for j = 0..k-1 in slot order (masked slots skipped).
 //
-// Persistent, warp-specialised CTAs.  Work item = (token, 1024-channel
-// segment); each CTA walks a contiguous range of items, so consecutive items
-// mostly share a token and its metadata.
+// Persistent, warp-specialised CTAs.  Work item = (group of T consecutive
+// tokens, 2048-channel segment) with T = max(1, 8 / k), so an item always
+// stages about 8 row segments of 4 KB whatever k is.  Each CTA walks a
+// contiguous range of items, so consecutive items mostly share a token group
+// and its metadata (the group's T*k slots and weights are contiguous).
 //   producer warp: per item, waits for a free stage of a shared-memory ring,
 //     writes the item's weights and valid-slot mask into the stage header and
 //     issues one 1-D bulk copy (cp.async.bulk, global -> shared, completing on
-//     the stage's "full" mbarrier) per valid slot row -- lane j copies row j.
-//     The next token's slots and weights are loaded one token ahead.
-//   4 consumer warps: per item, wait for "full", each thread folds its 8
-//     channels of the k staged rows in slot order, stores 16 bytes of bf16,
-//     and the warp releases the stage through its "empty" mbarrier.
-// The stages keep k * 2 KB * stages bytes per CTA in flight without any
-// registers holding them; waits are bounded (1 s, then MOE_ERR_TIMEOUT).
+//     the stage's "full" mbarrier) per valid slot row -- lane q copies row q.
+//     The next group's slots and weights are loaded one group ahead.
+//   8 consumer warps: per item, wait for "full"; each thread folds its 8
+//     channels of every token's k staged rows in slot order, stores 16 bytes
+//     of bf16 per token, and each warp releases the stage through the
+//     "empty" mbarrier.
+// Segment size, consumer warps and the ~64 KB stage budget per CTA were
+// chosen by timing variants on B200 (prefill and Mixtral shapes).  Waits are
+// bounded (1 s, then MOE_ERR_TIMEOUT).
 #include <algorithm>
 
 #include "moe_device.cuh"
@@ -29,15 +33,17 @@
 namespace moe {
 namespace {
 
-constexpr int kSeg = 1024;              // channels per work item
-constexpr int kSegBytes = kSeg * 2;     // one bf16 row segment
-constexpr int kConsumerWarps = 4;       // 128 threads x 8 channels = kSeg
+constexpr int kMaxSeg = 2048;           // channels per work item (k <= 8)
+constexpr int kConsumerWarps = 8;       // 256 threads x 8 channels = kMaxSeg
+constexpr int kStageRowsBytes = 8 * kMaxSeg * 2;  // row segments staged per item
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kHeaderBytes = 256;       // weights[32] + valid mask, per stage
 constexpr int kStageTarget = 64 * 1024; // shared bytes in flight per CTA
 constexpr int kMaxStages = 8;
 
 struct Layout {
+  int T;    // tokens per work item
+  int seg;  // channels per work item: 2048, narrower for k > 8 (32 KB per stage)
   int nstage;
   size_t stage_bytes;
   size_t bars_off, hdr_off, data_off, total;
@@ -45,7 +51,10 @@ struct Layout {
 
 __host__ __device__ inline Layout smem_layout(int k) {
   Layout L;
-  L.stage_bytes = static_cast<size_t>(k) * kSegBytes;
+  L.T = k >= 8 ? 1 : 8 / k;
+  const int rows = L.T * k;
+  L.seg = rows <= 8 ? kMaxSeg : (kStageRowsBytes / (rows * 2)) / 256 * 256;
+  L.stage_bytes = static_cast<size_t>(rows) * L.seg * 2;
   int ns = static_cast<int>(kStageTarget / L.stage_bytes);
   L.nstage = ns < 2 ? 2 : (ns > kMaxStages ? kMaxStages : ns);
   L.bars_off = 0;
@@ -55,7 +64,7 @@ __host__ __device__ inline Layout smem_layout(int k) {
   return L;
 }
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
     combine_bulk_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
                         const int32_t* __restrict__ token_slot, const float* __restrict__ topk_w,
                         uint16_t* __restrict__ out, int32_t* d_status) {
@@ -78,8 +87,12 @@ __global__ void __launch_bounds__(kThreads)
   pdl_wait();  // everything above touched shared memory only
   pdl_trigger();
 
-  const int segs = (H + kSeg - 1) / kSeg;
-  const long long items = static_cast<long long>(N) * segs;
+  const int T = L.T, TK = L.T * k;  // tokens and rows per item (TK <= 32)
+  const int seg = L.seg;
+  const uint32_t seg_bytes = static_cast<uint32_t>(seg) * 2u;
+  const int groups = (N + T - 1) / T;
+  const int segs = (H + seg - 1) / seg;
+  const long long items = static_cast<long long>(groups) * segs;
   const long long per = (items + gridDim.x - 1) / gridDim.x;
   const long long i0 = static_cast<long long>(blockIdx.x) * per;
   const long long i1 = i0 + per < items ? i0 + per : items;
@@ -91,46 +104,52 @@ __global__ void __launch_bounds__(kThreads)
     uint32_t phase = 0;
     long long issued = 0;
     bool ok = true;
-    int cur_t = -1, my_slot = -1, next_slot = -1;
+    // lane q < TK stands for row q of the group: token g*T + q/k, slot q%k;
+    // the group's entries are contiguous in token_slot / topk_w
+    const long long NK = static_cast<long long>(N) * k;
+    int cur_g = -1, my_slot = -1, next_slot = -1;
     float my_w = 0.0f, next_w = 0.0f;
     if (i0 < i1) {
-      const int t0 = static_cast<int>(i0 / segs);
-      if (lane < k) {
-        next_slot = token_slot[static_cast<size_t>(t0) * k + lane];
-        next_w = topk_w[static_cast<size_t>(t0) * k + lane];
+      const long long f = (i0 / segs) * TK + lane;
+      if (lane < TK && f < NK) {
+        next_slot = token_slot[f];
+        next_w = topk_w[f];
       }
     }
     for (long long it = i0; it < i1; ++it) {
-      const int t = static_cast<int>(it / segs);
-      const int s = static_cast<int>(it - static_cast<long long>(t) * segs);
-      if (t != cur_t) {
-        cur_t = t;
+      const int g = static_cast<int>(it / segs);
+      const int s = static_cast<int>(it - static_cast<long long>(g) * segs);
+      if (g != cur_g) {
+        cur_g = g;
         my_slot = next_slot;
         my_w = next_w;
-        if (lane < k && t + 1 < N) {  // one token ahead
-          next_slot = token_slot[static_cast<size_t>(t + 1) * k + lane];
-          next_w = topk_w[static_cast<size_t>(t + 1) * k + lane];
+        const long long f = static_cast<long long>(g + 1) * TK + lane;  // one group ahead
+        next_slot = -1;
+        next_w = 0.0f;
+        if (g + 1 < groups && lane < TK && f < NK) {
+          next_slot = token_slot[f];
+          next_w = topk_w[f];
         }
-        if (lane < k && (my_slot < -1 || my_slot >= S)) report_bad_index(d_status);
+        if (my_slot < -1 || my_slot >= S) report_bad_index(d_status);
       }
       if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
         report_timeout(d_status);
         ok = false;
         break;
       }
-      const int seg_ch = H - s * kSeg < kSeg ? H - s * kSeg : kSeg;
+      const int seg_ch = H - s * seg < seg ? H - s * seg : seg;
       const uint32_t row_bytes = static_cast<uint32_t>(seg_ch) * 2u;
-      const bool valid = lane < k && my_slot >= 0 && my_slot < S;
+      const bool valid = lane < TK && my_slot >= 0 && my_slot < S;
       const uint32_t vmask = __ballot_sync(kFullMask, valid);
       float* hw = reinterpret_cast<float*>(smem + L.hdr_off + static_cast<size_t>(stage) * kHeaderBytes);
-      if (lane < k) hw[lane] = my_w;
+      if (lane < TK) hw[lane] = my_w;
       if (lane == 0) reinterpret_cast<uint32_t*>(hw)[32] = vmask;
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), __popc(vmask) * row_bytes);
       __syncwarp();
       if (valid)
-        bulk_g2s(data + static_cast<uint32_t>(stage * L.stage_bytes) + lane * kSegBytes,
-                 y + static_cast<size_t>(my_slot) * H + static_cast<size_t>(s) * kSeg, row_bytes,
+        bulk_g2s(data + static_cast<uint32_t>(stage * L.stage_bytes) + lane * seg_bytes,
+                 y + static_cast<size_t>(my_slot) * H + static_cast<size_t>(s) * seg, row_bytes,
                  full_bar(stage));
       ++issued;
       if (++stage == L.nstage) {
@@ -151,45 +170,52 @@ __global__ void __launch_bounds__(kThreads)
     uint32_t phase = 0;
     const int c = threadIdx.x * 8;  // this thread's 8 channels of the segment
     for (long long it = i0; it < i1; ++it) {
-      const int t = static_cast<int>(it / segs);
-      const int s = static_cast<int>(it - static_cast<long long>(t) * segs);
+      const int g = static_cast<int>(it / segs);
+      const int s = static_cast<int>(it - static_cast<long long>(g) * segs);
       if (!mbar_wait(full_bar(stage), phase)) {
         report_timeout(d_status);
         break;
       }
-      const int seg_ch = H - s * kSeg < kSeg ? H - s * kSeg : kSeg;
+      const int seg_ch = H - s * seg < seg ? H - s * seg : seg;
       if (c < seg_ch) {
         const float* hw =
             reinterpret_cast<const float*>(smem + L.hdr_off + static_cast<size_t>(stage) * kHeaderBytes);
         const uint32_t vmask = reinterpret_cast<const uint32_t*>(hw)[32];
-        const uint32_t row0 = data + static_cast<uint32_t>(stage * L.stage_bytes) + c * 2;
-        float acc[8];
+        const uint32_t stage0 = data + static_cast<uint32_t>(stage * L.stage_bytes) + c * 2;
+        for (int u = 0; u < T; ++u) {
+          const int t = g * T + u;
+          if (t >= N) break;
+          const uint32_t row0 = stage0 + static_cast<uint32_t>(u * k) * seg_bytes;
+          const uint32_t umask = vmask >> (u * k);
+          const float* uw = hw + u * k;
+          float acc[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-        for (int j0 = 0; j0 < k; j0 += 8) {
-          uint4 v[8];
+          for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+          for (int j0 = 0; j0 < k; j0 += 8) {
+            uint4 v[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            if (j0 + u < k) v[u] = ld_shared_v4(row0 + (j0 + u) * kSegBytes);
+            for (int q = 0; q < 8; ++q)
+              if (j0 + q < k) v[q] = ld_shared_v4(row0 + (j0 + q) * seg_bytes);
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int j = j0 + u;
-            if (j >= k || !((vmask >> j) & 1u)) continue;
-            const float wj = hw[j];
-            const uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            for (int q = 0; q < 8; ++q) {
+              const int j = j0 + q;
+              if (j >= k || !((umask >> j) & 1u)) continue;
+              const float wj = uw[j];
+              const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              acc[2 * i] = __fmaf_rn(wj, bf16_lo(w4[i]), acc[2 * i]);
-              acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(w4[i]), acc[2 * i + 1]);
+              for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = __fmaf_rn(wj, bf16_lo(w4[i]), acc[2 * i]);
+                acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(w4[i]), acc[2 * i + 1]);
+              }
             }
           }
+          uint4 o;
+          o.x = pack_bf16x2(acc[0], acc[1]);
+          o.y = pack_bf16x2(acc[2], acc[3]);
+          o.z = pack_bf16x2(acc[4], acc[5]);
+          o.w = pack_bf16x2(acc[6], acc[7]);
+          st_stream_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * seg + c, o);
         }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        st_stream_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * kSeg + c, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty_bar(stage));
@@ -220,7 +246,8 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
                                                            L.total)) != cudaSuccess)
     return err;
   if (per_sm < 1) per_sm = 1;
-  const long long items = static_cast<long long>(N) * ((H + kSeg - 1) / kSeg);
+  const long long items =
+      static_cast<long long>((N + L.T - 1) / L.T) * ((H + L.seg - 1) / L.seg);
   const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
   return launch_pdl(combine_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total, stream,
                     static_cast<const uint16_t*>(y), N, H, k, token_slot, topk_w,
