@@ -53,7 +53,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle baseline CPU budget (s)")
     p.add_argument("--tokens", type=int, default=None,
                    help="override the workload's token count (profiling captures of a smaller case)")
     return p.parse_args()
@@ -96,6 +96,40 @@ def ncu_traffic(op: str, workload: str):
         return int(e["dram_bytes_per_launch"])
     except Exception:
         return None
+
+
+def launches_per_step(w) -> int:
+    """Kernels one step launches: gate, layout (one CTA-sized kernel when all
+    N*k entries fit one 1024-entry chunk, else count + assign), dispatch, combine."""
+    return 1 + (1 if w.N * w.k <= 1024 else 2) + 1 + 1
+
+
+def isolated_op_times(step_ops, flush, device, reps=30):
+    """Each op alone in its own CUDA graph (cold, clean L2 before every replay);
+    the empty graph's time is subtracted.  Inside the step an op can also pay for
+    the previous op's dirty L2 lines, which this isolates."""
+    ops = step_ops()
+    out = {}
+    for name in ["empty", *ops]:
+        a = torch.cuda.Event(enable_timing=True, external=True)
+        b = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            a.record(torch.cuda.current_stream(device))
+            if name != "empty":
+                ops[name]()
+            b.record(torch.cuda.current_stream(device))
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            g.replay()
+            b.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b) * 1e3)
+        ts.sort()
+        out[name] = ts[len(ts) // 2]
+    base = out.pop("empty")
+    return {k: round(max(0.0, v - base), 2) for k, v in out.items()}
 
 
 # ---------------------------------------------------------------- ranks
@@ -207,13 +241,18 @@ def oracle_sample_size(w, inp, budget_s):
 
 
 def cpu_baseline(w, inp, budget_s):
+    """Oracle passes over (a prefix of) the batch, repeated until budget_s of CPU work."""
     n, _ = oracle_sample_size(w, inp, budget_s)
-    t = time.perf_counter()
-    oracle_step(w, inp, n)
-    dt = time.perf_counter() - t
-    return {"value": n / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {n} of the {w.N} tokens of the {w.name} batch (seed 0), gate+layout+"
-                      f"dispatch+combine, single-threaded C, {dt:.1f} s"}
+    reps, t = 0, time.perf_counter()
+    while True:
+        oracle_step(w, inp, n)
+        reps += 1
+        dt = time.perf_counter() - t
+        if dt >= budget_s:
+            break
+    return {"value": n * reps / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{reps} pass(es) over the first {n} of the {w.N} tokens of the {w.name} batch "
+                      f"(seed 0): gate+layout+dispatch+combine, single-threaded C oracle, {dt:.1f} s"}
 
 
 def workload(args):
@@ -282,6 +321,16 @@ def run_ours(args, rank, world, device):
 
     flush = _Flush()
 
+    def step_ops():
+        return {
+            "gate": lambda: api.moe_topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
+                                              w.group_topn, topk_idx=idx, topk_w=wts),
+            "layout": lambda: api.moe_get_layout(idx, w.E, w.R, out=L),
+            "dispatch": lambda: api.moe_dispatch(x, L.token_slot, w.dtype_code, recv_x=recv,
+                                                 recv_scale=scale, d_status=L.status),
+            "combine": lambda: api.moe_combine(y, L.token_slot, wts, out=out, d_status=L.status),
+        }
+
     def step(ev=None):
         stream = torch.cuda.current_stream(device)  # the capture stream inside torch.cuda.graph
         if ev: ev[0].record(stream)
@@ -348,6 +397,8 @@ def run_ours(args, rank, world, device):
         raise RuntimeError(f"device status {int(L.status.item())} after the timed steps")
     max_total_ms = max_over_ranks(sum(step_ms), world, device)
 
+    isolated = isolated_op_times(step_ops, flush, device)
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world)
@@ -362,10 +413,13 @@ def run_ours(args, rank, world, device):
     other = "dispatch" if dominant == "combine" else "combine"
 
     def roof(n):
+        iso = isolated.get(n) or None
         return {"kernel": n, "bound": "hbm", "achieved": gbs[n], "peak": peak, "unit": "GB/s",
                 "frac": gbs[n] / peak, "peak_source": f"{peak_kind} hbm_gbs",
                 "traffic": ncu_traffic(n, w.name), "algorithmic_bytes": ab[n],
-                "avg_launch_us": 1e3 * avg[n]}
+                "avg_launch_us": 1e3 * avg[n],
+                "isolated_us": iso,
+                "isolated_frac": (ab[n] / (iso * 1e-6) / 1e9 / peak) if iso else None}
 
     line = {
         "impl": "ours", "metric": METRIC,
@@ -386,7 +440,8 @@ def run_ours(args, rank, world, device):
         "dispatch_combine_tokens_per_s": w.N * world / ((avg["dispatch"] + avg["combine"]) * 1e-3),
         "roofline": roof(dominant),
         "roofline_other": roof(other),
-        "gpu_launches": 10 * args.steps,  # 5 kernels per replay, two timed loops
+        "gpu_launches": 2 * launches_per_step(w) * args.steps,  # two timed loops
+        "isolated_us": isolated,
         "clocks": clk.summary(),
         "e2e": e2e,
     }
