@@ -87,6 +87,10 @@ def _declare(L):
     L.oracle_dispatch.restype = _I
     L.oracle_combine.argtypes = [_P, _I, _I, _I, _P, _P, _P]
     L.oracle_combine.restype = _I
+    L.oracle_dispatch_backward.argtypes = [_P, _I, _I, _I, _P, _P]
+    L.oracle_dispatch_backward.restype = _I
+    L.oracle_combine_backward.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P]
+    L.oracle_combine_backward.restype = _I
 
 
 def _ptr(a: np.ndarray):
@@ -226,3 +230,37 @@ def combine(y_bf16: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray):
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_combine: invalid argument")
     return out, st
+
+
+def dispatch_backward(grad_recv_bf16: np.ndarray, token_slot: np.ndarray):
+    """grad_x bf16 bits [N,H] = slot-order fp32 sum of each token's gradient rows; (grad_x, status)."""
+    grad_recv_bf16 = _c(grad_recv_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    N, k = token_slot.shape
+    H = grad_recv_bf16.shape[1]
+    gx = np.empty((N, H), np.uint16)
+    st = lib().oracle_dispatch_backward(_ptr(grad_recv_bf16), N, H, k, _ptr(token_slot), _ptr(gx))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_dispatch_backward: invalid argument")
+    return gx, st
+
+
+def combine_backward(grad_out_bf16: np.ndarray, y_bf16: np.ndarray, token_slot: np.ndarray,
+                     topk_w: np.ndarray):
+    """(grad_y bf16 bits [S,H] (rows no slot names stay 0), grad_w fp32 [N,k],
+    sum_c |g*y| float64 [N,k] (for error bounds), status)."""
+    grad_out_bf16 = _c(grad_out_bf16, np.uint16)
+    y_bf16 = _c(y_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    N, k = token_slot.shape
+    H = grad_out_bf16.shape[1]
+    gy = np.zeros((y_bf16.shape[0], H), np.uint16)
+    gw = np.empty((N, k), np.float32)
+    mag = np.empty((N, k), np.float64)
+    st = lib().oracle_combine_backward(_ptr(grad_out_bf16), _ptr(y_bf16), N, H, k, _ptr(token_slot),
+                                       _ptr(topk_w), _ptr(gy), _ptr(gw), _ptr(mag))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_combine_backward: invalid argument")
+    return gy, gw, mag, st
+

@@ -471,3 +471,75 @@ int oracle_combine(const uint16_t* y, int N, int H, int k,
     }
     return status;
 }
+
+/* ------------------------------------------------------------------ */
+/* Backward of dispatch and combine.  [EPv2] usage patterns: the backward
+ * pass of dispatch is a combine and the backward pass of combine is a
+ * dispatch.  Written out as the adjoints of the forward maps:
+ *
+ *  dispatch backward:  grad_x[t,c] = bf16_rne(acc), acc = +0.0f, then
+ *      acc = acc + grad_recv[token_slot[t,j], c] for j = 0..k-1 (slot order,
+ *      fp32, masked slots skipped).
+ *  combine backward:   for every valid slot s = token_slot[t,j]
+ *      grad_y[s,c]  = bf16_rne( fp32(topk_w[t,j] * grad_out[t,c]) )
+ *      grad_w[t,j]  = sum_c grad_out[t,c] * y[s,c], accumulated in double
+ *                     (exact products, 53-bit sum) and rounded to fp32;
+ *      a masked slot gets grad_w = 0 and writes no grad_y row.
+ * The kernels may sum grad_w in another order in fp32; their error bound
+ * follows from the arithmetic and is stated with the tests.            */
+/* ------------------------------------------------------------------ */
+int oracle_dispatch_backward(const uint16_t* grad_recv, int N, int H, int k,
+                             const int32_t* token_slot, uint16_t* grad_x)
+{
+    if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int64_t S = (int64_t)N * k;
+    for (int t = 0; t < N; ++t) {
+        for (int c = 0; c < H; ++c) {
+            float acc = 0.0f;
+            for (int j = 0; j < k; ++j) {
+                int32_t s = token_slot[(int64_t)t * k + j];
+                if (s == -1) continue;
+                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }
+                acc = acc + oracle_f32_from_bf16(grad_recv[(size_t)s * H + c]);
+            }
+            grad_x[(size_t)t * H + c] = oracle_bf16_from_f32(acc);
+        }
+    }
+    return status;
+}
+
+int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int N, int H, int k,
+                            const int32_t* token_slot, const float* topk_w,
+                            uint16_t* grad_y, float* grad_w, double* grad_w_abs)
+{
+    if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int64_t S = (int64_t)N * k;
+    for (int t = 0; t < N; ++t) {
+        const uint16_t* g = grad_out + (size_t)t * H;
+        for (int j = 0; j < k; ++j) {
+            int64_t i = (int64_t)t * k + j;
+            int32_t s = token_slot[i];
+            grad_w[i] = 0.0f;
+            if (grad_w_abs) grad_w_abs[i] = 0.0;
+            if (s == -1) continue;
+            if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }
+            const uint16_t* yr = y + (size_t)s * H;
+            uint16_t* gy = grad_y + (size_t)s * H;
+            double dot = 0.0, mag = 0.0;
+            for (int c = 0; c < H; ++c) {
+                float gc = oracle_f32_from_bf16(g[c]);
+                float prod = topk_w[i] * gc;
+                gy[c] = oracle_bf16_from_f32(prod);
+                double term = (double)gc * (double)oracle_f32_from_bf16(yr[c]);
+                dot += term;
+                mag += fabs(term);
+            }
+            grad_w[i] = (float)dot;
+            if (grad_w_abs) grad_w_abs[i] = mag;
+        }
+    }
+    return status;
+}
+

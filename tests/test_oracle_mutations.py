@@ -32,6 +32,11 @@ MUTANTS = {
     "bf16_ties_up": ("(lower == 0x8000u && (upper & 1u))", "(lower == 0x8000u)"),
     "combine_weight_index_dropped": ("acc = fmaf(topk_w[(int64_t)t * k + j], v, acc);",
                                      "acc = fmaf(topk_w[(int64_t)t * k], v, acc);"),
+    "dispatch_backward_skips_last_slot": ("            for (int j = 0; j < k; ++j) {\n                int32_t s = token_slot[(int64_t)t * k + j];\n                if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                acc = acc + ",
+                                          "            for (int j = 0; j + 1 < k; ++j) {\n                int32_t s = token_slot[(int64_t)t * k + j];\n                if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                acc = acc + "),
+    "combine_backward_weight_dropped": ("float prod = topk_w[i] * gc;", "float prod = gc;"),
+    "combine_backward_dot_wrong_row": ("double term = (double)gc * (double)oracle_f32_from_bf16(yr[c]);",
+                                       "double term = (double)gc * (double)oracle_f32_from_bf16(yr[0]);"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

@@ -480,3 +480,80 @@ def test_dispatch_combine_adjoint():
     wslot[L.token_slot.reshape(-1)] = w.reshape(-1)
     rhs = (O.bf16_to_f32(y).astype(np.float64) * O.bf16_to_f32(dg) * wslot[:, None]).sum()
     assert abs(lhs - rhs) <= 2.0**-8 * np.abs(O.bf16_to_f32(out).astype(np.float64) * O.bf16_to_f32(g)).sum()
+
+
+# ----------------------------------------------------------------- backward
+def test_dispatch_backward_is_slot_sum():
+    rng = np.random.default_rng(18)
+    N, H, k = 60, 40, 4
+    slot = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    slot[rng.random((N, k)) < 0.1] = -1
+    g = _bf16_bits(rng.integers(-8, 8, size=(N * k, H)))        # small integers: exact sums
+    gx, st = O.dispatch_backward(g, slot)
+    gv = O.bf16_to_f32(g).astype(np.float64)
+    ref = np.zeros((N, H))
+    for t in range(N):
+        for j in range(k):
+            if slot[t, j] >= 0:
+                ref[t] += gv[slot[t, j]]
+    assert st == O.OK and np.array_equal(O.bf16_to_f32(gx), ref.astype(np.float32))
+    # random values: within one bf16 ulp of the float64 sum
+    g2 = _bf16_bits(rng.normal(size=(N * k, H)))
+    gx2, _ = O.dispatch_backward(g2, slot)
+    gv2 = O.bf16_to_f32(g2).astype(np.float64)
+    ref2 = np.zeros((N, H))
+    for t in range(N):
+        for j in range(k):
+            if slot[t, j] >= 0:
+                ref2[t] += gv2[slot[t, j]]
+    got = O.bf16_to_f32(gx2).astype(np.float64)
+    assert (np.abs(got - ref2) <= 2.0**-8 * np.abs(ref2) + k * 2.0**-24 * np.abs(gv2).max() + 1e-30).all()
+
+
+def test_dispatch_backward_adjoint_of_dispatch():
+    """<dispatch_backward(G), x> = <G, dispatch(x)> in exact arithmetic."""
+    rng = np.random.default_rng(19)
+    N, H, E, k = 50, 32, 12, 3
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(N)]).astype(np.int32)
+    L = O.get_layout(idx, E, 3)
+    x = _bf16_bits(rng.integers(-4, 5, size=(N, H)))
+    G = _bf16_bits(rng.integers(-4, 5, size=(N * k, H)))
+    dx, _, _ = O.dispatch(x, L.token_slot, O.DT_BF16)
+    gx, _ = O.dispatch_backward(G, L.token_slot)
+    lhs = (O.bf16_to_f32(gx).astype(np.float64) * O.bf16_to_f32(x)).sum()
+    rhs = (O.bf16_to_f32(G).astype(np.float64) * O.bf16_to_f32(dx)).sum()
+    assert lhs == rhs
+
+
+def test_combine_backward_vs_torch_autograd():
+    rng = np.random.default_rng(20)
+    N, H, k = 24, 64, 4
+    S = N * k
+    slot = rng.permutation(S).astype(np.int32).reshape(N, k)
+    orphan = int(slot[3, 2])           # the row the masked slot would have used
+    slot[3, 2] = -1
+    w = rng.random((N, k)).astype(np.float32)
+    y = _bf16_bits(rng.normal(size=(S, H)))
+    g = _bf16_bits(rng.normal(size=(N, H)))
+    gy, gw, mag, st = O.combine_backward(g, y, slot, w)
+    assert st == O.OK
+    yt = torch.from_numpy(O.bf16_to_f32(y).astype(np.float64)).requires_grad_(True)
+    wt = torch.from_numpy(w.astype(np.float64)).requires_grad_(True)
+    st_ = torch.from_numpy(np.where(slot >= 0, slot, 0).astype(np.int64))
+    mask = torch.from_numpy((slot >= 0).astype(np.float64))
+    out = (wt[:, :, None] * mask[:, :, None] * yt[st_]).sum(1)
+    gt = torch.from_numpy(O.bf16_to_f32(g).astype(np.float64))
+    (out * gt).sum().backward()
+    # grad_w: the oracle sums in double, so it matches autograd to double rounding
+    assert np.allclose(gw, wt.grad.numpy(), rtol=1e-6, atol=1e-12)
+    assert gw[3, 2] == 0.0
+    # grad_y = bf16(fp32(w * g)) on every valid row; autograd's float64 value is within one rounding
+    valid = slot >= 0
+    ref_rows = torch.from_numpy((w[:, :, None] * O.bf16_to_f32(g)[:, None, :]).astype(np.float32))
+    ref_bits = ref_rows.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(gy[slot[valid]], ref_bits[valid])
+    ag = yt.grad.numpy()[slot[valid]]
+    assert np.all(np.abs(O.bf16_to_f32(gy[slot[valid]]) - ag) <= 2.0**-8 * np.abs(ag) + 1e-30)
+    assert not gy[orphan].any()        # no slot names it: never written
+    # magnitude sums bound the dot products
+    assert (np.abs(gw) <= mag * (1 + 1e-6) + 1e-30).all()
