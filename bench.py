@@ -53,6 +53,7 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-backward", action="store_true", help="skip timing the backward ops")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle baseline CPU budget (s)")
     p.add_argument("--tokens", type=int, default=None,
                    help="override the workload's token count (profiling captures of a smaller case)")
@@ -398,6 +399,33 @@ def run_ours(args, rank, world, device):
     max_total_ms = max_over_ranks(sum(step_ms), world, device)
 
     isolated = isolated_op_times(step_ops, flush, device)
+    backward = None
+    if not args.no_backward:
+        # backward ops on the same layout, timed alone (cold, clean L2)
+        gen = torch.Generator(device="cpu").manual_seed(1234)
+        grad_recv = torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
+        grad_out = torch.randn(w.N, w.H, generator=gen).to(torch.bfloat16).to(device)
+        y_b = y_in if y_in is not None else torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
+        grad_x = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
+        grad_y = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
+        grad_w = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
+
+        def bwd_ops():
+            return {
+                "dispatch_backward": lambda: api.moe_dispatch_backward(
+                    grad_recv, L.token_slot, grad_x=grad_x, d_status=L.status),
+                "combine_backward": lambda: api.moe_combine_backward(
+                    grad_out, y_b, L.token_slot, wts, grad_y=grad_y, grad_w=grad_w, d_status=L.status),
+            }
+        bt = isolated_op_times(bwd_ops, flush, device)
+        ab_all = algorithmic_bytes(w)
+        peak_b, _ = measured_peak()
+        backward = {n: {"us": bt[n], "gbs": ab_all[n] / (bt[n] * 1e-6) / 1e9 if bt[n] else None,
+                        "frac": ab_all[n] / (bt[n] * 1e-6) / 1e9 / peak_b if bt[n] else None,
+                        "algorithmic_bytes": ab_all[n]} for n in bt}
+        torch.cuda.synchronize(device)
+        if int(L.status.item()) != 0:
+            raise RuntimeError(f"device status {int(L.status.item())} after the backward ops")
 
     e2e = None
     if not args.no_e2e:
@@ -442,6 +470,7 @@ def run_ours(args, rank, world, device):
         "roofline_other": roof(other),
         "gpu_launches": 2 * launches_per_step(w) * args.steps,  # two timed loops
         "isolated_us": isolated,
+        "backward": backward,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

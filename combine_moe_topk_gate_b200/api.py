@@ -55,6 +55,10 @@ def _load() -> ctypes.CDLL:
     L.moe_dispatch.restype = I
     L.moe_combine.argtypes = [P, I, I, I, P, P, P, P, P]
     L.moe_combine.restype = I
+    L.moe_dispatch_backward.argtypes = [P, I, I, I, P, P, P, P]
+    L.moe_dispatch_backward.restype = I
+    L.moe_combine_backward.argtypes = [P, P, I, I, I, P, P, P, P, P, P]
+    L.moe_combine_backward.restype = I
     L.moe_e4m3_encode.argtypes = [P, SZ, P, P]
     L.moe_e4m3_encode.restype = I
     L.moe_status_string.argtypes = [I]
@@ -245,6 +249,46 @@ def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor,
                           _ptr(d_status), _stream(stream, y.device))
     _check(st, "moe_combine")
     return out
+
+
+def moe_dispatch_backward(grad_recv: torch.Tensor, token_slot: torch.Tensor, *, grad_x=None,
+                          d_status=None, stream=None) -> torch.Tensor:
+    """Gradient of dispatch: slot-order sum of each token's rows of ``grad_recv``
+    (bf16 [N*k,H]) -> bf16 [N,H]."""
+    _need(grad_recv, "grad_recv", torch.bfloat16)
+    _need(token_slot, "token_slot", torch.int32)
+    N, k = token_slot.shape
+    H = grad_recv.shape[1]
+    if grad_x is None:
+        grad_x = torch.empty((N, H), dtype=torch.bfloat16, device=grad_recv.device)
+    _need(grad_x, "grad_x", torch.bfloat16, (N, H))
+    st = _lib.moe_dispatch_backward(_ptr(grad_recv), N, H, k, _ptr(token_slot), _ptr(grad_x),
+                                    _ptr(d_status), _stream(stream, grad_recv.device))
+    _check(st, "moe_dispatch_backward")
+    return grad_x
+
+
+def moe_combine_backward(grad_out: torch.Tensor, y: torch.Tensor, token_slot: torch.Tensor,
+                         topk_w: torch.Tensor, *, grad_y=None, grad_w=None, d_status=None,
+                         stream=None):
+    """Gradients of combine: ``(grad_y bf16 [N*k,H], grad_w fp32 [N,k])``."""
+    _need(grad_out, "grad_out", torch.bfloat16)
+    _need(y, "y", torch.bfloat16)
+    _need(token_slot, "token_slot", torch.int32)
+    N, k = token_slot.shape
+    H = grad_out.shape[1]
+    _need(topk_w, "topk_w", torch.float32, (N, k))
+    if grad_y is None:
+        grad_y = torch.empty((N * k, H), dtype=torch.bfloat16, device=y.device)
+    if grad_w is None:
+        grad_w = torch.empty((N, k), dtype=torch.float32, device=y.device)
+    _need(grad_y, "grad_y", torch.bfloat16, (N * k, H))
+    _need(grad_w, "grad_w", torch.float32, (N, k))
+    st = _lib.moe_combine_backward(_ptr(grad_out), _ptr(y), N, H, k, _ptr(token_slot),
+                                   _ptr(topk_w), _ptr(grad_y), _ptr(grad_w), _ptr(d_status),
+                                   _stream(stream, y.device))
+    _check(st, "moe_combine_backward")
+    return grad_y, grad_w
 
 
 def moe_e4m3_encode(x: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:

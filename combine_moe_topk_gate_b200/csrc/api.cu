@@ -139,6 +139,41 @@ moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
                                        as_stream(stream)));
 }
 
+moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hidden, int k,
+                                   const int32_t* token_slot, void* grad_x, int32_t* d_status,
+                                   moe_stream_t stream) {
+  const int N = num_tokens, H = hidden;
+  if (N < 0 || H < 1 || k < 1 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  if (N == 0) return MOE_OK;
+  if (!grad_recv || !token_slot || !grad_x) return MOE_ERR_INVALID_ARG;
+  if (!aligned(grad_recv, 16) || !aligned(grad_x, 16) || !aligned(token_slot, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARG;
+  // the combine kernel with unit weights
+  return from_cuda(moe::launch_combine(grad_recv, N, H, k, token_slot, nullptr, grad_x, d_status,
+                                       as_stream(stream)));
+}
+
+moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_tokens, int hidden,
+                                  int k, const int32_t* token_slot, const float* topk_w,
+                                  void* grad_y, float* grad_w, int32_t* d_status,
+                                  moe_stream_t stream) {
+  const int N = num_tokens, H = hidden;
+  if (N < 0 || H < 1 || k < 1 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  if (N == 0) return MOE_OK;
+  if (!grad_out || !y || !token_slot || !topk_w || !grad_y || !grad_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned(grad_out, 16) || !aligned(y, 16) || !aligned(grad_y, 16) ||
+      !aligned(token_slot, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4) ||
+      !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_combine_backward(grad_out, y, N, H, k, token_slot, topk_w, grad_y,
+                                                grad_w, d_status, as_stream(stream)));
+}
+
 moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream) {
   if (n == 0) return MOE_OK;
   if (!in || !out || !aligned(in, 4)) return MOE_ERR_INVALID_ARG;

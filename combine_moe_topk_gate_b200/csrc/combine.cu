@@ -6,7 +6,9 @@
 // patterns: combine reduces the expert outputs back to the token.
 //
 //   out[t, c] = bf16_rne(acc),  acc = +0, then acc = fmaf(w[t,j], y[slot[t,j], c], acc)
-//   for j = 0..k-1 in slot order (masked slots skipped).
+//   for j = 0..k-1 in slot order (masked slots skipped).  With no weights
+//   (topk_w == nullptr) every weight is 1 and fmaf(1, v, acc) = acc + v: that
+//   is the backward of dispatch (the slot-order sum of a token's gradient rows).
 //
 // Persistent, warp-specialised CTAs.  Work item = (group of T consecutive
 // tokens, 2048-channel segment) with T = max(1, 8 / k), so an item always
@@ -113,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 3)
       const long long f = (i0 / segs) * TK + lane;
       if (lane < TK && f < NK) {
         next_slot = token_slot[f];
-        next_w = topk_w[f];
+        next_w = topk_w ? topk_w[f] : 1.0f;
       }
     }
     for (long long it = i0; it < i1; ++it) {
@@ -128,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 3)
         next_w = 0.0f;
         if (g + 1 < groups && lane < TK && f < NK) {
           next_slot = token_slot[f];
-          next_w = topk_w[f];
+          next_w = topk_w ? topk_w[f] : 1.0f;
         }
         if (my_slot < -1 || my_slot >= S) report_bad_index(d_status);
       }

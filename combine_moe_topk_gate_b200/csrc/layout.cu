@@ -247,6 +247,89 @@ __global__ void __launch_bounds__(kLayoutThreads)
   (void)lane;
 }
 
+// Whole layout in one CTA when every entry fits one chunk (N*k <= 1024, the
+// decode-sized batches): histogram, scan and ranks stay in shared memory, so
+// there is one launch and no workspace round trip.
+__global__ void __launch_bounds__(kLayoutThreads)
+    layout_single_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R,
+                         int32_t* __restrict__ expert_count, int32_t* __restrict__ expert_offset,
+                         int32_t* __restrict__ rank_count, int32_t* __restrict__ rank_offset,
+                         int32_t* __restrict__ rank_tokens, int32_t* __restrict__ token_slot,
+                         int32_t* __restrict__ slot_token, int32_t* d_status) {
+  extern __shared__ int32_t sm[];
+  const int nb = E + 1;
+  int32_t* off = sm;                              // nb: totals, then their exclusive scan
+  int32_t* wcnt = off + nb;                       // kLayoutWarps * nb
+  int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
+  int32_t* rtok = warp_sums + 32;                 // R
+  int32_t* sidx = rtok + R;                       // kLayoutThreads
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int ne = N * k;  // <= kLayoutThreads
+  const int nbits = 32 - __clz(E + 1);
+  const int epr = E / R;
+  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
+  for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  pdl_wait();
+  pdl_trigger();
+  int e = -1, b = -1;
+  if (tid < ne) {
+    e = topk_idx[tid];
+    sidx[tid] = e;
+    b = bucket_of(e, E);
+    if (b == E && e != -1) report_bad_index(d_status);
+  }
+  __syncthreads();
+  const unsigned same = warp_match(static_cast<unsigned>(b + 1), nbits);
+  const int in_warp = __popc(same & lanemask_lt());
+  if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
+  if (b >= 0 && b < E) {  // the token's first slot on this rank counts the token
+    const int r = e / epr;
+    const int j = tid % k;
+    bool first = true;
+    for (int jj = 0; jj < j; ++jj) {
+      const int e2 = sidx[tid - j + jj];
+      if (static_cast<unsigned>(e2) < static_cast<unsigned>(E) && e2 / epr == r) {
+        first = false;
+        break;
+      }
+    }
+    if (first) atomicAdd(&rtok[r], 1);
+  }
+  __syncthreads();
+  // per bucket: exclusive prefix over the warps, total into off[]
+  for (int bb = warp; bb < nb; bb += kLayoutWarps) {
+    const int v = wcnt[lane * nb + bb];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(kFullMask, incl, o);
+      if (lane >= o) incl += y;
+    }
+    wcnt[lane * nb + bb] = incl - v;
+    if (lane == 31) off[bb] = incl;
+  }
+  __syncthreads();
+  for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = off[i];
+  block_exclusive_scan(off, nb, warp_sums);
+  for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
+  for (int r = tid; r < R; r += kLayoutThreads) {
+    rank_offset[r] = off[r * epr];
+    rank_count[r] = off[(r + 1) * epr] - off[r * epr];
+    rank_tokens[r] = rtok[r];
+  }
+  if (tid == 0) rank_offset[R] = off[E];
+  if (tid < ne) {
+    const int slot = off[b] + wcnt[warp * nb + b] + in_warp;
+    if (b < E) {
+      token_slot[tid] = slot;
+      slot_token[slot] = tid / k;
+    } else {
+      token_slot[tid] = -1;
+      slot_token[slot] = -1;
+    }
+  }
+}
+
 }  // namespace
 
 size_t layout_workspace_bytes(int N, int k, int E, int R) {
@@ -262,13 +345,26 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
                           int32_t* slot_token, void* workspace, int32_t* d_status,
                           cudaStream_t stream) {
   const int C = num_chunks(N, k);
+  cudaError_t err;
+  if (static_cast<long long>(N) * k <= kLayoutThreads) {
+    const size_t smem = (static_cast<size_t>(E) + 1 + static_cast<size_t>(kLayoutWarps) * (E + 1) +
+                         32 + R + kLayoutThreads) *
+                        sizeof(int32_t);
+    if (smem > 48 * 1024) {
+      err = cudaFuncSetAttribute(layout_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+      if (err != cudaSuccess) return err;
+    }
+    return launch_pdl(layout_single_kernel, 1, kLayoutThreads, smem, stream, topk_idx, N, k, E, R,
+                      expert_count, expert_offset, rank_count, rank_offset, rank_tokens, token_slot,
+                      slot_token, d_status);
+  }
   int32_t* chunk_counts = static_cast<int32_t*>(workspace);
   int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
   const size_t smem_count = (static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
   const size_t smem_assign =
       (2 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
       sizeof(int32_t);
-  cudaError_t err;
   if (smem_count > 48 * 1024) {
     err = cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem_count));

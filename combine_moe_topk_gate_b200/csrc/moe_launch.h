@@ -28,6 +28,10 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
                            const float* topk_w, void* out, int32_t* d_status,
                            cudaStream_t stream);
 
+cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, int H, int k,
+                                    const int32_t* token_slot, const float* topk_w, void* grad_y,
+                                    float* grad_w, int32_t* d_status, cudaStream_t stream);
+
 cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream);
 
 }  // namespace moe

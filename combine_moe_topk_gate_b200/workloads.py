@@ -128,6 +128,10 @@ def algorithmic_bytes(w: Workload) -> dict:
         "layout": 4 * N * k + 8 * N * k + 4 * (4 * E + 3 * w.R),
         "dispatch": 2 * N * H + N * k * H * b + scales + 4 * N * k,
         "combine": 2 * N * k * H + 2 * N * H + 8 * N * k,
+        # backward: gradient rows in, token gradient out (dispatch); token
+        # gradient + expert rows in, scaled rows + weight gradients out (combine)
+        "dispatch_backward": 2 * N * k * H + 2 * N * H + 4 * N * k,
+        "combine_backward": 2 * N * H + 4 * N * k * H + 12 * N * k,
     }
 
 

@@ -221,6 +221,38 @@ moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
                          int32_t* d_status, moe_stream_t stream);
 
 /*
+ * moe_dispatch_backward -- gradient of dispatch: the sum of each token's
+ * gradient rows.  [EPv2] usage patterns: the backward pass of dispatch is a
+ * combine.  grad_recv bf16 [S, H] (one gradient row per receive slot),
+ * token_slot int32 [N, k] -> grad_x bf16 [N, H]:
+ *   grad_x[t, c] = bf16_rne(acc), acc = +0.0f, acc = acc + grad_recv[token_slot[t,j], c]
+ *   for j = 0..k-1 in slot order (fp32; masked slots skipped).
+ * (With FP8 dispatch the gradient passes the quantisation unchanged: grad_recv
+ * is the gradient with respect to the dequantised rows.)
+ * H % 8 == 0; grad_recv and grad_x 16-byte aligned.
+ */
+moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hidden, int k,
+                                   const int32_t* token_slot, void* grad_x, int32_t* d_status,
+                                   moe_stream_t stream);
+
+/*
+ * moe_combine_backward -- gradients of combine with respect to the expert
+ * outputs and the router weights.  [EPv2] usage patterns: the backward pass of
+ * combine is a dispatch.  For every valid slot s = token_slot[t,j]:
+ *   grad_y[s, c] = bf16_rne(fp32(topk_w[t,j] * grad_out[t,c]))   (grad_y bf16 [S, H])
+ *   grad_w[t, j] = sum_c grad_out[t,c] * y[s,c]                   (grad_w fp32 [N, k])
+ * grad_w is accumulated in fp32 in a fixed order (deterministic); its
+ * rounding error is at most (H - 1) * 2^-24 * sum_c |grad_out[t,c] * y[s,c]|
+ * (the products of two bf16 values are exact in fp32).  A masked slot gets
+ * grad_w = 0 and writes no grad_y row; rows no slot names are not written.
+ * H % 8 == 0; grad_out, y, grad_y 16-byte aligned.
+ */
+moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_tokens, int hidden,
+                                  int k, const int32_t* token_slot, const float* topk_w,
+                                  void* grad_y, float* grad_w, int32_t* d_status,
+                                  moe_stream_t stream);
+
+/*
  * moe_e4m3_encode -- the element encoder moe_dispatch uses, exposed on its
  * own: out[i] = e4m3 code of in[i], round to nearest even, finite values and
  * infinities beyond 448 saturated to +-448, zero keeps its sign, NaN -> NaN
