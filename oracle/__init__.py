@@ -27,6 +27,8 @@ GATE_SOFTMAX_RENORM = 1
 GATE_SIGMOID_GROUP = 2
 DT_BF16 = 0
 DT_FP8_E4M3 = 1
+DT_FP8_E4M3_TOKEN = 2
+DT_MXFP8_E4M3 = 3
 OK = 0
 ERR_INVALID_ARG = 1
 ERR_BAD_INDEX = 4
@@ -198,7 +200,9 @@ def get_layout(topk_idx: np.ndarray, E: int, R: int) -> Layout:
 
 def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
              recv_rows: int | None = None):
-    """Returns (recv_x, recv_scale or None, status).  Rows no slot names stay 0."""
+    """Returns (recv_x, recv_scale or None, status).  Rows no slot names stay 0.
+    recv_scale: fp32 [S, H/128] (per block), fp32 [S, 1] (per token) or uint8
+    E8M0 bytes [S, H/32] (MXFP8)."""
     x_bf16 = _c(x_bf16, np.uint16)
     token_slot = _c(token_slot, np.int32)
     N, H = x_bf16.shape
@@ -210,7 +214,12 @@ def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
         sp = None
     else:
         recv = np.zeros((S, H), np.uint8)
-        scale = np.zeros((S, H // 128), np.float32)
+        if dtype == DT_FP8_E4M3:
+            scale = np.zeros((S, H // 128), np.float32)
+        elif dtype == DT_FP8_E4M3_TOKEN:
+            scale = np.zeros((S, 1), np.float32)
+        else:                                   # MXFP8: E8M0 bytes, one per 32 channels
+            scale = np.zeros((S, H // 32), np.uint8)
         sp = _ptr(scale)
     st = lib().oracle_dispatch(_ptr(x_bf16), N, H, k, _ptr(token_slot), dtype, _ptr(recv), sp)
     if st == ERR_INVALID_ARG:

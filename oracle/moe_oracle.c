@@ -43,6 +43,8 @@
 
 #define DT_BF16 0
 #define DT_FP8_E4M3 1
+#define DT_FP8_E4M3_TOKEN 2
+#define DT_MXFP8_E4M3 3
 
 /* ------------------------------------------------------------------ */
 /* bit helpers                                                         */
@@ -392,13 +394,92 @@ int oracle_get_layout(const int32_t* topk_idx, int N, int k, int E, int R,
  * The same codes and scale go to every slot of the token.
  * A slot outside [-1, N*k) is skipped and reported.                    */
 /* ------------------------------------------------------------------ */
+/* Quantisation variants ([TK] list, "Quantisierung ... pro Token, pro Block"):
+ *  DT_FP8_E4M3_TOKEN: one fp32 scale per token row: amax over the whole row,
+ *      scale = amax / 448, codes e4m3(x * (448 / amax)) as for the blocks;
+ *      recv_scale is [S, 1].
+ *  DT_MXFP8_E4M3: OCP Microscaling MXFP8 -- blocks of 32 elements share the
+ *      scale X = 2^e with e = floor(log2(amax)) - 8 (8 = the largest exponent
+ *      of e4m3), clamped to [-127, 127]; elements e4m3(x * 2^-e), RNE,
+ *      saturating to 448 (x * 2^-e can reach 511.x); the scale is stored as
+ *      the E8M0 byte e + 127 in recv_scale viewed as uint8 [S, H/32].  An
+ *      all-zero block stores e = -127 (byte 0) and zero codes.               */
+static int floor_log2_pos(float a)   /* a > 0, finite: exact from the bits */
+{
+    uint32_t u = f32_bits(a);
+    int ex = (int)((u >> 23) & 0xFF);
+    if (ex > 0) return ex - 127;
+    int m = (int)(u & 0x7FFFFF), hb = 22;
+    while (!((m >> hb) & 1)) --hb;
+    return hb - 149;                 /* subnormal: 2^(hb - 23) * 2^-126 */
+}
+
+static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
+                                   const int32_t* token_slot, int dtype, uint8_t* recv_x,
+                                   float* recv_scale)
+{
+    int status = ORC_OK;
+    int64_t S = (int64_t)N * k;
+    int nb = dtype == DT_MXFP8_E4M3 ? H / 32 : 1;
+    uint8_t* q = (uint8_t*)malloc((size_t)H);
+    float* fsc = (float*)malloc(sizeof(float));
+    uint8_t* esc = (uint8_t*)malloc((size_t)nb);
+    for (int t = 0; t < N; ++t) {
+        const uint16_t* xr = x + (size_t)t * H;
+        if (dtype == DT_FP8_E4M3_TOKEN) {
+            float amax = 0.0f;
+            for (int c = 0; c < H; ++c) {
+                float v = fabsf(oracle_f32_from_bf16(xr[c]));
+                if (v > amax) amax = v;
+            }
+            float inv = 448.0f / amax;
+            fsc[0] = amax / 448.0f;
+            for (int c = 0; c < H; ++c) {
+                float v = oracle_f32_from_bf16(xr[c]);
+                q[c] = oracle_e4m3_encode((v == 0.0f) ? v : v * inv);
+            }
+        } else {
+            for (int b = 0; b < nb; ++b) {
+                float amax = 0.0f;
+                for (int c = b * 32; c < (b + 1) * 32; ++c) {
+                    float v = fabsf(oracle_f32_from_bf16(xr[c]));
+                    if (v > amax) amax = v;
+                }
+                int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+                esc[b] = (uint8_t)(e + 127);
+                float down = ldexpf(1.0f, -e);    /* e <= 119 for bf16 input: 2^-e is a normal float */
+                for (int c = b * 32; c < (b + 1) * 32; ++c) {
+                    float v = oracle_f32_from_bf16(xr[c]);
+                    q[c] = oracle_e4m3_encode((v == 0.0f) ? v : v * down);
+                }
+            }
+        }
+        for (int j = 0; j < k; ++j) {
+            int32_t s = token_slot[(int64_t)t * k + j];
+            if (s == -1) continue;
+            if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }
+            memcpy(recv_x + (size_t)s * H, q, (size_t)H);
+            if (dtype == DT_FP8_E4M3_TOKEN) recv_scale[s] = fsc[0];
+            else memcpy((uint8_t*)recv_scale + (size_t)s * nb, esc, (size_t)nb);
+        }
+    }
+    free(q); free(fsc); free(esc);
+    return status;
+}
+
 int oracle_dispatch(const uint16_t* x, int N, int H, int k,
                     const int32_t* token_slot, int dtype, void* recv_x,
                     float* recv_scale)
 {
     if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
     if (dtype == DT_FP8_E4M3 && H % 128 != 0) return ORC_ERR_INVALID_ARG;
-    if (dtype != DT_BF16 && dtype != DT_FP8_E4M3) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_MXFP8_E4M3 && H % 32 != 0) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_FP8_E4M3_TOKEN && H % 8 != 0) return ORC_ERR_INVALID_ARG;
+    if (dtype < DT_BF16 || dtype > DT_MXFP8_E4M3) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_FP8_E4M3_TOKEN || dtype == DT_MXFP8_E4M3)
+        return oracle_dispatch_variant(x, N, H, k, token_slot, dtype, (uint8_t*)recv_x, recv_scale);
     int status = ORC_OK;
     int64_t S = (int64_t)N * k;
     int nb = H / 128;

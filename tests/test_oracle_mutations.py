@@ -37,6 +37,9 @@ MUTANTS = {
     "combine_backward_weight_dropped": ("float prod = topk_w[i] * gc;", "float prod = gc;"),
     "combine_backward_dot_wrong_row": ("double term = (double)gc * (double)oracle_f32_from_bf16(yr[c]);",
                                        "double term = (double)gc * (double)oracle_f32_from_bf16(yr[0]);"),
+    "mxfp8_exponent_off_by_one": ("int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;",
+                                  "int e = (amax > 0.0f) ? floor_log2_pos(amax) - 7 : -127;"),
+    "fp8_token_scale_transposed": ("fsc[0] = amax / 448.0f;", "fsc[0] = 448.0f / amax;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

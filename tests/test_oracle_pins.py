@@ -557,3 +557,67 @@ def test_combine_backward_vs_torch_autograd():
     assert not gy[orphan].any()        # no slot names it: never written
     # magnitude sums bound the dot products
     assert (np.abs(gw) <= mag * (1 + 1e-6) + 1e-30).all()
+
+
+# ----------------------------------------------------------------- quantisation variants
+def test_mxfp8_worked_example():
+    g = _gold("mxfp8_block_worked_example.json")
+    row = np.zeros(32, np.float32)
+    for c, v in g["nonzero"].items():
+        row[int(c)] = v
+    x = _bf16_bits(row[None, :])
+    recv, sc, st = O.dispatch(x, np.array([[0]], np.int32), O.DT_MXFP8_E4M3)
+    assert sc.dtype == np.uint8 and sc[0, 0] == g["e8m0"]
+    for c, code in g["codes"].items():
+        assert recv[0, int(c)] == int(code, 16), c
+
+
+def test_mxfp8_properties():
+    rng = np.random.default_rng(21)
+    N, H, k = 30, 256, 3
+    xf = (rng.normal(size=(N, H)) * np.exp2(rng.integers(-20, 20, size=(N, 1)))).astype(np.float32)
+    xf[2, :32] = 0.0
+    xf[3, 32:64] = -0.0
+    x = _bf16_bits(xf)
+    ts = np.arange(N * k, dtype=np.int32).reshape(N, k)
+    recv, sc, st = O.dispatch(x, ts, O.DT_MXFP8_E4M3)
+    xv = O.bf16_to_f32(x).astype(np.float32).reshape(N, H // 32, 32)
+    amax = np.abs(xv).max(2)
+    mant, ex = np.frexp(amax.astype(np.float64))          # amax = mant * 2^ex, mant in [0.5, 1)
+    e = np.where(amax > 0, ex - 1 - 8, -127)
+    assert np.array_equal(sc[ts[:, 0]], (e + 127).astype(np.uint8))
+    for j in range(k):
+        assert np.array_equal(recv[ts[:, j]], recv[ts[:, 0]]) and np.array_equal(sc[ts[:, j]], sc[ts[:, 0]])
+    scaled = np.ldexp(xv.astype(np.float64), -e[:, :, None]).astype(np.float32)      # exact
+    ref = torch.from_numpy(np.clip(scaled, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    q = recv[ts[:, 0]].reshape(N, H // 32, 32)
+    assert np.array_equal(q, ref)
+    # the largest element of every non-zero block lands in [256, 448] (saturating above)
+    top = np.take_along_axis(q, np.abs(xv).argmax(2)[:, :, None], 2)[:, :, 0] & 0x7F
+    assert ((top[amax > 0] >= 0x78) & (top[amax > 0] <= 0x7E)).all()
+    assert (q[2, 0] == 0).all() and (q[3, 1] == 0x80).all() and sc[ts[2, 0], 0] == 0
+
+
+def test_fp8_per_token_properties():
+    rng = np.random.default_rng(22)
+    N, H, k = 20, 384, 2
+    xf = rng.normal(size=(N, H)).astype(np.float32) * np.exp2(rng.integers(-10, 10, size=(N, 1))).astype(np.float32)
+    xf[5] = 0.0
+    x = _bf16_bits(xf)
+    ts = np.arange(N * k, dtype=np.int32).reshape(N, k)
+    recv, sc, st = O.dispatch(x, ts, O.DT_FP8_E4M3_TOKEN)
+    xv = O.bf16_to_f32(x).astype(np.float32)
+    amax = np.abs(xv).max(1)
+    assert sc.shape == (N * k, 1)
+    assert np.array_equal(sc[ts[:, 1], 0], (amax / np.float32(448)).astype(np.float32))
+    with np.errstate(divide="ignore", invalid="ignore"):
+        inv = (np.float32(448) / amax).astype(np.float32)
+        prod = (xv * inv[:, None]).astype(np.float32)
+    prod = np.where(xv == 0, xv, prod)
+    ref = torch.from_numpy(np.clip(prod, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(recv[ts[:, 0]], ref) and np.array_equal(recv[ts[:, 1]], ref)
+    assert sc[ts[5, 0], 0] == 0.0 and (recv[ts[5, 0]] == 0).all()
+    # round trip within the e4m3 bound
+    deq = _torch_e4m3_decode_table()[recv[ts[:, 0]]] * sc[ts[:, 0]].astype(np.float64)
+    bound = np.maximum(2.0**-4 * np.abs(xv), 2.0**-10 * sc[ts[:, 0]]) * (1 + 2.0**-20)
+    assert (np.abs(deq - xv) <= bound).all()
