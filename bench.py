@@ -299,9 +299,10 @@ def run_ours(args, rank, world, device):
     idx = torch.empty((w.N, w.k), dtype=torch.int32, device=device)
     wts = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
     L = api.Layout.empty(w.N, w.k, w.E, w.R, device)
-    if w.dtype == "fp8":
+    if w.dtype != "bf16":
         recv = torch.empty((w.S, w.H), dtype=torch.uint8, device=device)
-        scale = torch.empty((w.S, w.H // 128), dtype=torch.float32, device=device)
+        shape, sdt = api.scale_shape(w.S, w.H, w.dtype_code)
+        scale = torch.empty(shape, dtype=sdt, device=device)
     else:
         recv = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
         scale = None
@@ -427,6 +428,29 @@ def run_ours(args, rank, world, device):
         if int(L.status.item()) != 0:
             raise RuntimeError(f"device status {int(L.status.item())} after the backward ops")
 
+    variants = None
+    if not args.no_backward:
+        # every dispatch payload type on this shape, each alone (cold, clean L2)
+        from combine_moe_topk_gate_b200.workloads import DTYPES, Workload
+        bufs = {}
+        for dname, code in DTYPES.items():
+            rx = torch.empty((w.S, w.H), dtype=torch.bfloat16 if code == 0 else torch.uint8, device=device)
+            shape, sdt = api.scale_shape(w.S, w.H, code)
+            bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
+
+        def var_ops():
+            return {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
+                                                                  d_status=L.status))
+                    for d, (c, rx, rs) in bufs.items()}
+        vt = isolated_op_times(var_ops, flush, device)
+        peak_v, _ = measured_peak()
+        variants = {}
+        for d, us in vt.items():
+            abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": d}))["dispatch"]
+            variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
+                           "algorithmic_bytes": abv}
+        del bufs
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world)
@@ -471,6 +495,7 @@ def run_ours(args, rank, world, device):
         "gpu_launches": 2 * launches_per_step(w) * args.steps,  # two timed loops
         "isolated_us": isolated,
         "backward": backward,
+        "dispatch_variants": variants,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

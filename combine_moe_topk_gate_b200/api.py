@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX, MOE_ERR_TIMEOUT = range(6)
 MOE_GATE_SOFTMAX, MOE_GATE_SOFTMAX_RENORM, MOE_GATE_SIGMOID_GROUP = range(3)
-MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3 = range(2)
+MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_TOKEN, MOE_DTYPE_MXFP8_E4M3 = range(4)
 MOE_MAX_EXPERTS = 1024
 MOE_MAX_TOPK = 32
 MOE_FP8_BLOCK = 128
@@ -49,7 +49,7 @@ def _load() -> ctypes.CDLL:
     L.moe_get_layout_noalloc.restype = I
     L.moe_recv_bytes.argtypes = [I, I, I, I]
     L.moe_recv_bytes.restype = SZ
-    L.moe_scale_bytes.argtypes = [I, I, I]
+    L.moe_scale_bytes.argtypes = [I, I, I, I]
     L.moe_scale_bytes.restype = SZ
     L.moe_dispatch.argtypes = [P, I, I, I, P, I, P, P, P, P]
     L.moe_dispatch.restype = I
@@ -202,15 +202,27 @@ def moe_recv_bytes(num_tokens: int, hidden: int, k: int, dtype: int) -> int:
     return int(_lib.moe_recv_bytes(num_tokens, hidden, k, dtype))
 
 
-def moe_scale_bytes(num_tokens: int, hidden: int, k: int) -> int:
-    return int(_lib.moe_scale_bytes(num_tokens, hidden, k))
+def moe_scale_bytes(num_tokens: int, hidden: int, k: int, dtype: int = MOE_DTYPE_FP8_E4M3) -> int:
+    return int(_lib.moe_scale_bytes(num_tokens, hidden, k, dtype))
+
+
+def scale_shape(S: int, H: int, dtype: int):
+    """(shape, torch dtype) of recv_scale for a payload type (None for BF16)."""
+    if dtype == MOE_DTYPE_FP8_E4M3:
+        return (S, H // MOE_FP8_BLOCK), torch.float32
+    if dtype == MOE_DTYPE_FP8_E4M3_TOKEN:
+        return (S, 1), torch.float32
+    if dtype == MOE_DTYPE_MXFP8_E4M3:
+        return (S, H // 32), torch.uint8
+    return None, None
 
 
 def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_x=None,
                  recv_scale=None, d_status=None, stream=None):
     """Scatter rows of ``x`` (bf16 [N,H]) to their receive rows.  Returns
     ``(recv_x, recv_scale)``: bf16 [N*k,H] and None, or uint8 e4m3 codes
-    [N*k,H] and fp32 [N*k,H/128]."""
+    [N*k,H] with fp32 [N*k,H/128] (per block), fp32 [N*k,1] (per token) or
+    uint8 E8M0 bytes [N*k,H/32] (MXFP8)."""
     _need(x, "x", torch.bfloat16)
     N, H = x.shape
     _need(token_slot, "token_slot", torch.int32)
@@ -222,12 +234,15 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
         _need(recv_x, "recv_x", torch.bfloat16, (S, H))
         recv_scale = None
     else:
+        shape, sdt = scale_shape(S, H, dtype)
+        if shape is None:
+            raise ValueError(f"unknown dispatch dtype {dtype}")
         if recv_x is None:
             recv_x = torch.empty((S, H), dtype=torch.uint8, device=x.device)
         if recv_scale is None:
-            recv_scale = torch.empty((S, H // MOE_FP8_BLOCK), dtype=torch.float32, device=x.device)
+            recv_scale = torch.empty(shape, dtype=sdt, device=x.device)
         _need(recv_x, "recv_x", torch.uint8, (S, H))
-        _need(recv_scale, "recv_scale", torch.float32, (S, H // MOE_FP8_BLOCK))
+        _need(recv_scale, "recv_scale", sdt, shape)
     st = _lib.moe_dispatch(_ptr(x), N, H, k, _ptr(token_slot), dtype, _ptr(recv_x),
                            _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
     _check(st, "moe_dispatch")

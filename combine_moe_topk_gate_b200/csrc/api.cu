@@ -94,14 +94,20 @@ size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
   return static_cast<size_t>(num_tokens) * k * hidden * esz;
 }
 
-size_t moe_scale_bytes(int num_tokens, int hidden, int k) {
+size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
   if (num_tokens < 0 || hidden < 1 || k < 1) return 0;
-  return static_cast<size_t>(num_tokens) * k * (hidden / MOE_FP8_BLOCK) * sizeof(float);
+  const size_t rows = static_cast<size_t>(num_tokens) * k;
+  switch (dtype) {
+    case MOE_DTYPE_FP8_E4M3: return rows * (hidden / MOE_FP8_BLOCK) * sizeof(float);
+    case MOE_DTYPE_FP8_E4M3_TOKEN: return rows * sizeof(float);
+    case MOE_DTYPE_MXFP8_E4M3: return rows * (hidden / 32);
+    default: return 0;
+  }
 }
 
 moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
                           const int32_t* token_slot, moe_dtype_t dtype, void* recv_x,
-                          float* recv_scale, int32_t* d_status, moe_stream_t stream) {
+                          void* recv_scale, int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
   if (N < 0 || H < 1 || k < 1) return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
@@ -110,12 +116,18 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
     if (H % 8 != 0) return MOE_ERR_INVALID_ARG;
   } else if (dtype == MOE_DTYPE_FP8_E4M3) {
     if (H % MOE_FP8_BLOCK != 0) return MOE_ERR_INVALID_ARG;
+  } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
+    if (H % 8 != 0) return MOE_ERR_INVALID_ARG;
+    if (H > 16384) return MOE_ERR_UNSUPPORTED;
+  } else if (dtype == MOE_DTYPE_MXFP8_E4M3) {
+    if (H % 32 != 0) return MOE_ERR_INVALID_ARG;
   } else {
     return MOE_ERR_INVALID_ARG;
   }
   if (N == 0) return MOE_OK;
   if (!x || !token_slot || !recv_x) return MOE_ERR_INVALID_ARG;
-  if (dtype == MOE_DTYPE_FP8_E4M3 && (!recv_scale || !aligned(recv_scale, 4)))
+  if (dtype != MOE_DTYPE_BF16 && !recv_scale) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_BF16 && !aligned(recv_scale, dtype == MOE_DTYPE_MXFP8_E4M3 ? 16 : 4))
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(token_slot, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;

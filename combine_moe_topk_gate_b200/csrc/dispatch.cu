@@ -87,6 +87,165 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// MXFP8 (OCP Microscaling): 32-element blocks share X = 2^e with
+// e = floor(log2(amax)) - 8, stored as the E8M0 byte e + 127; elements are
+// e4m3(x * 2^-e), saturating (x * 2^-e can reach 511.x).  Same work split as
+// the per-block kernel: lane owns 16 channels, 2 lanes = one block, a warp
+// covers 512 channels and gathers its 16 scale bytes into one 16-byte store.
+__device__ __forceinline__ int floor_log2_pos(float a) {  // a > 0, finite; exact
+  const uint32_t u = __float_as_uint(a);
+  const int ex = static_cast<int>((u >> 23) & 0xffu);
+  return ex ? ex - 127 : (31 - __clz(u & 0x7fffffu)) - 149;
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+    dispatch_mxfp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                          const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
+                          uint8_t* __restrict__ recv_e8m0, int32_t* d_status) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (H + 511) / 512;
+  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (item >= static_cast<long long>(N) * segs) return;
+  const int t = static_cast<int>(item / segs);
+  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
+  const int c0 = s * 512 + lane * 16;
+  const bool active = c0 < H;  // H % 32 == 0: whole 2-lane blocks are in or out
+  const long long S = static_cast<long long>(N) * k;
+  const int nblk = H / 32;
+  pdl_wait();
+  pdl_trigger();
+
+  const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (active) {
+    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
+    a = ld_stream(src);
+    b = ld_stream(src + 8);
+  }
+  float f[16];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    f[2 * i] = bf16_lo(w[i]);
+    f[2 * i + 1] = bf16_hi(w[i]);
+  }
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+  int e = amax > 0.0f ? floor_log2_pos(amax) - 8 : -127;
+  e = e < -127 ? -127 : (e > 127 ? 127 : e);
+  const float down = __int_as_float((127 - e) << 23);  // 2^-e; e <= 119 for bf16 input
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float p[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float v = f[4 * i + u];
+      p[u] = (v == 0.0f) ? v : __fmul_rn(v, down);  // exact scaling by a power of two
+    }
+    q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+  }
+  const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+  // the warp's 16 scale bytes (block i sits in lane 2i)
+  const uint32_t my_byte = static_cast<uint32_t>(e + 127);
+  uint32_t sw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    sw[i] = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) sw[i] |= (__shfl_sync(kFullMask, my_byte, 2 * (4 * i + u)) & 0xffu) << (8 * u);
+  }
+  const bool whole16 = (H % 512) == 0;  // 16-byte aligned, full 16 scale bytes per warp
+  for (int j = 0; j < k; ++j) {
+    const int slot = __shfl_sync(kFullMask, my_slot, j);
+    if (slot == -1) continue;
+    if (slot < -1 || slot >= S) {
+      if (lane == 0) report_bad_index(d_status);
+      continue;
+    }
+    if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
+    uint8_t* srow = recv_e8m0 + static_cast<size_t>(slot) * nblk;
+    if (whole16) {
+      if (lane == 0) st_v4(srow + s * 16, make_uint4(sw[0], sw[1], sw[2], sw[3]));
+    } else if (active && (lane & 1) == 0) {
+      srow[c0 >> 5] = static_cast<uint8_t>(my_byte);
+    }
+  }
+}
+
+// FP8 with one scale per token: one CTA per token, the row held in registers
+// (VPT 16-byte vectors per thread), amax reduced over the CTA, then the same
+// code rule as the blocks: scale = amax/448, codes e4m3(x * (448/amax)).
+constexpr int kTokenThreads = 256;
+
+template <int VPT>
+__global__ void __launch_bounds__(kTokenThreads)
+    dispatch_fp8_token_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                              const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
+                              float* __restrict__ recv_scale, int32_t* d_status) {
+  __shared__ float warp_max[kTokenThreads / 32];
+  __shared__ int slots[MOE_MAX_TOPK];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.x;
+  const int nvec = H / 8;
+  const long long S = static_cast<long long>(N) * k;
+  pdl_wait();
+  pdl_trigger();
+  if (tid < k) {
+    const int sl = token_slot[static_cast<size_t>(t) * k + tid];
+    slots[tid] = sl;
+    if (sl < -1 || sl >= S) report_bad_index(d_status);
+  }
+  uint4 v[VPT];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = i * kTokenThreads + tid;
+    v[i] = make_uint4(0, 0, 0, 0);
+    if (vi < nvec) v[i] = ld_stream(x + static_cast<size_t>(t) * H + static_cast<size_t>(vi) * 8);
+    const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[u])), fabsf(bf16_hi(w4[u]))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int w2 = 1; w2 < kTokenThreads / 32; ++w2) amax = fmaxf(amax, warp_max[w2]);
+  const float inv = __fdiv_rn(448.0f, amax);
+  const float scale = __fdiv_rn(amax, 448.0f);
+  uint2 q[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    float p[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float lo = bf16_lo(w4[u]), hi = bf16_hi(w4[u]);
+      p[2 * u] = (lo == 0.0f) ? lo : __fmul_rn(lo, inv);
+      p[2 * u + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, inv);
+    }
+    q[i].x = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+    q[i].y = e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16);
+  }
+  for (int j = 0; j < k; ++j) {
+    const int slot = slots[j];
+    if (slot < 0 || slot >= S) continue;
+    uint8_t* row = recv_x + static_cast<size_t>(slot) * H;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = i * kTokenThreads + tid;
+      if (vi < nvec) *reinterpret_cast<uint2*>(row + static_cast<size_t>(vi) * 8) = q[i];
+    }
+    if (tid == 0) recv_scale[slot] = scale;
+  }
+}
+
 // BF16: lane owns 8 channels (one 16-byte vector), a warp covers 256 channels.
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_bf16_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
@@ -133,15 +292,33 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
 }  // namespace
 
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            int dtype, void* recv_x, float* recv_scale, int32_t* d_status,
+                            int dtype, void* recv_x, void* recv_scale, int32_t* d_status,
                             cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
-  if (dtype == MOE_DTYPE_FP8_E4M3) {
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint8_t* r8 = static_cast<uint8_t*>(recv_x);
+  if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3) {
     const long long items = static_cast<long long>(N) * ((H + 511) / 512);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-    return launch_pdl(dispatch_fp8_kernel, blocks, kWarps * 32, 0, stream,
-                      static_cast<const uint16_t*>(x), N, H, k, token_slot,
-                      static_cast<uint8_t*>(recv_x), recv_scale, d_status);
+    if (dtype == MOE_DTYPE_FP8_E4M3)
+      return launch_pdl(dispatch_fp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
+                        token_slot, r8, static_cast<float*>(recv_scale), d_status);
+    return launch_pdl(dispatch_mxfp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
+                      token_slot, r8, static_cast<uint8_t*>(recv_scale), d_status);
+  } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
+    const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
+    float* sc = static_cast<float*>(recv_scale);
+    if (vpt <= 1)
+      return launch_pdl(dispatch_fp8_token_kernel<1>, N, kTokenThreads, 0, stream, xs, N, H, k,
+                        token_slot, r8, sc, d_status);
+    if (vpt <= 2)
+      return launch_pdl(dispatch_fp8_token_kernel<2>, N, kTokenThreads, 0, stream, xs, N, H, k,
+                        token_slot, r8, sc, d_status);
+    if (vpt <= 4)
+      return launch_pdl(dispatch_fp8_token_kernel<4>, N, kTokenThreads, 0, stream, xs, N, H, k,
+                        token_slot, r8, sc, d_status);
+    return launch_pdl(dispatch_fp8_token_kernel<8>, N, kTokenThreads, 0, stream, xs, N, H, k,
+                      token_slot, r8, sc, d_status);
   } else {
     const long long items = static_cast<long long>(N) * ((H + 255) / 256);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);

@@ -21,7 +21,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
                           cudaStream_t stream);
 
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            int dtype, void* recv_x, float* recv_scale, int32_t* d_status,
+                            int dtype, void* recv_x, void* recv_scale, int32_t* d_status,
                             cudaStream_t stream);
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,

@@ -29,7 +29,7 @@ from dataclasses import dataclass, field
 import torch
 
 GATE_KINDS = {"softmax": 0, "softmax_renorm": 1, "sigmoid_group": 2}
-DTYPES = {"bf16": 0, "fp8": 1}
+DTYPES = {"bf16": 0, "fp8": 1, "fp8_token": 2, "mxfp8": 3}
 
 
 @dataclass(frozen=True)
@@ -41,7 +41,7 @@ class Workload:
     k: int                 # experts per token
     R: int                 # logical EP ranks (partitions of the receive buffer)
     gate: str              # "softmax" | "softmax_renorm" | "sigmoid_group"
-    dtype: str             # dispatch payload: "bf16" | "fp8"
+    dtype: str             # dispatch payload: "bf16" | "fp8" | "fp8_token" | "mxfp8"
     expert_out: str        # "identity" (y = recv_x) | "random" (seeded bf16 y)
     n_groups: int = 1
     topk_groups: int = 1
@@ -121,8 +121,9 @@ def algorithmic_bytes(w: Workload) -> dict:
     """Bytes each step must move at least once (each token row read once,
     written k times; int32 metadata of the step included)."""
     N, H, E, k = w.N, w.H, w.E, w.k
-    b = 1 if w.dtype == "fp8" else 2
-    scales = 4 * N * k * (H // 128) if w.dtype == "fp8" else 0
+    b = 2 if w.dtype == "bf16" else 1
+    scales = {"fp8": 4 * N * k * (H // 128), "fp8_token": 4 * N * k,
+              "mxfp8": N * k * (H // 32)}.get(w.dtype, 0)
     return {
         "gate": 4 * N * E + 8 * N * k,
         "layout": 4 * N * k + 8 * N * k + 4 * (4 * E + 3 * w.R),

@@ -69,8 +69,10 @@ typedef enum {
 } moe_gate_kind_t;
 
 typedef enum {
-    MOE_DTYPE_BF16 = 0,          /* payload copied as bf16                            */
-    MOE_DTYPE_FP8_E4M3 = 1       /* payload quantised to e4m3, one fp32 scale / 128ch */
+    MOE_DTYPE_BF16 = 0,          /* payload copied as bf16                              */
+    MOE_DTYPE_FP8_E4M3 = 1,      /* e4m3, one fp32 scale per 128 channels               */
+    MOE_DTYPE_FP8_E4M3_TOKEN = 2,/* e4m3, one fp32 scale per token row                  */
+    MOE_DTYPE_MXFP8_E4M3 = 3     /* OCP MXFP8: e4m3, one E8M0 scale byte per 32 channels */
 } moe_dtype_t;
 
 typedef void* moe_stream_t;      /* a cudaStream_t */
@@ -177,8 +179,9 @@ moe_status_t moe_get_layout_noalloc(const int32_t* topk_idx, int num_tokens, int
 
 /* Receive-buffer payload bytes: N*k rows of H bf16 (2 B) or e4m3 (1 B). */
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
-/* FP8 scale bytes: N*k rows of H/128 fp32. */
-size_t moe_scale_bytes(int num_tokens, int hidden, int k);
+/* Scale bytes for the FP8 payloads: N*k rows of H/128 fp32 (per block), of one
+ * fp32 (per token) or of H/32 E8M0 bytes (MXFP8); 0 for BF16. */
+size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
 
 /*
  * moe_dispatch -- scatter each token's row to all of its receive rows.
@@ -196,12 +199,22 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k);
  *          product, IEEE rounding); zeros keep their sign (so an all-zero
  *          block gives scale 0 and zero codes).  H % 128 == 0; x, recv_x
  *          16-byte aligned, recv_scale 4-byte aligned.
+ *   FP8 per token ([TK]: "pro Token"): recv_x e4m3 [S, H], recv_scale fp32
+ *          [S, 1]: amax over the whole row, then the same rule as the
+ *          blocks.  H % 8 == 0 and H <= 16384.
+ *   MXFP8 (OCP Microscaling, the block-scaled FP8 of Blackwell's block-scaled
+ *          MMA): recv_x e4m3 [S, H], recv_scale viewed as uint8 [S, H/32].
+ *          Per 32-channel block: e = floor(log2(amax)) - 8 (clamped to
+ *          [-127, 127], -127 for an all-zero block), scale byte e + 127,
+ *          codes e4m3_rne_satfinite(x * 2^-e) (the power-of-two scaling is
+ *          exact; values up to 511.x saturate to 448).  H % 32 == 0;
+ *          recv_scale 16-byte aligned.
  *   Rows no slot names are not written.  A slot outside [-1, S) is skipped
  *   and reported through d_status.
  */
 moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
                           const int32_t* token_slot, moe_dtype_t dtype, void* recv_x,
-                          float* recv_scale, int32_t* d_status, moe_stream_t stream);
+                          void* recv_scale, int32_t* d_status, moe_stream_t stream);
 
 /*
  * moe_combine -- weighted gather-reduce of each token's k expert outputs.

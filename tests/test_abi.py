@@ -40,6 +40,9 @@ def test_size_queries(api):
     assert api.moe_recv_bytes(4096, 7168, 8, api.MOE_DTYPE_FP8_E4M3) == 4096 * 8 * 7168
     assert api.moe_recv_bytes(16384, 4096, 2, api.MOE_DTYPE_BF16) == 16384 * 2 * 4096 * 2
     assert api.moe_scale_bytes(4096, 7168, 8) == 4096 * 8 * 56 * 4
+    assert api.moe_scale_bytes(4096, 7168, 8, api.MOE_DTYPE_FP8_E4M3_TOKEN) == 4096 * 8 * 4
+    assert api.moe_scale_bytes(4096, 7168, 8, api.MOE_DTYPE_MXFP8_E4M3) == 4096 * 8 * 224
+    assert api.moe_scale_bytes(4096, 7168, 8, api.MOE_DTYPE_BF16) == 0
     ws = api.moe_layout_workspace_bytes(4096, 8, 256, 32)
     assert ws >= 256 and ws % 256 == 0
     assert api.moe_layout_workspace_bytes(0, 8, 256, 32) >= 256
@@ -100,6 +103,11 @@ def test_dispatch_combine_reject_bad_arguments(api):
     assert L.moe_dispatch(_P(), 10, 256, 2, _P(), FP8, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
     assert L.moe_dispatch(_P(0x1008), 10, 256, 2, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
     assert L.moe_dispatch(_P(), 10, 256, 2, _P(), 5, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    MX, TOK = api.MOE_DTYPE_MXFP8_E4M3, api.MOE_DTYPE_FP8_E4M3_TOKEN
+    assert L.moe_dispatch(_P(), 10, 272, 2, _P(), MX, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG  # H % 32
+    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), MX, _P(), _P(0x1008), None, None) == api.MOE_ERR_INVALID_ARG  # scales 16-B
+    assert L.moe_dispatch(_P(), 10, 20000, 2, _P(), TOK, _P(), _P(), None, None) == api.MOE_ERR_UNSUPPORTED
+    assert L.moe_dispatch(_P(), 10, 100, 2, _P(), TOK, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG  # H % 8
     assert L.moe_dispatch(_P(), 10, 256, 40, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_UNSUPPORTED
     assert L.moe_dispatch(None, 0, 256, 2, None, BF16, None, None, None, None) == api.MOE_OK
     assert L.moe_combine(_P(), 10, 100, 2, _P(), _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
