@@ -10,11 +10,12 @@
 // Selection keys.  A candidate (value v, expert e) is packed into 64 bits as
 // (order-preserving bits of v) << 32 | (0xffffffff - e), so a larger key means
 // a larger value and, on equal values, a lower index -- the tie rule.  -0.0 is
-// turned into +0.0 first so that the two compare equal.  One selection round
-// takes, per lane, the largest key below the previous winner and finds the
-// warp's largest with two redux.sync max operations (high word, then low word
-// among the lanes that hold the high maximum).  k rounds give the slots in
-// order.
+// turned into +0.0 first so that the two compare equal.  The warp's largest
+// key comes from two redux.sync max operations (high word, then low word among
+// the lanes that hold the high maximum); k rounds give the slots in order.
+// The lanes kernel sorts each lane's keys once, so a round is O(1) per lane
+// (offer the head, pop it if it won); the generic kernel scans its keys for
+// the largest one below the previous winner.
 //
 // Two kernels:
 //  * lanes kernel (E = 32*V): lane l holds experts [l*V, (l+1)*V) -- one
@@ -92,6 +93,52 @@ __device__ __forceinline__ void select_topk(const uint64_t (&key)[V], int k, int
   }
 }
 
+// Sorts a lane's keys, largest first, with a fixed comparator network
+// (Knuth's 19-comparator network for 8 keys).
+__device__ __forceinline__ void cswap_desc(uint64_t& a, uint64_t& b) {
+  const uint64_t hi = a > b ? a : b, lo = a > b ? b : a;
+  a = hi;
+  b = lo;
+}
+template <int V>
+__device__ __forceinline__ void sort_desc(uint64_t (&k)[V]) {
+  if constexpr (V == 2) {
+    cswap_desc(k[0], k[1]);
+  } else if constexpr (V == 4) {
+    cswap_desc(k[0], k[1]); cswap_desc(k[2], k[3]);
+    cswap_desc(k[0], k[2]); cswap_desc(k[1], k[3]);
+    cswap_desc(k[1], k[2]);
+  } else if constexpr (V == 8) {
+    cswap_desc(k[0], k[2]); cswap_desc(k[1], k[3]); cswap_desc(k[4], k[6]); cswap_desc(k[5], k[7]);
+    cswap_desc(k[0], k[4]); cswap_desc(k[1], k[5]); cswap_desc(k[2], k[6]); cswap_desc(k[3], k[7]);
+    cswap_desc(k[0], k[1]); cswap_desc(k[2], k[3]); cswap_desc(k[4], k[5]); cswap_desc(k[6], k[7]);
+    cswap_desc(k[2], k[4]); cswap_desc(k[3], k[5]);
+    cswap_desc(k[1], k[4]); cswap_desc(k[3], k[6]);
+    cswap_desc(k[1], k[2]); cswap_desc(k[3], k[4]); cswap_desc(k[5], k[6]);
+  }
+}
+
+// Selection over per-lane lists sorted largest first: a lane offers its head,
+// the warp's largest head wins, and the winning lane pops it.  Lane j
+// receives slot j; every lane gets the slot-order sum of the winners' values.
+template <int V>
+__device__ __forceinline__ void select_sorted(uint64_t (&key)[V], int k, int lane, int& sel_i,
+                                              float& sel_v, float& sum) {
+  for (int j = 0; j < k; ++j) {
+    const uint64_t win = warp_max_key(key[0]);
+    const float wv = key_value(win);
+    sum = (j == 0) ? wv : __fadd_rn(sum, wv);
+    if (lane == j) {
+      sel_i = key_index(win);
+      sel_v = wv;
+    }
+    const bool pop = win != 0 && key[0] == win;
+#pragma unroll
+    for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
+    key[V - 1] = pop ? 0 : key[V - 1];
+  }
+}
+
 // ------------------------------------------------------------------ lanes kernel
 // Softmax needs Z summed in ascending expert order: the exp terms go to shared
 // memory and lane 0 adds them one by one.
@@ -134,18 +181,11 @@ __global__ void __launch_bounds__(kGateWarps * 32)
     if (kind == MOE_GATE_SIGMOID_GROUP) {
 #pragma unroll
       for (int v = 0; v < V; ++v) key[v] = make_key(logistic(l[v]), e0 + v);
+      sort_desc<V>(key);
       // this lane's top-n, best first (key 0 pads when n > V)
       uint64_t top[topn];
-      uint64_t prev = ~0ull;
 #pragma unroll
-      for (int p = 0; p < topn; ++p) {
-        uint64_t best = 0;
-#pragma unroll
-        for (int v = 0; v < V; ++v)
-          if (key[v] < prev && key[v] > best) best = key[v];
-        top[p] = best;
-        prev = best;
-      }
+      for (int p = 0; p < topn; ++p) top[p] = p < V ? key[p < V ? p : 0] : 0;
       // merge with the other lanes of the group: top-n of two sorted lists is
       // max(a_i, b_{n-1-i}) (a bitonic sequence), then sorted again
 #pragma unroll
@@ -183,7 +223,7 @@ __global__ void __launch_bounds__(kGateWarps * 32)
 #pragma unroll
         for (int v = 0; v < V; ++v) key[v] = 0;
       }
-      select_topk<V>(key, k, lane, sel_i, sel_v, sum);
+      select_sorted<V>(key, k, lane, sel_i, sel_v, sum);
       if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
     } else {
       float m = l[0];
@@ -201,13 +241,9 @@ __global__ void __launch_bounds__(kGateWarps * 32)
       if (lane == 0)
         for (int i = 0; i < E; ++i) z = __fadd_rn(z, sh_exp[warp][i]);
       z = __shfl_sync(kFullMask, z, 0);
-      uint64_t prev = ~0ull;
+      sort_desc<V>(key);
       for (int j = 0; j < k; ++j) {
-        uint64_t best = 0;
-#pragma unroll
-        for (int v = 0; v < V; ++v)
-          if (key[v] < prev && key[v] > best) best = key[v];
-        const uint64_t win = warp_max_key(best);
+        const uint64_t win = warp_max_key(key[0]);
         const int wi = key_index(win);
         const float p = (wi >= 0 && wi < E) ? __fdiv_rn(sh_exp[warp][wi], z) : 0.0f;
         sum = (j == 0) ? p : __fadd_rn(sum, p);
@@ -215,7 +251,10 @@ __global__ void __launch_bounds__(kGateWarps * 32)
           sel_i = (wi >= 0 && wi < E) ? wi : -1;
           sel_v = p;
         }
-        prev = win;
+        const bool pop = win != 0 && key[0] == win;
+#pragma unroll
+        for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
+        key[V - 1] = pop ? 0 : key[V - 1];
       }
       if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
       __syncwarp();  // sh_exp is rewritten for the next token
