@@ -85,13 +85,18 @@ def _declare(L):
     L.oracle_topk_gate.restype = _I
     L.oracle_get_layout.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]
     L.oracle_get_layout.restype = _I
+    _L64 = ctypes.c_int64
+    L.oracle_get_layout_aligned.argtypes = [_P, _I, _I, _I, _I, _I, _L64, _P, _P, _P, _P, _P, _P, _P]
+    L.oracle_get_layout_aligned.restype = _I
     L.oracle_dispatch.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P]
     L.oracle_dispatch.restype = _I
-    L.oracle_combine.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+    L.oracle_dispatch_rows.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _P, _P]
+    L.oracle_dispatch_rows.restype = _I
+    L.oracle_combine.argtypes = [_P, _L64, _I, _I, _I, _P, _P, _P]
     L.oracle_combine.restype = _I
-    L.oracle_dispatch_backward.argtypes = [_P, _I, _I, _I, _P, _P]
+    L.oracle_dispatch_backward.argtypes = [_P, _L64, _I, _I, _I, _P, _P]
     L.oracle_dispatch_backward.restype = _I
-    L.oracle_combine_backward.argtypes = [_P, _P, _I, _I, _I, _P, _P, _P, _P, _P]
+    L.oracle_combine_backward.argtypes = [_P, _P, _L64, _I, _I, _I, _P, _P, _P, _P, _P]
     L.oracle_combine_backward.restype = _I
 
 
@@ -198,6 +203,24 @@ def get_layout(topk_idx: np.ndarray, E: int, R: int) -> Layout:
     return L
 
 
+def get_layout_aligned(topk_idx: np.ndarray, E: int, R: int, align: int, num_rows: int) -> Layout:
+    """Layout whose experts start at multiples of ``align`` rows; ``slot_token``
+    covers ``num_rows`` rows (-1 where no token lands)."""
+    topk_idx = _c(topk_idx, np.int32)
+    N, k = topk_idx.shape
+    L = Layout(np.empty(E, np.int32), np.empty(E + 1, np.int32), np.empty(R, np.int32),
+               np.empty(R + 1, np.int32), np.empty(R, np.int32), np.empty((N, k), np.int32),
+               np.empty(num_rows, np.int32), OK)
+    st = lib().oracle_get_layout_aligned(_ptr(topk_idx), N, k, E, R, align, num_rows,
+                                         _ptr(L.expert_count), _ptr(L.expert_offset),
+                                         _ptr(L.rank_count), _ptr(L.rank_offset), _ptr(L.rank_tokens),
+                                         _ptr(L.token_slot), _ptr(L.slot_token))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_get_layout_aligned: invalid argument")
+    L.status = st
+    return L
+
+
 def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
              recv_rows: int | None = None):
     """Returns (recv_x, recv_scale or None, status).  Rows no slot names stay 0.
@@ -221,7 +244,7 @@ def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
         else:                                   # MXFP8: E8M0 bytes, one per 32 channels
             scale = np.zeros((S, H // 32), np.uint8)
         sp = _ptr(scale)
-    st = lib().oracle_dispatch(_ptr(x_bf16), N, H, k, _ptr(token_slot), dtype, _ptr(recv), sp)
+    st = lib().oracle_dispatch_rows(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, dtype, _ptr(recv), sp)
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch: invalid argument")
     return recv, scale, st
@@ -235,7 +258,8 @@ def combine(y_bf16: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray):
     N, k = token_slot.shape
     H = y_bf16.shape[1]
     out = np.empty((N, H), np.uint16)
-    st = lib().oracle_combine(_ptr(y_bf16), N, H, k, _ptr(token_slot), _ptr(topk_w), _ptr(out))
+    st = lib().oracle_combine(_ptr(y_bf16), y_bf16.shape[0], N, H, k, _ptr(token_slot), _ptr(topk_w),
+                              _ptr(out))
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_combine: invalid argument")
     return out, st
@@ -248,7 +272,8 @@ def dispatch_backward(grad_recv_bf16: np.ndarray, token_slot: np.ndarray):
     N, k = token_slot.shape
     H = grad_recv_bf16.shape[1]
     gx = np.empty((N, H), np.uint16)
-    st = lib().oracle_dispatch_backward(_ptr(grad_recv_bf16), N, H, k, _ptr(token_slot), _ptr(gx))
+    st = lib().oracle_dispatch_backward(_ptr(grad_recv_bf16), grad_recv_bf16.shape[0], N, H, k,
+                                        _ptr(token_slot), _ptr(gx))
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch_backward: invalid argument")
     return gx, st
@@ -267,8 +292,8 @@ def combine_backward(grad_out_bf16: np.ndarray, y_bf16: np.ndarray, token_slot: 
     gy = np.zeros((y_bf16.shape[0], H), np.uint16)
     gw = np.empty((N, k), np.float32)
     mag = np.empty((N, k), np.float64)
-    st = lib().oracle_combine_backward(_ptr(grad_out_bf16), _ptr(y_bf16), N, H, k, _ptr(token_slot),
-                                       _ptr(topk_w), _ptr(gy), _ptr(gw), _ptr(mag))
+    st = lib().oracle_combine_backward(_ptr(grad_out_bf16), _ptr(y_bf16), y_bf16.shape[0], N, H, k,
+                                       _ptr(token_slot), _ptr(topk_w), _ptr(gy), _ptr(gw), _ptr(mag))
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_combine_backward: invalid argument")
     return gy, gw, mag, st

@@ -377,6 +377,78 @@ int oracle_get_layout(const int32_t* topk_idx, int N, int k, int E, int R,
 }
 
 /* ------------------------------------------------------------------ */
+/* GEMM-aligned layout.  [EPv2] mentions a "new GEMM layout" without
+ * defining it; the reading taken: each expert's rows start at a multiple of
+ * `align` so a grouped GEMM can tile every expert by align rows.
+ *   expert_offset[e] = sum_{e' < e} round_up(expert_count[e'], align)
+ *   token_slot[t,j]  = expert_offset[e] + (rank of (t,j) inside e, as before)
+ *   slot_token[s]    = the token of row s, -1 for every other row in
+ *                      [0, num_rows) (padding, masked tail, spare capacity)
+ *   rank_offset[r]   = expert_offset[r*E/R]; rank_count[r] = the rows of rank
+ *                      r's region, padding included.
+ * num_rows must be at least expert_offset[E] + (masked entries); N*k +
+ * E*(align-1) always suffices.  align = 1 is the packed layout.          */
+/* ------------------------------------------------------------------ */
+int oracle_get_layout_aligned(const int32_t* topk_idx, int N, int k, int E, int R,
+                              int align, int64_t num_rows, int32_t* expert_count,
+                              int32_t* expert_offset, int32_t* rank_count,
+                              int32_t* rank_offset, int32_t* rank_tokens,
+                              int32_t* token_slot, int32_t* slot_token)
+{
+    if (N < 0 || k < 1 || E < 1 || R < 1 || E % R != 0 || align < 1) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int epr = E / R;
+    int64_t S = (int64_t)N * k;
+    int64_t invalid = 0;
+    for (int e = 0; e < E; ++e) expert_count[e] = 0;
+    for (int64_t i = 0; i < S; ++i) {
+        int32_t e = topk_idx[i];
+        if (e >= 0 && e < E) expert_count[e] += 1;
+        else { invalid += 1; if (e != -1) status = ORC_ERR_BAD_INDEX; }
+    }
+    expert_offset[0] = 0;
+    for (int e = 0; e < E; ++e) {
+        int32_t padded = (expert_count[e] + align - 1) / align * align;
+        expert_offset[e + 1] = expert_offset[e] + padded;
+    }
+    if ((int64_t)expert_offset[E] + invalid > num_rows) return ORC_ERR_INVALID_ARG;
+    for (int64_t s = 0; s < num_rows; ++s) slot_token[s] = -1;
+    int32_t* cursor = (int32_t*)malloc(sizeof(int32_t) * (size_t)E);
+    for (int e = 0; e < E; ++e) cursor[e] = expert_offset[e];
+    for (int t = 0; t < N; ++t) {
+        for (int j = 0; j < k; ++j) {
+            int64_t i = (int64_t)t * k + j;
+            int32_t e = topk_idx[i];
+            if (e >= 0 && e < E) {
+                int32_t s = cursor[e]++;
+                token_slot[i] = s;
+                slot_token[s] = t;
+            } else {
+                token_slot[i] = -1;
+            }
+        }
+    }
+    free(cursor);
+    for (int r = 0; r < R; ++r) {
+        rank_offset[r] = expert_offset[r * epr];
+        rank_count[r] = expert_offset[(r + 1) * epr] - expert_offset[r * epr];
+        rank_tokens[r] = 0;
+    }
+    rank_offset[R] = expert_offset[E];
+    for (int t = 0; t < N; ++t) {
+        for (int r = 0; r < R; ++r) {
+            int hit = 0;
+            for (int j = 0; j < k; ++j) {
+                int32_t e = topk_idx[(int64_t)t * k + j];
+                if (e >= 0 && e < E && e / epr == r) hit = 1;
+            }
+            rank_tokens[r] += hit;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------ */
 /* Dispatch.  [pplx] Dispatch: each token's activations (with block scaling
  * factors when quantised) are sent to every expert it was routed to and
  * unpacked into one contiguous buffer per expert.  [EPv2] usage patterns:
@@ -415,11 +487,11 @@ static int floor_log2_pos(float a)   /* a > 0, finite: exact from the bits */
 }
 
 static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
-                                   const int32_t* token_slot, int dtype, uint8_t* recv_x,
-                                   float* recv_scale)
+                                   const int32_t* token_slot, int64_t num_rows, int dtype,
+                                   uint8_t* recv_x, float* recv_scale)
 {
     int status = ORC_OK;
-    int64_t S = (int64_t)N * k;
+    int64_t S = num_rows;
     int nb = dtype == DT_MXFP8_E4M3 ? H / 32 : 1;
     uint8_t* q = (uint8_t*)malloc((size_t)H);
     float* fsc = (float*)malloc(sizeof(float));
@@ -469,9 +541,20 @@ static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
     return status;
 }
 
+int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
+                         const int32_t* token_slot, int64_t num_rows, int dtype, void* recv_x,
+                         float* recv_scale);
 int oracle_dispatch(const uint16_t* x, int N, int H, int k,
                     const int32_t* token_slot, int dtype, void* recv_x,
                     float* recv_scale)
+{
+    return oracle_dispatch_rows(x, N, H, k, token_slot, (int64_t)N * k, dtype, recv_x, recv_scale);
+}
+
+/* the receive buffer holds num_rows rows (N*k for the packed layout) */
+int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
+                         const int32_t* token_slot, int64_t num_rows, int dtype, void* recv_x,
+                         float* recv_scale)
 {
     if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
     if (dtype == DT_FP8_E4M3 && H % 128 != 0) return ORC_ERR_INVALID_ARG;
@@ -479,7 +562,8 @@ int oracle_dispatch(const uint16_t* x, int N, int H, int k,
     if (dtype == DT_FP8_E4M3_TOKEN && H % 8 != 0) return ORC_ERR_INVALID_ARG;
     if (dtype < DT_BF16 || dtype > DT_MXFP8_E4M3) return ORC_ERR_INVALID_ARG;
     if (dtype == DT_FP8_E4M3_TOKEN || dtype == DT_MXFP8_E4M3)
-        return oracle_dispatch_variant(x, N, H, k, token_slot, dtype, (uint8_t*)recv_x, recv_scale);
+        return oracle_dispatch_variant(x, N, H, k, token_slot, num_rows, dtype, (uint8_t*)recv_x,
+                                       recv_scale);
     int status = ORC_OK;
     int64_t S = (int64_t)N * k;
     int nb = H / 128;
@@ -530,13 +614,13 @@ int oracle_dispatch(const uint16_t* x, int N, int H, int k,
  * Masked slots (-1) contribute nothing; other out-of-range slots are
  * skipped and reported.                                                */
 /* ------------------------------------------------------------------ */
-int oracle_combine(const uint16_t* y, int N, int H, int k,
+int oracle_combine(const uint16_t* y, int64_t num_rows, int N, int H, int k,
                    const int32_t* token_slot, const float* topk_w,
                    uint16_t* out)
 {
     if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
     int status = ORC_OK;
-    int64_t S = (int64_t)N * k;
+    int64_t S = num_rows;   /* rows of y */
     for (int t = 0; t < N; ++t) {
         for (int c = 0; c < H; ++c) {
             float acc = 0.0f;
@@ -569,12 +653,12 @@ int oracle_combine(const uint16_t* y, int N, int H, int k,
  * The kernels may sum grad_w in another order in fp32; their error bound
  * follows from the arithmetic and is stated with the tests.            */
 /* ------------------------------------------------------------------ */
-int oracle_dispatch_backward(const uint16_t* grad_recv, int N, int H, int k,
+int oracle_dispatch_backward(const uint16_t* grad_recv, int64_t num_rows, int N, int H, int k,
                              const int32_t* token_slot, uint16_t* grad_x)
 {
     if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
     int status = ORC_OK;
-    int64_t S = (int64_t)N * k;
+    int64_t S = num_rows;   /* rows of grad_recv */
     for (int t = 0; t < N; ++t) {
         for (int c = 0; c < H; ++c) {
             float acc = 0.0f;
@@ -590,13 +674,13 @@ int oracle_dispatch_backward(const uint16_t* grad_recv, int N, int H, int k,
     return status;
 }
 
-int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int N, int H, int k,
-                            const int32_t* token_slot, const float* topk_w,
+int oracle_combine_backward(const uint16_t* grad_out, const uint16_t* y, int64_t num_rows, int N,
+                            int H, int k, const int32_t* token_slot, const float* topk_w,
                             uint16_t* grad_y, float* grad_w, double* grad_w_abs)
 {
     if (N < 0 || H < 1 || k < 1) return ORC_ERR_INVALID_ARG;
     int status = ORC_OK;
-    int64_t S = (int64_t)N * k;
+    int64_t S = num_rows;   /* rows of y and grad_y */
     for (int t = 0; t < N; ++t) {
         const uint16_t* g = grad_out + (size_t)t * H;
         for (int j = 0; j < k; ++j) {

@@ -40,6 +40,8 @@ MUTANTS = {
     "mxfp8_exponent_off_by_one": ("int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;",
                                   "int e = (amax > 0.0f) ? floor_log2_pos(amax) - 7 : -127;"),
     "fp8_token_scale_transposed": ("fsc[0] = amax / 448.0f;", "fsc[0] = 448.0f / amax;"),
+    "aligned_layout_rounds_down": ("int32_t padded = (expert_count[e] + align - 1) / align * align;",
+                                   "int32_t padded = expert_count[e] / align * align;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

@@ -621,3 +621,42 @@ def test_fp8_per_token_properties():
     deq = _torch_e4m3_decode_table()[recv[ts[:, 0]]] * sc[ts[:, 0]].astype(np.float64)
     bound = np.maximum(2.0**-4 * np.abs(xv), 2.0**-10 * sc[ts[:, 0]]) * (1 + 2.0**-20)
     assert (np.abs(deq - xv) <= bound).all()
+
+
+# ----------------------------------------------------------------- aligned layout
+def test_layout_aligned_worked_example():
+    g = _gold("layout_aligned_worked_example.json")
+    L = O.get_layout_aligned(np.array(g["topk_idx"], np.int32), g["E"], g["R"], g["align"], g["num_rows"])
+    for key in ("expert_count", "expert_offset", "rank_count", "rank_offset", "rank_tokens",
+                "token_slot", "slot_token"):
+        assert getattr(L, key).tolist() == g[key], key
+
+
+@pytest.mark.parametrize("N,k,E,R,align,mask", [(200, 8, 256, 32, 128, 0.0), (333, 2, 8, 8, 16, 0.1),
+                                                (64, 6, 12, 3, 8, 0.3), (50, 3, 16, 4, 1, 0.0)])
+def test_layout_aligned_vs_naive(N, k, E, R, align, mask):
+    rng = np.random.default_rng(N + align)
+    idx = rng.integers(0, E, (N, k)).astype(np.int32)
+    idx[rng.random((N, k)) < mask] = -1
+    rows = N * k + E * (align - 1)
+    L = O.get_layout_aligned(idx, E, R, align, rows)
+    flat = idx.reshape(-1)
+    counts = np.array([(flat == e).sum() for e in range(E)])
+    padded = -(-counts // align) * align
+    off = np.concatenate([[0], np.cumsum(padded)])
+    assert np.array_equal(L.expert_count, counts) and np.array_equal(L.expert_offset, off)
+    assert (L.expert_offset % align == 0).all()
+    ts = np.full(N * k, -1)
+    st = np.full(rows, -1)
+    for e in range(E):
+        pos = np.nonzero(flat == e)[0]
+        ts[pos] = off[e] + np.arange(len(pos))
+        st[off[e] + np.arange(len(pos))] = pos // k
+    assert np.array_equal(L.token_slot.reshape(-1), ts)
+    assert np.array_equal(L.slot_token, st)
+    epr = E // R
+    assert np.array_equal(L.rank_offset, off[::epr])
+    assert np.array_equal(L.rank_count, np.diff(off[::epr]))
+    if align == 1:   # reduces to the packed layout
+        P = O.get_layout(idx, E, R)
+        assert np.array_equal(P.token_slot, L.token_slot) and np.array_equal(P.expert_offset, L.expert_offset)
