@@ -22,9 +22,16 @@ MUTANTS = {
     "softmax_renorm_dropped": ("for (int j = 0; j < k; ++j) ow[j] = ow[j] / ps;", "(void)ps;"),
     "group_score_drops_second": ("for (int j = 1; j < group_topn; ++j) sum = sum + gv[gsel[j]];", "(void)0;"),
     "group_candidates_wrong_index": ("cand[(size_t)gsel[j] * eg + i] = 1;", "cand[(size_t)j * eg + i] = 1;"),
-    "layout_slot_token_stores_slot_index": ("slot_token[s] = t;", "slot_token[s] = j;"),
-    "layout_rank_offset_wrong_index": ("rank_offset[r] = expert_offset[r * epr];", "rank_offset[r] = expert_offset[r];"),
-    "layout_rank_tokens_modulo": ("if (e >= 0 && e < E && e / epr == r) hit = 1;", "if (e >= 0 && e < E && e % epr == r) hit = 1;"),
+    "layout_slot_token_stores_slot_index": ("slot_token[s] = t;", "slot_token[s] = j;", 0),
+    "aligned_slot_token_stores_slot_index": ("slot_token[s] = t;", "slot_token[s] = j;", 1),
+    "layout_rank_offset_wrong_index": ("rank_count[r] = c;\n        rank_offset[r] = expert_offset[r * epr];",
+                                       "rank_count[r] = c;\n        rank_offset[r] = expert_offset[r];"),
+    "aligned_rank_offset_wrong_index": ("        rank_offset[r] = expert_offset[r * epr];\n        rank_count[r] = expert_offset[(r + 1) * epr]",
+                                        "        rank_offset[r] = expert_offset[r];\n        rank_count[r] = expert_offset[(r + 1) * epr]"),
+    "layout_rank_tokens_modulo": ("if (e >= 0 && e < E && e / epr == r) hit = 1;",
+                                  "if (e >= 0 && e < E && e % epr == r) hit = 1;", 0),
+    "aligned_rank_tokens_modulo": ("if (e >= 0 && e < E && e / epr == r) hit = 1;",
+                                   "if (e >= 0 && e < E && e % epr == r) hit = 1;", 1),
     "fp8_scale_transposed": ("sc[b] = amax / 448.0f;", "sc[b] = 448.0f / amax;"),
     "e4m3_ties_away": ("double m = nearbyint(q);                     /* ties to even */",
                        "double m = floor(q + 0.5);"),
@@ -50,10 +57,16 @@ MUTANTS = {
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_pins_catch_mutant(name, tmp_path):
     src = open(SRC).read()
-    old, new = MUTANTS[name]
-    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    old, new, *which = MUTANTS[name]
+    if which:   # the anchor occurs in more than one function: mutate occurrence which[0]
+        parts = src.split(old)
+        assert len(parts) > which[0] + 1, f"mutation anchor occurrence missing: {old!r}"
+        mutated = old.join(parts[:which[0] + 1]) + new + old.join(parts[which[0] + 1:])
+    else:
+        assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+        mutated = src.replace(old, new)
     mut = tmp_path / "moe_oracle_mut.c"
-    mut.write_text(src.replace(old, new))
+    mut.write_text(mutated)
     lib = tmp_path / "liboracle_mut.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
                            "-shared", "-w", "-o", str(lib), str(mut), "-lm"])
