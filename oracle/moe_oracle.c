@@ -464,7 +464,8 @@ int oracle_get_layout_aligned(const int32_t* topk_idx, int N, int k, int E, int 
  *           is what the product gives whenever inv is finite and defines
  *           the all-zero block (amax = 0, scale = 0).
  * The same codes and scale go to every slot of the token.
- * A slot outside [-1, N*k) is skipped and reported.                    */
+ * A slot outside [-1, num_rows) is skipped and reported (num_rows = N*k  
+ * for the packed layout, more for a padded one).                        */
 /* ------------------------------------------------------------------ */
 /* Quantisation variants ([TK] list, "Quantisierung ... pro Token, pro Block"):
  *  DT_FP8_E4M3_TOKEN: one fp32 scale per token row: amax over the whole row,
@@ -565,7 +566,7 @@ int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
         return oracle_dispatch_variant(x, N, H, k, token_slot, num_rows, dtype, (uint8_t*)recv_x,
                                        recv_scale);
     int status = ORC_OK;
-    int64_t S = (int64_t)N * k;
+    int64_t S = num_rows;
     int nb = H / 128;
     uint8_t* q = (uint8_t*)malloc((size_t)H);
     float* sc = (float*)malloc(sizeof(float) * (size_t)(nb > 0 ? nb : 1));

@@ -660,3 +660,51 @@ def test_layout_aligned_vs_naive(N, k, E, R, align, mask):
     if align == 1:   # reduces to the packed layout
         P = O.get_layout(idx, E, R)
         assert np.array_equal(P.token_slot, L.token_slot) and np.array_equal(P.expert_offset, L.expert_offset)
+
+
+@pytest.mark.parametrize("dtype", [O.DT_BF16, O.DT_FP8_E4M3, O.DT_FP8_E4M3_TOKEN, O.DT_MXFP8_E4M3])
+def test_ops_on_padded_buffer_are_relocations_of_packed(dtype):
+    """Where a token's rows sit in the receive buffer changes nothing else: every
+    op on the padded (aligned) buffer equals the packed op with its rows moved,
+    padding rows are never written, and no in-range slot is reported bad."""
+    rng = np.random.default_rng(7 + dtype)
+    N, k, E, R, H, align = 90, 3, 12, 4, 256, 16
+    idx = rng.integers(0, E, (N, k)).astype(np.int32)
+    idx[rng.random((N, k)) < 0.15] = -1
+    rows = N * k + E * (align - 1) + 5
+    P = O.get_layout(idx, E, R)
+    A = O.get_layout_aligned(idx, E, R, align, rows)
+    assert A.status == 0 and int(A.token_slot.max()) >= N * k       # some rows beyond N*k
+    x = rng.normal(size=(N, H)).astype(np.float32)
+    x_bits = (torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    valid = P.token_slot >= 0
+    sp, sa = P.token_slot[valid], A.token_slot[valid]
+
+    rp, cp, stp = O.dispatch(x_bits, P.token_slot, dtype)
+    ra, ca, sta = O.dispatch(x_bits, A.token_slot, dtype, recv_rows=rows)
+    assert stp == 0 and sta == 0
+    assert np.array_equal(ra[sa], rp[sp])
+    unused = A.slot_token < 0
+    assert (ra[unused] == 0).all()
+    if cp is not None:
+        assert np.array_equal(ca[sa], cp[sp]) and (ca[unused] == 0).all()
+
+    w = rng.random((N, k)).astype(np.float32)
+    yp = rng.integers(0, 1 << 16, (N * k, H), dtype=np.uint16) & 0xBFFF     # finite bf16 patterns
+    ya = np.zeros((rows, H), np.uint16)
+    ya[sa] = yp[sp]
+    ya[unused] = 0x7FC0                                                       # NaN padding must not leak
+    op, s1 = O.combine(yp, P.token_slot, w)
+    oa, s2 = O.combine(ya, A.token_slot, w)
+    assert s1 == 0 and s2 == 0 and np.array_equal(oa, op)
+
+    gp, s1 = O.dispatch_backward(yp, P.token_slot)
+    ga, s2 = O.dispatch_backward(ya, A.token_slot)
+    assert s1 == 0 and s2 == 0 and np.array_equal(ga, gp)
+
+    go = x_bits
+    gyp, gwp, mp, s1 = O.combine_backward(go, yp, P.token_slot, w)
+    gya, gwa, ma, s2 = O.combine_backward(go, ya, A.token_slot, w)
+    assert s1 == 0 and s2 == 0
+    assert np.array_equal(gya[sa], gyp[sp]) and (gya[unused] == 0).all()
+    assert np.array_equal(gwa, gwp) and np.array_equal(ma, mp)
