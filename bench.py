@@ -451,6 +451,40 @@ def run_ours(args, rank, world, device):
                            "algorithmic_bytes": abv}
         del bufs
 
+    aligned = None
+    if not args.no_backward:
+        # the GEMM-aligned layout (every expert's rows start at a multiple of
+        # 128, one M tile) and the ops on its padded buffer, each alone
+        A = 128
+        rows_a = api.moe_aligned_recv_rows(w.N, w.k, w.E, A)
+        La = api.Layout.empty(w.N, w.k, w.E, w.R, device, align=A)
+        api.moe_get_layout(idx, w.E, w.R, align=A, out=La)
+        rx_a = torch.empty((rows_a, w.H), dtype=recv.dtype, device=device)
+        shape_a, sdt_a = api.scale_shape(rows_a, w.H, w.dtype_code)
+        rs_a = torch.empty(shape_a, dtype=sdt_a, device=device) if shape_a else None
+        y_a = torch.empty((rows_a, w.H), dtype=torch.bfloat16, device=device).normal_()
+        out_a = torch.empty_like(out)
+
+        def al_ops():
+            return {
+                "layout": lambda: api.moe_get_layout(idx, w.E, w.R, align=A, out=La),
+                "dispatch": lambda: api.moe_dispatch(x, La.token_slot, w.dtype_code, recv_x=rx_a,
+                                                     recv_scale=rs_a, d_status=La.status),
+                "combine": lambda: api.moe_combine(y_a, La.token_slot, wts, out=out_a, d_status=La.status),
+            }
+        at = isolated_op_times(al_ops, flush, device)
+        torch.cuda.synchronize(device)
+        if int(La.status.item()) != 0:
+            raise RuntimeError(f"device status {int(La.status.item())} after the aligned ops")
+        peak_a, _ = measured_peak()
+        ab_a = algorithmic_bytes(w)
+        aligned = {"align": A, "recv_rows": rows_a,
+                   "padding_rows": int(rows_a - w.S),
+                   **{n: {"us": us, "frac": (ab_a[n] / (us * 1e-6) / 1e9 / peak_a)
+                          if us and n != "layout" else None}
+                      for n, us in at.items()}}
+        del rx_a, rs_a, y_a, La
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world)
@@ -496,6 +530,7 @@ def run_ours(args, rank, world, device):
         "isolated_us": isolated,
         "backward": backward,
         "dispatch_variants": variants,
+        "aligned_layout": aligned,
         "clocks": clk.summary(),
         "e2e": e2e,
     }

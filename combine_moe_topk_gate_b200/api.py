@@ -22,6 +22,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_BAD_INDE
 MOE_GATE_SOFTMAX, MOE_GATE_SOFTMAX_RENORM, MOE_GATE_SIGMOID_GROUP = range(3)
 MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_TOKEN, MOE_DTYPE_MXFP8_E4M3 = range(4)
 MOE_MAX_EXPERTS = 1024
+MOE_MAX_ALIGN = 4096
 MOE_MAX_TOPK = 32
 MOE_FP8_BLOCK = 128
 
@@ -45,19 +46,23 @@ def _load() -> ctypes.CDLL:
     L.moe_layout_workspace_bytes.restype = SZ
     L.moe_get_layout.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P, P]
     L.moe_get_layout.restype = I
+    L.moe_get_layout_aligned.argtypes = [P, I, I, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P, P]
+    L.moe_get_layout_aligned.restype = I
+    L.moe_aligned_recv_rows.argtypes = [I, I, I, I]
+    L.moe_aligned_recv_rows.restype = SZ
     L.moe_get_layout_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, P]
     L.moe_get_layout_noalloc.restype = I
     L.moe_recv_bytes.argtypes = [I, I, I, I]
     L.moe_recv_bytes.restype = SZ
     L.moe_scale_bytes.argtypes = [I, I, I, I]
     L.moe_scale_bytes.restype = SZ
-    L.moe_dispatch.argtypes = [P, I, I, I, P, I, P, P, P, P]
+    L.moe_dispatch.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
     L.moe_dispatch.restype = I
-    L.moe_combine.argtypes = [P, I, I, I, P, P, P, P, P]
+    L.moe_combine.argtypes = [P, I, I, I, P, I, P, P, P, P]
     L.moe_combine.restype = I
-    L.moe_dispatch_backward.argtypes = [P, I, I, I, P, P, P, P]
+    L.moe_dispatch_backward.argtypes = [P, I, I, I, P, I, P, P, P]
     L.moe_dispatch_backward.restype = I
-    L.moe_combine_backward.argtypes = [P, P, I, I, I, P, P, P, P, P, P]
+    L.moe_combine_backward.argtypes = [P, P, I, I, I, P, I, P, P, P, P, P]
     L.moe_combine_backward.restype = I
     L.moe_e4m3_encode.argtypes = [P, SZ, P, P]
     L.moe_e4m3_encode.restype = I
@@ -135,40 +140,58 @@ class Layout:
     rank_offset: torch.Tensor    # int32 [R+1]
     rank_tokens: torch.Tensor    # int32 [R]
     token_slot: torch.Tensor     # int32 [N, k]
-    slot_token: torch.Tensor     # int32 [N*k]
+    slot_token: torch.Tensor     # int32 [num_rows]
     workspace: torch.Tensor      # uint8 scratch
     status: torch.Tensor         # int32 [1] device status word
+    align: int = 1               # expert row alignment of the receive buffer
+
+    @property
+    def num_rows(self) -> int:
+        """Rows of the receive buffer this layout addresses."""
+        return self.slot_token.numel()
 
     @staticmethod
-    def empty(N: int, k: int, E: int, R: int, device) -> "Layout":
+    def empty(N: int, k: int, E: int, R: int, device, align: int = 1, num_rows: int | None = None) -> "Layout":
         i32 = dict(dtype=torch.int32, device=device)
         ws = moe_layout_workspace_bytes(N, k, E, R)
+        rows = num_rows if num_rows is not None else moe_aligned_recv_rows(N, k, E, align)
         return Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32),
                       torch.empty(R + 1, **i32), torch.empty(R, **i32), torch.empty((N, k), **i32),
-                      torch.empty(N * k, **i32), torch.empty(ws, dtype=torch.uint8, device=device),
-                      torch.zeros(1, **i32))
+                      torch.empty(rows, **i32), torch.empty(ws, dtype=torch.uint8, device=device),
+                      torch.zeros(1, **i32), align)
 
 
 def moe_layout_workspace_bytes(num_tokens: int, k: int, num_experts: int, num_ranks: int) -> int:
     return int(_lib.moe_layout_workspace_bytes(num_tokens, k, num_experts, num_ranks))
 
 
-def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, out: Layout | None = None,
-                   stream=None) -> Layout:
-    """Counts, offsets and token<->slot maps; fills (and returns) ``out``.  The
-    device status word ``out.status`` is not cleared here: zero it to start a
-    fresh error record."""
+def moe_aligned_recv_rows(num_tokens: int, k: int, num_experts: int, align: int) -> int:
+    return int(_lib.moe_aligned_recv_rows(num_tokens, k, num_experts, align))
+
+
+def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, align: int = 1,
+                   num_recv_rows: int | None = None, out: Layout | None = None, stream=None) -> Layout:
+    """Counts, offsets and token<->slot maps; fills (and returns) ``out``.
+    ``align > 1`` starts every expert's rows at a multiple of ``align``
+    (moe_get_layout_aligned); the receive buffer then has ``out.num_rows`` rows.
+    The device status word ``out.status`` is not cleared here: zero it to start
+    a fresh error record."""
     _need(topk_idx, "topk_idx", torch.int32)
     N, k = topk_idx.shape
     E, R = num_experts, num_ranks
     if out is None:
-        out = Layout.empty(N, k, E, R, topk_idx.device)
-    st = _lib.moe_get_layout(_ptr(topk_idx), N, k, E, R, _ptr(out.expert_count),
-                             _ptr(out.expert_offset), _ptr(out.rank_count), _ptr(out.rank_offset),
-                             _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token),
-                             _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
-                             _stream(stream, topk_idx.device))
-    _check(st, "moe_get_layout")
+        out = Layout.empty(N, k, E, R, topk_idx.device, align, num_recv_rows)
+    args = (_ptr(out.expert_count), _ptr(out.expert_offset), _ptr(out.rank_count),
+            _ptr(out.rank_offset), _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token),
+            _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
+            _stream(stream, topk_idx.device))
+    if align == 1 and out.num_rows == N * k:
+        st = _lib.moe_get_layout(_ptr(topk_idx), N, k, E, R, *args)
+        _check(st, "moe_get_layout")
+    else:
+        st = _lib.moe_get_layout_aligned(_ptr(topk_idx), N, k, E, R, align, out.num_rows, *args)
+        _check(st, "moe_get_layout_aligned")
+    out.align = align
     return out
 
 
@@ -218,7 +241,7 @@ def scale_shape(S: int, H: int, dtype: int):
 
 
 def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_x=None,
-                 recv_scale=None, d_status=None, stream=None):
+                 recv_scale=None, num_recv_rows: int | None = None, d_status=None, stream=None):
     """Scatter rows of ``x`` (bf16 [N,H]) to their receive rows.  Returns
     ``(recv_x, recv_scale)``: bf16 [N*k,H] and None, or uint8 e4m3 codes
     [N*k,H] with fp32 [N*k,H/128] (per block), fp32 [N*k,1] (per token) or
@@ -227,7 +250,7 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
     N, H = x.shape
     _need(token_slot, "token_slot", torch.int32)
     k = token_slot.shape[1]
-    S = N * k
+    S = num_recv_rows if num_recv_rows is not None else (recv_x.shape[0] if recv_x is not None else N * k)
     if dtype == MOE_DTYPE_BF16:
         if recv_x is None:
             recv_x = torch.empty((S, H), dtype=torch.bfloat16, device=x.device)
@@ -243,7 +266,7 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
             recv_scale = torch.empty(shape, dtype=sdt, device=x.device)
         _need(recv_x, "recv_x", torch.uint8, (S, H))
         _need(recv_scale, "recv_scale", sdt, shape)
-    st = _lib.moe_dispatch(_ptr(x), N, H, k, _ptr(token_slot), dtype, _ptr(recv_x),
+    st = _lib.moe_dispatch(_ptr(x), N, H, k, _ptr(token_slot), S, dtype, _ptr(recv_x),
                            _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
     _check(st, "moe_dispatch")
     return recv_x, recv_scale
@@ -260,7 +283,7 @@ def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor,
     if out is None:
         out = torch.empty((N, H), dtype=torch.bfloat16, device=y.device)
     _need(out, "out", torch.bfloat16, (N, H))
-    st = _lib.moe_combine(_ptr(y), N, H, k, _ptr(token_slot), _ptr(topk_w), _ptr(out),
+    st = _lib.moe_combine(_ptr(y), N, H, k, _ptr(token_slot), y.shape[0], _ptr(topk_w), _ptr(out),
                           _ptr(d_status), _stream(stream, y.device))
     _check(st, "moe_combine")
     return out
@@ -277,8 +300,8 @@ def moe_dispatch_backward(grad_recv: torch.Tensor, token_slot: torch.Tensor, *, 
     if grad_x is None:
         grad_x = torch.empty((N, H), dtype=torch.bfloat16, device=grad_recv.device)
     _need(grad_x, "grad_x", torch.bfloat16, (N, H))
-    st = _lib.moe_dispatch_backward(_ptr(grad_recv), N, H, k, _ptr(token_slot), _ptr(grad_x),
-                                    _ptr(d_status), _stream(stream, grad_recv.device))
+    st = _lib.moe_dispatch_backward(_ptr(grad_recv), N, H, k, _ptr(token_slot), grad_recv.shape[0],
+                                    _ptr(grad_x), _ptr(d_status), _stream(stream, grad_recv.device))
     _check(st, "moe_dispatch_backward")
     return grad_x
 
@@ -294,12 +317,12 @@ def moe_combine_backward(grad_out: torch.Tensor, y: torch.Tensor, token_slot: to
     H = grad_out.shape[1]
     _need(topk_w, "topk_w", torch.float32, (N, k))
     if grad_y is None:
-        grad_y = torch.empty((N * k, H), dtype=torch.bfloat16, device=y.device)
+        grad_y = torch.empty(tuple(y.shape), dtype=torch.bfloat16, device=y.device)
     if grad_w is None:
         grad_w = torch.empty((N, k), dtype=torch.float32, device=y.device)
-    _need(grad_y, "grad_y", torch.bfloat16, (N * k, H))
+    _need(grad_y, "grad_y", torch.bfloat16, tuple(y.shape))
     _need(grad_w, "grad_w", torch.float32, (N, k))
-    st = _lib.moe_combine_backward(_ptr(grad_out), _ptr(y), N, H, k, _ptr(token_slot),
+    st = _lib.moe_combine_backward(_ptr(grad_out), _ptr(y), N, H, k, _ptr(token_slot), y.shape[0],
                                    _ptr(topk_w), _ptr(grad_y), _ptr(grad_w), _ptr(d_status),
                                    _stream(stream, y.device))
     _check(st, "moe_combine_backward")

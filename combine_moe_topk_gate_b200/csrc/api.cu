@@ -22,7 +22,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 1; }
+int moe_abi_version(void) { return 2; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -64,28 +64,55 @@ size_t moe_layout_workspace_bytes(int num_tokens, int k, int num_experts, int nu
   return moe::layout_workspace_bytes(num_tokens, k, num_experts, num_ranks);
 }
 
-moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k, int num_experts,
-                            int num_ranks, int32_t* expert_count, int32_t* expert_offset,
-                            int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
-                            int32_t* token_slot, int32_t* slot_token, void* workspace,
-                            size_t workspace_bytes, int32_t* d_status, moe_stream_t stream) {
+size_t moe_aligned_recv_rows(int num_tokens, int k, int num_experts, int align) {
+  if (num_tokens < 0 || k < 1 || num_experts < 1 || align < 1) return 0;
+  return static_cast<size_t>(num_tokens) * k + static_cast<size_t>(num_experts) * (align - 1);
+}
+
+moe_status_t moe_get_layout_aligned(const int32_t* topk_idx, int num_tokens, int k,
+                                    int num_experts, int num_ranks, int align,
+                                    int num_recv_rows, int32_t* expert_count,
+                                    int32_t* expert_offset, int32_t* rank_count,
+                                    int32_t* rank_offset, int32_t* rank_tokens,
+                                    int32_t* token_slot, int32_t* slot_token, void* workspace,
+                                    size_t workspace_bytes, int32_t* d_status,
+                                    moe_stream_t stream) {
   const int N = num_tokens, E = num_experts, R = num_ranks;
   if (N < 0 || k < 1 || E < 1 || R < 1 || E % R != 0) return MOE_ERR_INVALID_ARG;
+  if (align < 1 || align > MOE_MAX_ALIGN) return MOE_ERR_INVALID_ARG;
   if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
-  if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  const long long need = static_cast<long long>(N) * k + static_cast<long long>(E) * (align - 1);
+  if (need > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  if (num_recv_rows < need) return MOE_ERR_INVALID_ARG;
   if (!expert_count || !expert_offset || !rank_count || !rank_offset || !rank_tokens ||
       !workspace)
     return MOE_ERR_INVALID_ARG;
-  if (N > 0 && (!topk_idx || !token_slot || !slot_token)) return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!topk_idx || !token_slot)) return MOE_ERR_INVALID_ARG;
+  if (num_recv_rows > 0 && !slot_token) return MOE_ERR_INVALID_ARG;
   if (workspace_bytes < moe::layout_workspace_bytes(N, k, E, R)) return MOE_ERR_INVALID_ARG;
   const void* ptrs[] = {topk_idx, expert_count, expert_offset, rank_count, rank_offset,
                         rank_tokens, token_slot, slot_token, d_status};
   for (const void* p : ptrs)
     if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_layout(topk_idx, N, k, E, R, expert_count, expert_offset,
-                                      rank_count, rank_offset, rank_tokens, token_slot,
-                                      slot_token, workspace, d_status, as_stream(stream)));
+  return from_cuda(moe::launch_layout(topk_idx, N, k, E, R, align, num_recv_rows, expert_count,
+                                      expert_offset, rank_count, rank_offset, rank_tokens,
+                                      token_slot, slot_token, workspace, d_status,
+                                      as_stream(stream)));
+}
+
+moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k, int num_experts,
+                            int num_ranks, int32_t* expert_count, int32_t* expert_offset,
+                            int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
+                            int32_t* token_slot, int32_t* slot_token, void* workspace,
+                            size_t workspace_bytes, int32_t* d_status, moe_stream_t stream) {
+  if (num_tokens < 0 || k < 1) return MOE_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(num_tokens) * k;
+  if (rows > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  return moe_get_layout_aligned(topk_idx, num_tokens, k, num_experts, num_ranks, 1,
+                                static_cast<int>(rows), expert_count, expert_offset, rank_count,
+                                rank_offset, rank_tokens, token_slot, slot_token, workspace,
+                                workspace_bytes, d_status, stream);
 }
 
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
@@ -106,10 +133,11 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
 }
 
 moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
-                          const int32_t* token_slot, moe_dtype_t dtype, void* recv_x,
-                          void* recv_scale, int32_t* d_status, moe_stream_t stream) {
+                          const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
+                          void* recv_x, void* recv_scale, int32_t* d_status,
+                          moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
-  if (N < 0 || H < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (N < 0 || H < 1 || k < 1 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
   if (dtype == MOE_DTYPE_BF16) {
@@ -131,15 +159,15 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
     return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(token_slot, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_dispatch(x, N, H, k, token_slot, dtype, recv_x, recv_scale,
-                                        d_status, as_stream(stream)));
+  return from_cuda(moe::launch_dispatch(x, N, H, k, token_slot, num_recv_rows, dtype, recv_x,
+                                        recv_scale, d_status, as_stream(stream)));
 }
 
 moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
-                         const int32_t* token_slot, const float* topk_w, void* out,
-                         int32_t* d_status, moe_stream_t stream) {
+                         const int32_t* token_slot, int num_recv_rows, const float* topk_w,
+                         void* out, int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
-  if (N < 0 || H < 1 || k < 1 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (N < 0 || H < 1 || k < 1 || H % 8 != 0 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
   if (N == 0) return MOE_OK;
@@ -147,15 +175,15 @@ moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
   if (!aligned(y, 16) || !aligned(out, 16) || !aligned(token_slot, 4) || !aligned(topk_w, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_combine(y, N, H, k, token_slot, topk_w, out, d_status,
-                                       as_stream(stream)));
+  return from_cuda(moe::launch_combine(y, N, H, k, token_slot, num_recv_rows, topk_w, out,
+                                       d_status, as_stream(stream)));
 }
 
 moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hidden, int k,
-                                   const int32_t* token_slot, void* grad_x, int32_t* d_status,
-                                   moe_stream_t stream) {
+                                   const int32_t* token_slot, int num_recv_rows, void* grad_x,
+                                   int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
-  if (N < 0 || H < 1 || k < 1 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (N < 0 || H < 1 || k < 1 || H % 8 != 0 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
   if (N == 0) return MOE_OK;
@@ -164,16 +192,16 @@ moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hi
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
   // the combine kernel with unit weights
-  return from_cuda(moe::launch_combine(grad_recv, N, H, k, token_slot, nullptr, grad_x, d_status,
-                                       as_stream(stream)));
+  return from_cuda(moe::launch_combine(grad_recv, N, H, k, token_slot, num_recv_rows, nullptr,
+                                       grad_x, d_status, as_stream(stream)));
 }
 
 moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_tokens, int hidden,
-                                  int k, const int32_t* token_slot, const float* topk_w,
-                                  void* grad_y, float* grad_w, int32_t* d_status,
-                                  moe_stream_t stream) {
+                                  int k, const int32_t* token_slot, int num_recv_rows,
+                                  const float* topk_w, void* grad_y, float* grad_w,
+                                  int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
-  if (N < 0 || H < 1 || k < 1 || H % 8 != 0) return MOE_ERR_INVALID_ARG;
+  if (N < 0 || H < 1 || k < 1 || H % 8 != 0 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
   if (N == 0) return MOE_OK;
@@ -182,8 +210,9 @@ moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_t
       !aligned(token_slot, 4) || !aligned(topk_w, 4) || !aligned(grad_w, 4) ||
       !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_combine_backward(grad_out, y, N, H, k, token_slot, topk_w, grad_y,
-                                                grad_w, d_status, as_stream(stream)));
+  return from_cuda(moe::launch_combine_backward(grad_out, y, N, H, k, token_slot, num_recv_rows,
+                                                topk_w, grad_y, grad_w, d_status,
+                                                as_stream(stream)));
 }
 
 moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream) {

@@ -63,7 +63,7 @@ __device__ __forceinline__ void consumer_barrier() {
 __global__ void __launch_bounds__(kThreads)
     combine_backward_bulk_kernel(const uint16_t* __restrict__ grad_out,
                                  const uint16_t* __restrict__ y, int N, int H, int k,
-                                 const int32_t* __restrict__ token_slot,
+                                 const int32_t* __restrict__ token_slot, long long S,
                                  const float* __restrict__ topk_w, uint16_t* __restrict__ grad_y,
                                  float* __restrict__ grad_w, int32_t* d_status) {
   extern __shared__ __align__(128) unsigned char smem[];
@@ -95,8 +95,7 @@ __global__ void __launch_bounds__(kThreads)
   const int g1 = g0 + gper < groups ? g0 + gper : groups;
   const long long i0 = static_cast<long long>(g0) * segs;
   const long long i1 = g1 > g0 ? static_cast<long long>(g1) * segs : i0;
-  const long long S = static_cast<long long>(N) * k;
-  const long long NK = S;
+  const long long NK = static_cast<long long>(N) * k;  // entries of token_slot / topk_w
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -252,8 +251,9 @@ __global__ void __launch_bounds__(kThreads)
 }  // namespace
 
 cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, int H, int k,
-                                    const int32_t* token_slot, const float* topk_w, void* grad_y,
-                                    float* grad_w, int32_t* d_status, cudaStream_t stream) {
+                                    const int32_t* token_slot, long long num_rows,
+                                    const float* topk_w, void* grad_y, float* grad_w,
+                                    int32_t* d_status, cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   const Layout L = smem_layout(k);
   cudaError_t err = cudaFuncSetAttribute(combine_backward_bulk_kernel,
@@ -272,7 +272,8 @@ cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, 
   const long long grid = std::min<long long>(groups, static_cast<long long>(sms) * per_sm);
   return launch_pdl(combine_backward_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total,
                     stream, static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y),
-                    N, H, k, token_slot, topk_w, static_cast<uint16_t*>(grad_y), grad_w, d_status);
+                    N, H, k, token_slot, num_rows, topk_w, static_cast<uint16_t*>(grad_y), grad_w,
+                    d_status);
 }
 
 }  // namespace moe

@@ -68,8 +68,9 @@ __host__ __device__ inline Layout smem_layout(int k) {
 
 __global__ void __launch_bounds__(kThreads, 3)
     combine_bulk_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
-                        const int32_t* __restrict__ token_slot, const float* __restrict__ topk_w,
-                        uint16_t* __restrict__ out, int32_t* d_status) {
+                        const int32_t* __restrict__ token_slot, long long S,
+                        const float* __restrict__ topk_w, uint16_t* __restrict__ out,
+                        int32_t* d_status) {
   extern __shared__ __align__(128) unsigned char smem[];
   const Layout L = smem_layout(k);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -98,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 3)
   const long long per = (items + gridDim.x - 1) / gridDim.x;
   const long long i0 = static_cast<long long>(blockIdx.x) * per;
   const long long i1 = i0 + per < items ? i0 + per : items;
-  const long long S = static_cast<long long>(N) * k;
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 }  // namespace
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
-                           const float* topk_w, void* out, int32_t* d_status,
+                           long long num_rows, const float* topk_w, void* out, int32_t* d_status,
                            cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   const Layout L = smem_layout(k);
@@ -252,7 +252,7 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
       static_cast<long long>((N + L.T - 1) / L.T) * ((H + L.seg - 1) / L.seg);
   const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
   return launch_pdl(combine_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total, stream,
-                    static_cast<const uint16_t*>(y), N, H, k, token_slot, topk_w,
+                    static_cast<const uint16_t*>(y), N, H, k, token_slot, num_rows, topk_w,
                     static_cast<uint16_t*>(out), d_status);
 }
 

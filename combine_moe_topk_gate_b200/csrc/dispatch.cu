@@ -24,8 +24,9 @@ constexpr int kWarps = 8;
 // a warp covers 512 channels.
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_fp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
-                        const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
-                        float* __restrict__ recv_scale, int32_t* d_status) {
+                        const int32_t* __restrict__ token_slot, long long S,
+                        uint8_t* __restrict__ recv_x, float* __restrict__ recv_scale,
+                        int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -34,7 +35,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
   const int c0 = s * 512 + lane * 16;
   const bool active = c0 < H;  // H % 128 == 0: whole 8-lane blocks are in or out
-  const long long S = static_cast<long long>(N) * k;
   const int nblk = H / 128;
   pdl_wait();
   pdl_trigger();
@@ -100,8 +100,9 @@ __device__ __forceinline__ int floor_log2_pos(float a) {  // a > 0, finite; exac
 
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_mxfp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
-                          const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
-                          uint8_t* __restrict__ recv_e8m0, int32_t* d_status) {
+                          const int32_t* __restrict__ token_slot, long long S,
+                          uint8_t* __restrict__ recv_x, uint8_t* __restrict__ recv_e8m0,
+                          int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -110,7 +111,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
   const int c0 = s * 512 + lane * 16;
   const bool active = c0 < H;  // H % 32 == 0: whole 2-lane blocks are in or out
-  const long long S = static_cast<long long>(N) * k;
   const int nblk = H / 32;
   pdl_wait();
   pdl_trigger();
@@ -183,14 +183,14 @@ constexpr int kTokenThreads = 256;
 template <int VPT>
 __global__ void __launch_bounds__(kTokenThreads)
     dispatch_fp8_token_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
-                              const int32_t* __restrict__ token_slot, uint8_t* __restrict__ recv_x,
-                              float* __restrict__ recv_scale, int32_t* d_status) {
+                              const int32_t* __restrict__ token_slot, long long S,
+                              uint8_t* __restrict__ recv_x, float* __restrict__ recv_scale,
+                              int32_t* d_status) {
   __shared__ float warp_max[kTokenThreads / 32];
   __shared__ int slots[MOE_MAX_TOPK];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
   const int nvec = H / 8;
-  const long long S = static_cast<long long>(N) * k;
   pdl_wait();
   pdl_trigger();
   if (tid < k) {
@@ -249,8 +249,8 @@ __global__ void __launch_bounds__(kTokenThreads)
 // BF16: lane owns 8 channels (one 16-byte vector), a warp covers 256 channels.
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_bf16_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
-                         const int32_t* __restrict__ token_slot, uint16_t* __restrict__ recv_x,
-                         int32_t* d_status) {
+                         const int32_t* __restrict__ token_slot, long long S,
+                         uint16_t* __restrict__ recv_x, int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 255) / 256;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -259,7 +259,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
   const int c0 = s * 256 + lane * 8;
   const bool active = c0 < H;  // H % 8 == 0
-  const long long S = static_cast<long long>(N) * k;
   pdl_wait();
   pdl_trigger();
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
@@ -292,8 +291,8 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
 }  // namespace
 
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            int dtype, void* recv_x, void* recv_scale, int32_t* d_status,
-                            cudaStream_t stream) {
+                            long long num_rows, int dtype, void* recv_x, void* recv_scale,
+                            int32_t* d_status, cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* r8 = static_cast<uint8_t*>(recv_x);
@@ -302,28 +301,28 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
     if (dtype == MOE_DTYPE_FP8_E4M3)
       return launch_pdl(dispatch_fp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
-                        token_slot, r8, static_cast<float*>(recv_scale), d_status);
+                        token_slot, num_rows, r8, static_cast<float*>(recv_scale), d_status);
     return launch_pdl(dispatch_mxfp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
-                      token_slot, r8, static_cast<uint8_t*>(recv_scale), d_status);
+                      token_slot, num_rows, r8, static_cast<uint8_t*>(recv_scale), d_status);
   } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
     const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
     float* sc = static_cast<float*>(recv_scale);
     if (vpt <= 1)
       return launch_pdl(dispatch_fp8_token_kernel<1>, N, kTokenThreads, 0, stream, xs, N, H, k,
-                        token_slot, r8, sc, d_status);
+                        token_slot, num_rows, r8, sc, d_status);
     if (vpt <= 2)
       return launch_pdl(dispatch_fp8_token_kernel<2>, N, kTokenThreads, 0, stream, xs, N, H, k,
-                        token_slot, r8, sc, d_status);
+                        token_slot, num_rows, r8, sc, d_status);
     if (vpt <= 4)
       return launch_pdl(dispatch_fp8_token_kernel<4>, N, kTokenThreads, 0, stream, xs, N, H, k,
-                        token_slot, r8, sc, d_status);
+                        token_slot, num_rows, r8, sc, d_status);
     return launch_pdl(dispatch_fp8_token_kernel<8>, N, kTokenThreads, 0, stream, xs, N, H, k,
-                      token_slot, r8, sc, d_status);
+                      token_slot, num_rows, r8, sc, d_status);
   } else {
     const long long items = static_cast<long long>(N) * ((H + 255) / 256);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
     return launch_pdl(dispatch_bf16_kernel, blocks, kWarps * 32, 0, stream,
-                      static_cast<const uint16_t*>(x), N, H, k, token_slot,
+                      static_cast<const uint16_t*>(x), N, H, k, token_slot, num_rows,
                       static_cast<uint16_t*>(recv_x), d_status);
   }
 }

@@ -128,6 +128,32 @@ __device__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_sums) {
   __syncthreads();
 }
 
+// Turns the per-bucket totals in off[] into exclusive row offsets, each
+// expert bucket rounded up to a multiple of `align` (1 = packed); cnt[] keeps
+// the totals.
+__device__ void aligned_offsets(int32_t* off, int32_t* cnt, int nb, int align,
+                                int32_t* warp_sums) {
+  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
+    const int v = off[i];
+    cnt[i] = v;
+    if (i < nb - 1) off[i] = (v + align - 1) / align * align;
+  }
+  __syncthreads();
+  block_exclusive_scan(off, nb, warp_sums);
+}
+
+// Rows no entry lands in get slot_token = -1: the padding after each expert
+// and every row after the masked tail.  CTA `cta` of `ncta` takes its share.
+__device__ void fill_unused_rows(const int32_t* off, const int32_t* cnt, int E, long long num_rows,
+                                 int32_t* slot_token, int cta, int ncta) {
+  for (int e = cta; e < E; e += ncta)
+    for (int i = off[e] + cnt[e] + threadIdx.x; i < off[e + 1]; i += blockDim.x) slot_token[i] = -1;
+  const long long tail0 = static_cast<long long>(off[E]) + cnt[E];
+  for (long long i = tail0 + static_cast<long long>(cta) * blockDim.x + threadIdx.x; i < num_rows;
+       i += static_cast<long long>(ncta) * blockDim.x)
+    slot_token[i] = -1;
+}
+
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_assign_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R, int C,
                          const int32_t* __restrict__ chunk_counts,
@@ -135,14 +161,15 @@ __global__ void __launch_bounds__(kLayoutThreads)
                          int32_t* __restrict__ expert_offset, int32_t* __restrict__ rank_count,
                          int32_t* __restrict__ rank_offset, int32_t* __restrict__ rank_tokens,
                          int32_t* __restrict__ token_slot, int32_t* __restrict__ slot_token,
-                         int32_t* d_status) {
+                         int align, long long num_rows, int32_t* d_status) {
   extern __shared__ int32_t sm[];
   const int nb = E + 1;
-  int32_t* off = sm;                 // nb: totals, then their exclusive scan
+  int32_t* off = sm;                 // nb: totals, then their exclusive (aligned) scan
   int32_t* base = off + nb;          // nb: first row of this chunk per bucket
   int32_t* wcnt = base + nb;         // kLayoutWarps * nb
   int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
   int32_t* rtok = warp_sums + 32;                 // R (CTA 0: tokens per rank)
+  int32_t* cnt = rtok + R;                        // nb: totals
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x;
   const int nbits = 32 - __clz(E + 1);
@@ -195,11 +222,12 @@ __global__ void __launch_bounds__(kLayoutThreads)
     }
   }
   __syncthreads();
+  // 2. bucket offsets (experts aligned), unused rows marked
+  aligned_offsets(off, cnt, nb, align, warp_sums);
   if (c == 0)
-    for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = off[i];
-  // 2. bucket offsets
-  block_exclusive_scan(off, nb, warp_sums);
+    for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
   for (int i = tid; i < nb; i += kLayoutThreads) base[i] += off[i];
+  fill_unused_rows(off, cnt, E, num_rows, slot_token, c, C);
   if (c == 0) {
     const int epr = E / R;
     for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
@@ -231,9 +259,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (tid < ne) {
     const int slot = base[b] + wcnt[warp * nb + b] + in_warp;
     const long long flat = t0 * k + tid;
-    // counts and ranks come from the same entries, so slot < N*k; the check
-    // only guards against topk_idx changing between the two launches
-    if (slot < 0 || static_cast<long long>(slot) >= static_cast<long long>(N) * k) {
+    // counts and ranks come from the same entries, so slot < num_rows; the
+    // check only guards against topk_idx changing between the two launches
+    if (slot < 0 || static_cast<long long>(slot) >= num_rows) {
       token_slot[flat] = -1;
       report_bad_index(d_status);
     } else if (b < E) {
@@ -255,7 +283,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
                          int32_t* __restrict__ expert_count, int32_t* __restrict__ expert_offset,
                          int32_t* __restrict__ rank_count, int32_t* __restrict__ rank_offset,
                          int32_t* __restrict__ rank_tokens, int32_t* __restrict__ token_slot,
-                         int32_t* __restrict__ slot_token, int32_t* d_status) {
+                         int32_t* __restrict__ slot_token, int align, long long num_rows,
+                         int32_t* d_status) {
   extern __shared__ int32_t sm[];
   const int nb = E + 1;
   int32_t* off = sm;                              // nb: totals, then their exclusive scan
@@ -263,6 +292,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
   int32_t* rtok = warp_sums + 32;                 // R
   int32_t* sidx = rtok + R;                       // kLayoutThreads
+  int32_t* cnt = sidx + kLayoutThreads;           // nb: totals
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ne = N * k;  // <= kLayoutThreads
   const int nbits = 32 - __clz(E + 1);
@@ -309,8 +339,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
     if (lane == 31) off[bb] = incl;
   }
   __syncthreads();
-  for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = off[i];
-  block_exclusive_scan(off, nb, warp_sums);
+  aligned_offsets(off, cnt, nb, align, warp_sums);
+  for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
+  fill_unused_rows(off, cnt, E, num_rows, slot_token, 0, 1);
   for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
   for (int r = tid; r < R; r += kLayoutThreads) {
     rank_offset[r] = off[r * epr];
@@ -339,16 +370,16 @@ size_t layout_workspace_bytes(int N, int k, int E, int R) {
   return bytes < 256 ? 256 : bytes;
 }
 
-cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
-                          int32_t* expert_count, int32_t* expert_offset, int32_t* rank_count,
-                          int32_t* rank_offset, int32_t* rank_tokens, int32_t* token_slot,
-                          int32_t* slot_token, void* workspace, int32_t* d_status,
-                          cudaStream_t stream) {
+cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, int align,
+                          long long num_rows, int32_t* expert_count, int32_t* expert_offset,
+                          int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
+                          int32_t* token_slot, int32_t* slot_token, void* workspace,
+                          int32_t* d_status, cudaStream_t stream) {
   const int C = num_chunks(N, k);
   cudaError_t err;
   if (static_cast<long long>(N) * k <= kLayoutThreads) {
-    const size_t smem = (static_cast<size_t>(E) + 1 + static_cast<size_t>(kLayoutWarps) * (E + 1) +
-                         32 + R + kLayoutThreads) *
+    const size_t smem = (2 * (static_cast<size_t>(E) + 1) +
+                         static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R + kLayoutThreads) *
                         sizeof(int32_t);
     if (smem > 48 * 1024) {
       err = cudaFuncSetAttribute(layout_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -357,13 +388,13 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
     }
     return launch_pdl(layout_single_kernel, 1, kLayoutThreads, smem, stream, topk_idx, N, k, E, R,
                       expert_count, expert_offset, rank_count, rank_offset, rank_tokens, token_slot,
-                      slot_token, d_status);
+                      slot_token, align, num_rows, d_status);
   }
   int32_t* chunk_counts = static_cast<int32_t*>(workspace);
   int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
   const size_t smem_count = (static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
   const size_t smem_assign =
-      (2 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
+      (3 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
       sizeof(int32_t);
   if (smem_count > 48 * 1024) {
     err = cudaFuncSetAttribute(layout_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -380,7 +411,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
   if (err != cudaSuccess) return err;
   return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
                     R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
-                    rank_offset, rank_tokens, token_slot, slot_token, d_status);
+                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
 }
 
 }  // namespace moe

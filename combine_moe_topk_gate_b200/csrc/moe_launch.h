@@ -14,23 +14,26 @@ cudaError_t launch_topk_gate(const float* logits, int N, int E, int k, int kind,
 
 size_t layout_workspace_bytes(int N, int k, int E, int R);
 
-cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R,
-                          int32_t* expert_count, int32_t* expert_offset, int32_t* rank_count,
-                          int32_t* rank_offset, int32_t* rank_tokens, int32_t* token_slot,
-                          int32_t* slot_token, void* workspace, int32_t* d_status,
-                          cudaStream_t stream);
+cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, int align,
+                          long long num_rows, int32_t* expert_count, int32_t* expert_offset,
+                          int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
+                          int32_t* token_slot, int32_t* slot_token, void* workspace,
+                          int32_t* d_status, cudaStream_t stream);
 
+// num_rows: rows of the receive buffer (N*k packed, more for aligned layouts);
+// slots outside [-1, num_rows) are skipped and reported.
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            int dtype, void* recv_x, void* recv_scale, int32_t* d_status,
-                            cudaStream_t stream);
+                            long long num_rows, int dtype, void* recv_x, void* recv_scale,
+                            int32_t* d_status, cudaStream_t stream);
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
-                           const float* topk_w, void* out, int32_t* d_status,
+                           long long num_rows, const float* topk_w, void* out, int32_t* d_status,
                            cudaStream_t stream);
 
 cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, int H, int k,
-                                    const int32_t* token_slot, const float* topk_w, void* grad_y,
-                                    float* grad_w, int32_t* d_status, cudaStream_t stream);
+                                    const int32_t* token_slot, long long num_rows,
+                                    const float* topk_w, void* grad_y, float* grad_w,
+                                    int32_t* d_status, cudaStream_t stream);
 
 cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream);
 

@@ -80,6 +80,7 @@ typedef void* moe_stream_t;      /* a cudaStream_t */
 #define MOE_MAX_EXPERTS 1024
 #define MOE_MAX_TOPK 32
 #define MOE_FP8_BLOCK 128
+#define MOE_MAX_ALIGN 4096
 
 /*
  * moe_topk_gate -- router top-k selection and weights.
@@ -142,6 +143,8 @@ size_t moe_layout_workspace_bytes(int num_tokens, int k, int num_experts, int nu
  *   workspace     device scratch of moe_layout_workspace_bytes() bytes, 16-byte
  *                 aligned; contents need no initialisation and are not kept.
  *   Limits: 1 <= E <= MOE_MAX_EXPERTS, 1 <= k <= MOE_MAX_TOPK, E % R == 0.
+ *   The receive buffer of this (packed) layout has S = N*k rows; pass S as
+ *   num_recv_rows to the calls below.
  */
 moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k,
                             int num_experts, int num_ranks, int32_t* expert_count,
@@ -149,6 +152,35 @@ moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k,
                             int32_t* rank_offset, int32_t* rank_tokens,
                             int32_t* token_slot, int32_t* slot_token, void* workspace,
                             size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
+
+/* Receive rows an aligned layout may need: N*k + E*(align - 1); 0 when an
+ * argument is out of range (N < 0, k < 1, E < 1, align < 1). */
+size_t moe_aligned_recv_rows(int num_tokens, int k, int num_experts, int align);
+
+/*
+ * moe_get_layout_aligned -- the layout with every expert's rows starting at a
+ * multiple of `align` (1 <= align <= MOE_MAX_ALIGN), so a grouped GEMM can
+ * tile each expert by align rows.  [EPv2] ElasticBuffer interface mentions a
+ * new GEMM layout without defining it; this is the reading taken.
+ *   expert_offset[e] = sum_{e' < e} round_up(expert_count[e'], align);
+ *   rank_offset[r]   = expert_offset[r*E/R], rank_count[r] = the rows of rank
+ *                      r's region (padding included);
+ *   token_slot, slot_token and rank_tokens as in moe_get_layout, except that
+ *   slot_token has num_recv_rows entries and is -1 on every row no token
+ *   lands in (padding, masked tail, spare rows).
+ *   num_recv_rows >= moe_aligned_recv_rows(N, k, E, align), else
+ *   MOE_ERR_INVALID_ARG; align outside [1, MOE_MAX_ALIGN] is
+ *   MOE_ERR_INVALID_ARG, and a padded layout of 2^31 rows or more
+ *   MOE_ERR_UNSUPPORTED.  align = 1 is exactly moe_get_layout.
+ */
+moe_status_t moe_get_layout_aligned(const int32_t* topk_idx, int num_tokens, int k,
+                                    int num_experts, int num_ranks, int align,
+                                    int num_recv_rows, int32_t* expert_count,
+                                    int32_t* expert_offset, int32_t* rank_count,
+                                    int32_t* rank_offset, int32_t* rank_tokens,
+                                    int32_t* token_slot, int32_t* slot_token, void* workspace,
+                                    size_t workspace_bytes, int32_t* d_status,
+                                    moe_stream_t stream);
 
 /*
  * moe_get_layout_noalloc -- moe_get_layout without a caller-provided
@@ -190,7 +222,9 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
  *   BF16 and FP8 dispatch.  [TK]: per-block FP8 quantisation.
  *
  *   x           bf16 [N, H] in.
- *   token_slot  int32 [N, k] from moe_get_layout.
+ *   token_slot  int32 [N, k] from moe_get_layout(_aligned).
+ *   num_recv_rows  rows S of the receive buffer (N*k packed, the aligned
+ *               layout's num_recv_rows otherwise); slots must lie in [-1, S).
  *   BF16:  recv_x bf16 [S, H]: recv_x[token_slot[t,j]] = x[t]; recv_scale unused.
  *          H % 8 == 0; x and recv_x 16-byte aligned.
  *   FP8:   recv_x e4m3 [S, H], recv_scale fp32 [S, H/128].  Per token and
@@ -213,8 +247,9 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
  *   and reported through d_status.
  */
 moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
-                          const int32_t* token_slot, moe_dtype_t dtype, void* recv_x,
-                          void* recv_scale, int32_t* d_status, moe_stream_t stream);
+                          const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
+                          void* recv_x, void* recv_scale, int32_t* d_status,
+                          moe_stream_t stream);
 
 /*
  * moe_combine -- weighted gather-reduce of each token's k expert outputs.
@@ -222,7 +257,8 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
  *   selected experts' outputs weighted by the router weights; [EPv2] usage
  *   patterns: combine reduces expert outputs back to the token.
  *
- *   y          bf16 [S, H] expert outputs, one row per receive slot.
+ *   y          bf16 [S, H] expert outputs, one row per receive slot (S =
+ *              num_recv_rows, see moe_dispatch).
  *   token_slot int32 [N, k], topk_w fp32 [N, k].
  *   out        bf16 [N, H]:  acc = +0.0f; for j = 0..k-1 (slot order):
  *              acc = fmaf(topk_w[t,j], y[token_slot[t,j], c], acc);
@@ -230,8 +266,8 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
  *              nothing.  H % 8 == 0; y and out 16-byte aligned.
  */
 moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
-                         const int32_t* token_slot, const float* topk_w, void* out,
-                         int32_t* d_status, moe_stream_t stream);
+                         const int32_t* token_slot, int num_recv_rows, const float* topk_w,
+                         void* out, int32_t* d_status, moe_stream_t stream);
 
 /*
  * moe_dispatch_backward -- gradient of dispatch: the sum of each token's
@@ -245,8 +281,8 @@ moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,
  * H % 8 == 0; grad_recv and grad_x 16-byte aligned.
  */
 moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hidden, int k,
-                                   const int32_t* token_slot, void* grad_x, int32_t* d_status,
-                                   moe_stream_t stream);
+                                   const int32_t* token_slot, int num_recv_rows, void* grad_x,
+                                   int32_t* d_status, moe_stream_t stream);
 
 /*
  * moe_combine_backward -- gradients of combine with respect to the expert
@@ -261,9 +297,9 @@ moe_status_t moe_dispatch_backward(const void* grad_recv, int num_tokens, int hi
  * H % 8 == 0; grad_out, y, grad_y 16-byte aligned.
  */
 moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_tokens, int hidden,
-                                  int k, const int32_t* token_slot, const float* topk_w,
-                                  void* grad_y, float* grad_w, int32_t* d_status,
-                                  moe_stream_t stream);
+                                  int k, const int32_t* token_slot, int num_recv_rows,
+                                  const float* topk_w, void* grad_y, float* grad_w,
+                                  int32_t* d_status, moe_stream_t stream);
 
 /*
  * moe_e4m3_encode -- the element encoder moe_dispatch uses, exposed on its

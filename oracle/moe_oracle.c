@@ -464,7 +464,7 @@ int oracle_get_layout_aligned(const int32_t* topk_idx, int N, int k, int E, int 
  *           is what the product gives whenever inv is finite and defines
  *           the all-zero block (amax = 0, scale = 0).
  * The same codes and scale go to every slot of the token.
- * A slot outside [-1, num_rows) is skipped and reported (num_rows = N*k  
+ * A slot outside [-1, num_rows) is skipped and reported (num_rows = N*k
  * for the packed layout, more for a padded one).                        */
 /* ------------------------------------------------------------------ */
 /* Quantisation variants ([TK] list, "Quantisierung ... pro Token, pro Block"):

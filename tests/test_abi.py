@@ -95,24 +95,58 @@ def test_layout_rejects_bad_arguments(api):
     assert call(N=1 << 29, k=8, wsb=1 << 40) == api.MOE_ERR_UNSUPPORTED   # N*k >= 2^31
 
 
+def test_aligned_layout_rejects_bad_arguments(api):
+    L = api.lib()
+    ws = api.moe_layout_workspace_bytes(100, 4, 16, 4)
+    need = api.moe_aligned_recv_rows(100, 4, 16, 64)
+    assert need == 100 * 4 + 16 * 63
+    assert api.moe_aligned_recv_rows(100, 4, 16, 1) == 400
+    assert api.moe_aligned_recv_rows(100, 4, 16, 0) == 0
+
+    def call(align=64, rows=need, slot_token=_P(), N=100, k=4, E=16, R=4):
+        return L.moe_get_layout_aligned(_P(), N, k, E, R, align, rows, _P(), _P(), _P(), _P(), _P(),
+                                        _P(), slot_token, _P(), ws, None, None)
+    assert call(align=0) == api.MOE_ERR_INVALID_ARG
+    assert call(align=api.MOE_MAX_ALIGN + 1) == api.MOE_ERR_INVALID_ARG
+    assert call(rows=need - 1) == api.MOE_ERR_INVALID_ARG      # buffer cannot hold the padded layout
+    assert call(slot_token=None) == api.MOE_ERR_INVALID_ARG
+    assert call(N=0, rows=16 * 63 - 1) == api.MOE_ERR_INVALID_ARG  # padding alone needs E*(align-1)
+    assert call(N=1 << 26, k=32, E=1024, R=4, align=4096, rows=(1 << 31) - 1) == api.MOE_ERR_UNSUPPORTED
+
+
 def test_dispatch_combine_reject_bad_arguments(api):
     L = api.lib()
     FP8, BF16 = api.MOE_DTYPE_FP8_E4M3, api.MOE_DTYPE_BF16
-    assert L.moe_dispatch(_P(), 10, 200, 2, _P(), FP8, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_dispatch(_P(), 10, 100, 2, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), FP8, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_dispatch(_P(0x1008), 10, 256, 2, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), 5, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    S = 20
+
+    def disp(x, N, H, k, dt, recv, scale, rows=S, ts=_P()):
+        return L.moe_dispatch(x, N, H, k, ts, rows, dt, recv, scale, None, None)
+    assert disp(_P(), 10, 200, 2, FP8, _P(), _P()) == api.MOE_ERR_INVALID_ARG
+    assert disp(_P(), 10, 100, 2, BF16, _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert disp(_P(), 10, 256, 2, FP8, _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert disp(_P(0x1008), 10, 256, 2, BF16, _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert disp(_P(), 10, 256, 2, 5, _P(), None) == api.MOE_ERR_INVALID_ARG
     MX, TOK = api.MOE_DTYPE_MXFP8_E4M3, api.MOE_DTYPE_FP8_E4M3_TOKEN
-    assert L.moe_dispatch(_P(), 10, 272, 2, _P(), MX, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG  # H % 32
-    assert L.moe_dispatch(_P(), 10, 256, 2, _P(), MX, _P(), _P(0x1008), None, None) == api.MOE_ERR_INVALID_ARG  # scales 16-B
-    assert L.moe_dispatch(_P(), 10, 20000, 2, _P(), TOK, _P(), _P(), None, None) == api.MOE_ERR_UNSUPPORTED
-    assert L.moe_dispatch(_P(), 10, 100, 2, _P(), TOK, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG  # H % 8
-    assert L.moe_dispatch(_P(), 10, 256, 40, _P(), BF16, _P(), None, None, None) == api.MOE_ERR_UNSUPPORTED
-    assert L.moe_dispatch(None, 0, 256, 2, None, BF16, None, None, None, None) == api.MOE_OK
-    assert L.moe_combine(_P(), 10, 100, 2, _P(), _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(_P(), 10, 256, 2, _P(), _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(_P(), 10, 256, 2, _P(), _P(), _P(0x1004), None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(None, 0, 256, 2, None, None, None, None, None) == api.MOE_OK
+    assert disp(_P(), 10, 272, 2, MX, _P(), _P()) == api.MOE_ERR_INVALID_ARG  # H % 32
+    assert disp(_P(), 10, 256, 2, MX, _P(), _P(0x1008)) == api.MOE_ERR_INVALID_ARG  # scales 16-B
+    assert disp(_P(), 10, 20000, 2, TOK, _P(), _P()) == api.MOE_ERR_UNSUPPORTED
+    assert disp(_P(), 10, 100, 2, TOK, _P(), _P()) == api.MOE_ERR_INVALID_ARG  # H % 8
+    assert disp(_P(), 10, 256, 40, BF16, _P(), None) == api.MOE_ERR_UNSUPPORTED
+    assert disp(_P(), 10, 256, 2, BF16, _P(), None, rows=-1) == api.MOE_ERR_INVALID_ARG
+    assert disp(None, 0, 256, 2, BF16, None, None, rows=0, ts=None) == api.MOE_OK
+
+    def comb(y, N, H, k, w, out, rows=S, ts=_P()):
+        return L.moe_combine(y, N, H, k, ts, rows, w, out, None, None)
+    assert comb(_P(), 10, 100, 2, _P(), _P()) == api.MOE_ERR_INVALID_ARG
+    assert comb(_P(), 10, 256, 2, _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert comb(_P(), 10, 256, 2, _P(), _P(0x1004)) == api.MOE_ERR_INVALID_ARG
+    assert comb(_P(), 10, 256, 2, _P(), _P(), rows=-5) == api.MOE_ERR_INVALID_ARG
+    assert comb(None, 0, 256, 2, None, None, rows=0, ts=None) == api.MOE_OK
+    assert L.moe_dispatch_backward(_P(), 10, 100, 2, _P(), S, _P(), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_backward(_P(), 10, 256, 2, _P(), -1, _P(), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_combine_backward(_P(), _P(), 10, 100, 2, _P(), S, _P(), _P(), _P(), None, None) \
+        == api.MOE_ERR_INVALID_ARG
+    assert L.moe_combine_backward(_P(), _P(), 10, 256, 2, _P(), -1, _P(), _P(), _P(), None, None) \
+        == api.MOE_ERR_INVALID_ARG
     assert L.moe_e4m3_encode(None, 0, None, None) == api.MOE_OK
     assert L.moe_e4m3_encode(None, 5, _P(), None) == api.MOE_ERR_INVALID_ARG
