@@ -29,6 +29,9 @@ DT_BF16 = 0
 DT_FP8_E4M3 = 1
 DT_FP8_E4M3_TOKEN = 2
 DT_MXFP8_E4M3 = 3
+SL_ROW_MAJOR = 0
+SL_MN_MAJOR = 1
+SL_MMA_TILED = 2
 OK = 0
 ERR_INVALID_ARG = 1
 ERR_BAD_INDEX = 4
@@ -92,6 +95,12 @@ def _declare(L):
     L.oracle_dispatch.restype = _I
     L.oracle_dispatch_rows.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _P, _P]
     L.oracle_dispatch_rows.restype = _I
+    L.oracle_scale_elems.argtypes = [_L64, _I, _I, _I]
+    L.oracle_scale_elems.restype = _L64
+    L.oracle_scale_index.argtypes = [_I, _L64, _I, _I, _L64, _I]
+    L.oracle_scale_index.restype = _L64
+    L.oracle_dispatch_scaled.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _I, _P, _P]
+    L.oracle_dispatch_scaled.restype = _I
     L.oracle_combine.argtypes = [_P, _L64, _I, _I, _I, _P, _P, _P]
     L.oracle_combine.restype = _I
     L.oracle_dispatch_backward.argtypes = [_P, _L64, _I, _I, _I, _P, _P]
@@ -247,6 +256,41 @@ def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
     st = lib().oracle_dispatch_rows(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, dtype, _ptr(recv), sp)
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch: invalid argument")
+    return recv, scale, st
+
+
+def scale_elems(num_rows: int, H: int, dtype: int, layout: int) -> int:
+    """Elements of the receive-scale buffer in ``layout`` (-1: layout not defined
+    for the payload type)."""
+    return int(lib().oracle_scale_elems(num_rows, H, dtype, layout))
+
+
+def scale_index(layout: int, num_rows: int, H: int, dtype: int, s: int, b: int) -> int:
+    """Element index of the scale of receive row ``s``, block ``b``."""
+    return int(lib().oracle_scale_index(layout, num_rows, H, dtype, s, b))
+
+
+def dispatch_scaled(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int, layout: int,
+                    recv_rows: int | None = None):
+    """dispatch with the receive scales in ``layout``: (recv_x, flat scale
+    buffer, status); positions no landed row owns stay 0."""
+    if layout == SL_ROW_MAJOR:
+        recv, scale, st = dispatch(x_bf16, token_slot, dtype, recv_rows)
+        return recv, (scale.reshape(-1) if scale is not None else None), st
+    x_bf16 = _c(x_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    N, H = x_bf16.shape
+    k = token_slot.shape[1]
+    S = N * k if recv_rows is None else recv_rows
+    n = scale_elems(S, H, dtype, layout)
+    if n < 0:
+        raise ValueError("oracle_dispatch_scaled: layout not defined for this payload")
+    recv = np.zeros((S, H), np.uint8)
+    scale = np.zeros(n, np.uint8 if dtype == DT_MXFP8_E4M3 else np.float32)
+    st = lib().oracle_dispatch_scaled(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, dtype, layout,
+                                      _ptr(recv), _ptr(scale))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_dispatch_scaled: invalid argument")
     return recv, scale, st
 
 

@@ -607,6 +607,92 @@ int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
 }
 
 /* ------------------------------------------------------------------ */
+/* Scale layouts for a grouped GEMM.  [EPv2] names "a new GEMM layout"
+ * without defining it and [TK] lists batched transposes; neither fixes
+ * where the receive scales go.  Reading: the same values in one of three
+ * places, for scale (s, b) of receive row s and scale block b, with B
+ * blocks per row (H/128 per-block FP8, 1 per-token FP8, H/32 MXFP8):
+ *   ROW_MAJOR   element s*B + b: what dispatch writes by default.
+ *   MN_MAJOR    element b*ld + s, ld = num_rows rounded up to 16 bytes of
+ *               scales (4 fp32 or 16 E8M0 bytes): each block's scales are
+ *               contiguous over the rows (the transposed, M-major scale
+ *               operand of a grouped GEMM), each column 16-byte aligned.
+ *   MMA_TILED   E8M0 only, B % 4 == 0: the order in which the block-scaled
+ *               tensor-core MMA takes its scale factors.  Rows are padded to
+ *               a multiple of 128; 128-row x 4-block atoms of 512 bytes are
+ *               stored row-major over (s / 128, b / 4); inside an atom,
+ *               row s and block b sit at byte
+ *               (s mod 32)*16 + ((s mod 128) / 32)*4 + (b mod 4).
+ * Positions of rows that no token lands in are not written.            */
+/* ------------------------------------------------------------------ */
+#define SL_ROW_MAJOR 0
+#define SL_MN_MAJOR 1
+#define SL_MMA_TILED 2
+
+static int scale_blocks(int H, int dtype)
+{
+    if (dtype == DT_FP8_E4M3) return H / 128;
+    if (dtype == DT_FP8_E4M3_TOKEN) return 1;
+    if (dtype == DT_MXFP8_E4M3) return H / 32;
+    return 0;
+}
+
+static int scale_elem_bytes(int dtype) { return dtype == DT_MXFP8_E4M3 ? 1 : 4; }
+
+static int64_t round_up64(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+/* elements the scale buffer holds in this layout; -1 where the layout does
+ * not apply to the payload type */
+int64_t oracle_scale_elems(int64_t num_rows, int H, int dtype, int layout)
+{
+    int B = scale_blocks(H, dtype);
+    if (num_rows < 0 || B < 1) return -1;
+    if (layout == SL_ROW_MAJOR) return num_rows * B;
+    if (layout == SL_MN_MAJOR) return (int64_t)B * round_up64(num_rows, 16 / scale_elem_bytes(dtype));
+    if (layout == SL_MMA_TILED && dtype == DT_MXFP8_E4M3 && B % 4 == 0)
+        return round_up64(num_rows, 128) * B;
+    return -1;
+}
+
+/* element index of scale (s, b); the layout must apply (see above) */
+int64_t oracle_scale_index(int layout, int64_t num_rows, int H, int dtype, int64_t s, int b)
+{
+    int B = scale_blocks(H, dtype);
+    if (layout == SL_MN_MAJOR) return (int64_t)b * round_up64(num_rows, 16 / scale_elem_bytes(dtype)) + s;
+    if (layout == SL_MMA_TILED) {
+        int64_t atom = (s / 128) * (B / 4) + b / 4;
+        return atom * 512 + (s % 32) * 16 + ((s % 128) / 32) * 4 + b % 4;
+    }
+    return s * B + b;
+}
+
+/* dispatch with the receive scales in `layout`: the row-major dispatch,
+ * then every landed row's scales moved to their place */
+int oracle_dispatch_scaled(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                           int64_t num_rows, int dtype, int layout, void* recv_x,
+                           void* recv_scale)
+{
+    if (layout == SL_ROW_MAJOR)
+        return oracle_dispatch_rows(x, N, H, k, token_slot, num_rows, dtype, recv_x,
+                                    (float*)recv_scale);
+    if (oracle_scale_elems(num_rows, H, dtype, layout) < 0) return ORC_ERR_INVALID_ARG;
+    int B = scale_blocks(H, dtype), es = scale_elem_bytes(dtype);
+    unsigned char* rows = (unsigned char*)calloc((size_t)(num_rows > 0 ? num_rows : 1) * B, (size_t)es);
+    int st = oracle_dispatch_rows(x, N, H, k, token_slot, num_rows, dtype, recv_x, (float*)rows);
+    if (st != ORC_ERR_INVALID_ARG) {
+        for (int64_t i = 0; i < (int64_t)N * k; ++i) {
+            int64_t s = token_slot[i];
+            if (s < 0 || s >= num_rows) continue;
+            for (int b = 0; b < B; ++b)
+                memcpy((unsigned char*)recv_scale + oracle_scale_index(layout, num_rows, H, dtype, s, b) * es,
+                       rows + (s * B + b) * es, (size_t)es);
+        }
+    }
+    free(rows);
+    return st;
+}
+
+/* ------------------------------------------------------------------ */
 /* Combine.  [pplx] Introduction and Combine: the token's output is the
  * average of its experts' outputs weighted by the router weights; [EPv2]
  * usage patterns: combine reduces the expert outputs back to the token.

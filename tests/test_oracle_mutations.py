@@ -49,6 +49,14 @@ MUTANTS = {
     "fp8_token_scale_transposed": ("fsc[0] = amax / 448.0f;", "fsc[0] = 448.0f / amax;"),
     "aligned_layout_rounds_down": ("int32_t padded = (expert_count[e] + align - 1) / align * align;",
                                    "int32_t padded = expert_count[e] / align * align;"),
+    "dispatch_rows_bound_by_packed_rows": ("    int status = ORC_OK;\n    int64_t S = num_rows;\n    int nb = H / 128;",
+                                           "    int status = ORC_OK;\n    int64_t S = (int64_t)N * k;\n    int nb = H / 128;"),
+    "mn_major_unpadded_stride": ("if (layout == SL_MN_MAJOR) return (int64_t)b * round_up64(num_rows, 16 / scale_elem_bytes(dtype)) + s;",
+                                 "if (layout == SL_MN_MAJOR) return (int64_t)b * num_rows + s;"),
+    "mma_tile_row_quarters_swapped": ("return atom * 512 + (s % 32) * 16 + ((s % 128) / 32) * 4 + b % 4;",
+                                      "return atom * 512 + ((s % 128) / 32) * 16 + (s % 32) * 4 + b % 4;"),
+    "mma_tile_atoms_column_major": ("int64_t atom = (s / 128) * (B / 4) + b / 4;",
+                                    "int64_t atom = (b / 4) * ((num_rows + 127) / 128) + s / 128;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

@@ -708,3 +708,70 @@ def test_ops_on_padded_buffer_are_relocations_of_packed(dtype):
     assert s1 == 0 and s2 == 0
     assert np.array_equal(gya[sa], gyp[sp]) and (gya[unused] == 0).all()
     assert np.array_equal(gwa, gwp) and np.array_equal(ma, mp)
+
+
+# ----------------------------------------------------------------- scale layouts
+def test_scale_layout_worked_offsets():
+    g = _gold("scale_layout_offsets.json")
+    for c in g["cases"]:
+        assert O.scale_elems(c["num_rows"], c["H"], c["dtype"], c["layout"]) == c["elems"], c
+        for s, b, off in c["points"]:
+            assert O.scale_index(c["layout"], c["num_rows"], c["H"], c["dtype"], s, b) == off, (c, s, b)
+    for layout, dtype, H, rows in g["undefined"]:
+        assert O.scale_elems(rows, H, dtype, layout) == -1
+
+
+def _scaled_case(dtype, seed=0, N=70, k=3, E=6, align=32):
+    rng = np.random.default_rng(seed)
+    H = 512
+    idx = rng.integers(0, E, (N, k)).astype(np.int32)
+    idx[rng.random((N, k)) < 0.1] = -1
+    rows = N * k + E * (align - 1)
+    A = O.get_layout_aligned(idx, E, 2, align, rows)
+    x = rng.normal(size=(N, H)) * np.exp2(rng.integers(-6, 6, (N, H // 32))).repeat(32, 1)
+    x_bits = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    return x_bits, A, rows
+
+
+@pytest.mark.parametrize("dtype", [O.DT_FP8_E4M3, O.DT_FP8_E4M3_TOKEN, O.DT_MXFP8_E4M3])
+def test_scale_layout_mn_major_is_padded_transpose(dtype):
+    x_bits, A, rows = _scaled_case(dtype)
+    r_recv, r_sc, _ = O.dispatch(x_bits, A.token_slot, dtype, recv_rows=rows)
+    m_recv, m_sc, st = O.dispatch_scaled(x_bits, A.token_slot, dtype, O.SL_MN_MAJOR, recv_rows=rows)
+    assert st == 0 and np.array_equal(m_recv, r_recv)
+    B = r_sc.shape[1]
+    ld = -(-rows // (16 // r_sc.itemsize)) * (16 // r_sc.itemsize)
+    assert m_sc.size == B * ld and (ld * r_sc.itemsize) % 16 == 0
+    assert np.array_equal(m_sc.reshape(B, ld)[:, :rows].T, r_sc)      # zeros where nothing lands
+    assert (m_sc.reshape(B, ld)[:, rows:] == 0).all()
+
+
+def test_scale_layout_mma_tiled_is_blocked_reshape():
+    """The tiled E8M0 layout, restated as array reshapes: rows s = 128 i + 32 j + r
+    and blocks b = 4 m + n go to index (i, m, r, j, n)."""
+    x_bits, A, rows = _scaled_case(O.DT_MXFP8_E4M3, seed=4)
+    _, r_sc, _ = O.dispatch(x_bits, A.token_slot, O.DT_MXFP8_E4M3, recv_rows=rows)
+    t_recv, t_sc, st = O.dispatch_scaled(x_bits, A.token_slot, O.DT_MXFP8_E4M3, O.SL_MMA_TILED,
+                                         recv_rows=rows)
+    assert st == 0
+    B = r_sc.shape[1]
+    Sp = -(-rows // 128) * 128
+    padded = np.zeros((Sp, B), np.uint8)
+    padded[:rows] = r_sc
+    want = padded.reshape(Sp // 128, 4, 32, B // 4, 4).transpose(0, 3, 2, 1, 4).reshape(-1)
+    assert np.array_equal(t_sc, want)
+    # with align = 128 every expert's scales are one contiguous run of whole atoms
+    x2, A2, rows2 = _scaled_case(O.DT_MXFP8_E4M3, seed=5, align=128)
+    _, t2, _ = O.dispatch_scaled(x2, A2.token_slot, O.DT_MXFP8_E4M3, O.SL_MMA_TILED, recv_rows=rows2)
+    _, r2, _ = O.dispatch(x2, A2.token_slot, O.DT_MXFP8_E4M3, recv_rows=rows2)
+    for e in range(len(A2.expert_count)):
+        lo, hi = A2.expert_offset[e], A2.expert_offset[e + 1]
+        seg = t2[lo * B: hi * B].reshape(-1, B // 4, 32, 4, 4).transpose(0, 3, 2, 1, 4).reshape(hi - lo, B)
+        assert np.array_equal(seg, r2[lo:hi])
+
+
+def test_scale_layout_rejects_undefined_pairs():
+    x_bits, A, rows = _scaled_case(O.DT_FP8_E4M3)
+    for dt, lay in ((O.DT_FP8_E4M3, O.SL_MMA_TILED), (O.DT_BF16, O.SL_MN_MAJOR)):
+        with pytest.raises(ValueError):
+            O.dispatch_scaled(x_bits, A.token_slot, dt, lay, recv_rows=rows)
