@@ -101,6 +101,8 @@ def _declare(L):
     L.oracle_scale_index.restype = _L64
     L.oracle_dispatch_scaled.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _I, _P, _P]
     L.oracle_dispatch_scaled.restype = _I
+    L.oracle_swiglu_quant.argtypes = [_P, _L64, _I, _P, _I, _I, _P, _P]
+    L.oracle_swiglu_quant.restype = _I
     L.oracle_combine.argtypes = [_P, _L64, _I, _I, _I, _P, _P, _P]
     L.oracle_combine.restype = _I
     L.oracle_dispatch_backward.argtypes = [_P, _L64, _I, _I, _I, _P, _P]
@@ -292,6 +294,34 @@ def dispatch_scaled(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int, layo
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch_scaled: invalid argument")
     return recv, scale, st
+
+
+def swiglu_quant(h_bf16: np.ndarray, slot_token: np.ndarray | None, dtype: int,
+                 layout: int = SL_ROW_MAJOR):
+    """a = silu(gate) * up of each row of ``h`` = [gate | up] (bf16 bits [S, 2I]),
+    quantised like a dispatched row: (out, flat scale buffer or None, status).
+    out is bf16 bits [S, I] (BF16) or e4m3 codes [S, I]; rows whose slot_token
+    is -1 are skipped (left 0)."""
+    h_bf16 = _c(h_bf16, np.uint16)
+    S, I2 = h_bf16.shape
+    I = I2 // 2
+    st_ptr = None
+    if slot_token is not None:
+        slot_token = _c(slot_token, np.int32)
+        assert slot_token.shape == (S,)
+        st_ptr = _ptr(slot_token)
+    out = np.zeros((S, I), np.uint16 if dtype == DT_BF16 else np.uint8)
+    scale, sp = None, None
+    if dtype != DT_BF16:
+        n = scale_elems(S, I, dtype, layout)
+        if n < 0:
+            raise ValueError("oracle_swiglu_quant: layout not defined for this payload")
+        scale = np.zeros(n, np.uint8 if dtype == DT_MXFP8_E4M3 else np.float32)
+        sp = _ptr(scale)
+    st = lib().oracle_swiglu_quant(_ptr(h_bf16), S, I, st_ptr, dtype, layout, _ptr(out), sp)
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_swiglu_quant: invalid argument")
+    return out, scale, st
 
 
 def combine(y_bf16: np.ndarray, token_slot: np.ndarray, topk_w: np.ndarray):

@@ -693,6 +693,92 @@ int oracle_dispatch_scaled(const uint16_t* x, int N, int H, int k, const int32_t
 }
 
 /* ------------------------------------------------------------------ */
+/* SwiGLU fused with quantisation.  [TK] list: SwiGLU combined with the
+ * quantisation operations.  Between an expert's two GEMMs the first one's
+ * output row h = [gate | up] (bf16, 2I channels; reading: the gate half
+ * first) becomes a = SiLU(gate) * up, quantised for the second GEMM.
+ * Reading (fp32, every operation rounded once):
+ *   silu(g) = g / (1 + dexp(-g))   (the textbook x * sigmoid(x), written
+ *                                   as one division)
+ *   a_c     = silu(g_c) * u_c
+ * a is quantised the way dispatch quantises a row, with these fp32 values
+ * in place of the bf16 ones: BF16 (a rounded to bf16), per-128-block FP8,
+ * per-row FP8 or MXFP8, scales in any layout of oracle_scale_index over
+ * num_rows rows.  Rows whose slot_token is -1 (padding of the aligned
+ * layout) are skipped; slot_token may be NULL (every row).             */
+/* ------------------------------------------------------------------ */
+static float silu_f32(float g)
+{
+    float e = oracle_dexp(-g);
+    float d = 1.0f + e;
+    return g / d;
+}
+
+/* quantise one fp32 row of n values: codes (or bf16) to out_row, fp32
+ * scales to fsc or E8M0 bytes to esc, one per block */
+static void quantize_f32_row(const float* a, int n, int dtype, void* out_row, float* fsc,
+                             uint8_t* esc)
+{
+    if (dtype == DT_BF16) {
+        for (int c = 0; c < n; ++c) ((uint16_t*)out_row)[c] = oracle_bf16_from_f32(a[c]);
+        return;
+    }
+    uint8_t* q = (uint8_t*)out_row;
+    int bw = dtype == DT_FP8_E4M3 ? 128 : (dtype == DT_MXFP8_E4M3 ? 32 : n);
+    for (int b = 0; b * bw < n; ++b) {
+        float amax = 0.0f;
+        for (int c = b * bw; c < (b + 1) * bw; ++c)
+            if (fabsf(a[c]) > amax) amax = fabsf(a[c]);
+        if (dtype == DT_MXFP8_E4M3) {
+            int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;
+            if (e < -127) e = -127;
+            if (e > 127) e = 127;
+            esc[b] = (uint8_t)(e + 127);
+            float down = ldexpf(1.0f, -e);   /* e <= 119 for finite a: a normal float */
+            for (int c = b * bw; c < (b + 1) * bw; ++c)
+                q[c] = oracle_e4m3_encode((a[c] == 0.0f) ? a[c] : a[c] * down);
+        } else {
+            float inv = 448.0f / amax;
+            fsc[b] = amax / 448.0f;
+            for (int c = b * bw; c < (b + 1) * bw; ++c)
+                q[c] = oracle_e4m3_encode((a[c] == 0.0f) ? a[c] : a[c] * inv);
+        }
+    }
+}
+
+int oracle_swiglu_quant(const uint16_t* h, int64_t num_rows, int I, const int32_t* slot_token,
+                        int dtype, int layout, void* out, void* out_scale)
+{
+    if (num_rows < 0 || I < 1 || dtype < DT_BF16 || dtype > DT_MXFP8_E4M3) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_FP8_E4M3 && I % 128 != 0) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_MXFP8_E4M3 && I % 32 != 0) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_BF16 ? layout != SL_ROW_MAJOR : oracle_scale_elems(num_rows, I, dtype, layout) < 0)
+        return ORC_ERR_INVALID_ARG;
+    int B = scale_blocks(I, dtype), es = scale_elem_bytes(dtype);
+    int ob = dtype == DT_BF16 ? 2 : 1;
+    float* a = (float*)malloc(sizeof(float) * (size_t)I);
+    float* fsc = (float*)malloc(sizeof(float) * (size_t)(B > 0 ? B : 1));
+    uint8_t* esc = (uint8_t*)malloc((size_t)(B > 0 ? B : 1));
+    for (int64_t s = 0; s < num_rows; ++s) {
+        if (slot_token && slot_token[s] < 0) continue;
+        const uint16_t* hr = h + (size_t)s * 2 * I;
+        for (int c = 0; c < I; ++c) {
+            float g = oracle_f32_from_bf16(hr[c]);
+            float u = oracle_f32_from_bf16(hr[I + c]);
+            a[c] = silu_f32(g) * u;
+        }
+        quantize_f32_row(a, I, dtype, (uint8_t*)out + (size_t)s * I * ob, fsc, esc);
+        for (int b = 0; b < B; ++b) {
+            const void* src = dtype == DT_MXFP8_E4M3 ? (const void*)&esc[b] : (const void*)&fsc[b];
+            memcpy((uint8_t*)out_scale + oracle_scale_index(layout, num_rows, I, dtype, s, b) * es,
+                   src, (size_t)es);
+        }
+    }
+    free(a); free(fsc); free(esc);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* Combine.  [pplx] Introduction and Combine: the token's output is the
  * average of its experts' outputs weighted by the router weights; [EPv2]
  * usage patterns: combine reduces the expert outputs back to the token.

@@ -57,6 +57,10 @@ MUTANTS = {
                                       "return atom * 512 + ((s % 128) / 32) * 16 + (s % 32) * 4 + b % 4;"),
     "mma_tile_atoms_column_major": ("int64_t atom = (s / 128) * (B / 4) + b / 4;",
                                     "int64_t atom = (b / 4) * ((num_rows + 127) / 128) + s / 128;"),
+    "silu_wrong_sign": ("float e = oracle_dexp(-g);", "float e = oracle_dexp(g);"),
+    "swiglu_halves_swapped": ("float g = oracle_f32_from_bf16(hr[c]);\n            float u = oracle_f32_from_bf16(hr[I + c]);",
+                              "float g = oracle_f32_from_bf16(hr[I + c]);\n            float u = oracle_f32_from_bf16(hr[c]);"),
+    "swiglu_padding_not_skipped": ("if (slot_token && slot_token[s] < 0) continue;", "(void)slot_token;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

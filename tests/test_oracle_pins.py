@@ -775,3 +775,81 @@ def test_scale_layout_rejects_undefined_pairs():
     for dt, lay in ((O.DT_FP8_E4M3, O.SL_MMA_TILED), (O.DT_BF16, O.SL_MN_MAJOR)):
         with pytest.raises(ValueError):
             O.dispatch_scaled(x_bits, A.token_slot, dt, lay, recv_rows=rows)
+
+
+# ----------------------------------------------------------------- SwiGLU + quantisation
+def _bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_swiglu_closed_forms():
+    g = np.array([0.0, -0.0, 20.0, 37.5, 1e4, -100.0, -1e30, 1.0], np.float32)
+    u = np.array([3.0, 3.0, 1.0, -2.0, 0.5, 1.0, 1.0, 1.0], np.float32)
+    I = len(g)
+    h = np.concatenate([_bf16(g), _bf16(u)])[None, :]
+    out, _, st = O.swiglu_quant(h, None, O.DT_BF16)
+    got = O.bf16_to_f32(out[0]).astype(np.float64)
+    gb, ub = O.bf16_to_f32(h[0, :I]).astype(np.float64), O.bf16_to_f32(h[0, I:]).astype(np.float64)
+    assert st == 0
+    assert got[0] == 0 and got[1] == 0
+    for i in (2, 3, 4):                                  # 1 + e^-g rounds to 1: silu(g) = g exactly
+        assert got[i] == O.bf16_to_f32(_bf16(np.float32(gb[i] * ub[i]))[None])[0]
+    assert -1e-36 < got[5] < 0                           # -100 / (1 + e^88): tiny, negative
+    assert got[6] == -0.0 or got[6] < 0                  # the exponent is clamped, no NaN
+    ref = 1.0 / (1.0 + math.exp(-1.0))                   # silu(1) * 1
+    assert abs(got[7] - ref) <= 2.0**-8 * ref
+
+
+def test_swiglu_vs_float64():
+    rng = np.random.default_rng(21)
+    S, I = 64, 256
+    h = _bf16(rng.normal(scale=2.0, size=(S, 2 * I)))
+    out, _, st = O.swiglu_quant(h, None, O.DT_BF16)
+    hf = O.bf16_to_f32(h).astype(np.float64)
+    g, u = hf[:, :I], hf[:, I:]
+    ref = g / (1.0 + np.exp(-g)) * u
+    got = O.bf16_to_f32(out).astype(np.float64)
+    ulp = np.spacing(np.abs(ref).astype(np.float32)).astype(np.float64) * 2.0**16   # one bf16 ulp
+    assert st == 0 and (np.abs(got - ref) <= ulp).all()
+    assert (np.abs(got - ref) <= 2.0**-8 * np.abs(ref) * (1 + 2.0**-6) + 1e-38).all()
+
+
+@pytest.mark.parametrize("dtype,layout", [(O.DT_FP8_E4M3, O.SL_ROW_MAJOR), (O.DT_FP8_E4M3, O.SL_MN_MAJOR),
+                                          (O.DT_FP8_E4M3_TOKEN, O.SL_ROW_MAJOR), (O.DT_MXFP8_E4M3, O.SL_ROW_MAJOR),
+                                          (O.DT_MXFP8_E4M3, O.SL_MMA_TILED), (O.DT_BF16, O.SL_ROW_MAJOR)])
+def test_swiglu_quant_equals_dispatch_of_exact_activations(dtype, layout):
+    """With gate >= 20 the SiLU is the identity (1 + e^-g rounds to 1) and with
+    up = +-1 or +-0 every a = silu(g) * u is an exact bf16 value: the fused op
+    must then quantise exactly as dispatch quantises that bf16 row."""
+    rng = np.random.default_rng(33 + dtype)
+    S, I = 40, 512
+    g = np.exp2(rng.integers(5, 21, (S, I))) * rng.uniform(1, 2, (S, I))
+    g = O.bf16_to_f32(_bf16(g)).astype(np.float32)
+    u = rng.choice(np.array([1.0, -1.0, 0.0, -0.0], np.float32), (S, I), p=[0.45, 0.45, 0.05, 0.05])
+    u[3] = 0.0                                           # an all-zero row
+    h = np.concatenate([_bf16(g), _bf16(u)], axis=1)
+    a = (g * u).astype(np.float32)
+    out, sc, st = O.swiglu_quant(h, None, dtype, layout)
+    slots = np.arange(S, dtype=np.int32)[:, None]
+    r_out, r_sc, rst = O.dispatch_scaled(_bf16(a), slots, dtype, layout)
+    assert st == 0 and rst == 0
+    assert np.array_equal(out, r_out)
+    if sc is not None:
+        assert np.array_equal(sc.view(np.uint8), r_sc.view(np.uint8))
+
+
+def test_swiglu_skips_padding_rows():
+    rng = np.random.default_rng(8)
+    S, I = 300, 128
+    h = _bf16(rng.normal(size=(S, 2 * I)))
+    slot_token = rng.integers(-1, 50, S).astype(np.int32)
+    full, fsc, _ = O.swiglu_quant(h, None, O.DT_FP8_E4M3)
+    part, psc, st = O.swiglu_quant(h, slot_token, O.DT_FP8_E4M3)
+    keep = slot_token >= 0
+    assert st == 0 and np.array_equal(part[keep], full[keep]) and (part[~keep] == 0).all()
+    assert np.array_equal(psc.reshape(S, -1)[keep], fsc.reshape(S, -1)[keep])
+    assert (psc.reshape(S, -1)[~keep] == 0).all()
+    for dt, lay, I_bad in ((O.DT_FP8_E4M3, O.SL_ROW_MAJOR, 96), (O.DT_BF16, O.SL_MN_MAJOR, 128),
+                           (O.DT_FP8_E4M3, O.SL_MMA_TILED, 128)):
+        with pytest.raises(ValueError):
+            O.swiglu_quant(h[:, :2 * I_bad], None, dt, lay)
