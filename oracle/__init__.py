@@ -29,6 +29,7 @@ DT_BF16 = 0
 DT_FP8_E4M3 = 1
 DT_FP8_E4M3_TOKEN = 2
 DT_MXFP8_E4M3 = 3
+DT_NVFP4 = 4
 SL_ROW_MAJOR = 0
 SL_MN_MAJOR = 1
 SL_MMA_TILED = 2
@@ -77,6 +78,10 @@ def _declare(L):
     L.oracle_e4m3_encode.restype = ctypes.c_uint8
     L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
     L.oracle_e4m3_decode.restype = ctypes.c_float
+    L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
+    L.oracle_e2m1_encode.restype = ctypes.c_uint8
+    L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
+    L.oracle_e2m1_decode.restype = ctypes.c_float
     L.oracle_bf16_from_f32.argtypes = [ctypes.c_float]
     L.oracle_bf16_from_f32.restype = ctypes.c_uint16
     L.oracle_f32_from_bf16.argtypes = [ctypes.c_uint16]
@@ -101,6 +106,8 @@ def _declare(L):
     L.oracle_scale_index.restype = _L64
     L.oracle_dispatch_scaled.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _I, _P, _P]
     L.oracle_dispatch_scaled.restype = _I
+    L.oracle_dispatch_nvfp4.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _P, _P, _P]
+    L.oracle_dispatch_nvfp4.restype = _I
     L.oracle_swiglu_quant.argtypes = [_P, _L64, _I, _P, _I, _I, _P, _P]
     L.oracle_swiglu_quant.restype = _I
     L.oracle_combine.argtypes = [_P, _L64, _I, _I, _I, _P, _P, _P]
@@ -131,6 +138,14 @@ def sigmoid(x: float) -> float:
 
 def e4m3_encode(f: float) -> int:
     return lib().oracle_e4m3_encode(f)
+
+
+def e2m1_encode(f: float) -> int:
+    return int(lib().oracle_e2m1_encode(f))
+
+
+def e2m1_decode(c: int) -> float:
+    return float(lib().oracle_e2m1_decode(c))
 
 
 def e4m3_decode(c: int) -> float:
@@ -294,6 +309,29 @@ def dispatch_scaled(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int, layo
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch_scaled: invalid argument")
     return recv, scale, st
+
+
+def dispatch_nvfp4(x_bf16: np.ndarray, token_slot: np.ndarray, layout: int = SL_ROW_MAJOR,
+                   recv_rows: int | None = None):
+    """NVFP4 dispatch: (recv_x packed e2m1 [S, H/2] uint8, block scales (flat
+    uint8, e4m3 codes in ``layout``), row scales fp32 [S], status).  Rows no
+    slot names stay 0."""
+    x_bf16 = _c(x_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    N, H = x_bf16.shape
+    k = token_slot.shape[1]
+    S = N * k if recv_rows is None else recv_rows
+    n = scale_elems(S, H, DT_NVFP4, layout)
+    if n < 0 or H % 64:
+        raise ValueError("oracle_dispatch_nvfp4: invalid argument")
+    recv = np.zeros((S, H // 2), np.uint8)
+    bs = np.zeros(n, np.uint8)
+    rs = np.zeros(S, np.float32)
+    st = lib().oracle_dispatch_nvfp4(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, layout, _ptr(recv),
+                                     _ptr(bs), _ptr(rs))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_dispatch_nvfp4: invalid argument")
+    return recv, bs, rs, st
 
 
 def swiglu_quant(h_bf16: np.ndarray, slot_token: np.ndarray | None, dtype: int,

@@ -45,6 +45,7 @@
 #define DT_FP8_E4M3 1
 #define DT_FP8_E4M3_TOKEN 2
 #define DT_MXFP8_E4M3 3
+#define DT_NVFP4 4
 
 /* ------------------------------------------------------------------ */
 /* bit helpers                                                         */
@@ -157,6 +158,30 @@ uint8_t oracle_e4m3_encode(float f)
 void oracle_e4m3_encode_array(const float* in, uint8_t* out, size_t n)
 {
     for (size_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(in[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* FP4 E2M1 (the OCP MX element type that NVFP4 uses: 1 sign, 2 exponent
+ * bits with bias 1, 1 mantissa bit; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6;
+ * no infinity, no NaN).  Encoding rounds to nearest, ties to the even
+ * mantissa, and saturates beyond 6 (infinity too) to +-6.  NaN inputs are
+ * outside the contract.                                                */
+/* ------------------------------------------------------------------ */
+float oracle_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (float)(s ? -v : v);
+}
+
+uint8_t oracle_e2m1_encode(float f)
+{
+    uint8_t sign = (f32_bits(f) >> 31) ? 0x8 : 0x0;
+    double a = fabs((double)f);
+    if (!(a < 6.0)) return sign | 0x7;           /* saturate (and NaN) */
+    if (a < 2.0) return sign | (uint8_t)nearbyint(a * 2.0);      /* steps of 0.5: codes 0..4 */
+    if (a < 4.0) return sign | (uint8_t)(2 + nearbyint(a));      /* 2, 3, 4 -> codes 4, 5, 6 */
+    return sign | (uint8_t)(4 + nearbyint(a * 0.5));              /* 4, 6 -> codes 6, 7 */
 }
 
 void oracle_dexp_array(const float* in, float* out, size_t n)
@@ -634,10 +659,11 @@ static int scale_blocks(int H, int dtype)
     if (dtype == DT_FP8_E4M3) return H / 128;
     if (dtype == DT_FP8_E4M3_TOKEN) return 1;
     if (dtype == DT_MXFP8_E4M3) return H / 32;
+    if (dtype == DT_NVFP4) return H / 16;
     return 0;
 }
 
-static int scale_elem_bytes(int dtype) { return dtype == DT_MXFP8_E4M3 ? 1 : 4; }
+static int scale_elem_bytes(int dtype) { return (dtype == DT_MXFP8_E4M3 || dtype == DT_NVFP4) ? 1 : 4; }
 
 static int64_t round_up64(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
@@ -649,7 +675,7 @@ int64_t oracle_scale_elems(int64_t num_rows, int H, int dtype, int layout)
     if (num_rows < 0 || B < 1) return -1;
     if (layout == SL_ROW_MAJOR) return num_rows * B;
     if (layout == SL_MN_MAJOR) return (int64_t)B * round_up64(num_rows, 16 / scale_elem_bytes(dtype));
-    if (layout == SL_MMA_TILED && dtype == DT_MXFP8_E4M3 && B % 4 == 0)
+    if (layout == SL_MMA_TILED && (dtype == DT_MXFP8_E4M3 || dtype == DT_NVFP4) && B % 4 == 0)
         return round_up64(num_rows, 128) * B;
     return -1;
 }
@@ -690,6 +716,72 @@ int oracle_dispatch_scaled(const uint16_t* x, int N, int H, int k, const int32_t
     }
     free(rows);
     return st;
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4 dispatch.  [EPv2] feature list (Hybrid-EP: NVFP4 support) and [TK]
+ * (FP4 conversion) name the format without its rule.  Reading, per token t
+ * (the per-token mode of [TK]), the two-level NVFP4 scaling with the
+ * token's row in place of the tensor:
+ *   amax_t = max_c |x[t,c]|,  g_t = amax_t / 2688 (448 * 6, the largest
+ *            e4m3 times the largest e2m1): the row's fp32 scale,
+ *   inv_t  = 2688 / amax_t,
+ *   per block b of 16 channels: sb = e4m3((amax_b / 6) * inv_t) if
+ *            amax_b > 0, else 0 (an unsigned e4m3 code),
+ *   r_b    = inv_t / e4m3_value(sb),
+ *   q_c    = e2m1(x_c * r_b)  (a zero keeps its sign, as in FP8),
+ * every operation in fp32 rounded once; x is recovered as
+ * e2m1_value(q) * e4m3_value(sb) * g_t.  Two codes per byte, channel 2i in
+ * the low nibble.  Block scales (one byte per 16 channels) in any layout of
+ * oracle_scale_index; the row scales fp32 [num_rows].  H % 64 == 0.    */
+/* ------------------------------------------------------------------ */
+int oracle_dispatch_nvfp4(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                          int64_t num_rows, int layout, uint8_t* recv_x, uint8_t* block_scale,
+                          float* row_scale)
+{
+    if (N < 0 || H < 64 || H % 64 != 0 || k < 1 || num_rows < 0) return ORC_ERR_INVALID_ARG;
+    if (oracle_scale_elems(num_rows, H, DT_NVFP4, layout) < 0) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    int B = H / 16;
+    uint8_t* q = (uint8_t*)malloc((size_t)H / 2);
+    uint8_t* sb = (uint8_t*)malloc((size_t)B);
+    for (int t = 0; t < N; ++t) {
+        const uint16_t* xr = x + (size_t)t * H;
+        float amax_t = 0.0f;
+        for (int c = 0; c < H; ++c) {
+            float v = fabsf(oracle_f32_from_bf16(xr[c]));
+            if (v > amax_t) amax_t = v;
+        }
+        float g = amax_t / 2688.0f;
+        float inv = 2688.0f / amax_t;
+        for (int b = 0; b < B; ++b) {
+            float amax_b = 0.0f;
+            for (int c = b * 16; c < (b + 1) * 16; ++c) {
+                float v = fabsf(oracle_f32_from_bf16(xr[c]));
+                if (v > amax_b) amax_b = v;
+            }
+            float sbf = (amax_b / 6.0f) * inv;
+            sb[b] = amax_b > 0.0f ? oracle_e4m3_encode(sbf) : 0;
+            float r = inv / oracle_e4m3_decode(sb[b]);
+            for (int c = b * 16; c < (b + 1) * 16; c += 2) {
+                float v0 = oracle_f32_from_bf16(xr[c]), v1 = oracle_f32_from_bf16(xr[c + 1]);
+                uint8_t lo = oracle_e2m1_encode(v0 == 0.0f ? v0 : v0 * r);
+                uint8_t hi = oracle_e2m1_encode(v1 == 0.0f ? v1 : v1 * r);
+                q[c / 2] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+        for (int j = 0; j < k; ++j) {
+            int32_t s = token_slot[(int64_t)t * k + j];
+            if (s == -1) continue;
+            if (s < -1 || s >= num_rows) { status = ORC_ERR_BAD_INDEX; continue; }
+            memcpy(recv_x + (size_t)s * (H / 2), q, (size_t)H / 2);
+            for (int b = 0; b < B; ++b)
+                block_scale[oracle_scale_index(layout, num_rows, H, DT_NVFP4, s, b)] = sb[b];
+            row_scale[s] = g;
+        }
+    }
+    free(q); free(sb);
+    return status;
 }
 
 /* ------------------------------------------------------------------ */

@@ -32,7 +32,8 @@ MUTANTS = {
                                   "if (e >= 0 && e < E && e % epr == r) hit = 1;", 0),
     "aligned_rank_tokens_modulo": ("if (e >= 0 && e < E && e / epr == r) hit = 1;",
                                    "if (e >= 0 && e < E && e % epr == r) hit = 1;", 1),
-    "fp8_scale_transposed": ("sc[b] = amax / 448.0f;", "sc[b] = 448.0f / amax;"),
+    "fp8_scale_transposed": (" sc[b] = amax / 448.0f;", " sc[b] = 448.0f / amax;"),
+    "swiglu_fp8_scale_transposed": ("fsc[b] = amax / 448.0f;", "fsc[b] = 448.0f / amax;"),
     "e4m3_ties_away": ("double m = nearbyint(q);                     /* ties to even */",
                        "double m = floor(q + 0.5);"),
     "e4m3_subnormal_step": ("double q = a * 512.0;", "double q = a * 256.0;"),
@@ -45,7 +46,9 @@ MUTANTS = {
     "combine_backward_dot_wrong_row": ("double term = (double)gc * (double)oracle_f32_from_bf16(yr[c]);",
                                        "double term = (double)gc * (double)oracle_f32_from_bf16(yr[0]);"),
     "mxfp8_exponent_off_by_one": ("int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;",
-                                  "int e = (amax > 0.0f) ? floor_log2_pos(amax) - 7 : -127;"),
+                                  "int e = (amax > 0.0f) ? floor_log2_pos(amax) - 7 : -127;", 0),
+    "swiglu_mxfp8_exponent_off_by_one": ("int e = (amax > 0.0f) ? floor_log2_pos(amax) - 8 : -127;",
+                                         "int e = (amax > 0.0f) ? floor_log2_pos(amax) - 7 : -127;", 1),
     "fp8_token_scale_transposed": ("fsc[0] = amax / 448.0f;", "fsc[0] = 448.0f / amax;"),
     "aligned_layout_rounds_down": ("int32_t padded = (expert_count[e] + align - 1) / align * align;",
                                    "int32_t padded = expert_count[e] / align * align;"),
@@ -61,6 +64,11 @@ MUTANTS = {
     "swiglu_halves_swapped": ("float g = oracle_f32_from_bf16(hr[c]);\n            float u = oracle_f32_from_bf16(hr[I + c]);",
                               "float g = oracle_f32_from_bf16(hr[I + c]);\n            float u = oracle_f32_from_bf16(hr[c]);"),
     "swiglu_padding_not_skipped": ("if (slot_token && slot_token[s] < 0) continue;", "(void)slot_token;"),
+    "nvfp4_nibbles_swapped": ("q[c / 2] = (uint8_t)(lo | (hi << 4));", "q[c / 2] = (uint8_t)(hi | (lo << 4));"),
+    "nvfp4_ratio_uses_unrounded_block_scale": ("float r = inv / oracle_e4m3_decode(sb[b]);", "float r = inv / sbf;"),
+    "nvfp4_block_scale_from_row_amax": ("float sbf = (amax_b / 6.0f) * inv;", "float sbf = (amax_t / 6.0f) * inv;"),
+    "nvfp4_row_scale_inverted": ("float g = amax_t / 2688.0f;", "float g = 2688.0f / amax_t;"),
+    "e2m1_ties_away": ("if (a < 2.0) return sign | (uint8_t)nearbyint(a * 2.0);", "if (a < 2.0) return sign | (uint8_t)floor(a * 2.0 + 0.5);"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

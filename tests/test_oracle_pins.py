@@ -853,3 +853,80 @@ def test_swiglu_skips_padding_rows():
                            (O.DT_FP8_E4M3, O.SL_MMA_TILED, 128)):
         with pytest.raises(ValueError):
             O.swiglu_quant(h[:, :2 * I_bad], None, dt, lay)
+
+
+# ----------------------------------------------------------------- FP4 E2M1 and NVFP4
+def test_e2m1_decode_table():
+    g = _gold("nvfp4_worked_example.json")
+    for c in range(16):
+        v = O.e2m1_decode(c)
+        assert v == g["e2m1_values"][c] and math.copysign(1, v) == math.copysign(1, g["e2m1_values"][c])
+
+
+def test_e2m1_encode_brute_force_nearest_even():
+    """Every bf16 value in [-8, 8] and a dense fp32 grid: the code of the nearest
+    E2M1 value, ties to the even mantissa bit, saturating beyond 6."""
+    mags = np.array([O.e2m1_decode(c) for c in range(8)])
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = O.bf16_to_f32(bits)
+    vals = vals[np.isfinite(vals) & (np.abs(vals) <= 8)]
+    vals = np.concatenate([vals, np.linspace(-7, 7, 20001, dtype=np.float32), mags.astype(np.float32) + 0.25])
+    for v in vals:
+        a = abs(float(v))
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        code = int(best[0]) if len(best) == 1 else int(best[best % 2 == 0][0])
+        if a >= 6:
+            code = 7
+        code |= 8 if math.copysign(1, float(v)) < 0 else 0
+        assert O.e2m1_encode(float(v)) == code, (v, O.e2m1_encode(float(v)), code)
+
+
+def test_nvfp4_worked_example():
+    g = _gold("nvfp4_worked_example.json")
+    x0 = np.array(g["x_token0"], np.float32)
+    x = np.stack([x0, x0 * np.float32(g["token1_factor"])])
+    xb = _bf16(x)
+    assert np.array_equal(O.bf16_to_f32(xb), x)                 # every value is exact in bf16
+    slots = np.array([[1], [0]], np.int32)                      # token 0 -> row 1, token 1 -> row 0
+    recv, bs, rs, st = O.dispatch_nvfp4(xb, slots)
+    assert st == 0
+    assert recv[1].tolist() == g["codes_token0"] and recv[0].tolist() == g["codes_token0"]
+    assert bs.reshape(2, -1)[1].tolist() == g["block_scales"] == bs.reshape(2, -1)[0].tolist()
+    assert rs.tolist() == [g["row_scales"][1], g["row_scales"][0]]
+    x2 = _bf16(np.array(g["x_token2"], np.float32)[None])
+    r2, b2, s2, st = O.dispatch_nvfp4(x2, np.array([[0]], np.int32))
+    assert st == 0 and r2[0].tolist() == g["codes_token2"] and b2.tolist() == g["block_scales_token2"]
+    assert s2.tolist() == [1.0]
+
+
+def test_nvfp4_round_trip_bound_and_tiled_layout():
+    rng = np.random.default_rng(12)
+    N, H, k = 50, 512, 2
+    x = rng.normal(size=(N, H)) * np.exp2(rng.integers(-8, 8, (N, H // 16))).repeat(16, 1)
+    x[3] = 0.0
+    xb = _bf16(x)
+    xf = O.bf16_to_f32(xb).astype(np.float64)
+    slots = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    recv, bs, rs, st = O.dispatch_nvfp4(xb, slots)
+    assert st == 0
+    lo, hi = recv & 0xF, recv >> 4
+    codes = np.stack([lo, hi], axis=-1).reshape(N * k, H)
+    dec = np.array([O.e2m1_decode(c) for c in range(16)])[codes]
+    sbv = np.array([O.e4m3_decode(c) for c in range(256)])[bs.reshape(N * k, -1)].repeat(16, 1)
+    deq = dec * sbv * rs.astype(np.float64)[:, None]
+    ref = xf[np.argsort(slots.reshape(-1)) // k]
+    amax_b = np.abs(ref).reshape(N * k, -1, 16).max(-1).repeat(16, 1)
+    bound = 1.07 * amax_b / 6 + 6.1 * 2.0**-10 * rs.astype(np.float64)[:, None]
+    assert (np.abs(deq - ref) <= bound).all()
+    # the largest element of each row decodes within 6.25 % (sb rounds by at most half an e4m3 step)
+    row_max = np.abs(ref).max(1)
+    assert (np.abs(np.abs(deq).max(1) - row_max) <= 0.0625 * row_max + 1e-30).all()
+    # tiled block scales are the same bytes in the block-scaled MMA's order
+    rows = N * k
+    _, bt, _, _ = O.dispatch_nvfp4(xb, slots, O.SL_MMA_TILED)
+    B = H // 16
+    Sp = -(-rows // 128) * 128
+    padded = np.zeros((Sp, B), np.uint8)
+    padded[:rows] = bs.reshape(rows, B)
+    assert np.array_equal(bt, padded.reshape(Sp // 128, 4, 32, B // 4, 4).transpose(0, 3, 2, 1, 4).reshape(-1))
