@@ -30,6 +30,7 @@ DT_FP8_E4M3 = 1
 DT_FP8_E4M3_TOKEN = 2
 DT_MXFP8_E4M3 = 3
 DT_NVFP4 = 4
+DT_E5M6 = 5
 SL_ROW_MAJOR = 0
 SL_MN_MAJOR = 1
 SL_MMA_TILED = 2
@@ -78,6 +79,10 @@ def _declare(L):
     L.oracle_e4m3_encode.restype = ctypes.c_uint8
     L.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
     L.oracle_e4m3_decode.restype = ctypes.c_float
+    L.oracle_e5m6_encode.argtypes = [ctypes.c_float]
+    L.oracle_e5m6_encode.restype = ctypes.c_uint16
+    L.oracle_e5m6_decode.argtypes = [ctypes.c_uint16]
+    L.oracle_e5m6_decode.restype = ctypes.c_float
     L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
     L.oracle_e2m1_encode.restype = ctypes.c_uint8
     L.oracle_e2m1_decode.argtypes = [ctypes.c_uint8]
@@ -106,6 +111,8 @@ def _declare(L):
     L.oracle_scale_index.restype = _L64
     L.oracle_dispatch_scaled.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _I, _P, _P]
     L.oracle_dispatch_scaled.restype = _I
+    L.oracle_dispatch_e5m6.argtypes = [_P, _I, _I, _I, _P, _L64, _P]
+    L.oracle_dispatch_e5m6.restype = _I
     L.oracle_dispatch_nvfp4.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _P, _P, _P]
     L.oracle_dispatch_nvfp4.restype = _I
     L.oracle_swiglu_quant.argtypes = [_P, _L64, _I, _P, _I, _I, _P, _P]
@@ -138,6 +145,28 @@ def sigmoid(x: float) -> float:
 
 def e4m3_encode(f: float) -> int:
     return lib().oracle_e4m3_encode(f)
+
+
+def e5m6_encode(f: float) -> int:
+    return int(lib().oracle_e5m6_encode(f))
+
+
+def e5m6_decode(c: int) -> float:
+    return float(lib().oracle_e5m6_decode(c))
+
+
+def dispatch_e5m6(x_bf16: np.ndarray, token_slot: np.ndarray, recv_rows: int | None = None):
+    """E5M6 dispatch: (recv_x uint8 [S, 3H/2] (two 12-bit codes per 3 bytes), status)."""
+    x_bf16 = _c(x_bf16, np.uint16)
+    token_slot = _c(token_slot, np.int32)
+    N, H = x_bf16.shape
+    k = token_slot.shape[1]
+    S = N * k if recv_rows is None else recv_rows
+    recv = np.zeros((S, H // 2 * 3), np.uint8)
+    st = lib().oracle_dispatch_e5m6(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, _ptr(recv))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_dispatch_e5m6: invalid argument")
+    return recv, st
 
 
 def e2m1_encode(f: float) -> int:

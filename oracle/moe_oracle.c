@@ -46,6 +46,7 @@
 #define DT_FP8_E4M3_TOKEN 2
 #define DT_MXFP8_E4M3 3
 #define DT_NVFP4 4
+#define DT_E5M6 5
 
 /* ------------------------------------------------------------------ */
 /* bit helpers                                                         */
@@ -158,6 +159,48 @@ uint8_t oracle_e4m3_encode(float f)
 void oracle_e4m3_encode_array(const float* in, uint8_t* out, size_t n)
 {
     for (size_t i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(in[i]);
+}
+
+/* ------------------------------------------------------------------ */
+/* E5M6, a 12-bit float.  [TK] lists E5M6 conversion without a definition.
+ * Reading: the IEEE-style binary format with 1 sign bit, 5 exponent bits
+ * (bias 15) and 6 fraction bits -- FP16 with its 4 lowest fraction bits
+ * dropped: exponent field 0 holds the subnormals m * 2^-20, field 31 the
+ * infinities and NaNs, largest finite 2^15 * (1 + 63/64) = 65024.
+ * Encoding rounds to nearest, ties to even, and saturates every finite value
+ * (and infinity) beyond 65024 to +-65024, as the FP8 encoders here do.
+ * Two codes are packed in three bytes, little endian: code 2i in bits
+ * 0..11, code 2i+1 in bits 12..23.                                      */
+/* ------------------------------------------------------------------ */
+float oracle_e5m6_decode(uint16_t c)
+{
+    int s = (c >> 11) & 1, e = (c >> 6) & 31, m = c & 63;
+    double v;
+    if (e == 31) return m ? NAN : (s ? -INFINITY : INFINITY);
+    if (e == 0) v = ldexp((double)m, -20);
+    else v = ldexp(1.0 + m / 64.0, e - 15);
+    return (float)(s ? -v : v);
+}
+
+uint16_t oracle_e5m6_encode(float f)
+{
+    uint16_t sign = (f32_bits(f) >> 31) ? 0x800 : 0x000;
+    if (isnan(f)) return sign | 0x7FF;
+    double a = fabs((double)f);
+    if (a >= 65024.0) return sign | 0x7BF;       /* saturate */
+    if (a < ldexp(1.0, -14)) {                   /* subnormal range */
+        double m = nearbyint(a * 1048576.0);     /* units of 2^-20, exact; ties to even */
+        return sign | (uint16_t)m;               /* m == 64 is the code of 2^-14 */
+    }
+    int ex;
+    frexp(a, &ex);
+    int unb = ex - 1;                            /* a in [2^unb, 2^(unb+1)) */
+    double q = (ldexp(a, -unb) - 1.0) * 64.0;    /* fraction in 64ths, exact */
+    double m = nearbyint(q);                     /* ties to even */
+    int biased = unb + 15;
+    if (m == 64.0) { m = 0.0; biased += 1; }
+    if (biased >= 31) return sign | 0x7BF;
+    return sign | (uint16_t)((biased << 6) | (int)m);
 }
 
 /* ------------------------------------------------------------------ */
@@ -716,6 +759,39 @@ int oracle_dispatch_scaled(const uint16_t* x, int N, int H, int k, const int32_t
     }
     free(rows);
     return st;
+}
+
+/* ------------------------------------------------------------------ */
+/* E5M6 dispatch: every element of the token's row encoded on its own (no
+ * scale), the packed row copied to each of the token's receive rows
+ * (3H/2 bytes).  H % 32 == 0.                                           */
+/* ------------------------------------------------------------------ */
+int oracle_dispatch_e5m6(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                         int64_t num_rows, uint8_t* recv_x)
+{
+    if (N < 0 || H < 32 || H % 32 != 0 || k < 1 || num_rows < 0) return ORC_ERR_INVALID_ARG;
+    int status = ORC_OK;
+    size_t rb = (size_t)H / 2 * 3;
+    uint8_t* q = (uint8_t*)malloc(rb);
+    for (int t = 0; t < N; ++t) {
+        const uint16_t* xr = x + (size_t)t * H;
+        for (int c = 0; c < H; c += 2) {
+            uint32_t c0 = oracle_e5m6_encode(oracle_f32_from_bf16(xr[c]));
+            uint32_t c1 = oracle_e5m6_encode(oracle_f32_from_bf16(xr[c + 1]));
+            uint32_t w = c0 | (c1 << 12);
+            q[c / 2 * 3 + 0] = (uint8_t)(w & 0xFF);
+            q[c / 2 * 3 + 1] = (uint8_t)((w >> 8) & 0xFF);
+            q[c / 2 * 3 + 2] = (uint8_t)((w >> 16) & 0xFF);
+        }
+        for (int j = 0; j < k; ++j) {
+            int32_t s = token_slot[(int64_t)t * k + j];
+            if (s == -1) continue;
+            if (s < -1 || s >= num_rows) { status = ORC_ERR_BAD_INDEX; continue; }
+            memcpy(recv_x + (size_t)s * rb, q, rb);
+        }
+    }
+    free(q);
+    return status;
 }
 
 /* ------------------------------------------------------------------ */

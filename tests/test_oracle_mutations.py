@@ -69,6 +69,10 @@ MUTANTS = {
     "nvfp4_block_scale_from_row_amax": ("float sbf = (amax_b / 6.0f) * inv;", "float sbf = (amax_t / 6.0f) * inv;"),
     "nvfp4_row_scale_inverted": ("float g = amax_t / 2688.0f;", "float g = 2688.0f / amax_t;"),
     "e2m1_ties_away": ("if (a < 2.0) return sign | (uint8_t)nearbyint(a * 2.0);", "if (a < 2.0) return sign | (uint8_t)floor(a * 2.0 + 0.5);"),
+    "e5m6_ties_away": ("    double m = nearbyint(q);                     /* ties to even */\n    int biased = unb + 15;",
+                       "    double m = floor(q + 0.5);\n    int biased = unb + 15;"),
+    "e5m6_subnormal_step": ("double m = nearbyint(a * 1048576.0);", "double m = nearbyint(a * 524288.0);"),
+    "e5m6_pack_overlaps": ("uint32_t w = c0 | (c1 << 12);", "uint32_t w = c0 | (c1 << 8);"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

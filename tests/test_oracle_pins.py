@@ -930,3 +930,59 @@ def test_nvfp4_round_trip_bound_and_tiled_layout():
     padded = np.zeros((Sp, B), np.uint8)
     padded[:rows] = bs.reshape(rows, B)
     assert np.array_equal(bt, padded.reshape(Sp // 128, 4, 32, B // 4, 4).transpose(0, 3, 2, 1, 4).reshape(-1))
+
+
+# ----------------------------------------------------------------- E5M6
+def test_e5m6_decode_is_truncated_fp16():
+    """E5M6 code c is the FP16 value with bits c << 4 (same exponent field and
+    bias, the top 6 of FP16's 10 fraction bits): checked for all 4096 codes
+    against numpy's float16."""
+    codes = np.arange(4096, dtype=np.uint16)
+    want = (codes << 4).astype(np.uint16).view(np.float16).astype(np.float64)
+    got = np.array([O.e5m6_decode(int(c)) for c in codes], np.float64)
+    same = (got == want) | (np.isnan(got) & np.isnan(want))
+    assert same.all()
+    assert np.array_equal(np.signbit(got[~np.isnan(got)]), np.signbit(want[~np.isnan(want)]))
+
+
+def test_e5m6_encode_brute_force_nearest_even():
+    codes = np.arange(0x7C0, dtype=np.int64)                     # non-negative finite codes
+    vals = (codes.astype(np.uint16) << 4).view(np.float16).astype(np.float64)
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    xs = O.bf16_to_f32(bits)
+    xs = np.concatenate([xs[np.isfinite(xs)], np.float32(vals[1:] - np.diff(vals) / 2),   # exact midpoints
+                         np.linspace(-70000, 70000, 4001, dtype=np.float32)])
+    for x in xs:
+        a = abs(float(x))
+        if a >= 65024.0:
+            code = 0x7BF
+        else:
+            i = int(np.searchsorted(vals, a))
+            cand = [j for j in (i - 1, i) if 0 <= j < len(vals)]
+            d = [abs(vals[j] - a) for j in cand]
+            best = [cand[n] for n in range(len(cand)) if d[n] == min(d)]
+            code = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        code |= 0x800 if math.copysign(1, float(x)) < 0 else 0
+        assert O.e5m6_encode(float(x)) == code, (x, hex(O.e5m6_encode(float(x))), hex(code))
+
+
+def test_dispatch_e5m6_packs_two_codes_in_three_bytes():
+    rng = np.random.default_rng(17)
+    N, H, k = 30, 96, 3
+    x = _bf16(rng.normal(size=(N, H)) * np.exp2(rng.integers(-24, 17, (N, H))))
+    slots = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    slots[4, 2] = -1
+    recv, st = O.dispatch_e5m6(x, slots)
+    assert st == 0 and recv.shape == (N * k, H // 2 * 3)
+    w = recv.reshape(N * k, H // 2, 3).astype(np.uint32)
+    word = w[..., 0] | (w[..., 1] << 8) | (w[..., 2] << 16)
+    codes = np.stack([word & 0xFFF, word >> 12], -1).reshape(N * k, H)
+    xf = O.bf16_to_f32(x)
+    for t in range(N):
+        for j in range(k):
+            s = slots[t, j]
+            if s < 0:
+                continue
+            assert [O.e5m6_encode(float(v)) for v in xf[t]] == codes[s].tolist()
+    unused = np.setdiff1d(np.arange(N * k), slots.ravel())          # the masked slot's row
+    assert len(unused) == 1 and (recv[unused] == 0).all()
