@@ -115,6 +115,8 @@ def _declare(L):
     L.oracle_dispatch_e5m6.restype = _I
     L.oracle_dispatch_nvfp4.argtypes = [_P, _I, _I, _I, _P, _L64, _I, _P, _P, _P]
     L.oracle_dispatch_nvfp4.restype = _I
+    L.oracle_quant_fp8_channel.argtypes = [_P, _L64, _I, _I, _P, _P, _I, _P, _P]
+    L.oracle_quant_fp8_channel.restype = _I
     L.oracle_swiglu_quant.argtypes = [_P, _L64, _I, _P, _I, _I, _P, _P]
     L.oracle_swiglu_quant.restype = _I
     L.oracle_combine.argtypes = [_P, _L64, _I, _I, _I, _P, _P, _P]
@@ -361,6 +363,24 @@ def dispatch_nvfp4(x_bf16: np.ndarray, token_slot: np.ndarray, layout: int = SL_
     if st == ERR_INVALID_ARG:
         raise ValueError("oracle_dispatch_nvfp4: invalid argument")
     return recv, bs, rs, st
+
+
+def quant_fp8_channel(recv_bf16: np.ndarray, expert_offset: np.ndarray, expert_count: np.ndarray,
+                      transpose: bool = False):
+    """Per-(expert, channel) FP8 of the receive rows: (codes [S, H] or [H, S],
+    scales fp32 [E, H], status); rows outside the experts' landed ranges stay 0."""
+    recv_bf16 = _c(recv_bf16, np.uint16)
+    expert_offset = _c(expert_offset, np.int32)
+    expert_count = _c(expert_count, np.int32)
+    S, H = recv_bf16.shape
+    E = len(expert_count)
+    out = np.zeros((H, S) if transpose else (S, H), np.uint8)
+    scale = np.zeros((E, H), np.float32)
+    st = lib().oracle_quant_fp8_channel(_ptr(recv_bf16), S, H, E, _ptr(expert_offset), _ptr(expert_count),
+                                        int(transpose), _ptr(out), _ptr(scale))
+    if st == ERR_INVALID_ARG:
+        raise ValueError("oracle_quant_fp8_channel: invalid argument")
+    return out, scale, st
 
 
 def swiglu_quant(h_bf16: np.ndarray, slot_token: np.ndarray | None, dtype: int,

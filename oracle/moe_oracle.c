@@ -861,6 +861,50 @@ int oracle_dispatch_nvfp4(const uint16_t* x, int N, int H, int k, const int32_t*
 }
 
 /* ------------------------------------------------------------------ */
+/* Per-channel FP8 of the receive buffer.  [TK] lists FP8 quantisation "per
+ * channel" (and batched transposes) without a formula.  Reading: an
+ * expert's receive rows are the contracted dimension of its weight-gradient
+ * GEMM (dW_e = X_e^T dY_e), so one scale per (expert, channel) factors out
+ * of it.  Per expert e and channel c, over the rows
+ * s in [expert_offset[e], expert_offset[e] + expert_count[e]):
+ *   amax = max |x[s,c]|,  scale[e,c] = amax / 448,
+ *   code = e4m3(x[s,c] * (448 / amax))   (zeros keep their sign)
+ * -- the per-block FP8 rule with the block = one channel of one expert.
+ * Codes are written row-major [num_rows, H] or transposed [H, num_rows]
+ * (channel-major); rows outside every expert's landed range (padding of the
+ * aligned layout) are not written.                                      */
+/* ------------------------------------------------------------------ */
+int oracle_quant_fp8_channel(const uint16_t* x, int64_t num_rows, int H, int E,
+                             const int32_t* expert_offset, const int32_t* expert_count,
+                             int transpose, uint8_t* out, float* scale)
+{
+    if (num_rows < 0 || H < 1 || E < 1 || expert_offset[0] < 0 || expert_offset[E] > num_rows)
+        return ORC_ERR_INVALID_ARG;
+    for (int e = 0; e < E; ++e)
+        if (expert_count[e] < 0 || expert_offset[e] + expert_count[e] > expert_offset[e + 1])
+            return ORC_ERR_INVALID_ARG;
+    for (int e = 0; e < E; ++e) {
+        int64_t r0 = expert_offset[e], r1 = r0 + expert_count[e];
+        for (int c = 0; c < H; ++c) {
+            float amax = 0.0f;
+            for (int64_t s = r0; s < r1; ++s) {
+                float v = fabsf(oracle_f32_from_bf16(x[(size_t)s * H + c]));
+                if (v > amax) amax = v;
+            }
+            float inv = 448.0f / amax;
+            scale[(size_t)e * H + c] = amax / 448.0f;
+            for (int64_t s = r0; s < r1; ++s) {
+                float v = oracle_f32_from_bf16(x[(size_t)s * H + c]);
+                uint8_t q = oracle_e4m3_encode((v == 0.0f) ? v : v * inv);
+                if (transpose) out[(size_t)c * num_rows + s] = q;
+                else out[(size_t)s * H + c] = q;
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* SwiGLU fused with quantisation.  [TK] list: SwiGLU combined with the
  * quantisation operations.  Between an expert's two GEMMs the first one's
  * output row h = [gate | up] (bf16, 2I channels; reading: the gate half

@@ -73,6 +73,10 @@ MUTANTS = {
                        "    double m = floor(q + 0.5);\n    int biased = unb + 15;"),
     "e5m6_subnormal_step": ("double m = nearbyint(a * 1048576.0);", "double m = nearbyint(a * 524288.0);"),
     "e5m6_pack_overlaps": ("uint32_t w = c0 | (c1 << 12);", "uint32_t w = c0 | (c1 << 8);"),
+    "fp8_channel_amax_over_padded_block": ("int64_t r0 = expert_offset[e], r1 = r0 + expert_count[e];",
+                                           "int64_t r0 = expert_offset[e], r1 = expert_offset[e + 1];"),
+    "fp8_channel_transpose_index": ("if (transpose) out[(size_t)c * num_rows + s] = q;",
+                                    "if (transpose) out[(size_t)c * H + s] = q;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

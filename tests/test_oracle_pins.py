@@ -986,3 +986,50 @@ def test_dispatch_e5m6_packs_two_codes_in_three_bytes():
             assert [O.e5m6_encode(float(v)) for v in xf[t]] == codes[s].tolist()
     unused = np.setdiff1d(np.arange(N * k), slots.ravel())          # the masked slot's row
     assert len(unused) == 1 and (recv[unused] == 0).all()
+
+
+# ----------------------------------------------------------------- per-channel FP8
+def _channel_case(seed=0, align=16):
+    rng = np.random.default_rng(seed)
+    N, k, E, H = 120, 3, 10, 96
+    idx = rng.integers(0, E, (N, k)).astype(np.int32)
+    idx[rng.random((N, k)) < 0.1] = -1
+    idx[idx == 7] = -1                                   # an expert with no rows
+    rows = N * k + E * (align - 1)
+    L = O.get_layout_aligned(idx, E, 2, align, rows)
+    x = rng.normal(size=(rows, H)) * np.exp2(rng.integers(-10, 10, (1, H)))   # per-channel magnitudes
+    x[:, 5] = 0.0                                        # an all-zero channel
+    return _bf16(x), L, rows
+
+
+def test_fp8_channel_equals_per_token_rule_on_transposed_columns():
+    """Channel c of expert e, read as one 'token row' of the expert's landed rows
+    (zero-padded to a multiple of 8), quantised by the per-token FP8 dispatch:
+    the same codes and the same scale."""
+    x, L, rows = _channel_case()
+    codes, sc, st = O.quant_fp8_channel(x, L.expert_offset, L.expert_count)
+    assert st == 0
+    for e in range(len(L.expert_count)):
+        r0, n = int(L.expert_offset[e]), int(L.expert_count[e])
+        if n == 0:
+            assert (sc[e] == 0).all()
+            continue
+        cols = np.zeros((x.shape[1], -(-n // 8) * 8), np.uint16)
+        cols[:, :n] = x[r0:r0 + n].T
+        tq, ts, tst = O.dispatch(cols, np.arange(x.shape[1], dtype=np.int32)[:, None], O.DT_FP8_E4M3_TOKEN)
+        assert tst == 0
+        assert np.array_equal(codes[r0:r0 + n].T, tq[:, :n])
+        assert np.array_equal(sc[e].view(np.uint32), ts[:, 0].view(np.uint32))
+
+
+def test_fp8_channel_transposed_and_padding():
+    x, L, rows = _channel_case(3, align=32)
+    c0, s0, _ = O.quant_fp8_channel(x, L.expert_offset, L.expert_count)
+    c1, s1, st = O.quant_fp8_channel(x, L.expert_offset, L.expert_count, transpose=True)
+    assert st == 0 and np.array_equal(c1, c0.T) and np.array_equal(s0, s1)
+    landed = L.slot_token >= 0
+    assert (c0[~landed] == 0).all()                      # padding rows are not written
+    x2 = x.copy()
+    x2[~landed] = 0x7F80                                 # +inf in the padding must not matter
+    c2, s2, _ = O.quant_fp8_channel(x2, L.expert_offset, L.expert_count)
+    assert np.array_equal(c2, c0) and np.array_equal(s2, s0)
