@@ -438,10 +438,25 @@ def run_ours(args, rank, world, device):
             shape, sdt = api.scale_shape(w.S, w.H, code)
             bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
 
+        nv = None
+        if w.H % 64 == 0:
+            nv = (torch.empty((w.S, w.H // 2), dtype=torch.uint8, device=device),
+                  torch.empty((w.S, w.H // 16), dtype=torch.uint8, device=device),
+                  torch.empty((w.S,), dtype=torch.float32, device=device))
+
+        e5 = torch.empty((w.S, w.H // 2 * 3), dtype=torch.uint8, device=device) if w.H % 32 == 0 else None
+
         def var_ops():
-            return {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
-                                                                  d_status=L.status))
-                    for d, (c, rx, rs) in bufs.items()}
+            ops = {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
+                                                                 d_status=L.status))
+                   for d, (c, rx, rs) in bufs.items()}
+            if nv is not None:
+                ops["nvfp4"] = lambda: api.moe_dispatch_nvfp4(x, L.token_slot, recv_x=nv[0], block_scale=nv[1],
+                                                              row_scale=nv[2], d_status=L.status)
+            if e5 is not None:
+                ops["e5m6"] = lambda: api.moe_dispatch(x, L.token_slot, api.MOE_DTYPE_E5M6, recv_x=e5,
+                                                       d_status=L.status)
+            return ops
         vt = isolated_op_times(var_ops, flush, device)
         peak_v, _ = measured_peak()
         variants = {}
@@ -449,12 +464,13 @@ def run_ours(args, rank, world, device):
             abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": d}))["dispatch"]
             variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
                            "algorithmic_bytes": abv}
-        del bufs
+        del bufs, nv, e5
 
     aligned = None
     if not args.no_backward:
         # the GEMM-aligned layout (every expert's rows start at a multiple of
         # 128, one M tile) and the ops on its padded buffer, each alone
+        from combine_moe_topk_gate_b200.workloads import Workload
         A = 128
         rows_a = api.moe_aligned_recv_rows(w.N, w.k, w.E, A)
         La = api.Layout.empty(w.N, w.k, w.E, w.R, device, align=A)
@@ -465,25 +481,64 @@ def run_ours(args, rank, world, device):
         y_a = torch.empty((rows_a, w.H), dtype=torch.bfloat16, device=device).normal_()
         out_a = torch.empty_like(out)
 
+        # the same rows with the scales laid out for the grouped GEMM: MN-major
+        # (per-block FP8) and the block-scaled MMA's tiled E8M0 atoms (MXFP8)
+        gemm_scales = {}
+        if w.H % 128 == 0:
+            rx8 = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
+            for nm, dt, lay in (("dispatch_fp8_mn_major", api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR),
+                                ("dispatch_mxfp8_mma_tiled", api.MOE_DTYPE_MXFP8_E4M3, api.MOE_SCALE_MMA_TILED)):
+                shp, sdt = api.scale_shape(rows_a, w.H, dt, lay)
+                gemm_scales[nm] = (dt, lay, torch.empty(shp, dtype=sdt, device=device))
+
+        # SwiGLU + FP8 quantisation between the expert GEMMs, on the same padded
+        # rows: h = [gate | up] of the first GEMM (seeded, resident), I = the
+        # experts' intermediate width (2048 for the 7168-wide configs, 14336
+        # for Mixtral 8x7B)
+        inter = 14336 if w.name == "mixtral" else 2048
+        h_a = torch.empty((rows_a, 2 * inter), dtype=torch.bfloat16, device=device).normal_()
+        sw_out = torch.empty((rows_a, inter), dtype=torch.uint8, device=device)
+        shp, sdt = api.scale_shape(rows_a, inter, api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR)
+        sw_sc = torch.empty(shp, dtype=sdt, device=device)
+
+        # per-(expert, channel) FP8 of a bf16 receive buffer (the weight-gradient
+        # GEMM's operand); y_a doubles as that buffer
+        ch_out = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
+        ch_sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+
         def al_ops():
-            return {
+            ops = {
+                "quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
+                    y_a, La.expert_offset, La.expert_count, out=ch_out, scale=ch_sc, d_status=La.status),
+                "swiglu_fp8_mn_major": lambda: api.moe_swiglu_quant(
+                    h_a, api.MOE_DTYPE_FP8_E4M3, slot_token=La.slot_token, scale_layout=api.MOE_SCALE_MN_MAJOR,
+                    out=sw_out, out_scale=sw_sc),
                 "layout": lambda: api.moe_get_layout(idx, w.E, w.R, align=A, out=La),
                 "dispatch": lambda: api.moe_dispatch(x, La.token_slot, w.dtype_code, recv_x=rx_a,
                                                      recv_scale=rs_a, d_status=La.status),
                 "combine": lambda: api.moe_combine(y_a, La.token_slot, wts, out=out_a, d_status=La.status),
             }
+            for nm, (dt, lay, buf) in gemm_scales.items():
+                ops[nm] = (lambda dt=dt, lay=lay, buf=buf: api.moe_dispatch(
+                    x, La.token_slot, dt, recv_x=rx8, recv_scale=buf, scale_layout=lay, d_status=La.status))
+            return ops
         at = isolated_op_times(al_ops, flush, device)
         torch.cuda.synchronize(device)
         if int(La.status.item()) != 0:
             raise RuntimeError(f"device status {int(La.status.item())} after the aligned ops")
         peak_a, _ = measured_peak()
         ab_a = algorithmic_bytes(w)
+        landed = int((La.slot_token >= 0).sum().item())
+        ab_a["quant_fp8_channel"] = landed * w.H * 3 + 4 * w.E * w.H + 8 * w.E
+        ab_a["swiglu_fp8_mn_major"] = landed * (4 * inter + inter + 4 * (inter // 128)) + 4 * rows_a
+        ab_a["dispatch_fp8_mn_major"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "fp8"}))["dispatch"]
+        ab_a["dispatch_mxfp8_mma_tiled"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "mxfp8"}))["dispatch"]
         aligned = {"align": A, "recv_rows": rows_a,
-                   "padding_rows": int(rows_a - w.S),
+                   "padding_rows": int(rows_a - w.S), "swiglu_inter": inter, "landed_rows": landed,
                    **{n: {"us": us, "frac": (ab_a[n] / (us * 1e-6) / 1e9 / peak_a)
                           if us and n != "layout" else None}
                       for n, us in at.items()}}
-        del rx_a, rs_a, y_a, La
+        del rx_a, rs_a, y_a, La, gemm_scales, h_a, sw_out, sw_sc, ch_out, ch_sc
 
     e2e = None
     if not args.no_e2e:

@@ -20,9 +20,13 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX, MOE_ERR_TIMEOUT = range(6)
 MOE_GATE_SOFTMAX, MOE_GATE_SOFTMAX_RENORM, MOE_GATE_SIGMOID_GROUP = range(3)
-MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_TOKEN, MOE_DTYPE_MXFP8_E4M3 = range(4)
+(MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_TOKEN, MOE_DTYPE_MXFP8_E4M3, MOE_DTYPE_NVFP4,
+ MOE_DTYPE_E5M6) = range(6)
 MOE_MAX_EXPERTS = 1024
 MOE_MAX_ALIGN = 4096
+MOE_SCALE_ROW_MAJOR = 0
+MOE_SCALE_MN_MAJOR = 1
+MOE_SCALE_MMA_TILED = 2
 MOE_MAX_TOPK = 32
 MOE_FP8_BLOCK = 128
 
@@ -58,6 +62,16 @@ def _load() -> ctypes.CDLL:
     L.moe_scale_bytes.restype = SZ
     L.moe_dispatch.argtypes = [P, I, I, I, P, I, I, P, P, P, P]
     L.moe_dispatch.restype = I
+    L.moe_dispatch_ex.argtypes = [P, I, I, I, P, I, I, I, P, P, P, P]
+    L.moe_dispatch_ex.restype = I
+    L.moe_recv_scale_bytes.argtypes = [I, I, I, I]
+    L.moe_recv_scale_bytes.restype = SZ
+    L.moe_dispatch_nvfp4.argtypes = [P, I, I, I, P, I, I, P, P, P, P, P]
+    L.moe_dispatch_nvfp4.restype = I
+    L.moe_quant_fp8_channel.argtypes = [P, I, I, I, P, P, I, P, P, P, P]
+    L.moe_quant_fp8_channel.restype = I
+    L.moe_swiglu_quant.argtypes = [P, I, I, P, I, I, P, P, P]
+    L.moe_swiglu_quant.restype = I
     L.moe_combine.argtypes = [P, I, I, I, P, I, P, P, P, P]
     L.moe_combine.restype = I
     L.moe_dispatch_backward.argtypes = [P, I, I, I, P, I, P, P, P]
@@ -229,23 +243,43 @@ def moe_scale_bytes(num_tokens: int, hidden: int, k: int, dtype: int = MOE_DTYPE
     return int(_lib.moe_scale_bytes(num_tokens, hidden, k, dtype))
 
 
-def scale_shape(S: int, H: int, dtype: int):
-    """(shape, torch dtype) of recv_scale for a payload type (None for BF16)."""
+def moe_recv_scale_bytes(num_recv_rows: int, hidden: int, dtype: int, scale_layout: int) -> int:
+    return int(_lib.moe_recv_scale_bytes(num_recv_rows, hidden, dtype, scale_layout))
+
+
+def scale_shape(S: int, H: int, dtype: int, scale_layout: int = 0):
+    """(shape, torch dtype) of recv_scale for a payload type (None for BF16):
+    row-major [S, B]; MN-major [B, ld]; MMA-tiled flat bytes."""
+    if scale_layout != MOE_SCALE_ROW_MAJOR:
+        nbytes = moe_recv_scale_bytes(S, H, dtype, scale_layout)
+        if nbytes == 0:
+            return None, None
+        sdt = torch.uint8 if dtype in (MOE_DTYPE_MXFP8_E4M3, MOE_DTYPE_NVFP4) else torch.float32
+        if scale_layout == MOE_SCALE_MMA_TILED:
+            return (nbytes,), sdt
+        B = {MOE_DTYPE_FP8_E4M3: H // MOE_FP8_BLOCK, MOE_DTYPE_FP8_E4M3_TOKEN: 1,
+             MOE_DTYPE_MXFP8_E4M3: H // 32, MOE_DTYPE_NVFP4: H // 16}[dtype]
+        es = 1 if sdt == torch.uint8 else 4
+        return (B, nbytes // es // B), sdt
     if dtype == MOE_DTYPE_FP8_E4M3:
         return (S, H // MOE_FP8_BLOCK), torch.float32
     if dtype == MOE_DTYPE_FP8_E4M3_TOKEN:
         return (S, 1), torch.float32
     if dtype == MOE_DTYPE_MXFP8_E4M3:
         return (S, H // 32), torch.uint8
+    if dtype == MOE_DTYPE_NVFP4:
+        return (S, H // 16), torch.uint8
     return None, None
 
 
 def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_x=None,
-                 recv_scale=None, num_recv_rows: int | None = None, d_status=None, stream=None):
+                 recv_scale=None, num_recv_rows: int | None = None, scale_layout: int = 0,
+                 d_status=None, stream=None):
     """Scatter rows of ``x`` (bf16 [N,H]) to their receive rows.  Returns
-    ``(recv_x, recv_scale)``: bf16 [N*k,H] and None, or uint8 e4m3 codes
-    [N*k,H] with fp32 [N*k,H/128] (per block), fp32 [N*k,1] (per token) or
-    uint8 E8M0 bytes [N*k,H/32] (MXFP8)."""
+    ``(recv_x, recv_scale)``: bf16 [S,H] and None, or uint8 e4m3 codes
+    [S,H] with fp32 [S,H/128] (per block), fp32 [S,1] (per token) or
+    uint8 E8M0 bytes [S,H/32] (MXFP8), row-major; ``scale_layout`` selects
+    the MN-major or MMA-tiled scale layouts (moe_dispatch_ex)."""
     _need(x, "x", torch.bfloat16)
     N, H = x.shape
     _need(token_slot, "token_slot", torch.int32)
@@ -256,20 +290,110 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
             recv_x = torch.empty((S, H), dtype=torch.bfloat16, device=x.device)
         _need(recv_x, "recv_x", torch.bfloat16, (S, H))
         recv_scale = None
+    elif dtype == MOE_DTYPE_E5M6:
+        if recv_x is None:
+            recv_x = torch.empty((S, H // 2 * 3), dtype=torch.uint8, device=x.device)
+        _need(recv_x, "recv_x", torch.uint8, (S, H // 2 * 3))
+        recv_scale = None
     else:
-        shape, sdt = scale_shape(S, H, dtype)
+        shape, sdt = scale_shape(S, H, dtype, scale_layout)
         if shape is None:
-            raise ValueError(f"unknown dispatch dtype {dtype}")
+            raise ValueError(f"dispatch dtype {dtype} has no scale layout {scale_layout}")
         if recv_x is None:
             recv_x = torch.empty((S, H), dtype=torch.uint8, device=x.device)
         if recv_scale is None:
             recv_scale = torch.empty(shape, dtype=sdt, device=x.device)
         _need(recv_x, "recv_x", torch.uint8, (S, H))
         _need(recv_scale, "recv_scale", sdt, shape)
-    st = _lib.moe_dispatch(_ptr(x), N, H, k, _ptr(token_slot), S, dtype, _ptr(recv_x),
-                           _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
+    st = _lib.moe_dispatch_ex(_ptr(x), N, H, k, _ptr(token_slot), S, dtype, scale_layout,
+                              _ptr(recv_x), _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
     _check(st, "moe_dispatch")
     return recv_x, recv_scale
+
+
+def moe_dispatch_nvfp4(x: torch.Tensor, token_slot: torch.Tensor, *, scale_layout: int = 0,
+                       recv_x=None, block_scale=None, row_scale=None, num_recv_rows: int | None = None,
+                       d_status=None, stream=None):
+    """NVFP4 dispatch: returns ``(recv_x uint8 [S, H/2] (two e2m1 codes per
+    byte, even channel in the low nibble), block_scale (e4m3 codes, one per
+    16 channels, in ``scale_layout``), row_scale fp32 [S])``."""
+    _need(x, "x", torch.bfloat16)
+    N, H = x.shape
+    _need(token_slot, "token_slot", torch.int32)
+    k = token_slot.shape[1]
+    S = num_recv_rows if num_recv_rows is not None else (recv_x.shape[0] if recv_x is not None else N * k)
+    shape, _ = scale_shape(S, H, MOE_DTYPE_NVFP4, scale_layout)
+    if shape is None:
+        raise ValueError(f"NVFP4 has no scale layout {scale_layout} for hidden {H}")
+    if recv_x is None:
+        recv_x = torch.empty((S, H // 2), dtype=torch.uint8, device=x.device)
+    if block_scale is None:
+        block_scale = torch.empty(shape, dtype=torch.uint8, device=x.device)
+    if row_scale is None:
+        row_scale = torch.empty((S,), dtype=torch.float32, device=x.device)
+    _need(recv_x, "recv_x", torch.uint8, (S, H // 2))
+    _need(block_scale, "block_scale", torch.uint8, shape)
+    _need(row_scale, "row_scale", torch.float32, (S,))
+    st = _lib.moe_dispatch_nvfp4(_ptr(x), N, H, k, _ptr(token_slot), S, scale_layout, _ptr(recv_x),
+                                 _ptr(block_scale), _ptr(row_scale), _ptr(d_status), _stream(stream, x.device))
+    _check(st, "moe_dispatch_nvfp4")
+    return recv_x, block_scale, row_scale
+
+
+def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, expert_count: torch.Tensor, *,
+                          transpose: bool = False, out=None, scale=None, d_status=None, stream=None):
+    """Per-(expert, channel) FP8 of the receive rows ``recv`` (bf16 [S, H]) over
+    each expert's landed rows; returns ``(codes uint8 [S, H] or [H, S], scale
+    fp32 [E, H])``."""
+    _need(recv, "recv", torch.bfloat16)
+    S, H = recv.shape
+    _need(expert_count, "expert_count", torch.int32)
+    E = expert_count.numel()
+    _need(expert_offset, "expert_offset", torch.int32, (E + 1,))
+    shape = (H, S) if transpose else (S, H)
+    if out is None:
+        out = torch.empty(shape, dtype=torch.uint8, device=recv.device)
+    if scale is None:
+        scale = torch.empty((E, H), dtype=torch.float32, device=recv.device)
+    _need(out, "out", torch.uint8, shape)
+    _need(scale, "scale", torch.float32, (E, H))
+    st = _lib.moe_quant_fp8_channel(_ptr(recv), S, H, E, _ptr(expert_offset), _ptr(expert_count),
+                                    int(transpose), _ptr(out), _ptr(scale), _ptr(d_status),
+                                    _stream(stream, recv.device))
+    _check(st, "moe_quant_fp8_channel")
+    return out, scale
+
+
+def moe_swiglu_quant(h: torch.Tensor, dtype: int, *, slot_token=None, scale_layout: int = 0,
+                     out=None, out_scale=None, stream=None):
+    """a = silu(gate) * up for every row of ``h`` = [gate | up] (bf16 [S, 2I]),
+    stored as bf16 [S, I] or quantised like a dispatched row (e4m3 [S, I] plus
+    scales in ``scale_layout``).  Rows whose ``slot_token`` (int32 [S]) is
+    negative are skipped.  Returns ``(out, out_scale)``."""
+    _need(h, "h", torch.bfloat16)
+    S, I2 = h.shape
+    I = I2 // 2
+    if slot_token is not None:
+        _need(slot_token, "slot_token", torch.int32, (S,))
+    if dtype == MOE_DTYPE_BF16:
+        if out is None:
+            out = torch.empty((S, I), dtype=torch.bfloat16, device=h.device)
+        _need(out, "out", torch.bfloat16, (S, I))
+        out_scale = None
+    else:
+        shape, sdt = scale_shape(S, I, dtype, scale_layout)
+        if shape is None:
+            raise ValueError(f"swiglu dtype {dtype} has no scale layout {scale_layout}")
+        if out is None:
+            out = torch.empty((S, I), dtype=torch.uint8, device=h.device)
+        if out_scale is None:
+            out_scale = torch.empty(shape, dtype=sdt, device=h.device)
+        _need(out, "out", torch.uint8, (S, I))
+        _need(out_scale, "out_scale", sdt, shape)
+    st = _lib.moe_swiglu_quant(_ptr(h), S, I, _ptr(slot_token), dtype, scale_layout, _ptr(out),
+                               _ptr(out_scale), _stream(stream, h.device))
+    _check(st, "moe_swiglu_quant")
+    return out, out_scale
 
 
 def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor, *, out=None,

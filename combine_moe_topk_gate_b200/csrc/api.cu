@@ -22,7 +22,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 2; }
+int moe_abi_version(void) { return 3; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -117,7 +117,9 @@ moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k, int 
 
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
   if (num_tokens < 0 || hidden < 1 || k < 1) return 0;
-  const size_t esz = dtype == MOE_DTYPE_FP8_E4M3 ? 1 : 2;
+  const size_t esz = dtype == MOE_DTYPE_BF16 ? 2 : 1;
+  if (dtype == MOE_DTYPE_NVFP4) return static_cast<size_t>(num_tokens) * k * (hidden / 2);
+  if (dtype == MOE_DTYPE_E5M6) return static_cast<size_t>(num_tokens) * k * (hidden / 2 * 3);
   return static_cast<size_t>(num_tokens) * k * hidden * esz;
 }
 
@@ -128,16 +130,139 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
     case MOE_DTYPE_FP8_E4M3: return rows * (hidden / MOE_FP8_BLOCK) * sizeof(float);
     case MOE_DTYPE_FP8_E4M3_TOKEN: return rows * sizeof(float);
     case MOE_DTYPE_MXFP8_E4M3: return rows * (hidden / 32);
+    case MOE_DTYPE_NVFP4: return rows * (hidden / 16);  /* block scales; + 4 bytes per row */
     default: return 0;
   }
+}
+
+static int scale_blocks(int H, moe_dtype_t dtype) {
+  switch (dtype) {
+    case MOE_DTYPE_FP8_E4M3: return H / MOE_FP8_BLOCK;
+    case MOE_DTYPE_FP8_E4M3_TOKEN: return 1;
+    case MOE_DTYPE_MXFP8_E4M3: return H / 32;
+    case MOE_DTYPE_NVFP4: return H / 16;
+    default: return 0;
+  }
+}
+
+// whether `layout` is defined for the payload type (and its block count)
+static bool scale_layout_defined(int H, moe_dtype_t dtype, moe_scale_layout_t layout) {
+  if (layout == MOE_SCALE_ROW_MAJOR) return true;
+  if (dtype == MOE_DTYPE_BF16 || scale_blocks(H, dtype) < 1) return false;
+  if (layout == MOE_SCALE_MN_MAJOR) return true;
+  return layout == MOE_SCALE_MMA_TILED &&
+         (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) && scale_blocks(H, dtype) % 4 == 0;
+}
+
+size_t moe_recv_scale_bytes(int num_recv_rows, int hidden, moe_dtype_t dtype,
+                            moe_scale_layout_t layout) {
+  if (num_recv_rows < 0 || hidden < 1 || !scale_layout_defined(hidden, dtype, layout)) return 0;
+  const size_t B = static_cast<size_t>(scale_blocks(hidden, dtype));
+  const size_t es = (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) ? 1 : sizeof(float);
+  const size_t rows = static_cast<size_t>(num_recv_rows);
+  switch (layout) {
+    case MOE_SCALE_MN_MAJOR: return B * static_cast<size_t>(moe::scale_ld(num_recv_rows, dtype)) * es;
+    case MOE_SCALE_MMA_TILED: return (rows + 127) / 128 * 128 * B;
+    default: return rows * B * es;
+  }
+}
+
+moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,
+                                   const int32_t* expert_offset, const int32_t* expert_count,
+                                   int transpose, void* out, float* scale, int32_t* d_status,
+                                   moe_stream_t stream) {
+  if (num_rows < 0 || hidden < 1 || num_experts < 1) return MOE_ERR_INVALID_ARG;
+  if (hidden % 128 != 0 || (transpose != 0 && transpose != 1)) return MOE_ERR_INVALID_ARG;
+  if (num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
+  if (!expert_offset || !expert_count || !scale || (num_rows > 0 && (!recv || !out)))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(recv, 16) || !aligned(out, 4) || !aligned(scale, 4) || !aligned(expert_offset, 4) ||
+      !aligned(expert_count, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_quant_fp8_channel(recv, num_rows, hidden, num_experts, expert_offset,
+                                                 expert_count, transpose != 0, out, scale, d_status,
+                                                 as_stream(stream)));
+}
+
+moe_status_t moe_swiglu_quant(const void* h, int num_rows, int inter, const int32_t* slot_token,
+                              moe_dtype_t dtype, moe_scale_layout_t scale_layout, void* out,
+                              void* out_scale, moe_stream_t stream) {
+  if (num_rows < 0 || inter < 1) return MOE_ERR_INVALID_ARG;
+  if (scale_layout != MOE_SCALE_ROW_MAJOR && scale_layout != MOE_SCALE_MN_MAJOR &&
+      scale_layout != MOE_SCALE_MMA_TILED)
+    return MOE_ERR_INVALID_ARG;
+  switch (dtype) {
+    case MOE_DTYPE_BF16:
+      if (inter % 16 != 0) return MOE_ERR_INVALID_ARG;
+      break;
+    case MOE_DTYPE_FP8_E4M3:
+      if (inter % MOE_FP8_BLOCK != 0) return MOE_ERR_INVALID_ARG;
+      break;
+    case MOE_DTYPE_FP8_E4M3_TOKEN:
+      if (inter % 8 != 0) return MOE_ERR_INVALID_ARG;
+      if (inter > 16384) return MOE_ERR_UNSUPPORTED;
+      break;
+    case MOE_DTYPE_MXFP8_E4M3:
+      if (inter % 32 != 0) return MOE_ERR_INVALID_ARG;
+      break;
+    default:
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (!scale_layout_defined(inter, dtype, scale_layout)) return MOE_ERR_INVALID_ARG;
+  // one warp per (row, 512 channels), 8 warps per CTA: the grid must fit
+  if (static_cast<long long>(num_rows) * ((inter + 511) / 512) / 8 >= kMaxRows)
+    return MOE_ERR_UNSUPPORTED;
+  if (num_rows == 0) return MOE_OK;
+  if (!h || !out) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_BF16 && !out_scale) return MOE_ERR_INVALID_ARG;
+  const int scale_align =
+      (dtype == MOE_DTYPE_MXFP8_E4M3 || scale_layout != MOE_SCALE_ROW_MAJOR) ? 16 : 4;
+  if (!aligned(h, 16) || !aligned(out, 16) || !aligned(slot_token, 4)) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_BF16 && !aligned(out_scale, scale_align)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_swiglu_quant(h, num_rows, inter, slot_token, dtype, scale_layout,
+                                            out, out_scale, as_stream(stream)));
+}
+
+moe_status_t moe_dispatch_nvfp4(const void* x, int num_tokens, int hidden, int k,
+                                const int32_t* token_slot, int num_recv_rows,
+                                moe_scale_layout_t scale_layout, void* recv_x,
+                                void* recv_block_scale, float* recv_row_scale, int32_t* d_status,
+                                moe_stream_t stream) {
+  const int N = num_tokens, H = hidden;
+  if (N < 0 || H < 1 || k < 1 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (H % 64 != 0) return MOE_ERR_INVALID_ARG;
+  if (scale_layout != MOE_SCALE_ROW_MAJOR && scale_layout != MOE_SCALE_MN_MAJOR &&
+      scale_layout != MOE_SCALE_MMA_TILED)
+    return MOE_ERR_INVALID_ARG;
+  if (k > MOE_MAX_TOPK || H > 16384) return MOE_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  if (N == 0) return MOE_OK;
+  if (!x || !token_slot || !recv_x || !recv_block_scale || !recv_row_scale) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(recv_block_scale, 16) ||
+      !aligned(recv_row_scale, 4) || !aligned(token_slot, 4) || !aligned(d_status, 4))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_dispatch_nvfp4(x, N, H, k, token_slot, num_recv_rows, scale_layout,
+                                              recv_x, recv_block_scale, recv_row_scale, d_status,
+                                              as_stream(stream)));
 }
 
 moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
                           const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
                           void* recv_x, void* recv_scale, int32_t* d_status,
                           moe_stream_t stream) {
+  return moe_dispatch_ex(x, num_tokens, hidden, k, token_slot, num_recv_rows, dtype,
+                         MOE_SCALE_ROW_MAJOR, recv_x, recv_scale, d_status, stream);
+}
+
+moe_status_t moe_dispatch_ex(const void* x, int num_tokens, int hidden, int k,
+                             const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
+                             moe_scale_layout_t scale_layout, void* recv_x, void* recv_scale,
+                             int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
   if (N < 0 || H < 1 || k < 1 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
+  if (scale_layout != MOE_SCALE_ROW_MAJOR && scale_layout != MOE_SCALE_MN_MAJOR &&
+      scale_layout != MOE_SCALE_MMA_TILED)
+    return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
   if (dtype == MOE_DTYPE_BF16) {
@@ -149,18 +274,24 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
     if (H > 16384) return MOE_ERR_UNSUPPORTED;
   } else if (dtype == MOE_DTYPE_MXFP8_E4M3) {
     if (H % 32 != 0) return MOE_ERR_INVALID_ARG;
+  } else if (dtype == MOE_DTYPE_E5M6) {
+    if (H % 32 != 0) return MOE_ERR_INVALID_ARG;
   } else {
     return MOE_ERR_INVALID_ARG;
   }
+  if (!scale_layout_defined(H, dtype, scale_layout)) return MOE_ERR_INVALID_ARG;
   if (N == 0) return MOE_OK;
   if (!x || !token_slot || !recv_x) return MOE_ERR_INVALID_ARG;
-  if (dtype != MOE_DTYPE_BF16 && !recv_scale) return MOE_ERR_INVALID_ARG;
-  if (dtype != MOE_DTYPE_BF16 && !aligned(recv_scale, dtype == MOE_DTYPE_MXFP8_E4M3 ? 16 : 4))
-    return MOE_ERR_INVALID_ARG;
+  const bool scaled = dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_E5M6;
+  if (scaled && !recv_scale) return MOE_ERR_INVALID_ARG;
+  const int scale_align =
+      (dtype == MOE_DTYPE_MXFP8_E4M3 || scale_layout != MOE_SCALE_ROW_MAJOR) ? 16 : 4;
+  if (scaled && !aligned(recv_scale, scale_align)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(token_slot, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_dispatch(x, N, H, k, token_slot, num_recv_rows, dtype, recv_x,
-                                        recv_scale, d_status, as_stream(stream)));
+  return from_cuda(moe::launch_dispatch(x, N, H, k, token_slot, num_recv_rows, dtype,
+                                        scale_layout, recv_x, recv_scale, d_status,
+                                        as_stream(stream)));
 }
 
 moe_status_t moe_combine(const void* y, int num_tokens, int hidden, int k,

@@ -22,11 +22,12 @@ constexpr int kWarps = 8;
 
 // FP8: lane owns 16 channels (two 16-byte loads), 8 lanes = one 128-block,
 // a warp covers 512 channels.
+template <int SL>
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_fp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                         const int32_t* __restrict__ token_slot, long long S,
                         uint8_t* __restrict__ recv_x, float* __restrict__ recv_scale,
-                        int32_t* d_status) {
+                        long long ld, int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -82,7 +83,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     if (active) {
       st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
-      if ((lane & 7) == 0) recv_scale[static_cast<size_t>(slot) * nblk + (c0 >> 7)] = scale;
+      if ((lane & 7) == 0) recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
     }
   }
 }
@@ -92,17 +93,13 @@ __global__ void __launch_bounds__(kWarps * 32)
 // e4m3(x * 2^-e), saturating (x * 2^-e can reach 511.x).  Same work split as
 // the per-block kernel: lane owns 16 channels, 2 lanes = one block, a warp
 // covers 512 channels and gathers its 16 scale bytes into one 16-byte store.
-__device__ __forceinline__ int floor_log2_pos(float a) {  // a > 0, finite; exact
-  const uint32_t u = __float_as_uint(a);
-  const int ex = static_cast<int>((u >> 23) & 0xffu);
-  return ex ? ex - 127 : (31 - __clz(u & 0x7fffffu)) - 149;
-}
 
+template <int SL>
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_mxfp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                           const int32_t* __restrict__ token_slot, long long S,
                           uint8_t* __restrict__ recv_x, uint8_t* __restrict__ recv_e8m0,
-                          int32_t* d_status) {
+                          long long ld, int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
@@ -166,11 +163,24 @@ __global__ void __launch_bounds__(kWarps * 32)
       continue;
     }
     if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
-    uint8_t* srow = recv_e8m0 + static_cast<size_t>(slot) * nblk;
-    if (whole16) {
-      if (lane == 0) st_v4(srow + s * 16, make_uint4(sw[0], sw[1], sw[2], sw[3]));
-    } else if (active && (lane & 1) == 0) {
-      srow[c0 >> 5] = static_cast<uint8_t>(my_byte);
+    if constexpr (SL == MOE_SCALE_ROW_MAJOR) {
+      uint8_t* srow = recv_e8m0 + static_cast<size_t>(slot) * nblk;
+      if (whole16) {
+        if (lane == 0) st_v4(srow + s * 16, make_uint4(sw[0], sw[1], sw[2], sw[3]));
+      } else if (active && (lane & 1) == 0) {
+        srow[c0 >> 5] = static_cast<uint8_t>(my_byte);
+      }
+    } else if constexpr (SL == MOE_SCALE_MMA_TILED) {
+      // blocks 4i..4i+3 are 4 consecutive bytes of one atom (nblk % 4 == 0):
+      // lane i < 4 stores word i of the warp's 16 blocks
+      const int b0 = s * 16 + 4 * lane;
+      if (lane < 4 && b0 < nblk) {
+        const uint32_t word = lane == 0 ? sw[0] : lane == 1 ? sw[1] : lane == 2 ? sw[2] : sw[3];
+        *reinterpret_cast<uint32_t*>(recv_e8m0 + scale_at<SL>(slot, b0, nblk, ld)) = word;
+      }
+    } else {
+      if (active && (lane & 1) == 0)
+        recv_e8m0[scale_at<SL>(slot, c0 >> 5, nblk, ld)] = static_cast<uint8_t>(my_byte);
     }
   }
 }
@@ -246,6 +256,167 @@ __global__ void __launch_bounds__(kTokenThreads)
   }
 }
 
+// NVFP4: one CTA per token, one 16-channel block per thread vector (VPT per
+// thread).  Row amax over the CTA, then per block: sb = e4m3((amax_b / 6) *
+// (2688 / amax_row)), r = (2688 / amax_row) / value(sb), codes e2m1(x * r);
+// row scale g = amax_row / 2688.  Four neighbouring threads hold four
+// consecutive blocks, so their scale bytes go out as one 32-bit word
+// (H % 64 == 0).
+template <int VPT, int SL>
+__global__ void __launch_bounds__(kTokenThreads)
+    dispatch_nvfp4_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                          const int32_t* __restrict__ token_slot, long long S,
+                          uint8_t* __restrict__ recv_x, uint8_t* __restrict__ block_scale,
+                          float* __restrict__ row_scale, long long ld, int32_t* d_status) {
+  __shared__ float warp_max[kTokenThreads / 32];
+  __shared__ int slots[MOE_MAX_TOPK];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = blockIdx.x;
+  const int nvec = H / 16, B = H / 16;
+  pdl_wait();
+  pdl_trigger();
+  if (tid < k) {
+    const int sl = token_slot[static_cast<size_t>(t) * k + tid];
+    slots[tid] = sl;
+    if (sl < -1 || sl >= S) report_bad_index(d_status);
+  }
+  float f[VPT][16];
+  float bmax[VPT];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = i * kTokenThreads + tid;
+    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    if (vi < nvec) {
+      const uint16_t* src = x + static_cast<size_t>(t) * H + static_cast<size_t>(vi) * 16;
+      a = ld_stream(src);
+      b = ld_stream(src + 8);
+    }
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    bmax[i] = 0.0f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      f[i][2 * u] = bf16_lo(w[u]);
+      f[i][2 * u + 1] = bf16_hi(w[u]);
+      bmax[i] = fmaxf(bmax[i], fmaxf(fabsf(f[i][2 * u]), fabsf(f[i][2 * u + 1])));
+    }
+    amax = fmaxf(amax, bmax[i]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  amax = warp_max[0];
+#pragma unroll
+  for (int w2 = 1; w2 < kTokenThreads / 32; ++w2) amax = fmaxf(amax, warp_max[w2]);
+  const float g = __fdiv_rn(amax, 2688.0f);
+  const float inv = __fdiv_rn(2688.0f, amax);
+  uint2 q[VPT];
+  uint32_t sword[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const float sbf = __fmul_rn(__fdiv_rn(bmax[i], 6.0f), inv);
+    const uint32_t sb = bmax[i] > 0.0f ? (e4m3x2(sbf, 0.0f) & 0xffu) : 0u;
+    const float r = __fdiv_rn(inv, e4m3_value(sb));
+    float p[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) p[u] = (f[i][u] == 0.0f) ? f[i][u] : __fmul_rn(f[i][u], r);
+    q[i] = make_uint2(e2m1x8(p), e2m1x8(p + 8));
+    // bytes of blocks vi..vi+3 (threads lane..lane+3) into lane % 4 == 0
+    uint32_t word = sb;
+    word |= (__shfl_down_sync(kFullMask, sb, 1) & 0xffu) << 8;
+    word |= (__shfl_down_sync(kFullMask, sb, 2) & 0xffu) << 16;
+    word |= (__shfl_down_sync(kFullMask, sb, 3) & 0xffu) << 24;
+    sword[i] = SL == MOE_SCALE_MN_MAJOR ? sb : word;
+  }
+  for (int j = 0; j < k; ++j) {
+    const int slot = slots[j];
+    if (slot < 0 || slot >= S) continue;
+    uint8_t* row = recv_x + static_cast<size_t>(slot) * (H / 2);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = i * kTokenThreads + tid;
+      if (vi < nvec) {
+        *reinterpret_cast<uint2*>(row + static_cast<size_t>(vi) * 8) = q[i];
+        if constexpr (SL == MOE_SCALE_MN_MAJOR) {
+          block_scale[scale_at<SL>(slot, vi, B, ld)] = static_cast<uint8_t>(sword[i]);
+        } else if ((lane & 3) == 0) {
+          *reinterpret_cast<uint32_t*>(block_scale + scale_at<SL>(slot, vi, B, ld)) = sword[i];
+        }
+      }
+    }
+    if (tid == 0) row_scale[slot] = g;
+  }
+}
+
+// E5M6 (12-bit float: FP16 without its 4 lowest fraction bits), rounded to
+// nearest even, saturating to +-65024.  Normal range: rebias the fp32
+// exponent (127 -> 15) and round the fraction to 6 bits in the integer
+// domain; subnormals (|f| < 2^-14) in units of 2^-20, rounded by adding
+// 1.5 * 2^23 (the product |f| * 2^20 is exact and below 64).
+__device__ __forceinline__ uint32_t e5m6_code(float f) {
+  const uint32_t u = __float_as_uint(f);
+  const uint32_t sign = (u >> 20) & 0x800u;
+  const uint32_t a = u & 0x7fffffffu;
+  if (a > 0x7f800000u) return sign | 0x7ffu;  // NaN
+  if (a >= 0x38800000u) {
+    const uint32_t r = a - (112u << 23);
+    const uint32_t c = (r + 0xffffu + ((r >> 17) & 1u)) >> 17;
+    return sign | (c >= 0x7c0u ? 0x7bfu : c);
+  }
+  const float t = __fadd_rn(__fmul_rn(__uint_as_float(a), 0x1p20f), 12582912.0f);
+  return sign | (__float_as_uint(t) - 0x4B400000u);
+}
+
+// E5M6 dispatch: lane owns 16 channels (two 16-byte loads) -> 16 codes ->
+// 24 bytes (two codes per 3 bytes, little endian), stored as three 8-byte
+// streaming stores; a warp writes 768 contiguous bytes of each receive row.
+__global__ void __launch_bounds__(kWarps * 32)
+    dispatch_e5m6_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
+                         const int32_t* __restrict__ token_slot, long long S,
+                         uint8_t* __restrict__ recv_x, int32_t* d_status) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (H + 511) / 512;
+  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (item >= static_cast<long long>(N) * segs) return;
+  const int t = static_cast<int>(item / segs);
+  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
+  const int c0 = s * 512 + lane * 16;
+  const bool active = c0 < H;  // H % 32 == 0: 16 whole channels or none
+  pdl_wait();
+  pdl_trigger();
+  const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
+  uint4 a = make_uint4(0, 0, 0, 0), b = a;
+  if (active) {
+    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
+    a = ld_stream(src);
+    b = ld_stream(src + 8);
+  }
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t p[8];  // 24-bit pairs
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = e5m6_code(bf16_lo(w[i])) | (e5m6_code(bf16_hi(w[i])) << 12);
+  const uint2 o0 = make_uint2(p[0] | (p[1] << 24), (p[1] >> 8) | (p[2] << 16));
+  const uint2 o1 = make_uint2((p[2] >> 16) | (p[3] << 8), p[4] | (p[5] << 24));
+  const uint2 o2 = make_uint2((p[5] >> 8) | (p[6] << 16), (p[6] >> 16) | (p[7] << 8));
+  const size_t row_bytes = static_cast<size_t>(H) / 2 * 3;
+  for (int j = 0; j < k; ++j) {
+    const int slot = __shfl_sync(kFullMask, my_slot, j);
+    if (slot == -1) continue;
+    if (slot < -1 || slot >= S) {
+      if (lane == 0) report_bad_index(d_status);
+      continue;
+    }
+    if (active) {
+      uint2* dst = reinterpret_cast<uint2*>(recv_x + static_cast<size_t>(slot) * row_bytes +
+                                            static_cast<size_t>(c0) / 2 * 3);
+      __stcs(dst, o0);
+      __stcs(dst + 1, o1);
+      __stcs(dst + 2, o2);
+    }
+  }
+}
+
 // BF16: lane owns 8 channels (one 16-byte vector), a warp covers 256 channels.
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_bf16_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
@@ -290,20 +461,39 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
 
 }  // namespace
 
+long long scale_ld(long long num_rows, int dtype) {
+  const long long per16 =
+      (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) ? 16 : 4;  // scales per 16 bytes
+  return (num_rows + per16 - 1) / per16 * per16;
+}
+
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            long long num_rows, int dtype, void* recv_x, void* recv_scale,
-                            int32_t* d_status, cudaStream_t stream) {
+                            long long num_rows, int dtype, int scale_layout, void* recv_x,
+                            void* recv_scale, int32_t* d_status, cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* r8 = static_cast<uint8_t*>(recv_x);
+  const long long ld = scale_ld(num_rows, dtype);
   if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3) {
     const long long items = static_cast<long long>(N) * ((H + 511) / 512);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-    if (dtype == MOE_DTYPE_FP8_E4M3)
-      return launch_pdl(dispatch_fp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
-                        token_slot, num_rows, r8, static_cast<float*>(recv_scale), d_status);
-    return launch_pdl(dispatch_mxfp8_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k,
-                      token_slot, num_rows, r8, static_cast<uint8_t*>(recv_scale), d_status);
+    float* f32 = static_cast<float*>(recv_scale);
+    uint8_t* e8 = static_cast<uint8_t*>(recv_scale);
+    if (dtype == MOE_DTYPE_FP8_E4M3) {
+      if (scale_layout == MOE_SCALE_MN_MAJOR)
+        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,
+                          xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+      return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_ROW_MAJOR>, blocks, kWarps * 32, 0, stream,
+                        xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+    }
+    if (scale_layout == MOE_SCALE_MN_MAJOR)
+      return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,
+                        xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
+    if (scale_layout == MOE_SCALE_MMA_TILED)
+      return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_MMA_TILED>, blocks, kWarps * 32, 0, stream,
+                        xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
+    return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_ROW_MAJOR>, blocks, kWarps * 32, 0, stream,
+                      xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
   } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
     const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
     float* sc = static_cast<float*>(recv_scale);
@@ -318,6 +508,11 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
                         token_slot, num_rows, r8, sc, d_status);
     return launch_pdl(dispatch_fp8_token_kernel<8>, N, kTokenThreads, 0, stream, xs, N, H, k,
                       token_slot, num_rows, r8, sc, d_status);
+  } else if (dtype == MOE_DTYPE_E5M6) {
+    const long long items = static_cast<long long>(N) * ((H + 511) / 512);
+    const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+    return launch_pdl(dispatch_e5m6_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
+                      num_rows, r8, d_status);
   } else {
     const long long items = static_cast<long long>(N) * ((H + 255) / 256);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
@@ -325,6 +520,40 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
                       static_cast<const uint16_t*>(x), N, H, k, token_slot, num_rows,
                       static_cast<uint16_t*>(recv_x), d_status);
   }
+}
+
+template <int SL>
+cudaError_t launch_nvfp4(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                         long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
+                         float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
+  const int vpt = (H / 16 + kTokenThreads - 1) / kTokenThreads;
+  if (vpt <= 1)
+    return launch_pdl(dispatch_nvfp4_kernel<1, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
+                      token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
+  if (vpt <= 2)
+    return launch_pdl(dispatch_nvfp4_kernel<2, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
+                      token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
+  return launch_pdl(dispatch_nvfp4_kernel<4, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
+                    token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
+}
+
+cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int32_t* token_slot,
+                                  long long num_rows, int scale_layout, void* recv_x,
+                                  void* block_scale, float* row_scale, int32_t* d_status,
+                                  cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  uint8_t* r8 = static_cast<uint8_t*>(recv_x);
+  uint8_t* bs = static_cast<uint8_t*>(block_scale);
+  const long long ld = scale_ld(num_rows, MOE_DTYPE_NVFP4);
+  if (scale_layout == MOE_SCALE_MN_MAJOR)
+    return launch_nvfp4<MOE_SCALE_MN_MAJOR>(xs, N, H, k, token_slot, num_rows, r8, bs, row_scale,
+                                            ld, d_status, stream);
+  if (scale_layout == MOE_SCALE_MMA_TILED)
+    return launch_nvfp4<MOE_SCALE_MMA_TILED>(xs, N, H, k, token_slot, num_rows, r8, bs, row_scale,
+                                             ld, d_status, stream);
+  return launch_nvfp4<MOE_SCALE_ROW_MAJOR>(xs, N, H, k, token_slot, num_rows, r8, bs, row_scale,
+                                           ld, d_status, stream);
 }
 
 cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream) {

@@ -21,6 +21,9 @@ constexpr unsigned kFullMask = 0xffffffffu;
 // two fused steps (ln2 = head + tail, head = floor(ln2 * 2^16) / 2^16 so that
 // n*head is exact), e^r by its Taylor series to r^7/7! (Horner), 2^n built
 // from the exponent field.  y is clamped to [-87, 88] so 2^n stays normal.
+// The nearest integer (ties to even) comes from adding 1.5 * 2^23: the sum's
+// unit in the last place is 1, so the addition itself rounds y*log2(e) to an
+// integer, which then sits in the low mantissa bits (|y*log2(e)| <= 127).
 __device__ __forceinline__ float fixed_exp(float y) {
   constexpr float kLog2e = 1.44269504088896340736f;
   constexpr float kLn2Head = 0.693145751953125f;          // 45426 / 65536
@@ -28,8 +31,10 @@ __device__ __forceinline__ float fixed_exp(float y) {
   constexpr float kInv2 = 0.5f, kInv6 = 1.0f / 6.0f, kInv24 = 1.0f / 24.0f;
   constexpr float kInv120 = 1.0f / 120.0f, kInv720 = 1.0f / 720.0f;
   constexpr float kInv5040 = 1.0f / 5040.0f;
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   y = fminf(fmaxf(y, -87.0f), 88.0f);
-  const float n = rintf(__fmul_rn(y, kLog2e));
+  const float t = __fadd_rn(__fmul_rn(y, kLog2e), kRound);
+  const float n = __fsub_rn(t, kRound);
   float r = __fmaf_rn(-n, kLn2Head, y);
   r = __fmaf_rn(-n, kLn2Tail, r);
   float p = kInv5040;
@@ -40,7 +45,7 @@ __device__ __forceinline__ float fixed_exp(float y) {
   p = __fmaf_rn(p, r, kInv2);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  const float two_n = __int_as_float((static_cast<int>(n) + 127) << 23);
+  const float two_n = __int_as_float((__float_as_int(t) - 0x4B400000 + 127) << 23);
   return __fmul_rn(p, two_n);
 }
 
@@ -75,6 +80,69 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
   if (nan_lo) v = (v & 0xff00u) | ((__float_as_uint(lo) >> 24) & 0x80u) | 0x7fu;
   if (nan_hi) v = (v & 0x00ffu) | ((((__float_as_uint(hi) >> 24) & 0x80u) | 0x7fu) << 8);
   return v;
+}
+
+// ---------------------------------------------------------------- scales
+// floor(log2(a)) for a > 0 finite, exact from the bits (subnormals too)
+__device__ __forceinline__ int floor_log2_pos(float a) {  // a > 0, finite; exact
+  const uint32_t u = __float_as_uint(a);
+  const int ex = static_cast<int>((u >> 23) & 0xffu);
+  return ex ? ex - 127 : (31 - __clz(u & 0x7fffffu)) - 149;
+}
+
+// Receive-scale layouts (moe_scale_layout_t): element of scale (row s, block b)
+// for B blocks per row.  MN-major: column b is contiguous over the rows with
+// leading dimension ld (the row count padded to 16 bytes).  MMA-tiled (E8M0):
+// 128-row x 4-block atoms of 512 bytes, row-major over atoms, row s / block b
+// at byte (s % 32) * 16 + ((s % 128) / 32) * 4 + b % 4 inside the atom -- the
+// order the block-scaled tensor-core MMA takes scale factors in.
+template <int SL>
+__device__ __forceinline__ size_t scale_at(long long s, int b, int B, long long ld) {
+  if constexpr (SL == MOE_SCALE_MN_MAJOR) {
+    return static_cast<size_t>(b) * ld + s;
+  } else if constexpr (SL == MOE_SCALE_MMA_TILED) {
+    const size_t atom = static_cast<size_t>(s >> 7) * (B >> 2) + (b >> 2);
+    return atom * 512 + (s & 31) * 16 + ((s >> 5) & 3) * 4 + (b & 3);
+  } else {
+    return static_cast<size_t>(s) * B + b;
+  }
+}
+
+// e4m3x2 for inputs that are never NaN (the codes of finite values and of
+// +-infinity equal e4m3x2's; a NaN input gives an unspecified code).
+__device__ __forceinline__ uint32_t e4m3x2_nonan(float lo, float hi) {
+  const float clo = fminf(fmaxf(lo, -448.0f), 448.0f);
+  const float chi = fminf(fmaxf(hi, -448.0f), 448.0f);
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(chi), "f"(clo));
+  return r;
+}
+
+// ---------------------------------------------------------------- e2m1
+// Eight floats -> eight FP4 E2M1 codes packed in a word, value i in bits
+// 4i..4i+3 (so the even channel of each byte sits in its low nibble).  Round
+// to nearest even; values beyond +-6 (infinities too) are clamped to +-6
+// first.  cvt puts its first source in the upper nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float* p) {
+  float c[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) c[i] = fminf(fmaxf(p[i], -6.0f), 6.0f);
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(c[0]), "f"(c[1]), "f"(c[2]), "f"(c[3]), "f"(c[4]), "f"(c[5]), "f"(c[6]), "f"(c[7]));
+  return r;
+}
+
+// value of a non-negative e4m3 code (no NaN), exact
+__device__ __forceinline__ float e4m3_value(uint32_t c) {
+  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : __fmul_rn(static_cast<float>(m), 0x1p-9f);
 }
 
 // ---------------------------------------------------------------- memory

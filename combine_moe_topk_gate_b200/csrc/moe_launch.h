@@ -23,8 +23,21 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
 // num_rows: rows of the receive buffer (N*k packed, more for aligned layouts);
 // slots outside [-1, num_rows) are skipped and reported.
 cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* token_slot,
-                            long long num_rows, int dtype, void* recv_x, void* recv_scale,
-                            int32_t* d_status, cudaStream_t stream);
+                            long long num_rows, int dtype, int scale_layout, void* recv_x,
+                            void* recv_scale, int32_t* d_status, cudaStream_t stream);
+// leading dimension of MN-major scales: num_rows padded to 16 bytes of scales
+long long scale_ld(long long num_rows, int dtype);
+cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int32_t* token_slot,
+                                  long long num_rows, int scale_layout, void* recv_x,
+                                  void* block_scale, float* row_scale, int32_t* d_status,
+                                  cudaStream_t stream);
+cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, int E,
+                                     const int32_t* expert_offset, const int32_t* expert_count,
+                                     bool transpose, void* out, float* scale, int32_t* d_status,
+                                     cudaStream_t stream);
+cudaError_t launch_swiglu_quant(const void* h, long long num_rows, int I, const int32_t* slot_token,
+                                int dtype, int scale_layout, void* out, void* out_scale,
+                                cudaStream_t stream);
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
                            long long num_rows, const float* topk_w, void* out, int32_t* d_status,

@@ -121,13 +121,13 @@ def algorithmic_bytes(w: Workload) -> dict:
     """Bytes each step must move at least once (each token row read once,
     written k times; int32 metadata of the step included)."""
     N, H, E, k = w.N, w.H, w.E, w.k
-    b = 2 if w.dtype == "bf16" else 1
+    row = {"bf16": 2 * H, "nvfp4": H // 2, "e5m6": H // 2 * 3}.get(w.dtype, H)   # payload bytes of a receive row
     scales = {"fp8": 4 * N * k * (H // 128), "fp8_token": 4 * N * k,
-              "mxfp8": N * k * (H // 32)}.get(w.dtype, 0)
+              "mxfp8": N * k * (H // 32), "nvfp4": N * k * (H // 16) + 4 * N * k}.get(w.dtype, 0)
     return {
         "gate": 4 * N * E + 8 * N * k,
         "layout": 4 * N * k + 8 * N * k + 4 * (4 * E + 3 * w.R),
-        "dispatch": 2 * N * H + N * k * H * b + scales + 4 * N * k,
+        "dispatch": 2 * N * H + N * k * row + scales + 4 * N * k,
         "combine": 2 * N * k * H + 2 * N * H + 8 * N * k,
         # backward: gradient rows in, token gradient out (dispatch); token
         # gradient + expert rows in, scaled rows + weight gradients out (combine)

@@ -72,8 +72,19 @@ typedef enum {
     MOE_DTYPE_BF16 = 0,          /* payload copied as bf16                              */
     MOE_DTYPE_FP8_E4M3 = 1,      /* e4m3, one fp32 scale per 128 channels               */
     MOE_DTYPE_FP8_E4M3_TOKEN = 2,/* e4m3, one fp32 scale per token row                  */
-    MOE_DTYPE_MXFP8_E4M3 = 3     /* OCP MXFP8: e4m3, one E8M0 scale byte per 32 channels */
+    MOE_DTYPE_MXFP8_E4M3 = 3,    /* OCP MXFP8: e4m3, one E8M0 scale byte per 32 channels */
+    MOE_DTYPE_NVFP4 = 4,         /* e2m1, one e4m3 scale per 16 channels + fp32 per row  */
+    MOE_DTYPE_E5M6 = 5           /* 12-bit float (FP16 minus 4 fraction bits), no scale  */
 } moe_dtype_t;
+
+/* Where the receive scales go (moe_dispatch_ex).  Scale (s, b) is that of
+ * receive row s and scale block b; a row has B blocks (H/128 per-block FP8,
+ * 1 per-token FP8, H/32 MXFP8). */
+typedef enum {
+    MOE_SCALE_ROW_MAJOR = 0,     /* element s*B + b                                      */
+    MOE_SCALE_MN_MAJOR = 1,      /* element b*ld + s, ld = S padded to 16 bytes of scales */
+    MOE_SCALE_MMA_TILED = 2      /* E8M0 only: block-scaled MMA scale-factor atoms        */
+} moe_scale_layout_t;
 
 typedef void* moe_stream_t;      /* a cudaStream_t */
 
@@ -243,6 +254,12 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
  *          codes e4m3_rne_satfinite(x * 2^-e) (the power-of-two scaling is
  *          exact; values up to 511.x saturate to 448).  H % 32 == 0;
  *          recv_scale 16-byte aligned.
+ *   E5M6 ([TK]: E5M6 conversion; the format is not defined there, reading:
+ *          IEEE-style 1-5-6 bits, bias 15, i.e. FP16 with its 4 lowest
+ *          fraction bits dropped; round to nearest even, saturating to
+ *          +-65024): recv_x uint8 [S, 3H/2], two 12-bit codes per 3 bytes
+ *          (code 2i in bits 0..11 of the little-endian 24-bit group);
+ *          recv_scale unused.  H % 32 == 0.
  *   Rows no slot names are not written.  A slot outside [-1, S) is skipped
  *   and reported through d_status.
  */
@@ -250,6 +267,118 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
                           const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
                           void* recv_x, void* recv_scale, int32_t* d_status,
                           moe_stream_t stream);
+
+/*
+ * moe_dispatch_ex -- moe_dispatch with the receive scales laid out for the
+ * grouped GEMM that consumes them.  [EPv2] ElasticBuffer interface names a
+ * new GEMM layout without defining it and [TK] lists batched transposes;
+ * the reading taken is one of three places for the same values:
+ *   MOE_SCALE_ROW_MAJOR  as moe_dispatch.
+ *   MOE_SCALE_MN_MAJOR   per-block FP8, per-token FP8 or MXFP8: scale (s, b)
+ *        at element b*ld + s with ld = S rounded up to 4 (fp32) or 16 (E8M0):
+ *        each block's scales are contiguous over the rows, every column
+ *        16-byte aligned -- the transposed (M-major) scale operand of a
+ *        grouped GEMM.
+ *   MOE_SCALE_MMA_TILED  MXFP8 with H % 128 == 0: the order in which the
+ *        block-scaled tensor-core MMA takes scale factors.  Rows are padded
+ *        to a multiple of 128; 128-row x 4-block atoms of 512 bytes follow
+ *        each other row-major over (s/128, b/4); inside an atom, row s and
+ *        block b sit at byte (s%32)*16 + ((s%128)/32)*4 + b%4.  With the
+ *        aligned layout at align 128 every expert's scales are a contiguous
+ *        run of whole atoms.
+ *   recv_scale holds moe_recv_scale_bytes(S, H, dtype, scale_layout) bytes,
+ *   16-byte aligned for the MN-major and tiled layouts.  Only positions of
+ *   rows a token lands in are written.  A layout the payload type does not
+ *   have (BF16 with any but row-major, per-block FP8 tiled) is
+ *   MOE_ERR_INVALID_ARG.  Everything else is as in moe_dispatch.
+ */
+moe_status_t moe_dispatch_ex(const void* x, int num_tokens, int hidden, int k,
+                             const int32_t* token_slot, int num_recv_rows, moe_dtype_t dtype,
+                             moe_scale_layout_t scale_layout, void* recv_x, void* recv_scale,
+                             int32_t* d_status, moe_stream_t stream);
+
+/* Bytes of recv_scale for S receive rows in `scale_layout`; 0 for BF16 and
+ * for a layout the payload type does not have. */
+size_t moe_recv_scale_bytes(int num_recv_rows, int hidden, moe_dtype_t dtype,
+                            moe_scale_layout_t scale_layout);
+
+/*
+ * moe_dispatch_nvfp4 -- moe_dispatch with an NVFP4 payload, the FP4 format of
+ * Blackwell's block-scaled tensor-core MMA.  [EPv2] feature list (Hybrid-EP:
+ * NVFP4 support) and [TK] (FP4 conversion) name the format without a rule;
+ * the reading is two-level NVFP4 scaling with the token's row in place of
+ * the tensor (the per-token mode of [TK]).  Per token t:
+ *   amax_t = max |x[t,:]|, row scale g_t = amax_t / 2688 (= 448 * 6),
+ *   inv_t = 2688 / amax_t; per block b of 16 channels:
+ *   sb = e4m3((amax_b / 6) * inv_t) (0 for an all-zero block),
+ *   codes e2m1(x * (inv_t / value(sb))), round to nearest even, saturating
+ *   to +-6; zeros keep their sign.  Every operation is fp32, rounded once;
+ *   x ~ e2m1 * value(sb) * g_t.
+ *   recv_x            uint8 [S, H/2]: two codes per byte, channel 2i in the
+ *                     low nibble (the operand order of FP4 MMA).
+ *   recv_block_scale  e4m3 codes, one per 16 channels, in scale_layout
+ *                     (moe_recv_scale_bytes(S, H, MOE_DTYPE_NVFP4, layout)
+ *                     bytes); the tiled layout is the FP4 block-scaled MMA's.
+ *   recv_row_scale    fp32 [S]: g of the token in each row.
+ *   Limits: H % 64 == 0, H <= 16384; x, recv_x, recv_block_scale 16-byte
+ *   aligned.  Slots, masks and errors as in moe_dispatch.
+ */
+moe_status_t moe_dispatch_nvfp4(const void* x, int num_tokens, int hidden, int k,
+                                const int32_t* token_slot, int num_recv_rows,
+                                moe_scale_layout_t scale_layout, void* recv_x,
+                                void* recv_block_scale, float* recv_row_scale, int32_t* d_status,
+                                moe_stream_t stream);
+
+/*
+ * moe_quant_fp8_channel -- per-(expert, channel) FP8 of the receive buffer,
+ * for each expert's weight-gradient GEMM.  [TK] list: FP8 quantisation "pro
+ * Kanal" and batched transposes, no formula; reading: an expert's rows are
+ * the contracted dimension of dW_e = X_e^T dY_e, so one scale per (expert,
+ * channel) factors out of it.  Per expert e and channel c over the landed
+ * rows [expert_offset[e], expert_offset[e] + expert_count[e]):
+ *   amax = max |x|, scale[e*H + c] = amax / 448,
+ *   code = e4m3(x * (448 / amax)) (fp32, rounded once each; zeros keep
+ *   their sign) -- the per-block rule with the block = one channel of one
+ *   expert.
+ *   recv           bf16 [S, H] in (S = num_rows), 16-byte aligned.
+ *   expert_offset  int32 [E+1], expert_count int32 [E]: device arrays, e.g.
+ *                  from moe_get_layout_aligned; an expert whose range leaves
+ *                  [0, S) is skipped and reported through d_status.
+ *   transpose      0: out e4m3 [S, H] row-major; 1: out e4m3 [H, S]
+ *                  (channel-major, the K-major operand).
+ *   scale          fp32 [E, H] out (0 for an expert with no rows).
+ *   Padding rows (outside every expert's landed range) are not written.
+ *   H % 128 == 0, 1 <= E <= MOE_MAX_EXPERTS.
+ */
+moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,
+                                   const int32_t* expert_offset, const int32_t* expert_count,
+                                   int transpose, void* out, float* scale, int32_t* d_status,
+                                   moe_stream_t stream);
+
+/*
+ * moe_swiglu_quant -- SwiGLU between an expert's two GEMMs, fused with the
+ * quantisation the second GEMM reads.  [TK] list: SwiGLU combined with the
+ * quantisation operations (the formula is not on the pages; reading below).
+ *   h           bf16 [S, 2I] in: row s = [gate | up], the first GEMM's output
+ *               for receive row s (gate half first).
+ *   slot_token  int32 [S] from moe_get_layout(_aligned), or NULL: rows with
+ *               slot_token < 0 (padding) are skipped and their outputs left
+ *               as they were.
+ *   a_c = silu(g_c) * u_c with silu(g) = g / (1 + exp(-g)), in fp32 with
+ *   every operation rounded once and exp the gate's fixed routine.
+ *   out / out_scale: a as bf16 [S, I] (dtype BF16, out_scale unused), or
+ *   e4m3 [S, I] with scales exactly as moe_dispatch_ex produces them from a
+ *   row (per-128-block FP8, per-row FP8, MXFP8) with the fp32 a in place of
+ *   the bf16 input, in `scale_layout` over S rows (moe_recv_scale_bytes(S,
+ *   I, dtype, scale_layout) bytes).
+ *   Limits: I % 16 == 0 (BF16), % 128 (FP8 per block), % 8 and <= 16384
+ *   (per row), % 32 (MXFP8; % 128 for the tiled scales); h and out 16-byte
+ *   aligned; out_scale aligned as in moe_dispatch_ex.  S == 0 enqueues
+ *   nothing.
+ */
+moe_status_t moe_swiglu_quant(const void* h, int num_rows, int inter, const int32_t* slot_token,
+                              moe_dtype_t dtype, moe_scale_layout_t scale_layout, void* out,
+                              void* out_scale, moe_stream_t stream);
 
 /*
  * moe_combine -- weighted gather-reduce of each token's k expert outputs.

@@ -125,7 +125,7 @@ def test_dispatch_combine_reject_bad_arguments(api):
     assert disp(_P(), 10, 100, 2, BF16, _P(), None) == api.MOE_ERR_INVALID_ARG
     assert disp(_P(), 10, 256, 2, FP8, _P(), None) == api.MOE_ERR_INVALID_ARG
     assert disp(_P(0x1008), 10, 256, 2, BF16, _P(), None) == api.MOE_ERR_INVALID_ARG
-    assert disp(_P(), 10, 256, 2, 5, _P(), None) == api.MOE_ERR_INVALID_ARG
+    assert disp(_P(), 10, 256, 2, 9, _P(), None) == api.MOE_ERR_INVALID_ARG
     MX, TOK = api.MOE_DTYPE_MXFP8_E4M3, api.MOE_DTYPE_FP8_E4M3_TOKEN
     assert disp(_P(), 10, 272, 2, MX, _P(), _P()) == api.MOE_ERR_INVALID_ARG  # H % 32
     assert disp(_P(), 10, 256, 2, MX, _P(), _P(0x1008)) == api.MOE_ERR_INVALID_ARG  # scales 16-B
@@ -150,3 +150,109 @@ def test_dispatch_combine_reject_bad_arguments(api):
         == api.MOE_ERR_INVALID_ARG
     assert L.moe_e4m3_encode(None, 0, None, None) == api.MOE_OK
     assert L.moe_e4m3_encode(None, 5, _P(), None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_scale_layout_sizes_and_validation(api):
+    L = api.lib()
+    FP8, TOK, MX, BF16 = (api.MOE_DTYPE_FP8_E4M3, api.MOE_DTYPE_FP8_E4M3_TOKEN,
+                          api.MOE_DTYPE_MXFP8_E4M3, api.MOE_DTYPE_BF16)
+    ROW, MN, TILED = api.MOE_SCALE_ROW_MAJOR, api.MOE_SCALE_MN_MAJOR, api.MOE_SCALE_MMA_TILED
+    # payload bytes: every e4m3 payload is one byte per element
+    for dt in (FP8, TOK, MX):
+        assert api.moe_recv_bytes(10, 256, 2, dt) == 10 * 2 * 256
+    assert api.moe_recv_scale_bytes(10, 256, FP8, ROW) == 10 * 2 * 4
+    assert api.moe_recv_scale_bytes(10, 256, FP8, MN) == 2 * 12 * 4        # ld = 12 (16 bytes)
+    assert api.moe_recv_scale_bytes(10, 256, TOK, MN) == 12 * 4
+    assert api.moe_recv_scale_bytes(10, 256, MX, MN) == 8 * 16              # ld = 16 bytes
+    assert api.moe_recv_scale_bytes(300, 256, MX, TILED) == 384 * 8         # rows padded to 128
+    assert api.moe_recv_scale_bytes(300, 224, MX, TILED) == 0               # 7 blocks: not a multiple of 4
+    assert api.moe_recv_scale_bytes(300, 256, FP8, TILED) == 0
+    assert api.moe_recv_scale_bytes(300, 256, BF16, MN) == 0
+    assert api.scale_shape(10, 256, FP8, MN) == ((2, 12), api.torch.float32)
+    assert api.scale_shape(300, 256, MX, TILED) == ((3072,), api.torch.uint8)
+
+    def disp(dt, lay, H=256, scale=_P(), rows=20):
+        return L.moe_dispatch_ex(_P(), 10, H, 2, _P(), rows, dt, lay, _P(), scale, None, None)
+    assert disp(FP8, TILED) == api.MOE_ERR_INVALID_ARG
+    assert disp(TOK, TILED) == api.MOE_ERR_INVALID_ARG
+    assert disp(BF16, MN, scale=None) == api.MOE_ERR_INVALID_ARG
+    assert disp(MX, TILED, H=224) == api.MOE_ERR_INVALID_ARG
+    assert disp(MX, 3) == api.MOE_ERR_INVALID_ARG
+    assert disp(FP8, MN, scale=_P(0x1004)) == api.MOE_ERR_INVALID_ARG   # 16-byte alignment
+    assert disp(FP8, ROW, H=200) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_ex(None, 0, 256, 2, None, 0, MX, TILED, None, None, None, None) == api.MOE_OK
+
+
+def test_swiglu_quant_rejects_bad_arguments(api):
+    L = api.lib()
+    FP8, TOK, MX, BF16 = (api.MOE_DTYPE_FP8_E4M3, api.MOE_DTYPE_FP8_E4M3_TOKEN,
+                          api.MOE_DTYPE_MXFP8_E4M3, api.MOE_DTYPE_BF16)
+    ROW, MN, TILED = api.MOE_SCALE_ROW_MAJOR, api.MOE_SCALE_MN_MAJOR, api.MOE_SCALE_MMA_TILED
+
+    def call(dt, I, lay=ROW, rows=10, h=_P(), out=_P(), sc=_P(), st=None):
+        return L.moe_swiglu_quant(h, rows, I, st, dt, lay, out, sc, None)
+    assert call(FP8, 192) == api.MOE_ERR_INVALID_ARG          # I % 128
+    assert call(MX, 48) == api.MOE_ERR_INVALID_ARG            # I % 32
+    assert call(MX, 96, TILED) == api.MOE_ERR_INVALID_ARG     # tiled needs I % 128
+    assert call(BF16, 24) == api.MOE_ERR_INVALID_ARG          # I % 16
+    assert call(BF16, 256, MN) == api.MOE_ERR_INVALID_ARG     # bf16 has no scales
+    assert call(TOK, 20000) == api.MOE_ERR_UNSUPPORTED
+    assert call(FP8, 256, TILED) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, 7) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, sc=None) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, h=_P(0x1008)) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, MN, sc=_P(0x1004)) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, st=_P(0x1002)) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, rows=-1) == api.MOE_ERR_INVALID_ARG
+    assert call(FP8, 256, rows=0, h=None, out=None, sc=None) == api.MOE_OK
+
+
+def test_nvfp4_sizes_and_validation(api):
+    L = api.lib()
+    NV = api.MOE_DTYPE_NVFP4
+    assert api.moe_recv_bytes(10, 256, 2, NV) == 10 * 2 * 128
+    assert api.moe_scale_bytes(10, 256, 2, NV) == 10 * 2 * 16
+    assert api.moe_recv_scale_bytes(300, 256, NV, api.MOE_SCALE_MMA_TILED) == 384 * 16
+    assert api.moe_recv_scale_bytes(10, 256, NV, api.MOE_SCALE_MN_MAJOR) == 16 * 16
+    assert api.scale_shape(10, 256, NV) == ((10, 16), api.torch.uint8)
+
+    def call(H=256, lay=0, bs=_P(), rs=_P(), x=_P(), rows=20):
+        return L.moe_dispatch_nvfp4(x, 10, H, 2, _P(), rows, lay, _P(), bs, rs, None, None)
+    assert call(H=96) == api.MOE_ERR_INVALID_ARG            # H % 64
+    assert call(H=32768) == api.MOE_ERR_UNSUPPORTED
+    assert call(lay=5) == api.MOE_ERR_INVALID_ARG
+    assert call(rs=None) == api.MOE_ERR_INVALID_ARG
+    assert call(bs=_P(0x1004)) == api.MOE_ERR_INVALID_ARG    # 16-byte aligned block scales
+    assert call(x=_P(0x1008)) == api.MOE_ERR_INVALID_ARG
+    assert call(rows=-1) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_nvfp4(None, 0, 256, 2, None, 0, 0, None, None, None, None, None) == api.MOE_OK
+    # the other entry points do not take NVFP4
+    assert L.moe_dispatch_ex(_P(), 10, 256, 2, _P(), 20, NV, 0, _P(), _P(), None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_swiglu_quant(_P(), 10, 256, None, NV, 0, _P(), _P(), None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_e5m6_sizes_and_validation(api):
+    L = api.lib()
+    E5 = api.MOE_DTYPE_E5M6
+    assert api.moe_recv_bytes(10, 256, 2, E5) == 10 * 2 * 384
+    assert api.moe_scale_bytes(10, 256, 2, E5) == 0
+    assert api.moe_recv_scale_bytes(10, 256, E5, api.MOE_SCALE_MN_MAJOR) == 0
+    assert L.moe_dispatch_ex(_P(), 10, 272, 2, _P(), 20, E5, 0, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_ex(_P(), 10, 256, 2, _P(), 20, E5, 1, _P(), None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch_ex(None, 0, 256, 2, None, 0, E5, 0, None, None, None, None) == api.MOE_OK
+
+
+def test_quant_fp8_channel_rejects_bad_arguments(api):
+    L = api.lib()
+
+    def call(S=64, H=256, E=4, tr=0, recv=_P(), out=_P(), sc=_P(), off=_P(), cnt=_P()):
+        return L.moe_quant_fp8_channel(recv, S, H, E, off, cnt, tr, out, sc, None, None)
+    assert call(H=192) == api.MOE_ERR_INVALID_ARG           # H % 128
+    assert call(E=0) == api.MOE_ERR_INVALID_ARG
+    assert call(E=2000) == api.MOE_ERR_UNSUPPORTED
+    assert call(tr=2) == api.MOE_ERR_INVALID_ARG
+    assert call(sc=None) == api.MOE_ERR_INVALID_ARG
+    assert call(off=None) == api.MOE_ERR_INVALID_ARG
+    assert call(recv=_P(0x1008)) == api.MOE_ERR_INVALID_ARG
+    assert call(out=_P(0x1002)) == api.MOE_ERR_INVALID_ARG
+    assert call(S=-1) == api.MOE_ERR_INVALID_ARG

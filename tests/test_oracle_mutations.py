@@ -35,7 +35,7 @@ MUTANTS = {
     "fp8_scale_transposed": (" sc[b] = amax / 448.0f;", " sc[b] = 448.0f / amax;"),
     "swiglu_fp8_scale_transposed": ("fsc[b] = amax / 448.0f;", "fsc[b] = 448.0f / amax;"),
     "e4m3_ties_away": ("double m = nearbyint(q);                     /* ties to even */",
-                       "double m = floor(q + 0.5);"),
+                       "double m = floor(q + 0.5);", 0),
     "e4m3_subnormal_step": ("double q = a * 512.0;", "double q = a * 256.0;"),
     "bf16_ties_up": ("(lower == 0x8000u && (upper & 1u))", "(lower == 0x8000u)"),
     "combine_weight_index_dropped": ("acc = fmaf(topk_w[(int64_t)t * k + j], v, acc);",
@@ -82,24 +82,42 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTANTS))
-def test_pins_catch_mutant(name, tmp_path):
+def _mutated_source(name: str) -> str:
     src = open(SRC).read()
     old, new, *which = MUTANTS[name]
     if which:   # the anchor occurs in more than one function: mutate occurrence which[0]
         parts = src.split(old)
         assert len(parts) > which[0] + 1, f"mutation anchor occurrence missing: {old!r}"
-        mutated = old.join(parts[:which[0] + 1]) + new + old.join(parts[which[0] + 1:])
-    else:
-        assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
-        mutated = src.replace(old, new)
-    mut = tmp_path / "moe_oracle_mut.c"
-    mut.write_text(mutated)
-    lib = tmp_path / "liboracle_mut.so"
+        return old.join(parts[:which[0] + 1]) + new + old.join(parts[which[0] + 1:])
+    assert src.count(old) == 1, f"mutation anchor not found once: {old!r}"
+    return src.replace(old, new)
+
+
+def _run_mutant(name: str, work) -> tuple[int, str]:
+    """Build the mutated oracle and run the pin suite against it: (return code, tail)."""
+    mut = work / f"{name}.c"
+    mut.write_text(_mutated_source(name))
+    lib = work / f"lib{name}.so"
     subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC",
                            "-shared", "-w", "-o", str(lib), str(mut), "-lm"])
     env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
                         os.path.join(ROOT, "tests", "test_oracle_pins.py")],
-                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, f"pins did not catch mutant {name}:\n{r.stdout[-2000:]}"
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    return r.returncode, r.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def mutant_results(tmp_path_factory):
+    """Every mutant's pin run, several at a time (each is its own process)."""
+    from concurrent.futures import ThreadPoolExecutor
+    work = tmp_path_factory.mktemp("mutants")
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as pool:
+        futs = {n: pool.submit(_run_mutant, n, work) for n in sorted(MUTANTS)}
+        return {n: f.result() for n, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, mutant_results):
+    code, tail = mutant_results[name]
+    assert code != 0, f"pins did not catch mutant {name}:\n{tail}"
