@@ -31,9 +31,11 @@ DT_FP8_E4M3_TOKEN = 2
 DT_MXFP8_E4M3 = 3
 DT_NVFP4 = 4
 DT_E5M6 = 5
+DT_FP8_UE8M0 = 6
 SL_ROW_MAJOR = 0
 SL_MN_MAJOR = 1
 SL_MMA_TILED = 2
+SL_MN_MAJOR_PACK4 = 3
 OK = 0
 ERR_INVALID_ARG = 1
 ERR_BAD_INDEX = 4
@@ -298,6 +300,8 @@ def dispatch(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int,
             scale = np.zeros((S, H // 128), np.float32)
         elif dtype == DT_FP8_E4M3_TOKEN:
             scale = np.zeros((S, 1), np.float32)
+        elif dtype == DT_FP8_UE8M0:                 # UE8M0 bytes, one per 128 channels
+            scale = np.zeros((S, H // 128), np.uint8)
         else:                                   # MXFP8: E8M0 bytes, one per 32 channels
             scale = np.zeros((S, H // 32), np.uint8)
         sp = _ptr(scale)
@@ -334,7 +338,7 @@ def dispatch_scaled(x_bf16: np.ndarray, token_slot: np.ndarray, dtype: int, layo
     if n < 0:
         raise ValueError("oracle_dispatch_scaled: layout not defined for this payload")
     recv = np.zeros((S, H), np.uint8)
-    scale = np.zeros(n, np.uint8 if dtype == DT_MXFP8_E4M3 else np.float32)
+    scale = np.zeros(n, np.uint8 if dtype in (DT_MXFP8_E4M3, DT_FP8_UE8M0) else np.float32)
     st = lib().oracle_dispatch_scaled(_ptr(x_bf16), N, H, k, _ptr(token_slot), S, dtype, layout,
                                       _ptr(recv), _ptr(scale))
     if st == ERR_INVALID_ARG:

@@ -47,6 +47,7 @@
 #define DT_MXFP8_E4M3 3
 #define DT_NVFP4 4
 #define DT_E5M6 5
+#define DT_FP8_UE8M0 6
 
 /* ------------------------------------------------------------------ */
 /* bit helpers                                                         */
@@ -561,7 +562,7 @@ static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
 {
     int status = ORC_OK;
     int64_t S = num_rows;
-    int nb = dtype == DT_MXFP8_E4M3 ? H / 32 : 1;
+    int nb = dtype == DT_FP8_E4M3_TOKEN ? 1 : (dtype == DT_FP8_UE8M0 ? H / 128 : H / 32);
     uint8_t* q = (uint8_t*)malloc((size_t)H);
     float* fsc = (float*)malloc(sizeof(float));
     uint8_t* esc = (uint8_t*)malloc((size_t)nb);
@@ -578,6 +579,31 @@ static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
             for (int c = 0; c < H; ++c) {
                 float v = oracle_f32_from_bf16(xr[c]);
                 q[c] = oracle_e4m3_encode((v == 0.0f) ? v : v * inv);
+            }
+        } else if (dtype == DT_FP8_UE8M0) {
+            /* 1x128 blocks, power-of-two scale 2^e with e = ceil(log2(amax/448)):
+             * the smallest power of two not below the fp32 quotient */
+            for (int b = 0; b < nb; ++b) {
+                float amax = 0.0f;
+                for (int c = b * 128; c < (b + 1) * 128; ++c) {
+                    float v = fabsf(oracle_f32_from_bf16(xr[c]));
+                    if (v > amax) amax = v;
+                }
+                int e = -127;
+                if (amax > 0.0f) {
+                    float qt = amax / 448.0f;
+                    int fe;
+                    double fr = frexp((double)qt, &fe);     /* qt = fr * 2^fe, fr in [0.5, 1) */
+                    e = (fr == 0.5) ? fe - 1 : fe;
+                }
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+                esc[b] = (uint8_t)(e + 127);
+                float down = ldexpf(1.0f, -e);    /* e <= 120 for bf16 input: 2^-e is a normal float */
+                for (int c = b * 128; c < (b + 1) * 128; ++c) {
+                    float v = oracle_f32_from_bf16(xr[c]);
+                    q[c] = oracle_e4m3_encode((v == 0.0f) ? v : v * down);
+                }
             }
         } else {
             for (int b = 0; b < nb; ++b) {
@@ -629,8 +655,9 @@ int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
     if (dtype == DT_FP8_E4M3 && H % 128 != 0) return ORC_ERR_INVALID_ARG;
     if (dtype == DT_MXFP8_E4M3 && H % 32 != 0) return ORC_ERR_INVALID_ARG;
     if (dtype == DT_FP8_E4M3_TOKEN && H % 8 != 0) return ORC_ERR_INVALID_ARG;
-    if (dtype < DT_BF16 || dtype > DT_MXFP8_E4M3) return ORC_ERR_INVALID_ARG;
-    if (dtype == DT_FP8_E4M3_TOKEN || dtype == DT_MXFP8_E4M3)
+    if (dtype == DT_FP8_UE8M0 && H % 128 != 0) return ORC_ERR_INVALID_ARG;
+    if ((dtype < DT_BF16 || dtype > DT_MXFP8_E4M3) && dtype != DT_FP8_UE8M0) return ORC_ERR_INVALID_ARG;
+    if (dtype == DT_FP8_E4M3_TOKEN || dtype == DT_MXFP8_E4M3 || dtype == DT_FP8_UE8M0)
         return oracle_dispatch_variant(x, N, H, k, token_slot, num_rows, dtype, (uint8_t*)recv_x,
                                        recv_scale);
     int status = ORC_OK;
@@ -691,11 +718,18 @@ int oracle_dispatch_rows(const uint16_t* x, int N, int H, int k,
  *               stored row-major over (s / 128, b / 4); inside an atom,
  *               row s and block b sit at byte
  *               (s mod 32)*16 + ((s mod 128) / 32)*4 + (b mod 4).
+ *   MN_MAJOR_PACK4  one-byte scales of 1x128 blocks (UE8M0): four
+ *               consecutive blocks of a row form one 32-bit word (block
+ *               4j+i in byte i), and the words are MN-major -- word (s, j)
+ *               at word index j*ld + s, ld = num_rows rounded up to 4 --
+ *               the packed power-of-two scale operand of a 1x128-scaled
+ *               FP8 GEMM.
  * Positions of rows that no token lands in are not written.            */
 /* ------------------------------------------------------------------ */
 #define SL_ROW_MAJOR 0
 #define SL_MN_MAJOR 1
 #define SL_MMA_TILED 2
+#define SL_MN_MAJOR_PACK4 3
 
 static int scale_blocks(int H, int dtype)
 {
@@ -703,10 +737,14 @@ static int scale_blocks(int H, int dtype)
     if (dtype == DT_FP8_E4M3_TOKEN) return 1;
     if (dtype == DT_MXFP8_E4M3) return H / 32;
     if (dtype == DT_NVFP4) return H / 16;
+    if (dtype == DT_FP8_UE8M0) return H / 128;
     return 0;
 }
 
-static int scale_elem_bytes(int dtype) { return (dtype == DT_MXFP8_E4M3 || dtype == DT_NVFP4) ? 1 : 4; }
+static int scale_elem_bytes(int dtype)
+{
+    return (dtype == DT_MXFP8_E4M3 || dtype == DT_NVFP4 || dtype == DT_FP8_UE8M0) ? 1 : 4;
+}
 
 static int64_t round_up64(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
@@ -720,6 +758,8 @@ int64_t oracle_scale_elems(int64_t num_rows, int H, int dtype, int layout)
     if (layout == SL_MN_MAJOR) return (int64_t)B * round_up64(num_rows, 16 / scale_elem_bytes(dtype));
     if (layout == SL_MMA_TILED && (dtype == DT_MXFP8_E4M3 || dtype == DT_NVFP4) && B % 4 == 0)
         return round_up64(num_rows, 128) * B;
+    if (layout == SL_MN_MAJOR_PACK4 && dtype == DT_FP8_UE8M0)
+        return (int64_t)((B + 3) / 4) * 4 * round_up64(num_rows, 4);
     return -1;
 }
 
@@ -732,6 +772,8 @@ int64_t oracle_scale_index(int layout, int64_t num_rows, int H, int dtype, int64
         int64_t atom = (s / 128) * (B / 4) + b / 4;
         return atom * 512 + (s % 32) * 16 + ((s % 128) / 32) * 4 + b % 4;
     }
+    if (layout == SL_MN_MAJOR_PACK4)   /* 32-bit words of 4 blocks, the words MN-major */
+        return (int64_t)(b / 4) * 4 * round_up64(num_rows, 4) + s * 4 + b % 4;
     return s * B + b;
 }
 

@@ -77,6 +77,10 @@ MUTANTS = {
                                            "int64_t r0 = expert_offset[e], r1 = expert_offset[e + 1];"),
     "fp8_channel_transpose_index": ("if (transpose) out[(size_t)c * num_rows + s] = q;",
                                     "if (transpose) out[(size_t)c * H + s] = q;"),
+    "ue8m0_floor_instead_of_ceil": ("e = (fr == 0.5) ? fe - 1 : fe;", "e = fe - 1;"),
+    "ue8m0_ceil_misses_powers_of_two": ("e = (fr == 0.5) ? fe - 1 : fe;", "e = fe;"),
+    "pack4_words_row_major": ("return (int64_t)(b / 4) * 4 * round_up64(num_rows, 4) + s * 4 + b % 4;",
+                              "return s * 4 * (int64_t)((B + 3) / 4) + (int64_t)(b / 4) * 4 + b % 4;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
                                         "if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                if (s == -1) s = 0;\n                float v"),
 }

@@ -1033,3 +1033,57 @@ def test_fp8_channel_transposed_and_padding():
     x2[~landed] = 0x7F80                                 # +inf in the padding must not matter
     c2, s2, _ = O.quant_fp8_channel(x2, L.expert_offset, L.expert_count)
     assert np.array_equal(c2, c0) and np.array_equal(s2, s0)
+
+
+# ----------------------------------------------------------------- FP8 with UE8M0 (power-of-two) 1x128 scales
+def test_ue8m0_worked_example():
+    g = _gold("ue8m0_worked_example.json")
+    H = g["H"]
+    x = np.zeros((len(g["tokens"]), H), np.float32)
+    for t, tok in enumerate(g["tokens"]):
+        for c, v in tok["values"].items():
+            x[t, int(c)] = v
+    xb = _bf16(x)
+    assert np.array_equal(O.bf16_to_f32(xb), x)
+    recv, sc, st = O.dispatch(xb, np.arange(len(x), dtype=np.int32)[:, None], O.DT_FP8_UE8M0)
+    assert st == 0
+    for t, tok in enumerate(g["tokens"]):
+        want = np.zeros(H, np.uint8)
+        for c, code in tok["codes"].items():
+            want[int(c)] = code
+        assert recv[t].tolist() == want.tolist(), t
+        assert sc[t].tolist() == tok["scale_bytes"], t
+
+
+def test_ue8m0_is_smallest_power_of_two_not_below_quotient():
+    rng = np.random.default_rng(31)
+    N, H = 64, 1024
+    x = rng.normal(size=(N, H)) * np.exp2(rng.integers(-20, 20, (N, H // 128))).repeat(128, 1)
+    x[::7, :128] = 0.0
+    xb = _bf16(x)
+    xf = O.bf16_to_f32(xb)
+    recv, sc, st = O.dispatch(xb, np.arange(N, dtype=np.int32)[:, None], O.DT_FP8_UE8M0)
+    assert st == 0
+    e = sc.astype(np.int64) - 127
+    amax = np.abs(xf).reshape(N, -1, 128).max(-1)
+    q = (amax / np.float32(448)).astype(np.float32).astype(np.float64)
+    live = amax > 0
+    assert (np.exp2(e[live] - 1.0) < q[live]).all() and (q[live] <= np.exp2(e[live].astype(np.float64))).all()
+    assert (sc[~live] == 0).all()
+    scaled = (xf * np.exp2(-e.repeat(128, 1)).astype(np.float32)).astype(np.float32)
+    assert np.array_equal(recv, O.e4m3_encode_array(scaled))
+
+
+def test_pack4_layout_is_word_transpose():
+    rng = np.random.default_rng(5)
+    N, k, H = 33, 2, 768                                  # 6 blocks: two words, the second half full
+    x = _bf16(rng.normal(size=(N, H)) * np.exp2(rng.integers(-9, 9, (N, H // 128))).repeat(128, 1))
+    slots = rng.permutation(N * k).astype(np.int32).reshape(N, k)
+    _, row, _ = O.dispatch(x, slots, O.DT_FP8_UE8M0)
+    _, packed, st = O.dispatch_scaled(x, slots, O.DT_FP8_UE8M0, O.SL_MN_MAJOR_PACK4)
+    assert st == 0
+    S, B = row.shape
+    ld, G = -(-S // 4) * 4, -(-B // 4)
+    padded = np.zeros((ld, G * 4), np.uint8)
+    padded[:S, :B] = row
+    assert np.array_equal(packed, padded.reshape(ld, G, 4).transpose(1, 0, 2).reshape(-1))
