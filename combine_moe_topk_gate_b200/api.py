@@ -21,12 +21,13 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA, MOE_ERR_BAD_INDEX, MOE_ERR_TIMEOUT = range(6)
 MOE_GATE_SOFTMAX, MOE_GATE_SOFTMAX_RENORM, MOE_GATE_SIGMOID_GROUP = range(3)
 (MOE_DTYPE_BF16, MOE_DTYPE_FP8_E4M3, MOE_DTYPE_FP8_E4M3_TOKEN, MOE_DTYPE_MXFP8_E4M3, MOE_DTYPE_NVFP4,
- MOE_DTYPE_E5M6) = range(6)
+ MOE_DTYPE_E5M6, MOE_DTYPE_FP8_E4M3_UE8M0) = range(7)
 MOE_MAX_EXPERTS = 1024
 MOE_MAX_ALIGN = 4096
 MOE_SCALE_ROW_MAJOR = 0
 MOE_SCALE_MN_MAJOR = 1
 MOE_SCALE_MMA_TILED = 2
+MOE_SCALE_MN_MAJOR_PACK4 = 3
 MOE_MAX_TOPK = 32
 MOE_FP8_BLOCK = 128
 
@@ -254,11 +255,13 @@ def scale_shape(S: int, H: int, dtype: int, scale_layout: int = 0):
         nbytes = moe_recv_scale_bytes(S, H, dtype, scale_layout)
         if nbytes == 0:
             return None, None
-        sdt = torch.uint8 if dtype in (MOE_DTYPE_MXFP8_E4M3, MOE_DTYPE_NVFP4) else torch.float32
-        if scale_layout == MOE_SCALE_MMA_TILED:
+        sdt = torch.uint8 if dtype in (MOE_DTYPE_MXFP8_E4M3, MOE_DTYPE_NVFP4, MOE_DTYPE_FP8_E4M3_UE8M0) \
+            else torch.float32
+        if scale_layout in (MOE_SCALE_MMA_TILED, MOE_SCALE_MN_MAJOR_PACK4):
             return (nbytes,), sdt
         B = {MOE_DTYPE_FP8_E4M3: H // MOE_FP8_BLOCK, MOE_DTYPE_FP8_E4M3_TOKEN: 1,
-             MOE_DTYPE_MXFP8_E4M3: H // 32, MOE_DTYPE_NVFP4: H // 16}[dtype]
+             MOE_DTYPE_MXFP8_E4M3: H // 32, MOE_DTYPE_NVFP4: H // 16,
+             MOE_DTYPE_FP8_E4M3_UE8M0: H // MOE_FP8_BLOCK}[dtype]
         es = 1 if sdt == torch.uint8 else 4
         return (B, nbytes // es // B), sdt
     if dtype == MOE_DTYPE_FP8_E4M3:
@@ -269,6 +272,8 @@ def scale_shape(S: int, H: int, dtype: int, scale_layout: int = 0):
         return (S, H // 32), torch.uint8
     if dtype == MOE_DTYPE_NVFP4:
         return (S, H // 16), torch.uint8
+    if dtype == MOE_DTYPE_FP8_E4M3_UE8M0:
+        return (S, H // MOE_FP8_BLOCK), torch.uint8
     return None, None
 
 

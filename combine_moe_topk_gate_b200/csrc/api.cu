@@ -131,6 +131,7 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {
     case MOE_DTYPE_FP8_E4M3_TOKEN: return rows * sizeof(float);
     case MOE_DTYPE_MXFP8_E4M3: return rows * (hidden / 32);
     case MOE_DTYPE_NVFP4: return rows * (hidden / 16);  /* block scales; + 4 bytes per row */
+    case MOE_DTYPE_FP8_E4M3_UE8M0: return rows * (hidden / MOE_FP8_BLOCK);
     default: return 0;
   }
 }
@@ -141,8 +142,13 @@ static int scale_blocks(int H, moe_dtype_t dtype) {
     case MOE_DTYPE_FP8_E4M3_TOKEN: return 1;
     case MOE_DTYPE_MXFP8_E4M3: return H / 32;
     case MOE_DTYPE_NVFP4: return H / 16;
+    case MOE_DTYPE_FP8_E4M3_UE8M0: return H / MOE_FP8_BLOCK;
     default: return 0;
   }
+}
+
+static bool byte_scales(moe_dtype_t dtype) {
+  return dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4 || dtype == MOE_DTYPE_FP8_E4M3_UE8M0;
 }
 
 // whether `layout` is defined for the payload type (and its block count)
@@ -150,6 +156,7 @@ static bool scale_layout_defined(int H, moe_dtype_t dtype, moe_scale_layout_t la
   if (layout == MOE_SCALE_ROW_MAJOR) return true;
   if (dtype == MOE_DTYPE_BF16 || scale_blocks(H, dtype) < 1) return false;
   if (layout == MOE_SCALE_MN_MAJOR) return true;
+  if (layout == MOE_SCALE_MN_MAJOR_PACK4) return dtype == MOE_DTYPE_FP8_E4M3_UE8M0;
   return layout == MOE_SCALE_MMA_TILED &&
          (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) && scale_blocks(H, dtype) % 4 == 0;
 }
@@ -158,11 +165,12 @@ size_t moe_recv_scale_bytes(int num_recv_rows, int hidden, moe_dtype_t dtype,
                             moe_scale_layout_t layout) {
   if (num_recv_rows < 0 || hidden < 1 || !scale_layout_defined(hidden, dtype, layout)) return 0;
   const size_t B = static_cast<size_t>(scale_blocks(hidden, dtype));
-  const size_t es = (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) ? 1 : sizeof(float);
+  const size_t es = byte_scales(dtype) ? 1 : sizeof(float);
   const size_t rows = static_cast<size_t>(num_recv_rows);
   switch (layout) {
     case MOE_SCALE_MN_MAJOR: return B * static_cast<size_t>(moe::scale_ld(num_recv_rows, dtype)) * es;
     case MOE_SCALE_MMA_TILED: return (rows + 127) / 128 * 128 * B;
+    case MOE_SCALE_MN_MAJOR_PACK4: return (B + 3) / 4 * 4 * ((rows + 3) / 4 * 4);
     default: return rows * B * es;
   }
 }
@@ -176,7 +184,7 @@ moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, i
   if (num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
   if (!expert_offset || !expert_count || !scale || (num_rows > 0 && (!recv || !out)))
     return MOE_ERR_INVALID_ARG;
-  if (!aligned(recv, 16) || !aligned(out, 4) || !aligned(scale, 4) || !aligned(expert_offset, 4) ||
+  if (!aligned(recv, 16) || !aligned(out, 16) || !aligned(scale, 4) || !aligned(expert_offset, 4) ||
       !aligned(expert_count, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_quant_fp8_channel(recv, num_rows, hidden, num_experts, expert_offset,
@@ -209,9 +217,8 @@ moe_status_t moe_swiglu_quant(const void* h, int num_rows, int inter, const int3
       return MOE_ERR_INVALID_ARG;
   }
   if (!scale_layout_defined(inter, dtype, scale_layout)) return MOE_ERR_INVALID_ARG;
-  // one warp per (row, 512 channels), 8 warps per CTA: the grid must fit
-  if (static_cast<long long>(num_rows) * ((inter + 511) / 512) / 8 >= kMaxRows)
-    return MOE_ERR_UNSUPPORTED;
+  // grid: y = 512-channel segments of a row (at most 65535)
+  if ((inter + 511) / 512 > 65535) return MOE_ERR_UNSUPPORTED;
   if (num_rows == 0) return MOE_OK;
   if (!h || !out) return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_DTYPE_BF16 && !out_scale) return MOE_ERR_INVALID_ARG;
@@ -260,8 +267,7 @@ moe_status_t moe_dispatch_ex(const void* x, int num_tokens, int hidden, int k,
                              int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, H = hidden;
   if (N < 0 || H < 1 || k < 1 || num_recv_rows < 0) return MOE_ERR_INVALID_ARG;
-  if (scale_layout != MOE_SCALE_ROW_MAJOR && scale_layout != MOE_SCALE_MN_MAJOR &&
-      scale_layout != MOE_SCALE_MMA_TILED)
+  if (scale_layout < MOE_SCALE_ROW_MAJOR || scale_layout > MOE_SCALE_MN_MAJOR_PACK4)
     return MOE_ERR_INVALID_ARG;
   if (k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
   if (static_cast<long long>(N) * k > kMaxRows) return MOE_ERR_UNSUPPORTED;
@@ -276,6 +282,8 @@ moe_status_t moe_dispatch_ex(const void* x, int num_tokens, int hidden, int k,
     if (H % 32 != 0) return MOE_ERR_INVALID_ARG;
   } else if (dtype == MOE_DTYPE_E5M6) {
     if (H % 32 != 0) return MOE_ERR_INVALID_ARG;
+  } else if (dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
+    if (H % MOE_FP8_BLOCK != 0) return MOE_ERR_INVALID_ARG;
   } else {
     return MOE_ERR_INVALID_ARG;
   }
@@ -284,8 +292,7 @@ moe_status_t moe_dispatch_ex(const void* x, int num_tokens, int hidden, int k,
   if (!x || !token_slot || !recv_x) return MOE_ERR_INVALID_ARG;
   const bool scaled = dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_E5M6;
   if (scaled && !recv_scale) return MOE_ERR_INVALID_ARG;
-  const int scale_align =
-      (dtype == MOE_DTYPE_MXFP8_E4M3 || scale_layout != MOE_SCALE_ROW_MAJOR) ? 16 : 4;
+  const int scale_align = (byte_scales(dtype) || scale_layout != MOE_SCALE_ROW_MAJOR) ? 16 : 4;
   if (scaled && !aligned(recv_scale, scale_align)) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(recv_x, 16) || !aligned(token_slot, 4) || !aligned(d_status, 4))
     return MOE_ERR_INVALID_ARG;

@@ -22,7 +22,20 @@ constexpr int kWarps = 8;
 
 // FP8: lane owns 16 channels (two 16-byte loads), 8 lanes = one 128-block,
 // a warp covers 512 channels.
-template <int SL>
+// ceil(log2(q)) for q > 0 finite, exact from the bits (subnormals too)
+__device__ __forceinline__ int ceil_log2_pos(float q) {
+  const uint32_t u = __float_as_uint(q);
+  const uint32_t m = u & 0x7fffffu;
+  const int ex = static_cast<int>((u >> 23) & 0xffu);
+  if (ex) return ex - 127 + (m != 0u);
+  const int fl = (31 - __clz(m)) - 149;
+  return fl + ((m & (m - 1u)) != 0u);
+}
+
+// UE8M0 = true: power-of-two scale 2^e per 128-block with e = ceil(log2(amax /
+// 448)) of the fp32 quotient, stored as the byte e + 127; codes e4m3(x * 2^-e)
+// (exact scaling, so a zero keeps its sign without a select).
+template <int SL, bool UE8M0 = false>
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_fp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                         const int32_t* __restrict__ token_slot, long long S,
@@ -60,8 +73,19 @@ __global__ void __launch_bounds__(kWarps * 32)
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-  const float inv = __fdiv_rn(448.0f, amax);
-  const float scale = __fdiv_rn(amax, 448.0f);
+  float inv, scale = 0.0f;
+  uint32_t sword = 0;  // UE8M0: the warp's 4 block bytes (block i in byte i)
+  if constexpr (UE8M0) {
+    int e = amax > 0.0f ? ceil_log2_pos(__fdiv_rn(amax, 448.0f)) : -127;
+    e = e < -127 ? -127 : (e > 127 ? 127 : e);
+    inv = __int_as_float((127 - e) << 23);  // 2^-e; e <= 120 for bf16 input
+    const uint32_t byte = static_cast<uint32_t>(e + 127);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sword |= (__shfl_sync(kFullMask, byte, 8 * i) & 0xffu) << (8 * i);
+  } else {
+    inv = __fdiv_rn(448.0f, amax);
+    scale = __fdiv_rn(amax, 448.0f);
+  }
   uint32_t q[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -69,7 +93,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float v = f[4 * i + u];
-      p[u] = (v == 0.0f) ? v : __fmul_rn(v, inv);  // zero keeps its sign
+      p[u] = (UE8M0 || v != 0.0f) ? __fmul_rn(v, inv) : v;  // zero keeps its sign
     }
     q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
   }
@@ -81,9 +105,19 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (lane == 0) report_bad_index(d_status);
       continue;
     }
-    if (active) {
-      st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
-      if ((lane & 7) == 0) recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
+    if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
+    if constexpr (!UE8M0) {
+      if (active && (lane & 7) == 0) recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
+    } else {
+      uint8_t* sb = reinterpret_cast<uint8_t*>(recv_scale);
+      if constexpr (SL == MOE_SCALE_MN_MAJOR_PACK4) {
+        // the warp's 4 blocks are exactly word s of the row
+        if (lane == 0) *reinterpret_cast<uint32_t*>(sb + scale_at<SL>(slot, 4 * s, nblk, ld)) = sword;
+      } else if (SL == MOE_SCALE_ROW_MAJOR && (nblk & 3) == 0) {
+        if (lane == 0) *reinterpret_cast<uint32_t*>(sb + static_cast<size_t>(slot) * nblk + 4 * s) = sword;
+      } else if (active && (lane & 7) == 0) {
+        sb[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = static_cast<uint8_t>(sword >> (lane & 24));
+      }
     }
   }
 }
@@ -280,26 +314,26 @@ __global__ void __launch_bounds__(kTokenThreads)
     slots[tid] = sl;
     if (sl < -1 || sl >= S) report_bad_index(d_status);
   }
-  float f[VPT][16];
+  // the raw bf16 words stay live across the row reduction (8 registers per
+  // block rather than 16 unpacked floats)
+  uint4 va[VPT], vb[VPT];
   float bmax[VPT];
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = i * kTokenThreads + tid;
-    uint4 a = make_uint4(0, 0, 0, 0), b = a;
+    va[i] = make_uint4(0, 0, 0, 0);
+    vb[i] = va[i];
     if (vi < nvec) {
       const uint16_t* src = x + static_cast<size_t>(t) * H + static_cast<size_t>(vi) * 16;
-      a = ld_stream(src);
-      b = ld_stream(src + 8);
+      va[i] = ld_stream(src);
+      vb[i] = ld_stream(src + 8);
     }
-    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    const uint32_t w[8] = {va[i].x, va[i].y, va[i].z, va[i].w, vb[i].x, vb[i].y, vb[i].z, vb[i].w};
     bmax[i] = 0.0f;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      f[i][2 * u] = bf16_lo(w[u]);
-      f[i][2 * u + 1] = bf16_hi(w[u]);
-      bmax[i] = fmaxf(bmax[i], fmaxf(fabsf(f[i][2 * u]), fabsf(f[i][2 * u + 1])));
-    }
+    for (int u = 0; u < 8; ++u)
+      bmax[i] = fmaxf(bmax[i], fmaxf(fabsf(bf16_lo(w[u])), fabsf(bf16_hi(w[u]))));
     amax = fmaxf(amax, bmax[i]);
   }
 #pragma unroll
@@ -318,9 +352,21 @@ __global__ void __launch_bounds__(kTokenThreads)
     const float sbf = __fmul_rn(__fdiv_rn(bmax[i], 6.0f), inv);
     const uint32_t sb = bmax[i] > 0.0f ? (e4m3x2(sbf, 0.0f) & 0xffu) : 0u;
     const float r = __fdiv_rn(inv, e4m3_value(sb));
-    float p[16];
+    const uint32_t w[8] = {va[i].x, va[i].y, va[i].z, va[i].w, vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+    float f[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) p[u] = (f[i][u] == 0.0f) ? f[i][u] : __fmul_rn(f[i][u], r);
+    for (int u = 0; u < 8; ++u) {
+      f[2 * u] = bf16_lo(w[u]);
+      f[2 * u + 1] = bf16_hi(w[u]);
+    }
+    float p[16];
+    if (r <= 3.402823466e38f) {  // finite: the product keeps a zero's sign
+#pragma unroll
+      for (int u = 0; u < 16; ++u) p[u] = __fmul_rn(f[u], r);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) p[u] = (f[u] == 0.0f) ? f[u] : __fmul_rn(f[u], r);
+    }
     q[i] = make_uint2(e2m1x8(p), e2m1x8(p + 8));
     // bytes of blocks vi..vi+3 (threads lane..lane+3) into lane % 4 == 0
     uint32_t word = sb;
@@ -369,13 +415,16 @@ __device__ __forceinline__ uint32_t e5m6_code(float f) {
 }
 
 // E5M6 dispatch: lane owns 16 channels (two 16-byte loads) -> 16 codes ->
-// 24 bytes (two codes per 3 bytes, little endian), stored as three 8-byte
-// streaming stores; a warp writes 768 contiguous bytes of each receive row.
+// 24 bytes (two codes per 3 bytes, little endian).  The warp's 768 bytes are
+// staged in shared memory and leave as 16-byte streaming stores covering 512
+// and 256 contiguous bytes (lanes 0..31, then 0..15), so no sector is
+// written in pieces.
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_e5m6_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                          const int32_t* __restrict__ token_slot, long long S,
                          uint8_t* __restrict__ recv_x, int32_t* d_status) {
-  const int lane = threadIdx.x & 31;
+  __shared__ __align__(16) uint2 stage[kWarps][96];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int segs = (H + 511) / 512;
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   if (item >= static_cast<long long>(N) * segs) return;
@@ -396,9 +445,16 @@ __global__ void __launch_bounds__(kWarps * 32)
   uint32_t p[8];  // 24-bit pairs
 #pragma unroll
   for (int i = 0; i < 8; ++i) p[i] = e5m6_code(bf16_lo(w[i])) | (e5m6_code(bf16_hi(w[i])) << 12);
-  const uint2 o0 = make_uint2(p[0] | (p[1] << 24), (p[1] >> 8) | (p[2] << 16));
-  const uint2 o1 = make_uint2((p[2] >> 16) | (p[3] << 8), p[4] | (p[5] << 24));
-  const uint2 o2 = make_uint2((p[5] >> 8) | (p[6] << 16), (p[6] >> 16) | (p[7] << 8));
+  stage[warp][3 * lane] = make_uint2(p[0] | (p[1] << 24), (p[1] >> 8) | (p[2] << 16));
+  stage[warp][3 * lane + 1] = make_uint2((p[2] >> 16) | (p[3] << 8), p[4] | (p[5] << 24));
+  stage[warp][3 * lane + 2] = make_uint2((p[5] >> 8) | (p[6] << 16), (p[6] >> 16) | (p[7] << 8));
+  __syncwarp();
+  // 16-byte chunk c of the warp's 768 bytes: lanes take c = lane and c = 32 + lane
+  const uint4* st4 = reinterpret_cast<const uint4*>(stage[warp]);
+  const uint4 v0 = st4[lane];
+  const uint4 v1 = lane < 16 ? st4[32 + lane] : make_uint4(0, 0, 0, 0);
+  // the segment's live bytes: 24 per active lane (the last segment of a row may be short)
+  const int live = (H - s * 512 < 512 ? H - s * 512 : 512) / 16 * 24;
   const size_t row_bytes = static_cast<size_t>(H) / 2 * 3;
   for (int j = 0; j < k; ++j) {
     const int slot = __shfl_sync(kFullMask, my_slot, j);
@@ -407,13 +463,9 @@ __global__ void __launch_bounds__(kWarps * 32)
       if (lane == 0) report_bad_index(d_status);
       continue;
     }
-    if (active) {
-      uint2* dst = reinterpret_cast<uint2*>(recv_x + static_cast<size_t>(slot) * row_bytes +
-                                            static_cast<size_t>(c0) / 2 * 3);
-      __stcs(dst, o0);
-      __stcs(dst + 1, o1);
-      __stcs(dst + 2, o2);
-    }
+    uint8_t* dst = recv_x + static_cast<size_t>(slot) * row_bytes + static_cast<size_t>(s) * 768;
+    if (16 * lane < live) st_stream_v4(dst + 16 * lane, v0);
+    if (lane < 16 && 512 + 16 * lane < live) st_stream_v4(dst + 512 + 16 * lane, v1);
   }
 }
 
@@ -462,8 +514,10 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
 }  // namespace
 
 long long scale_ld(long long num_rows, int dtype) {
-  const long long per16 =
-      (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4) ? 16 : 4;  // scales per 16 bytes
+  const long long per16 = (dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_NVFP4 ||
+                           dtype == MOE_DTYPE_FP8_E4M3_UE8M0)
+                              ? 16
+                              : 4;  // scales per 16 bytes
   return (num_rows + per16 - 1) / per16 * per16;
 }
 
@@ -474,11 +528,22 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* r8 = static_cast<uint8_t*>(recv_x);
   const long long ld = scale_ld(num_rows, dtype);
-  if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3) {
+  if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
     const long long items = static_cast<long long>(N) * ((H + 511) / 512);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
     float* f32 = static_cast<float*>(recv_scale);
     uint8_t* e8 = static_cast<uint8_t*>(recv_scale);
+    if (dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
+      if (scale_layout == MOE_SCALE_MN_MAJOR)
+        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR, true>, blocks, kWarps * 32, 0, stream,
+                          xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+      if (scale_layout == MOE_SCALE_MN_MAJOR_PACK4)
+        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR_PACK4, true>, blocks, kWarps * 32, 0,
+                          stream, xs, N, H, k, token_slot, num_rows, r8, f32, (num_rows + 3) / 4 * 4,
+                          d_status);
+      return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_ROW_MAJOR, true>, blocks, kWarps * 32, 0, stream,
+                        xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+    }
     if (dtype == MOE_DTYPE_FP8_E4M3) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
         return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,

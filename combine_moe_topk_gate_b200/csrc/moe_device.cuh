@@ -103,6 +103,9 @@ __device__ __forceinline__ size_t scale_at(long long s, int b, int B, long long 
   } else if constexpr (SL == MOE_SCALE_MMA_TILED) {
     const size_t atom = static_cast<size_t>(s >> 7) * (B >> 2) + (b >> 2);
     return atom * 512 + (s & 31) * 16 + ((s >> 5) & 3) * 4 + (b & 3);
+  } else if constexpr (SL == MOE_SCALE_MN_MAJOR_PACK4) {
+    // 32-bit words of 4 consecutive blocks, MN-major; ld = rows rounded up to 4
+    return static_cast<size_t>(b >> 2) * 4 * ld + static_cast<size_t>(s) * 4 + (b & 3);
   } else {
     return static_cast<size_t>(s) * B + b;
   }

@@ -10,12 +10,13 @@
 // zeros keeping their sign.  Codes go out row-major [S, H] (read MN-major by
 // the GEMM) or transposed [H, S] (K-major); padding rows are not touched.
 //
-// One CTA per (expert, 128-channel slab), 8 warps, each lane owning 4
-// channels (one 8-byte load per row).  Pass 1 reduces the slab's amax over
-// the expert's rows; pass 2 reads the same rows again -- from L2, the slab of
-// one expert is small -- and writes the codes: 4 bytes per lane and row
-// (row-major), or through a shared-memory tile of 32 rows so that each warp
-// store covers 32 consecutive rows of one channel (transposed).
+// One CTA per (expert, 256-channel slab), 8 warps, each lane owning 8
+// channels (one 16-byte load per row, 512 contiguous bytes per warp).  Pass
+// 1 reduces the slab's amax over the expert's rows, eight loads in flight per
+// lane; pass 2 reads the same rows again -- from L2, the slab of one expert
+// is small -- and writes the codes: 8 bytes per lane and row (row-major), or
+// through a shared-memory tile of 32 rows so that each warp store covers 32
+// consecutive rows of one channel (transposed).
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
@@ -24,12 +25,33 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarpsPerCta = kThreads / 32;
-constexpr int kSlab = 128;
+constexpr int kSlab = 256;
 
-__device__ __forceinline__ uint2 ld_nc_v2(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+// L2 eviction policies: pass 1 marks the slab's lines evict-last so that pass
+// 2 finds them in L2 despite the stream of other CTAs' loads and stores;
+// pass 2 and the code stores are evict-first (nothing reads them again here).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ld_hint(const void* ptr, uint64_t pol) {
+  uint4 r;  // not volatile: independent loads may be scheduled together
+  asm("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(ptr), "l"(pol));
   return r;
+}
+__device__ __forceinline__ void st_hint_v2(void* ptr, uint2 v, uint64_t pol) {
+  // no memory clobber: the codes are never read back here, so loads of x may
+  // move ahead of these stores
+  asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(ptr), "r"(v.x), "r"(v.y),
+               "l"(pol));
 }
 
 template <bool TRANSPOSE>
@@ -40,71 +62,113 @@ __global__ void __launch_bounds__(kThreads)
                              float* __restrict__ scale, int32_t* d_status) {
   __shared__ float part[kWarpsPerCta][kSlab];
   __shared__ float inv_s[kSlab];
-  __shared__ uint8_t tile[kSlab][33];  // transposed path: 32 rows per channel (+1 against conflicts)
+  __shared__ uint8_t tile[TRANSPOSE ? kSlab : 1][33];  // transposed: 32 rows per channel (+1: banks)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int slab = blockIdx.x, e = blockIdx.y;
-  const int c0 = slab * kSlab + lane * 4;
+  const int c0 = slab * kSlab + lane * 8;
+  const bool active = c0 < H;  // H % 128 == 0: 8 whole channels or none
   pdl_wait();
   pdl_trigger();
-  long long r0 = expert_offset[e];
+  const long long r0 = expert_offset[e];
   const long long n = expert_count[e];
   if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert
     if (tid == 0 && slab == 0) report_bad_index(d_status);
     return;
   }
   const long long r1 = r0 + n;
+  const uint16_t* col = x + c0;
+  const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
 
-  // pass 1: amax of the lane's 4 channels over the warp's rows
-  float m[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 4
-  for (long long s = r0 + warp; s < r1; s += kWarpsPerCta) {
-    const uint2 v = ld_nc_v2(x + static_cast<size_t>(s) * H + c0);
-    m[0] = fmaxf(m[0], fabsf(bf16_lo(v.x)));
-    m[1] = fmaxf(m[1], fabsf(bf16_hi(v.x)));
-    m[2] = fmaxf(m[2], fabsf(bf16_lo(v.y)));
-    m[3] = fmaxf(m[3], fabsf(bf16_hi(v.y)));
+  // pass 1: amax of the lane's 8 channels over the warp's rows
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+  if (active) {
+    long long s = r0 + warp;
+    for (; s + 7 * kWarpsPerCta < r1; s += 8 * kWarpsPerCta) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = ld_hint(col + static_cast<size_t>(s + u * kWarpsPerCta) * H, keep);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          m[2 * j] = fmaxf(m[2 * j], fabsf(bf16_lo(w[j])));
+          m[2 * j + 1] = fmaxf(m[2 * j + 1], fabsf(bf16_hi(w[j])));
+        }
+      }
+    }
+    for (; s < r1; s += kWarpsPerCta) {
+      const uint4 v = ld_hint(col + static_cast<size_t>(s) * H, keep);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        m[2 * j] = fmaxf(m[2 * j], fabsf(bf16_lo(w[j])));
+        m[2 * j + 1] = fmaxf(m[2 * j + 1], fabsf(bf16_hi(w[j])));
+      }
+    }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) part[warp][lane * 4 + i] = m[i];
+  for (int i = 0; i < 8; ++i) part[warp][lane * 8 + i] = m[i];
   __syncthreads();
-  if (tid < kSlab) {
-    float a = part[0][tid];
+  {
+    const int c = tid;  // kThreads == kSlab: one channel per thread
+    float a = part[0][c];
 #pragma unroll
-    for (int w = 1; w < kWarpsPerCta; ++w) a = fmaxf(a, part[w][tid]);
-    inv_s[tid] = __fdiv_rn(448.0f, a);
-    scale[static_cast<size_t>(e) * H + slab * kSlab + tid] = __fdiv_rn(a, 448.0f);
+    for (int w = 1; w < kWarpsPerCta; ++w) a = fmaxf(a, part[w][c]);
+    inv_s[c] = __fdiv_rn(448.0f, a);
+    if (slab * kSlab + c < H) scale[static_cast<size_t>(e) * H + slab * kSlab + c] = __fdiv_rn(a, 448.0f);
   }
   __syncthreads();
-  float inv[4];
+  float inv[8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) inv[i] = inv_s[lane * 4 + i];
+  for (int i = 0; i < 8; ++i) inv[i] = inv_s[lane * 8 + i];
 
-  // pass 2: codes
-  auto codes_of = [&](long long s) -> uint32_t {
-    const uint2 v = ld_nc_v2(x + static_cast<size_t>(s) * H + c0);
-    const float f[4] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y)};
-    float p[4];
+  // pass 2: codes of one row's 8 channels
+  auto codes_of_v = [&](uint4 v) -> uint2 {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    float p[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) p[i] = (f[i] == 0.0f) ? f[i] : __fmul_rn(f[i], inv[i]);
-    return e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+    for (int j = 0; j < 4; ++j) {
+      const float lo = bf16_lo(w[j]), hi = bf16_hi(w[j]);
+      p[2 * j] = (lo == 0.0f) ? lo : __fmul_rn(lo, inv[2 * j]);
+      p[2 * j + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, inv[2 * j + 1]);
+    }
+    return make_uint2(e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16),
+                      e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16));
   };
+  auto codes_of = [&](long long s) -> uint2 { return codes_of_v(ld_hint(col + static_cast<size_t>(s) * H, done)); };
   if constexpr (!TRANSPOSE) {
-    for (long long s = r0 + warp; s < r1; s += kWarpsPerCta)
-      *reinterpret_cast<uint32_t*>(out + static_cast<size_t>(s) * H + c0) = codes_of(s);
+    if (active) {
+      long long s = r0 + warp;
+      for (; s + 3 * kWarpsPerCta < r1; s += 4 * kWarpsPerCta) {  // four rows' loads in flight
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = ld_hint(col + static_cast<size_t>(s + u * kWarpsPerCta) * H, done);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_hint_v2(out + static_cast<size_t>(s + u * kWarpsPerCta) * H + c0, codes_of_v(v[u]), done);
+      }
+      for (; s < r1; s += kWarpsPerCta) st_hint_v2(out + static_cast<size_t>(s) * H + c0, codes_of(s), done);
+    }
   } else {
     for (long long s0 = r0; s0 < r1; s0 += 32) {
       // warp w fills rows s0 + w, s0 + w + 8, ... of the 32-row tile
       for (int rr = warp; rr < 32; rr += kWarpsPerCta) {
         const long long s = s0 + rr;
-        const uint32_t q = s < r1 ? codes_of(s) : 0u;
+        const uint2 q = (active && s < r1) ? codes_of(s) : make_uint2(0, 0);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tile[lane * 4 + i][rr] = static_cast<uint8_t>(q >> (8 * i));
+        for (int i = 0; i < 4; ++i) {
+          tile[lane * 8 + i][rr] = static_cast<uint8_t>(q.x >> (8 * i));
+          tile[lane * 8 + 4 + i][rr] = static_cast<uint8_t>(q.y >> (8 * i));
+        }
       }
       __syncthreads();
       // warp w writes channels w, w + 8, ...: lane = row, 32 consecutive bytes
       const long long s = s0 + lane;
       for (int c = warp; c < kSlab; c += kWarpsPerCta)
-        if (s < r1) out[static_cast<size_t>(slab * kSlab + c) * S + s] = tile[c][lane];
+        if (s < r1 && slab * kSlab + c < H) out[static_cast<size_t>(slab * kSlab + c) * S + s] = tile[c][lane];
       __syncthreads();
     }
   }
@@ -116,7 +180,7 @@ cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, i
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,
                                      cudaStream_t stream) {
-  const dim3 grid(H / kSlab, E);
+  const dim3 grid((H + kSlab - 1) / kSlab, E);
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* o = static_cast<uint8_t*>(out);
   if (transpose)

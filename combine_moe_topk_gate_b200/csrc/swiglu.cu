@@ -63,12 +63,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1)  // (..., 1): no register cap,
     swiglu_quant_kernel(const uint16_t* __restrict__ h, long long S, int I,
                         const int32_t* __restrict__ slot_token, void* __restrict__ out,
                         void* __restrict__ out_scale, long long ld) {
+  // grid: x = groups of kWarps rows, y = 512-channel segment (no division)
   const int lane = threadIdx.x & 31;
-  const int segs = (I + 511) / 512;
-  const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  if (item >= S * segs) return;
-  const long long row = item / segs;
-  const int seg = static_cast<int>(item - row * segs);
+  const long long row = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  if (row >= S) return;
+  const int seg = blockIdx.y;
   const int c0 = seg * 512 + lane * 16;
   const bool active = c0 < I;  // I % 16 == 0: a lane's 16 channels are all in or all out
   pdl_wait();
@@ -211,9 +210,8 @@ __global__ void __launch_bounds__(kRowThreads, 1)
 template <int DT, int SL>
 cudaError_t launch_warp_kernel(const uint16_t* h, long long S, int I, const int32_t* slot_token,
                                void* out, void* out_scale, long long ld, cudaStream_t stream) {
-  const long long items = S * ((I + 511) / 512);
-  const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  return launch_pdl(swiglu_quant_kernel<DT, SL>, blocks, kWarps * 32, 0, stream, h, S, I,
+  const dim3 grid(static_cast<unsigned>((S + kWarps - 1) / kWarps), (I + 511) / 512);
+  return launch_pdl(swiglu_quant_kernel<DT, SL>, grid, kWarps * 32, 0, stream, h, S, I,
                     slot_token, out, out_scale, ld);
 }
 

@@ -29,7 +29,7 @@ from dataclasses import dataclass, field
 import torch
 
 GATE_KINDS = {"softmax": 0, "softmax_renorm": 1, "sigmoid_group": 2}
-DTYPES = {"bf16": 0, "fp8": 1, "fp8_token": 2, "mxfp8": 3}
+DTYPES = {"bf16": 0, "fp8": 1, "fp8_token": 2, "mxfp8": 3, "fp8_ue8m0": 6}
 
 
 @dataclass(frozen=True)
@@ -123,7 +123,8 @@ def algorithmic_bytes(w: Workload) -> dict:
     N, H, E, k = w.N, w.H, w.E, w.k
     row = {"bf16": 2 * H, "nvfp4": H // 2, "e5m6": H // 2 * 3}.get(w.dtype, H)   # payload bytes of a receive row
     scales = {"fp8": 4 * N * k * (H // 128), "fp8_token": 4 * N * k,
-              "mxfp8": N * k * (H // 32), "nvfp4": N * k * (H // 16) + 4 * N * k}.get(w.dtype, 0)
+              "mxfp8": N * k * (H // 32), "nvfp4": N * k * (H // 16) + 4 * N * k,
+              "fp8_ue8m0": N * k * (H // 128)}.get(w.dtype, 0)
     return {
         "gate": 4 * N * E + 8 * N * k,
         "layout": 4 * N * k + 8 * N * k + 4 * (4 * E + 3 * w.R),

@@ -74,7 +74,8 @@ typedef enum {
     MOE_DTYPE_FP8_E4M3_TOKEN = 2,/* e4m3, one fp32 scale per token row                  */
     MOE_DTYPE_MXFP8_E4M3 = 3,    /* OCP MXFP8: e4m3, one E8M0 scale byte per 32 channels */
     MOE_DTYPE_NVFP4 = 4,         /* e2m1, one e4m3 scale per 16 channels + fp32 per row  */
-    MOE_DTYPE_E5M6 = 5           /* 12-bit float (FP16 minus 4 fraction bits), no scale  */
+    MOE_DTYPE_E5M6 = 5,          /* 12-bit float (FP16 minus 4 fraction bits), no scale  */
+    MOE_DTYPE_FP8_E4M3_UE8M0 = 6 /* e4m3, one power-of-two (UE8M0 byte) scale per 128     */
 } moe_dtype_t;
 
 /* Where the receive scales go (moe_dispatch_ex).  Scale (s, b) is that of
@@ -83,7 +84,8 @@ typedef enum {
 typedef enum {
     MOE_SCALE_ROW_MAJOR = 0,     /* element s*B + b                                      */
     MOE_SCALE_MN_MAJOR = 1,      /* element b*ld + s, ld = S padded to 16 bytes of scales */
-    MOE_SCALE_MMA_TILED = 2      /* E8M0 only: block-scaled MMA scale-factor atoms        */
+    MOE_SCALE_MMA_TILED = 2,     /* E8M0 only: block-scaled MMA scale-factor atoms        */
+    MOE_SCALE_MN_MAJOR_PACK4 = 3 /* UE8M0 only: 4 blocks per 32-bit word, words MN-major  */
 } moe_scale_layout_t;
 
 typedef void* moe_stream_t;      /* a cudaStream_t */
@@ -254,6 +256,12 @@ size_t moe_scale_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
  *          codes e4m3_rne_satfinite(x * 2^-e) (the power-of-two scaling is
  *          exact; values up to 511.x saturate to 448).  H % 32 == 0;
  *          recv_scale 16-byte aligned.
+ *   FP8 with power-of-two scales (MOE_DTYPE_FP8_E4M3_UE8M0; [TK] lists
+ *          power-of-two scales, the rule is a reading): per 128-channel
+ *          block e = ceil(log2(amax / 448)) of the fp32 quotient (-127 for an
+ *          all-zero block, clamped to [-127, 127]), scale byte e + 127,
+ *          codes e4m3_rne_satfinite(x * 2^-e); recv_scale uint8 [S, H/128].
+ *          H % 128 == 0, recv_scale 16-byte aligned.
  *   E5M6 ([TK]: E5M6 conversion; the format is not defined there, reading:
  *          IEEE-style 1-5-6 bits, bias 15, i.e. FP16 with its 4 lowest
  *          fraction bits dropped; round to nearest even, saturating to
@@ -286,6 +294,11 @@ moe_status_t moe_dispatch(const void* x, int num_tokens, int hidden, int k,
  *        block b sit at byte (s%32)*16 + ((s%128)/32)*4 + b%4.  With the
  *        aligned layout at align 128 every expert's scales are a contiguous
  *        run of whole atoms.
+ *   MOE_SCALE_MN_MAJOR_PACK4  FP8 with UE8M0 scales: four consecutive blocks
+ *        of a row form one 32-bit word (block 4j+i in byte i; bytes of
+ *        blocks past H/128 are written as 0) and the words are MN-major,
+ *        word (s, j) at j*ld + s with ld = S rounded up to 4 -- the packed
+ *        power-of-two scale operand of a 1x128-scaled FP8 GEMM.
  *   recv_scale holds moe_recv_scale_bytes(S, H, dtype, scale_layout) bytes,
  *   16-byte aligned for the MN-major and tiled layouts.  Only positions of
  *   rows a token lands in are written.  A layout the payload type does not
@@ -340,7 +353,7 @@ moe_status_t moe_dispatch_nvfp4(const void* x, int num_tokens, int hidden, int k
  *   code = e4m3(x * (448 / amax)) (fp32, rounded once each; zeros keep
  *   their sign) -- the per-block rule with the block = one channel of one
  *   expert.
- *   recv           bf16 [S, H] in (S = num_rows), 16-byte aligned.
+ *   recv           bf16 [S, H] in (S = num_rows); recv and out 16-byte aligned.
  *   expert_offset  int32 [E+1], expert_count int32 [E]: device arrays, e.g.
  *                  from moe_get_layout_aligned; an expert whose range leaves
  *                  [0, S) is skipped and reported through d_status.

@@ -256,3 +256,25 @@ def test_quant_fp8_channel_rejects_bad_arguments(api):
     assert call(recv=_P(0x1008)) == api.MOE_ERR_INVALID_ARG
     assert call(out=_P(0x1002)) == api.MOE_ERR_INVALID_ARG
     assert call(S=-1) == api.MOE_ERR_INVALID_ARG
+
+
+def test_ue8m0_and_pack4_sizes_and_validation(api):
+    L = api.lib()
+    U8, FP8, MX = api.MOE_DTYPE_FP8_E4M3_UE8M0, api.MOE_DTYPE_FP8_E4M3, api.MOE_DTYPE_MXFP8_E4M3
+    P4 = api.MOE_SCALE_MN_MAJOR_PACK4
+    assert api.moe_recv_bytes(10, 768, 2, U8) == 10 * 2 * 768
+    assert api.moe_scale_bytes(10, 768, 2, U8) == 10 * 2 * 6
+    assert api.moe_recv_scale_bytes(10, 768, U8, P4) == 2 * 4 * 12          # 6 blocks -> 2 words, rows -> 12
+    assert api.moe_recv_scale_bytes(10, 768, U8, api.MOE_SCALE_MN_MAJOR) == 6 * 16
+    assert api.moe_recv_scale_bytes(10, 768, U8, api.MOE_SCALE_MMA_TILED) == 0
+    assert api.moe_recv_scale_bytes(10, 768, MX, P4) == 0
+    assert api.scale_shape(10, 768, U8) == ((10, 6), api.torch.uint8)
+    assert api.scale_shape(10, 768, U8, P4) == ((96,), api.torch.uint8)
+
+    def disp(dt, lay, H=768, sc=_P()):
+        return L.moe_dispatch_ex(_P(), 10, H, 2, _P(), 20, dt, lay, _P(), sc, None, None)
+    assert disp(U8, 0, H=192) == api.MOE_ERR_INVALID_ARG                  # H % 128
+    assert disp(U8, api.MOE_SCALE_MMA_TILED) == api.MOE_ERR_INVALID_ARG
+    assert disp(FP8, P4) == api.MOE_ERR_INVALID_ARG
+    assert disp(U8, 4) == api.MOE_ERR_INVALID_ARG
+    assert disp(U8, 0, sc=_P(0x1004)) == api.MOE_ERR_INVALID_ARG           # byte scales: 16-byte aligned

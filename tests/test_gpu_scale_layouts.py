@@ -175,3 +175,30 @@ def test_mn_major_fp8_scales_feed_blockwise_gemm():
     mag_ref = deq.abs() @ wdeq.abs().t()
     err = (out.float().cpu().to(torch.float64) - ref).abs()
     assert (err <= 2.0**-8 * ref.abs() + 2.0**-14 * mag_ref).all()
+
+
+@pytest.mark.parametrize("layout", [0, 1, 3])
+@pytest.mark.parametrize("case", CASES, ids=[f"{w.name}-a{a}" for w, a, _ in CASES])
+def test_ue8m0_parity(case, layout):
+    """FP8 with power-of-two (UE8M0) 1x128 scales, row-major, MN-major and
+    packed MN-major scales, against the oracle over whole zeroed buffers."""
+    from combine_moe_topk_gate_b200 import api
+    w, align, frac = case
+    dev = torch.device("cuda", 0)
+    inp, L, rows = _routed(w, align, frac, seed=8)
+    g = torch.Generator().manual_seed(3)
+    x = (inp.x.float() * torch.exp2(torch.randint(-30, 20, (w.N, w.H // 128), generator=g).float())
+         .repeat_interleave(128, 1)).to(torch.bfloat16)
+    x[0] = 0.0
+    code = api.MOE_DTYPE_FP8_E4M3_UE8M0
+    shape, sdt = api.scale_shape(rows, w.H, code, layout)
+    sc = torch.zeros(shape, dtype=sdt, device=dev)
+    rx = torch.zeros((rows, w.H), dtype=torch.uint8, device=dev)
+    api.moe_dispatch(x.to(dev), L.token_slot, code, recv_x=rx, recv_scale=sc, num_recv_rows=rows,
+                     scale_layout=layout, d_status=L.status)
+    torch.cuda.synchronize()
+    assert int(L.status.item()) == 0
+    r_recv, r_sc, st = O.dispatch_scaled(bf16_bits(x), L.token_slot.cpu().numpy(), code, layout, recv_rows=rows)
+    assert st == 0
+    assert np.array_equal(rx.cpu().numpy(), r_recv)
+    assert np.array_equal(sc.cpu().numpy().reshape(-1), r_sc.reshape(-1))
