@@ -107,7 +107,13 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
     if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
     if constexpr (!UE8M0) {
-      if (active && (lane & 7) == 0) recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
+      if (active && (lane & 7) == 0) {
+        if constexpr (SL == MOE_SCALE_ROW_MAJOR)
+          recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
+        else
+          st_keep_b32(recv_scale + scale_at<SL>(slot, c0 >> 7, nblk, ld), __float_as_uint(scale),
+                      l2_evict_last_policy());
+      }
     } else {
       uint8_t* sb = reinterpret_cast<uint8_t*>(recv_scale);
       if constexpr (SL == MOE_SCALE_MN_MAJOR_PACK4) {
@@ -210,11 +216,11 @@ __global__ void __launch_bounds__(kWarps * 32)
       const int b0 = s * 16 + 4 * lane;
       if (lane < 4 && b0 < nblk) {
         const uint32_t word = lane == 0 ? sw[0] : lane == 1 ? sw[1] : lane == 2 ? sw[2] : sw[3];
-        *reinterpret_cast<uint32_t*>(recv_e8m0 + scale_at<SL>(slot, b0, nblk, ld)) = word;
+        st_keep_b32(recv_e8m0 + scale_at<SL>(slot, b0, nblk, ld), word, l2_evict_last_policy());
       }
     } else {
       if (active && (lane & 1) == 0)
-        recv_e8m0[scale_at<SL>(slot, c0 >> 5, nblk, ld)] = static_cast<uint8_t>(my_byte);
+        st_keep_b8(recv_e8m0 + scale_at<SL>(slot, c0 >> 5, nblk, ld), my_byte, l2_evict_last_policy());
     }
   }
 }

@@ -148,6 +148,22 @@ __device__ __forceinline__ float e4m3_value(uint32_t c) {
   return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : __fmul_rn(static_cast<float>(m), 0x1p-9f);
 }
 
+// ---------------------------------------------------------------- L2 policy
+// Scale tables written in pieces (MN-major, tiled): keep their lines in L2
+// (evict-last) until every piece has arrived, so that the stream of payload
+// stores does not push half-written sectors out to DRAM.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void st_keep_b32(void* ptr, uint32_t v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol));
+}
+__device__ __forceinline__ void st_keep_b8(void* ptr, uint32_t v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.b8 [%0], %1, %2;" ::"l"(ptr), "r"(v), "l"(pol));
+}
+
 // ---------------------------------------------------------------- memory
 // Read-once streaming load of 16 bytes: not kept in L1 (the rows of x in
 // dispatch and y in combine are touched by exactly one warp).
