@@ -79,10 +79,16 @@ __global__ void __launch_bounds__(kThreads)
   const uint16_t* col = x + c0;
   const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
 
-  // pass 1: amax of the lane's 8 channels over the warp's rows
-  float m[8];
+  // pass 1: amax of the lane's 8 channels over the warp's rows, on packed
+  // bf16 pairs (|x| and max are exact in bf16, so the result is the fp32 amax)
+  __nv_bfloat162 m2[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = 0.0f;
+  for (int j = 0; j < 4; ++j) m2[j] = __floats2bfloat162_rn(0.0f, 0.0f);
+  auto fold = [&](uint4 v) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m2[j] = __hmax2(m2[j], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
+  };
   if (active) {
     long long s = r0 + warp;
     for (; s + 7 * kWarpsPerCta < r1; s += 8 * kWarpsPerCta) {
@@ -90,27 +96,15 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
       for (int u = 0; u < 8; ++u) v[u] = ld_hint(col + static_cast<size_t>(s + u * kWarpsPerCta) * H, keep);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          m[2 * j] = fmaxf(m[2 * j], fabsf(bf16_lo(w[j])));
-          m[2 * j + 1] = fmaxf(m[2 * j + 1], fabsf(bf16_hi(w[j])));
-        }
-      }
+      for (int u = 0; u < 8; ++u) fold(v[u]);
     }
-    for (; s < r1; s += kWarpsPerCta) {
-      const uint4 v = ld_hint(col + static_cast<size_t>(s) * H, keep);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        m[2 * j] = fmaxf(m[2 * j], fabsf(bf16_lo(w[j])));
-        m[2 * j + 1] = fmaxf(m[2 * j + 1], fabsf(bf16_hi(w[j])));
-      }
-    }
+    for (; s < r1; s += kWarpsPerCta) fold(ld_hint(col + static_cast<size_t>(s) * H, keep));
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) part[warp][lane * 8 + i] = m[i];
+  for (int j = 0; j < 4; ++j) {
+    part[warp][lane * 8 + 2 * j] = __low2float(m2[j]);
+    part[warp][lane * 8 + 2 * j + 1] = __high2float(m2[j]);
+  }
   __syncthreads();
   {
     const int c = tid;  // kThreads == kSlab: one channel per thread
@@ -122,21 +116,34 @@ __global__ void __launch_bounds__(kThreads)
   }
   __syncthreads();
   float inv[8];
+  bool finite = true;  // every 448/amax of the lane finite: products keep zero signs
 #pragma unroll
-  for (int i = 0; i < 8; ++i) inv[i] = inv_s[lane * 8 + i];
+  for (int i = 0; i < 8; ++i) {
+    inv[i] = inv_s[lane * 8 + i];
+    finite = finite && inv[i] <= 3.402823466e38f;
+  }
 
-  // pass 2: codes of one row's 8 channels
+  // pass 2: codes of one row's 8 channels (x * inv of finite bf16 is never
+  // NaN, so the encoder without NaN handling gives the same codes)
   auto codes_of_v = [&](uint4 v) -> uint2 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float p[8];
+    if (finite) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float lo = bf16_lo(w[j]), hi = bf16_hi(w[j]);
-      p[2 * j] = (lo == 0.0f) ? lo : __fmul_rn(lo, inv[2 * j]);
-      p[2 * j + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, inv[2 * j + 1]);
+      for (int j = 0; j < 4; ++j) {
+        p[2 * j] = __fmul_rn(bf16_lo(w[j]), inv[2 * j]);
+        p[2 * j + 1] = __fmul_rn(bf16_hi(w[j]), inv[2 * j + 1]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = bf16_lo(w[j]), hi = bf16_hi(w[j]);
+        p[2 * j] = (lo == 0.0f) ? lo : __fmul_rn(lo, inv[2 * j]);
+        p[2 * j + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, inv[2 * j + 1]);
+      }
     }
-    return make_uint2(e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16),
-                      e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16));
+    return make_uint2(e4m3x2_nonan(p[0], p[1]) | (e4m3x2_nonan(p[2], p[3]) << 16),
+                      e4m3x2_nonan(p[4], p[5]) | (e4m3x2_nonan(p[6], p[7]) << 16));
   };
   auto codes_of = [&](long long s) -> uint2 { return codes_of_v(ld_hint(col + static_cast<size_t>(s) * H, done)); };
   if constexpr (!TRANSPOSE) {

@@ -38,6 +38,7 @@ def test_quant_fp8_channel_parity(case, transpose):
     g = torch.Generator().manual_seed(9)
     recv = torch.randn(rows, w.H, generator=g) * torch.exp2(torch.randint(-12, 12, (1, w.H), generator=g).float())
     recv[:, 3] = 0.0
+    recv[:, 7] = torch.randn(rows, generator=g) * 1e-39     # a channel of bf16 subnormals only
     landed = (L.slot_token >= 0).cpu()
     recv[~landed] = float("inf")
     recv = recv.to(torch.bfloat16)
