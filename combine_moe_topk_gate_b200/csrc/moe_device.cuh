@@ -49,9 +49,10 @@ __device__ __forceinline__ float fixed_exp(float y) {
   return __fmul_rn(p, two_n);
 }
 
-// 1 / (1 + e^-x), each operation rounded once.
+// 1 / (1 + e^-x), each operation rounded once (the correctly rounded
+// reciprocal is the correctly rounded quotient 1 / d).
 __device__ __forceinline__ float logistic(float x) {
-  return __fdiv_rn(1.0f, __fadd_rn(1.0f, fixed_exp(-x)));
+  return __frcp_rn(__fadd_rn(1.0f, fixed_exp(-x)));
 }
 
 // ---------------------------------------------------------------- bf16
