@@ -229,12 +229,85 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 }
 
+// Small batches (N*k <= kSmallEntries, the decode-sized ones): one warp per
+// (token, 256 channels), each lane 8 channels.  The lane loads its 16 bytes of
+// all k rows at once -- one memory round trip instead of the pipeline's
+// copy-then-fold per item -- and folds them in slot order exactly as the
+// pipelined kernel does (acc = fma(w_j, y_j, acc), invalid slots skipped).
+constexpr int kSmallEntries = 4096;
+constexpr int kSmallWarps = 8;
+
+__global__ void __launch_bounds__(kSmallWarps * 32)
+    combine_regs_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
+                        const int32_t* __restrict__ token_slot, long long S,
+                        const float* __restrict__ topk_w, uint16_t* __restrict__ out,
+                        int32_t* d_status) {
+  const int lane = threadIdx.x & 31;
+  const int segs = (H + 255) / 256;
+  const int item = blockIdx.x * kSmallWarps + (threadIdx.x >> 5);  // N*k <= 4096: fits an int
+  const int t = item / segs;
+  if (t >= N) return;
+  const int s = item - t * segs;
+  const int c0 = s * 256 + lane * 8;
+  const bool active = c0 < H;  // H % 8 == 0
+  pdl_wait();
+  pdl_trigger();
+  int my_slot = -1;
+  float my_w = 0.0f;
+  if (lane < k) {
+    my_slot = token_slot[static_cast<size_t>(t) * k + lane];
+    my_w = topk_w ? topk_w[static_cast<size_t>(t) * k + lane] : 1.0f;
+    if (s == 0 && (my_slot < -1 || my_slot >= S)) report_bad_index(d_status);
+  }
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+  for (int j0 = 0; j0 < k; j0 += 8) {
+    uint4 v[8];
+    int slot[8];
+    float w[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      slot[q] = __shfl_sync(kFullMask, my_slot, (j0 + q) & 31);
+      w[q] = __shfl_sync(kFullMask, my_w, (j0 + q) & 31);
+      const bool ok = j0 + q < k && slot[q] >= 0 && slot[q] < S;
+      if (!ok) slot[q] = -1;
+      v[q] = make_uint4(0, 0, 0, 0);
+      if (ok && active) v[q] = ld_stream(y + static_cast<size_t>(slot[q]) * H + c0);
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (slot[q] < 0) continue;
+      const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc[2 * i] = __fmaf_rn(w[q], bf16_lo(w4[i]), acc[2 * i]);
+        acc[2 * i + 1] = __fmaf_rn(w[q], bf16_hi(w4[i]), acc[2 * i + 1]);
+      }
+    }
+  }
+  if (active) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    st_stream_v4(out + static_cast<size_t>(t) * H + c0, o);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
                            long long num_rows, const float* topk_w, void* out, int32_t* d_status,
                            cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
+  if (static_cast<long long>(N) * k <= kSmallEntries) {
+    const int items = N * ((H + 255) / 256);
+    return launch_pdl(combine_regs_kernel, static_cast<unsigned>((items + kSmallWarps - 1) / kSmallWarps),
+                      kSmallWarps * 32, 0, stream, static_cast<const uint16_t*>(y), N, H, k, token_slot,
+                      num_rows, topk_w, static_cast<uint16_t*>(out), d_status);
+  }
   const Layout L = smem_layout(k);
   cudaError_t err = cudaFuncSetAttribute(combine_bulk_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
