@@ -296,104 +296,135 @@ __global__ void __launch_bounds__(kTokenThreads)
   }
 }
 
-// NVFP4: one CTA per token, one 16-channel block per thread vector (VPT per
-// thread).  Row amax over the CTA, then per block: sb = e4m3((amax_b / 6) *
-// (2688 / amax_row)), r = (2688 / amax_row) / value(sb), codes e2m1(x * r);
-// row scale g = amax_row / 2688.  Four neighbouring threads hold four
-// consecutive blocks, so their scale bytes go out as one 32-bit word
-// (H % 64 == 0).
-template <int VPT, int SL>
-__global__ void __launch_bounds__(kTokenThreads)
+// NVFP4: one 128-thread CTA per token.  One thread copies the token's row
+// into shared memory with a 1-D bulk copy (no tensor map, no multicast) that
+// completes on an mbarrier; the CTA then works from shared memory, so the row
+// does not occupy registers and about 15 tokens fit per SM.  Each thread owns
+// the 16-channel blocks tid, tid + 128, ... (BPT of them): block maxima, the
+// CTA-wide row amax (row scale g = amax / 2688, inv = 2688 / amax), then per
+// block sb = e4m3((amax_b / 6) * inv), r = inv / value(sb), codes e2m1(x * r).
+// Four neighbouring threads hold four consecutive blocks, so their scale
+// bytes leave as one 32-bit word (H % 64 == 0).  The copy's wait is bounded
+// (MOE_ERR_TIMEOUT).
+constexpr int kNvThreads = 128;
+
+template <int BPT, int SL>
+__global__ void __launch_bounds__(kNvThreads)
     dispatch_nvfp4_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                           const int32_t* __restrict__ token_slot, long long S,
                           uint8_t* __restrict__ recv_x, uint8_t* __restrict__ block_scale,
                           float* __restrict__ row_scale, long long ld, int32_t* d_status) {
-  __shared__ float warp_max[kTokenThreads / 32];
+  extern __shared__ __align__(128) unsigned char smem[];  // mbarrier at 0, the row from 128
+  __shared__ float warp_max[kNvThreads / 32];
   __shared__ int slots[MOE_MAX_TOPK];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
-  const int nvec = H / 16, B = H / 16;
+  const int nb = H / 16;
+  const uint32_t bar = smem_addr(smem);
+  const uint32_t row = smem_addr(smem + 128);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(H) * 2u);
+    bulk_g2s(row, x + static_cast<size_t>(t) * H, static_cast<uint32_t>(H) * 2u, bar);
+  }
   if (tid < k) {
     const int sl = token_slot[static_cast<size_t>(t) * k + tid];
     slots[tid] = sl;
     if (sl < -1 || sl >= S) report_bad_index(d_status);
   }
-  // the raw bf16 words stay live across the row reduction (8 registers per
-  // block rather than 16 unpacked floats)
-  uint4 va[VPT], vb[VPT];
-  float bmax[VPT];
+  // one thread takes the bounded wait, so the give-up decision is the same
+  // for the whole CTA (no thread may leave while others reach a barrier);
+  // after it every thread observes the completed phase, which makes the
+  // copied bytes visible to it
+  __shared__ int copy_ok;
+  if (tid == 0) {
+    copy_ok = mbar_wait(bar, 0) ? 1 : 0;
+    if (!copy_ok) {
+      report_timeout(d_status);
+      mbar_wait(bar, 0);  // bounded again: the copy must land before the CTA may exit
+    }
+  }
+  __syncthreads();
+  if (!copy_ok) return;
+  mbar_wait(bar, 0);  // the phase has completed: returns at once (and is bounded regardless)
+
+  float bmax[BPT];
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int vi = i * kTokenThreads + tid;
-    va[i] = make_uint4(0, 0, 0, 0);
-    vb[i] = va[i];
-    if (vi < nvec) {
-      const uint16_t* src = x + static_cast<size_t>(t) * H + static_cast<size_t>(vi) * 16;
-      va[i] = ld_stream(src);
-      vb[i] = ld_stream(src + 8);
-    }
-    const uint32_t w[8] = {va[i].x, va[i].y, va[i].z, va[i].w, vb[i].x, vb[i].y, vb[i].z, vb[i].w};
+  for (int i = 0; i < BPT; ++i) {
+    const int b = tid + i * kNvThreads;
     bmax[i] = 0.0f;
+    if (b < nb) {
+      const uint4 va = ld_shared_v4(row + b * 32), vb = ld_shared_v4(row + b * 32 + 16);
+      const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
-      bmax[i] = fmaxf(bmax[i], fmaxf(fabsf(bf16_lo(w[u])), fabsf(bf16_hi(w[u]))));
+      for (int u = 0; u < 8; ++u) bmax[i] = fmaxf(bmax[i], fmaxf(fabsf(bf16_lo(w[u])), fabsf(bf16_hi(w[u]))));
+    }
     amax = fmaxf(amax, bmax[i]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
   if (lane == 0) warp_max[warp] = amax;
   __syncthreads();
-  amax = warp_max[0];
-#pragma unroll
-  for (int w2 = 1; w2 < kTokenThreads / 32; ++w2) amax = fmaxf(amax, warp_max[w2]);
+  amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
   const float g = __fdiv_rn(amax, 2688.0f);
   const float inv = __fdiv_rn(2688.0f, amax);
-  uint2 q[VPT];
-  uint32_t sword[VPT];
+  uint2 q[BPT];
+  uint32_t sword[BPT];
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
+  for (int i = 0; i < BPT; ++i) {
+    const int b = tid + i * kNvThreads;
     const float sbf = __fmul_rn(__fdiv_rn(bmax[i], 6.0f), inv);
     const uint32_t sb = bmax[i] > 0.0f ? (e4m3x2(sbf, 0.0f) & 0xffu) : 0u;
-    const float r = __fdiv_rn(inv, e4m3_value(sb));
-    const uint32_t w[8] = {va[i].x, va[i].y, va[i].z, va[i].w, vb[i].x, vb[i].y, vb[i].z, vb[i].w};
-    float f[16];
+    q[i] = make_uint2(0, 0);
+    if (b < nb) {
+      const float r = __fdiv_rn(inv, e4m3_value(sb));
+      const uint4 va = ld_shared_v4(row + b * 32), vb = ld_shared_v4(row + b * 32 + 16);
+      const uint32_t w[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+      float p[16];
+      if (r <= 3.402823466e38f) {  // finite: the product keeps a zero's sign
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      f[2 * u] = bf16_lo(w[u]);
-      f[2 * u + 1] = bf16_hi(w[u]);
+        for (int u = 0; u < 8; ++u) {
+          p[2 * u] = __fmul_rn(bf16_lo(w[u]), r);
+          p[2 * u + 1] = __fmul_rn(bf16_hi(w[u]), r);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float lo = bf16_lo(w[u]), hi = bf16_hi(w[u]);
+          p[2 * u] = (lo == 0.0f) ? lo : __fmul_rn(lo, r);
+          p[2 * u + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, r);
+        }
+      }
+      q[i] = make_uint2(e2m1x8(p), e2m1x8(p + 8));
     }
-    float p[16];
-    if (r <= 3.402823466e38f) {  // finite: the product keeps a zero's sign
-#pragma unroll
-      for (int u = 0; u < 16; ++u) p[u] = __fmul_rn(f[u], r);
-    } else {
-#pragma unroll
-      for (int u = 0; u < 16; ++u) p[u] = (f[u] == 0.0f) ? f[u] : __fmul_rn(f[u], r);
-    }
-    q[i] = make_uint2(e2m1x8(p), e2m1x8(p + 8));
-    // bytes of blocks vi..vi+3 (threads lane..lane+3) into lane % 4 == 0
+    // bytes of blocks b..b+3 (threads tid..tid+3) into tid % 4 == 0
     uint32_t word = sb;
     word |= (__shfl_down_sync(kFullMask, sb, 1) & 0xffu) << 8;
     word |= (__shfl_down_sync(kFullMask, sb, 2) & 0xffu) << 16;
     word |= (__shfl_down_sync(kFullMask, sb, 3) & 0xffu) << 24;
     sword[i] = SL == MOE_SCALE_MN_MAJOR ? sb : word;
   }
+  const size_t row_bytes = static_cast<size_t>(H) / 2;
   for (int j = 0; j < k; ++j) {
     const int slot = slots[j];
     if (slot < 0 || slot >= S) continue;
-    uint8_t* row = recv_x + static_cast<size_t>(slot) * (H / 2);
+    uint8_t* dst = recv_x + static_cast<size_t>(slot) * row_bytes;
 #pragma unroll
-    for (int i = 0; i < VPT; ++i) {
-      const int vi = i * kTokenThreads + tid;
-      if (vi < nvec) {
-        *reinterpret_cast<uint2*>(row + static_cast<size_t>(vi) * 8) = q[i];
+    for (int i = 0; i < BPT; ++i) {
+      const int b = tid + i * kNvThreads;
+      if (b < nb) {
+        *reinterpret_cast<uint2*>(dst + static_cast<size_t>(b) * 8) = q[i];
         if constexpr (SL == MOE_SCALE_MN_MAJOR) {
-          block_scale[scale_at<SL>(slot, vi, B, ld)] = static_cast<uint8_t>(sword[i]);
-        } else if ((lane & 3) == 0) {
-          *reinterpret_cast<uint32_t*>(block_scale + scale_at<SL>(slot, vi, B, ld)) = sword[i];
+          block_scale[scale_at<SL>(slot, b, nb, ld)] = static_cast<uint8_t>(sword[i]);
+        } else if ((tid & 3) == 0) {
+          *reinterpret_cast<uint32_t*>(block_scale + scale_at<SL>(slot, b, nb, ld)) = sword[i];
         }
       }
     }
@@ -593,19 +624,31 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   }
 }
 
+template <int BPT, int SL>
+cudaError_t launch_nvfp4_bpt(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                             long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
+                             float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
+  const size_t smem = 128 + static_cast<size_t>(H) * 2;  // H <= 16384: at most 32 KB + 128
+  return launch_pdl(dispatch_nvfp4_kernel<BPT, SL>, N, kNvThreads, smem, stream, x, N, H, k,
+                    token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
+}
+
 template <int SL>
 cudaError_t launch_nvfp4(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                          long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
                          float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
-  const int vpt = (H / 16 + kTokenThreads - 1) / kTokenThreads;
-  if (vpt <= 1)
-    return launch_pdl(dispatch_nvfp4_kernel<1, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
-                      token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
-  if (vpt <= 2)
-    return launch_pdl(dispatch_nvfp4_kernel<2, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
-                      token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
-  return launch_pdl(dispatch_nvfp4_kernel<4, SL>, N, kTokenThreads, 0, stream, x, N, H, k,
-                    token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
+  const int bpt = (H / 16 + kNvThreads - 1) / kNvThreads;  // blocks per thread, <= 8
+  if (bpt <= 1)
+    return launch_nvfp4_bpt<1, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
+                                   d_status, stream);
+  if (bpt <= 2)
+    return launch_nvfp4_bpt<2, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
+                                   d_status, stream);
+  if (bpt <= 4)
+    return launch_nvfp4_bpt<4, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
+                                   d_status, stream);
+  return launch_nvfp4_bpt<8, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
+                                 d_status, stream);
 }
 
 cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int32_t* token_slot,
