@@ -190,14 +190,14 @@ __global__ void __launch_bounds__(kLayoutThreads)
     e = topk_idx[t0 * k + tid];
     b = bucket_of(e, E);
   }
-  // 1. column sums over chunks: all chunks (totals) and chunks before c.  All
-  //    threads load the C x nb counts in one pass (one L2 round trip) and add
-  //    them into shared memory.
-  for (int i = tid; i < nb; i += kLayoutThreads) off[i] = base[i] = 0;
-  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
+  // 1. column sums over chunks: all chunks (totals) and chunks before c,
+  //    without atomics.  P threads per bucket each add a contiguous range of
+  //    chunks (independent L2 loads); their partials go to shared memory (the
+  //    warp-count array, zeroed only after) and one thread per bucket folds
+  //    them.
   for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
-  __syncthreads();
   if (c == 0) {  // block-uniform: CTA 0 also sums the per-chunk tokens per rank
+    __syncthreads();
     const int total_vals = C * R;
     for (int i = tid; i < total_vals; i += kLayoutThreads) {
       const int v = chunk_rtok[i];
@@ -205,25 +205,35 @@ __global__ void __launch_bounds__(kLayoutThreads)
     }
   }
   {
-    const int total_vals = C * nb;
-    constexpr int kBatch = 16;
-    for (int i0 = 0; i0 < total_vals; i0 += kBatch * kLayoutThreads) {
-      int v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * kLayoutThreads + tid;
-        v[u] = i < total_vals ? chunk_counts[i] : 0;
+    const int P = min(16, max(1, kLayoutThreads / nb));  // 2 * nb * P <= kLayoutWarps * nb
+    const int Lc = (C + P - 1) / P;
+    int32_t* ptot = wcnt;           // [nb][P] partial totals
+    int32_t* ppre = wcnt + nb * P;  // [nb][P] partial sums of the chunks before c
+    for (int item = tid; item < nb * P; item += kLayoutThreads) {
+      const int bb = item / P, p = item - bb * P;
+      const int ca = p * Lc, cb = min(C, ca + Lc);
+      int tot = 0, pre = 0;
+#pragma unroll 4
+      for (int cc = ca; cc < cb; ++cc) {
+        const int v = chunk_counts[static_cast<size_t>(cc) * nb + bb];
+        tot += v;
+        pre += cc < c ? v : 0;
       }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * kLayoutThreads + tid;
-        if (v[u] != 0) {
-          const int cc = i / nb, bb = i - cc * nb;
-          atomicAdd(&off[bb], v[u]);
-          if (cc < c) atomicAdd(&base[bb], v[u]);
-        }
-      }
+      ptot[item] = tot;
+      ppre[item] = pre;
     }
+    __syncthreads();
+    for (int bb = tid; bb < nb; bb += kLayoutThreads) {
+      int tot = 0, pre = 0;
+      for (int p = 0; p < P; ++p) {
+        tot += ptot[bb * P + p];
+        pre += ppre[bb * P + p];
+      }
+      off[bb] = tot;
+      base[bb] = pre;
+    }
+    __syncthreads();
+    for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
   }
   __syncthreads();
   // 2. bucket offsets (experts aligned), unused rows marked
