@@ -69,6 +69,8 @@ def _load() -> ctypes.CDLL:
     L.moe_recv_scale_bytes.restype = SZ
     L.moe_dispatch_nvfp4.argtypes = [P, I, I, I, P, I, I, P, P, P, P, P]
     L.moe_dispatch_nvfp4.restype = I
+    L.moe_selftest_bounded_wait.argtypes = [P, P]
+    L.moe_selftest_bounded_wait.restype = I
     L.moe_quant_fp8_channel.argtypes = [P, I, I, I, P, P, I, P, P, P, P]
     L.moe_quant_fp8_channel.restype = I
     L.moe_swiglu_quant.argtypes = [P, I, I, P, I, I, P, P, P]
@@ -343,6 +345,14 @@ def moe_dispatch_nvfp4(x: torch.Tensor, token_slot: torch.Tensor, *, scale_layou
                                  _ptr(block_scale), _ptr(row_scale), _ptr(d_status), _stream(stream, x.device))
     _check(st, "moe_dispatch_nvfp4")
     return recv_x, block_scale, row_scale
+
+
+def moe_selftest_bounded_wait(d_status: torch.Tensor, stream=None) -> None:
+    """Runs the pipelined kernels' bounded wait on an mbarrier nothing completes;
+    after about a second MOE_ERR_TIMEOUT is recorded in ``d_status``."""
+    _need(d_status, "d_status", torch.int32, (1,))
+    _check(_lib.moe_selftest_bounded_wait(_ptr(d_status), _stream(stream, d_status.device)),
+           "moe_selftest_bounded_wait")
 
 
 def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, expert_count: torch.Tensor, *,

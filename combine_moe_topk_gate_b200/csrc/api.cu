@@ -175,6 +175,11 @@ size_t moe_recv_scale_bytes(int num_recv_rows, int hidden, moe_dtype_t dtype,
   }
 }
 
+moe_status_t moe_selftest_bounded_wait(int32_t* d_status, moe_stream_t stream) {
+  if (!d_status || !aligned(d_status, 4)) return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_bounded_wait_selftest(d_status, as_stream(stream)));
+}
+
 moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,
                                    const int32_t* expert_offset, const int32_t* expert_count,
                                    int transpose, void* out, float* scale, int32_t* d_status,

@@ -225,10 +225,14 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-// FP8 with one scale per token: one CTA per token, the row held in registers
-// (VPT 16-byte vectors per thread), amax reduced over the CTA, then the same
-// code rule as the blocks: scale = amax/448, codes e4m3(x * (448/amax)).
-constexpr int kTokenThreads = 256;
+// FP8 with one scale per token: one 128-thread CTA per token.  One thread
+// copies the row into shared memory with a 1-D bulk copy (no tensor map, no
+// multicast) completing on an mbarrier; the CTA reduces the row amax from
+// shared memory and codes its VPT 8-channel vectors per thread with the
+// block rule: scale = amax/448, codes e4m3(x * (448/amax)).  The row does not
+// occupy registers, so many tokens are in flight per SM.  The copy's wait is
+// bounded (MOE_ERR_TIMEOUT), the give-up decision taken by one thread.
+constexpr int kTokenThreads = 128;
 
 template <int VPT>
 __global__ void __launch_bounds__(kTokenThreads)
@@ -236,61 +240,89 @@ __global__ void __launch_bounds__(kTokenThreads)
                               const int32_t* __restrict__ token_slot, long long S,
                               uint8_t* __restrict__ recv_x, float* __restrict__ recv_scale,
                               int32_t* d_status) {
+  extern __shared__ __align__(128) unsigned char smem[];  // mbarrier at 0, the row from 128
   __shared__ float warp_max[kTokenThreads / 32];
   __shared__ int slots[MOE_MAX_TOPK];
+  __shared__ int copy_ok;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
   const int nvec = H / 8;
+  const uint32_t bar = smem_addr(smem);
+  const uint32_t row = smem_addr(smem + 128);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init_fence();
+  }
+  __syncthreads();
   pdl_wait();
   pdl_trigger();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(H) * 2u);
+    bulk_g2s(row, x + static_cast<size_t>(t) * H, static_cast<uint32_t>(H) * 2u, bar);
+  }
   if (tid < k) {
     const int sl = token_slot[static_cast<size_t>(t) * k + tid];
     slots[tid] = sl;
     if (sl < -1 || sl >= S) report_bad_index(d_status);
   }
-  uint4 v[VPT];
+  if (tid == 0) {
+    copy_ok = mbar_wait(bar, 0) ? 1 : 0;
+    if (!copy_ok) {
+      report_timeout(d_status);
+      mbar_wait(bar, 0);  // bounded again: the copy must land before the CTA may exit
+    }
+  }
+  __syncthreads();
+  if (!copy_ok) return;
+  mbar_wait(bar, 0);  // the phase has completed: returns at once (and is bounded regardless)
+
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int vi = i * kTokenThreads + tid;
-    v[i] = make_uint4(0, 0, 0, 0);
-    if (vi < nvec) v[i] = ld_stream(x + static_cast<size_t>(t) * H + static_cast<size_t>(vi) * 8);
-    const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+    if (vi < nvec) {
+      const uint4 v = ld_shared_v4(row + vi * 16);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[u])), fabsf(bf16_hi(w4[u]))));
+      for (int u = 0; u < 4; ++u)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[u])), fabsf(bf16_hi(w4[u]))));
+    }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
   if (lane == 0) warp_max[warp] = amax;
   __syncthreads();
-  amax = warp_max[0];
-#pragma unroll
-  for (int w2 = 1; w2 < kTokenThreads / 32; ++w2) amax = fmaxf(amax, warp_max[w2]);
+  amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
   const float inv = __fdiv_rn(448.0f, amax);
   const float scale = __fdiv_rn(amax, 448.0f);
+  const bool finite = inv <= 3.402823466e38f;  // then the product keeps a zero's sign
   uint2 q[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
-    const uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-    float p[8];
+    const int vi = i * kTokenThreads + tid;
+    q[i] = make_uint2(0, 0);
+    if (vi < nvec) {
+      const uint4 v = ld_shared_v4(row + vi * 16);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      float p[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float lo = bf16_lo(w4[u]), hi = bf16_hi(w4[u]);
-      p[2 * u] = (lo == 0.0f) ? lo : __fmul_rn(lo, inv);
-      p[2 * u + 1] = (hi == 0.0f) ? hi : __fmul_rn(hi, inv);
+      for (int u = 0; u < 4; ++u) {
+        const float lo = bf16_lo(w4[u]), hi = bf16_hi(w4[u]);
+        p[2 * u] = (finite || lo != 0.0f) ? __fmul_rn(lo, inv) : lo;
+        p[2 * u + 1] = (finite || hi != 0.0f) ? __fmul_rn(hi, inv) : hi;
+      }
+      q[i].x = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+      q[i].y = e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16);
     }
-    q[i].x = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
-    q[i].y = e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16);
   }
   for (int j = 0; j < k; ++j) {
     const int slot = slots[j];
     if (slot < 0 || slot >= S) continue;
-    uint8_t* row = recv_x + static_cast<size_t>(slot) * H;
+    uint8_t* dst = recv_x + static_cast<size_t>(slot) * H;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int vi = i * kTokenThreads + tid;
-      if (vi < nvec) *reinterpret_cast<uint2*>(row + static_cast<size_t>(vi) * 8) = q[i];
+      if (vi < nvec) *reinterpret_cast<uint2*>(dst + static_cast<size_t>(vi) * 8) = q[i];
     }
     if (tid == 0) recv_scale[slot] = scale;
   }
@@ -597,18 +629,20 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_ROW_MAJOR>, blocks, kWarps * 32, 0, stream,
                       xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
   } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
+    // vectors of 8 channels per thread; H <= 16384 -> at most 16
     const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
     float* sc = static_cast<float*>(recv_scale);
-    if (vpt <= 1)
-      return launch_pdl(dispatch_fp8_token_kernel<1>, N, kTokenThreads, 0, stream, xs, N, H, k,
-                        token_slot, num_rows, r8, sc, d_status);
+    const size_t smem = 128 + static_cast<size_t>(H) * 2;
     if (vpt <= 2)
-      return launch_pdl(dispatch_fp8_token_kernel<2>, N, kTokenThreads, 0, stream, xs, N, H, k,
+      return launch_pdl(dispatch_fp8_token_kernel<2>, N, kTokenThreads, smem, stream, xs, N, H, k,
                         token_slot, num_rows, r8, sc, d_status);
     if (vpt <= 4)
-      return launch_pdl(dispatch_fp8_token_kernel<4>, N, kTokenThreads, 0, stream, xs, N, H, k,
+      return launch_pdl(dispatch_fp8_token_kernel<4>, N, kTokenThreads, smem, stream, xs, N, H, k,
                         token_slot, num_rows, r8, sc, d_status);
-    return launch_pdl(dispatch_fp8_token_kernel<8>, N, kTokenThreads, 0, stream, xs, N, H, k,
+    if (vpt <= 8)
+      return launch_pdl(dispatch_fp8_token_kernel<8>, N, kTokenThreads, smem, stream, xs, N, H, k,
+                        token_slot, num_rows, r8, sc, d_status);
+    return launch_pdl(dispatch_fp8_token_kernel<16>, N, kTokenThreads, smem, stream, xs, N, H, k,
                       token_slot, num_rows, r8, sc, d_status);
   } else if (dtype == MOE_DTYPE_E5M6) {
     const long long items = static_cast<long long>(N) * ((H + 511) / 512);

@@ -35,6 +35,7 @@ cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, i
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,
                                      cudaStream_t stream);
+cudaError_t launch_bounded_wait_selftest(int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_swiglu_quant(const void* h, long long num_rows, int I, const int32_t* slot_token,
                                 int dtype, int scale_layout, void* out, void* out_scale,
                                 cudaStream_t stream);

@@ -454,6 +454,16 @@ moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(moe_status_t status);
 
+/*
+ * moe_selftest_bounded_wait -- diagnostics: runs the bounded wait that the
+ * pipelined kernels (combine, combine backward, NVFP4 dispatch) use on an
+ * mbarrier that nothing completes.  After about one second the wait gives up
+ * and MOE_ERR_TIMEOUT is recorded in *d_status (device memory, 4-byte
+ * aligned), exactly as a kernel whose copy never lands would report it; the
+ * context stays usable.  No fault, trap or hang is involved.
+ */
+moe_status_t moe_selftest_bounded_wait(int32_t* d_status, moe_stream_t stream);
+
 /* ABI version: bumped when a signature or a documented behaviour changes. */
 int moe_abi_version(void);
 

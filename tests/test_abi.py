@@ -278,3 +278,9 @@ def test_ue8m0_and_pack4_sizes_and_validation(api):
     assert disp(FP8, P4) == api.MOE_ERR_INVALID_ARG
     assert disp(U8, 4) == api.MOE_ERR_INVALID_ARG
     assert disp(U8, 0, sc=_P(0x1004)) == api.MOE_ERR_INVALID_ARG           # byte scales: 16-byte aligned
+
+
+def test_selftest_rejects_bad_arguments(api):
+    L = api.lib()
+    assert L.moe_selftest_bounded_wait(None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_selftest_bounded_wait(_P(0x1002), None) == api.MOE_ERR_INVALID_ARG
