@@ -60,6 +60,10 @@ __device__ __forceinline__ void consumer_barrier() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumers) : "memory");
 }
 
+// KT > 0: k == KT is known at compile time (1, 2, 4 or 8), so the group holds
+// exactly 8 slots and the consumers keep 8 dot partials with constant indices;
+// KT == 0 serves any k (up to 32 slots per group).
+template <int KT>
 __global__ void __launch_bounds__(kThreads)
     combine_backward_bulk_kernel(const uint16_t* __restrict__ grad_out,
                                  const uint16_t* __restrict__ y, int N, int H, int k,
@@ -164,9 +168,10 @@ __global__ void __launch_bounds__(kThreads)
     int stage = 0;
     uint32_t phase = 0;
     const int c = threadIdx.x * 8;
-    float dot[32];
+    constexpr int kDots = KT > 0 ? (KT >= 8 ? KT : 8) : 32;  // >= TK
+    float dot[kDots];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) dot[q] = 0.0f;
+    for (int q = 0; q < kDots; ++q) dot[q] = 0.0f;
     bool failed = false;
     for (long long it = i0; it < i1; ++it) {
       const int g = static_cast<int>(it / segs);
@@ -181,38 +186,58 @@ __global__ void __launch_bounds__(kThreads)
       const uint32_t vmask = reinterpret_cast<const uint32_t*>(hw)[32];
       if (!failed && c < seg_ch) {
         const uint32_t st0 = data + static_cast<uint32_t>(stage * L.stage_bytes) + c * 2;
-        for (int u = 0; u < T; ++u) {
-          const int t = g * T + u;
-          if (t >= N) break;
+        // slot q of the group (token q / k): dot partial of grad_out . y, and
+        // grad_y = w * grad_out
+        auto slot_work = [&](int q, const float(&gf)[8]) {
+          const uint4 yv = ld_shared_v4(st0 + q * seg_bytes);
+          const uint32_t y4[4] = {yv.x, yv.y, yv.z, yv.w};
+          float d = dot[q];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            d = __fmaf_rn(gf[2 * i], bf16_lo(y4[i]), d);
+            d = __fmaf_rn(gf[2 * i + 1], bf16_hi(y4[i]), d);
+          }
+          dot[q] = d;
+          const float wq = hw[q];
+          const int slot = reinterpret_cast<const int32_t*>(hw)[64 + q];
+          uint4 o;
+          o.x = pack_bf16x2(__fmul_rn(wq, gf[0]), __fmul_rn(wq, gf[1]));
+          o.y = pack_bf16x2(__fmul_rn(wq, gf[2]), __fmul_rn(wq, gf[3]));
+          o.z = pack_bf16x2(__fmul_rn(wq, gf[4]), __fmul_rn(wq, gf[5]));
+          o.w = pack_bf16x2(__fmul_rn(wq, gf[6]), __fmul_rn(wq, gf[7]));
+          st_stream_v4(grad_y + static_cast<size_t>(slot) * H + static_cast<size_t>(s) * seg + c, o);
+        };
+        auto grad_row = [&](int u, float(&gf)[8]) {
           const uint4 gv = ld_shared_v4(st0 + (TK + u) * seg_bytes);
           const uint32_t g4[4] = {gv.x, gv.y, gv.z, gv.w};
-          float gf[8];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             gf[2 * i] = bf16_lo(g4[i]);
             gf[2 * i + 1] = bf16_hi(g4[i]);
           }
+        };
+        if constexpr (KT > 0) {
+          constexpr int TT = kDots / KT;  // == L.T
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
-            if (q >= TK) break;
-            if (q / k != u || !((vmask >> q) & 1u)) continue;
-            const uint4 yv = ld_shared_v4(st0 + q * seg_bytes);
-            const uint32_t y4[4] = {yv.x, yv.y, yv.z, yv.w};
-            float d = dot[q];
+          for (int u = 0; u < TT; ++u) {
+            if (g * TT + u >= N) break;
+            float gf[8];
+            grad_row(u, gf);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              d = __fmaf_rn(gf[2 * i], bf16_lo(y4[i]), d);
-              d = __fmaf_rn(gf[2 * i + 1], bf16_hi(y4[i]), d);
+            for (int j = 0; j < KT; ++j)
+              if ((vmask >> (u * KT + j)) & 1u) slot_work(u * KT + j, gf);
+          }
+        } else {
+          for (int u = 0; u < T; ++u) {
+            if (g * T + u >= N) break;
+            float gf[8];
+            grad_row(u, gf);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              if (q >= TK) break;
+              if (q / k != u || !((vmask >> q) & 1u)) continue;
+              slot_work(q, gf);
             }
-            dot[q] = d;
-            const float wq = hw[q];
-            const int slot = reinterpret_cast<const int32_t*>(hw)[64 + q];
-            uint4 o;
-            o.x = pack_bf16x2(__fmul_rn(wq, gf[0]), __fmul_rn(wq, gf[1]));
-            o.y = pack_bf16x2(__fmul_rn(wq, gf[2]), __fmul_rn(wq, gf[3]));
-            o.z = pack_bf16x2(__fmul_rn(wq, gf[4]), __fmul_rn(wq, gf[5]));
-            o.w = pack_bf16x2(__fmul_rn(wq, gf[6]), __fmul_rn(wq, gf[7]));
-            st_stream_v4(grad_y + static_cast<size_t>(slot) * H + static_cast<size_t>(s) * seg + c, o);
           }
         }
       }
@@ -225,7 +250,7 @@ __global__ void __launch_bounds__(kThreads)
       if (s == segs - 1) {
         // the group's last segment: reduce the partial dots and write grad_w
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < kDots; ++q) {
           if (q >= TK) break;
           float d = dot[q];
 #pragma unroll
@@ -248,15 +273,12 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
-}  // namespace
-
-cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, int H, int k,
-                                    const int32_t* token_slot, long long num_rows,
-                                    const float* topk_w, void* grad_y, float* grad_w,
-                                    int32_t* d_status, cudaStream_t stream) {
-  if (N == 0) return cudaSuccess;
+template <int KT>
+cudaError_t launch_bulk(const void* grad_out, const void* y, int N, int H, int k,
+                        const int32_t* token_slot, long long num_rows, const float* topk_w,
+                        void* grad_y, float* grad_w, int32_t* d_status, cudaStream_t stream) {
   const Layout L = smem_layout(k);
-  cudaError_t err = cudaFuncSetAttribute(combine_backward_bulk_kernel,
+  cudaError_t err = cudaFuncSetAttribute(combine_backward_bulk_kernel<KT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L.total));
   if (err != cudaSuccess) return err;
@@ -264,16 +286,32 @@ cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, 
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
     return err;
-  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_backward_bulk_kernel,
+  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_backward_bulk_kernel<KT>,
                                                            kThreads, L.total)) != cudaSuccess)
     return err;
   if (per_sm < 1) per_sm = 1;
   const long long groups = (N + L.T - 1) / L.T;
   const long long grid = std::min<long long>(groups, static_cast<long long>(sms) * per_sm);
-  return launch_pdl(combine_backward_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total,
+  return launch_pdl(combine_backward_bulk_kernel<KT>, static_cast<unsigned>(grid), kThreads, L.total,
                     stream, static_cast<const uint16_t*>(grad_out), static_cast<const uint16_t*>(y),
                     N, H, k, token_slot, num_rows, topk_w, static_cast<uint16_t*>(grad_y), grad_w,
                     d_status);
+}
+
+}  // namespace
+
+cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, int H, int k,
+                                    const int32_t* token_slot, long long num_rows,
+                                    const float* topk_w, void* grad_y, float* grad_w,
+                                    int32_t* d_status, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  switch (k) {
+    case 1: return launch_bulk<1>(grad_out, y, N, H, k, token_slot, num_rows, topk_w, grad_y, grad_w, d_status, stream);
+    case 2: return launch_bulk<2>(grad_out, y, N, H, k, token_slot, num_rows, topk_w, grad_y, grad_w, d_status, stream);
+    case 4: return launch_bulk<4>(grad_out, y, N, H, k, token_slot, num_rows, topk_w, grad_y, grad_w, d_status, stream);
+    case 8: return launch_bulk<8>(grad_out, y, N, H, k, token_slot, num_rows, topk_w, grad_y, grad_w, d_status, stream);
+    default: return launch_bulk<0>(grad_out, y, N, H, k, token_slot, num_rows, topk_w, grad_y, grad_w, d_status, stream);
+  }
 }
 
 }  // namespace moe

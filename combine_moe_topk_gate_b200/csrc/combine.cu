@@ -66,6 +66,9 @@ __host__ __device__ inline Layout smem_layout(int k) {
   return L;
 }
 
+// KT > 0: k == KT is known at compile time (1, 2, 4 or 8), so the consumers'
+// loops over tokens and slots unroll exactly; KT == 0 serves any k.
+template <int KT>
 __global__ void __launch_bounds__(kThreads, 3)
     combine_bulk_kernel(const uint16_t* __restrict__ y, int N, int H, int k,
                         const int32_t* __restrict__ token_slot, long long S,
@@ -184,6 +187,38 @@ __global__ void __launch_bounds__(kThreads, 3)
             reinterpret_cast<const float*>(smem + L.hdr_off + static_cast<size_t>(stage) * kHeaderBytes);
         const uint32_t vmask = reinterpret_cast<const uint32_t*>(hw)[32];
         const uint32_t stage0 = data + static_cast<uint32_t>(stage * L.stage_bytes) + c * 2;
+        if constexpr (KT > 0) {
+          constexpr int TT = KT >= 8 ? 1 : 8 / KT;  // == L.T
+#pragma unroll
+          for (int u = 0; u < TT; ++u) {
+            const int t = g * TT + u;
+            if (t >= N) break;
+            const uint32_t row0 = stage0 + static_cast<uint32_t>(u * KT) * seg_bytes;
+            uint4 v[KT];
+#pragma unroll
+            for (int q = 0; q < KT; ++q) v[q] = ld_shared_v4(row0 + q * seg_bytes);
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+            for (int q = 0; q < KT; ++q) {
+              if (!((vmask >> (u * KT + q)) & 1u)) continue;  // masked slot: rows not staged
+              const float wj = hw[u * KT + q];
+              const uint32_t w4[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                acc[2 * i] = __fmaf_rn(wj, bf16_lo(w4[i]), acc[2 * i]);
+                acc[2 * i + 1] = __fmaf_rn(wj, bf16_hi(w4[i]), acc[2 * i + 1]);
+              }
+            }
+            uint4 o;
+            o.x = pack_bf16x2(acc[0], acc[1]);
+            o.y = pack_bf16x2(acc[2], acc[3]);
+            o.z = pack_bf16x2(acc[4], acc[5]);
+            o.w = pack_bf16x2(acc[6], acc[7]);
+            st_stream_v4(out + static_cast<size_t>(t) * H + static_cast<size_t>(s) * seg + c, o);
+          }
+        } else
         for (int u = 0; u < T; ++u) {
           const int t = g * T + u;
           if (t >= N) break;
@@ -296,6 +331,31 @@ __global__ void __launch_bounds__(kSmallWarps * 32)
   }
 }
 
+template <int KT>
+cudaError_t launch_bulk(const void* y, int N, int H, int k, const int32_t* token_slot,
+                        long long num_rows, const float* topk_w, void* out, int32_t* d_status,
+                        cudaStream_t stream) {
+  const Layout L = smem_layout(k);
+  cudaError_t err = cudaFuncSetAttribute(combine_bulk_kernel<KT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(L.total));
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return err;
+  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel<KT>, kThreads,
+                                                           L.total)) != cudaSuccess)
+    return err;
+  if (per_sm < 1) per_sm = 1;
+  const long long items =
+      static_cast<long long>((N + L.T - 1) / L.T) * ((H + L.seg - 1) / L.seg);
+  const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
+  return launch_pdl(combine_bulk_kernel<KT>, static_cast<unsigned>(grid), kThreads, L.total, stream,
+                    static_cast<const uint16_t*>(y), N, H, k, token_slot, num_rows, topk_w,
+                    static_cast<uint16_t*>(out), d_status);
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* token_slot,
@@ -308,25 +368,13 @@ cudaError_t launch_combine(const void* y, int N, int H, int k, const int32_t* to
                       kSmallWarps * 32, 0, stream, static_cast<const uint16_t*>(y), N, H, k, token_slot,
                       num_rows, topk_w, static_cast<uint16_t*>(out), d_status);
   }
-  const Layout L = smem_layout(k);
-  cudaError_t err = cudaFuncSetAttribute(combine_bulk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(L.total));
-  if (err != cudaSuccess) return err;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
-    return err;
-  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_bulk_kernel, kThreads,
-                                                           L.total)) != cudaSuccess)
-    return err;
-  if (per_sm < 1) per_sm = 1;
-  const long long items =
-      static_cast<long long>((N + L.T - 1) / L.T) * ((H + L.seg - 1) / L.seg);
-  const long long grid = std::min<long long>(items, static_cast<long long>(sms) * per_sm);
-  return launch_pdl(combine_bulk_kernel, static_cast<unsigned>(grid), kThreads, L.total, stream,
-                    static_cast<const uint16_t*>(y), N, H, k, token_slot, num_rows, topk_w,
-                    static_cast<uint16_t*>(out), d_status);
+  switch (k) {
+    case 1: return launch_bulk<1>(y, N, H, k, token_slot, num_rows, topk_w, out, d_status, stream);
+    case 2: return launch_bulk<2>(y, N, H, k, token_slot, num_rows, topk_w, out, d_status, stream);
+    case 4: return launch_bulk<4>(y, N, H, k, token_slot, num_rows, topk_w, out, d_status, stream);
+    case 8: return launch_bulk<8>(y, N, H, k, token_slot, num_rows, topk_w, out, d_status, stream);
+    default: return launch_bulk<0>(y, N, H, k, token_slot, num_rows, topk_w, out, d_status, stream);
+  }
 }
 
 }  // namespace moe

@@ -37,7 +37,9 @@ def _layout(w, inp, dev, masked_frac=0.0, seed=0):
 CASES = [("prefill", 0.0), ("mixtral", 0.0), ("decode", 0.05), ("tiny", 0.1)]
 EXTRA = [Workload("bwd_k32", 64, 264, 64, 32, 4, "softmax_renorm", "bf16", "random"),
          Workload("bwd_k3", 333, 136, 24, 3, 6, "softmax", "bf16", "random"),
-         Workload("bwd_k1", 100, 512, 16, 1, 4, "softmax", "bf16", "random")]
+         Workload("bwd_k1", 100, 512, 16, 1, 4, "softmax", "bf16", "random"),
+         Workload("bwd_k2", 333, 200, 16, 2, 4, "softmax", "bf16", "random"),
+         Workload("bwd_k4", 301, 264, 32, 4, 4, "softmax_renorm", "bf16", "random")]
 
 
 @pytest.mark.parametrize("w", [WORKLOADS[n] for n, _ in CASES] + EXTRA,

@@ -106,6 +106,23 @@ def test_masked_and_invalid_ids():
     assert g1["status"] == O.ERR_BAD_INDEX
 
 
+@pytest.mark.parametrize("k", [1, 2, 4, 5, 8])
+def test_bulk_combine_every_k_with_masked_slots(k):
+    """Sizes past the register kernel (N * k > 4096) so the pipelined kernel
+    runs, with its compile-time k (1, 2, 4, 8) or generic (5) consumer; a ragged
+    last token group and 10 % masked slots."""
+    E = 32
+    N = 4096 // k + 37
+    w = Workload(f"bulk_k{k}", N, 264, E, k, 4, "softmax", "bf16", "random")
+    inp = make_inputs(w, 7)
+    rng = np.random.default_rng(k)
+    idx = np.stack([rng.choice(E, k, replace=False) for _ in range(N)]).astype(np.int32)
+    idx[rng.random(idx.shape) < 0.1] = -1
+    g, r = run_gpu(w, inp, topk_idx=torch.from_numpy(idx)), run_oracle(w, inp, topk_idx=idx)
+    compare(g, r)
+    assert g["status"] == 0
+
+
 def test_bad_slots_in_dispatch_and_combine():
     from combine_moe_topk_gate_b200 import api
     N, H, k = 64, 256, 2
