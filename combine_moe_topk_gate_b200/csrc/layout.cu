@@ -44,6 +44,17 @@ __device__ __forceinline__ int bucket_of(int e, int E) {
   return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : E;
 }
 
+// True when none of the token's slots before slot j (ids at tok[0..j)) has an
+// expert of the rank whose experts are [lo, lo + epr); ids outside [0, E)
+// never match because that range lies inside it.  The loads are independent.
+__device__ __forceinline__ bool first_on_rank(const int32_t* tok, int j, int lo, int epr) {
+  bool first = true;
+#pragma unroll 4
+  for (int jj = 0; jj < j; ++jj)
+    first = first && static_cast<unsigned>(tok[jj]) - static_cast<unsigned>(lo) >= static_cast<unsigned>(epr);
+  return first;
+}
+
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_count_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R,
                         int32_t* __restrict__ chunk_counts, int32_t* __restrict__ chunk_rtok,
@@ -52,6 +63,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   int32_t* hist = sm;           // E + 1
   int32_t* rtok = hist + E + 1;  // R
   int32_t* sidx = rtok + R;      // kLayoutThreads
+  int32_t* rank_of = sidx + kLayoutThreads;  // E: rank of each expert
   const int tid = threadIdx.x, lane = tid & 31;
   const int c = blockIdx.x;
   const int tc = tokens_per_chunk(k);
@@ -59,8 +71,12 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int nt = static_cast<int>(min(static_cast<long long>(tc), N - t0));
   const int ne = nt > 0 ? nt * k : 0;
   const int nbits = 32 - __clz(E + 1);  // bucket + 1 lies in [0, E + 1]
+  // data-independent setup (overlaps the predecessor's tail under PDL)
+  const int epr = E / R;
+  const int j = tid % k;  // slot of this entry inside its token
   for (int i = tid; i <= E; i += kLayoutThreads) hist[i] = 0;
   for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  for (int i = tid; i < E; i += kLayoutThreads) rank_of[i] = i / epr;
   pdl_wait();
   pdl_trigger();
   int e = -1;
@@ -76,18 +92,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (b >= 0 && (same & lanemask_lt()) == 0) atomicAdd(&hist[b], __popc(same));
   if (b >= 0 && b < E) {
     // the token's first slot landing on this rank counts the token once
-    const int epr = E / R;
-    const int r = e / epr;
-    const int j = tid % k;
-    bool first = true;
-    for (int jj = 0; jj < j; ++jj) {
-      const int e2 = sidx[tid - j + jj];
-      if (static_cast<unsigned>(e2) < static_cast<unsigned>(E) && e2 / epr == r) {
-        first = false;
-        break;
-      }
-    }
-    if (first) atomicAdd(&rtok[r], 1);
+    const int r = rank_of[e];
+    if (first_on_rank(sidx + tid - j, j, r * epr, epr)) atomicAdd(&rtok[r], 1);
   }
   (void)lane;
   __syncthreads();
@@ -128,6 +134,26 @@ __device__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_sums) {
   __syncthreads();
 }
 
+// Exclusive prefix over the warps of every bucket of the [kLayoutWarps][nb]
+// count matrix, in place: one thread per bucket, its loads issued eight at a
+// time (independent addresses) and summed in registers.  Returns the
+// bucket's total.
+__device__ __forceinline__ int warp_prefix_of_bucket(int32_t* wcnt, int nb, int bb) {
+  int acc = 0;
+#pragma unroll
+  for (int w0 = 0; w0 < kLayoutWarps; w0 += 8) {
+    int v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = wcnt[(w0 + i) * nb + bb];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      wcnt[(w0 + i) * nb + bb] = acc;
+      acc += v[i];
+    }
+  }
+  return acc;
+}
+
 // Turns the per-bucket totals in off[] into exclusive row offsets, each
 // expert bucket rounded up to a multiple of `align` (1 = packed); cnt[] keeps
 // the totals.
@@ -136,7 +162,7 @@ __device__ void aligned_offsets(int32_t* off, int32_t* cnt, int nb, int align,
   for (int i = threadIdx.x; i < nb; i += blockDim.x) {
     const int v = off[i];
     cnt[i] = v;
-    if (i < nb - 1) off[i] = (v + align - 1) / align * align;
+    if (i < nb - 1 && align > 1) off[i] = (v + align - 1) / align * align;
   }
   __syncthreads();
   block_exclusive_scan(off, nb, warp_sums);
@@ -177,6 +203,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c = blockIdx.x;
   const int nbits = 32 - __clz(E + 1);
+  const int my_tok = tid / k;  // token of this entry inside the chunk
   pdl_wait();
   pdl_trigger();
 
@@ -257,18 +284,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int in_warp = __popc(same & lanemask_lt());
   if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
   __syncthreads();
-  // exclusive prefix over the 32 warps of every bucket: one warp per bucket
-  // at a time, lane w holding warp w's count
-  for (int bb = warp; bb < nb; bb += kLayoutWarps) {
-    const int v = wcnt[lane * nb + bb];
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFullMask, incl, o);
-      if (lane >= o) incl += y;
-    }
-    wcnt[lane * nb + bb] = incl - v;
-  }
+  // exclusive prefix over the 32 warps of every bucket
+  for (int bb = tid; bb < nb; bb += kLayoutThreads) warp_prefix_of_bucket(wcnt, nb, bb);
   __syncthreads();
   if (tid < ne) {
     const int slot = base[b] + wcnt[warp * nb + b] + in_warp;
@@ -280,7 +297,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
       report_bad_index(d_status);
     } else if (b < E) {
       token_slot[flat] = slot;
-      slot_token[slot] = static_cast<int32_t>(t0 + tid / k);
+      slot_token[slot] = static_cast<int32_t>(t0 + my_tok);
     } else {
       token_slot[flat] = -1;
       slot_token[slot] = -1;
@@ -307,12 +324,16 @@ __global__ void __launch_bounds__(kLayoutThreads)
   int32_t* rtok = warp_sums + 32;                 // R
   int32_t* sidx = rtok + R;                       // kLayoutThreads
   int32_t* cnt = sidx + kLayoutThreads;           // nb: totals
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* rank_of = cnt + nb;                    // E: rank of each expert
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int ne = N * k;  // <= kLayoutThreads
   const int nbits = 32 - __clz(E + 1);
   const int epr = E / R;
+  // data-independent setup (overlaps the predecessor's tail under PDL)
+  const int my_tok = tid / k, j = tid - my_tok * k;
   for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
   for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
+  for (int i = tid; i < E; i += kLayoutThreads) rank_of[i] = i / epr;
   pdl_wait();
   pdl_trigger();
   int e = -1, b = -1;
@@ -327,31 +348,12 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const int in_warp = __popc(same & lanemask_lt());
   if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
   if (b >= 0 && b < E) {  // the token's first slot on this rank counts the token
-    const int r = e / epr;
-    const int j = tid % k;
-    bool first = true;
-    for (int jj = 0; jj < j; ++jj) {
-      const int e2 = sidx[tid - j + jj];
-      if (static_cast<unsigned>(e2) < static_cast<unsigned>(E) && e2 / epr == r) {
-        first = false;
-        break;
-      }
-    }
-    if (first) atomicAdd(&rtok[r], 1);
+    const int r = rank_of[e];
+    if (first_on_rank(sidx + tid - j, j, r * epr, epr)) atomicAdd(&rtok[r], 1);
   }
   __syncthreads();
   // per bucket: exclusive prefix over the warps, total into off[]
-  for (int bb = warp; bb < nb; bb += kLayoutWarps) {
-    const int v = wcnt[lane * nb + bb];
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(kFullMask, incl, o);
-      if (lane >= o) incl += y;
-    }
-    wcnt[lane * nb + bb] = incl - v;
-    if (lane == 31) off[bb] = incl;
-  }
+  for (int bb = tid; bb < nb; bb += kLayoutThreads) off[bb] = warp_prefix_of_bucket(wcnt, nb, bb);
   __syncthreads();
   aligned_offsets(off, cnt, nb, align, warp_sums);
   for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
     const int slot = off[b] + wcnt[warp * nb + b] + in_warp;
     if (b < E) {
       token_slot[tid] = slot;
-      slot_token[slot] = tid / k;
+      slot_token[slot] = my_tok;
     } else {
       token_slot[tid] = -1;
       slot_token[slot] = -1;
@@ -393,7 +395,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
   cudaError_t err;
   if (static_cast<long long>(N) * k <= kLayoutThreads) {
     const size_t smem = (2 * (static_cast<size_t>(E) + 1) +
-                         static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R + kLayoutThreads) *
+                         static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R + kLayoutThreads + E) *
                         sizeof(int32_t);
     if (smem > 48 * 1024) {
       err = cudaFuncSetAttribute(layout_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -406,7 +408,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
   }
   int32_t* chunk_counts = static_cast<int32_t*>(workspace);
   int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
-  const size_t smem_count = (static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
+  const size_t smem_count = (2 * static_cast<size_t>(E) + 1 + R + kLayoutThreads) * sizeof(int32_t);
   const size_t smem_assign =
       (3 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
       sizeof(int32_t);
