@@ -42,12 +42,17 @@ EXTRA = [Workload("bwd_k32", 64, 264, 64, 32, 4, "softmax_renorm", "bf16", "rand
          Workload("bwd_k4", 301, 264, 32, 4, 4, "softmax_renorm", "bf16", "random")]
 
 
+# masked slots reach every compile-time k of the backward consumer (1, 2, 4, 8)
+# and the generic one (3, 32)
+MASKED_EXTRA = {"bwd_k32": 0.1, "bwd_k3": 0.15, "bwd_k1": 0.2, "bwd_k2": 0.1, "bwd_k4": 0.1}
+
+
 @pytest.mark.parametrize("w", [WORKLOADS[n] for n, _ in CASES] + EXTRA,
                          ids=[n for n, _ in CASES] + [w.name for w in EXTRA])
 def test_backward_parity(w):
     from combine_moe_topk_gate_b200 import api
     dev = torch.device("cuda", 0)
-    masked = dict(CASES).get(w.name, 0.0)
+    masked = dict(CASES).get(w.name, MASKED_EXTRA.get(w.name, 0.0))
     inp = make_inputs(w, 5, with_y=False)
     idx, wts, L = _layout(w, inp, dev, masked)
     gen = torch.Generator().manual_seed(11)
