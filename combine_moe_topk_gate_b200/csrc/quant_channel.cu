@@ -17,6 +17,14 @@
 // is small -- and writes the codes: 8 bytes per lane and row (row-major), or
 // through a shared-memory tile of 32 rows so that each warp store covers 32
 // consecutive rows of one channel (transposed).
+//
+// With few experts (thousands of rows each) one CTA per (expert, slab) is
+// too little parallelism, so Q > 1 CTAs form a thread-block cluster per
+// (expert, slab), each taking a 32-row-aligned share of the expert's rows:
+// every CTA reduces its share's per-channel amax, the cluster combines them
+// through distributed shared memory between two hardware cluster barriers,
+// and each CTA writes the codes of its own rows.  A max is exact in any
+// order, so every Q gives the same bits.
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
@@ -54,7 +62,7 @@ __device__ __forceinline__ void st_hint_v2(void* ptr, uint2 v, uint64_t pol) {
                "l"(pol));
 }
 
-template <bool TRANSPOSE>
+template <bool TRANSPOSE, bool CLUSTER>
 __global__ void __launch_bounds__(kThreads)
     quant_fp8_channel_kernel(const uint16_t* __restrict__ x, long long S, int H, int E,
                              const int32_t* __restrict__ expert_offset,
@@ -62,20 +70,27 @@ __global__ void __launch_bounds__(kThreads)
                              float* __restrict__ scale, int32_t* d_status) {
   __shared__ float part[kWarpsPerCta][kSlab];
   __shared__ float inv_s[kSlab];
+  __shared__ float cta_amax[CLUSTER ? kSlab : 1];  // this CTA's share, read by the cluster
   __shared__ uint8_t tile[TRANSPOSE ? kSlab : 1][33];  // transposed: 32 rows per channel (+1: banks)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int slab = blockIdx.x, e = blockIdx.y;
+  // cluster: x = slab * Q + rank, the Q CTAs of a cluster share (expert, slab)
+  const int Q = CLUSTER ? static_cast<int>(gridDim.x / ((H + kSlab - 1) / kSlab)) : 1;
+  const int q = CLUSTER ? static_cast<int>(cluster_rank()) : 0;
+  const int slab = CLUSTER ? static_cast<int>(blockIdx.x) / Q : static_cast<int>(blockIdx.x);
+  const int e = blockIdx.y;
   const int c0 = slab * kSlab + lane * 8;
   const bool active = c0 < H;  // H % 128 == 0: 8 whole channels or none
   pdl_wait();
   pdl_trigger();
   const long long r0 = expert_offset[e];
   const long long n = expert_count[e];
-  if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert
-    if (tid == 0 && slab == 0) report_bad_index(d_status);
-    return;
+  if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert (the
+    if (tid == 0 && slab == 0) report_bad_index(d_status);  // whole cluster returns:
+    return;                                                   // e is the same for all)
   }
-  const long long r1 = r0 + n;
+  const long long share = CLUSTER ? ((n + Q - 1) / Q + 31) / 32 * 32 : n;  // rows per CTA
+  const long long rb = r0 + q * share < r0 + n ? r0 + q * share : r0 + n;  // this CTA's rows
+  const long long r1 = rb + share < r0 + n ? rb + share : r0 + n;
   const uint16_t* col = x + c0;
   const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
 
@@ -90,7 +105,7 @@ __global__ void __launch_bounds__(kThreads)
     for (int j = 0; j < 4; ++j) m2[j] = __hmax2(m2[j], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
   };
   if (active) {
-    long long s = r0 + warp;
+    long long s = rb + warp;
     for (; s + 7 * kWarpsPerCta < r1; s += 8 * kWarpsPerCta) {
       uint4 v[8];
 #pragma unroll
@@ -111,8 +126,17 @@ __global__ void __launch_bounds__(kThreads)
     float a = part[0][c];
 #pragma unroll
     for (int w = 1; w < kWarpsPerCta; ++w) a = fmaxf(a, part[w][c]);
+    if constexpr (CLUSTER) {
+      cta_amax[c] = a;
+      cluster_arrive();  // every CTA's share published ...
+      cluster_wait();
+      a = 0.0f;
+      for (int r = 0; r < Q; ++r) a = fmaxf(a, ld_peer_shared_f32(&cta_amax[c], static_cast<uint32_t>(r)));
+      cluster_arrive();  // ... and read; the matching wait comes before the exit
+    }
     inv_s[c] = __fdiv_rn(448.0f, a);
-    if (slab * kSlab + c < H) scale[static_cast<size_t>(e) * H + slab * kSlab + c] = __fdiv_rn(a, 448.0f);
+    if (q == 0 && slab * kSlab + c < H)
+      scale[static_cast<size_t>(e) * H + slab * kSlab + c] = __fdiv_rn(a, 448.0f);
   }
   __syncthreads();
   float inv[8];
@@ -148,7 +172,7 @@ __global__ void __launch_bounds__(kThreads)
   auto codes_of = [&](long long s) -> uint2 { return codes_of_v(ld_hint(col + static_cast<size_t>(s) * H, done)); };
   if constexpr (!TRANSPOSE) {
     if (active) {
-      long long s = r0 + warp;
+      long long s = rb + warp;
       for (; s + 3 * kWarpsPerCta < r1; s += 4 * kWarpsPerCta) {  // four rows' loads in flight
         uint4 v[4];
 #pragma unroll
@@ -160,7 +184,7 @@ __global__ void __launch_bounds__(kThreads)
       for (; s < r1; s += kWarpsPerCta) st_hint_v2(out + static_cast<size_t>(s) * H + c0, codes_of(s), done);
     }
   } else {
-    for (long long s0 = r0; s0 < r1; s0 += 32) {
+    for (long long s0 = rb; s0 < r1; s0 += 32) {
       // warp w fills rows s0 + w, s0 + w + 8, ... of the 32-row tile
       for (int rr = warp; rr < 32; rr += kWarpsPerCta) {
         const long long s = s0 + rr;
@@ -179,6 +203,7 @@ __global__ void __launch_bounds__(kThreads)
       __syncthreads();
     }
   }
+  if constexpr (CLUSTER) cluster_wait();  // no CTA leaves while a peer may still read its share
 }
 
 }  // namespace
@@ -187,13 +212,26 @@ cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, i
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,
                                      cudaStream_t stream) {
-  const dim3 grid((H + kSlab - 1) / kSlab, E);
+  const int slabs = (H + kSlab - 1) / kSlab;
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* o = static_cast<uint8_t*>(out);
+  // CTAs per (expert, slab): about 512 rows each on average, at most 8 (the
+  // portable cluster size); 1 keeps the plain launch
+  const long long avg_rows = E > 0 ? num_rows / E : 0;
+  const int Q = avg_rows >= 4096 ? 8 : avg_rows >= 2048 ? 4 : avg_rows >= 1024 ? 2 : 1;
+  if (Q > 1) {
+    const dim3 grid(slabs * Q, E);
+    if (transpose)
+      return launch_pdl_cluster(quant_fp8_channel_kernel<true, true>, grid, kThreads, 0, stream, Q, xs,
+                                num_rows, H, E, expert_offset, expert_count, o, scale, d_status);
+    return launch_pdl_cluster(quant_fp8_channel_kernel<false, true>, grid, kThreads, 0, stream, Q, xs,
+                              num_rows, H, E, expert_offset, expert_count, o, scale, d_status);
+  }
+  const dim3 grid(slabs, E);
   if (transpose)
-    return launch_pdl(quant_fp8_channel_kernel<true>, grid, kThreads, 0, stream, xs, num_rows, H, E,
+    return launch_pdl(quant_fp8_channel_kernel<true, false>, grid, kThreads, 0, stream, xs, num_rows, H, E,
                       expert_offset, expert_count, o, scale, d_status);
-  return launch_pdl(quant_fp8_channel_kernel<false>, grid, kThreads, 0, stream, xs, num_rows, H, E,
+  return launch_pdl(quant_fp8_channel_kernel<false, false>, grid, kThreads, 0, stream, xs, num_rows, H, E,
                     expert_offset, expert_count, o, scale, d_status);
 }
 

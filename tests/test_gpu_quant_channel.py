@@ -17,6 +17,11 @@ CASES = [
     (WORKLOADS["decode"], 128, 0.0),
     (WORKLOADS["prefill"], 128, 0.0),
     (Workload("ch_ragged", 300, 384, 40, 3, 8, "softmax", "bf16", "random"), 8, 0.25),
+    # few experts with thousands of rows each: several CTAs per (expert, slab),
+    # combined through a thread-block cluster (2, 4 and 8 CTAs)
+    (Workload("ch_q2", 1100, 256, 2, 2, 2, "softmax", "bf16", "random"), 128, 0.1),
+    (Workload("ch_q4", 3000, 384, 2, 2, 2, "softmax", "bf16", "random"), 32, 0.3),
+    (Workload("ch_q8", 8192, 384, 4, 2, 2, "softmax", "bf16", "random"), 128, 0.2),
 ]
 
 
@@ -73,3 +78,34 @@ def test_quant_fp8_channel_reports_bad_ranges():
     api.moe_quant_fp8_channel(recv, off, cnt_bad, d_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == O.ERR_BAD_INDEX
+
+
+@pytest.mark.parametrize("transpose", [False, True])
+def test_clustered_split_with_empty_experts(transpose):
+    """40 000 rows over 4 experts (8 CTAs per expert and slab), experts 1 and 3
+    empty, expert 2 with 37 rows: the empty and short experts' CTAs still meet
+    the cluster barriers, and nothing outside the landed rows is touched."""
+    from combine_moe_topk_gate_b200 import api
+    dev = torch.device("cuda", 0)
+    N, H, E = 40000, 256, 4
+    idx = torch.zeros((N, 1), dtype=torch.int32)
+    idx[:37, 0] = 2
+    L = api.moe_get_layout(idx.to(dev), E, 2)
+    g = torch.Generator().manual_seed(12)
+    recv = (torch.randn(N, H, generator=g) * torch.exp2(torch.randint(-8, 8, (1, H), generator=g).float()))
+    recv[5000:5100, 17] = 300.0                                  # a channel maximum deep inside one share
+    recv = recv.to(torch.bfloat16)
+    shape = (H, N) if transpose else (N, H)
+    out = torch.zeros(shape, dtype=torch.uint8, device=dev)
+    sc = torch.full((E, H), 5.0, dtype=torch.float32, device=dev)
+    api.moe_quant_fp8_channel(recv.to(dev), L.expert_offset, L.expert_count, transpose=transpose, out=out,
+                              scale=sc, d_status=L.status)
+    torch.cuda.synchronize()
+    assert int(L.status.item()) == 0
+    off, cnt = L.expert_offset.cpu().numpy(), L.expert_count.cpu().numpy()
+    assert list(cnt) == [N - 37, 0, 37, 0]
+    r_out, r_sc, st = O.quant_fp8_channel(bf16_bits(recv), off, cnt, transpose=transpose)
+    assert st == 0
+    assert np.array_equal(out.cpu().numpy(), r_out)
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), r_sc.view(np.uint32))
+    assert (sc.cpu().numpy()[[1, 3]] == 0).all()
