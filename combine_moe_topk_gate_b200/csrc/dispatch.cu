@@ -35,7 +35,11 @@ __device__ __forceinline__ int ceil_log2_pos(float q) {
 // UE8M0 = true: power-of-two scale 2^e per 128-block with e = ceil(log2(amax /
 // 448)) of the fp32 quotient, stored as the byte e + 127; codes e4m3(x * 2^-e)
 // (exact scaling, so a zero keeps its sign without a select).
-template <int SL, bool UE8M0 = false>
+// SPW = segments per warp: with SPW = 2 a warp owns two neighbouring
+// 512-channel segments of its token and issues both segments' loads before
+// working on the first, twice the bytes in flight per warp -- for small k,
+// where reading x is most of the traffic and load latency sets the pace.
+template <int SL, bool UE8M0 = false, int SPW = 1>
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_fp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                         const int32_t* __restrict__ token_slot, long long S,
@@ -43,86 +47,99 @@ __global__ void __launch_bounds__(kWarps * 32)
                         long long ld, int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
+  const int groups = (segs + SPW - 1) / SPW;  // work items per token
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(N) * segs) return;
-  const int t = static_cast<int>(item / segs);
-  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
-  const int c0 = s * 512 + lane * 16;
-  const bool active = c0 < H;  // H % 128 == 0: whole 8-lane blocks are in or out
+  if (item >= static_cast<long long>(N) * groups) return;
+  const int t = static_cast<int>(item / groups);
+  const int s0 = static_cast<int>(item - static_cast<long long>(t) * groups) * SPW;
   const int nblk = H / 128;
   pdl_wait();
   pdl_trigger();
 
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
-  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-  if (active) {
-    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
-    a = ld_stream(src);
-    b = ld_stream(src + 8);
-  }
-  float f[16];
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint4 av[SPW], bv[SPW];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    f[2 * i] = bf16_lo(w[i]);
-    f[2 * i + 1] = bf16_hi(w[i]);
-  }
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
-  amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-  float inv, scale = 0.0f;
-  uint32_t sword = 0;  // UE8M0: the warp's 4 block bytes (block i in byte i)
-  if constexpr (UE8M0) {
-    int e = amax > 0.0f ? ceil_log2_pos(__fdiv_rn(amax, 448.0f)) : -127;
-    e = e < -127 ? -127 : (e > 127 ? 127 : e);
-    inv = __int_as_float((127 - e) << 23);  // 2^-e; e <= 120 for bf16 input
-    const uint32_t byte = static_cast<uint32_t>(e + 127);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sword |= (__shfl_sync(kFullMask, byte, 8 * i) & 0xffu) << (8 * i);
-  } else {
-    inv = __fdiv_rn(448.0f, amax);
-    scale = __fdiv_rn(amax, 448.0f);
-  }
-  uint32_t q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float p[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float v = f[4 * i + u];
-      p[u] = (UE8M0 || v != 0.0f) ? __fmul_rn(v, inv) : v;  // zero keeps its sign
+  for (int u = 0; u < SPW; ++u) {
+    const int c0 = (s0 + u) * 512 + lane * 16;
+    av[u] = make_uint4(0, 0, 0, 0);
+    bv[u] = make_uint4(0, 0, 0, 0);
+    if (c0 < H) {  // H % 128 == 0: whole 8-lane blocks are in or out
+      const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
+      av[u] = ld_stream(src);
+      bv[u] = ld_stream(src + 8);
     }
-    q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
   }
-  const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
-  for (int j = 0; j < k; ++j) {
-    const int slot = __shfl_sync(kFullMask, my_slot, j);
-    if (slot == -1) continue;
-    if (slot < -1 || slot >= S) {
-      if (lane == 0) report_bad_index(d_status);
-      continue;
+#pragma unroll
+  for (int u = 0; u < SPW; ++u) {
+    const int s = s0 + u;
+    if (s >= segs) break;  // warp-uniform
+    const int c0 = s * 512 + lane * 16;
+    const bool active = c0 < H;
+    const uint4 a = av[u], b = bv[u];
+    float f[16];
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      f[2 * i] = bf16_lo(w[i]);
+      f[2 * i + 1] = bf16_hi(w[i]);
     }
-    if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
-    if constexpr (!UE8M0) {
-      if (active && (lane & 7) == 0) {
-        if constexpr (SL == MOE_SCALE_ROW_MAJOR)
-          recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
-        else
-          st_keep_b32(recv_scale + scale_at<SL>(slot, c0 >> 7, nblk, ld), __float_as_uint(scale),
-                      l2_evict_last_policy());
-      }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
+    float inv, scale = 0.0f;
+    uint32_t sword = 0;  // UE8M0: the warp's 4 block bytes (block i in byte i)
+    if constexpr (UE8M0) {
+      int e = amax > 0.0f ? ceil_log2_pos(__fdiv_rn(amax, 448.0f)) : -127;
+      e = e < -127 ? -127 : (e > 127 ? 127 : e);
+      inv = __int_as_float((127 - e) << 23);  // 2^-e; e <= 120 for bf16 input
+      const uint32_t byte = static_cast<uint32_t>(e + 127);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sword |= (__shfl_sync(kFullMask, byte, 8 * i) & 0xffu) << (8 * i);
     } else {
-      uint8_t* sb = reinterpret_cast<uint8_t*>(recv_scale);
-      if constexpr (SL == MOE_SCALE_MN_MAJOR_PACK4) {
-        // the warp's 4 blocks are exactly word s of the row
-        if (lane == 0) *reinterpret_cast<uint32_t*>(sb + scale_at<SL>(slot, 4 * s, nblk, ld)) = sword;
-      } else if (SL == MOE_SCALE_ROW_MAJOR && (nblk & 3) == 0) {
-        if (lane == 0) *reinterpret_cast<uint32_t*>(sb + static_cast<size_t>(slot) * nblk + 4 * s) = sword;
-      } else if (active && (lane & 7) == 0) {
-        sb[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = static_cast<uint8_t>(sword >> (lane & 24));
+      inv = __fdiv_rn(448.0f, amax);
+      scale = __fdiv_rn(amax, 448.0f);
+    }
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float p[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float xv = f[4 * i + v];
+        p[v] = (UE8M0 || xv != 0.0f) ? __fmul_rn(xv, inv) : xv;  // zero keeps its sign
+      }
+      q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+    }
+    const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
+    for (int j = 0; j < k; ++j) {
+      const int slot = __shfl_sync(kFullMask, my_slot, j);
+      if (slot == -1) continue;
+      if (slot < -1 || slot >= S) {
+        if (lane == 0 && u == 0) report_bad_index(d_status);
+        continue;
+      }
+      if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
+      if constexpr (!UE8M0) {
+        if (active && (lane & 7) == 0) {
+          if constexpr (SL == MOE_SCALE_ROW_MAJOR)
+            recv_scale[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = scale;
+          else
+            st_keep_b32(recv_scale + scale_at<SL>(slot, c0 >> 7, nblk, ld), __float_as_uint(scale),
+                        l2_evict_last_policy());
+        }
+      } else {
+        uint8_t* sb = reinterpret_cast<uint8_t*>(recv_scale);
+        if constexpr (SL == MOE_SCALE_MN_MAJOR_PACK4) {
+          // the warp's 4 blocks are exactly word s of the row
+          if (lane == 0) *reinterpret_cast<uint32_t*>(sb + scale_at<SL>(slot, 4 * s, nblk, ld)) = sword;
+        } else if (SL == MOE_SCALE_ROW_MAJOR && (nblk & 3) == 0) {
+          if (lane == 0) *reinterpret_cast<uint32_t*>(sb + static_cast<size_t>(slot) * nblk + 4 * s) = sword;
+        } else if (active && (lane & 7) == 0) {
+          sb[scale_at<SL>(slot, c0 >> 7, nblk, ld)] = static_cast<uint8_t>(sword >> (lane & 24));
+        }
       }
     }
   }
@@ -580,6 +597,21 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
   }
 }
 
+template <int SL, bool UE8M0>
+cudaError_t launch_fp8(bool two, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                       long long num_rows, uint8_t* recv_x, float* recv_scale, long long ld,
+                       int32_t* d_status, cudaStream_t stream) {
+  const int segs = (H + 511) / 512;
+  const int spw = two ? 2 : 1;
+  const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
+  const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+  if (two)
+    return launch_pdl(dispatch_fp8_kernel<SL, UE8M0, 2>, blocks, kWarps * 32, 0, stream, x, N, H, k,
+                      token_slot, num_rows, recv_x, recv_scale, ld, d_status);
+  return launch_pdl(dispatch_fp8_kernel<SL, UE8M0, 1>, blocks, kWarps * 32, 0, stream, x, N, H, k,
+                    token_slot, num_rows, recv_x, recv_scale, ld, d_status);
+}
+
 }  // namespace
 
 long long scale_ld(long long num_rows, int dtype) {
@@ -602,23 +634,24 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
     float* f32 = static_cast<float*>(recv_scale);
     uint8_t* e8 = static_cast<uint8_t*>(recv_scale);
+    // two segments per warp when k <= 4 (reads of x dominate), else one
+    const bool two = k <= 4;
     if (dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
-        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR, true>, blocks, kWarps * 32, 0, stream,
-                          xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+        return launch_fp8<MOE_SCALE_MN_MAJOR, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                    d_status, stream);
       if (scale_layout == MOE_SCALE_MN_MAJOR_PACK4)
-        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR_PACK4, true>, blocks, kWarps * 32, 0,
-                          stream, xs, N, H, k, token_slot, num_rows, r8, f32, (num_rows + 3) / 4 * 4,
-                          d_status);
-      return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_ROW_MAJOR, true>, blocks, kWarps * 32, 0, stream,
-                        xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+        return launch_fp8<MOE_SCALE_MN_MAJOR_PACK4, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32,
+                                                          (num_rows + 3) / 4 * 4, d_status, stream);
+      return launch_fp8<MOE_SCALE_ROW_MAJOR, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                   d_status, stream);
     }
     if (dtype == MOE_DTYPE_FP8_E4M3) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
-        return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,
-                          xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
-      return launch_pdl(dispatch_fp8_kernel<MOE_SCALE_ROW_MAJOR>, blocks, kWarps * 32, 0, stream,
-                        xs, N, H, k, token_slot, num_rows, r8, f32, ld, d_status);
+        return launch_fp8<MOE_SCALE_MN_MAJOR, false>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                     d_status, stream);
+      return launch_fp8<MOE_SCALE_ROW_MAJOR, false>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                    d_status, stream);
     }
     if (scale_layout == MOE_SCALE_MN_MAJOR)
       return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,

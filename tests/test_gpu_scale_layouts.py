@@ -23,6 +23,10 @@ CASES = [
     (Workload("sl_ragged", 1500, 384, 96, 6, 8, "softmax_renorm", "fp8", "random"), 32, 0.2),
     (Workload("sl_small", 37, 640, 16, 3, 4, "softmax", "fp8", "random"), 1, 0.0),
     (WORKLOADS["prefill"], 128, 0.0),
+    # k <= 4: the FP8 kernels take two 512-channel segments per warp; 1152
+    # channels = 3 segments, so the last warp of a token has one segment
+    (Workload("sl_k2_odd", 600, 1152, 16, 2, 4, "softmax", "fp8", "random"), 16, 0.1),
+    (Workload("sl_k4", 300, 2048, 32, 4, 8, "softmax_renorm", "fp8", "random"), 128, 0.05),
 ]
 
 
