@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 // the per-block kernel: lane owns 16 channels, 2 lanes = one block, a warp
 // covers 512 channels and gathers its 16 scale bytes into one 16-byte store.
 
-template <int SL>
+template <int SL, int SPW = 1>  // SPW: segments per warp, as in the FP8 kernel
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_mxfp8_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                           const int32_t* __restrict__ token_slot, long long S,
@@ -159,23 +159,35 @@ __global__ void __launch_bounds__(kWarps * 32)
                           long long ld, int32_t* d_status) {
   const int lane = threadIdx.x & 31;
   const int segs = (H + 511) / 512;
+  const int groups = (segs + SPW - 1) / SPW;  // work items per token
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(N) * segs) return;
-  const int t = static_cast<int>(item / segs);
-  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
-  const int c0 = s * 512 + lane * 16;
-  const bool active = c0 < H;  // H % 32 == 0: whole 2-lane blocks are in or out
+  if (item >= static_cast<long long>(N) * groups) return;
+  const int t = static_cast<int>(item / groups);
+  const int s0 = static_cast<int>(item - static_cast<long long>(t) * groups) * SPW;
   const int nblk = H / 32;
   pdl_wait();
   pdl_trigger();
 
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
-  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-  if (active) {
-    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
-    a = ld_stream(src);
-    b = ld_stream(src + 8);
+  uint4 av[SPW], bv[SPW];
+#pragma unroll
+  for (int u = 0; u < SPW; ++u) {
+    const int cu = (s0 + u) * 512 + lane * 16;
+    av[u] = make_uint4(0, 0, 0, 0);
+    bv[u] = make_uint4(0, 0, 0, 0);
+    if (cu < H) {  // H % 32 == 0: whole 2-lane blocks are in or out
+      const uint16_t* src = x + static_cast<size_t>(t) * H + cu;
+      av[u] = ld_stream(src);
+      bv[u] = ld_stream(src + 8);
+    }
   }
+#pragma unroll
+  for (int u = 0; u < SPW; ++u) {
+  const int s = s0 + u;
+  if (s >= segs) break;  // warp-uniform
+  const int c0 = s * 512 + lane * 16;
+  const bool active = c0 < H;
+  const uint4 a = av[u], b = bv[u];
   float f[16];
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -216,7 +228,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int slot = __shfl_sync(kFullMask, my_slot, j);
     if (slot == -1) continue;
     if (slot < -1 || slot >= S) {
-      if (lane == 0) report_bad_index(d_status);
+      if (lane == 0 && u == 0) report_bad_index(d_status);
       continue;
     }
     if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
@@ -240,6 +252,7 @@ __global__ void __launch_bounds__(kWarps * 32)
         st_keep_b8(recv_e8m0 + scale_at<SL>(slot, c0 >> 5, nblk, ld), my_byte, l2_evict_last_policy());
     }
   }
+  }  // segments of the warp
 }
 
 // FP8 with one scale per token: one 128-thread CTA per token.  One thread
@@ -504,7 +517,8 @@ __device__ __forceinline__ uint32_t e5m6_code(float f) {
 // 24 bytes (two codes per 3 bytes, little endian).  The warp's 768 bytes are
 // staged in shared memory and leave as 16-byte streaming stores covering 512
 // and 256 contiguous bytes (lanes 0..31, then 0..15), so no sector is
-// written in pieces.
+// written in pieces.  SPW: segments per warp, as in the FP8 kernel.
+template <int SPW = 1>
 __global__ void __launch_bounds__(kWarps * 32)
     dispatch_e5m6_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                          const int32_t* __restrict__ token_slot, long long S,
@@ -512,25 +526,36 @@ __global__ void __launch_bounds__(kWarps * 32)
   __shared__ __align__(16) uint2 stage[kWarps][96];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int segs = (H + 511) / 512;
+  const int groups = (segs + SPW - 1) / SPW;  // work items per token
   const long long item = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  if (item >= static_cast<long long>(N) * segs) return;
-  const int t = static_cast<int>(item / segs);
-  const int s = static_cast<int>(item - static_cast<long long>(t) * segs);
-  const int c0 = s * 512 + lane * 16;
-  const bool active = c0 < H;  // H % 32 == 0: 16 whole channels or none
+  if (item >= static_cast<long long>(N) * groups) return;
+  const int t = static_cast<int>(item / groups);
+  const int s0 = static_cast<int>(item - static_cast<long long>(t) * groups) * SPW;
   pdl_wait();
   pdl_trigger();
   const int my_slot = lane < k ? token_slot[static_cast<size_t>(t) * k + lane] : -1;
-  uint4 a = make_uint4(0, 0, 0, 0), b = a;
-  if (active) {
-    const uint16_t* src = x + static_cast<size_t>(t) * H + c0;
-    a = ld_stream(src);
-    b = ld_stream(src + 8);
+  uint4 av[SPW], bv[SPW];
+#pragma unroll
+  for (int u = 0; u < SPW; ++u) {
+    const int cu = (s0 + u) * 512 + lane * 16;
+    av[u] = make_uint4(0, 0, 0, 0);
+    bv[u] = av[u];
+    if (cu < H) {  // H % 32 == 0: 16 whole channels or none
+      const uint16_t* src = x + static_cast<size_t>(t) * H + cu;
+      av[u] = ld_stream(src);
+      bv[u] = ld_stream(src + 8);
+    }
   }
+#pragma unroll
+  for (int u = 0; u < SPW; ++u) {
+  const int s = s0 + u;
+  if (s >= segs) break;  // warp-uniform
+  const uint4 a = av[u], b = bv[u];
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
   uint32_t p[8];  // 24-bit pairs
 #pragma unroll
   for (int i = 0; i < 8; ++i) p[i] = e5m6_code(bf16_lo(w[i])) | (e5m6_code(bf16_hi(w[i])) << 12);
+  if (u > 0) __syncwarp();  // every lane has read the previous segment's stage
   stage[warp][3 * lane] = make_uint2(p[0] | (p[1] << 24), (p[1] >> 8) | (p[2] << 16));
   stage[warp][3 * lane + 1] = make_uint2((p[2] >> 16) | (p[3] << 8), p[4] | (p[5] << 24));
   stage[warp][3 * lane + 2] = make_uint2((p[5] >> 8) | (p[6] << 16), (p[6] >> 16) | (p[7] << 8));
@@ -546,13 +571,14 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int slot = __shfl_sync(kFullMask, my_slot, j);
     if (slot == -1) continue;
     if (slot < -1 || slot >= S) {
-      if (lane == 0) report_bad_index(d_status);
+      if (lane == 0 && u == 0) report_bad_index(d_status);
       continue;
     }
     uint8_t* dst = recv_x + static_cast<size_t>(slot) * row_bytes + static_cast<size_t>(s) * 768;
     if (16 * lane < live) st_stream_v4(dst + 16 * lane, v0);
     if (lane < 16 && 512 + 16 * lane < live) st_stream_v4(dst + 512 + 16 * lane, v1);
   }
+  }  // segments of the warp
 }
 
 // BF16: lane owns 8 channels (one 16-byte vector), a warp covers 256 channels.
@@ -612,6 +638,21 @@ cudaError_t launch_fp8(bool two, const uint16_t* x, int N, int H, int k, const i
                     token_slot, num_rows, recv_x, recv_scale, ld, d_status);
 }
 
+template <int SL>
+cudaError_t launch_mx(bool two, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+                      long long num_rows, uint8_t* recv_x, uint8_t* recv_e8m0, long long ld,
+                      int32_t* d_status, cudaStream_t stream) {
+  const int segs = (H + 511) / 512;
+  const int spw = two ? 2 : 1;
+  const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
+  const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+  if (two)
+    return launch_pdl(dispatch_mxfp8_kernel<SL, 2>, blocks, kWarps * 32, 0, stream, x, N, H, k, token_slot,
+                      num_rows, recv_x, recv_e8m0, ld, d_status);
+  return launch_pdl(dispatch_mxfp8_kernel<SL, 1>, blocks, kWarps * 32, 0, stream, x, N, H, k, token_slot,
+                    num_rows, recv_x, recv_e8m0, ld, d_status);
+}
+
 }  // namespace
 
 long long scale_ld(long long num_rows, int dtype) {
@@ -630,8 +671,6 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   uint8_t* r8 = static_cast<uint8_t*>(recv_x);
   const long long ld = scale_ld(num_rows, dtype);
   if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
-    const long long items = static_cast<long long>(N) * ((H + 511) / 512);
-    const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
     float* f32 = static_cast<float*>(recv_scale);
     uint8_t* e8 = static_cast<uint8_t*>(recv_scale);
     // two segments per warp when k <= 4 (reads of x dominate), else one
@@ -654,13 +693,13 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
                                                     d_status, stream);
     }
     if (scale_layout == MOE_SCALE_MN_MAJOR)
-      return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_MN_MAJOR>, blocks, kWarps * 32, 0, stream,
-                        xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
+      return launch_mx<MOE_SCALE_MN_MAJOR>(two, xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status,
+                                           stream);
     if (scale_layout == MOE_SCALE_MMA_TILED)
-      return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_MMA_TILED>, blocks, kWarps * 32, 0, stream,
-                        xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
-    return launch_pdl(dispatch_mxfp8_kernel<MOE_SCALE_ROW_MAJOR>, blocks, kWarps * 32, 0, stream,
-                      xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status);
+      return launch_mx<MOE_SCALE_MMA_TILED>(two, xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status,
+                                            stream);
+    return launch_mx<MOE_SCALE_ROW_MAJOR>(two, xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status,
+                                          stream);
   } else if (dtype == MOE_DTYPE_FP8_E4M3_TOKEN) {
     // vectors of 8 channels per thread; H <= 16384 -> at most 16
     const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
@@ -678,9 +717,14 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     return launch_pdl(dispatch_fp8_token_kernel<16>, N, kTokenThreads, smem, stream, xs, N, H, k,
                       token_slot, num_rows, r8, sc, d_status);
   } else if (dtype == MOE_DTYPE_E5M6) {
-    const long long items = static_cast<long long>(N) * ((H + 511) / 512);
+    const int segs = (H + 511) / 512;
+    const int spw = k <= 4 ? 2 : 1;  // as the FP8 kernels
+    const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-    return launch_pdl(dispatch_e5m6_kernel, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
+    if (spw == 2)
+      return launch_pdl(dispatch_e5m6_kernel<2>, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
+                        num_rows, r8, d_status);
+    return launch_pdl(dispatch_e5m6_kernel<1>, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
                       num_rows, r8, d_status);
   } else {
     const long long items = static_cast<long long>(N) * ((H + 255) / 256);

@@ -25,7 +25,13 @@ CASES = [_variant(P, "fp8_token"), _variant(P, "mxfp8"),
          Workload("mx_small_h", 77, 96, 16, 3, 4, "softmax", "mxfp8", "random"),
          Workload("tok_ragged", 257, 200, 12, 3, 3, "softmax_renorm", "fp8_token", "random"),
          Workload("tok_max_h", 40, 16384, 32, 4, 4, "softmax", "fp8_token", "random"),
-         Workload("tok_min_h", 50, 8, 8, 2, 2, "softmax", "fp8_token", "random")]
+         Workload("tok_min_h", 50, 8, 8, 2, 2, "softmax", "fp8_token", "random"),
+         # k <= 4: two 512-channel segments per warp; 1536 = 3 whole segments
+         # (16-byte scale stores), 1184 = 2 whole + 160 channels
+         Workload("mx_k2", 500, 1536, 16, 2, 4, "softmax", "mxfp8", "random"),
+         Workload("mx_k4_ragged", 300, 1184, 16, 4, 4, "softmax_renorm", "mxfp8", "random"),
+         Workload("fp8_k2", 500, 1536, 16, 2, 4, "softmax", "fp8", "random"),
+         Workload("fp8_k1_ragged", 333, 1152, 8, 1, 2, "softmax", "fp8", "random")]
 
 
 @pytest.mark.parametrize("w", CASES, ids=[w.name for w in CASES])
