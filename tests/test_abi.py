@@ -284,3 +284,32 @@ def test_selftest_rejects_bad_arguments(api):
     L = api.lib()
     assert L.moe_selftest_bounded_wait(None, None) == api.MOE_ERR_INVALID_ARG
     assert L.moe_selftest_bounded_wait(_P(0x1002), None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_scale_buffer_sizes_agree_with_the_oracle(api):
+    """For every payload type and scale layout, the three independent size
+    rules agree: the library's moe_recv_scale_bytes, the binding's
+    scale_shape, and the oracle's scale_elems x element size.  Undefined
+    pairs are 0 bytes / None / -1 on the three sides."""
+    import math
+
+    import oracle as O
+    elem = {api.MOE_DTYPE_FP8_E4M3: 4, api.MOE_DTYPE_FP8_E4M3_TOKEN: 4, api.MOE_DTYPE_MXFP8_E4M3: 1,
+            api.MOE_DTYPE_NVFP4: 1, api.MOE_DTYPE_FP8_E4M3_UE8M0: 1}
+    layouts = [api.MOE_SCALE_ROW_MAJOR, api.MOE_SCALE_MN_MAJOR, api.MOE_SCALE_MMA_TILED,
+               api.MOE_SCALE_MN_MAJOR_PACK4]
+    checked = 0
+    for dtype, es in elem.items():
+        for lay in layouts:
+            for rows in (1, 3, 4, 15, 16, 127, 128, 129, 1000, 65280):
+                for H in (128, 256, 640, 1024, 7168):
+                    nbytes = api.moe_recv_scale_bytes(rows, H, dtype, lay)
+                    n_or = O.scale_elems(rows, H, dtype, lay)
+                    shape, sdt = api.scale_shape(rows, H, dtype, lay)
+                    if n_or < 0:
+                        assert nbytes == 0 and shape is None, (dtype, lay, rows, H)
+                        continue
+                    assert nbytes == n_or * es, (dtype, lay, rows, H, nbytes, n_or)
+                    assert shape is not None and math.prod(shape) * (1 if sdt == api.torch.uint8 else 4) == nbytes
+                    checked += 1
+    assert checked > 300
