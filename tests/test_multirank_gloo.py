@@ -92,3 +92,24 @@ def test_two_ranks_shard_tokens_and_aggregate():
     out, _ = O.combine(y_full, L.token_slot, wts)
     assert np.array_equal(res["idx"], idx)
     assert np.array_equal(res["out"], out)
+
+
+def test_reference_arm_rank0_prints_other_ranks_exit_quietly():
+    """The comparison arm (the CPU oracle) under a 2-rank launch: rank 0 prints
+    the one JSON line, rank 1 exits 0 without work or output."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+           "--steps", "2", "--warmup", "3"]
+    outs = []
+    for rank in (0, 1):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+        r = subprocess.run(cmd, capture_output=True, text=True, timeout=300, env=env, cwd=root)
+        assert r.returncode == 0, r.stderr[-2000:]
+        outs.append(r.stdout.strip())
+    line = json.loads(outs[0].splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert outs[1] == ""
