@@ -128,6 +128,26 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> torch.T
     return t
 
 
+def _status(d_status: torch.Tensor | None) -> torch.Tensor | None:
+    """The optional device status word: int32 on the GPU, at least one element."""
+    if d_status is not None:
+        _need(d_status, "d_status", torch.int32)
+        if d_status.numel() < 1:
+            raise ValueError("d_status must hold at least one int32")
+    return d_status
+
+
+def _launch(fn, where: str, tensors, *args) -> None:
+    """Calls an entry point that launches kernels.  The library launches on
+    the calling thread's current CUDA device, so every tensor of the call
+    must sit on one device, which is made current for the call."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"{where}: tensors on {sorted(str(d) for d in devs)}; all must be on one CUDA device")
+    with torch.cuda.device(devs.pop()):
+        _check(fn(*args), where)
+
+
 # ---------------------------------------------------------------- gate
 def moe_topk_gate(logits: torch.Tensor, k: int, kind: int, n_groups: int = 1,
                   topk_groups: int = 1, group_topn: int = 1, *, topk_idx=None, topk_w=None,
@@ -141,9 +161,8 @@ def moe_topk_gate(logits: torch.Tensor, k: int, kind: int, n_groups: int = 1,
         topk_w = torch.empty((N, k), dtype=torch.float32, device=logits.device)
     _need(topk_idx, "topk_idx", torch.int32, (N, k))
     _need(topk_w, "topk_w", torch.float32, (N, k))
-    st = _lib.moe_topk_gate(_ptr(logits), N, E, k, kind, n_groups, topk_groups, group_topn,
-                            _ptr(topk_idx), _ptr(topk_w), _stream(stream, logits.device))
-    _check(st, "moe_topk_gate")
+    _launch(_lib.moe_topk_gate, "moe_topk_gate", (logits, topk_idx, topk_w), _ptr(logits), N, E, k, kind,
+            n_groups, topk_groups, group_topn, _ptr(topk_idx), _ptr(topk_w), _stream(stream, logits.device))
     return topk_idx, topk_w
 
 
@@ -178,6 +197,18 @@ class Layout:
                       torch.zeros(1, **i32), align)
 
 
+def _check_layout(out: Layout, N: int, k: int, E: int, R: int, workspace: bool = True) -> None:
+    """A caller-supplied layout must have the shapes of the batch it is filled
+    for: the kernels write every one of its arrays."""
+    for name, shape in (("expert_count", (E,)), ("expert_offset", (E + 1,)), ("rank_count", (R,)),
+                        ("rank_offset", (R + 1,)), ("rank_tokens", (R,)), ("token_slot", (N, k))):
+        _need(getattr(out, name), f"out.{name}", torch.int32, shape)
+    _need(out.slot_token, "out.slot_token", torch.int32, (out.slot_token.numel(),))
+    if workspace:
+        _need(out.workspace, "out.workspace", torch.uint8, (out.workspace.numel(),))
+    _status(out.status)
+
+
 def moe_layout_workspace_bytes(num_tokens: int, k: int, num_experts: int, num_ranks: int) -> int:
     return int(_lib.moe_layout_workspace_bytes(num_tokens, k, num_experts, num_ranks))
 
@@ -198,16 +229,18 @@ def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, 
     E, R = num_experts, num_ranks
     if out is None:
         out = Layout.empty(N, k, E, R, topk_idx.device, align, num_recv_rows)
+    _check_layout(out, N, k, E, R)
     args = (_ptr(out.expert_count), _ptr(out.expert_offset), _ptr(out.rank_count),
             _ptr(out.rank_offset), _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token),
             _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
             _stream(stream, topk_idx.device))
+    tensors = (topk_idx, out.expert_count, out.expert_offset, out.rank_count, out.rank_offset,
+               out.rank_tokens, out.token_slot, out.slot_token, out.workspace, _status(out.status))
     if align == 1 and out.num_rows == N * k:
-        st = _lib.moe_get_layout(_ptr(topk_idx), N, k, E, R, *args)
-        _check(st, "moe_get_layout")
+        _launch(_lib.moe_get_layout, "moe_get_layout", tensors, _ptr(topk_idx), N, k, E, R, *args)
     else:
-        st = _lib.moe_get_layout_aligned(_ptr(topk_idx), N, k, E, R, align, out.num_rows, *args)
-        _check(st, "moe_get_layout_aligned")
+        _launch(_lib.moe_get_layout_aligned, "moe_get_layout_aligned", tensors, _ptr(topk_idx), N, k, E, R,
+                align, out.num_rows, *args)
     out.align = align
     return out
 
@@ -228,12 +261,13 @@ def moe_get_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_ranks: 
     E, R = num_experts, num_ranks
     if out is None:
         out = Layout.empty(N, k, E, R, topk_idx.device)
-    st = _lib.moe_get_layout_noalloc(_ptr(topk_idx), N, k, E, R, _ptr(out.expert_count),
-                                     _ptr(out.expert_offset), _ptr(out.rank_count),
-                                     _ptr(out.rank_offset), _ptr(out.rank_tokens),
-                                     _ptr(out.token_slot), _ptr(out.slot_token), _ptr(out.status),
-                                     _stream(stream, topk_idx.device))
-    _check(st, "moe_get_layout_noalloc")
+    _check_layout(out, N, k, E, R, workspace=False)
+    tensors = (topk_idx, out.expert_count, out.expert_offset, out.rank_count, out.rank_offset,
+               out.rank_tokens, out.token_slot, out.slot_token, _status(out.status))
+    _launch(_lib.moe_get_layout_noalloc, "moe_get_layout_noalloc", tensors, _ptr(topk_idx), N, k, E, R,
+            _ptr(out.expert_count), _ptr(out.expert_offset), _ptr(out.rank_count), _ptr(out.rank_offset),
+            _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token), _ptr(out.status),
+            _stream(stream, topk_idx.device))
     return out
 
 
@@ -312,9 +346,9 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
             recv_scale = torch.empty(shape, dtype=sdt, device=x.device)
         _need(recv_x, "recv_x", torch.uint8, (S, H))
         _need(recv_scale, "recv_scale", sdt, shape)
-    st = _lib.moe_dispatch_ex(_ptr(x), N, H, k, _ptr(token_slot), S, dtype, scale_layout,
-                              _ptr(recv_x), _ptr(recv_scale), _ptr(d_status), _stream(stream, x.device))
-    _check(st, "moe_dispatch")
+    _launch(_lib.moe_dispatch_ex, "moe_dispatch", (x, token_slot, recv_x, recv_scale, _status(d_status)),
+            _ptr(x), N, H, k, _ptr(token_slot), S, dtype, scale_layout, _ptr(recv_x), _ptr(recv_scale),
+            _ptr(d_status), _stream(stream, x.device))
     return recv_x, recv_scale
 
 
@@ -341,9 +375,10 @@ def moe_dispatch_nvfp4(x: torch.Tensor, token_slot: torch.Tensor, *, scale_layou
     _need(recv_x, "recv_x", torch.uint8, (S, H // 2))
     _need(block_scale, "block_scale", torch.uint8, shape)
     _need(row_scale, "row_scale", torch.float32, (S,))
-    st = _lib.moe_dispatch_nvfp4(_ptr(x), N, H, k, _ptr(token_slot), S, scale_layout, _ptr(recv_x),
-                                 _ptr(block_scale), _ptr(row_scale), _ptr(d_status), _stream(stream, x.device))
-    _check(st, "moe_dispatch_nvfp4")
+    _launch(_lib.moe_dispatch_nvfp4, "moe_dispatch_nvfp4",
+            (x, token_slot, recv_x, block_scale, row_scale, _status(d_status)), _ptr(x), N, H, k,
+            _ptr(token_slot), S, scale_layout, _ptr(recv_x), _ptr(block_scale), _ptr(row_scale),
+            _ptr(d_status), _stream(stream, x.device))
     return recv_x, block_scale, row_scale
 
 
@@ -351,8 +386,8 @@ def moe_selftest_bounded_wait(d_status: torch.Tensor, stream=None) -> None:
     """Runs the pipelined kernels' bounded wait on an mbarrier nothing completes;
     after about a second MOE_ERR_TIMEOUT is recorded in ``d_status``."""
     _need(d_status, "d_status", torch.int32, (1,))
-    _check(_lib.moe_selftest_bounded_wait(_ptr(d_status), _stream(stream, d_status.device)),
-           "moe_selftest_bounded_wait")
+    _launch(_lib.moe_selftest_bounded_wait, "moe_selftest_bounded_wait", (d_status,), _ptr(d_status),
+            _stream(stream, d_status.device))
 
 
 def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, expert_count: torch.Tensor, *,
@@ -372,10 +407,10 @@ def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, exper
         scale = torch.empty((E, H), dtype=torch.float32, device=recv.device)
     _need(out, "out", torch.uint8, shape)
     _need(scale, "scale", torch.float32, (E, H))
-    st = _lib.moe_quant_fp8_channel(_ptr(recv), S, H, E, _ptr(expert_offset), _ptr(expert_count),
-                                    int(transpose), _ptr(out), _ptr(scale), _ptr(d_status),
-                                    _stream(stream, recv.device))
-    _check(st, "moe_quant_fp8_channel")
+    _launch(_lib.moe_quant_fp8_channel, "moe_quant_fp8_channel",
+            (recv, expert_offset, expert_count, out, scale, _status(d_status)), _ptr(recv), S, H, E,
+            _ptr(expert_offset), _ptr(expert_count), int(transpose), _ptr(out), _ptr(scale), _ptr(d_status),
+            _stream(stream, recv.device))
     return out, scale
 
 
@@ -405,9 +440,8 @@ def moe_swiglu_quant(h: torch.Tensor, dtype: int, *, slot_token=None, scale_layo
             out_scale = torch.empty(shape, dtype=sdt, device=h.device)
         _need(out, "out", torch.uint8, (S, I))
         _need(out_scale, "out_scale", sdt, shape)
-    st = _lib.moe_swiglu_quant(_ptr(h), S, I, _ptr(slot_token), dtype, scale_layout, _ptr(out),
-                               _ptr(out_scale), _stream(stream, h.device))
-    _check(st, "moe_swiglu_quant")
+    _launch(_lib.moe_swiglu_quant, "moe_swiglu_quant", (h, slot_token, out, out_scale), _ptr(h), S, I,
+            _ptr(slot_token), dtype, scale_layout, _ptr(out), _ptr(out_scale), _stream(stream, h.device))
     return out, out_scale
 
 
@@ -422,9 +456,8 @@ def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor,
     if out is None:
         out = torch.empty((N, H), dtype=torch.bfloat16, device=y.device)
     _need(out, "out", torch.bfloat16, (N, H))
-    st = _lib.moe_combine(_ptr(y), N, H, k, _ptr(token_slot), y.shape[0], _ptr(topk_w), _ptr(out),
-                          _ptr(d_status), _stream(stream, y.device))
-    _check(st, "moe_combine")
+    _launch(_lib.moe_combine, "moe_combine", (y, token_slot, topk_w, out, _status(d_status)), _ptr(y), N, H,
+            k, _ptr(token_slot), y.shape[0], _ptr(topk_w), _ptr(out), _ptr(d_status), _stream(stream, y.device))
     return out
 
 
@@ -439,9 +472,9 @@ def moe_dispatch_backward(grad_recv: torch.Tensor, token_slot: torch.Tensor, *, 
     if grad_x is None:
         grad_x = torch.empty((N, H), dtype=torch.bfloat16, device=grad_recv.device)
     _need(grad_x, "grad_x", torch.bfloat16, (N, H))
-    st = _lib.moe_dispatch_backward(_ptr(grad_recv), N, H, k, _ptr(token_slot), grad_recv.shape[0],
-                                    _ptr(grad_x), _ptr(d_status), _stream(stream, grad_recv.device))
-    _check(st, "moe_dispatch_backward")
+    _launch(_lib.moe_dispatch_backward, "moe_dispatch_backward", (grad_recv, token_slot, grad_x, _status(d_status)),
+            _ptr(grad_recv), N, H, k, _ptr(token_slot), grad_recv.shape[0], _ptr(grad_x), _ptr(d_status),
+            _stream(stream, grad_recv.device))
     return grad_x
 
 
@@ -461,10 +494,10 @@ def moe_combine_backward(grad_out: torch.Tensor, y: torch.Tensor, token_slot: to
         grad_w = torch.empty((N, k), dtype=torch.float32, device=y.device)
     _need(grad_y, "grad_y", torch.bfloat16, tuple(y.shape))
     _need(grad_w, "grad_w", torch.float32, (N, k))
-    st = _lib.moe_combine_backward(_ptr(grad_out), _ptr(y), N, H, k, _ptr(token_slot), y.shape[0],
-                                   _ptr(topk_w), _ptr(grad_y), _ptr(grad_w), _ptr(d_status),
-                                   _stream(stream, y.device))
-    _check(st, "moe_combine_backward")
+    _launch(_lib.moe_combine_backward, "moe_combine_backward",
+            (grad_out, y, token_slot, topk_w, grad_y, grad_w, _status(d_status)), _ptr(grad_out), _ptr(y), N, H,
+            k, _ptr(token_slot), y.shape[0], _ptr(topk_w), _ptr(grad_y), _ptr(grad_w), _ptr(d_status),
+            _stream(stream, y.device))
     return grad_y, grad_w
 
 
@@ -474,8 +507,8 @@ def moe_e4m3_encode(x: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     _need(out, "out", torch.uint8, x.shape)
-    st = _lib.moe_e4m3_encode(_ptr(x), x.numel(), _ptr(out), _stream(stream, x.device))
-    _check(st, "moe_e4m3_encode")
+    _launch(_lib.moe_e4m3_encode, "moe_e4m3_encode", (x, out), _ptr(x), x.numel(), _ptr(out),
+            _stream(stream, x.device))
     return out
 
 

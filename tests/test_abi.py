@@ -313,3 +313,17 @@ def test_scale_buffer_sizes_agree_with_the_oracle(api):
                     assert shape is not None and math.prod(shape) * (1 if sdt == api.torch.uint8 else 4) == nbytes
                     checked += 1
     assert checked > 300
+
+
+def test_binding_rejects_mixed_devices_and_bad_status_words(api):
+    """The binding's own checks, before anything is called: tensors of one
+    call on two devices, and a status word that is not device int32."""
+    import torch
+    called = []
+    with pytest.raises(ValueError, match="one CUDA device"):
+        api._launch(lambda *a: called.append(a) or 0, "probe",
+                    (torch.empty(1), torch.empty(1, device="meta")), 1, 2)
+    assert not called
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        api._status(torch.zeros(1, dtype=torch.int32))
+    assert api._status(None) is None

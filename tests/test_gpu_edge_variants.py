@@ -117,3 +117,20 @@ def test_swiglu_single_row_every_layout():
         if sc is not None:
             assert np.array_equal(np.ascontiguousarray(sc.cpu().numpy().reshape(-1)).view(np.uint8),
                                   r_sc.view(np.uint8)), (dt, lay)
+
+
+def test_mismatched_layout_handle_is_rejected_before_launch():
+    """A caller-supplied layout sized for another batch raises in the binding;
+    nothing is launched, so nothing can be written out of bounds."""
+    from combine_moe_topk_gate_b200 import api
+    idx = torch.zeros((10, 2), dtype=torch.int32, device=DEV)
+    with pytest.raises(ValueError, match="out.token_slot"):
+        api.moe_get_layout(idx, 4, 2, out=api.Layout.empty(8, 2, 4, 2, DEV))       # 8 tokens, not 10
+    with pytest.raises(ValueError, match="out.expert_count"):
+        api.moe_get_layout(idx, 4, 2, out=api.Layout.empty(10, 2, 8, 2, DEV))      # 8 experts, not 4
+    with pytest.raises(ValueError, match="out.rank_count"):
+        api.moe_get_layout_noalloc(idx, 4, 2, out=api.Layout.empty(10, 2, 4, 4, DEV))  # 4 ranks, not 2
+    with pytest.raises(ValueError, match="d_status"):
+        api.moe_combine(torch.zeros((20, 64), dtype=torch.bfloat16, device=DEV), idx,
+                        torch.zeros((10, 2), dtype=torch.float32, device=DEV),
+                        d_status=torch.zeros(1, dtype=torch.int32))                   # host status word
