@@ -144,8 +144,12 @@ def _launch(fn, where: str, tensors, *args) -> None:
     devs = {t.device for t in tensors if t is not None}
     if len(devs) != 1:
         raise ValueError(f"{where}: tensors on {sorted(str(d) for d in devs)}; all must be on one CUDA device")
-    with torch.cuda.device(devs.pop()):
+    dev = devs.pop()
+    if dev.index == torch.cuda.current_device():
         _check(fn(*args), where)
+    else:
+        with torch.cuda.device(dev):
+            _check(fn(*args), where)
 
 
 # ---------------------------------------------------------------- gate
