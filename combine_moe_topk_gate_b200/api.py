@@ -111,8 +111,16 @@ def _ptr(t: torch.Tensor | None):
 
 
 def _stream(stream, device) -> ctypes.c_void_p:
+    """The stream handle to enqueue on: the device's current stream, or the
+    caller's stream, which must belong to the tensors' device (the library
+    launches on the current device, and a stream of another device there is
+    a CUDA error)."""
     if stream is None:
         stream = torch.cuda.current_stream(device)
+    else:
+        sdev = getattr(stream, "device", None)
+        if sdev is not None and device is not None and torch.device(sdev) != torch.device(device):
+            raise ValueError(f"stream is on {sdev}, the tensors on {device}")
     return ctypes.c_void_p(stream.cuda_stream)
 
 
@@ -126,6 +134,15 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None) -> torch.T
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
+
+
+def _slots_of(token_slot: torch.Tensor, N: int) -> int:
+    """k of a token_slot array that must describe the N tokens of x: int32 [N, k]
+    (the kernels read N*k slots)."""
+    _need(token_slot, "token_slot", torch.int32)
+    if token_slot.dim() != 2 or token_slot.shape[0] != N:
+        raise ValueError(f"token_slot must have shape ({N}, k), got {tuple(token_slot.shape)}")
+    return int(token_slot.shape[1])
 
 
 def _status(d_status: torch.Tensor | None) -> torch.Tensor | None:
@@ -191,9 +208,13 @@ class Layout:
         return self.slot_token.numel()
 
     @staticmethod
-    def empty(N: int, k: int, E: int, R: int, device, align: int = 1, num_rows: int | None = None) -> "Layout":
+    def empty(N: int, k: int, E: int, R: int, device, align: int = 1, num_rows: int | None = None,
+              workspace: bool = True) -> "Layout":
+        """Uninitialised arrays for an N x k batch over E experts and R ranks;
+        ``workspace=False`` gives a 0-byte workspace (for the no-workspace
+        entry point)."""
         i32 = dict(dtype=torch.int32, device=device)
-        ws = moe_layout_workspace_bytes(N, k, E, R)
+        ws = moe_layout_workspace_bytes(N, k, E, R) if workspace else 0
         rows = num_rows if num_rows is not None else moe_aligned_recv_rows(N, k, E, align)
         return Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32),
                       torch.empty(R + 1, **i32), torch.empty(R, **i32), torch.empty((N, k), **i32),
@@ -264,14 +285,19 @@ def moe_get_layout_noalloc(topk_idx: torch.Tensor, num_experts: int, num_ranks: 
     N, k = topk_idx.shape
     E, R = num_experts, num_ranks
     if out is None:
-        out = Layout.empty(N, k, E, R, topk_idx.device)
+        out = Layout.empty(N, k, E, R, topk_idx.device, workspace=False)
     _check_layout(out, N, k, E, R, workspace=False)
+    # the entry point writes the packed layout: exactly N*k receive rows
+    if out.slot_token.numel() != N * k:
+        raise ValueError(f"out.slot_token must have N*k = {N * k} entries for the packed layout, "
+                         f"got {out.slot_token.numel()}")
     tensors = (topk_idx, out.expert_count, out.expert_offset, out.rank_count, out.rank_offset,
                out.rank_tokens, out.token_slot, out.slot_token, _status(out.status))
     _launch(_lib.moe_get_layout_noalloc, "moe_get_layout_noalloc", tensors, _ptr(topk_idx), N, k, E, R,
             _ptr(out.expert_count), _ptr(out.expert_offset), _ptr(out.rank_count), _ptr(out.rank_offset),
             _ptr(out.rank_tokens), _ptr(out.token_slot), _ptr(out.slot_token), _ptr(out.status),
             _stream(stream, topk_idx.device))
+    out.align = 1
     return out
 
 
@@ -327,8 +353,7 @@ def moe_dispatch(x: torch.Tensor, token_slot: torch.Tensor, dtype: int, *, recv_
     the MN-major or MMA-tiled scale layouts (moe_dispatch_ex)."""
     _need(x, "x", torch.bfloat16)
     N, H = x.shape
-    _need(token_slot, "token_slot", torch.int32)
-    k = token_slot.shape[1]
+    k = _slots_of(token_slot, N)
     S = num_recv_rows if num_recv_rows is not None else (recv_x.shape[0] if recv_x is not None else N * k)
     if dtype == MOE_DTYPE_BF16:
         if recv_x is None:
@@ -364,8 +389,7 @@ def moe_dispatch_nvfp4(x: torch.Tensor, token_slot: torch.Tensor, *, scale_layou
     16 channels, in ``scale_layout``), row_scale fp32 [S])``."""
     _need(x, "x", torch.bfloat16)
     N, H = x.shape
-    _need(token_slot, "token_slot", torch.int32)
-    k = token_slot.shape[1]
+    k = _slots_of(token_slot, N)
     S = num_recv_rows if num_recv_rows is not None else (recv_x.shape[0] if recv_x is not None else N * k)
     shape, _ = scale_shape(S, H, MOE_DTYPE_NVFP4, scale_layout)
     if shape is None:
@@ -453,6 +477,8 @@ def moe_combine(y: torch.Tensor, token_slot: torch.Tensor, topk_w: torch.Tensor,
                 d_status=None, stream=None) -> torch.Tensor:
     """Weighted gather-reduce of expert outputs ``y`` (bf16 [N*k,H]) -> bf16 [N,H]."""
     _need(y, "y", torch.bfloat16)
+    if y.dim() != 2:
+        raise ValueError(f"y must be 2-D [S, H], got {tuple(y.shape)}")
     _need(token_slot, "token_slot", torch.int32)
     N, k = token_slot.shape
     H = y.shape[1]
@@ -470,6 +496,8 @@ def moe_dispatch_backward(grad_recv: torch.Tensor, token_slot: torch.Tensor, *, 
     """Gradient of dispatch: slot-order sum of each token's rows of ``grad_recv``
     (bf16 [N*k,H]) -> bf16 [N,H]."""
     _need(grad_recv, "grad_recv", torch.bfloat16)
+    if grad_recv.dim() != 2:
+        raise ValueError(f"grad_recv must be 2-D [S, H], got {tuple(grad_recv.shape)}")
     _need(token_slot, "token_slot", torch.int32)
     N, k = token_slot.shape
     H = grad_recv.shape[1]
@@ -486,11 +514,13 @@ def moe_combine_backward(grad_out: torch.Tensor, y: torch.Tensor, token_slot: to
                          topk_w: torch.Tensor, *, grad_y=None, grad_w=None, d_status=None,
                          stream=None):
     """Gradients of combine: ``(grad_y bf16 [N*k,H], grad_w fp32 [N,k])``."""
-    _need(grad_out, "grad_out", torch.bfloat16)
-    _need(y, "y", torch.bfloat16)
     _need(token_slot, "token_slot", torch.int32)
     N, k = token_slot.shape
-    H = grad_out.shape[1]
+    _need(y, "y", torch.bfloat16)
+    if y.dim() != 2:
+        raise ValueError(f"y must be 2-D [S, H], got {tuple(y.shape)}")
+    H = y.shape[1]
+    _need(grad_out, "grad_out", torch.bfloat16, (N, H))
     _need(topk_w, "topk_w", torch.float32, (N, k))
     if grad_y is None:
         grad_y = torch.empty(tuple(y.shape), dtype=torch.bfloat16, device=y.device)

@@ -7,18 +7,13 @@ with CUDA events; the same command is what a profiler capture of that op runs.
 ops: gate, layout, dispatch_<payload> (bf16, fp8, fp8_token, mxfp8, nvfp4,
 e5m6), combine, dispatch_backward, combine_backward, swiglu_fp8 (R receive
 rows of h = [gate | up], I channels each), quant_fp8_channel (the aligned
-receive buffer at align 128); hbm_rates (no op of the path: read-only,
-write-only and copy rates of plain library calls on 1 GiB buffers, the
-context for the write-heavy dispatch).  The first five launches are warm-up; the
+receive buffer at align 128).  The first five launches are warm-up; the
 timed ones follow (each launch reuses resident inputs, so a capture of launch
 6 or later sees the steady state).
 """
 from __future__ import annotations
 
 import argparse
-import ctypes
-import glob
-import os
 
 import torch
 
@@ -90,40 +85,6 @@ def build(op: str, workload: str, rows: int | None, inter: int, device):
     raise SystemExit(f"unknown op {op}")
 
 
-def hbm_rates(device, reps: int) -> None:
-    """HBM rates of library calls on 1 GiB buffers, CUDA events, back to back
-    (each buffer is 8x the L2): fp32 sum (read), fill and cudaMemsetAsync
-    (write), copy (read + write)."""
-    n = 1 << 30
-    a = torch.full((n,), 1, dtype=torch.uint8, device=device)
-    b = torch.full((n,), 2, dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream(device)
-
-    def rate(fn, nbytes):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize(device)
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record()
-        for _ in range(reps):
-            fn()
-        t1.record()
-        t1.synchronize()
-        us = t0.elapsed_time(t1) / reps * 1e3
-        return f"{us:.1f} us, {nbytes / us / 1e3:.0f} GB/s"
-
-    af = a.view(torch.float32)
-    print("read  (torch sum, fp32)   ", rate(lambda: af.sum(), n))
-    print("write (torch fill_)       ", rate(lambda: a.fill_(3), n))
-    libs = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
-                                  "libcudart.so*"))
-    if libs:
-        rt = ctypes.CDLL(libs[0])
-        rt.cudaMemsetAsync.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p]
-        print("write (cudaMemsetAsync)   ", rate(lambda: rt.cudaMemsetAsync(a.data_ptr(), 0, n, stream.cuda_stream), n))
-    print("copy  (torch copy_)       ", rate(lambda: b.copy_(a), 2 * n))
-
-
 def main() -> None:
     p = argparse.ArgumentParser()
     p.add_argument("op")
@@ -133,9 +94,6 @@ def main() -> None:
     p.add_argument("--inter", type=int, default=2048)
     a = p.parse_args()
     device = torch.device("cuda", 0)
-    if a.op == "hbm_rates":
-        hbm_rates(device, a.reps)
-        return
     launch, nbytes = build(a.op, a.workload, a.rows, a.inter, device)
     for _ in range(5):
         launch()

@@ -134,3 +134,46 @@ def test_mismatched_layout_handle_is_rejected_before_launch():
         api.moe_combine(torch.zeros((20, 64), dtype=torch.bfloat16, device=DEV), idx,
                         torch.zeros((10, 2), dtype=torch.float32, device=DEV),
                         d_status=torch.zeros(1, dtype=torch.int32))                   # host status word
+    # the no-workspace entry point writes the packed layout's N*k rows: a
+    # handle with another row count (or an aligned one) is refused
+    with pytest.raises(ValueError, match="N\\*k"):
+        api.moe_get_layout_noalloc(idx, 4, 2, out=api.Layout.empty(10, 2, 4, 2, DEV, num_rows=12))
+    with pytest.raises(ValueError, match="N\\*k"):
+        api.moe_get_layout_noalloc(idx, 4, 2, out=api.Layout.empty(10, 2, 4, 2, DEV, align=8))
+
+
+def test_shape_mismatches_are_rejected_before_launch():
+    """Arrays whose shapes disagree with the batch raise in the binding before
+    any kernel could read or write past them."""
+    from combine_moe_topk_gate_b200 import api
+    x = torch.zeros((10, 128), dtype=torch.bfloat16, device=DEV)
+    short = torch.zeros((8, 2), dtype=torch.int32, device=DEV)      # 8 tokens' slots for 10 tokens
+    for dt in (api.MOE_DTYPE_BF16, api.MOE_DTYPE_FP8_E4M3):
+        with pytest.raises(ValueError, match="token_slot"):
+            api.moe_dispatch(x, short, dt)
+    with pytest.raises(ValueError, match="token_slot"):
+        api.moe_dispatch_nvfp4(x, short)
+    with pytest.raises(ValueError, match="token_slot"):
+        api.moe_dispatch(x, torch.zeros((12, 2), dtype=torch.int32, device=DEV), 0)
+    slots = torch.zeros((10, 2), dtype=torch.int32, device=DEV)
+    w = torch.zeros((10, 2), dtype=torch.float32, device=DEV)
+    y = torch.zeros((20, 128), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ValueError, match="grad_out"):   # fewer rows than tokens
+        api.moe_combine_backward(torch.zeros((9, 128), dtype=torch.bfloat16, device=DEV), y, slots, w)
+    with pytest.raises(ValueError, match="grad_out"):   # another width than y
+        api.moe_combine_backward(torch.zeros((10, 64), dtype=torch.bfloat16, device=DEV), y, slots, w)
+    with pytest.raises(ValueError, match="y must be 2-D"):
+        api.moe_combine(torch.zeros(20 * 128, dtype=torch.bfloat16, device=DEV), slots, w)
+    with pytest.raises(ValueError, match="grad_recv"):
+        api.moe_dispatch_backward(torch.zeros(20 * 128, dtype=torch.bfloat16, device=DEV), slots)
+
+
+def test_stream_of_another_device_is_rejected():
+    from combine_moe_topk_gate_b200 import api
+
+    class _OtherDeviceStream:
+        device = torch.device("cuda", torch.cuda.device_count())   # a device that is not the tensors'
+        cuda_stream = 0
+    logits = torch.zeros((4, 8), dtype=torch.float32, device=DEV)
+    with pytest.raises(ValueError, match="stream is on"):
+        api.moe_topk_gate(logits, 2, api.MOE_GATE_SOFTMAX, stream=_OtherDeviceStream())
