@@ -22,7 +22,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 3; }
+int moe_abi_version(void) { return 4; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -356,6 +356,14 @@ moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_t
   return from_cuda(moe::launch_combine_backward(grad_out, y, N, H, k, token_slot, num_recv_rows,
                                                 topk_w, grad_y, grad_w, d_status,
                                                 as_stream(stream)));
+}
+
+moe_status_t moe_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
+                           moe_stream_t stream) {
+  if (n == 0) return MOE_OK;
+  if ((!exp_out && !sigmoid_out) || !aligned(exp_out, 16) || !aligned(sigmoid_out, 16))
+    return MOE_ERR_INVALID_ARG;
+  return from_cuda(moe::launch_gate_math(first, n, exp_out, sigmoid_out, as_stream(stream)));
 }
 
 moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream) {

@@ -451,6 +451,25 @@ moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_t
  */
 moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream);
 
+/*
+ * moe_gate_math -- diagnostics: the gate's exp and sigmoid, exposed on their
+ * own (as moe_e4m3_encode exposes dispatch's encoder).  For i in [0, n) the
+ * input x_i is the fp32 whose bit pattern is (first + i) mod 2^32, so one
+ * call can cover any run of patterns without an input array:
+ *   exp_out[i]     = the exp every gate kind uses (Cody-Waite reduction with
+ *                    ln2 split into a 16-bit head and a tail, degree-7 Taylor
+ *                    polynomial by Horner, input clamped to [-87, 88] by
+ *                    IEEE min/max, so a NaN input is taken as -87);
+ *   sigmoid_out[i] = 1 / (1 + exp(-x_i)), each operation rounded once, the
+ *                    score of the group-limited kind.
+ * "DeepSeek, DeepEP 오픈소스 공개", Topic Body: group-limited gating, whose
+ * group scores are sums of these sigmoids.  Either output may be NULL (not
+ * both); outputs are device fp32 arrays of n elements, 16-byte aligned.
+ * n may be 0.
+ */
+moe_status_t moe_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
+                           moe_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(moe_status_t status);
 

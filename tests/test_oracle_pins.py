@@ -56,6 +56,11 @@ def test_dexp_vs_float64_exp_dense():
 def test_dexp_saturation_and_monotone():
     assert O.dexp(-100.0) == O.dexp(-87.0)
     assert O.dexp(100.0) == O.dexp(88.0)
+    assert O.dexp(float("inf")) == O.dexp(88.0) and O.dexp(float("-inf")) == O.dexp(-87.0)
+    # the clamp takes a NaN input to -87 (NaN is outside the contract; the
+    # routine is total so that every fp32 pattern has a defined result)
+    assert O.dexp(float("nan")) == O.dexp(-87.0)
+    assert O.sigmoid(float("nan")) == O.sigmoid(87.0) == 1.0
     x = np.sort(np.random.default_rng(2).uniform(-90, 90, 500_000).astype(np.float32))
     assert (np.diff(O.dexp_array(x)) >= 0).all()
 
