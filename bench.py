@@ -53,7 +53,10 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--no-backward", action="store_true", help="skip timing the backward ops")
+    p.add_argument("--no-backward", action="store_true",
+                   help="skip timing the backward ops, the dispatch payload variants and the aligned layout")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the per-workload summary of the other four workloads")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle baseline CPU budget (s)")
     p.add_argument("--tokens", type=int, default=None,
                    help="override the workload's token count (profiling captures of a smaller case)")
@@ -67,6 +70,32 @@ def describe(w) -> str:
     return (f"{w.name}: N={w.N} tokens, H={w.H}, E={w.E} experts, top-{w.k}, {gate}, "
             f"R={w.R} logical ranks, {w.dtype.upper()} dispatch, BF16 combine, "
             f"expert outputs {'= dispatched rows' if w.expert_out == 'identity' else 'seeded bf16 N(0,1)'}")
+
+
+def config_of(w, world: int) -> dict:
+    """The workload description both arms print (ours and the oracle arm)."""
+    return {"workload": describe(w), "tokens_per_gpu": w.N, "hidden": w.H, "experts": w.E,
+            "topk": w.k, "logical_ranks": w.R, "payload": f"x bf16, dispatch {w.dtype}, out bf16",
+            "l2": "flushed before every step, outside the events: a write of 2x the L2 size, "
+                  "then a read of another 2x L2 buffer (the step starts cold and clean)",
+            "timing": "step captured once as a CUDA graph and replayed; step time from events "
+                      "at the graph's ends, per-op times from a second graph with event nodes "
+                      "between the ops; medians over the timed steps",
+            "parallelism": f"replicas x{world} (tokens sharded, no collective)"}
+
+
+def host_description() -> dict:
+    """Host cores and CPU model (the machine the oracle baseline runs on)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
 
 
 def measured_peak():
@@ -253,7 +282,8 @@ def cpu_baseline(w, inp, budget_s):
             break
     return {"value": n * reps / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{reps} pass(es) over the first {n} of the {w.N} tokens of the {w.name} batch "
-                      f"(seed 0): gate+layout+dispatch+combine, single-threaded C oracle, {dt:.1f} s"}
+                      f"(seed 0): gate+layout+dispatch+combine, single-threaded C oracle, {dt:.1f} s",
+            **host_description()}
 
 
 def workload(args):
@@ -279,278 +309,347 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic", "config": {"workload": describe(w), "tokens_per_step": n},
+        "data": "synthetic", "config": config_of(w, world),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"first {n} of {w.N} tokens per step, single-threaded C oracle"},
+                         "sample": f"each step: gate+layout+dispatch+combine over the first {n} of the "
+                                   f"{w.N} tokens of the {w.name} batch (seed 0), single-threaded C oracle",
+                         **host_description()},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------- our arm
+OPS = ("gate", "layout", "dispatch", "combine")
+
+
+class L2Flush:
+    """Before every timed step: write a buffer of twice the L2 size (evicts
+    every line), then read another one (so the lines left behind are clean,
+    not dirty lines the next step would have to write back)."""
+
+    def __init__(self, device):
+        l2 = torch.cuda.get_device_properties(device).L2_cache_size
+        self.w = torch.empty(2 * l2, dtype=torch.uint8, device=device)
+        self.r = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=device)
+
+    def zero_(self):
+        self.w.zero_()
+        self.r.max()
+
+
+class StepRunner:
+    """Device buffers of one workload and the four calls of one step, each
+    through the library's public binding."""
+
+    def __init__(self, api, w, inp, device):
+        self.api, self.w, self.device = api, w, device
+        self.logits = inp.logits.to(device)
+        self.x = inp.x.to(device)
+        self.y_in = inp.y.to(device) if inp.y is not None else None
+        self.idx = torch.empty((w.N, w.k), dtype=torch.int32, device=device)
+        self.wts = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
+        self.L = api.Layout.empty(w.N, w.k, w.E, w.R, device)
+        if w.dtype != "bf16":
+            self.recv = torch.empty((w.S, w.H), dtype=torch.uint8, device=device)
+            shape, sdt = api.scale_shape(w.S, w.H, w.dtype_code)
+            self.scale = torch.empty(shape, dtype=sdt, device=device)
+        else:
+            self.recv = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
+            self.scale = None
+        self.out = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
+        self.y = self.recv if w.expert_out == "identity" else self.y_in
+
+    def ops(self, stream=None):
+        api, w, L = self.api, self.w, self.L
+        return {
+            "gate": lambda: api.moe_topk_gate(self.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
+                                              w.group_topn, topk_idx=self.idx, topk_w=self.wts, stream=stream),
+            "layout": lambda: api.moe_get_layout(self.idx, w.E, w.R, out=L, stream=stream),
+            "dispatch": lambda: api.moe_dispatch(self.x, L.token_slot, w.dtype_code, recv_x=self.recv,
+                                                 recv_scale=self.scale, d_status=L.status, stream=stream),
+            "combine": lambda: api.moe_combine(self.y, L.token_slot, self.wts, out=self.out,
+                                               d_status=L.status, stream=stream),
+        }
+
+    def step(self, ev=None):
+        stream = torch.cuda.current_stream(self.device)  # the capture stream inside torch.cuda.graph
+        for j, fn in enumerate(self.ops(stream).values()):
+            if ev:
+                ev[j].record(stream)
+            fn()
+        if ev:
+            ev[len(OPS)].record(stream)
+
+    def check_status(self, when: str):
+        if int(self.L.status.item()) != 0:
+            raise RuntimeError(f"device status {int(self.L.status.item())} {when}")
+
+    def capture(self, flush, warmup: int):
+        """Eager warm-up, then the step captured once as a CUDA graph and
+        replayed, so the timed interval is device time of the kernels back to
+        back (their launches overlap through programmatic dependent launch),
+        not the binding's launch overhead.  graph_step has events only at its
+        ends and gives the step time; graph_ops has an event-record node
+        between the ops (which also cuts the launch overlap) and gives the
+        per-op breakdown."""
+        for _ in range(warmup):
+            flush.zero_()
+            self.step()
+        torch.cuda.synchronize(self.device)
+        self.check_status("after warm-up")
+        dev = self.device
+        self.ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        self.graph_step = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_step):
+            self.ends[0].record(torch.cuda.current_stream(dev))
+            self.step()
+            self.ends[1].record(torch.cuda.current_stream(dev))
+        self.evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(OPS) + 1)]
+        self.graph_ops = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_ops):
+            self.step(self.evs)
+        for _ in range(warmup):
+            for g in (self.graph_step, self.graph_ops):
+                flush.zero_()
+                g.replay()
+        torch.cuda.synchronize(dev)
+
+    def timed(self, steps: int, flush):
+        """(step times in ms, {op: [ms]}) over `steps` replays of each graph."""
+        step_ms, per_op = [], {n: [] for n in OPS}
+        for _ in range(steps):
+            flush.zero_()
+            self.graph_step.replay()
+            self.ends[1].synchronize()
+            step_ms.append(self.ends[0].elapsed_time(self.ends[1]))
+        for _ in range(steps):
+            flush.zero_()
+            self.graph_ops.replay()
+            self.evs[-1].synchronize()
+            for j, n in enumerate(OPS):
+                per_op[n].append(self.evs[j].elapsed_time(self.evs[j + 1]))
+        torch.cuda.synchronize(self.device)
+        self.check_status("after the timed steps")
+        return step_ms, per_op
+
+
+def summary_of(w, step_ms, per_op, isolated, peak, world=1) -> dict:
+    """Medians of one workload's timed steps, with the dispatch and combine
+    roofline fractions (in the step and alone).  Decode- and tiny-sized steps
+    move a few MB and are bound by launch and memory latency, not bandwidth:
+    their fractions are reported but do not describe the kernels' bound."""
+    ab = algorithmic_bytes(w)
+    med = {n: statistics.median(v) * 1e3 for n, v in per_op.items()}
+    st = statistics.median(step_ms) * 1e3
+    latency_bound = ab["combine"] < 64e6
+    ops = {}
+    for n in ("dispatch", "combine"):
+        iso = isolated.get(n) or None
+        ops[n] = {"in_step_us": round(med[n], 2), "frac": ab[n] / (med[n] * 1e-6) / 1e9 / peak,
+                  "isolated_us": iso, "isolated_frac": (ab[n] / (iso * 1e-6) / 1e9 / peak) if iso else None,
+                  "algorithmic_bytes": ab[n]}
+    return {"config": describe(w), "tokens": w.N,
+            "step_us": {"median": round(st, 2), "mean": round(statistics.mean(step_ms) * 1e3, 2),
+                        "min": round(min(step_ms) * 1e3, 2), "max": round(max(step_ms) * 1e3, 2)},
+            "tokens_per_s": w.N * world / (st * 1e-6),
+            "per_op_us": {n: round(v, 2) for n, v in med.items()},
+            "dispatch_combine_tokens_per_s": w.N * world / ((med["dispatch"] + med["combine"]) * 1e-6),
+            **ops, "bound": "latency" if latency_bound else "hbm"}
+
+
+def other_workloads(api, main, device, steps, warmup, flush, peak) -> dict:
+    """Every other workload measured the same way (seed 0), one after another."""
+    res = {}
+    for name in ("tiny", "decode", "prefill", "skewed", "mixtral"):
+        if name == main:
+            continue
+        w = WORKLOADS[name]
+        r = StepRunner(api, w, make_inputs(w, 0), device)
+        r.capture(flush, warmup)
+        step_ms, per_op = r.timed(steps, flush)
+        iso = isolated_op_times(r.ops, flush, device)
+        res[name] = summary_of(w, step_ms, per_op, iso, peak)
+        del r
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, device):
     from combine_moe_topk_gate_b200 import api
     w = workload(args)
     inp = make_inputs(w, rank)
     stream = torch.cuda.current_stream(device)
-    logits = inp.logits.to(device)
-    x = inp.x.to(device)
-    y_in = inp.y.to(device) if inp.y is not None else None
-    idx = torch.empty((w.N, w.k), dtype=torch.int32, device=device)
-    wts = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
-    L = api.Layout.empty(w.N, w.k, w.E, w.R, device)
-    if w.dtype != "bf16":
-        recv = torch.empty((w.S, w.H), dtype=torch.uint8, device=device)
-        shape, sdt = api.scale_shape(w.S, w.H, w.dtype_code)
-        scale = torch.empty(shape, dtype=sdt, device=device)
-    else:
-        recv = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
-        scale = None
-    out = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
-    y = recv if w.expert_out == "identity" else y_in
-    l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    flush_w = torch.empty(2 * l2, dtype=torch.uint8, device=device)
-    flush_r = torch.zeros(2 * l2 // 4, dtype=torch.float32, device=device)
-
-    class _Flush:
-        # write a buffer of twice the L2 size (evicts every line), then read
-        # another one (so the lines left behind are clean, not dirty lines the
-        # next step would have to write back)
-        @staticmethod
-        def zero_():
-            flush_w.zero_()
-            flush_r.max()
-
-    flush = _Flush()
-
-    def step_ops():
-        return {
-            "gate": lambda: api.moe_topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
-                                              w.group_topn, topk_idx=idx, topk_w=wts),
-            "layout": lambda: api.moe_get_layout(idx, w.E, w.R, out=L),
-            "dispatch": lambda: api.moe_dispatch(x, L.token_slot, w.dtype_code, recv_x=recv,
-                                                 recv_scale=scale, d_status=L.status),
-            "combine": lambda: api.moe_combine(y, L.token_slot, wts, out=out, d_status=L.status),
-        }
-
-    def step(ev=None):
-        stream = torch.cuda.current_stream(device)  # the capture stream inside torch.cuda.graph
-        if ev: ev[0].record(stream)
-        api.moe_topk_gate(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn,
-                          topk_idx=idx, topk_w=wts, stream=stream)
-        if ev: ev[1].record(stream)
-        api.moe_get_layout(idx, w.E, w.R, out=L, stream=stream)
-        if ev: ev[2].record(stream)
-        api.moe_dispatch(x, L.token_slot, w.dtype_code, recv_x=recv, recv_scale=scale,
-                         d_status=L.status, stream=stream)
-        if ev: ev[3].record(stream)
-        api.moe_combine(y, L.token_slot, wts, out=out, d_status=L.status, stream=stream)
-        if ev: ev[4].record(stream)
-
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    torch.cuda.synchronize(device)
-    if int(L.status.item()) != 0:
-        raise RuntimeError(f"device status {int(L.status.item())} after warm-up")
-
-    # The step is captured once as a CUDA graph and replayed, so the timed
-    # interval is device time of the 5 kernels back to back (their launches
-    # overlap through programmatic dependent launch), not the Python binding's
-    # launch overhead.  graph_step has events only at its ends and gives the
-    # step time; graph_ops has an event-record node between the ops (which
-    # also cuts the launch overlap) and gives the per-op breakdown.
-    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-    graph_step = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_step):
-        ends[0].record(torch.cuda.current_stream(device))
-        step()
-        ends[1].record(torch.cuda.current_stream(device))
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-    graph_ops = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph_ops):
-        step(evs)
-    for _ in range(args.warmup):
-        for g in (graph_step, graph_ops):
-            flush.zero_()
-            g.replay()
-    torch.cuda.synchronize(device)
-    per_op = {n: [] for n in ("gate", "layout", "dispatch", "combine")}
-    step_ms = []
+    flush = L2Flush(device)
+    r = StepRunner(api, w, inp, device)
+    r.capture(flush, args.warmup)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
     with ClockSampler(device.index) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            graph_step.replay()
-            ends[1].synchronize()
-            step_ms.append(ends[0].elapsed_time(ends[1]))
-        for i in range(args.steps):
-            flush.zero_()
-            graph_ops.replay()
-            evs[4].synchronize()
-            for j, n in enumerate(per_op):
-                per_op[n].append(evs[j].elapsed_time(evs[j + 1]))
-        torch.cuda.synchronize(device)
-    if world > 1:
-        torch.distributed.barrier()
-    if int(L.status.item()) != 0:
-        raise RuntimeError(f"device status {int(L.status.item())} after the timed steps")
-    max_total_ms = max_over_ranks(sum(step_ms), world, device)
+        step_ms, per_op = r.timed(args.steps, flush)
+        if world > 1:
+            torch.distributed.barrier()
+        max_total_ms = max_over_ranks(sum(step_ms), world, device)
 
-    isolated = isolated_op_times(step_ops, flush, device)
-    backward = None
-    if not args.no_backward:
-        # backward ops on the same layout, timed alone (cold, clean L2)
-        gen = torch.Generator(device="cpu").manual_seed(1234)
-        grad_recv = torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
-        grad_out = torch.randn(w.N, w.H, generator=gen).to(torch.bfloat16).to(device)
-        y_b = y_in if y_in is not None else torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
-        grad_x = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
-        grad_y = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
-        grad_w = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
+        isolated = isolated_op_times(r.ops, flush, device)
+        L, idx, wts, x, y_in, out = r.L, r.idx, r.wts, r.x, r.y_in, r.out
+        recv = r.recv
+        peak, peak_kind = measured_peak()
+        workloads = None
+        if world == 1 and not args.no_workloads and args.tokens is None:
+            workloads = {w.name: summary_of(w, step_ms, per_op, isolated, peak)}
+            workloads.update(other_workloads(api, w.name, device, args.steps, args.warmup, flush, peak))
+        backward = None
+        if not args.no_backward:
+            # backward ops on the same layout, timed alone (cold, clean L2)
+            gen = torch.Generator(device="cpu").manual_seed(1234)
+            grad_recv = torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
+            grad_out = torch.randn(w.N, w.H, generator=gen).to(torch.bfloat16).to(device)
+            y_b = y_in if y_in is not None else torch.randn(w.S, w.H, generator=gen).to(torch.bfloat16).to(device)
+            grad_x = torch.empty((w.N, w.H), dtype=torch.bfloat16, device=device)
+            grad_y = torch.empty((w.S, w.H), dtype=torch.bfloat16, device=device)
+            grad_w = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
 
-        def bwd_ops():
-            return {
-                "dispatch_backward": lambda: api.moe_dispatch_backward(
-                    grad_recv, L.token_slot, grad_x=grad_x, d_status=L.status),
-                "combine_backward": lambda: api.moe_combine_backward(
-                    grad_out, y_b, L.token_slot, wts, grad_y=grad_y, grad_w=grad_w, d_status=L.status),
-            }
-        bt = isolated_op_times(bwd_ops, flush, device)
-        ab_all = algorithmic_bytes(w)
-        peak_b, _ = measured_peak()
-        backward = {n: {"us": bt[n], "gbs": ab_all[n] / (bt[n] * 1e-6) / 1e9 if bt[n] else None,
-                        "frac": ab_all[n] / (bt[n] * 1e-6) / 1e9 / peak_b if bt[n] else None,
-                        "algorithmic_bytes": ab_all[n]} for n in bt}
-        torch.cuda.synchronize(device)
-        if int(L.status.item()) != 0:
-            raise RuntimeError(f"device status {int(L.status.item())} after the backward ops")
+            def bwd_ops():
+                return {
+                    "dispatch_backward": lambda: api.moe_dispatch_backward(
+                        grad_recv, L.token_slot, grad_x=grad_x, d_status=L.status),
+                    "combine_backward": lambda: api.moe_combine_backward(
+                        grad_out, y_b, L.token_slot, wts, grad_y=grad_y, grad_w=grad_w, d_status=L.status),
+                }
+            bt = isolated_op_times(bwd_ops, flush, device)
+            ab_all = algorithmic_bytes(w)
+            peak_b, _ = measured_peak()
+            backward = {n: {"us": bt[n], "gbs": ab_all[n] / (bt[n] * 1e-6) / 1e9 if bt[n] else None,
+                            "frac": ab_all[n] / (bt[n] * 1e-6) / 1e9 / peak_b if bt[n] else None,
+                            "algorithmic_bytes": ab_all[n]} for n in bt}
+            torch.cuda.synchronize(device)
+            if int(L.status.item()) != 0:
+                raise RuntimeError(f"device status {int(L.status.item())} after the backward ops")
 
-    variants = None
-    if not args.no_backward:
-        # every dispatch payload type on this shape, each alone (cold, clean L2)
-        from combine_moe_topk_gate_b200.workloads import DTYPES, Workload
-        bufs = {}
-        for dname, code in DTYPES.items():
-            rx = torch.empty((w.S, w.H), dtype=torch.bfloat16 if code == 0 else torch.uint8, device=device)
-            shape, sdt = api.scale_shape(w.S, w.H, code)
-            bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
+        variants = None
+        if not args.no_backward:
+            # every dispatch payload type on this shape, each alone (cold, clean L2)
+            from combine_moe_topk_gate_b200.workloads import DTYPES, Workload
+            bufs = {}
+            for dname, code in DTYPES.items():
+                rx = torch.empty((w.S, w.H), dtype=torch.bfloat16 if code == 0 else torch.uint8, device=device)
+                shape, sdt = api.scale_shape(w.S, w.H, code)
+                bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
 
-        nv = None
-        if w.H % 64 == 0:
-            nv = (torch.empty((w.S, w.H // 2), dtype=torch.uint8, device=device),
-                  torch.empty((w.S, w.H // 16), dtype=torch.uint8, device=device),
-                  torch.empty((w.S,), dtype=torch.float32, device=device))
+            nv = None
+            if w.H % 64 == 0:
+                nv = (torch.empty((w.S, w.H // 2), dtype=torch.uint8, device=device),
+                      torch.empty((w.S, w.H // 16), dtype=torch.uint8, device=device),
+                      torch.empty((w.S,), dtype=torch.float32, device=device))
 
-        e5 = torch.empty((w.S, w.H // 2 * 3), dtype=torch.uint8, device=device) if w.H % 32 == 0 else None
+            e5 = torch.empty((w.S, w.H // 2 * 3), dtype=torch.uint8, device=device) if w.H % 32 == 0 else None
 
-        def var_ops():
-            ops = {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
-                                                                 d_status=L.status))
-                   for d, (c, rx, rs) in bufs.items()}
-            if nv is not None:
-                ops["nvfp4"] = lambda: api.moe_dispatch_nvfp4(x, L.token_slot, recv_x=nv[0], block_scale=nv[1],
-                                                              row_scale=nv[2], d_status=L.status)
-            if e5 is not None:
-                ops["e5m6"] = lambda: api.moe_dispatch(x, L.token_slot, api.MOE_DTYPE_E5M6, recv_x=e5,
-                                                       d_status=L.status)
-            return ops
-        vt = isolated_op_times(var_ops, flush, device)
-        peak_v, _ = measured_peak()
-        variants = {}
-        for d, us in vt.items():
-            abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": d}))["dispatch"]
-            variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
-                           "algorithmic_bytes": abv}
-        del bufs, nv, e5
+            def var_ops():
+                ops = {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
+                                                                     d_status=L.status))
+                       for d, (c, rx, rs) in bufs.items()}
+                if nv is not None:
+                    ops["nvfp4"] = lambda: api.moe_dispatch_nvfp4(x, L.token_slot, recv_x=nv[0], block_scale=nv[1],
+                                                                  row_scale=nv[2], d_status=L.status)
+                if e5 is not None:
+                    ops["e5m6"] = lambda: api.moe_dispatch(x, L.token_slot, api.MOE_DTYPE_E5M6, recv_x=e5,
+                                                           d_status=L.status)
+                return ops
+            vt = isolated_op_times(var_ops, flush, device)
+            peak_v, _ = measured_peak()
+            variants = {}
+            for d, us in vt.items():
+                abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": d}))["dispatch"]
+                variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
+                               "algorithmic_bytes": abv}
+            del bufs, nv, e5
 
-    aligned = None
-    if not args.no_backward:
-        # the GEMM-aligned layout (every expert's rows start at a multiple of
-        # 128, one M tile) and the ops on its padded buffer, each alone
-        from combine_moe_topk_gate_b200.workloads import Workload
-        A = 128
-        rows_a = api.moe_aligned_recv_rows(w.N, w.k, w.E, A)
-        La = api.Layout.empty(w.N, w.k, w.E, w.R, device, align=A)
-        api.moe_get_layout(idx, w.E, w.R, align=A, out=La)
-        rx_a = torch.empty((rows_a, w.H), dtype=recv.dtype, device=device)
-        shape_a, sdt_a = api.scale_shape(rows_a, w.H, w.dtype_code)
-        rs_a = torch.empty(shape_a, dtype=sdt_a, device=device) if shape_a else None
-        y_a = torch.empty((rows_a, w.H), dtype=torch.bfloat16, device=device).normal_()
-        out_a = torch.empty_like(out)
+        aligned = None
+        if not args.no_backward:
+            # the GEMM-aligned layout (every expert's rows start at a multiple of
+            # 128, one M tile) and the ops on its padded buffer, each alone
+            from combine_moe_topk_gate_b200.workloads import Workload
+            A = 128
+            rows_a = api.moe_aligned_recv_rows(w.N, w.k, w.E, A)
+            La = api.Layout.empty(w.N, w.k, w.E, w.R, device, align=A)
+            api.moe_get_layout(idx, w.E, w.R, align=A, out=La)
+            rx_a = torch.empty((rows_a, w.H), dtype=recv.dtype, device=device)
+            shape_a, sdt_a = api.scale_shape(rows_a, w.H, w.dtype_code)
+            rs_a = torch.empty(shape_a, dtype=sdt_a, device=device) if shape_a else None
+            y_a = torch.empty((rows_a, w.H), dtype=torch.bfloat16, device=device).normal_()
+            out_a = torch.empty_like(out)
 
-        # the same rows with the scales laid out for the grouped GEMM: MN-major
-        # (per-block FP8) and the block-scaled MMA's tiled E8M0 atoms (MXFP8)
-        gemm_scales = {}
-        if w.H % 128 == 0:
-            rx8 = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
-            for nm, dt, lay in (("dispatch_fp8_mn_major", api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR),
-                                ("dispatch_mxfp8_mma_tiled", api.MOE_DTYPE_MXFP8_E4M3, api.MOE_SCALE_MMA_TILED)):
-                shp, sdt = api.scale_shape(rows_a, w.H, dt, lay)
-                gemm_scales[nm] = (dt, lay, torch.empty(shp, dtype=sdt, device=device))
+            # the same rows with the scales laid out for the grouped GEMM: MN-major
+            # (per-block FP8) and the block-scaled MMA's tiled E8M0 atoms (MXFP8)
+            gemm_scales = {}
+            if w.H % 128 == 0:
+                rx8 = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
+                for nm, dt, lay in (("dispatch_fp8_mn_major", api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR),
+                                    ("dispatch_mxfp8_mma_tiled", api.MOE_DTYPE_MXFP8_E4M3, api.MOE_SCALE_MMA_TILED)):
+                    shp, sdt = api.scale_shape(rows_a, w.H, dt, lay)
+                    gemm_scales[nm] = (dt, lay, torch.empty(shp, dtype=sdt, device=device))
 
-        # SwiGLU + FP8 quantisation between the expert GEMMs, on the same padded
-        # rows: h = [gate | up] of the first GEMM (seeded, resident), I = the
-        # experts' intermediate width (2048 for the 7168-wide configs, 14336
-        # for Mixtral 8x7B)
-        inter = 14336 if w.name == "mixtral" else 2048
-        h_a = torch.empty((rows_a, 2 * inter), dtype=torch.bfloat16, device=device).normal_()
-        sw_out = torch.empty((rows_a, inter), dtype=torch.uint8, device=device)
-        shp, sdt = api.scale_shape(rows_a, inter, api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR)
-        sw_sc = torch.empty(shp, dtype=sdt, device=device)
+            # SwiGLU + FP8 quantisation between the expert GEMMs, on the same padded
+            # rows: h = [gate | up] of the first GEMM (seeded, resident), I = the
+            # experts' intermediate width (2048 for the 7168-wide configs, 14336
+            # for Mixtral 8x7B)
+            inter = 14336 if w.name == "mixtral" else 2048
+            h_a = torch.empty((rows_a, 2 * inter), dtype=torch.bfloat16, device=device).normal_()
+            sw_out = torch.empty((rows_a, inter), dtype=torch.uint8, device=device)
+            shp, sdt = api.scale_shape(rows_a, inter, api.MOE_DTYPE_FP8_E4M3, api.MOE_SCALE_MN_MAJOR)
+            sw_sc = torch.empty(shp, dtype=sdt, device=device)
 
-        # per-(expert, channel) FP8 of a bf16 receive buffer (the weight-gradient
-        # GEMM's operand); y_a doubles as that buffer
-        ch_out = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
-        ch_sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+            # per-(expert, channel) FP8 of a bf16 receive buffer (the weight-gradient
+            # GEMM's operand); y_a doubles as that buffer
+            ch_out = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
+            ch_sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
 
-        def al_ops():
-            ops = {
-                "quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
-                    y_a, La.expert_offset, La.expert_count, out=ch_out, scale=ch_sc, d_status=La.status),
-                "swiglu_fp8_mn_major": lambda: api.moe_swiglu_quant(
-                    h_a, api.MOE_DTYPE_FP8_E4M3, slot_token=La.slot_token, scale_layout=api.MOE_SCALE_MN_MAJOR,
-                    out=sw_out, out_scale=sw_sc),
-                "layout": lambda: api.moe_get_layout(idx, w.E, w.R, align=A, out=La),
-                "dispatch": lambda: api.moe_dispatch(x, La.token_slot, w.dtype_code, recv_x=rx_a,
-                                                     recv_scale=rs_a, d_status=La.status),
-                "combine": lambda: api.moe_combine(y_a, La.token_slot, wts, out=out_a, d_status=La.status),
-            }
-            for nm, (dt, lay, buf) in gemm_scales.items():
-                ops[nm] = (lambda dt=dt, lay=lay, buf=buf: api.moe_dispatch(
-                    x, La.token_slot, dt, recv_x=rx8, recv_scale=buf, scale_layout=lay, d_status=La.status))
-            return ops
-        at = isolated_op_times(al_ops, flush, device)
-        torch.cuda.synchronize(device)
-        if int(La.status.item()) != 0:
-            raise RuntimeError(f"device status {int(La.status.item())} after the aligned ops")
-        peak_a, _ = measured_peak()
-        ab_a = algorithmic_bytes(w)
-        landed = int((La.slot_token >= 0).sum().item())
-        ab_a["quant_fp8_channel"] = landed * w.H * 3 + 4 * w.E * w.H + 8 * w.E
-        ab_a["swiglu_fp8_mn_major"] = landed * (4 * inter + inter + 4 * (inter // 128)) + 4 * rows_a
-        ab_a["dispatch_fp8_mn_major"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "fp8"}))["dispatch"]
-        ab_a["dispatch_mxfp8_mma_tiled"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "mxfp8"}))["dispatch"]
-        aligned = {"align": A, "recv_rows": rows_a,
-                   "padding_rows": int(rows_a - w.S), "swiglu_inter": inter, "landed_rows": landed,
-                   **{n: {"us": us, "frac": (ab_a[n] / (us * 1e-6) / 1e9 / peak_a)
-                          if us and n != "layout" else None}
-                      for n, us in at.items()}}
-        del rx_a, rs_a, y_a, La, gemm_scales, h_a, sw_out, sw_sc, ch_out, ch_sc
+            def al_ops():
+                ops = {
+                    "quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
+                        y_a, La.expert_offset, La.expert_count, out=ch_out, scale=ch_sc, d_status=La.status),
+                    "swiglu_fp8_mn_major": lambda: api.moe_swiglu_quant(
+                        h_a, api.MOE_DTYPE_FP8_E4M3, slot_token=La.slot_token, scale_layout=api.MOE_SCALE_MN_MAJOR,
+                        out=sw_out, out_scale=sw_sc),
+                    "layout": lambda: api.moe_get_layout(idx, w.E, w.R, align=A, out=La),
+                    "dispatch": lambda: api.moe_dispatch(x, La.token_slot, w.dtype_code, recv_x=rx_a,
+                                                         recv_scale=rs_a, d_status=La.status),
+                    "combine": lambda: api.moe_combine(y_a, La.token_slot, wts, out=out_a, d_status=La.status),
+                }
+                for nm, (dt, lay, buf) in gemm_scales.items():
+                    ops[nm] = (lambda dt=dt, lay=lay, buf=buf: api.moe_dispatch(
+                        x, La.token_slot, dt, recv_x=rx8, recv_scale=buf, scale_layout=lay, d_status=La.status))
+                return ops
+            at = isolated_op_times(al_ops, flush, device)
+            torch.cuda.synchronize(device)
+            if int(La.status.item()) != 0:
+                raise RuntimeError(f"device status {int(La.status.item())} after the aligned ops")
+            peak_a, _ = measured_peak()
+            ab_a = algorithmic_bytes(w)
+            landed = int((La.slot_token >= 0).sum().item())
+            ab_a["quant_fp8_channel"] = landed * w.H * 3 + 4 * w.E * w.H + 8 * w.E
+            ab_a["swiglu_fp8_mn_major"] = landed * (4 * inter + inter + 4 * (inter // 128)) + 4 * rows_a
+            ab_a["dispatch_fp8_mn_major"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "fp8"}))["dispatch"]
+            ab_a["dispatch_mxfp8_mma_tiled"] = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "mxfp8"}))["dispatch"]
+            aligned = {"align": A, "recv_rows": rows_a,
+                       "padding_rows": int(rows_a - w.S), "swiglu_inter": inter, "landed_rows": landed,
+                       **{n: {"us": us, "frac": (ab_a[n] / (us * 1e-6) / 1e9 / peak_a)
+                              if us and n != "layout" else None}
+                          for n, us in at.items()}}
+            del rx_a, rs_a, y_a, La, gemm_scales, h_a, sw_out, sw_sc, ch_out, ch_sc
 
     e2e = None
     if not args.no_e2e:
-        e2e = measure_e2e(args, w, inp, device, stream, step, logits, x, y_in, out, flush, world)
+        e2e = measure_e2e(args, w, inp, device, stream, r.step, r.logits, r.x, r.y_in, r.out, flush, world)
 
     if rank != 0:
         return
     ab = algorithmic_bytes(w)
-    peak, peak_kind = measured_peak()
-    avg = {n: sum(v) / len(v) for n, v in per_op.items()}
-    gbs = {n: ab[n] / (avg[n] * 1e-3) / 1e9 for n in avg}
-    dominant = max(("dispatch", "combine"), key=lambda n: avg[n])
+    med = {n: statistics.median(v) for n, v in per_op.items()}
+    gbs = {n: ab[n] / (med[n] * 1e-3) / 1e9 for n in med}
+    dominant = max(("dispatch", "combine"), key=lambda n: med[n])
     other = "dispatch" if dominant == "combine" else "combine"
 
     def roof(n):
@@ -558,7 +657,7 @@ def run_ours(args, rank, world, device):
         return {"kernel": n, "bound": "hbm", "achieved": gbs[n], "peak": peak, "unit": "GB/s",
                 "frac": gbs[n] / peak, "peak_source": f"{peak_kind} hbm_gbs",
                 "traffic": ncu_traffic(n, w.name), "algorithmic_bytes": ab[n],
-                "avg_launch_us": 1e3 * avg[n],
+                "median_launch_us": 1e3 * med[n],
                 "isolated_us": iso,
                 "isolated_frac": (ab[n] / (iso * 1e-6) / 1e9 / peak) if iso else None}
 
@@ -568,21 +667,16 @@ def run_ours(args, rank, world, device):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": max_total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": describe(w), "tokens_per_gpu": w.N, "hidden": w.H, "experts": w.E,
-                   "topk": w.k, "logical_ranks": w.R, "payload": f"x bf16, dispatch {w.dtype}, out bf16",
-                   "l2": "flushed before every step, outside the events: a write of 2x the L2 size, "
-                         "then a read of another 2x L2 buffer (the step starts cold and clean)",
-                   "timing": "step captured once as a CUDA graph and replayed; step time from events "
-                             "at the graph's ends, per-op times from a second graph with event nodes "
-                             "between the ops",
-                   "parallelism": f"replicas x{world} (tokens sharded, no collective)"},
-        "per_op_us": {n: 1e3 * v for n, v in avg.items()},
+        "config": config_of(w, world),
+        "step_us_median": statistics.median(step_ms) * 1e3,
+        "per_op_us": {n: 1e3 * v for n, v in med.items()},
         "per_op_gbs": gbs,
-        "dispatch_combine_tokens_per_s": w.N * world / ((avg["dispatch"] + avg["combine"]) * 1e-3),
+        "dispatch_combine_tokens_per_s": w.N * world / ((med["dispatch"] + med["combine"]) * 1e-3),
         "roofline": roof(dominant),
         "roofline_other": roof(other),
-        "gpu_launches": 2 * launches_per_step(w) * args.steps,  # two timed loops
+        "gpu_launches": 2 * launches_per_step(w) * args.steps,  # the two timed loops of the main workload
         "isolated_us": isolated,
+        "workloads": workloads,
         "backward": backward,
         "dispatch_variants": variants,
         "aligned_layout": aligned,

@@ -172,11 +172,13 @@ __device__ void aligned_offsets(int32_t* off, int32_t* cnt, int nb, int align,
 // (align > 1 only) and every row after the masked tail.  CTA `cta` of `ncta`
 // takes its share; inside it one warp per expert, lanes over the rows.
 __device__ void fill_unused_rows(const int32_t* off, const int32_t* cnt, int E, int align,
-                                 long long num_rows, int32_t* slot_token, int cta, int ncta) {
+                                 long long num_rows, int32_t* slot_token, int cta, int ncta,
+                                 int32_t* d_status) {
   if (align > 1) {
     const int nw = blockDim.x >> 5, lane = threadIdx.x & 31;
     for (int e = cta * nw + (threadIdx.x >> 5); e < E; e += ncta * nw)
-      for (int i = off[e] + cnt[e] + lane; i < off[e + 1]; i += 32) slot_token[i] = -1;
+      for (int i = off[e] + cnt[e] + lane; i < off[e + 1]; i += 32)
+        if (derived_row_ok(i, num_rows, d_status)) slot_token[i] = -1;
   }
   const long long tail0 = static_cast<long long>(off[E]) + cnt[E];
   for (long long i = tail0 + static_cast<long long>(cta) * blockDim.x + threadIdx.x; i < num_rows;
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (c == 0)
     for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
   for (int i = tid; i < nb; i += kLayoutThreads) base[i] += off[i];
-  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, c, C);
+  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, c, C, d_status);
   if (c == 0) {
     const int epr = E / R;
     for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
@@ -357,7 +359,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   __syncthreads();
   aligned_offsets(off, cnt, nb, align, warp_sums);
   for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
-  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, 0, 1);
+  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, 0, 1, d_status);
   for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
   for (int r = tid; r < R; r += kLayoutThreads) {
     rank_offset[r] = off[r * epr];
@@ -367,7 +369,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (tid == 0) rank_offset[R] = off[E];
   if (tid < ne) {
     const int slot = off[b] + wcnt[warp * nb + b] + in_warp;
-    if (b < E) {
+    if (!derived_row_ok(slot, num_rows, d_status)) {
+      token_slot[tid] = -1;
+    } else if (b < E) {
       token_slot[tid] = slot;
       slot_token[slot] = my_tok;
     } else {

@@ -9,6 +9,9 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "moe.h"
 
@@ -222,6 +225,26 @@ __device__ __forceinline__ void report_timeout(int32_t* d_status) {
   if (d_status) *reinterpret_cast<volatile int32_t*>(d_status) = MOE_ERR_TIMEOUT;
 }
 
+// Bounds-checked build (compiled with -DMOE_BOUNDS_CHECK): a receive-row
+// index a kernel derives itself -- from the layout's own counts and offsets,
+// not read from a caller's array (those are always checked) -- is also tested
+// against the buffer's rows before it is written; one outside [0, rows) is
+// skipped and reported as MOE_ERR_BAD_INDEX.  In the default build the test
+// compiles to nothing: the indices follow from counts of the same entries.
+__device__ __forceinline__ bool derived_row_ok(long long row, long long rows, int32_t* d_status) {
+#ifdef MOE_BOUNDS_CHECK
+  if (row < 0 || row >= rows) {
+    report_bad_index(d_status);
+    return false;
+  }
+#else
+  (void)row;
+  (void)rows;
+  (void)d_status;
+#endif
+  return true;
+}
+
 // ---------------------------------------------------------------- mbarrier + bulk copy
 // 1-D bulk copies (cp.async.bulk, no tensor map, no multicast) complete on an
 // mbarrier in the issuing CTA's shared memory.  Every wait is bounded.
@@ -301,10 +324,34 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+// Launch trace: with MOE_DEBUG set in the environment (to anything but "" or
+// "0"), every launch through launch_pdl / launch_pdl_cluster prints the
+// kernel's name and launch configuration on stderr.  The variable is read once
+// per process.
+inline bool debug_launches() {
+  static const bool on = [] {
+    const char* v = getenv("MOE_DEBUG");
+    return v != nullptr && v[0] != '\0' && strcmp(v, "0") != 0;
+  }();
+  return on;
+}
+
+inline void trace_launch(const void* kernel, dim3 grid, dim3 block, size_t smem, unsigned cluster_x) {
+  if (!debug_launches()) return;
+  const char* name = nullptr;
+  if (cudaFuncGetName(&name, kernel) != cudaSuccess || name == nullptr) {
+    (void)cudaGetLastError();
+    name = "(unknown kernel)";
+  }
+  fprintf(stderr, "[moe] launch %s grid=(%u,%u,%u) block=(%u,%u,%u) smem=%zu cluster=%u pdl=1\n", name,
+          grid.x, grid.y, grid.z, block.x, block.y, block.z, smem, cluster_x);
+}
+
 // Launch with the programmatic stream-serialisation attribute (see pdl_wait).
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                               cudaStream_t stream, Args... args) {
+  trace_launch(reinterpret_cast<const void*>(kernel), grid, block, smem, 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -324,6 +371,7 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 template <typename... KArgs, typename... Args>
 inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                                       cudaStream_t stream, unsigned cluster_x, Args... args) {
+  trace_launch(reinterpret_cast<const void*>(kernel), grid, block, smem, cluster_x);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
