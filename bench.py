@@ -129,9 +129,11 @@ def ncu_traffic(op: str, workload: str):
 
 
 def launches_per_step(w) -> int:
-    """Kernels one step launches: gate, layout (one CTA-sized kernel when all
-    N*k entries fit one 1024-entry chunk, else count + assign), dispatch, combine."""
-    return 1 + (1 if w.N * w.k <= 1024 else 2) + 1 + 1
+    """Kernels one step launches: routing (one launch when all N*k entries fit
+    one 1024-entry chunk and E = 32, 64, 128 or 256, else the counting gate +
+    the assignment), dispatch, combine."""
+    lanes_gate = w.E % 32 == 0 and (w.E // 32) in (1, 2, 4, 8)
+    return (1 if w.N * w.k <= 1024 and lanes_gate else 2) + 1 + 1
 
 
 def isolated_op_times(step_ops, flush, device, reps=30):
@@ -320,7 +322,7 @@ def run_reference(args, rank, world):
 
 
 # ---------------------------------------------------------------- our arm
-OPS = ("gate", "layout", "dispatch", "combine")
+OPS = ("route", "dispatch", "combine")
 
 
 class L2Flush:
@@ -349,7 +351,11 @@ class StepRunner:
         self.y_in = inp.y.to(device) if inp.y is not None else None
         self.idx = torch.empty((w.N, w.k), dtype=torch.int32, device=device)
         self.wts = torch.empty((w.N, w.k), dtype=torch.float32, device=device)
-        self.L = api.Layout.empty(w.N, w.k, w.E, w.R, device)
+        self.L = api.Layout.empty(w.N, w.k, w.E, w.R, device, route=True)
+        # the same two steps as separate calls (timed alone, for the breakdown)
+        self.idx2 = torch.empty_like(self.idx)
+        self.wts2 = torch.empty_like(self.wts)
+        self.L2 = api.Layout.empty(w.N, w.k, w.E, w.R, device)
         if w.dtype != "bf16":
             self.recv = torch.empty((w.S, w.H), dtype=torch.uint8, device=device)
             shape, sdt = api.scale_shape(w.S, w.H, w.dtype_code)
@@ -361,15 +367,25 @@ class StepRunner:
         self.y = self.recv if w.expert_out == "identity" else self.y_in
 
     def ops(self, stream=None):
+        """The step: gate and layout in one call (moe_route), dispatch, combine."""
         api, w, L = self.api, self.w, self.L
         return {
-            "gate": lambda: api.moe_topk_gate(self.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
-                                              w.group_topn, topk_idx=self.idx, topk_w=self.wts, stream=stream),
-            "layout": lambda: api.moe_get_layout(self.idx, w.E, w.R, out=L, stream=stream),
+            "route": lambda: api.moe_route(self.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
+                                           w.group_topn, w.R, topk_idx=self.idx, topk_w=self.wts, out=L,
+                                           stream=stream),
             "dispatch": lambda: api.moe_dispatch(self.x, L.token_slot, w.dtype_code, recv_x=self.recv,
                                                  recv_scale=self.scale, d_status=L.status, stream=stream),
             "combine": lambda: api.moe_combine(self.y, L.token_slot, self.wts, out=self.out,
                                                d_status=L.status, stream=stream),
+        }
+
+    def separate_ops(self, stream=None):
+        """Gate and layout as the two separate calls."""
+        api, w = self.api, self.w
+        return {
+            "gate": lambda: api.moe_topk_gate(self.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
+                                              w.group_topn, topk_idx=self.idx2, topk_w=self.wts2, stream=stream),
+            "layout": lambda: api.moe_get_layout(self.idx2, w.E, w.R, out=self.L2, stream=stream),
         }
 
     def step(self, ev=None):
@@ -440,6 +456,7 @@ def summary_of(w, step_ms, per_op, isolated, peak, world=1) -> dict:
     move a few MB and are bound by launch and memory latency, not bandwidth:
     their fractions are reported but do not describe the kernels' bound."""
     ab = algorithmic_bytes(w)
+    ab["route"] = ab["gate"] + ab["layout"]
     med = {n: statistics.median(v) * 1e3 for n, v in per_op.items()}
     st = statistics.median(step_ms) * 1e3
     latency_bound = ab["combine"] < 64e6
@@ -454,6 +471,8 @@ def summary_of(w, step_ms, per_op, isolated, peak, world=1) -> dict:
                         "min": round(min(step_ms) * 1e3, 2), "max": round(max(step_ms) * 1e3, 2)},
             "tokens_per_s": w.N * world / (st * 1e-6),
             "per_op_us": {n: round(v, 2) for n, v in med.items()},
+            "per_op_us_mean": {n: round(statistics.mean(v) * 1e3, 2) for n, v in per_op.items()},
+            "isolated_us": isolated,
             "dispatch_combine_tokens_per_s": w.N * world / ((med["dispatch"] + med["combine"]) * 1e-6),
             **ops, "bound": "latency" if latency_bound else "hbm"}
 
@@ -469,6 +488,7 @@ def other_workloads(api, main, device, steps, warmup, flush, peak) -> dict:
         r.capture(flush, warmup)
         step_ms, per_op = r.timed(steps, flush)
         iso = isolated_op_times(r.ops, flush, device)
+        iso.update(isolated_op_times(r.separate_ops, flush, device))
         res[name] = summary_of(w, step_ms, per_op, iso, peak)
         del r
         torch.cuda.empty_cache()
@@ -493,7 +513,9 @@ def run_ours(args, rank, world, device):
         max_total_ms = max_over_ranks(sum(step_ms), world, device)
 
         isolated = isolated_op_times(r.ops, flush, device)
-        L, idx, wts, x, y_in, out = r.L, r.idx, r.wts, r.x, r.y_in, r.out
+        isolated.update(isolated_op_times(r.separate_ops, flush, device))
+        L, idx, wts, x, y_in, out = r.L2, r.idx, r.wts, r.x, r.y_in, r.out
+        api.moe_get_layout(idx, w.E, w.R, out=L)   # the separate-call handle, for the sections below
         recv = r.recv
         peak, peak_kind = measured_peak()
         workloads = None
@@ -647,6 +669,7 @@ def run_ours(args, rank, world, device):
     if rank != 0:
         return
     ab = algorithmic_bytes(w)
+    ab["route"] = ab["gate"] + ab["layout"]
     med = {n: statistics.median(v) for n, v in per_op.items()}
     gbs = {n: ab[n] / (med[n] * 1e-3) / 1e9 for n in med}
     dominant = max(("dispatch", "combine"), key=lambda n: med[n])

@@ -59,6 +59,10 @@ def _load() -> ctypes.CDLL:
     L.moe_aligned_recv_rows.restype = SZ
     L.moe_get_layout_noalloc.argtypes = [P, I, I, I, I, P, P, P, P, P, P, P, P, P]
     L.moe_get_layout_noalloc.restype = I
+    L.moe_route_workspace_bytes.argtypes = [I, I, I, I]
+    L.moe_route_workspace_bytes.restype = SZ
+    L.moe_route.argtypes = [P, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, SZ, P, P]
+    L.moe_route.restype = I
     L.moe_recv_bytes.argtypes = [I, I, I, I]
     L.moe_recv_bytes.restype = SZ
     L.moe_scale_bytes.argtypes = [I, I, I, I]
@@ -213,11 +217,17 @@ class Layout:
 
     @staticmethod
     def empty(N: int, k: int, E: int, R: int, device, align: int = 1, num_rows: int | None = None,
-              workspace: bool = True) -> "Layout":
+              workspace: bool = True, route: bool = False) -> "Layout":
         """Uninitialised arrays for an N x k batch over E experts and R ranks;
         ``workspace=False`` gives a 0-byte workspace (for the no-workspace
-        entry point)."""
+        entry point); ``route=True`` a zeroed workspace of moe_route's size
+        (moe_route keeps it zero; do not pass it to moe_get_layout)."""
         i32 = dict(dtype=torch.int32, device=device)
+        if route:
+            ws = moe_route_workspace_bytes(N, k, E, R)
+            layout = Layout.empty(N, k, E, R, device, align, num_rows, workspace=False)
+            layout.workspace = torch.zeros(ws, dtype=torch.uint8, device=device)
+            return layout
         ws = moe_layout_workspace_bytes(N, k, E, R) if workspace else 0
         rows = num_rows if num_rows is not None else moe_aligned_recv_rows(N, k, E, align)
         return Layout(torch.empty(E, **i32), torch.empty(E + 1, **i32), torch.empty(R, **i32),
@@ -236,6 +246,10 @@ def _check_layout(out: Layout, N: int, k: int, E: int, R: int, workspace: bool =
     if workspace:
         _need(out.workspace, "out.workspace", torch.uint8, (out.workspace.numel(),))
     _status(out.status)
+
+
+def moe_route_workspace_bytes(num_tokens: int, k: int, num_experts: int, num_ranks: int) -> int:
+    return int(_lib.moe_route_workspace_bytes(num_tokens, k, num_experts, num_ranks))
 
 
 def moe_layout_workspace_bytes(num_tokens: int, k: int, num_experts: int, num_ranks: int) -> int:
@@ -272,6 +286,41 @@ def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, 
                 align, out.num_rows, *args)
     out.align = align
     return out
+
+
+def moe_route(logits: torch.Tensor, k: int, kind: int, n_groups: int, topk_groups: int, group_topn: int,
+              num_ranks: int, *, align: int = 1, num_recv_rows: int | None = None, topk_idx=None, topk_w=None,
+              out: Layout | None = None, stream=None):
+    """Gate and layout in one call (moe_route): returns ``(topk_idx, topk_w,
+    layout)`` equal to ``moe_topk_gate`` followed by ``moe_get_layout``.
+    ``out.workspace`` must be a zeroed moe_route workspace
+    (``Layout.empty(..., route=True)``), which every call leaves zero."""
+    _need(logits, "logits", torch.float32)
+    N, E = logits.shape
+    R = num_ranks
+    if topk_idx is None:
+        topk_idx = torch.empty((N, k), dtype=torch.int32, device=logits.device)
+    if topk_w is None:
+        topk_w = torch.empty((N, k), dtype=torch.float32, device=logits.device)
+    _need(topk_idx, "topk_idx", torch.int32, (N, k))
+    _need(topk_w, "topk_w", torch.float32, (N, k))
+    if out is None:
+        out = Layout.empty(N, k, E, R, logits.device, align, num_recv_rows, route=True)
+    _check_layout(out, N, k, E, R)
+    need = moe_route_workspace_bytes(N, k, E, R)
+    if out.workspace.numel() < need:
+        raise ValueError(f"out.workspace must hold moe_route_workspace_bytes = {need} bytes "
+                         f"(Layout.empty(..., route=True)), got {out.workspace.numel()}")
+    rows = out.num_rows
+    tensors = (logits, topk_idx, topk_w, out.expert_count, out.expert_offset, out.rank_count, out.rank_offset,
+               out.rank_tokens, out.token_slot, out.slot_token, out.workspace, _status(out.status))
+    _launch(_lib.moe_route, "moe_route", tensors, _ptr(logits), N, E, k, kind, n_groups, topk_groups, group_topn,
+            R, align, rows, _ptr(topk_idx), _ptr(topk_w), _ptr(out.expert_count), _ptr(out.expert_offset),
+            _ptr(out.rank_count), _ptr(out.rank_offset), _ptr(out.rank_tokens), _ptr(out.token_slot),
+            _ptr(out.slot_token), _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
+            _stream(stream, logits.device))
+    out.align = align
+    return topk_idx, topk_w, out
 
 
 MOE_LAYOUT_NOALLOC_SCRATCH_BYTES = 1 << 20

@@ -22,7 +22,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 4; }
+int moe_abi_version(void) { return 5; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -113,6 +113,53 @@ moe_status_t moe_get_layout(const int32_t* topk_idx, int num_tokens, int k, int 
                                 static_cast<int>(rows), expert_count, expert_offset, rank_count,
                                 rank_offset, rank_tokens, token_slot, slot_token, workspace,
                                 workspace_bytes, d_status, stream);
+}
+
+size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num_ranks) {
+  if (num_tokens < 0 || k < 1 || num_experts < 1 || num_ranks < 1) return 0;
+  return moe::route_workspace_bytes(num_tokens, k, num_experts, num_ranks);
+}
+
+moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int k,
+                       moe_gate_kind_t kind, int n_groups, int topk_groups, int group_topn,
+                       int num_ranks, int align, int num_recv_rows, int32_t* topk_idx,
+                       float* topk_w, int32_t* expert_count, int32_t* expert_offset,
+                       int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
+                       int32_t* token_slot, int32_t* slot_token, void* workspace,
+                       size_t workspace_bytes, int32_t* d_status, moe_stream_t stream) {
+  const int N = num_tokens, E = num_experts, R = num_ranks;
+  // the gate's checks
+  if (N < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (E > MOE_MAX_EXPERTS || k > MOE_MAX_TOPK) return MOE_ERR_UNSUPPORTED;
+  if (kind == MOE_GATE_SIGMOID_GROUP) {
+    if (n_groups < 1 || E % n_groups != 0) return MOE_ERR_INVALID_ARG;
+    const int eg = E / n_groups;
+    if (topk_groups < 1 || topk_groups > n_groups) return MOE_ERR_INVALID_ARG;
+    if (group_topn < 1 || group_topn > eg) return MOE_ERR_INVALID_ARG;
+    if (static_cast<long long>(topk_groups) * eg < k) return MOE_ERR_INVALID_ARG;
+  } else if (kind != MOE_GATE_SOFTMAX && kind != MOE_GATE_SOFTMAX_RENORM) {
+    return MOE_ERR_INVALID_ARG;
+  }
+  // the layout's checks
+  if (R < 1 || E % R != 0) return MOE_ERR_INVALID_ARG;
+  if (align < 1 || align > MOE_MAX_ALIGN) return MOE_ERR_INVALID_ARG;
+  const long long need = static_cast<long long>(N) * k + static_cast<long long>(E) * (align - 1);
+  if (need > kMaxRows) return MOE_ERR_UNSUPPORTED;
+  if (num_recv_rows < need) return MOE_ERR_INVALID_ARG;
+  if (!expert_count || !expert_offset || !rank_count || !rank_offset || !rank_tokens || !workspace)
+    return MOE_ERR_INVALID_ARG;
+  if (N > 0 && (!logits || !topk_idx || !topk_w || !token_slot)) return MOE_ERR_INVALID_ARG;
+  if (num_recv_rows > 0 && !slot_token) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < moe::route_workspace_bytes(N, k, E, R)) return MOE_ERR_INVALID_ARG;
+  const void* ptrs[] = {logits, topk_idx, topk_w, expert_count, expert_offset, rank_count,
+                        rank_offset, rank_tokens, token_slot, slot_token, d_status};
+  for (const void* p : ptrs)
+    if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return MOE_ERR_INVALID_ARG;
+  const moe::RouteOut out{expert_count, expert_offset, rank_count, rank_offset, rank_tokens,
+                          token_slot,   slot_token,    align,      num_recv_rows, d_status};
+  return from_cuda(moe::launch_route(logits, N, E, k, kind, n_groups, topk_groups, group_topn, R,
+                                     topk_idx, topk_w, out, workspace, as_stream(stream)));
 }
 
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype) {

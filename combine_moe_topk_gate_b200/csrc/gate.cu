@@ -25,6 +25,7 @@
 //    merges give every lane its group's top-n, summed largest first.
 //  * generic kernel (any E <= 1024): lane l holds experts l, l+32, ...; group
 //    scores come from a per-warp shared-memory scan.
+#include "layout_impl.cuh"
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
@@ -139,131 +140,206 @@ __device__ __forceinline__ void select_sorted(uint64_t (&key)[V], int k, int lan
   }
 }
 
+// Per-chunk counting for the fused routing path (moe_route): the layout's
+// chunk histograms (entries per bucket, bucket E = masked) and per-chunk
+// tokens per rank, accumulated with atomics into zeroed workspace while the
+// gate's registers still hold each token's choices.  counts == NULL: off.
+struct ChunkCount {
+  int32_t* counts;  // [C][E + 1]
+  int32_t* rtok;    // [C][R]
+  int E, R, epr;    // experts, ranks, experts per rank
+  int tpc;          // tokens per chunk
+};
+
+// Lane j < k holds the token's slot j (expert sel_i, or -1).  The token is
+// counted once per rank, at its first slot on that rank.
+__device__ __forceinline__ void count_token(const ChunkCount& cc, int t, int k, int lane, int sel_i) {
+  const bool valid = static_cast<unsigned>(sel_i) < static_cast<unsigned>(cc.E);
+  const int r = valid ? sel_i / cc.epr : -1;
+  bool first = valid;
+  for (int jj = 0; jj < k; ++jj) {  // k is warp-uniform: every lane shuffles
+    const int rj = __shfl_sync(kFullMask, r, jj);
+    first = first && !(jj < lane && rj == r);
+  }
+  if (lane < k) {
+    const size_t c = static_cast<size_t>(t / cc.tpc);
+    atomicAdd(&cc.counts[c * (cc.E + 1) + (valid ? sel_i : cc.E)], 1);
+    if (first) atomicAdd(&cc.rtok[c * cc.R + r], 1);
+  }
+}
+
 // ------------------------------------------------------------------ lanes kernel
+template <int V, int TOPN>
+__device__ __forceinline__ void gate_lanes_token(const float* __restrict__ logits, int t, int k,
+                                                 int kind, int LPG_log2, int TG, float* sh_exp,
+                                                 int lane, int32_t* __restrict__ topk_idx,
+                                                 float* __restrict__ topk_w, const ChunkCount& cc) {
+  constexpr int E = 32 * V;
+  constexpr int topn = TOPN;  // group score = sum of the TOPN best scores of a group
+  const int e0 = lane * V;
+  const float* row = logits + static_cast<size_t>(t) * E + e0;
+  float l[V];
+  if constexpr (V % 4 == 0) {
+#pragma unroll
+    for (int q = 0; q < V / 4; ++q) {
+      const float4 f = reinterpret_cast<const float4*>(row)[q];
+      l[4 * q] = f.x;
+      l[4 * q + 1] = f.y;
+      l[4 * q + 2] = f.z;
+      l[4 * q + 3] = f.w;
+    }
+  } else if constexpr (V == 2) {
+    const float2 f = *reinterpret_cast<const float2*>(row);
+    l[0] = f.x;
+    l[1] = f.y;
+  } else {
+    l[0] = row[0];
+  }
+  uint64_t key[V];
+  int sel_i = -1;
+  float sel_v = 0.0f, sum = 0.0f;
+
+  if (kind == MOE_GATE_SIGMOID_GROUP) {
+#pragma unroll
+    for (int v = 0; v < V; ++v) key[v] = make_key(logistic(l[v]), e0 + v);
+    sort_desc<V>(key);
+    // this lane's top-n, best first (key 0 pads when n > V)
+    uint64_t top[topn];
+#pragma unroll
+    for (int p = 0; p < topn; ++p) top[p] = p < V ? key[p < V ? p : 0] : 0;
+    // merge with the other lanes of the group: top-n of two sorted lists is
+    // max(a_i, b_{n-1-i}) (a bitonic sequence), then sorted again
+#pragma unroll
+    for (int step = 0; step < 5; ++step) {  // LPG <= 32 lanes: at most 5 merges
+      if (step >= LPG_log2) break;            // warp-uniform
+      const int m = 1 << step;
+      uint64_t other[topn], mrg[topn];
+#pragma unroll
+      for (int p = 0; p < topn; ++p) other[p] = shfl_xor_key(top[p], m);
+#pragma unroll
+      for (int p = 0; p < topn; ++p) mrg[p] = top[p] > other[topn - 1 - p] ? top[p] : other[topn - 1 - p];
+      // sort the merged keys, largest first
+#pragma unroll
+      for (int a = 0; a < topn; ++a)
+#pragma unroll
+        for (int b = topn - 1; b > a; --b)
+          if (mrg[b] > mrg[b - 1]) {
+            const uint64_t tmp = mrg[b];
+            mrg[b] = mrg[b - 1];
+            mrg[b - 1] = tmp;
+          }
+#pragma unroll
+      for (int p = 0; p < topn; ++p) top[p] = mrg[p];
+    }
+    float gscore = key_value(top[0]);
+#pragma unroll
+    for (int p = 1; p < topn; ++p) gscore = __fadd_rn(gscore, key_value(top[p]));
+    // rank of this lane's group among all groups (group h leads lanes h*LPG..)
+    const int g = lane >> LPG_log2;
+    const int G = 32 >> LPG_log2;
+    const uint64_t gkey = make_key(gscore, g);
+    int before = 0;
+    for (int h = 0; h < G; ++h) before += shfl_key(gkey, h << LPG_log2) > gkey ? 1 : 0;
+    if (before >= TG) {
+#pragma unroll
+      for (int v = 0; v < V; ++v) key[v] = 0;
+    }
+    select_sorted<V>(key, k, lane, sel_i, sel_v, sum);
+    if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
+  } else {
+    float m = l[0];
+#pragma unroll
+    for (int v = 1; v < V; ++v) m = fmaxf(m, l[v]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      sh_exp[e0 + v] = fixed_exp(__fsub_rn(l[v], m));
+      key[v] = make_key(l[v], e0 + v);
+    }
+    __syncwarp();
+    float z = 0.0f;
+    if (lane == 0)
+      for (int i = 0; i < E; ++i) z = __fadd_rn(z, sh_exp[i]);
+    z = __shfl_sync(kFullMask, z, 0);
+    sort_desc<V>(key);
+    for (int j = 0; j < k; ++j) {
+      const uint64_t win = warp_max_key(key[0]);
+      const int wi = key_index(win);
+      const float p = (wi >= 0 && wi < E) ? __fdiv_rn(sh_exp[wi], z) : 0.0f;
+      sum = (j == 0) ? p : __fadd_rn(sum, p);
+      if (lane == j) {
+        sel_i = (wi >= 0 && wi < E) ? wi : -1;
+        sel_v = p;
+      }
+      const bool pop = win != 0 && key[0] == win;
+#pragma unroll
+      for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
+      key[V - 1] = pop ? 0 : key[V - 1];
+    }
+    if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
+    __syncwarp();  // sh_exp is rewritten for the next token
+  }
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
+    topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
+  }
+  if (cc.counts != nullptr) count_token(cc, t, k, lane, sel_i);
+}
+
 // Softmax needs Z summed in ascending expert order: the exp terms go to shared
-// memory and lane 0 adds them one by one.
+// memory (one row per warp) and lane 0 adds them one by one.
 template <int V, int TOPN>
 __global__ void __launch_bounds__(kGateWarps * 32)
     topk_gate_lanes_kernel(const float* __restrict__ logits, int N, int k, int kind, int LPG_log2,
-                           int TG, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
-  constexpr int E = 32 * V;
-  constexpr int topn = TOPN;  // group score = sum of the TOPN best scores of a group
-  __shared__ float sh_exp[kGateWarps][E];
+                           int TG, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                           ChunkCount cc) {
+  __shared__ float sh_exp[kGateWarps][32 * V];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int e0 = lane * V;
   pdl_wait();
   pdl_trigger();
+  for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps)
+    gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, sh_exp[warp], lane, topk_idx, topk_w, cc);
+}
 
-  for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
-    const float* row = logits + static_cast<size_t>(t) * E + e0;
-    float l[V];
-    if constexpr (V % 4 == 0) {
-#pragma unroll
-      for (int q = 0; q < V / 4; ++q) {
-        const float4 f = reinterpret_cast<const float4*>(row)[q];
-        l[4 * q] = f.x;
-        l[4 * q + 1] = f.y;
-        l[4 * q + 2] = f.z;
-        l[4 * q + 3] = f.w;
-      }
-    } else if constexpr (V == 2) {
-      const float2 f = *reinterpret_cast<const float2*>(row);
-      l[0] = f.x;
-      l[1] = f.y;
-    } else {
-      l[0] = row[0];
-    }
-    uint64_t key[V];
-    int sel_i = -1;
-    float sel_v = 0.0f, sum = 0.0f;
-
-    if (kind == MOE_GATE_SIGMOID_GROUP) {
-#pragma unroll
-      for (int v = 0; v < V; ++v) key[v] = make_key(logistic(l[v]), e0 + v);
-      sort_desc<V>(key);
-      // this lane's top-n, best first (key 0 pads when n > V)
-      uint64_t top[topn];
-#pragma unroll
-      for (int p = 0; p < topn; ++p) top[p] = p < V ? key[p < V ? p : 0] : 0;
-      // merge with the other lanes of the group: top-n of two sorted lists is
-      // max(a_i, b_{n-1-i}) (a bitonic sequence), then sorted again
-#pragma unroll
-      for (int step = 0; step < 5; ++step) {  // LPG <= 32 lanes: at most 5 merges
-        if (step >= LPG_log2) break;            // warp-uniform
-        const int m = 1 << step;
-        uint64_t other[topn], mrg[topn];
-#pragma unroll
-        for (int p = 0; p < topn; ++p) other[p] = shfl_xor_key(top[p], m);
-#pragma unroll
-        for (int p = 0; p < topn; ++p) mrg[p] = top[p] > other[topn - 1 - p] ? top[p] : other[topn - 1 - p];
-        // sort the merged keys, largest first
-#pragma unroll
-        for (int a = 0; a < topn; ++a)
-#pragma unroll
-          for (int b = topn - 1; b > a; --b)
-            if (mrg[b] > mrg[b - 1]) {
-              const uint64_t tmp = mrg[b];
-              mrg[b] = mrg[b - 1];
-              mrg[b - 1] = tmp;
-            }
-#pragma unroll
-        for (int p = 0; p < topn; ++p) top[p] = mrg[p];
-      }
-      float gscore = key_value(top[0]);
-#pragma unroll
-      for (int p = 1; p < topn; ++p) gscore = __fadd_rn(gscore, key_value(top[p]));
-      // rank of this lane's group among all groups (group h leads lanes h*LPG..)
-      const int g = lane >> LPG_log2;
-      const int G = 32 >> LPG_log2;
-      const uint64_t gkey = make_key(gscore, g);
-      int before = 0;
-      for (int h = 0; h < G; ++h) before += shfl_key(gkey, h << LPG_log2) > gkey ? 1 : 0;
-      if (before >= TG) {
-#pragma unroll
-        for (int v = 0; v < V; ++v) key[v] = 0;
-      }
-      select_sorted<V>(key, k, lane, sel_i, sel_v, sum);
-      if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
-    } else {
-      float m = l[0];
-#pragma unroll
-      for (int v = 1; v < V; ++v) m = fmaxf(m, l[v]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        sh_exp[warp][e0 + v] = fixed_exp(__fsub_rn(l[v], m));
-        key[v] = make_key(l[v], e0 + v);
-      }
-      __syncwarp();
-      float z = 0.0f;
-      if (lane == 0)
-        for (int i = 0; i < E; ++i) z = __fadd_rn(z, sh_exp[warp][i]);
-      z = __shfl_sync(kFullMask, z, 0);
-      sort_desc<V>(key);
-      for (int j = 0; j < k; ++j) {
-        const uint64_t win = warp_max_key(key[0]);
-        const int wi = key_index(win);
-        const float p = (wi >= 0 && wi < E) ? __fdiv_rn(sh_exp[warp][wi], z) : 0.0f;
-        sum = (j == 0) ? p : __fadd_rn(sum, p);
-        if (lane == j) {
-          sel_i = (wi >= 0 && wi < E) ? wi : -1;
-          sel_v = p;
-        }
-        const bool pop = win != 0 && key[0] == win;
-#pragma unroll
-        for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
-        key[V - 1] = pop ? 0 : key[V - 1];
-      }
-      if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
-      __syncwarp();  // sh_exp is rewritten for the next token
-    }
-    if (lane < k) {
-      topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
-      topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
-    }
-  }
+// ------------------------------------------------------------------ fused routing, small batches
+// Gate and layout in one launch when every entry fits one layout chunk
+// (N*k <= kLayoutThreads): CTAs of kLayoutWarps warps, one token per warp.
+// Each CTA publishes its tokens' choices (fence, then an arrival on a counter
+// in the caller's zeroed workspace); the CTA that arrives last -- every
+// other CTA's outputs are visible to it by then -- builds the whole layout
+// with the single-CTA layout body and puts the counter back to zero.  No CTA
+// waits for another.
+template <int V, int TOPN>
+__global__ void __launch_bounds__(kLayoutThreads)
+    route_small_kernel(const float* __restrict__ logits, int N, int k, int kind, int LPG_log2, int TG,
+                       int32_t* __restrict__ topk_idx, float* __restrict__ topk_w, int R,
+                       int32_t* __restrict__ expert_count, int32_t* __restrict__ expert_offset,
+                       int32_t* __restrict__ rank_count, int32_t* __restrict__ rank_offset,
+                       int32_t* __restrict__ rank_tokens, int32_t* __restrict__ token_slot,
+                       int32_t* __restrict__ slot_token, int align, long long num_rows,
+                       int32_t* d_status, unsigned* done) {
+  extern __shared__ int32_t sm[];  // gate: one row of E floats per warp; then the layout's words
+  __shared__ int last_cta;
+  constexpr int E = 32 * V;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  const int t = blockIdx.x * kLayoutWarps + warp;
+  const ChunkCount none{nullptr, nullptr, E, 1, E, 1};
+  if (t < N)
+    gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, reinterpret_cast<float*>(sm) + warp * E,
+                              lane, topk_idx, topk_w, none);
+  __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) last_cta = atomicAdd(done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 // ------------------------------------------------------------------ generic kernel
@@ -272,7 +348,7 @@ template <int V>
 __global__ void __launch_bounds__(kGateWarps * 32)
     topk_gate_generic_kernel(const float* __restrict__ logits, int N, int E, int k, int kind,
                              int G, int TG, int topn, int32_t* __restrict__ topk_idx,
-                             float* __restrict__ topk_w) {
+                             float* __restrict__ topk_w, ChunkCount cc) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -385,6 +461,7 @@ __global__ void __launch_bounds__(kGateWarps * 32)
       topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
       topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
     }
+    if (cc.counts != nullptr) count_token(cc, t, k, lane, sel_i);
     __syncwarp();  // the next token reuses this warp's shared memory
   }
 }
@@ -397,7 +474,7 @@ unsigned grid_for(int N) {
 
 template <int V>
 cudaError_t launch_generic(const float* logits, int N, int E, int k, int kind, int G, int TG,
-                           int topn, int32_t* idx, float* w, cudaStream_t stream) {
+                           int topn, int32_t* idx, float* w, const ChunkCount& cc, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(kGateWarps) * (E + 2 * G) * sizeof(float);
   if (smem > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(topk_gate_generic_kernel<V>,
@@ -406,24 +483,24 @@ cudaError_t launch_generic(const float* logits, int N, int E, int k, int kind, i
     if (err != cudaSuccess) return err;
   }
   return launch_pdl(topk_gate_generic_kernel<V>, grid_for(N), kGateWarps * 32, smem, stream, logits,
-                    N, E, k, kind, G, TG, topn, idx, w);
+                    N, E, k, kind, G, TG, topn, idx, w, cc);
 }
 
 template <int V, int TOPN>
 cudaError_t launch_lanes_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
-                           int32_t* idx, float* w, cudaStream_t stream) {
+                           int32_t* idx, float* w, const ChunkCount& cc, cudaStream_t stream) {
   return launch_pdl(topk_gate_lanes_kernel<V, TOPN>, grid_for(N), kGateWarps * 32, 0, stream,
-                    logits, N, k, kind, lpg_log2, TG, idx, w);
+                    logits, N, k, kind, lpg_log2, TG, idx, w, cc);
 }
 
 template <int V>
 cudaError_t launch_lanes(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
-                         int topn, int32_t* idx, float* w, cudaStream_t stream) {
+                         int topn, int32_t* idx, float* w, const ChunkCount& cc, cudaStream_t stream) {
   switch (topn) {
-    case 1: return launch_lanes_n<V, 1>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
-    case 2: return launch_lanes_n<V, 2>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
-    case 3: return launch_lanes_n<V, 3>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
-    default: return launch_lanes_n<V, 4>(logits, N, k, kind, lpg_log2, TG, idx, w, stream);
+    case 1: return launch_lanes_n<V, 1>(logits, N, k, kind, lpg_log2, TG, idx, w, cc, stream);
+    case 2: return launch_lanes_n<V, 2>(logits, N, k, kind, lpg_log2, TG, idx, w, cc, stream);
+    case 3: return launch_lanes_n<V, 3>(logits, N, k, kind, lpg_log2, TG, idx, w, cc, stream);
+    default: return launch_lanes_n<V, 4>(logits, N, k, kind, lpg_log2, TG, idx, w, cc, stream);
   }
 }
 
@@ -472,39 +549,127 @@ cudaError_t launch_gate_math(uint32_t first, size_t n, float* exp_out, float* si
   return cudaGetLastError();
 }
 
+namespace {
+
+// Which gate kernel a shape takes: the lanes kernel when E = 32*V with V a
+// power of two up to 8, rows 16-byte aligned and (group kind) groups made of
+// whole lanes with topn <= 4; lpg_log2 = log2(lanes per group).
+struct GatePlan {
+  bool lanes;
+  int V, lpg_log2, G, TG, topn;
+};
+
+GatePlan plan_gate(const float* logits, int E, int kind, int n_groups, int topk_groups,
+                   int group_topn) {
+  GatePlan p{false, E / 32, 0, n_groups, topk_groups, group_topn};
+  if (kind != MOE_GATE_SIGMOID_GROUP) p.G = p.TG = p.topn = 1;
+  p.lanes = E % 32 == 0 && log2_exact(p.V) >= 0 && p.V <= 8 &&
+            (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
+  if (p.lanes && kind == MOE_GATE_SIGMOID_GROUP) {
+    const int eg = E / p.G;
+    p.lpg_log2 = (eg % p.V == 0) ? log2_exact(eg / p.V) : -1;
+    p.lanes = p.lpg_log2 >= 0 && p.topn <= kMaxTopn;
+  }
+  return p;
+}
+
+cudaError_t launch_gate(const float* logits, int N, int E, int k, int kind, const GatePlan& p,
+                        int32_t* topk_idx, float* topk_w, const ChunkCount& cc, cudaStream_t stream) {
+  if (p.lanes) {
+    switch (p.V) {
+      case 1: return launch_lanes<1>(logits, N, k, kind, p.lpg_log2, p.TG, p.topn, topk_idx, topk_w, cc, stream);
+      case 2: return launch_lanes<2>(logits, N, k, kind, p.lpg_log2, p.TG, p.topn, topk_idx, topk_w, cc, stream);
+      case 4: return launch_lanes<4>(logits, N, k, kind, p.lpg_log2, p.TG, p.topn, topk_idx, topk_w, cc, stream);
+      default: return launch_lanes<8>(logits, N, k, kind, p.lpg_log2, p.TG, p.topn, topk_idx, topk_w, cc, stream);
+    }
+  }
+  const int per_lane = (E + 31) / 32;
+  const int G = p.G, TG = p.TG, topn = p.topn;
+  if (per_lane <= 1) return launch_generic<1>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+  if (per_lane <= 2) return launch_generic<2>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+  if (per_lane <= 4) return launch_generic<4>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+  if (per_lane <= 8) return launch_generic<8>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+  if (per_lane <= 16) return launch_generic<16>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+  return launch_generic<32>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
+}
+
+template <int V, int TOPN>
+cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
+                                 int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
+                                 cudaStream_t stream) {
+  constexpr int E = 32 * V;
+  const size_t words = layout_single_smem_words(E, R);
+  const size_t smem = (words > static_cast<size_t>(kLayoutWarps) * E ? words : static_cast<size_t>(kLayoutWarps) * E) *
+                      sizeof(int32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(route_small_kernel<V, TOPN>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  const unsigned grid = static_cast<unsigned>((N + kLayoutWarps - 1) / kLayoutWarps);
+  return launch_pdl(route_small_kernel<V, TOPN>, grid, kLayoutThreads, smem, stream, logits, N, k, kind,
+                    lpg_log2, TG, idx, w, R, o.expert_count, o.expert_offset, o.rank_count, o.rank_offset,
+                    o.rank_tokens, o.token_slot, o.slot_token, o.align, o.num_rows, o.d_status, done);
+}
+
+template <int V>
+cudaError_t launch_route_small(const float* logits, int N, int k, int kind, const GatePlan& p, int32_t* idx,
+                               float* w, int R, const RouteOut& o, unsigned* done, cudaStream_t stream) {
+  switch (p.topn) {
+    case 1: return launch_route_small_n<V, 1>(logits, N, k, kind, p.lpg_log2, p.TG, idx, w, R, o, done, stream);
+    case 2: return launch_route_small_n<V, 2>(logits, N, k, kind, p.lpg_log2, p.TG, idx, w, R, o, done, stream);
+    case 3: return launch_route_small_n<V, 3>(logits, N, k, kind, p.lpg_log2, p.TG, idx, w, R, o, done, stream);
+    default: return launch_route_small_n<V, 4>(logits, N, k, kind, p.lpg_log2, p.TG, idx, w, R, o, done, stream);
+  }
+}
+
+}  // namespace
+
+size_t route_workspace_bytes(int N, int k, int E, int R) {
+  return kRouteCounterBytes + layout_workspace_bytes(N, k, E, R);
+}
+
+cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int n_groups,
+                         int topk_groups, int group_topn, int R, int32_t* topk_idx, float* topk_w,
+                         const RouteOut& o, void* workspace, cudaStream_t stream) {
+  const GatePlan p = plan_gate(logits, E, kind, n_groups, topk_groups, group_topn);
+  unsigned* done = static_cast<unsigned*>(workspace);
+  int32_t* chunks = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kRouteCounterBytes);
+  if (N == 0 || static_cast<long long>(N) * k <= kLayoutThreads) {
+    if (N > 0 && p.lanes) {
+      switch (p.V) {
+        case 1: return launch_route_small<1>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
+        case 2: return launch_route_small<2>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
+        case 4: return launch_route_small<4>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
+        default: return launch_route_small<8>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
+      }
+    }
+    // other expert counts (or no tokens): gate, then the one-CTA layout
+    cudaError_t err = launch_topk_gate(logits, N, E, k, kind, n_groups, topk_groups, group_topn, topk_idx,
+                                       topk_w, stream);
+    if (err != cudaSuccess) return err;
+    return launch_layout(topk_idx, N, k, E, R, o.align, o.num_rows, o.expert_count, o.expert_offset,
+                         o.rank_count, o.rank_offset, o.rank_tokens, o.token_slot, o.slot_token, chunks,
+                         o.d_status, stream);
+  }
+  // gate with the per-chunk counts folded in, then the assignment (which
+  // leaves the counts zeroed again)
+  const int C = (N + kLayoutThreads / k - 1) / (kLayoutThreads / k);
+  const ChunkCount cc{chunks, chunks + static_cast<size_t>(C) * (E + 1), E, R, E / R, kLayoutThreads / k};
+  cudaError_t err = launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, cc, stream);
+  if (err != cudaSuccess) return err;
+  return launch_layout_assign_zeroing(topk_idx, N, k, E, R, o.align, o.num_rows, o.expert_count,
+                                      o.expert_offset, o.rank_count, o.rank_offset, o.rank_tokens,
+                                      o.token_slot, o.slot_token, chunks, done, o.d_status, stream);
+}
+
 cudaError_t launch_topk_gate(const float* logits, int N, int E, int k, int kind, int n_groups,
                              int topk_groups, int group_topn, int32_t* topk_idx, float* topk_w,
                              cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
-  int G = n_groups, TG = topk_groups, topn = group_topn;
-  if (kind != MOE_GATE_SIGMOID_GROUP) G = TG = topn = 1;
-
-  // lanes kernel: E = 32*V with V a power of two up to 8, 16-byte aligned rows,
-  // and (group kind) groups made of whole lanes with topn <= 4
-  const int V = E / 32;
-  bool lanes = E % 32 == 0 && log2_exact(V) >= 0 && V <= 8 &&
-               (reinterpret_cast<uintptr_t>(logits) & 15) == 0;
-  int lpg_log2 = 0;
-  if (lanes && kind == MOE_GATE_SIGMOID_GROUP) {
-    const int eg = E / G;
-    lpg_log2 = (eg % V == 0) ? log2_exact(eg / V) : -1;
-    lanes = lpg_log2 >= 0 && topn <= kMaxTopn;
-  }
-  if (lanes) {
-    switch (V) {
-      case 1: return launch_lanes<1>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
-      case 2: return launch_lanes<2>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
-      case 4: return launch_lanes<4>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
-      default: return launch_lanes<8>(logits, N, k, kind, lpg_log2, TG, topn, topk_idx, topk_w, stream);
-    }
-  }
-  const int per_lane = (E + 31) / 32;
-  if (per_lane <= 1) return launch_generic<1>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 2) return launch_generic<2>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 4) return launch_generic<4>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 8) return launch_generic<8>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  if (per_lane <= 16) return launch_generic<16>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
-  return launch_generic<32>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, stream);
+  const GatePlan p = plan_gate(logits, E, kind, n_groups, topk_groups, group_topn);
+  const ChunkCount none{nullptr, nullptr, E, 1, E, 1};
+  return launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, none, stream);
 }
 
 }  // namespace moe

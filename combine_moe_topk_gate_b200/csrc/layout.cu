@@ -22,38 +22,11 @@
 //           counts and offsets.  The row of entry (t, j) in expert e is the
 //           number of entries routed to e before it in (t, j) order, so the
 //           result is deterministic.
-#include "moe_device.cuh"
+#include "layout_impl.cuh"
 #include "moe_launch.h"
 
 namespace moe {
 namespace {
-
-constexpr int kLayoutThreads = 1024;
-constexpr int kLayoutWarps = kLayoutThreads / 32;
-
-__host__ __device__ __forceinline__ int tokens_per_chunk(int k) { return kLayoutThreads / k; }
-
-__host__ __device__ __forceinline__ int num_chunks(int N, int k) {
-  const int tc = tokens_per_chunk(k);
-  const int c = (N + tc - 1) / tc;
-  return c > 0 ? c : 1;
-}
-
-// bucket of an entry: its expert, E for masked (-1) and invalid ids
-__device__ __forceinline__ int bucket_of(int e, int E) {
-  return (static_cast<unsigned>(e) < static_cast<unsigned>(E)) ? e : E;
-}
-
-// True when none of the token's slots before slot j (ids at tok[0..j)) has an
-// expert of the rank whose experts are [lo, lo + epr); ids outside [0, E)
-// never match because that range lies inside it.  The loads are independent.
-__device__ __forceinline__ bool first_on_rank(const int32_t* tok, int j, int lo, int epr) {
-  bool first = true;
-#pragma unroll 4
-  for (int jj = 0; jj < j; ++jj)
-    first = first && static_cast<unsigned>(tok[jj]) - static_cast<unsigned>(lo) >= static_cast<unsigned>(epr);
-  return first;
-}
 
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_count_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R,
@@ -102,90 +75,6 @@ __global__ void __launch_bounds__(kLayoutThreads)
   for (int i = tid; i < R; i += kLayoutThreads) chunk_rtok[static_cast<size_t>(c) * R + i] = rtok[i];
 }
 
-// Exclusive scan of a[0..n) in shared memory, n <= 2 * kLayoutThreads.
-__device__ void block_exclusive_scan(int32_t* a, int n, int32_t* warp_sums) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i0 = 2 * tid, i1 = 2 * tid + 1;
-  const int x0 = i0 < n ? a[i0] : 0;
-  const int x1 = i1 < n ? a[i1] : 0;
-  const int s = x0 + x1;
-  int incl = s;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(kFullMask, incl, off);
-    if (lane >= off) incl += y;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int v = warp_sums[lane];
-    int wi = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(kFullMask, wi, off);
-      if (lane >= off) wi += y;
-    }
-    warp_sums[lane] = wi - v;
-  }
-  __syncthreads();
-  const int excl = warp_sums[warp] + incl - s;
-  if (i0 < n) a[i0] = excl;
-  if (i1 < n) a[i1] = excl + x0;
-  __syncthreads();
-}
-
-// Exclusive prefix over the warps of every bucket of the [kLayoutWarps][nb]
-// count matrix, in place: one thread per bucket, its loads issued eight at a
-// time (independent addresses) and summed in registers.  Returns the
-// bucket's total.
-__device__ __forceinline__ int warp_prefix_of_bucket(int32_t* wcnt, int nb, int bb) {
-  int acc = 0;
-#pragma unroll
-  for (int w0 = 0; w0 < kLayoutWarps; w0 += 8) {
-    int v[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = wcnt[(w0 + i) * nb + bb];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      wcnt[(w0 + i) * nb + bb] = acc;
-      acc += v[i];
-    }
-  }
-  return acc;
-}
-
-// Turns the per-bucket totals in off[] into exclusive row offsets, each
-// expert bucket rounded up to a multiple of `align` (1 = packed); cnt[] keeps
-// the totals.
-__device__ void aligned_offsets(int32_t* off, int32_t* cnt, int nb, int align,
-                                int32_t* warp_sums) {
-  for (int i = threadIdx.x; i < nb; i += blockDim.x) {
-    const int v = off[i];
-    cnt[i] = v;
-    if (i < nb - 1 && align > 1) off[i] = (v + align - 1) / align * align;
-  }
-  __syncthreads();
-  block_exclusive_scan(off, nb, warp_sums);
-}
-
-// Rows no entry lands in get slot_token = -1: the padding after each expert
-// (align > 1 only) and every row after the masked tail.  CTA `cta` of `ncta`
-// takes its share; inside it one warp per expert, lanes over the rows.
-__device__ void fill_unused_rows(const int32_t* off, const int32_t* cnt, int E, int align,
-                                 long long num_rows, int32_t* slot_token, int cta, int ncta,
-                                 int32_t* d_status) {
-  if (align > 1) {
-    const int nw = blockDim.x >> 5, lane = threadIdx.x & 31;
-    for (int e = cta * nw + (threadIdx.x >> 5); e < E; e += ncta * nw)
-      for (int i = off[e] + cnt[e] + lane; i < off[e + 1]; i += 32)
-        if (derived_row_ok(i, num_rows, d_status)) slot_token[i] = -1;
-  }
-  const long long tail0 = static_cast<long long>(off[E]) + cnt[E];
-  for (long long i = tail0 + static_cast<long long>(cta) * blockDim.x + threadIdx.x; i < num_rows;
-       i += static_cast<long long>(ncta) * blockDim.x)
-    slot_token[i] = -1;
-}
-
 __global__ void __launch_bounds__(kLayoutThreads)
     layout_assign_kernel(const int32_t* __restrict__ topk_idx, int N, int k, int E, int R, int C,
                          const int32_t* __restrict__ chunk_counts,
@@ -193,8 +82,10 @@ __global__ void __launch_bounds__(kLayoutThreads)
                          int32_t* __restrict__ expert_offset, int32_t* __restrict__ rank_count,
                          int32_t* __restrict__ rank_offset, int32_t* __restrict__ rank_tokens,
                          int32_t* __restrict__ token_slot, int32_t* __restrict__ slot_token,
-                         int align, long long num_rows, int32_t* d_status) {
+                         int align, long long num_rows, int32_t* d_status, unsigned* done,
+                         int32_t* ws_clear, long long ws_words) {
   extern __shared__ int32_t sm[];
+  __shared__ int last_cta;
   const int nb = E + 1;
   int32_t* off = sm;                 // nb: totals, then their exclusive (aligned) scan
   int32_t* base = off + nb;          // nb: first row of this chunk per bucket
@@ -306,6 +197,19 @@ __global__ void __launch_bounds__(kLayoutThreads)
     }
   }
   (void)lane;
+  // Fused routing (done != NULL): the chunk counts were accumulated with
+  // atomics into zeroed workspace.  Every CTA has read them before it gets
+  // here, so the last CTA to arrive zeroes them (and the arrival counter)
+  // for the next call.  No CTA waits for another.
+  if (done != nullptr) {
+    __syncthreads();
+    if (tid == 0) last_cta = atomicAdd(done, 1u) == static_cast<unsigned>(C - 1);
+    __syncthreads();
+    if (last_cta) {
+      for (long long i = tid; i < ws_words; i += kLayoutThreads) ws_clear[i] = 0;
+      if (tid == 0) *done = 0u;
+    }
+  }
 }
 
 // Whole layout in one CTA when every entry fits one chunk (N*k <= 1024, the
@@ -319,66 +223,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
                          int32_t* __restrict__ slot_token, int align, long long num_rows,
                          int32_t* d_status) {
   extern __shared__ int32_t sm[];
-  const int nb = E + 1;
-  int32_t* off = sm;                              // nb: totals, then their exclusive scan
-  int32_t* wcnt = off + nb;                       // kLayoutWarps * nb
-  int32_t* warp_sums = wcnt + kLayoutWarps * nb;  // 32
-  int32_t* rtok = warp_sums + 32;                 // R
-  int32_t* sidx = rtok + R;                       // kLayoutThreads
-  int32_t* cnt = sidx + kLayoutThreads;           // nb: totals
-  int32_t* rank_of = cnt + nb;                    // E: rank of each expert
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int ne = N * k;  // <= kLayoutThreads
-  const int nbits = 32 - __clz(E + 1);
-  const int epr = E / R;
-  // data-independent setup (overlaps the predecessor's tail under PDL)
-  const int my_tok = tid / k, j = tid - my_tok * k;
-  for (int i = tid; i < kLayoutWarps * nb; i += kLayoutThreads) wcnt[i] = 0;
-  for (int i = tid; i < R; i += kLayoutThreads) rtok[i] = 0;
-  for (int i = tid; i < E; i += kLayoutThreads) rank_of[i] = i / epr;
-  pdl_wait();
-  pdl_trigger();
-  int e = -1, b = -1;
-  if (tid < ne) {
-    e = topk_idx[tid];
-    sidx[tid] = e;
-    b = bucket_of(e, E);
-    if (b == E && e != -1) report_bad_index(d_status);
-  }
-  __syncthreads();
-  const unsigned same = warp_match(static_cast<unsigned>(b + 1), nbits);
-  const int in_warp = __popc(same & lanemask_lt());
-  if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
-  if (b >= 0 && b < E) {  // the token's first slot on this rank counts the token
-    const int r = rank_of[e];
-    if (first_on_rank(sidx + tid - j, j, r * epr, epr)) atomicAdd(&rtok[r], 1);
-  }
-  __syncthreads();
-  // per bucket: exclusive prefix over the warps, total into off[]
-  for (int bb = tid; bb < nb; bb += kLayoutThreads) off[bb] = warp_prefix_of_bucket(wcnt, nb, bb);
-  __syncthreads();
-  aligned_offsets(off, cnt, nb, align, warp_sums);
-  for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
-  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, 0, 1, d_status);
-  for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
-  for (int r = tid; r < R; r += kLayoutThreads) {
-    rank_offset[r] = off[r * epr];
-    rank_count[r] = off[(r + 1) * epr] - off[r * epr];
-    rank_tokens[r] = rtok[r];
-  }
-  if (tid == 0) rank_offset[R] = off[E];
-  if (tid < ne) {
-    const int slot = off[b] + wcnt[warp * nb + b] + in_warp;
-    if (!derived_row_ok(slot, num_rows, d_status)) {
-      token_slot[tid] = -1;
-    } else if (b < E) {
-      token_slot[tid] = slot;
-      slot_token[slot] = my_tok;
-    } else {
-      token_slot[tid] = -1;
-      slot_token[slot] = -1;
-    }
-  }
+  layout_single_body<true>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                           rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
 }
 
 }  // namespace
@@ -398,9 +244,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
   const int C = num_chunks(N, k);
   cudaError_t err;
   if (static_cast<long long>(N) * k <= kLayoutThreads) {
-    const size_t smem = (2 * (static_cast<size_t>(E) + 1) +
-                         static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R + kLayoutThreads + E) *
-                        sizeof(int32_t);
+    const size_t smem = layout_single_smem_words(E, R) * sizeof(int32_t);
     if (smem > 48 * 1024) {
       err = cudaFuncSetAttribute(layout_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem));
@@ -431,7 +275,31 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
   if (err != cudaSuccess) return err;
   return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
                     R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
-                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status,
+                    static_cast<unsigned*>(nullptr), static_cast<int32_t*>(nullptr), 0LL);
+}
+
+cudaError_t launch_layout_assign_zeroing(const int32_t* topk_idx, int N, int k, int E, int R,
+                                         int align, long long num_rows, int32_t* expert_count,
+                                         int32_t* expert_offset, int32_t* rank_count,
+                                         int32_t* rank_offset, int32_t* rank_tokens,
+                                         int32_t* token_slot, int32_t* slot_token,
+                                         int32_t* chunk_counts, unsigned* done, int32_t* d_status,
+                                         cudaStream_t stream) {
+  const int C = num_chunks(N, k);
+  int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
+  const size_t smem_assign =
+      (3 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
+      sizeof(int32_t);
+  if (smem_assign > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(layout_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem_assign));
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
+                    R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
+                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status, done,
+                    chunk_counts, static_cast<long long>(C) * (E + 1 + R));
 }
 
 }  // namespace moe

@@ -222,6 +222,45 @@ moe_status_t moe_get_layout_noalloc(const int32_t* topk_idx, int num_tokens, int
                                     int32_t* token_slot, int32_t* slot_token, int32_t* d_status,
                                     moe_stream_t stream);
 
+/* Bytes of device workspace moe_route needs for these sizes (a multiple of
+ * 256).  Zero it once before the first call (cudaMemset); every call leaves
+ * it zero again. */
+size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num_ranks);
+
+/*
+ * moe_route -- moe_topk_gate and moe_get_layout_aligned in one call, with the
+ * layout's counting folded into the gate: the routing decision and the
+ * dispatch handle come out of one enqueue.  [EPv2] usage patterns: build the
+ * routing handle on the GPU without a CPU synchronisation and reuse it for
+ * dispatch and combine; DeepGEMM "Mega MoE" news: fewer, overlapped launches
+ * (programmatic dependent launch).
+ *   Arguments and outputs are exactly those of the two calls (topk_idx and
+ *   topk_w as moe_topk_gate writes them, the layout arrays as
+ *   moe_get_layout_aligned writes them for those ids; align = 1 and
+ *   num_recv_rows = N*k give the packed layout), and so are the results, bit
+ *   for bit.
+ *   workspace  moe_route_workspace_bytes(N, k, E, R) bytes, 16-byte aligned,
+ *              ZERO before the first call; each call leaves it zero (the
+ *              kernels accumulate counts in it with atomics and the last CTA
+ *              clears them).  Do not share it with moe_get_layout, which
+ *              leaves its workspace dirty, nor between calls whose GPU work
+ *              overlaps.
+ *   How: when N*k <= 1024 and E = 32, 64, 128 or 256 (groups of whole lanes
+ *   for the group kind), one launch: each CTA gates 32 tokens and the CTA
+ *   that finishes last builds the layout.  Otherwise the gate launch also
+ *   counts every 1024-entry chunk's experts and ranks while it holds the
+ *   choices, and one assignment launch follows (two launches instead of
+ *   three).
+ *   Errors as in the two calls (host checks of both, then d_status).
+ */
+moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int k,
+                       moe_gate_kind_t kind, int n_groups, int topk_groups, int group_topn,
+                       int num_ranks, int align, int num_recv_rows, int32_t* topk_idx,
+                       float* topk_w, int32_t* expert_count, int32_t* expert_offset,
+                       int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
+                       int32_t* token_slot, int32_t* slot_token, void* workspace,
+                       size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
+
 /* Receive-buffer payload bytes: N*k rows of H bf16 (2 B) or e4m3 (1 B). */
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);
 /* Scale bytes for the FP8 payloads: N*k rows of H/128 fp32 (per block), of one
@@ -459,7 +498,7 @@ moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream
  *   exp_out[i]     = the exp every gate kind uses (Cody-Waite reduction with
  *                    ln2 split into a 16-bit head and a tail, degree-7 Taylor
  *                    polynomial by Horner, input clamped to [-87, 88] by
- *                    IEEE min/max, so a NaN input is taken as -87);
+ *                    comparisons, so every NaN input is taken as -87);
  *   sigmoid_out[i] = 1 / (1 + exp(-x_i)), each operation rounded once, the
  *                    score of the group-limited kind.
  * "DeepSeek, DeepEP 오픈소스 공개", Topic Body: group-limited gating, whose

@@ -91,10 +91,11 @@ float oracle_dexp(float y)
     const float c2 = 1.0f / 2.0f, c3 = 1.0f / 6.0f, c4 = 1.0f / 24.0f;
     const float c5 = 1.0f / 120.0f, c6 = 1.0f / 720.0f, c7 = 1.0f / 5040.0f;
 
-    /* clamp to [-87, 88]; fmaxf / fminf return the other operand when one
-     * is NaN, so a NaN input (outside the gate's contract) is clamped to -87
-     * and the routine is defined on every fp32 pattern */
-    y = fminf(fmaxf(y, -87.0f), 88.0f);
+    /* clamp to [-87, 88] by comparisons: any NaN input (outside the gate's
+     * contract; quiet or signalling) fails the first test and becomes -87,
+     * so the routine is defined on every fp32 pattern */
+    if (!(y > -87.0f)) y = -87.0f;
+    if (y > 88.0f) y = 88.0f;
     float t = y * log2e;        /* one fp32 rounding */
     float n = rintf(t);         /* nearest integer, ties to even */
     float r = fmaf(-n, ln2_head, y);

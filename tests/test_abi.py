@@ -335,3 +335,22 @@ def test_gate_math_rejects_bad_arguments(api):
     assert L.moe_gate_math(0, 16, None, None, None) == api.MOE_ERR_INVALID_ARG
     assert L.moe_gate_math(0, 16, 260, None, None) == api.MOE_ERR_INVALID_ARG   # not 16-byte aligned
     assert L.moe_gate_math(0, 16, None, 264, None) == api.MOE_ERR_INVALID_ARG
+
+
+def test_route_rejects_bad_arguments(api):
+    L = api.lib()
+    p = 256
+    ws = api.moe_route_workspace_bytes(64, 8, 256, 8)
+    assert ws == api.moe_layout_workspace_bytes(64, 8, 256, 8) + 256 and ws % 256 == 0
+    args = lambda **kw: [kw.get("logits", p), kw.get("N", 64), kw.get("E", 256), kw.get("k", 8),
+                         kw.get("kind", api.MOE_GATE_SIGMOID_GROUP), kw.get("G", 8), kw.get("TG", 4),
+                         kw.get("topn", 2), kw.get("R", 8), kw.get("align", 1), kw.get("rows", 512),
+                         p, p, p, p, p, p, p, p, p, kw.get("ws", p), kw.get("wsb", ws), None, None]
+    assert L.moe_route(*args(k=0)) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_route(*args(R=3)) == api.MOE_ERR_INVALID_ARG                 # E % R != 0
+    assert L.moe_route(*args(G=3)) == api.MOE_ERR_INVALID_ARG                 # E % G != 0
+    assert L.moe_route(*args(rows=511)) == api.MOE_ERR_INVALID_ARG            # fewer rows than N*k
+    assert L.moe_route(*args(wsb=ws - 1)) == api.MOE_ERR_INVALID_ARG          # short workspace
+    assert L.moe_route(*args(ws=p + 4)) == api.MOE_ERR_INVALID_ARG            # workspace not 16-byte aligned
+    assert L.moe_route(*args(E=2048, k=8, G=8)) == api.MOE_ERR_UNSUPPORTED
+    assert L.moe_route(*args(align=0)) == api.MOE_ERR_INVALID_ARG

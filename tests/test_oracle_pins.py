@@ -59,8 +59,9 @@ def test_dexp_saturation_and_monotone():
     assert O.dexp(float("inf")) == O.dexp(88.0) and O.dexp(float("-inf")) == O.dexp(-87.0)
     # the clamp takes a NaN input to -87 (NaN is outside the contract; the
     # routine is total so that every fp32 pattern has a defined result)
-    assert O.dexp(float("nan")) == O.dexp(-87.0)
-    assert O.sigmoid(float("nan")) == O.sigmoid(87.0) == 1.0
+    nans = np.array([0x7F800001, 0x7FC00000, 0x7FFFFFFF, 0xFF800001, 0xFFC00000], dtype=np.uint32).view(np.float32)
+    assert (O.dexp_array(nans) == np.float32(O.dexp(-87.0))).all()        # signalling and quiet NaNs alike
+    assert (O.sigmoid_array(nans) == np.float32(1.0)).all()
     x = np.sort(np.random.default_rng(2).uniform(-90, 90, 500_000).astype(np.float32))
     assert (np.diff(O.dexp_array(x)) >= 0).all()
 
