@@ -367,12 +367,13 @@ class StepRunner:
         self.y = self.recv if w.expert_out == "identity" else self.y_in
 
     def ops(self, stream=None):
-        """The step: gate and layout in one call (moe_route), dispatch, combine."""
+        """The step: gate and layout in one call (moe_route, which also has L2
+        fetch x for the dispatch that follows), dispatch, combine."""
         api, w, L = self.api, self.w, self.L
         return {
             "route": lambda: api.moe_route(self.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups,
                                            w.group_topn, w.R, topk_idx=self.idx, topk_w=self.wts, out=L,
-                                           stream=stream),
+                                           prefetch=self.x, stream=stream),
             "dispatch": lambda: api.moe_dispatch(self.x, L.token_slot, w.dtype_code, recv_x=self.recv,
                                                  recv_scale=self.scale, d_status=L.status, stream=stream),
             "combine": lambda: api.moe_combine(self.y, L.token_slot, self.wts, out=self.out,

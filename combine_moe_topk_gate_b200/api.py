@@ -61,7 +61,7 @@ def _load() -> ctypes.CDLL:
     L.moe_get_layout_noalloc.restype = I
     L.moe_route_workspace_bytes.argtypes = [I, I, I, I]
     L.moe_route_workspace_bytes.restype = SZ
-    L.moe_route.argtypes = [P, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, SZ, P, P]
+    L.moe_route.argtypes = [P, I, I, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, SZ, P, SZ, P, P]
     L.moe_route.restype = I
     L.moe_recv_bytes.argtypes = [I, I, I, I]
     L.moe_recv_bytes.restype = SZ
@@ -290,11 +290,13 @@ def moe_get_layout(topk_idx: torch.Tensor, num_experts: int, num_ranks: int, *, 
 
 def moe_route(logits: torch.Tensor, k: int, kind: int, n_groups: int, topk_groups: int, group_topn: int,
               num_ranks: int, *, align: int = 1, num_recv_rows: int | None = None, topk_idx=None, topk_w=None,
-              out: Layout | None = None, stream=None):
+              out: Layout | None = None, prefetch: torch.Tensor | None = None, stream=None):
     """Gate and layout in one call (moe_route): returns ``(topk_idx, topk_w,
     layout)`` equal to ``moe_topk_gate`` followed by ``moe_get_layout``.
     ``out.workspace`` must be a zeroed moe_route workspace
-    (``Layout.empty(..., route=True)``), which every call leaves zero."""
+    (``Layout.empty(..., route=True)``), which every call leaves zero.
+    ``prefetch``: a CUDA tensor read next (e.g. x before moe_dispatch), fetched
+    into L2 while the routing kernels run (a hint; no result changes)."""
     _need(logits, "logits", torch.float32)
     N, E = logits.shape
     R = num_ranks
@@ -312,13 +314,18 @@ def moe_route(logits: torch.Tensor, k: int, kind: int, n_groups: int, topk_group
         raise ValueError(f"out.workspace must hold moe_route_workspace_bytes = {need} bytes "
                          f"(Layout.empty(..., route=True)), got {out.workspace.numel()}")
     rows = out.num_rows
+    pf_bytes = 0
+    if prefetch is not None:
+        if not prefetch.is_cuda or not prefetch.is_contiguous():
+            raise ValueError("prefetch must be a contiguous CUDA tensor")
+        pf_bytes = prefetch.numel() * prefetch.element_size() // 16 * 16
     tensors = (logits, topk_idx, topk_w, out.expert_count, out.expert_offset, out.rank_count, out.rank_offset,
-               out.rank_tokens, out.token_slot, out.slot_token, out.workspace, _status(out.status))
+               out.rank_tokens, out.token_slot, out.slot_token, out.workspace, _status(out.status), prefetch)
     _launch(_lib.moe_route, "moe_route", tensors, _ptr(logits), N, E, k, kind, n_groups, topk_groups, group_topn,
             R, align, rows, _ptr(topk_idx), _ptr(topk_w), _ptr(out.expert_count), _ptr(out.expert_offset),
             _ptr(out.rank_count), _ptr(out.rank_offset), _ptr(out.rank_tokens), _ptr(out.token_slot),
-            _ptr(out.slot_token), _ptr(out.workspace), out.workspace.numel(), _ptr(out.status),
-            _stream(stream, logits.device))
+            _ptr(out.slot_token), _ptr(out.workspace), out.workspace.numel(),
+            _ptr(prefetch) if pf_bytes else None, pf_bytes, _ptr(out.status), _stream(stream, logits.device))
     out.align = align
     return topk_idx, topk_w, out
 

@@ -11,6 +11,7 @@
 namespace {
 
 constexpr long long kMaxRows = 0x7fffffffLL;  // int32 slot ids
+constexpr size_t kMaxPrefetchBytes = size_t(64) << 20;  // moe_route's L2 prefetch: half the L2 at most
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -22,7 +23,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 5; }
+int moe_abi_version(void) { return 6; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -126,7 +127,8 @@ moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int
                        float* topk_w, int32_t* expert_count, int32_t* expert_offset,
                        int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
                        int32_t* token_slot, int32_t* slot_token, void* workspace,
-                       size_t workspace_bytes, int32_t* d_status, moe_stream_t stream) {
+                       size_t workspace_bytes, const void* prefetch, size_t prefetch_bytes,
+                       int32_t* d_status, moe_stream_t stream) {
   const int N = num_tokens, E = num_experts, R = num_ranks;
   // the gate's checks
   if (N < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
@@ -156,8 +158,11 @@ moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int
   for (const void* p : ptrs)
     if (!aligned(p, 4)) return MOE_ERR_INVALID_ARG;
   if (!aligned(workspace, 16)) return MOE_ERR_INVALID_ARG;
-  const moe::RouteOut out{expert_count, expert_offset, rank_count, rank_offset, rank_tokens,
-                          token_slot,   slot_token,    align,      num_recv_rows, d_status};
+  if (prefetch_bytes > 0 && (!prefetch || !aligned(prefetch, 16))) return MOE_ERR_INVALID_ARG;
+  const size_t pf_bytes = prefetch_bytes < kMaxPrefetchBytes ? prefetch_bytes : kMaxPrefetchBytes;
+  const moe::RouteOut out{expert_count, expert_offset, rank_count, rank_offset,
+                          rank_tokens,  token_slot,    slot_token, align,
+                          num_recv_rows, d_status,     pf_bytes ? prefetch : nullptr, pf_bytes};
   return from_cuda(moe::launch_route(logits, N, E, k, kind, n_groups, topk_groups, group_topn, R,
                                      topk_idx, topk_w, out, workspace, as_stream(stream)));
 }

@@ -149,6 +149,8 @@ struct ChunkCount {
   int32_t* rtok;    // [C][R]
   int E, R, epr;    // experts, ranks, experts per rank
   int tpc;          // tokens per chunk
+  const char* prefetch;             // the caller's next input, fetched into L2 meanwhile
+  unsigned long long prefetch_bytes;
 };
 
 // Lane j < k holds the token's slot j (expert sel_i, or -1).  The token is
@@ -299,6 +301,7 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   const int warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
+  prefetch_share_l2(cc.prefetch, cc.prefetch_bytes);
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps)
     gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, sh_exp[warp], lane, topk_idx, topk_w, cc);
 }
@@ -319,15 +322,17 @@ __global__ void __launch_bounds__(kLayoutThreads)
                        int32_t* __restrict__ rank_count, int32_t* __restrict__ rank_offset,
                        int32_t* __restrict__ rank_tokens, int32_t* __restrict__ token_slot,
                        int32_t* __restrict__ slot_token, int align, long long num_rows,
-                       int32_t* d_status, unsigned* done) {
+                       int32_t* d_status, unsigned* done, const char* prefetch,
+                       unsigned long long prefetch_bytes) {
   extern __shared__ int32_t sm[];  // gate: one row of E floats per warp; then the layout's words
   __shared__ int last_cta;
   constexpr int E = 32 * V;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
+  prefetch_share_l2(prefetch, prefetch_bytes);
   const int t = blockIdx.x * kLayoutWarps + warp;
-  const ChunkCount none{nullptr, nullptr, E, 1, E, 1};
+  const ChunkCount none{nullptr, nullptr, E, 1, E, 1, nullptr, 0};
   if (t < N)
     gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, reinterpret_cast<float*>(sm) + warp * E,
                               lane, topk_idx, topk_w, none);
@@ -358,6 +363,7 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   const int eg = E / G;
   pdl_wait();
   pdl_trigger();
+  prefetch_share_l2(cc.prefetch, cc.prefetch_bytes);
 
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
     const float* row = logits + static_cast<size_t>(t) * E;
@@ -597,6 +603,7 @@ template <int V, int TOPN>
 cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
                                  int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
                                  cudaStream_t stream) {
+  const char* pf = static_cast<const char*>(o.prefetch);
   constexpr int E = 32 * V;
   const size_t words = layout_single_smem_words(E, R);
   const size_t smem = (words > static_cast<size_t>(kLayoutWarps) * E ? words : static_cast<size_t>(kLayoutWarps) * E) *
@@ -609,7 +616,8 @@ cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, in
   const unsigned grid = static_cast<unsigned>((N + kLayoutWarps - 1) / kLayoutWarps);
   return launch_pdl(route_small_kernel<V, TOPN>, grid, kLayoutThreads, smem, stream, logits, N, k, kind,
                     lpg_log2, TG, idx, w, R, o.expert_count, o.expert_offset, o.rank_count, o.rank_offset,
-                    o.rank_tokens, o.token_slot, o.slot_token, o.align, o.num_rows, o.d_status, done);
+                    o.rank_tokens, o.token_slot, o.slot_token, o.align, o.num_rows, o.d_status, done, pf,
+                    static_cast<unsigned long long>(o.prefetch_bytes));
 }
 
 template <int V>
@@ -644,9 +652,14 @@ cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int
         default: return launch_route_small<8>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
       }
     }
-    // other expert counts (or no tokens): gate, then the one-CTA layout
-    cudaError_t err = launch_topk_gate(logits, N, E, k, kind, n_groups, topk_groups, group_topn, topk_idx,
-                                       topk_w, stream);
+    // other expert counts (or no tokens): gate (with the prefetch), then the
+    // one-CTA layout
+    cudaError_t err = cudaSuccess;
+    if (N > 0) {
+      const ChunkCount pf{nullptr, nullptr, E, 1, E, 1, static_cast<const char*>(o.prefetch),
+                          static_cast<unsigned long long>(o.prefetch_bytes)};
+      err = launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, pf, stream);
+    }
     if (err != cudaSuccess) return err;
     return launch_layout(topk_idx, N, k, E, R, o.align, o.num_rows, o.expert_count, o.expert_offset,
                          o.rank_count, o.rank_offset, o.rank_tokens, o.token_slot, o.slot_token, chunks,
@@ -655,7 +668,8 @@ cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int
   // gate with the per-chunk counts folded in, then the assignment (which
   // leaves the counts zeroed again)
   const int C = (N + kLayoutThreads / k - 1) / (kLayoutThreads / k);
-  const ChunkCount cc{chunks, chunks + static_cast<size_t>(C) * (E + 1), E, R, E / R, kLayoutThreads / k};
+  const ChunkCount cc{chunks, chunks + static_cast<size_t>(C) * (E + 1), E, R, E / R, kLayoutThreads / k,
+                      static_cast<const char*>(o.prefetch), static_cast<unsigned long long>(o.prefetch_bytes)};
   cudaError_t err = launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, cc, stream);
   if (err != cudaSuccess) return err;
   return launch_layout_assign_zeroing(topk_idx, N, k, E, R, o.align, o.num_rows, o.expert_count,
@@ -668,7 +682,7 @@ cudaError_t launch_topk_gate(const float* logits, int N, int E, int k, int kind,
                              cudaStream_t stream) {
   if (N == 0) return cudaSuccess;
   const GatePlan p = plan_gate(logits, E, kind, n_groups, topk_groups, group_topn);
-  const ChunkCount none{nullptr, nullptr, E, 1, E, 1};
+  const ChunkCount none{nullptr, nullptr, E, 1, E, 1, nullptr, 0};
   return launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, none, stream);
 }
 

@@ -312,6 +312,27 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// Asks L2 to fetch [src, src + bytes) (bulk prefetch: no data returns to the
+// SM, nothing waits on it; src and bytes multiples of 16).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// CTA blockIdx.x of gridDim.x prefetches its share of [base, base + bytes)
+// into L2 (thread 0 issues it in pieces of at most 64 KiB).  base 16-byte
+// aligned; bytes is rounded down to a multiple of 16.
+__device__ __forceinline__ void prefetch_share_l2(const char* base, unsigned long long bytes) {
+  if (base == nullptr || threadIdx.x != 0) return;
+  bytes &= ~15ull;
+  const unsigned long long per = ((bytes + gridDim.x - 1) / gridDim.x + 15) & ~15ull;
+  unsigned long long b = per * blockIdx.x;
+  const unsigned long long e = b + per < bytes ? b + per : bytes;
+  for (; b < e; b += 65536) {
+    const unsigned long long n = e - b < 65536 ? e - b : 65536;
+    prefetch_l2_bulk(base + b, static_cast<uint32_t>(n));
+  }
+}
+
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"

@@ -27,6 +27,8 @@ struct RouteOut {
   int align;
   long long num_rows;
   int32_t* d_status;
+  const void* prefetch;   // optional: a buffer the caller reads next, fetched into L2
+  size_t prefetch_bytes;
 };
 
 // Fused routing workspace: an arrival counter in the first kRouteCounterBytes,

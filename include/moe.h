@@ -251,6 +251,15 @@ size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num
  *   counts every 1024-entry chunk's experts and ranks while it holds the
  *   choices, and one assignment launch follows (two launches instead of
  *   three).
+ *   prefetch   optional device buffer the caller reads next -- typically x,
+ *              which moe_dispatch reads right after this call -- and its size
+ *              in bytes (NULL / 0: none; 16-byte aligned, a multiple of 16
+ *              bytes is used; at most the first 64 MiB).  While gating and
+ *              layout run (latency-bound, little traffic) the kernels ask L2
+ *              to fetch it, so the next kernel reads it from L2.  A hint
+ *              only: it changes no result, and the buffer must simply be
+ *              readable (it is fetched after this call's predecessors
+ *              finished, as any read of the call would be).
  *   Errors as in the two calls (host checks of both, then d_status).
  */
 moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int k,
@@ -259,7 +268,8 @@ moe_status_t moe_route(const float* logits, int num_tokens, int num_experts, int
                        float* topk_w, int32_t* expert_count, int32_t* expert_offset,
                        int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
                        int32_t* token_slot, int32_t* slot_token, void* workspace,
-                       size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
+                       size_t workspace_bytes, const void* prefetch, size_t prefetch_bytes,
+                       int32_t* d_status, moe_stream_t stream);
 
 /* Receive-buffer payload bytes: N*k rows of H bf16 (2 B) or e4m3 (1 B). */
 size_t moe_recv_bytes(int num_tokens, int hidden, int k, moe_dtype_t dtype);

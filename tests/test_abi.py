@@ -345,7 +345,8 @@ def test_route_rejects_bad_arguments(api):
     args = lambda **kw: [kw.get("logits", p), kw.get("N", 64), kw.get("E", 256), kw.get("k", 8),
                          kw.get("kind", api.MOE_GATE_SIGMOID_GROUP), kw.get("G", 8), kw.get("TG", 4),
                          kw.get("topn", 2), kw.get("R", 8), kw.get("align", 1), kw.get("rows", 512),
-                         p, p, p, p, p, p, p, p, p, kw.get("ws", p), kw.get("wsb", ws), None, None]
+                         p, p, p, p, p, p, p, p, p, kw.get("ws", p), kw.get("wsb", ws),
+                         kw.get("pf", None), kw.get("pfb", 0), None, None]
     assert L.moe_route(*args(k=0)) == api.MOE_ERR_INVALID_ARG
     assert L.moe_route(*args(R=3)) == api.MOE_ERR_INVALID_ARG                 # E % R != 0
     assert L.moe_route(*args(G=3)) == api.MOE_ERR_INVALID_ARG                 # E % G != 0
@@ -354,3 +355,5 @@ def test_route_rejects_bad_arguments(api):
     assert L.moe_route(*args(ws=p + 4)) == api.MOE_ERR_INVALID_ARG            # workspace not 16-byte aligned
     assert L.moe_route(*args(E=2048, k=8, G=8)) == api.MOE_ERR_UNSUPPORTED
     assert L.moe_route(*args(align=0)) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_route(*args(pf=None, pfb=4096)) == api.MOE_ERR_INVALID_ARG     # prefetch size without a buffer
+    assert L.moe_route(*args(pf=p + 8, pfb=4096)) == api.MOE_ERR_INVALID_ARG    # prefetch not 16-byte aligned

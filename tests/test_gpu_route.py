@@ -111,3 +111,25 @@ def test_route_rejects_a_short_workspace():
     L = api.Layout.empty(w.N, w.k, w.E, w.R, "cuda")      # moe_get_layout's size: 256 bytes short
     with pytest.raises(ValueError, match="workspace"):
         api.moe_route(logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn, w.R, out=L)
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "mixtral"])
+def test_route_with_l2_prefetch_gives_the_same_results(name):
+    """The prefetch region (x of the dispatch that follows, more than the
+    64 MiB cap on the Mixtral shape) is a hint: results are unchanged, and a
+    dispatch right after still matches the oracle."""
+    from combine_moe_topk_gate_b200 import api
+    w = WORKLOADS[name]
+    inp = make_inputs(w, 2, with_y=False)
+    x = inp.x.cuda()
+    idx, wts, L = api.moe_route(inp.logits.cuda(), w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn, w.R,
+                                prefetch=x)
+    recv, scale = api.moe_dispatch(x, L.token_slot, w.dtype_code, d_status=L.status)
+    torch.cuda.synchronize()
+    _check(w, inp, idx.cpu().numpy(), wts.cpu().numpy(), L)
+    from _harness import bf16_bits
+    r_recv, r_scale, _ = O.dispatch(bf16_bits(inp.x), L.token_slot.cpu().numpy(), w.dtype_code)
+    got = recv.cpu().numpy() if w.dtype != "bf16" else bf16_bits(recv)
+    assert np.array_equal(got, r_recv)
+    if scale is not None:
+        assert np.array_equal(scale.cpu().numpy().view(np.uint8), r_scale.view(np.uint8))
