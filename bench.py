@@ -491,9 +491,39 @@ def other_workloads(api, main, device, steps, warmup, flush, peak) -> dict:
         iso = isolated_op_times(r.ops, flush, device)
         iso.update(isolated_op_times(r.separate_ops, flush, device))
         res[name] = summary_of(w, step_ms, per_op, iso, peak)
+        res[name]["quant_fp8_channel"] = channel_fp8_time(api, r, flush, device, peak)
         del r
         torch.cuda.empty_cache()
     return res
+
+
+def channel_fp8_time(api, r, flush, device, peak, align: int = 128) -> dict:
+    """Per-(expert, channel) FP8 of a seeded bf16 receive buffer laid out by
+    this batch's GEMM-aligned layout (the weight-gradient GEMM's operand),
+    alone with a clean cold L2; bytes = the landed rows read once and their
+    codes written once, plus the scales."""
+    w = r.w
+    api.moe_route(r.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn, w.R,
+                  topk_idx=r.idx, topk_w=r.wts, out=r.L)
+    rows = api.moe_aligned_recv_rows(w.N, w.k, w.E, align)
+    La = api.Layout.empty(w.N, w.k, w.E, w.R, device, align=align)
+    api.moe_get_layout(r.idx, w.E, w.R, align=align, out=La)
+    y = torch.empty((rows, w.H), dtype=torch.bfloat16, device=device).normal_(generator=torch.Generator(
+        device=device).manual_seed(11))
+    out = torch.empty((rows, w.H), dtype=torch.uint8, device=device)
+    sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+    us = isolated_op_times(lambda: {"quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
+        y, La.expert_offset, La.expert_count, out=out, scale=sc, d_status=La.status)}, flush, device)
+    us = us["quant_fp8_channel"]
+    counts = La.expert_count.cpu()
+    landed = int(counts.sum().item())
+    nbytes = landed * w.H * 3 + 4 * w.E * w.H + 8 * w.E
+    torch.cuda.synchronize(device)
+    if int(La.status.item()) != 0:
+        raise RuntimeError(f"device status {int(La.status.item())} after the per-channel FP8")
+    return {"us": us, "frac": nbytes / (us * 1e-6) / 1e9 / peak if us else None, "algorithmic_bytes": nbytes,
+            "landed_rows": landed, "max_expert_rows": int(counts.max().item()),
+            "mean_expert_rows": landed / w.E}
 
 
 def run_ours(args, rank, world, device):
@@ -522,6 +552,7 @@ def run_ours(args, rank, world, device):
         workloads = None
         if world == 1 and not args.no_workloads and args.tokens is None:
             workloads = {w.name: summary_of(w, step_ms, per_op, isolated, peak)}
+            workloads[w.name]["quant_fp8_channel"] = channel_fp8_time(api, r, flush, device, peak)
             workloads.update(other_workloads(api, w.name, device, args.steps, args.warmup, flush, peak))
         backward = None
         if not args.no_backward:

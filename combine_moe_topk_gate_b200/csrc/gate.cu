@@ -33,6 +33,7 @@ namespace moe {
 namespace {
 
 constexpr int kGateWarps = 8;
+constexpr int kSmallRouteTokens = 8;  // tokens gated per CTA on the one-launch routing path
 constexpr int kMaxTopn = 4;
 
 // Order-preserving map of a float onto uint32 (larger float -> larger code).
@@ -308,7 +309,10 @@ __global__ void __launch_bounds__(kGateWarps * 32)
 
 // ------------------------------------------------------------------ fused routing, small batches
 // Gate and layout in one launch when every entry fits one layout chunk
-// (N*k <= kLayoutThreads): CTAs of kLayoutWarps warps, one token per warp.
+// (N*k <= kLayoutThreads): CTAs of kLayoutThreads threads of which the first
+// kSmallRouteTokens warps gate one token each (as many tokens per SM as the
+// gate kernel's CTAs take, so the gating spreads over as many SMs); all
+// kLayoutWarps warps of the last CTA build the layout.
 // Each CTA publishes its tokens' choices (fence, then an arrival on a counter
 // in the caller's zeroed workspace); the CTA that arrives last -- every
 // other CTA's outputs are visible to it by then -- builds the whole layout
@@ -331,9 +335,9 @@ __global__ void __launch_bounds__(kLayoutThreads)
   pdl_wait();
   pdl_trigger();
   prefetch_share_l2(prefetch, prefetch_bytes);
-  const int t = blockIdx.x * kLayoutWarps + warp;
+  const int t = blockIdx.x * kSmallRouteTokens + warp;
   const ChunkCount none{nullptr, nullptr, E, 1, E, 1, nullptr, 0};
-  if (t < N)
+  if (warp < kSmallRouteTokens && t < N)
     gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, reinterpret_cast<float*>(sm) + warp * E,
                               lane, topk_idx, topk_w, none);
   __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
@@ -613,7 +617,7 @@ cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, in
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  const unsigned grid = static_cast<unsigned>((N + kLayoutWarps - 1) / kLayoutWarps);
+  const unsigned grid = static_cast<unsigned>((N + kSmallRouteTokens - 1) / kSmallRouteTokens);
   return launch_pdl(route_small_kernel<V, TOPN>, grid, kLayoutThreads, smem, stream, logits, N, k, kind,
                     lpg_log2, TG, idx, w, R, o.expert_count, o.expert_offset, o.rank_count, o.rank_offset,
                     o.rank_tokens, o.token_slot, o.slot_token, o.align, o.num_rows, o.d_status, done, pf,

@@ -246,7 +246,7 @@ size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num
  *              leaves its workspace dirty, nor between calls whose GPU work
  *              overlaps.
  *   How: when N*k <= 1024 and E = 32, 64, 128 or 256 (groups of whole lanes
- *   for the group kind), one launch: each CTA gates 32 tokens and the CTA
+ *   for the group kind), one launch: each CTA gates 8 tokens and the CTA
  *   that finishes last builds the layout.  Otherwise the gate launch also
  *   counts every 1024-entry chunk's experts and ranks while it holds the
  *   choices, and one assignment launch follows (two launches instead of
