@@ -17,13 +17,12 @@ CASES = [
     (WORKLOADS["decode"], 128, 0.0),
     (WORKLOADS["prefill"], 128, 0.0),
     (Workload("ch_ragged", 300, 384, 40, 3, 8, "softmax", "bf16", "random"), 8, 0.25),
-    # few experts with thousands of rows each: narrow channel slabs (down to
-    # 16 channels) so that every unit of work stays small; H = 384 caps the
-    # slab at 128 channels
+    # few experts with thousands of rows each: several CTAs per (expert, slab),
+    # combined through a thread-block cluster (2, 4 and 8 CTAs)
     (Workload("ch_q2", 1100, 256, 2, 2, 2, "softmax", "bf16", "random"), 128, 0.1),
     (Workload("ch_q4", 3000, 384, 2, 2, 2, "softmax", "bf16", "random"), 32, 0.3),
     (Workload("ch_q8", 8192, 384, 4, 2, 2, "softmax", "bf16", "random"), 128, 0.2),
-    # skewed loads: hot experts (narrow slabs) next to cold ones (wide slabs)
+    # skewed loads: hot experts next to cold ones
     (Workload("ch_zipf", 4096, 512, 64, 8, 8, "sigmoid_group", "fp8", "random", 8, 4, 2, bias="zipf1.1"), 128, 0.0),
     (Workload("ch_mixtral", 16384, 512, 8, 2, 8, "softmax_renorm", "bf16", "identity", bias="expert0+2"), 128, 0.0),
 ]
@@ -85,11 +84,10 @@ def test_quant_fp8_channel_reports_bad_ranges():
 
 
 @pytest.mark.parametrize("transpose", [False, True])
-def test_big_expert_next_to_empty_and_short_ones(transpose):
-    """40 000 rows over 4 experts: expert 0 with almost all rows (16-channel
-    slabs), experts 1 and 3 empty (their scales must still be written as 0),
-    expert 2 with 37 rows (256-channel slabs); nothing outside the landed rows
-    is touched."""
+def test_clustered_split_with_empty_experts(transpose):
+    """40 000 rows over 4 experts (8 CTAs per expert and slab), experts 1 and 3
+    empty, expert 2 with 37 rows: the empty and short experts' CTAs still meet
+    the cluster barriers, and nothing outside the landed rows is touched."""
     from combine_moe_topk_gate_b200 import api
     dev = torch.device("cuda", 0)
     N, H, E = 40000, 256, 4
