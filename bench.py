@@ -130,10 +130,12 @@ def ncu_traffic(op: str, workload: str):
 
 def launches_per_step(w) -> int:
     """Kernels one step launches: routing (one launch when all N*k entries fit
-    one 1024-entry chunk and E = 32, 64, 128 or 256, else the counting gate +
-    the assignment), dispatch, combine."""
+    one 1024-entry chunk and E = 32, 64, 128 or 256; else the gate and the
+    layout's one or two launches), dispatch, combine."""
     lanes_gate = w.E % 32 == 0 and (w.E // 32) in (1, 2, 4, 8)
-    return (1 if w.N * w.k <= 1024 and lanes_gate else 2) + 1 + 1
+    small = w.N * w.k <= 1024
+    route = 1 if small and lanes_gate else (2 if small else 3)
+    return route + 1 + 1
 
 
 def isolated_op_times(step_ops, flush, device, reps=30):

@@ -221,7 +221,7 @@ class Layout:
         """Uninitialised arrays for an N x k batch over E experts and R ranks;
         ``workspace=False`` gives a 0-byte workspace (for the no-workspace
         entry point); ``route=True`` a zeroed workspace of moe_route's size
-        (moe_route keeps it zero; do not pass it to moe_get_layout)."""
+        (moe_route keeps its first 256 bytes, an arrival counter, zero)."""
         i32 = dict(dtype=torch.int32, device=device)
         if route:
             ws = moe_route_workspace_bytes(N, k, E, R)
@@ -293,8 +293,8 @@ def moe_route(logits: torch.Tensor, k: int, kind: int, n_groups: int, topk_group
               out: Layout | None = None, prefetch: torch.Tensor | None = None, stream=None):
     """Gate and layout in one call (moe_route): returns ``(topk_idx, topk_w,
     layout)`` equal to ``moe_topk_gate`` followed by ``moe_get_layout``.
-    ``out.workspace`` must be a zeroed moe_route workspace
-    (``Layout.empty(..., route=True)``), which every call leaves zero.
+    ``out.workspace`` must be a moe_route workspace whose first 256 bytes are
+    zero (``Layout.empty(..., route=True)``); every call leaves them zero.
     ``prefetch``: a CUDA tensor read next (e.g. x before moe_dispatch), fetched
     into L2 while the routing kernels run (a hint; no result changes)."""
     _need(logits, "logits", torch.float32)

@@ -82,10 +82,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
                          int32_t* __restrict__ expert_offset, int32_t* __restrict__ rank_count,
                          int32_t* __restrict__ rank_offset, int32_t* __restrict__ rank_tokens,
                          int32_t* __restrict__ token_slot, int32_t* __restrict__ slot_token,
-                         int align, long long num_rows, int32_t* d_status, unsigned* done,
-                         int32_t* ws_clear, long long ws_words) {
+                         int align, long long num_rows, int32_t* d_status) {
   extern __shared__ int32_t sm[];
-  __shared__ int last_cta;
   const int nb = E + 1;
   int32_t* off = sm;                 // nb: totals, then their exclusive (aligned) scan
   int32_t* base = off + nb;          // nb: first row of this chunk per bucket
@@ -197,19 +195,6 @@ __global__ void __launch_bounds__(kLayoutThreads)
     }
   }
   (void)lane;
-  // Fused routing (done != NULL): the chunk counts were accumulated with
-  // atomics into zeroed workspace.  Every CTA has read them before it gets
-  // here, so the last CTA to arrive zeroes them (and the arrival counter)
-  // for the next call.  No CTA waits for another.
-  if (done != nullptr) {
-    __syncthreads();
-    if (tid == 0) last_cta = atomicAdd(done, 1u) == static_cast<unsigned>(C - 1);
-    __syncthreads();
-    if (last_cta) {
-      for (long long i = tid; i < ws_words; i += kLayoutThreads) ws_clear[i] = 0;
-      if (tid == 0) *done = 0u;
-    }
-  }
 }
 
 // Whole layout in one CTA when every entry fits one chunk (N*k <= 1024, the
@@ -275,31 +260,7 @@ cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, i
   if (err != cudaSuccess) return err;
   return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
                     R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
-                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status,
-                    static_cast<unsigned*>(nullptr), static_cast<int32_t*>(nullptr), 0LL);
-}
-
-cudaError_t launch_layout_assign_zeroing(const int32_t* topk_idx, int N, int k, int E, int R,
-                                         int align, long long num_rows, int32_t* expert_count,
-                                         int32_t* expert_offset, int32_t* rank_count,
-                                         int32_t* rank_offset, int32_t* rank_tokens,
-                                         int32_t* token_slot, int32_t* slot_token,
-                                         int32_t* chunk_counts, unsigned* done, int32_t* d_status,
-                                         cudaStream_t stream) {
-  const int C = num_chunks(N, k);
-  int32_t* chunk_rtok = chunk_counts + static_cast<size_t>(C) * (E + 1);
-  const size_t smem_assign =
-      (3 * (static_cast<size_t>(E) + 1) + static_cast<size_t>(kLayoutWarps) * (E + 1) + 32 + R) *
-      sizeof(int32_t);
-  if (smem_assign > 48 * 1024) {
-    cudaError_t err = cudaFuncSetAttribute(layout_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem_assign));
-    if (err != cudaSuccess) return err;
-  }
-  return launch_pdl(layout_assign_kernel, C, kLayoutThreads, smem_assign, stream, topk_idx, N, k, E,
-                    R, C, chunk_counts, chunk_rtok, expert_count, expert_offset, rank_count,
-                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status, done,
-                    chunk_counts, static_cast<long long>(C) * (E + 1 + R));
+                    rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
 }
 
 }  // namespace moe

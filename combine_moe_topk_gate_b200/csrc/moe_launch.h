@@ -31,21 +31,15 @@ struct RouteOut {
   size_t prefetch_bytes;
 };
 
-// Fused routing workspace: an arrival counter in the first kRouteCounterBytes,
-// then the layout's per-chunk counts; zero before the first call, left zero
-// by every call.
+// Routing workspace: an arrival counter in the first kRouteCounterBytes (zero
+// before the first call, left zero by every call), then the layout's
+// per-chunk counts (scratch).
 constexpr size_t kRouteCounterBytes = 256;
 size_t route_workspace_bytes(int N, int k, int E, int R);
 cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int n_groups,
                          int topk_groups, int group_topn, int R, int32_t* topk_idx, float* topk_w,
                          const RouteOut& out, void* workspace, cudaStream_t stream);
-cudaError_t launch_layout_assign_zeroing(const int32_t* topk_idx, int N, int k, int E, int R,
-                                         int align, long long num_rows, int32_t* expert_count,
-                                         int32_t* expert_offset, int32_t* rank_count,
-                                         int32_t* rank_offset, int32_t* rank_tokens,
-                                         int32_t* token_slot, int32_t* slot_token,
-                                         int32_t* chunk_counts, unsigned* done, int32_t* d_status,
-                                         cudaStream_t stream);
+
 
 cudaError_t launch_layout(const int32_t* topk_idx, int N, int k, int E, int R, int align,
                           long long num_rows, int32_t* expert_count, int32_t* expert_offset,

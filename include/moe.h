@@ -223,34 +223,31 @@ moe_status_t moe_get_layout_noalloc(const int32_t* topk_idx, int num_tokens, int
                                     moe_stream_t stream);
 
 /* Bytes of device workspace moe_route needs for these sizes (a multiple of
- * 256).  Zero it once before the first call (cudaMemset); every call leaves
- * it zero again. */
+ * 256).  Its first 256 bytes must be zero before the first call (cudaMemset
+ * the whole buffer once); every call leaves them zero. */
 size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num_ranks);
 
 /*
- * moe_route -- moe_topk_gate and moe_get_layout_aligned in one call, with the
- * layout's counting folded into the gate: the routing decision and the
- * dispatch handle come out of one enqueue.  [EPv2] usage patterns: build the
- * routing handle on the GPU without a CPU synchronisation and reuse it for
- * dispatch and combine; DeepGEMM "Mega MoE" news: fewer, overlapped launches
- * (programmatic dependent launch).
+ * moe_route -- moe_topk_gate and moe_get_layout_aligned in one call: the
+ * routing decision and the dispatch handle come out of one enqueue.
+ * [EPv2] usage patterns: build the routing handle on the GPU without a CPU
+ * synchronisation and reuse it for dispatch and combine; DeepGEMM "Mega MoE"
+ * news: fewer, overlapped launches (programmatic dependent launch).
  *   Arguments and outputs are exactly those of the two calls (topk_idx and
  *   topk_w as moe_topk_gate writes them, the layout arrays as
  *   moe_get_layout_aligned writes them for those ids; align = 1 and
  *   num_recv_rows = N*k give the packed layout), and so are the results, bit
  *   for bit.
- *   workspace  moe_route_workspace_bytes(N, k, E, R) bytes, 16-byte aligned,
- *              ZERO before the first call; each call leaves it zero (the
- *              kernels accumulate counts in it with atomics and the last CTA
- *              clears them).  Do not share it with moe_get_layout, which
- *              leaves its workspace dirty, nor between calls whose GPU work
- *              overlaps.
+ *   workspace  moe_route_workspace_bytes(N, k, E, R) bytes, 16-byte aligned.
+ *              The first 256 bytes hold an arrival counter: zero before the
+ *              first call, left zero by every call; the rest is scratch.  Do
+ *              not share it between calls whose GPU work overlaps.
  *   How: when N*k <= 1024 and E = 32, 64, 128 or 256 (groups of whole lanes
  *   for the group kind), one launch: each CTA gates 8 tokens and the CTA
- *   that finishes last builds the layout.  Otherwise the gate launch also
- *   counts every 1024-entry chunk's experts and ranks while it holds the
- *   choices, and one assignment launch follows (two launches instead of
- *   three).
+ *   that arrives last on the counter builds the layout.  Otherwise the gate
+ *   launch and the layout's launches follow each other with programmatic
+ *   dependent launch (for large batches three overlapped launches measured
+ *   faster than a gate that also counts).
  *   prefetch   optional device buffer the caller reads next -- typically x,
  *              which moe_dispatch reads right after this call -- and its size
  *              in bytes (NULL / 0: none; 16-byte aligned, a multiple of 16

@@ -58,7 +58,7 @@ def test_launches_per_step():
     bench = _bench()
     assert bench.launches_per_step(WORKLOADS["tiny"]) == 4      # E = 8: gate, then the one-CTA layout
     assert bench.launches_per_step(WORKLOADS["decode"]) == 3    # N*k = 1024: still one launch
-    assert bench.launches_per_step(WORKLOADS["prefill"]) == 4   # counting gate + assignment
+    assert bench.launches_per_step(WORKLOADS["prefill"]) == 5   # gate, count, assign
 
 
 def test_whole_job_rate_is_tokens_over_time():
