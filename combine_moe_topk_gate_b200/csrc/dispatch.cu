@@ -623,15 +623,22 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
   }
 }
 
+// Segments per warp: reading x is most of the traffic when k is small, and
+// load latency then sets the pace, so each warp issues the loads of several
+// neighbouring 512-channel segments before working on the first.
+int segments_per_warp(int k) { return k <= 2 ? 4 : k <= 4 ? 2 : 1; }
+
 template <int SL, bool UE8M0>
-cudaError_t launch_fp8(bool two, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+cudaError_t launch_fp8(int spw, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                        long long num_rows, uint8_t* recv_x, float* recv_scale, long long ld,
                        int32_t* d_status, cudaStream_t stream) {
   const int segs = (H + 511) / 512;
-  const int spw = two ? 2 : 1;
   const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
   const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  if (two)
+  if (spw == 4)
+    return launch_pdl(dispatch_fp8_kernel<SL, UE8M0, 4>, blocks, kWarps * 32, 0, stream, x, N, H, k,
+                      token_slot, num_rows, recv_x, recv_scale, ld, d_status);
+  if (spw == 2)
     return launch_pdl(dispatch_fp8_kernel<SL, UE8M0, 2>, blocks, kWarps * 32, 0, stream, x, N, H, k,
                       token_slot, num_rows, recv_x, recv_scale, ld, d_status);
   return launch_pdl(dispatch_fp8_kernel<SL, UE8M0, 1>, blocks, kWarps * 32, 0, stream, x, N, H, k,
@@ -639,14 +646,16 @@ cudaError_t launch_fp8(bool two, const uint16_t* x, int N, int H, int k, const i
 }
 
 template <int SL>
-cudaError_t launch_mx(bool two, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
+cudaError_t launch_mx(int spw, const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                       long long num_rows, uint8_t* recv_x, uint8_t* recv_e8m0, long long ld,
                       int32_t* d_status, cudaStream_t stream) {
   const int segs = (H + 511) / 512;
-  const int spw = two ? 2 : 1;
   const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
   const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
-  if (two)
+  if (spw == 4)
+    return launch_pdl(dispatch_mxfp8_kernel<SL, 4>, blocks, kWarps * 32, 0, stream, x, N, H, k, token_slot,
+                      num_rows, recv_x, recv_e8m0, ld, d_status);
+  if (spw == 2)
     return launch_pdl(dispatch_mxfp8_kernel<SL, 2>, blocks, kWarps * 32, 0, stream, x, N, H, k, token_slot,
                       num_rows, recv_x, recv_e8m0, ld, d_status);
   return launch_pdl(dispatch_mxfp8_kernel<SL, 1>, blocks, kWarps * 32, 0, stream, x, N, H, k, token_slot,
@@ -673,8 +682,7 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   if (dtype == MOE_DTYPE_FP8_E4M3 || dtype == MOE_DTYPE_MXFP8_E4M3 || dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
     float* f32 = static_cast<float*>(recv_scale);
     uint8_t* e8 = static_cast<uint8_t*>(recv_scale);
-    // two segments per warp when k <= 4 (reads of x dominate), else one
-    const bool two = k <= 4;
+    const int two = segments_per_warp(k);
     if (dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
         return launch_fp8<MOE_SCALE_MN_MAJOR, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
@@ -718,9 +726,12 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
                       token_slot, num_rows, r8, sc, d_status);
   } else if (dtype == MOE_DTYPE_E5M6) {
     const int segs = (H + 511) / 512;
-    const int spw = k <= 4 ? 2 : 1;  // as the FP8 kernels
+    const int spw = segments_per_warp(k);  // as the FP8 kernels
     const long long items = static_cast<long long>(N) * ((segs + spw - 1) / spw);
     const unsigned blocks = static_cast<unsigned>((items + kWarps - 1) / kWarps);
+    if (spw == 4)
+      return launch_pdl(dispatch_e5m6_kernel<4>, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
+                        num_rows, r8, d_status);
     if (spw == 2)
       return launch_pdl(dispatch_e5m6_kernel<2>, blocks, kWarps * 32, 0, stream, xs, N, H, k, token_slot,
                         num_rows, r8, d_status);
