@@ -340,6 +340,11 @@ cudaError_t launch_bulk(const void* y, int N, int H, int k, const int32_t* token
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(L.total));
   if (err != cudaSuccess) return err;
+  // keep the shared-memory side of the L1/shared split large enough for the
+  // CTAs per SM the stage budget is sized for
+  err = cudaFuncSetAttribute(combine_bulk_kernel<KT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
   int dev = 0, sms = 0, per_sm = 0;
   if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
   if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)

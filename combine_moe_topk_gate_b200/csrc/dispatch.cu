@@ -678,18 +678,42 @@ __global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
     uint32_t phase = 0;
     long long issued = 0;
     bool ok = true;
+    // a group's slot ids (nt * k <= 4 * 32), lane q holding entries q, q + 32,
+    // ...; the next group's are loaded one group ahead, so the load latency
+    // stays off the path of the copies
+    constexpr int kSlotRegs = kRingTokens * MOE_MAX_TOPK / 32;
+    int cur[kSlotRegs], nxt[kSlotRegs];
+    int cur_g = -1;
+    auto load_group = [&](int g, int (&dst)[kSlotRegs]) {
+      const long long base = static_cast<long long>(g) * kRingTokens * k;
+      const long long lim = static_cast<long long>(N) * k;
+#pragma unroll
+      for (int i = 0; i < kSlotRegs; ++i) {
+        const long long q = base + lane + 32 * i;
+        dst[i] = (lane + 32 * i < kRingTokens * k && q < lim) ? token_slot[q] : -1;
+      }
+    };
+    if (i0 < i1) load_group(static_cast<int>(i0 / segs), nxt);
     for (long long it = i0; it < i1; ++it) {
       const int g = static_cast<int>(it / segs);
       const int s = static_cast<int>(it - static_cast<long long>(g) * segs);
       const int t0 = g * kRingTokens;
       const int nt = N - t0 < kRingTokens ? N - t0 : kRingTokens;
+      if (g != cur_g) {
+        cur_g = g;
+#pragma unroll
+        for (int i = 0; i < kSlotRegs; ++i) cur[i] = nxt[i];
+        if (g + 1 < groups) load_group(g + 1, nxt);
+      }
       if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
         report_timeout(d_status);
         ok = false;
         break;
       }
       int32_t* hdr = hdr0 + stage * (kRingHeader / 4);
-      for (int q = lane; q < nt * k; q += 32) hdr[q] = token_slot[static_cast<size_t>(t0) * k + q];
+#pragma unroll
+      for (int i = 0; i < kSlotRegs; ++i)
+        if (lane + 32 * i < nt * k) hdr[lane + 32 * i] = cur[i];
       const int seg_ch = H - s * kRingSeg < kRingSeg ? H - s * kRingSeg : kRingSeg;
       const uint32_t row_bytes = static_cast<uint32_t>(seg_ch) * 2u;
       __syncwarp();
@@ -796,12 +820,24 @@ template <int SL, bool UE8M0>
 cudaError_t launch_fp8_ring(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                             long long num_rows, uint8_t* recv_x, void* recv_scale, long long ld,
                             int32_t* d_status, cudaStream_t stream) {
-  cudaError_t err = cudaFuncSetAttribute(dispatch_fp8_ring_kernel<SL, UE8M0>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kRingSmem));
+  auto kernel = dispatch_fp8_ring_kernel<SL, UE8M0>;
+  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kRingSmem));
   if (err != cudaSuccess) return err;
+  // the ring needs the shared-memory side of the L1/shared split to keep
+  // kRingCtasPerSm CTAs resident on every SM
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (err != cudaSuccess) return err;
+  int dev = 0, sms = 0, per_sm = 0;
+  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRingThreads, kRingSmem)) != cudaSuccess)
+    return err;
+  if (per_sm < 1) per_sm = 1;
   const long long groups = (N + kRingTokens - 1) / kRingTokens;
   const long long items = groups * ((H + kRingSeg - 1) / kRingSeg);
-  const long long slots = 148ll * kRingCtasPerSm;
+  const long long slots = static_cast<long long>(sms) * per_sm;
   const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
   return launch_pdl(dispatch_fp8_ring_kernel<SL, UE8M0>, grid, kRingThreads, kRingSmem, stream, x, N, H, k,
                     token_slot, num_rows, recv_x, recv_scale, ld, d_status);
@@ -818,6 +854,14 @@ __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
     out[2 * i] = static_cast<uint8_t>(v & 0xff);
     if (2 * i + 1 < n) out[2 * i + 1] = static_cast<uint8_t>(v >> 8);
   }
+}
+
+// The CTA-per-token kernels keep the token's row in shared memory; many CTAs
+// per SM need the shared-memory side of the L1/shared split at its largest.
+template <typename K>
+cudaError_t prefer_shared(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              cudaSharedmemCarveoutMaxShared);
 }
 
 // Segments per warp: reading x is most of the traffic when k is small, and
@@ -910,6 +954,11 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     const int vpt = (H / 8 + kTokenThreads - 1) / kTokenThreads;
     float* sc = static_cast<float*>(recv_scale);
     const size_t smem = 128 + static_cast<size_t>(H) * 2;
+    cudaError_t err = vpt <= 2 ? prefer_shared(dispatch_fp8_token_kernel<2>)
+                    : vpt <= 4 ? prefer_shared(dispatch_fp8_token_kernel<4>)
+                    : vpt <= 8 ? prefer_shared(dispatch_fp8_token_kernel<8>)
+                               : prefer_shared(dispatch_fp8_token_kernel<16>);
+    if (err != cudaSuccess) return err;
     if (vpt <= 2)
       return launch_pdl(dispatch_fp8_token_kernel<2>, N, kTokenThreads, smem, stream, xs, N, H, k,
                         token_slot, num_rows, r8, sc, d_status);
@@ -948,6 +997,8 @@ cudaError_t launch_nvfp4_bpt(const uint16_t* x, int N, int H, int k, const int32
                              long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
                              float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
   const size_t smem = 128 + static_cast<size_t>(H) * 2;  // H <= 16384: at most 32 KB + 128
+  cudaError_t err = prefer_shared(dispatch_nvfp4_kernel<BPT, SL>);
+  if (err != cudaSuccess) return err;
   return launch_pdl(dispatch_nvfp4_kernel<BPT, SL>, N, kNvThreads, smem, stream, x, N, H, k,
                     token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
 }

@@ -323,8 +323,12 @@ __global__ void __launch_bounds__(kLayoutThreads)
   __syncthreads();
   if (!last_cta) return;
   __threadfence();
-  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
-                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  if (N <= kMaskMaxTokens)  // the gate names distinct experts per token: bitmask ranks
+    layout_mask_body(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
+                     rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  else
+    layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                              rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
   if (threadIdx.x == 0) *done = 0u;
 }
 
@@ -585,7 +589,9 @@ cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, in
                                  cudaStream_t stream) {
   const char* pf = static_cast<const char*>(o.prefetch);
   constexpr int E = 32 * V;
-  const size_t words = layout_single_smem_words(E, R);
+  size_t words = layout_single_smem_words(E, R);
+  const size_t mask_words = layout_mask_smem_words(E, R, N);
+  if (N <= kMaskMaxTokens && mask_words > words) words = mask_words;
   const size_t smem = (words > static_cast<size_t>(kLayoutWarps) * E ? words : static_cast<size_t>(kLayoutWarps) * E) *
                       sizeof(int32_t);
   if (smem > 48 * 1024) {
