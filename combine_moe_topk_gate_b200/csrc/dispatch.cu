@@ -926,20 +926,20 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
     const int two = segments_per_warp(k);
     if (dtype == MOE_DTYPE_FP8_E4M3_UE8M0) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
-        return launch_fp8_ring<MOE_SCALE_MN_MAJOR, true>(xs, N, H, k, token_slot, num_rows, r8, e8, ld,
-                                                         d_status, stream);
+        return launch_fp8<MOE_SCALE_MN_MAJOR, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                    d_status, stream);
       if (scale_layout == MOE_SCALE_MN_MAJOR_PACK4)
         return launch_fp8<MOE_SCALE_MN_MAJOR_PACK4, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32,
                                                           (num_rows + 3) / 4 * 4, d_status, stream);
-      return launch_fp8_ring<MOE_SCALE_ROW_MAJOR, true>(xs, N, H, k, token_slot, num_rows, r8, e8, ld,
-                                                        d_status, stream);
+      return launch_fp8<MOE_SCALE_ROW_MAJOR, true>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                   d_status, stream);
     }
     if (dtype == MOE_DTYPE_FP8_E4M3) {
       if (scale_layout == MOE_SCALE_MN_MAJOR)
-        return launch_fp8_ring<MOE_SCALE_MN_MAJOR, false>(xs, N, H, k, token_slot, num_rows, r8, f32, ld,
-                                                          d_status, stream);
-      return launch_fp8_ring<MOE_SCALE_ROW_MAJOR, false>(xs, N, H, k, token_slot, num_rows, r8, f32, ld,
-                                                         d_status, stream);
+        return launch_fp8<MOE_SCALE_MN_MAJOR, false>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                     d_status, stream);
+      return launch_fp8<MOE_SCALE_ROW_MAJOR, false>(two, xs, N, H, k, token_slot, num_rows, r8, f32, ld,
+                                                    d_status, stream);
     }
     if (scale_layout == MOE_SCALE_MN_MAJOR)
       return launch_mx<MOE_SCALE_MN_MAJOR>(two, xs, N, H, k, token_slot, num_rows, r8, e8, ld, d_status,

@@ -238,7 +238,7 @@ __device__ __forceinline__ void layout_mask_body(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ne = N * k;
   const int epr = E / R;
-  for (int i = tid; i < (E + R) * W; i += kLayoutThreads) emask[i] = 0u;
+  for (int i = tid; i < E * W; i += kLayoutThreads) emask[i] = 0u;
   __syncthreads();
   int e = -1, t = 0;
   bool valid = false;
@@ -247,14 +247,19 @@ __device__ __forceinline__ void layout_mask_body(
     t = tid / k;
     valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
     if (!valid && e != -1) report_bad_index(d_status);
-    if (valid) {
-      atomicOr(&emask[e * W + (t >> 5)], 1u << (t & 31));
-      atomicOr(&rmask[(e / epr) * W + (t >> 5)], 1u << (t & 31));
-    }
+    if (valid) atomicOr(&emask[e * W + (t >> 5)], 1u << (t & 31));
   }
   const bool masked = tid < ne && !valid;
   const unsigned mb = __ballot_sync(kFullMask, masked);
   if (lane == 0) wmasked[warp] = __popc(mb);
+  __syncthreads();
+  // tokens of each rank: the OR of its experts' masks (no contended atomics)
+  for (int i = tid; i < R * W; i += kLayoutThreads) {
+    const int r = i / W, w = i - r * W;
+    uint32_t m = 0u;
+    for (int ee = r * epr; ee < (r + 1) * epr; ++ee) m |= emask[ee * W + w];
+    rmask[i] = m;
+  }
   __syncthreads();
   // per-bucket totals: experts from their masks, the tail from the warps
   for (int b = tid; b < nb; b += kLayoutThreads) {
