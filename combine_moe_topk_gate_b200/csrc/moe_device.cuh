@@ -23,8 +23,10 @@ constexpr unsigned kFullMask = 0xffffffffu;
 // e^y = 2^n * e^r, n = nearest integer to y*log2(e), r = y - n*ln2 removed in
 // two fused steps (ln2 = head + tail, head = floor(ln2 * 2^16) / 2^16 so that
 // n*head is exact), e^r by its Taylor series to r^7/7! (Horner), 2^n built
-// from the exponent field.  y is clamped to [-87, 88] so 2^n stays normal
-// (by comparisons, so that every NaN, quiet or signalling, becomes -87).
+// from the exponent field.  y is clamped to [-87, 88] so 2^n stays normal;
+// the hardware max returns its other operand for any NaN, quiet or
+// signalling, so every NaN becomes -87 (as the definition's comparisons do;
+// checked on all 2^32 patterns).
 // The nearest integer (ties to even) comes from adding 1.5 * 2^23: the sum's
 // unit in the last place is 1, so the addition itself rounds y*log2(e) to an
 // integer, which then sits in the low mantissa bits (|y*log2(e)| <= 127).
@@ -36,8 +38,7 @@ __device__ __forceinline__ float fixed_exp(float y) {
   constexpr float kInv120 = 1.0f / 120.0f, kInv720 = 1.0f / 720.0f;
   constexpr float kInv5040 = 1.0f / 5040.0f;
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  y = y > -87.0f ? y : -87.0f;  // a NaN input fails the test and becomes -87
-  y = y < 88.0f ? y : 88.0f;
+  y = fminf(fmaxf(y, -87.0f), 88.0f);  // the GPU's max returns -87 for every NaN
   const float t = __fadd_rn(__fmul_rn(y, kLog2e), kRound);
   const float n = __fsub_rn(t, kRound);
   float r = __fmaf_rn(-n, kLn2Head, y);
@@ -50,7 +51,9 @@ __device__ __forceinline__ float fixed_exp(float y) {
   p = __fmaf_rn(p, r, kInv2);
   p = __fmaf_rn(p, r, 1.0f);
   p = __fmaf_rn(p, r, 1.0f);
-  const float two_n = __int_as_float((__float_as_int(t) - 0x4B400000 + 127) << 23);
+  // t's bits are 0x4B400000 + n, whose low 9 bits shifted up by 23 are n's
+  // exponent field; one multiply-add builds 2^n = (n + 127) << 23
+  const float two_n = __uint_as_float((__float_as_uint(t) << 23) + 0x3F800000u);
   return __fmul_rn(p, two_n);
 }
 
