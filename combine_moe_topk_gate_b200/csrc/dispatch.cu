@@ -610,239 +610,6 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
-// ------------------------------------------------------------------ pipelined FP8 dispatch
-// Persistent, warp-specialised CTAs, the combine pipeline turned around.
-// Work item = (group of kRingTokens consecutive tokens, 2048-channel
-// segment).  Each CTA walks a contiguous range of items.
-//   producer warp: per item, waits for a free stage of a shared-memory ring,
-//     writes the group's receive slots into the stage header and issues one
-//     1-D bulk copy (cp.async.bulk global -> shared, no tensor map, no
-//     multicast) per token row segment, completing on the stage's "full"
-//     mbarrier -- many KB of x in flight per SM, independent of how long the
-//     consumers take to quantise and store.
-//   8 consumer warps: per item, wait for "full"; each thread quantises its 8
-//     channels of every staged token (amax over the 16 threads of a
-//     128-channel block by shuffles, the same scale rules as the warp kernel)
-//     and stores 8 code bytes to each of the token's k receive rows plus the
-//     block scale; each warp then releases the stage through "empty".
-// Every wait is bounded (1 s, then MOE_ERR_TIMEOUT).
-constexpr int kRingSeg = 2048;                 // channels per staged row segment
-constexpr int kRingConsumerWarps = 8;          // 256 threads x 8 channels = kRingSeg
-constexpr int kRingThreads = (kRingConsumerWarps + 1) * 32;
-constexpr int kRingTokens = 4;                 // token rows per stage
-constexpr int kRingStages = 6;                 // stages per CTA
-constexpr int kRingRowBytes = kRingSeg * 2;
-constexpr int kRingHeader = kRingTokens * MOE_MAX_TOPK * 4;  // slot ids of the stage's tokens
-constexpr size_t kRingSmem = 128 + static_cast<size_t>(kRingStages) * (kRingHeader + kRingTokens * kRingRowBytes);
-constexpr int kRingCtasPerSm = 2;
-
-__device__ __forceinline__ void st_stream_v2(void* p, uint2 v) {
-  asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
-}
-
-template <int SL, bool UE8M0>
-__global__ void __launch_bounds__(kRingThreads, kRingCtasPerSm)
-    dispatch_fp8_ring_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
-                             const int32_t* __restrict__ token_slot, long long S,
-                             uint8_t* __restrict__ recv_x, void* __restrict__ recv_scale, long long ld,
-                             int32_t* d_status) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t bars = smem_addr(smem);  // full[s] at bars + 8s, empty[s] at bars + 64 + 8s
-  auto full_bar = [&](int st) { return bars + 8u * st; };
-  auto empty_bar = [&](int st) { return bars + 64u + 8u * st; };
-  int32_t* hdr0 = reinterpret_cast<int32_t*>(smem + 128);
-  const uint32_t data = smem_addr(smem + 128 + kRingStages * kRingHeader);
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < kRingStages; ++st) {
-      mbar_init(full_bar(st), 1);
-      mbar_init(empty_bar(st), kRingConsumerWarps);
-    }
-    mbar_init_fence();
-  }
-  __syncthreads();
-  pdl_wait();  // everything above touched shared memory only
-  pdl_trigger();
-
-  const int nblk = H / 128;
-  const int groups = (N + kRingTokens - 1) / kRingTokens;
-  const int segs = (H + kRingSeg - 1) / kRingSeg;
-  const long long items = static_cast<long long>(groups) * segs;
-  const long long per = (items + gridDim.x - 1) / gridDim.x;
-  const long long i0 = static_cast<long long>(blockIdx.x) * per;
-  const long long i1 = i0 + per < items ? i0 + per : items;
-
-  if (warp == kRingConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    int stage = 0;
-    uint32_t phase = 0;
-    long long issued = 0;
-    bool ok = true;
-    // a group's slot ids (nt * k <= 4 * 32), lane q holding entries q, q + 32,
-    // ...; the next group's are loaded one group ahead, so the load latency
-    // stays off the path of the copies
-    constexpr int kSlotRegs = kRingTokens * MOE_MAX_TOPK / 32;
-    int cur[kSlotRegs], nxt[kSlotRegs];
-    int cur_g = -1;
-    auto load_group = [&](int g, int (&dst)[kSlotRegs]) {
-      const long long base = static_cast<long long>(g) * kRingTokens * k;
-      const long long lim = static_cast<long long>(N) * k;
-#pragma unroll
-      for (int i = 0; i < kSlotRegs; ++i) {
-        const long long q = base + lane + 32 * i;
-        dst[i] = (lane + 32 * i < kRingTokens * k && q < lim) ? token_slot[q] : -1;
-      }
-    };
-    if (i0 < i1) load_group(static_cast<int>(i0 / segs), nxt);
-    for (long long it = i0; it < i1; ++it) {
-      const int g = static_cast<int>(it / segs);
-      const int s = static_cast<int>(it - static_cast<long long>(g) * segs);
-      const int t0 = g * kRingTokens;
-      const int nt = N - t0 < kRingTokens ? N - t0 : kRingTokens;
-      if (g != cur_g) {
-        cur_g = g;
-#pragma unroll
-        for (int i = 0; i < kSlotRegs; ++i) cur[i] = nxt[i];
-        if (g + 1 < groups) load_group(g + 1, nxt);
-      }
-      if (!mbar_wait(empty_bar(stage), phase ^ 1u)) {
-        report_timeout(d_status);
-        ok = false;
-        break;
-      }
-      int32_t* hdr = hdr0 + stage * (kRingHeader / 4);
-#pragma unroll
-      for (int i = 0; i < kSlotRegs; ++i)
-        if (lane + 32 * i < nt * k) hdr[lane + 32 * i] = cur[i];
-      const int seg_ch = H - s * kRingSeg < kRingSeg ? H - s * kRingSeg : kRingSeg;
-      const uint32_t row_bytes = static_cast<uint32_t>(seg_ch) * 2u;
-      __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), static_cast<uint32_t>(nt) * row_bytes);
-      __syncwarp();
-      if (lane < nt)
-        bulk_g2s(data + static_cast<uint32_t>(stage * kRingTokens + lane) * kRingRowBytes,
-                 x + static_cast<size_t>(t0 + lane) * H + static_cast<size_t>(s) * kRingSeg, row_bytes,
-                 full_bar(stage));
-      ++issued;
-      if (++stage == kRingStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-    if (!ok) {
-      // let the copies already issued land before the CTA may exit
-      const long long n = issued < kRingStages ? issued : kRingStages;
-      for (long long q = issued - n; q < issued; ++q)
-        mbar_wait(full_bar(static_cast<int>(q % kRingStages)), static_cast<uint32_t>((q / kRingStages) & 1));
-    }
-  } else {
-    // ------------------------------------------------------------ consumers
-    int stage = 0;
-    uint32_t phase = 0;
-    const int c = threadIdx.x * 8;  // this thread's 8 channels of the segment
-    for (long long it = i0; it < i1; ++it) {
-      const int g = static_cast<int>(it / segs);
-      const int s = static_cast<int>(it - static_cast<long long>(g) * segs);
-      const int t0 = g * kRingTokens;
-      const int nt = N - t0 < kRingTokens ? N - t0 : kRingTokens;
-      if (!mbar_wait(full_bar(stage), phase)) {
-        report_timeout(d_status);
-        break;
-      }
-      const int seg_ch = H - s * kRingSeg < kRingSeg ? H - s * kRingSeg : kRingSeg;
-      const bool active = c < seg_ch;  // seg_ch % 128 == 0: whole 16-thread blocks are in or out
-      const int col = s * kRingSeg + c;
-      const int32_t* hdr = hdr0 + stage * (kRingHeader / 4);
-      for (int u = 0; u < nt; ++u) {
-        // every thread takes part in the shuffles; the inactive ones read
-        // stale bytes of the stage and store nothing
-        const uint4 v = ld_shared_v4(data + static_cast<uint32_t>(stage * kRingTokens + u) * kRingRowBytes + c * 2);
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        float f[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          f[2 * i] = bf16_lo(w[i]);
-          f[2 * i + 1] = bf16_hi(w[i]);
-        }
-        float amax = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-#pragma unroll
-        for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
-        float inv, scale = 0.0f;
-        uint32_t ebyte = 0;
-        if constexpr (UE8M0) {
-          int e = amax > 0.0f ? ceil_log2_pos(__fdiv_rn(amax, 448.0f)) : -127;
-          e = e < -127 ? -127 : (e > 127 ? 127 : e);
-          inv = __int_as_float((127 - e) << 23);  // 2^-e; e <= 120 for bf16 input
-          ebyte = static_cast<uint32_t>(e + 127);
-        } else {
-          inv = __fdiv_rn(448.0f, amax);
-          scale = __fdiv_rn(amax, 448.0f);
-        }
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = (UE8M0 || f[i] != 0.0f) ? __fmul_rn(f[i], inv) : f[i];  // zero keeps its sign
-        const uint2 q = make_uint2(e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16),
-                                   e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16));
-        if (!active) continue;
-        for (int j = 0; j < k; ++j) {
-          const int slot = hdr[u * k + j];
-          if (slot == -1) continue;
-          if (slot < -1 || slot >= S) {
-            if ((threadIdx.x & 15) == 0 && c == 0) report_bad_index(d_status);
-            continue;
-          }
-          st_stream_v2(recv_x + static_cast<size_t>(slot) * H + col, q);
-          if ((lane & 15) == 0) {
-            if constexpr (UE8M0) {
-              static_cast<uint8_t*>(recv_scale)[scale_at<SL>(slot, col >> 7, nblk, ld)] = static_cast<uint8_t>(ebyte);
-            } else if constexpr (SL == MOE_SCALE_ROW_MAJOR) {
-              static_cast<float*>(recv_scale)[scale_at<SL>(slot, col >> 7, nblk, ld)] = scale;
-            } else {
-              st_keep_b32(static_cast<float*>(recv_scale) + scale_at<SL>(slot, col >> 7, nblk, ld),
-                          __float_as_uint(scale), l2_evict_last_policy());
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty_bar(stage));
-      if (++stage == kRingStages) {
-        stage = 0;
-        phase ^= 1u;
-      }
-    }
-  }
-}
-
-template <int SL, bool UE8M0>
-cudaError_t launch_fp8_ring(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
-                            long long num_rows, uint8_t* recv_x, void* recv_scale, long long ld,
-                            int32_t* d_status, cudaStream_t stream) {
-  auto kernel = dispatch_fp8_ring_kernel<SL, UE8M0>;
-  cudaError_t err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kRingSmem));
-  if (err != cudaSuccess) return err;
-  // the ring needs the shared-memory side of the L1/shared split to keep
-  // kRingCtasPerSm CTAs resident on every SM
-  err = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-  if (err != cudaSuccess) return err;
-  int dev = 0, sms = 0, per_sm = 0;
-  if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
-  if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
-  if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kRingThreads, kRingSmem)) != cudaSuccess)
-    return err;
-  if (per_sm < 1) per_sm = 1;
-  const long long groups = (N + kRingTokens - 1) / kRingTokens;
-  const long long items = groups * ((H + kRingSeg - 1) / kRingSeg);
-  const long long slots = static_cast<long long>(sms) * per_sm;
-  const unsigned grid = static_cast<unsigned>(items < slots ? items : slots);
-  return launch_pdl(dispatch_fp8_ring_kernel<SL, UE8M0>, grid, kRingThreads, kRingSmem, stream, x, N, H, k,
-                    token_slot, num_rows, recv_x, recv_scale, ld, d_status);
-}
-
 __global__ void e4m3_encode_kernel(const float* __restrict__ in, size_t n,
                                    uint8_t* __restrict__ out) {
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
