@@ -112,4 +112,13 @@ def test_reference_arm_rank0_prints_other_ranks_exit_quietly():
     line = json.loads(outs[0].splitlines()[-1])
     assert line["impl"] == "reference" and line["n_gpus"] == 2 and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["host_cores"] == os.cpu_count()
     assert outs[1] == ""
+    # the comparison arm describes the workload exactly as our arm does
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_cfg", os.path.join(root, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from combine_moe_topk_gate_b200.workloads import WORKLOADS as W
+    assert line["config"] == bench.config_of(W["tiny"], 2)
+    assert line["metric"] == bench.METRIC and line["unit"] == "tokens/s" and line["higher_is_better"] is True
