@@ -130,11 +130,10 @@ def ncu_traffic(op: str, workload: str):
 
 def launches_per_step(w) -> int:
     """Kernels one step launches: routing (one launch when all N*k entries fit
-    one 1024-entry chunk and E = 32, 64, 128 or 256; else the gate and the
-    layout's one or two launches), dispatch, combine."""
-    lanes_gate = w.E % 32 == 0 and (w.E // 32) in (1, 2, 4, 8)
+    one 1024-entry chunk and E <= 512; else the gate and the layout's one or
+    two launches), dispatch, combine."""
     small = w.N * w.k <= 1024
-    route = 1 if small and lanes_gate else (2 if small else 3)
+    route = 1 if small and w.E <= 512 else (2 if small else 3)
     return route + 1 + 1
 
 

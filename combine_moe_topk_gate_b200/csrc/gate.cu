@@ -333,7 +333,121 @@ __global__ void __launch_bounds__(kLayoutThreads)
 }
 
 // ------------------------------------------------------------------ generic kernel
-// Per-warp shared memory: vals[E] (scores or exp terms), gscore[G], gkeep[G].
+// One token by one warp for any E <= 1024: lane l holds experts l, l + 32,
+// ...; per-warp shared memory vals[E] (scores or exp terms), gscore[G],
+// gkeep[G] (group kind) -- wsm points at this warp's E + 2G words.
+template <int V>
+__device__ __forceinline__ void gate_generic_token(const float* __restrict__ logits, int t, int E, int k,
+                                                   int kind, int G, int TG, int topn, float* wsm, int lane,
+                                                   int32_t* __restrict__ topk_idx, float* __restrict__ topk_w) {
+  float* vals = wsm;
+  float* gscore = vals + E;
+  int* gkeep = reinterpret_cast<int*>(gscore + G);
+  const int eg = E / G;
+  const float* row = logits + static_cast<size_t>(t) * E;
+  float l[V];
+  uint64_t key[V];
+#pragma unroll
+  for (int v = 0; v < V; ++v) {
+    const int e = v * 32 + lane;
+    l[v] = e < E ? row[e] : 0.0f;
+  }
+  int sel_i = -1;
+  float sel_v = 0.0f, sum = 0.0f;
+
+  if (kind == MOE_GATE_SIGMOID_GROUP) {
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int e = v * 32 + lane;
+      if (e < E) {
+        const float s = logistic(l[v]);
+        vals[e] = s;
+        key[v] = make_key(s, e);
+      } else {
+        key[v] = 0;
+      }
+    }
+    __syncwarp();
+    // group score: the topn best scores of the group, added best first
+    for (int g = lane; g < G; g += 32) {
+      const float* gv = vals + g * eg;
+      uint64_t prev = ~0ull;
+      float gs = 0.0f;
+      for (int p = 0; p < topn; ++p) {
+        uint64_t best = 0;
+        for (int i = 0; i < eg; ++i) {
+          const uint64_t kv = make_key(gv[i], i);
+          if (kv < prev && kv > best) best = kv;
+        }
+        gs = (p == 0) ? key_value(best) : __fadd_rn(gs, key_value(best));
+        prev = best;
+      }
+      gscore[g] = gs;
+    }
+    __syncwarp();
+    // a group is kept when fewer than TG groups rank before it
+    for (int g = lane; g < G; g += 32) {
+      const uint64_t mine = make_key(gscore[g], g);
+      int before = 0;
+      for (int h = 0; h < G; ++h) before += make_key(gscore[h], h) > mine ? 1 : 0;
+      gkeep[g] = before < TG;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int e = v * 32 + lane;
+      if (e < E && !gkeep[e / eg]) key[v] = 0;
+    }
+    select_topk<V>(key, k, lane, sel_i, sel_v, sum);
+    if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
+  } else {
+    float m = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+      if (v * 32 + lane < E) m = fmaxf(m, l[v]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const int e = v * 32 + lane;
+      if (e < E) {
+        vals[e] = fixed_exp(__fsub_rn(l[v], m));
+        key[v] = make_key(l[v], e);
+      } else {
+        key[v] = 0;
+      }
+    }
+    __syncwarp();
+    float z = 0.0f;
+    if (lane == 0)
+      for (int i = 0; i < E; ++i) z = __fadd_rn(z, vals[i]);
+    z = __shfl_sync(kFullMask, z, 0);
+    uint64_t prev = ~0ull;
+    for (int j = 0; j < k; ++j) {
+      uint64_t best = 0;
+#pragma unroll
+      for (int v = 0; v < V; ++v)
+        if (key[v] < prev && key[v] > best) best = key[v];
+      const uint64_t win = warp_max_key(best);
+      const int wi = key_index(win);
+      // only NaN logits can leave a round without a candidate
+      const float p = (wi >= 0 && wi < E) ? __fdiv_rn(vals[wi], z) : 0.0f;
+      sum = (j == 0) ? p : __fadd_rn(sum, p);
+      if (lane == j) {
+        sel_i = (wi >= 0 && wi < E) ? wi : -1;
+        sel_v = p;
+      }
+      prev = win;
+    }
+    if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
+  }
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
+    topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
+  }
+  __syncwarp();  // the next token reuses this warp's shared memory
+}
+
 template <int V>
 __global__ void __launch_bounds__(kGateWarps * 32)
     topk_gate_generic_kernel(const float* __restrict__ logits, int N, int E, int k, int kind,
@@ -342,118 +456,49 @@ __global__ void __launch_bounds__(kGateWarps * 32)
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  float* vals = smem + warp * (E + 2 * G);
-  float* gscore = vals + E;
-  int* gkeep = reinterpret_cast<int*>(gscore + G);
-  const int eg = E / G;
   pdl_wait();
   pdl_trigger();
   prefetch_share_l2(cc.prefetch, cc.prefetch_bytes);
+  for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps)
+    gate_generic_token<V>(logits, t, E, k, kind, G, TG, topn, smem + warp * (E + 2 * G), lane, topk_idx,
+                          topk_w);
+}
 
-  for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps) {
-    const float* row = logits + static_cast<size_t>(t) * E;
-    float l[V];
-    uint64_t key[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) {
-      const int e = v * 32 + lane;
-      l[v] = e < E ? row[e] : 0.0f;
-    }
-    int sel_i = -1;
-    float sel_v = 0.0f, sum = 0.0f;
-
-    if (kind == MOE_GATE_SIGMOID_GROUP) {
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int e = v * 32 + lane;
-        if (e < E) {
-          const float s = logistic(l[v]);
-          vals[e] = s;
-          key[v] = make_key(s, e);
-        } else {
-          key[v] = 0;
-        }
-      }
-      __syncwarp();
-      // group score: the topn best scores of the group, added best first
-      for (int g = lane; g < G; g += 32) {
-        const float* gv = vals + g * eg;
-        uint64_t prev = ~0ull;
-        float gs = 0.0f;
-        for (int p = 0; p < topn; ++p) {
-          uint64_t best = 0;
-          for (int i = 0; i < eg; ++i) {
-            const uint64_t kv = make_key(gv[i], i);
-            if (kv < prev && kv > best) best = kv;
-          }
-          gs = (p == 0) ? key_value(best) : __fadd_rn(gs, key_value(best));
-          prev = best;
-        }
-        gscore[g] = gs;
-      }
-      __syncwarp();
-      // a group is kept when fewer than TG groups rank before it
-      for (int g = lane; g < G; g += 32) {
-        const uint64_t mine = make_key(gscore[g], g);
-        int before = 0;
-        for (int h = 0; h < G; ++h) before += make_key(gscore[h], h) > mine ? 1 : 0;
-        gkeep[g] = before < TG;
-      }
-      __syncwarp();
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int e = v * 32 + lane;
-        if (e < E && !gkeep[e / eg]) key[v] = 0;
-      }
-      select_topk<V>(key, k, lane, sel_i, sel_v, sum);
-      if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
-    } else {
-      float m = -INFINITY;
-#pragma unroll
-      for (int v = 0; v < V; ++v)
-        if (v * 32 + lane < E) m = fmaxf(m, l[v]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(kFullMask, m, off));
-#pragma unroll
-      for (int v = 0; v < V; ++v) {
-        const int e = v * 32 + lane;
-        if (e < E) {
-          vals[e] = fixed_exp(__fsub_rn(l[v], m));
-          key[v] = make_key(l[v], e);
-        } else {
-          key[v] = 0;
-        }
-      }
-      __syncwarp();
-      float z = 0.0f;
-      if (lane == 0)
-        for (int i = 0; i < E; ++i) z = __fadd_rn(z, vals[i]);
-      z = __shfl_sync(kFullMask, z, 0);
-      uint64_t prev = ~0ull;
-      for (int j = 0; j < k; ++j) {
-        uint64_t best = 0;
-#pragma unroll
-        for (int v = 0; v < V; ++v)
-          if (key[v] < prev && key[v] > best) best = key[v];
-        const uint64_t win = warp_max_key(best);
-        const int wi = key_index(win);
-        // only NaN logits can leave a round without a candidate
-        const float p = (wi >= 0 && wi < E) ? __fdiv_rn(vals[wi], z) : 0.0f;
-        sum = (j == 0) ? p : __fadd_rn(sum, p);
-        if (lane == j) {
-          sel_i = (wi >= 0 && wi < E) ? wi : -1;
-          sel_v = p;
-        }
-        prev = win;
-      }
-      if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
-    }
-    if (lane < k) {
-      topk_idx[static_cast<size_t>(t) * k + lane] = sel_i;
-      topk_w[static_cast<size_t>(t) * k + lane] = sel_v;
-    }
-    __syncwarp();  // the next token reuses this warp's shared memory
-  }
+// One-launch routing for the expert counts the lanes kernel does not take:
+// as route_small_kernel, with the generic gate (shared memory per warp).
+template <int V>
+__global__ void __launch_bounds__(kLayoutThreads)
+    route_small_generic_kernel(const float* __restrict__ logits, int N, int E, int k, int kind, int G,
+                               int TG, int topn, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
+                               int R, int32_t* __restrict__ expert_count, int32_t* __restrict__ expert_offset,
+                               int32_t* __restrict__ rank_count, int32_t* __restrict__ rank_offset,
+                               int32_t* __restrict__ rank_tokens, int32_t* __restrict__ token_slot,
+                               int32_t* __restrict__ slot_token, int align, long long num_rows,
+                               int32_t* d_status, unsigned* done, const char* prefetch,
+                               unsigned long long prefetch_bytes) {
+  extern __shared__ int32_t sm[];
+  __shared__ int last_cta;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait();
+  pdl_trigger();
+  prefetch_share_l2(prefetch, prefetch_bytes);
+  const int t = blockIdx.x * kSmallRouteTokens + warp;
+  if (warp < kSmallRouteTokens && t < N)
+    gate_generic_token<V>(logits, t, E, k, kind, G, TG, topn, reinterpret_cast<float*>(sm) + warp * (E + 2 * G),
+                          lane, topk_idx, topk_w);
+  __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) last_cta = atomicAdd(done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+  if (N <= kMaskMaxTokens)  // the gate names distinct experts per token: bitmask ranks
+    layout_mask_body(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
+                     rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  else
+    layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                              rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 unsigned grid_for(int N) {
@@ -617,6 +662,39 @@ cudaError_t launch_route_small(const float* logits, int N, int k, int kind, cons
   }
 }
 
+template <int V>
+cudaError_t launch_route_small_generic_v(const float* logits, int N, int E, int k, int kind, const GatePlan& p,
+                                         int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
+                                         cudaStream_t stream) {
+  size_t words = layout_single_smem_words(E, R);
+  const size_t mask_words = layout_mask_smem_words(E, R, N);
+  if (N <= kMaskMaxTokens && mask_words > words) words = mask_words;
+  const size_t gate_words = static_cast<size_t>(kSmallRouteTokens) * (E + 2 * p.G);
+  if (gate_words > words) words = gate_words;
+  const size_t smem = words * sizeof(int32_t);
+  if (smem > 48 * 1024) {
+    cudaError_t err = cudaFuncSetAttribute(route_small_generic_kernel<V>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  const unsigned grid = static_cast<unsigned>((N + kSmallRouteTokens - 1) / kSmallRouteTokens);
+  return launch_pdl(route_small_generic_kernel<V>, grid, kLayoutThreads, smem, stream, logits, N, E, k, kind,
+                    p.G, p.TG, p.topn, idx, w, R, o.expert_count, o.expert_offset, o.rank_count, o.rank_offset,
+                    o.rank_tokens, o.token_slot, o.slot_token, o.align, o.num_rows, o.d_status, done,
+                    static_cast<const char*>(o.prefetch), static_cast<unsigned long long>(o.prefetch_bytes));
+}
+
+cudaError_t launch_route_small_generic(const float* logits, int N, int E, int k, int kind, const GatePlan& p,
+                                       int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
+                                       cudaStream_t stream) {
+  const int per_lane = (E + 31) / 32;
+  if (per_lane <= 1) return launch_route_small_generic_v<1>(logits, N, E, k, kind, p, idx, w, R, o, done, stream);
+  if (per_lane <= 2) return launch_route_small_generic_v<2>(logits, N, E, k, kind, p, idx, w, R, o, done, stream);
+  if (per_lane <= 4) return launch_route_small_generic_v<4>(logits, N, E, k, kind, p, idx, w, R, o, done, stream);
+  if (per_lane <= 8) return launch_route_small_generic_v<8>(logits, N, E, k, kind, p, idx, w, R, o, done, stream);
+  return launch_route_small_generic_v<16>(logits, N, E, k, kind, p, idx, w, R, o, done, stream);
+}
+
 }  // namespace
 
 size_t route_workspace_bytes(int N, int k, int E, int R) {
@@ -638,14 +716,16 @@ cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int
         default: return launch_route_small<8>(logits, N, k, kind, p, topk_idx, topk_w, R, o, done, stream);
       }
     }
-    // other expert counts (or no tokens): gate (with the prefetch), then the
-    // one-CTA layout
-    cudaError_t err = cudaSuccess;
+    // other expert counts up to 512: the generic gate in the same one-launch
+    // scheme (beyond 512 its 32 keys per lane do not fit the registers a
+    // 1024-thread CTA leaves, so the gate and the one-CTA layout launch apart)
+    if (N > 0 && E <= 512)
+      return launch_route_small_generic(logits, N, E, k, kind, p, topk_idx, topk_w, R, o, done, stream);
     if (N > 0) {
       const GateExtras pf{static_cast<const char*>(o.prefetch), static_cast<unsigned long long>(o.prefetch_bytes)};
-      err = launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, pf, stream);
+      cudaError_t err = launch_gate(logits, N, E, k, kind, p, topk_idx, topk_w, pf, stream);
+      if (err != cudaSuccess) return err;
     }
-    if (err != cudaSuccess) return err;
     return launch_layout(topk_idx, N, k, E, R, o.align, o.num_rows, o.expert_count, o.expert_offset,
                          o.rank_count, o.rank_offset, o.rank_tokens, o.token_slot, o.slot_token, chunks,
                          o.d_status, stream);

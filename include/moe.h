@@ -242,12 +242,12 @@ size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num
  *              The first 256 bytes hold an arrival counter: zero before the
  *              first call, left zero by every call; the rest is scratch.  Do
  *              not share it between calls whose GPU work overlaps.
- *   How: when N*k <= 1024 and E = 32, 64, 128 or 256 (groups of whole lanes
- *   for the group kind), one launch: each CTA gates 8 tokens and the CTA
- *   that arrives last on the counter builds the layout.  Otherwise the gate
- *   launch and the layout's launches follow each other with programmatic
- *   dependent launch (for large batches three overlapped launches measured
- *   faster than a gate that also counts).
+ *   How: when N*k <= 1024 and E <= 512, one launch: each CTA gates 8 tokens
+ *   and the CTA that arrives last on the counter builds the layout (from
+ *   per-expert token bitmasks when N <= 256).  Otherwise the gate launch and
+ *   the layout's launches follow each other with programmatic dependent
+ *   launch (for large batches three overlapped launches measured faster than
+ *   a gate that also counts).
  *   prefetch   optional device buffer the caller reads next -- typically x,
  *              which moe_dispatch reads right after this call -- and its size
  *              in bytes (NULL / 0: none; 16-byte aligned, a multiple of 16

@@ -56,7 +56,7 @@ def test_dispatch_bytes_per_payload(dtype, row, scale):
 
 def test_launches_per_step():
     bench = _bench()
-    assert bench.launches_per_step(WORKLOADS["tiny"]) == 4      # E = 8: gate, then the one-CTA layout
+    assert bench.launches_per_step(WORKLOADS["tiny"]) == 3      # E = 8: the generic gate, still one launch
     assert bench.launches_per_step(WORKLOADS["decode"]) == 3    # N*k = 1024: still one launch
     assert bench.launches_per_step(WORKLOADS["prefill"]) == 5   # gate, count, assign
 

@@ -1,9 +1,9 @@
 """Routing in one call (moe_route: gate and layout) through the C ABI, against
 the CPU oracle's gate followed by its layout, bit for bit, on the five
 workloads and on the shapes that pick each of its paths: the one-launch path
-(N*k <= 1024 with E = 32*V, the last CTA builds the layout -- from per-expert
-token bitmasks when N <= 256, else from per-warp counts), the gate and layout
-launches for larger batches, and the generic gate for other expert counts.  The arrival counter (the workspace's first 256 bytes) must be zero
+(N*k <= 1024 with E <= 512, lanes or generic gate; the last CTA builds the
+layout -- from per-expert token bitmasks when N <= 256, else from per-warp
+counts), the gate and layout launches for larger batches or more experts.  The arrival counter (the workspace's first 256 bytes) must be zero
 again after every call, so calls in a row on one workspace agree too."""
 import numpy as np
 import pytest
@@ -59,7 +59,8 @@ SHAPES = [
     Workload("small_n300", 300, 64, 64, 2, 8, "softmax_renorm", "bf16", "random"),        # one launch, warp-count ranks
     Workload("e64_group", 700, 64, 64, 6, 8, "sigmoid_group", "fp8", "random", 8, 3, 2),
     Workload("e128_k1", 1000, 64, 128, 1, 4, "softmax_renorm", "bf16", "random"),
-    Workload("e33_small", 100, 64, 33, 5, 3, "softmax", "bf16", "random"),                          # fallback
+    Workload("e33_small", 100, 64, 33, 5, 3, "softmax", "bf16", "random"),                          # generic, one launch
+    Workload("e600_small", 40, 64, 600, 6, 6, "sigmoid_group", "fp8", "random", 12, 4, 2),       # generic, two launches
     Workload("e33_large", 900, 64, 33, 5, 3, "softmax", "bf16", "random"),                          # generic + counts
     Workload("max_E_max_k", 64, 64, 1024, 32, 16, "softmax_renorm", "bf16", "random"),
     Workload("max_E_group", 300, 64, 1024, 32, 32, "sigmoid_group", "fp8", "random", 32, 8, 3),
