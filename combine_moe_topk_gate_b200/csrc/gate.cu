@@ -323,12 +323,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   __syncthreads();
   if (!last_cta) return;
   __threadfence();
-  if (N <= kMaskMaxTokens)  // the gate names distinct experts per token: bitmask ranks
-    layout_mask_body(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
-                     rank_tokens, token_slot, slot_token, align, num_rows, d_status);
-  else
-    layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
-                              rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
   if (threadIdx.x == 0) *done = 0u;
 }
 
@@ -492,12 +488,8 @@ __global__ void __launch_bounds__(kLayoutThreads)
   __syncthreads();
   if (!last_cta) return;
   __threadfence();
-  if (N <= kMaskMaxTokens)  // the gate names distinct experts per token: bitmask ranks
-    layout_mask_body(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
-                     rank_tokens, token_slot, slot_token, align, num_rows, d_status);
-  else
-    layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
-                              rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
   if (threadIdx.x == 0) *done = 0u;
 }
 
@@ -635,8 +627,6 @@ cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, in
   const char* pf = static_cast<const char*>(o.prefetch);
   constexpr int E = 32 * V;
   size_t words = layout_single_smem_words(E, R);
-  const size_t mask_words = layout_mask_smem_words(E, R, N);
-  if (N <= kMaskMaxTokens && mask_words > words) words = mask_words;
   const size_t smem = (words > static_cast<size_t>(kLayoutWarps) * E ? words : static_cast<size_t>(kLayoutWarps) * E) *
                       sizeof(int32_t);
   if (smem > 48 * 1024) {
@@ -667,8 +657,6 @@ cudaError_t launch_route_small_generic_v(const float* logits, int N, int E, int 
                                          int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
                                          cudaStream_t stream) {
   size_t words = layout_single_smem_words(E, R);
-  const size_t mask_words = layout_mask_smem_words(E, R, N);
-  if (N <= kMaskMaxTokens && mask_words > words) words = mask_words;
   const size_t gate_words = static_cast<size_t>(kSmallRouteTokens) * (E + 2 * p.G);
   if (gate_words > words) words = gate_words;
   const size_t smem = words * sizeof(int32_t);

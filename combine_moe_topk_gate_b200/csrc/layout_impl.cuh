@@ -206,106 +206,5 @@ __device__ __forceinline__ void layout_single_body(
   }
 }
 
-// Words of shared memory layout_mask_body needs for E experts, R ranks and
-// N tokens (N <= kMaskMaxTokens).
-constexpr int kMaskMaxTokens = 256;
-__host__ __device__ __forceinline__ size_t layout_mask_smem_words(int E, int R, int N) {
-  const int W = (N + 31) / 32;
-  return static_cast<size_t>(E) * W + static_cast<size_t>(R) * W + 2 * (static_cast<size_t>(E) + 1) + 32 + 32 + 4;
-}
-
-// The layout of N <= kMaskMaxTokens tokens whose k ids come from the gate,
-// so a token never names one expert twice, built by one CTA of
-// kLayoutThreads threads (N*k <= kLayoutThreads).  Every expert keeps the
-// set of its tokens as a bitmask; the row of entry (t, j) in expert e is the
-// number of tokens before t in that set (a popcount of the bits below t),
-// which is the rank in (token, slot) order because t has only one entry in
-// e.  Masked and invalid ids go to the tail bucket in flat order.  The
-// entries were written by other CTAs of this grid and made visible by the
-// caller's fence; they are read from L2 (ld.global.cg).
-__device__ __forceinline__ void layout_mask_body(
-    int32_t* sm, const int32_t* topk_idx, int N, int k, int E, int R, int32_t* expert_count,
-    int32_t* expert_offset, int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
-    int32_t* token_slot, int32_t* slot_token, int align, long long num_rows, int32_t* d_status) {
-  const int W = (N + 31) / 32;
-  const int nb = E + 1;
-  uint32_t* emask = reinterpret_cast<uint32_t*>(sm);  // E * W: tokens of each expert
-  uint32_t* rmask = emask + static_cast<size_t>(E) * W;  // R * W: tokens of each rank
-  int32_t* off = reinterpret_cast<int32_t*>(rmask + static_cast<size_t>(R) * W);  // nb
-  int32_t* cnt = off + nb;                                                          // nb
-  int32_t* warp_sums = cnt + nb;                                                    // 32
-  int32_t* wmasked = warp_sums + 32;                                                // 32: masked entries per warp
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int ne = N * k;
-  const int epr = E / R;
-  for (int i = tid; i < E * W; i += kLayoutThreads) emask[i] = 0u;
-  __syncthreads();
-  int e = -1, t = 0;
-  bool valid = false;
-  if (tid < ne) {
-    e = __ldcg(topk_idx + tid);
-    t = tid / k;
-    valid = static_cast<unsigned>(e) < static_cast<unsigned>(E);
-    if (!valid && e != -1) report_bad_index(d_status);
-    if (valid) atomicOr(&emask[e * W + (t >> 5)], 1u << (t & 31));
-  }
-  const bool masked = tid < ne && !valid;
-  const unsigned mb = __ballot_sync(kFullMask, masked);
-  if (lane == 0) wmasked[warp] = __popc(mb);
-  __syncthreads();
-  // tokens of each rank: the OR of its experts' masks (no contended atomics)
-  for (int i = tid; i < R * W; i += kLayoutThreads) {
-    const int r = i / W, w = i - r * W;
-    uint32_t m = 0u;
-    for (int ee = r * epr; ee < (r + 1) * epr; ++ee) m |= emask[ee * W + w];
-    rmask[i] = m;
-  }
-  __syncthreads();
-  // per-bucket totals: experts from their masks, the tail from the warps
-  for (int b = tid; b < nb; b += kLayoutThreads) {
-    int c = 0;
-    if (b < E) {
-      for (int w = 0; w < W; ++w) c += __popc(emask[b * W + w]);
-    } else {
-      for (int w = 0; w < kLayoutWarps; ++w) c += wmasked[w];
-    }
-    off[b] = c;
-  }
-  for (int r = tid; r < R; r += kLayoutThreads) {
-    int c = 0;
-    for (int w = 0; w < W; ++w) c += __popc(rmask[r * W + w]);
-    rank_tokens[r] = c;
-  }
-  __syncthreads();
-  aligned_offsets(off, cnt, nb, align, warp_sums);
-  for (int i = tid; i < E; i += kLayoutThreads) expert_count[i] = cnt[i];
-  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, 0, 1, d_status);
-  for (int i = tid; i <= E; i += kLayoutThreads) expert_offset[i] = off[i];
-  for (int r = tid; r < R; r += kLayoutThreads) {
-    rank_offset[r] = off[r * epr];
-    rank_count[r] = off[(r + 1) * epr] - off[r * epr];
-  }
-  if (tid == 0) rank_offset[R] = off[E];
-  if (tid < ne) {
-    int slot;
-    if (valid) {
-      const uint32_t* m = emask + e * W;
-      int before = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
-      for (int w = 0; w < (t >> 5); ++w) before += __popc(m[w]);
-      slot = off[e] + before;
-    } else {
-      int before = __popc(mb & lanemask_lt());
-      for (int w = 0; w < warp; ++w) before += wmasked[w];
-      slot = off[E] + before;
-    }
-    if (!derived_row_ok(slot, num_rows, d_status)) {
-      token_slot[tid] = -1;
-    } else {
-      token_slot[tid] = valid ? slot : -1;
-      slot_token[slot] = valid ? t : -1;
-    }
-  }
-}
-
 }  // namespace
 }  // namespace moe

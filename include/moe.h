@@ -243,8 +243,8 @@ size_t moe_route_workspace_bytes(int num_tokens, int k, int num_experts, int num
  *              first call, left zero by every call; the rest is scratch.  Do
  *              not share it between calls whose GPU work overlaps.
  *   How: when N*k <= 1024 and E <= 512, one launch: each CTA gates 8 tokens
- *   and the CTA that arrives last on the counter builds the layout (from
- *   per-expert token bitmasks when N <= 256).  Otherwise the gate launch and
+ *   and the CTA that arrives last on the counter builds the layout.
+ *   Otherwise the gate launch and
  *   the layout's launches follow each other with programmatic dependent
  *   launch (for large batches three overlapped launches measured faster than
  *   a gate that also counts).

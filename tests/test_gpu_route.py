@@ -2,8 +2,7 @@
 the CPU oracle's gate followed by its layout, bit for bit, on the five
 workloads and on the shapes that pick each of its paths: the one-launch path
 (N*k <= 1024 with E <= 512, lanes or generic gate; the last CTA builds the
-layout -- from per-expert token bitmasks when N <= 256, else from per-warp
-counts), the gate and layout launches for larger batches or more experts.  The arrival counter (the workspace's first 256 bytes) must be zero
+layout), the gate and layout launches for larger batches or more experts.  The arrival counter (the workspace's first 256 bytes) must be zero
 again after every call, so calls in a row on one workspace agree too."""
 import numpy as np
 import pytest
@@ -55,8 +54,8 @@ SHAPES = [
     Workload("small_path_edge", 128, 64, 256, 8, 8, "sigmoid_group", "fp8", "random", 8, 4, 2),      # N*k = 1024
     Workload("large_path_edge", 129, 64, 256, 8, 8, "sigmoid_group", "fp8", "random", 8, 4, 2),      # 1032
     Workload("one_token", 1, 64, 32, 1, 1, "softmax", "bf16", "random"),
-    Workload("mask_edge_256", 256, 64, 128, 4, 4, "softmax_renorm", "bf16", "random"),   # bitmask ranks, 8 words
-    Workload("small_n300", 300, 64, 64, 2, 8, "softmax_renorm", "bf16", "random"),        # one launch, warp-count ranks
+    Workload("small_n256", 256, 64, 128, 4, 4, "softmax_renorm", "bf16", "random"),
+    Workload("small_n300", 300, 64, 64, 2, 8, "softmax_renorm", "bf16", "random"),
     Workload("e64_group", 700, 64, 64, 6, 8, "sigmoid_group", "fp8", "random", 8, 3, 2),
     Workload("e128_k1", 1000, 64, 128, 1, 4, "softmax_renorm", "bf16", "random"),
     Workload("e33_small", 100, 64, 33, 5, 3, "softmax", "bf16", "random"),                          # generic, one launch
