@@ -122,41 +122,24 @@ __device__ __forceinline__ void sort_desc(uint64_t (&k)[V]) {
   }
 }
 
-// Per-lane lists sorted largest first, kept in the warp's shared column
-// (key v of lane l at sh_key[v * 32 + l]; a lane reads only its own column):
-// a lane offers its head, the warp's largest head wins, and the winning lane
-// moves its head on -- one shared load per round instead of shifting the
-// list through registers.
+// Selection over per-lane lists sorted largest first: a lane offers its head,
+// the warp's largest head wins, and the winning lane pops it.  Lane j
+// receives slot j; every lane gets the slot-order sum of the winners' values.
 template <int V>
-__device__ __forceinline__ uint64_t stash_sorted(const uint64_t (&key)[V], uint64_t* sh_key, int lane) {
-#pragma unroll
-  for (int v = 1; v < V; ++v) sh_key[v * 32 + lane] = key[v];
-  return key[0];
-}
-template <int V>
-__device__ __forceinline__ uint64_t next_head(const uint64_t* sh_key, int lane, int& head, uint64_t offer,
-                                              uint64_t win) {
-  if (win == 0 || offer != win) return offer;
-  ++head;
-  return head < V ? sh_key[head * 32 + lane] : 0;
-}
-
-// Selection rounds over the stashed lists.  Lane j receives slot j; every
-// lane gets the slot-order sum of the winners' values.
-template <int V>
-__device__ __forceinline__ void select_sorted(const uint64_t (&key)[V], uint64_t* sh_key, int k, int lane,
-                                              int& sel_i, float& sel_v, float& sum) {
-  uint64_t offer = stash_sorted<V>(key, sh_key, lane);
-  int head = 0;
+__device__ __forceinline__ void select_sorted(uint64_t (&key)[V], int k, int lane, int& sel_i,
+                                              float& sel_v, float& sum) {
   for (int j = 0; j < k; ++j) {
-    const uint64_t win = warp_max_key(offer);
+    const uint64_t win = warp_max_key(key[0]);
     const float wv = key_value(win);
     sum = (j == 0) ? wv : __fadd_rn(sum, wv);
     if (lane == j) {
       sel_i = key_index(win);
       sel_v = wv;
     }
-    offer = next_head<V>(sh_key, lane, head, offer, win);
+    const bool pop = win != 0 && key[0] == win;
+#pragma unroll
+    for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
+    key[V - 1] = pop ? 0 : key[V - 1];
   }
 }
 
@@ -172,7 +155,7 @@ struct GateExtras {
 template <int V, int TOPN>
 __device__ __forceinline__ void gate_lanes_token(const float* __restrict__ logits, int t, int k,
                                                  int kind, int LPG_log2, int TG, float* sh_exp,
-                                                 uint64_t* sh_key, int lane, int32_t* __restrict__ topk_idx,
+                                                 int lane, int32_t* __restrict__ topk_idx,
                                                  float* __restrict__ topk_w, const GateExtras& cc) {
   constexpr int E = 32 * V;
   constexpr int topn = TOPN;  // group score = sum of the TOPN best scores of a group
@@ -244,7 +227,7 @@ __device__ __forceinline__ void gate_lanes_token(const float* __restrict__ logit
 #pragma unroll
       for (int v = 0; v < V; ++v) key[v] = 0;
     }
-    select_sorted<V>(key, sh_key, k, lane, sel_i, sel_v, sum);
+    select_sorted<V>(key, k, lane, sel_i, sel_v, sum);
     if (lane < k) sel_v = __fdiv_rn(sel_v, sum);
   } else {
     float m = l[0];
@@ -263,10 +246,8 @@ __device__ __forceinline__ void gate_lanes_token(const float* __restrict__ logit
       for (int i = 0; i < E; ++i) z = __fadd_rn(z, sh_exp[i]);
     z = __shfl_sync(kFullMask, z, 0);
     sort_desc<V>(key);
-    uint64_t offer = stash_sorted<V>(key, sh_key, lane);
-    int head = 0;
     for (int j = 0; j < k; ++j) {
-      const uint64_t win = warp_max_key(offer);
+      const uint64_t win = warp_max_key(key[0]);
       const int wi = key_index(win);
       const float p = (wi >= 0 && wi < E) ? __fdiv_rn(sh_exp[wi], z) : 0.0f;
       sum = (j == 0) ? p : __fadd_rn(sum, p);
@@ -274,7 +255,10 @@ __device__ __forceinline__ void gate_lanes_token(const float* __restrict__ logit
         sel_i = (wi >= 0 && wi < E) ? wi : -1;
         sel_v = p;
       }
-      offer = next_head<V>(sh_key, lane, head, offer, win);
+      const bool pop = win != 0 && key[0] == win;
+#pragma unroll
+      for (int v = 0; v + 1 < V; ++v) key[v] = pop ? key[v + 1] : key[v];
+      key[V - 1] = pop ? 0 : key[V - 1];
     }
     if (lane < k && kind == MOE_GATE_SOFTMAX_RENORM) sel_v = __fdiv_rn(sel_v, sum);
     __syncwarp();  // sh_exp is rewritten for the next token
@@ -293,15 +277,13 @@ __global__ void __launch_bounds__(kGateWarps * 32)
                            int TG, int32_t* __restrict__ topk_idx, float* __restrict__ topk_w,
                            GateExtras cc) {
   __shared__ float sh_exp[kGateWarps][32 * V];
-  __shared__ uint64_t sh_key[kGateWarps][32 * V];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   pdl_wait();
   pdl_trigger();
   prefetch_share_l2(cc.prefetch, cc.prefetch_bytes);
   for (int t = blockIdx.x * kGateWarps + warp; t < N; t += gridDim.x * kGateWarps)
-    gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, sh_exp[warp], sh_key[warp], lane, topk_idx,
-                              topk_w, cc);
+    gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, sh_exp[warp], lane, topk_idx, topk_w, cc);
 }
 
 // ------------------------------------------------------------------ fused routing, small batches
@@ -365,8 +347,7 @@ __global__ void __launch_bounds__(kLayoutThreads)
   const GateExtras none{nullptr, 0};
   if (warp < kSmallRouteTokens && t < N)
     gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, reinterpret_cast<float*>(sm) + warp * E,
-                              reinterpret_cast<uint64_t*>(sm + kSmallRouteTokens * E) + warp * E, lane,
-                              topk_idx, topk_w, none);
+                              lane, topk_idx, topk_w, none);
   route_small_layout(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
                      rank_tokens, token_slot, slot_token, align, num_rows, d_status, done, &last_cta);
 }
@@ -675,8 +656,7 @@ cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, in
                                  cudaStream_t stream) {
   const char* pf = static_cast<const char*>(o.prefetch);
   constexpr int E = 32 * V;
-  // gate rows: E floats of exp terms and E 64-bit keys per warp
-  const size_t smem = route_small_smem_words(N, k, E, R, static_cast<size_t>(kSmallRouteTokens) * 3 * E) * sizeof(int32_t);
+  const size_t smem = route_small_smem_words(N, k, E, R, static_cast<size_t>(kSmallRouteTokens) * E) * sizeof(int32_t);
   if (smem > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(route_small_kernel<V, TOPN>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
