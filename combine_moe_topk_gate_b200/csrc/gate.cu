@@ -25,8 +25,6 @@
 //    merges give every lane its group's top-n, summed largest first.
 //  * generic kernel (any E <= 1024): lane l holds experts l, l+32, ...; group
 //    scores come from a per-warp shared-memory scan.
-#include <algorithm>
-
 #include "layout_impl.cuh"
 #include "moe_device.cuh"
 #include "moe_launch.h"
@@ -287,35 +285,6 @@ __global__ void __launch_bounds__(kGateWarps * 32)
 }
 
 // ------------------------------------------------------------------ fused routing, small batches
-// After a routing CTA gated its tokens: rank its chunk (when the split layout
-// applies), publish (fence, then an arrival on the counter), and in the CTA
-// that arrives last finish the layout and put the counter back to zero.
-__device__ __forceinline__ void route_small_layout(
-    int32_t* sm, int32_t* topk_idx, int N, int k, int E, int R, int32_t* expert_count,
-    int32_t* expert_offset, int32_t* rank_count, int32_t* rank_offset, int32_t* rank_tokens,
-    int32_t* token_slot, int32_t* slot_token, int align, long long num_rows, int32_t* d_status,
-    unsigned* done, int* last_cta) {
-  const bool split = route_split_ok(N, k, E);
-  int32_t* ws_hist = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(done) + kRouteCounterBytes);
-  int32_t* ws_rtok = ws_hist + static_cast<size_t>(route_chunks(N)) * (E + 1);
-  __syncthreads();  // the CTA's gate outputs (global) and its shared rows are settled
-  if (split)
-    route_chunk_rank(sm, topk_idx, N, k, E, R, blockIdx.x, ws_hist, ws_rtok, token_slot, d_status);
-  __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
-  __syncthreads();
-  if (threadIdx.x == 0) *last_cta = atomicAdd(done, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!*last_cta) return;
-  __threadfence();
-  if (split)
-    route_split_finish(sm, topk_idx, N, k, E, R, ws_hist, ws_rtok, expert_count, expert_offset, rank_count,
-                       rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
-  else
-    layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
-                              rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
-  if (threadIdx.x == 0) *done = 0u;
-}
-
 // Gate and layout in one launch when every entry fits one layout chunk
 // (N*k <= kLayoutThreads): CTAs of kLayoutThreads threads of which the first
 // kSmallRouteTokens warps gate one token each (as many tokens per SM as the
@@ -348,8 +317,15 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (warp < kSmallRouteTokens && t < N)
     gate_lanes_token<V, TOPN>(logits, t, k, kind, LPG_log2, TG, reinterpret_cast<float*>(sm) + warp * E,
                               lane, topk_idx, topk_w, none);
-  route_small_layout(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
-                     rank_tokens, token_slot, slot_token, align, num_rows, d_status, done, &last_cta);
+  __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) last_cta = atomicAdd(done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 // ------------------------------------------------------------------ generic kernel
@@ -506,8 +482,15 @@ __global__ void __launch_bounds__(kLayoutThreads)
   if (warp < kSmallRouteTokens && t < N)
     gate_generic_token<V>(logits, t, E, k, kind, G, TG, topn, reinterpret_cast<float*>(sm) + warp * (E + 2 * G),
                           lane, topk_idx, topk_w);
-  route_small_layout(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count, rank_offset,
-                     rank_tokens, token_slot, slot_token, align, num_rows, d_status, done, &last_cta);
+  __threadfence();  // this thread's outputs reach device scope before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) last_cta = atomicAdd(done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+  layout_single_body<false>(sm, topk_idx, N, k, E, R, expert_count, expert_offset, rank_count,
+                            rank_offset, rank_tokens, token_slot, slot_token, align, num_rows, d_status);
+  if (threadIdx.x == 0) *done = 0u;
 }
 
 unsigned grid_for(int N) {
@@ -637,26 +620,15 @@ cudaError_t launch_gate(const float* logits, int N, int E, int k, int kind, cons
   return launch_generic<32>(logits, N, E, k, kind, G, TG, topn, topk_idx, topk_w, cc, stream);
 }
 
-// Shared words of a one-launch routing CTA: the gate's rows, then the
-// layout's (split: a chunk's ranks, the last CTA's sums; else the one-CTA body).
-size_t route_small_smem_words(int N, int k, int E, int R, size_t gate_words) {
-  size_t need = gate_words;
-  if (route_split_ok(N, k, E)) {
-    need = std::max(need, route_chunk_smem_words(E, R));
-    need = std::max(need, route_finish_smem_words(N, E));
-  } else {
-    need = std::max(need, layout_single_smem_words(E, R));
-  }
-  return need;
-}
-
 template <int V, int TOPN>
 cudaError_t launch_route_small_n(const float* logits, int N, int k, int kind, int lpg_log2, int TG,
                                  int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
                                  cudaStream_t stream) {
   const char* pf = static_cast<const char*>(o.prefetch);
   constexpr int E = 32 * V;
-  const size_t smem = route_small_smem_words(N, k, E, R, static_cast<size_t>(kSmallRouteTokens) * E) * sizeof(int32_t);
+  size_t words = layout_single_smem_words(E, R);
+  const size_t smem = (words > static_cast<size_t>(kLayoutWarps) * E ? words : static_cast<size_t>(kLayoutWarps) * E) *
+                      sizeof(int32_t);
   if (smem > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(route_small_kernel<V, TOPN>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -684,8 +656,10 @@ template <int V>
 cudaError_t launch_route_small_generic_v(const float* logits, int N, int E, int k, int kind, const GatePlan& p,
                                          int32_t* idx, float* w, int R, const RouteOut& o, unsigned* done,
                                          cudaStream_t stream) {
-  const size_t smem =
-      route_small_smem_words(N, k, E, R, static_cast<size_t>(kSmallRouteTokens) * (E + 2 * p.G)) * sizeof(int32_t);
+  size_t words = layout_single_smem_words(E, R);
+  const size_t gate_words = static_cast<size_t>(kSmallRouteTokens) * (E + 2 * p.G);
+  if (gate_words > words) words = gate_words;
+  const size_t smem = words * sizeof(int32_t);
   if (smem > 48 * 1024) {
     cudaError_t err = cudaFuncSetAttribute(route_small_generic_kernel<V>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -712,9 +686,7 @@ cudaError_t launch_route_small_generic(const float* logits, int N, int E, int k,
 }  // namespace
 
 size_t route_workspace_bytes(int N, int k, int E, int R) {
-  const size_t lay = layout_workspace_bytes(N, k, E, R);
-  const size_t split = (route_split_ws_words(N, E, R) * sizeof(int32_t) + 255) / 256 * 256;
-  return kRouteCounterBytes + (lay > split ? lay : split);
+  return kRouteCounterBytes + layout_workspace_bytes(N, k, E, R);
 }
 
 cudaError_t launch_route(const float* logits, int N, int E, int k, int kind, int n_groups,

@@ -206,154 +206,5 @@ __device__ __forceinline__ void layout_single_body(
   }
 }
 
-// ------------------------------------------------------------------ one-launch routing layout
-// The layout split over the CTAs of a routing launch that each gated
-// kRouteChunkTokens tokens (a chunk).  Every CTA ranks its own chunk's
-// entries (bucket = expert, E for masked / invalid ids) and publishes the
-// chunk's histogram and tokens per rank; the CTA that arrives last only sums
-// the small per-chunk histograms into offsets and places every entry.
-constexpr int kRouteChunkTokens = 8;
-constexpr int kRouteChunkThreads = 256;  // entries of a chunk: kRouteChunkTokens * k <= 256
-constexpr int kRouteMaxChunkWords = 16384;  // chunks x buckets the last CTA keeps in shared memory
-
-__host__ __device__ __forceinline__ int route_chunks(int N) { return (N + kRouteChunkTokens - 1) / kRouteChunkTokens; }
-
-// true when the split layout applies (else the one-CTA body builds it all)
-__host__ __device__ __forceinline__ bool route_split_ok(int N, int k, int E) {
-  return k * kRouteChunkTokens <= kRouteChunkThreads &&
-         static_cast<long long>(route_chunks(N)) * (E + 1) <= kRouteMaxChunkWords;
-}
-
-// Words of workspace (after the arrival counter) the split layout uses.
-__host__ __device__ __forceinline__ size_t route_split_ws_words(int N, int E, int R) {
-  return static_cast<size_t>(route_chunks(N)) * (E + 1 + R);
-}
-
-// Shared words route_chunk_rank needs: wcnt[8][E+1] + ids[256] + rtok[R].
-__host__ __device__ __forceinline__ size_t route_chunk_smem_words(int E, int R) {
-  return static_cast<size_t>(kRouteChunkThreads / 32) * (E + 1) + kRouteChunkThreads + R;
-}
-
-// Per chunk c (this CTA): entry i = (token c*8 + i/k, slot i%k) for i < ne.
-// Writes hist[c][0..E] (entries per bucket), rtok[c][0..R) (tokens with an
-// expert on rank r) and, into token_slot[global entry], the entry's rank
-// among the chunk's entries of its bucket in (token, slot) order.  The ids
-// come from topk_idx (written by this CTA's warps, visible after the
-// caller's __syncthreads).  All threads of the CTA call it.
-__device__ __forceinline__ void route_chunk_rank(int32_t* sm, const int32_t* topk_idx, int N, int k, int E,
-                                                 int R, int c, int32_t* ws_hist, int32_t* ws_rtok,
-                                                 int32_t* token_slot, int32_t* d_status) {
-  const int nb = E + 1;
-  constexpr int W = kRouteChunkThreads / 32;
-  int32_t* wcnt = sm;                    // W * nb
-  int32_t* ids = wcnt + W * nb;          // kRouteChunkThreads
-  int32_t* rtok = ids + kRouteChunkThreads;  // R
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int t0 = c * kRouteChunkTokens;
-  const int nt = N - t0 < kRouteChunkTokens ? N - t0 : kRouteChunkTokens;
-  const int ne = nt * k;
-  const int epr = E / R;
-  for (int i = tid; i < W * nb; i += blockDim.x) wcnt[i] = 0;
-  for (int i = tid; i < R; i += blockDim.x) rtok[i] = 0;
-  int e = -1, b = -1;
-  if (tid < ne) {
-    e = topk_idx[static_cast<size_t>(t0) * k + tid];
-    ids[tid] = e;
-    b = bucket_of(e, E);
-    if (b == E && e != -1) report_bad_index(d_status);
-  }
-  __syncthreads();
-  unsigned same = 0;
-  int in_warp = 0;
-  if (tid < kRouteChunkThreads) {
-    same = warp_match(static_cast<unsigned>(b + 1), 32 - __clz(E + 1));
-    in_warp = __popc(same & lanemask_lt());
-    if (b >= 0 && in_warp == 0) wcnt[warp * nb + b] = __popc(same);
-    if (b >= 0 && b < E) {  // the token's first slot on this rank counts the token
-      const int j = tid % k, r = e / epr;
-      if (first_on_rank(ids + tid - j, j, r * epr, epr)) atomicAdd(&rtok[r], 1);
-    }
-  }
-  __syncthreads();
-  // exclusive prefix over the chunk's warps of every bucket; totals out
-  for (int bb = tid; bb < nb; bb += blockDim.x) {
-    int acc = 0;
-#pragma unroll
-    for (int w = 0; w < W; ++w) {
-      const int v = wcnt[w * nb + bb];
-      wcnt[w * nb + bb] = acc;
-      acc += v;
-    }
-    ws_hist[static_cast<size_t>(c) * nb + bb] = acc;
-  }
-  __syncthreads();
-  if (tid < ne) token_slot[static_cast<size_t>(t0) * k + tid] = wcnt[warp * nb + b] + in_warp;
-  for (int r = tid; r < R; r += blockDim.x) ws_rtok[static_cast<size_t>(c) * R + r] = rtok[r];
-}
-
-// Shared words route_split_finish needs.
-__host__ __device__ __forceinline__ size_t route_finish_smem_words(int N, int E) {
-  return static_cast<size_t>(route_chunks(N)) * (E + 1) + 2 * (static_cast<size_t>(E) + 1) + 32;
-}
-
-// The last CTA (kLayoutThreads threads): per-bucket column prefix over the
-// C chunks, offsets (rows of each expert rounded up to `align`), counts,
-// ranks' sums, then every entry's row = offset + chunk base + rank.  The
-// per-chunk data and the ids come from other CTAs (made visible by their
-// fences before their arrivals) and are read from L2.
-__device__ __forceinline__ void route_split_finish(
-    int32_t* sm, const int32_t* topk_idx, int N, int k, int E, int R, const int32_t* ws_hist,
-    const int32_t* ws_rtok, int32_t* expert_count, int32_t* expert_offset, int32_t* rank_count,
-    int32_t* rank_offset, int32_t* rank_tokens, int32_t* token_slot, int32_t* slot_token, int align,
-    long long num_rows, int32_t* d_status) {
-  const int nb = E + 1, C = route_chunks(N);
-  int32_t* base = sm;                            // C * nb: first rank of chunk c in bucket b
-  int32_t* off = base + static_cast<size_t>(C) * nb;  // nb
-  int32_t* cnt = off + nb;                       // nb
-  int32_t* warp_sums = cnt + nb;                 // 32
-  const int tid = threadIdx.x;
-  const int epr = E / R;
-  for (int bb = tid; bb < nb; bb += blockDim.x) {
-    int acc = 0;
-    for (int c = 0; c < C; ++c) {
-      const int v = __ldcg(ws_hist + static_cast<size_t>(c) * nb + bb);
-      base[c * nb + bb] = acc;
-      acc += v;
-    }
-    off[bb] = acc;
-  }
-  for (int r = tid; r < R; r += blockDim.x) {
-    int acc = 0;
-    for (int c = 0; c < C; ++c) acc += __ldcg(ws_rtok + static_cast<size_t>(c) * R + r);
-    rank_tokens[r] = acc;
-  }
-  __syncthreads();
-  aligned_offsets(off, cnt, nb, align, warp_sums);
-  for (int i = tid; i < E; i += blockDim.x) expert_count[i] = cnt[i];
-  fill_unused_rows(off, cnt, E, align, num_rows, slot_token, 0, 1, d_status);
-  for (int i = tid; i <= E; i += blockDim.x) expert_offset[i] = off[i];
-  for (int r = tid; r < R; r += blockDim.x) {
-    rank_offset[r] = off[r * epr];
-    rank_count[r] = off[(r + 1) * epr] - off[r * epr];
-  }
-  if (tid == 0) rank_offset[R] = off[E];
-  const int ne = N * k;
-  for (int i = tid; i < ne; i += blockDim.x) {
-    const int e = __ldcg(topk_idx + i);
-    const int b = bucket_of(e, E);
-    const int c = (i / k) / kRouteChunkTokens;
-    const int slot = off[b] + base[c * nb + b] + __ldcg(token_slot + i);
-    if (!derived_row_ok(slot, num_rows, d_status)) {
-      token_slot[i] = -1;
-    } else if (b < E) {
-      token_slot[i] = slot;
-      slot_token[slot] = i / k;
-    } else {
-      token_slot[i] = -1;
-      slot_token[slot] = -1;
-    }
-  }
-}
-
 }  // namespace
 }  // namespace moe
