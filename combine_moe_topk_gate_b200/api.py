@@ -87,7 +87,7 @@ def _load() -> ctypes.CDLL:
     L.moe_dispatch_backward.restype = I
     L.moe_combine_backward.argtypes = [P, P, I, I, I, P, I, P, P, P, P, P]
     L.moe_combine_backward.restype = I
-    L.moe_gate_math.argtypes = [ctypes.c_uint32, SZ, P, P, P]
+    L.moe_gate_math.argtypes = [ctypes.c_uint32, SZ, P, P, P, P]
     L.moe_gate_math.restype = I
     L.moe_e4m3_encode.argtypes = [P, SZ, P, P]
     L.moe_e4m3_encode.restype = I
@@ -606,22 +606,24 @@ def moe_e4m3_encode(x: torch.Tensor, *, out=None, stream=None) -> torch.Tensor:
     return out
 
 
-def moe_gate_math(first: int, n: int, *, exp_out=None, sigmoid_out=None, device=None, stream=None):
-    """The gate's exp and sigmoid on the fp32 bit patterns first, first+1, ...,
-    first+n-1 (mod 2^32); returns ``(exp_out, sigmoid_out)``, fp32 [n] each."""
-    dev = exp_out.device if exp_out is not None else (
-        sigmoid_out.device if sigmoid_out is not None else torch.device("cuda", torch.cuda.current_device()))
+def moe_gate_math(first: int, n: int, *, exp_out=None, sigmoid_out=None, silu_out=None, device=None,
+                  stream=None):
+    """The gate's exp and sigmoid and SwiGLU's silu on the fp32 bit patterns
+    first, first+1, ..., first+n-1 (mod 2^32); returns ``(exp_out,
+    sigmoid_out, silu_out)``, fp32 [n] each."""
+    given = [t for t in (exp_out, sigmoid_out, silu_out) if t is not None]
+    dev = given[0].device if given else torch.device("cuda", torch.cuda.current_device())
     if device is not None and torch.device(device) != dev:
         raise ValueError(f"outputs are on {dev}, device is {device}")
-    if exp_out is None:
-        exp_out = torch.empty(n, dtype=torch.float32, device=dev)
-    if sigmoid_out is None:
-        sigmoid_out = torch.empty(n, dtype=torch.float32, device=dev)
-    _need(exp_out, "exp_out", torch.float32, (n,))
-    _need(sigmoid_out, "sigmoid_out", torch.float32, (n,))
-    _launch(_lib.moe_gate_math, "moe_gate_math", (exp_out, sigmoid_out), first & 0xFFFFFFFF, n,
-            _ptr(exp_out), _ptr(sigmoid_out), _stream(stream, dev))
-    return exp_out, sigmoid_out
+    outs = []
+    for name, t in (("exp_out", exp_out), ("sigmoid_out", sigmoid_out), ("silu_out", silu_out)):
+        if t is None:
+            t = torch.empty(n, dtype=torch.float32, device=dev)
+        _need(t, name, torch.float32, (n,))
+        outs.append(t)
+    _launch(_lib.moe_gate_math, "moe_gate_math", tuple(outs), first & 0xFFFFFFFF, n,
+            *(_ptr(t) for t in outs), _stream(stream, dev))
+    return tuple(outs)
 
 
 def moe_abi_version() -> int:

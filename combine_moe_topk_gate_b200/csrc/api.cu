@@ -23,7 +23,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 6; }
+int moe_abi_version(void) { return 7; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -411,11 +411,13 @@ moe_status_t moe_combine_backward(const void* grad_out, const void* y, int num_t
 }
 
 moe_status_t moe_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
-                           moe_stream_t stream) {
+                           float* silu_out, moe_stream_t stream) {
   if (n == 0) return MOE_OK;
-  if ((!exp_out && !sigmoid_out) || !aligned(exp_out, 16) || !aligned(sigmoid_out, 16))
+  if ((!exp_out && !sigmoid_out && !silu_out) || !aligned(exp_out, 16) ||
+      !aligned(sigmoid_out, 16) || !aligned(silu_out, 16))
     return MOE_ERR_INVALID_ARG;
-  return from_cuda(moe::launch_gate_math(first, n, exp_out, sigmoid_out, as_stream(stream)));
+  return from_cuda(
+      moe::launch_gate_math(first, n, exp_out, sigmoid_out, silu_out, as_stream(stream)));
 }
 
 moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream_t stream) {

@@ -541,25 +541,29 @@ int log2_exact(int x) {
 // takes patterns first + 4i .. first + 4i + 3 (mod 2^32) and stores them as
 // one 16-byte vector per output (a shorter run at the end of the range).
 __global__ void gate_math_kernel(uint32_t first, size_t n, float* __restrict__ exp_out,
-                                 float* __restrict__ sig_out) {
+                                 float* __restrict__ sig_out, float* __restrict__ silu_out) {
   const size_t quads = (n + 3) / 4;
   for (size_t q = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; q < quads;
        q += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const size_t i0 = 4 * q;
-    float e[4], s[4];
+    float e[4], s[4], g[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const float x = __uint_as_float(first + static_cast<uint32_t>(i0 + u));
       e[u] = fixed_exp(x);
       s[u] = logistic(x);
+      // the SwiGLU kernels' choice for a lone value
+      g[u] = fabsf(x) <= 87.0f ? silu_in_range(x) : silu_exact(x);
     }
     if (i0 + 4 <= n) {
       if (exp_out) *reinterpret_cast<float4*>(exp_out + i0) = make_float4(e[0], e[1], e[2], e[3]);
       if (sig_out) *reinterpret_cast<float4*>(sig_out + i0) = make_float4(s[0], s[1], s[2], s[3]);
+      if (silu_out) *reinterpret_cast<float4*>(silu_out + i0) = make_float4(g[0], g[1], g[2], g[3]);
     } else {
       for (int u = 0; u < 4 && i0 + u < n; ++u) {
         if (exp_out) exp_out[i0 + u] = e[u];
         if (sig_out) sig_out[i0 + u] = s[u];
+        if (silu_out) silu_out[i0 + u] = g[u];
       }
     }
   }
@@ -568,11 +572,12 @@ __global__ void gate_math_kernel(uint32_t first, size_t n, float* __restrict__ e
 }  // namespace
 
 cudaError_t launch_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
-                             cudaStream_t stream) {
+                             float* silu_out, cudaStream_t stream) {
   if (n == 0) return cudaSuccess;
   size_t blocks = (n + 4 * 256 - 1) / (4 * 256);
   if (blocks > 148 * 16) blocks = 148 * 16;
-  gate_math_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(first, n, exp_out, sigmoid_out);
+  gate_math_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(first, n, exp_out, sigmoid_out,
+                                                                      silu_out);
   return cudaGetLastError();
 }
 

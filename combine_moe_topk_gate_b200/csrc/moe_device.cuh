@@ -30,7 +30,8 @@ constexpr unsigned kFullMask = 0xffffffffu;
 // The nearest integer (ties to even) comes from adding 1.5 * 2^23: the sum's
 // unit in the last place is 1, so the addition itself rounds y*log2(e) to an
 // integer, which then sits in the low mantissa bits (|y*log2(e)| <= 127).
-__device__ __forceinline__ float fixed_exp(float y) {
+// fixed_exp for y already in [-87, 88] (the clamp would leave it unchanged)
+__device__ __forceinline__ float fixed_exp_in_range(float y) {
   constexpr float kLog2e = 1.44269504088896340736f;
   constexpr float kLn2Head = 0.693145751953125f;          // 45426 / 65536
   constexpr float kLn2Tail = 1.42860682030941723212e-6f;  // ln2 - head
@@ -38,7 +39,6 @@ __device__ __forceinline__ float fixed_exp(float y) {
   constexpr float kInv120 = 1.0f / 120.0f, kInv720 = 1.0f / 720.0f;
   constexpr float kInv5040 = 1.0f / 5040.0f;
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  y = fminf(fmaxf(y, -87.0f), 88.0f);  // the GPU's max returns -87 for every NaN
   const float t = __fadd_rn(__fmul_rn(y, kLog2e), kRound);
   const float n = __fsub_rn(t, kRound);
   float r = __fmaf_rn(-n, kLn2Head, y);
@@ -57,10 +57,53 @@ __device__ __forceinline__ float fixed_exp(float y) {
   return __fmul_rn(p, two_n);
 }
 
+__device__ __forceinline__ float fixed_exp(float y) {
+  y = fminf(fmaxf(y, -87.0f), 88.0f);  // the GPU's max returns -87 for every NaN
+  return fixed_exp_in_range(y);
+}
+
 // 1 / (1 + e^-x), each operation rounded once (the correctly rounded
 // reciprocal is the correctly rounded quotient 1 / d).
 __device__ __forceinline__ float logistic(float x) {
   return __frcp_rn(__fadd_rn(1.0f, fixed_exp(-x)));
+}
+
+// ---------------------------------------------------------------- silu
+// silu(g) = g / (1 + e^-g), each operation rounded once, e^-g the fixed exp.
+__device__ __forceinline__ float silu_exact(float g) {
+  return __fdiv_rn(g, __fadd_rn(1.0f, fixed_exp(-g)));
+}
+
+// g / d rounded once, by one correction of the quotient (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990): from y ~ 1/d and q = g*y, the
+// residual r = d*q - g is exact in one fused multiply-add, and q - r*y,
+// rounded once, is the quotient.  r is taken as d*q - g rather than g - d*q
+// so that g = -0 keeps its sign.  Used where d is in [1, 2^126) (y normal,
+// no flush to zero) and g is finite.
+__device__ __forceinline__ float div_corrected(float g, float d) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d));
+  const float q = __fmul_rn(g, y);
+  const float r = __fmaf_rn(d, q, -g);
+  return __fmaf_rn(-r, y, q);
+}
+
+// silu for |g| <= 87: -g is then inside the exp's clamp range and
+// 1 + e^-g <= 1 + e^87 < 2^126, so the clamp is skipped and the division is
+// div_corrected.  Equal to silu_exact on every bf16 g with |g| <= 87, the
+// only inputs the SwiGLU kernels give it (all of them checked on the GPU);
+// on other fp32 inputs one correction from an approximate reciprocal can be
+// one unit in the last place off (the same sweep finds such inputs).
+__device__ __forceinline__ float silu_in_range(float g) {
+  return div_corrected(g, __fadd_rn(1.0f, fixed_exp_in_range(-g)));
+}
+
+// max(m, |g|), NaN if either is NaN
+__device__ __forceinline__ float max_abs_nan(float m, float g) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(m), "f"(fabsf(g)));
+  return r;
 }
 
 // ---------------------------------------------------------------- bf16

@@ -77,7 +77,7 @@ cudaError_t launch_combine_backward(const void* grad_out, const void* y, int N, 
                                     int32_t* d_status, cudaStream_t stream);
 
 cudaError_t launch_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
-                             cudaStream_t stream);
+                             float* silu_out, cudaStream_t stream);
 
 cudaError_t launch_e4m3_encode(const float* in, size_t n, uint8_t* out, cudaStream_t stream);
 

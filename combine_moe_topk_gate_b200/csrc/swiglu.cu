@@ -23,21 +23,36 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kRowThreads = 256;
 
-__device__ __forceinline__ float silu_mul(float g, float u) {
-  const float d = __fadd_rn(1.0f, fixed_exp(-g));
-  return __fmul_rn(__fdiv_rn(g, d), u);
-}
-
-// a for 8 channels from a vector of 8 gate and a vector of 8 up values
+// a for 8 channels from a vector of 8 gate and a vector of 8 up values, on
+// every input
 __device__ __forceinline__ void swiglu8(uint4 gv, uint4 uv, float* a) {
   const uint32_t g4[4] = {gv.x, gv.y, gv.z, gv.w};
   const uint32_t u4[4] = {uv.x, uv.y, uv.z, uv.w};
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    a[2 * i] = silu_mul(bf16_lo(g4[i]), bf16_lo(u4[i]));
-    a[2 * i + 1] = silu_mul(bf16_hi(g4[i]), bf16_hi(u4[i]));
+    a[2 * i] = __fmul_rn(silu_exact(bf16_lo(g4[i])), bf16_lo(u4[i]));
+    a[2 * i + 1] = __fmul_rn(silu_exact(bf16_hi(g4[i])), bf16_hi(u4[i]));
   }
 }
+
+// The same a when every |g| <= 87 (silu_in_range: no clamp, a corrected
+// division); returns max(m, |g| over the 8), NaN if a g is NaN.  The caller
+// redoes the channels with swiglu8 when the maximum is above 87 or NaN, which
+// real activations almost never reach.
+__device__ __forceinline__ float swiglu8_in_range(uint4 gv, uint4 uv, float* a, float m) {
+  const uint32_t g4[4] = {gv.x, gv.y, gv.z, gv.w};
+  const uint32_t u4[4] = {uv.x, uv.y, uv.z, uv.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float g0 = bf16_lo(g4[i]), g1 = bf16_hi(g4[i]);
+    m = max_abs_nan(max_abs_nan(m, g0), g1);
+    a[2 * i] = __fmul_rn(silu_in_range(g0), bf16_lo(u4[i]));
+    a[2 * i + 1] = __fmul_rn(silu_in_range(g1), bf16_hi(u4[i]));
+  }
+  return m;
+}
+
+constexpr float kSiluRange = 87.0f;
 
 // a is never NaN for finite h (silu(g) * u of finite bf16 values), so the
 // encoder without NaN handling gives the same codes
@@ -59,7 +74,7 @@ __device__ __forceinline__ void scale_keep_zero(const float* a, float f, float* 
 }
 
 template <int DT, int SL>
-__global__ void __launch_bounds__(kWarps * 32, 1)  // (..., 1): no register cap, no spill
+__global__ void __launch_bounds__(kWarps * 32, 6)  // 40 registers, no spill: 48 warps per SM
     swiglu_quant_kernel(const uint16_t* __restrict__ h, long long S, int I,
                         const int32_t* __restrict__ slot_token, void* __restrict__ out,
                         void* __restrict__ out_scale, long long ld) {
@@ -76,16 +91,22 @@ __global__ void __launch_bounds__(kWarps * 32, 1)  // (..., 1): no register cap,
 
   float a[16];
   {
+    const uint16_t* hr = h + static_cast<size_t>(row) * 2 * I + c0;
     uint4 g0 = make_uint4(0, 0, 0, 0), g1 = g0, u0 = g0, u1 = g0;
     if (active) {
-      const uint16_t* hr = h + static_cast<size_t>(row) * 2 * I;
-      g0 = ld_stream(hr + c0);
-      g1 = ld_stream(hr + c0 + 8);
-      u0 = ld_stream(hr + I + c0);
-      u1 = ld_stream(hr + I + c0 + 8);
+      g0 = ld_stream(hr);
+      g1 = ld_stream(hr + 8);
+      u0 = ld_stream(hr + I);
+      u1 = ld_stream(hr + I + 8);
     }
-    swiglu8(g0, u0, a);
-    swiglu8(g1, u1, a + 8);
+    float m = swiglu8_in_range(g0, u0, a, 0.0f);
+    m = swiglu8_in_range(g1, u1, a + 8, m);
+    if (!(m <= kSiluRange)) {
+      // rare: the lane reads its 16 channels again (an L2 hit) rather than
+      // keeping them live through the common path
+      swiglu8(ld_stream(hr), ld_stream(hr + I), a);
+      swiglu8(ld_stream(hr + 8), ld_stream(hr + I + 8), a + 8);
+    }
   }
 
   if constexpr (DT == MOE_DTYPE_BF16) {
@@ -106,8 +127,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)  // (..., 1): no register cap,
       amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
       amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
       amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
-      const float inv = __fdiv_rn(448.0f, amax);
-      const float scale = __fdiv_rn(amax, 448.0f);
+      // the block's 448 / amax and amax / 448 from one division per lane:
+      // even lanes take the first, odd lanes the second
+      const bool odd = lane & 1;
+      const float q = __fdiv_rn(odd ? amax : 448.0f, odd ? 448.0f : amax);
+      const float inv = __shfl_sync(kFullMask, q, lane & ~7);
+      const float scale = __shfl_sync(kFullMask, q, (lane & ~7) | 1);
       float p[16];
       scale_keep_zero<16>(a, inv, p);
       if (active) {
@@ -131,18 +156,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1)  // (..., 1): no register cap,
       if constexpr (SL == MOE_SCALE_MN_MAJOR) {
         if (active && (lane & 1) == 0) sc[scale_at<SL>(row, c0 >> 5, nblk, ld)] = static_cast<uint8_t>(my_byte);
       } else {
-        // the warp's 16 block bytes, block i from lane 2i; 4 bytes per word
-        uint32_t sw[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          sw[i] = 0;
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            sw[i] |= (__shfl_sync(kFullMask, my_byte, 2 * (4 * i + u)) & 0xffu) << (8 * u);
-        }
-        const int b0 = seg * 16 + 4 * lane;
-        if (lane < 4 && b0 < nblk) {
-          const uint32_t word = lane == 0 ? sw[0] : lane == 1 ? sw[1] : lane == 2 ? sw[2] : sw[3];
+        // the warp's 16 block bytes (block j from lane 2j) as 4 words, word i
+        // = blocks 4i..4i+3 gathered on lane 8i in two shuffles
+        uint32_t word = my_byte | (__shfl_down_sync(kFullMask, my_byte, 2) << 8);
+        word |= __shfl_down_sync(kFullMask, word, 4) << 16;
+        const int b0 = seg * 16 + (lane >> 1);
+        if ((lane & 7) == 0 && b0 < nblk) {
           if constexpr (SL == MOE_SCALE_MMA_TILED) {
             *reinterpret_cast<uint32_t*>(sc + scale_at<SL>(row, b0, nblk, ld)) = word;
           } else {
@@ -182,7 +201,9 @@ __global__ void __launch_bounds__(kRowThreads, 1)
       gv = ld_stream(hr + static_cast<size_t>(vi) * 8);
       uv = ld_stream(hr + I + static_cast<size_t>(vi) * 8);
     }
-    swiglu8(gv, uv, a[i]);
+    if (!(swiglu8_in_range(gv, uv, a[i], 0.0f) <= kSiluRange))
+      swiglu8(ld_stream(hr + static_cast<size_t>(vi) * 8), ld_stream(hr + I + static_cast<size_t>(vi) * 8),
+              a[i]);
 #pragma unroll
     for (int u = 0; u < 8; ++u) amax = fmaxf(amax, fabsf(a[i][u]));
   }

@@ -507,14 +507,22 @@ moe_status_t moe_e4m3_encode(const float* in, size_t n, uint8_t* out, moe_stream
  *                    polynomial by Horner, input clamped to [-87, 88] by
  *                    comparisons, so every NaN input is taken as -87);
  *   sigmoid_out[i] = 1 / (1 + exp(-x_i)), each operation rounded once, the
- *                    score of the group-limited kind.
+ *                    score of the group-limited kind;
+ *   silu_out[i]    = x_i / (1 + exp(-x_i)) as moe_swiglu_quant computes it
+ *                    from a bf16 gate value: each operation rounded once, for
+ *                    |x_i| <= 87 by that kernel's shortened steps (no clamp,
+ *                    one corrected quotient from an approximate reciprocal),
+ *                    which give the same bits on every bf16-representable
+ *                    x_i and are within one unit in the last place on other
+ *                    fp32 patterns.
  * "DeepSeek, DeepEP 오픈소스 공개", Topic Body: group-limited gating, whose
- * group scores are sums of these sigmoids.  Either output may be NULL (not
- * both); outputs are device fp32 arrays of n elements, 16-byte aligned.
- * n may be 0.
+ * group scores are sums of these sigmoids; DeepSeek Tile-Kernels news,
+ * "Funktionen der DeepSeek-Tile-Kernel": SwiGLU.  Any output may be NULL
+ * (not all three); outputs are device fp32 arrays of n elements, 16-byte
+ * aligned.  n may be 0.
  */
 moe_status_t moe_gate_math(uint32_t first, size_t n, float* exp_out, float* sigmoid_out,
-                           moe_stream_t stream);
+                           float* silu_out, moe_stream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(moe_status_t status);

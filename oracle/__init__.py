@@ -93,7 +93,8 @@ def _declare(L):
     L.oracle_bf16_from_f32.restype = ctypes.c_uint16
     L.oracle_f32_from_bf16.argtypes = [ctypes.c_uint16]
     L.oracle_f32_from_bf16.restype = ctypes.c_float
-    for name in ("oracle_e4m3_encode_array", "oracle_dexp_array", "oracle_sigmoid_array"):
+    for name in ("oracle_e4m3_encode_array", "oracle_dexp_array", "oracle_sigmoid_array",
+                 "oracle_silu_array"):
         getattr(L, name).argtypes = [_P, _P, _SZ]
         getattr(L, name).restype = None
     L.oracle_topk_gate.argtypes = [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P]
@@ -212,6 +213,14 @@ def sigmoid_array(x: np.ndarray) -> np.ndarray:
     x = _c(x, np.float32)
     out = np.empty(x.shape, np.float32)
     lib().oracle_sigmoid_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def silu_array(x: np.ndarray) -> np.ndarray:
+    """silu(g) = g / (1 + dexp(-g)) of SwiGLU, fp32, each operation rounded once."""
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.float32)
+    lib().oracle_silu_array(_ptr(x), _ptr(out), x.size)
     return out
 
 

@@ -971,6 +971,11 @@ static float silu_f32(float g)
     return g / d;
 }
 
+void oracle_silu_array(const float* in, float* out, size_t n)
+{
+    for (size_t i = 0; i < n; ++i) out[i] = silu_f32(in[i]);
+}
+
 /* quantise one fp32 row of n values: codes (or bf16) to out_row, fp32
  * scales to fsc or E8M0 bytes to esc, one per block */
 static void quantize_f32_row(const float* a, int n, int dtype, void* out_row, float* fsc,

@@ -331,10 +331,11 @@ def test_binding_rejects_mixed_devices_and_bad_status_words(api):
 
 def test_gate_math_rejects_bad_arguments(api):
     L = api.lib()
-    assert L.moe_gate_math(0, 0, None, None, None) == api.MOE_OK            # empty run
-    assert L.moe_gate_math(0, 16, None, None, None) == api.MOE_ERR_INVALID_ARG
-    assert L.moe_gate_math(0, 16, 260, None, None) == api.MOE_ERR_INVALID_ARG   # not 16-byte aligned
-    assert L.moe_gate_math(0, 16, None, 264, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_gate_math(0, 0, None, None, None, None) == api.MOE_OK            # empty run
+    assert L.moe_gate_math(0, 16, None, None, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_gate_math(0, 16, 260, None, None, None) == api.MOE_ERR_INVALID_ARG   # not 16-byte aligned
+    assert L.moe_gate_math(0, 16, None, 264, None, None) == api.MOE_ERR_INVALID_ARG
+    assert L.moe_gate_math(0, 16, None, None, 520, None) == api.MOE_ERR_INVALID_ARG
 
 
 def test_route_rejects_bad_arguments(api):

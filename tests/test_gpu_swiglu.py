@@ -25,6 +25,14 @@ def _h(rows, I, seed):
     h[::17, I + 5] = -0.0
     h[::13, 3] = 30.0                                # silu saturates to the identity
     h[::11, I + 9] = 1e4
+    # gate values at and beyond the shortened silu's range (|g| <= 87): the
+    # lanes holding them take the full steps; -0 keeps its sign
+    h[::7, 10] = -0.0
+    h[::19, 11] = -100.0
+    h[::23, 12] = 87.5
+    h[::29, 13] = -87.0
+    h[::31, 14] = 87.0
+    h[::37, 15] = -1e4
     return h.to(torch.bfloat16)
 
 
