@@ -493,9 +493,64 @@ def other_workloads(api, main, device, steps, warmup, flush, peak) -> dict:
         iso.update(isolated_op_times(r.separate_ops, flush, device))
         res[name] = summary_of(w, step_ms, per_op, iso, peak)
         res[name]["quant_fp8_channel"] = channel_fp8_time(api, r, flush, device, peak)
+        if name in ("mixtral", "skewed"):   # top-2 / H = 4096 and the skewed top-8 shape
+            api.moe_route(r.logits, w.k, w.gate_kind, w.n_groups, w.topk_groups, w.group_topn, w.R,
+                          topk_idx=r.idx, topk_w=r.wts, out=r.L)
+            res[name]["dispatch_variants"] = dispatch_variant_times(api, w, r.x, r.L, flush, device)
         del r
         torch.cuda.empty_cache()
     return res
+
+
+def dispatch_variant_times(api, w, x, L, flush, device) -> dict:
+    """Every dispatch payload type on this batch's layout, each alone (cold,
+    clean L2): µs, fraction of the measured copy peak, algorithmic bytes."""
+    from combine_moe_topk_gate_b200.workloads import DTYPES, Workload
+    bufs = {}
+    for dname, code in DTYPES.items():
+        rx = torch.empty((w.S, w.H), dtype=torch.bfloat16 if code == 0 else torch.uint8, device=device)
+        shape, sdt = api.scale_shape(w.S, w.H, code)
+        bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
+    nv = None
+    if w.H % 64 == 0:
+        nv = (torch.empty((w.S, w.H // 2), dtype=torch.uint8, device=device),
+              torch.empty((w.S, w.H // 16), dtype=torch.uint8, device=device),
+              torch.empty((w.S,), dtype=torch.float32, device=device))
+    e5 = torch.empty((w.S, w.H // 2 * 3), dtype=torch.uint8, device=device) if w.H % 32 == 0 else None
+    tiled = None
+    if w.H % 128 == 0:   # MXFP8 with the block-scaled MMA's tiled E8M0 scales
+        shape_t, sdt_t = api.scale_shape(w.S, w.H, api.MOE_DTYPE_MXFP8_E4M3, api.MOE_SCALE_MMA_TILED)
+        if shape_t:
+            tiled = (torch.empty((w.S, w.H), dtype=torch.uint8, device=device),
+                     torch.empty(shape_t, dtype=sdt_t, device=device))
+
+    def var_ops():
+        ops = {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
+                                                             d_status=L.status))
+               for d, (c, rx, rs) in bufs.items()}
+        if nv is not None:
+            ops["nvfp4"] = lambda: api.moe_dispatch_nvfp4(x, L.token_slot, recv_x=nv[0], block_scale=nv[1],
+                                                          row_scale=nv[2], d_status=L.status)
+        if e5 is not None:
+            ops["e5m6"] = lambda: api.moe_dispatch(x, L.token_slot, api.MOE_DTYPE_E5M6, recv_x=e5,
+                                                   d_status=L.status)
+        if tiled is not None:
+            ops["mxfp8_mma_tiled"] = lambda: api.moe_dispatch(
+                x, L.token_slot, api.MOE_DTYPE_MXFP8_E4M3, recv_x=tiled[0], recv_scale=tiled[1],
+                scale_layout=api.MOE_SCALE_MMA_TILED, d_status=L.status)
+        return ops
+    vt = isolated_op_times(var_ops, flush, device)
+    peak_v, _ = measured_peak()
+    variants = {}
+    for d, us in vt.items():
+        abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": "mxfp8" if d == "mxfp8_mma_tiled" else d}))
+        abv = abv["dispatch"]
+        variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
+                       "algorithmic_bytes": abv}
+    torch.cuda.synchronize(device)
+    if int(L.status.item()) != 0:
+        raise RuntimeError(f"device status {int(L.status.item())} after the dispatch variants")
+    return variants
 
 
 def channel_fp8_time(api, r, flush, device, peak, align: int = 128) -> dict:
@@ -513,8 +568,10 @@ def channel_fp8_time(api, r, flush, device, peak, align: int = 128) -> dict:
         device=device).manual_seed(11))
     out = torch.empty((rows, w.H), dtype=torch.uint8, device=device)
     sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+    ws = torch.zeros(api.moe_quant_fp8_channel_workspace_bytes(w.E, w.H), dtype=torch.uint8, device=device)
     us = isolated_op_times(lambda: {"quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
-        y, La.expert_offset, La.expert_count, out=out, scale=sc, d_status=La.status)}, flush, device)
+        y, La.expert_offset, La.expert_count, out=out, scale=sc, workspace=ws, d_status=La.status)}, flush,
+        device)
     us = us["quant_fp8_channel"]
     counts = La.expert_count.cpu()
     landed = int(counts.sum().item())
@@ -585,41 +642,7 @@ def run_ours(args, rank, world, device):
 
         variants = None
         if not args.no_backward:
-            # every dispatch payload type on this shape, each alone (cold, clean L2)
-            from combine_moe_topk_gate_b200.workloads import DTYPES, Workload
-            bufs = {}
-            for dname, code in DTYPES.items():
-                rx = torch.empty((w.S, w.H), dtype=torch.bfloat16 if code == 0 else torch.uint8, device=device)
-                shape, sdt = api.scale_shape(w.S, w.H, code)
-                bufs[dname] = (code, rx, torch.empty(shape, dtype=sdt, device=device) if shape else None)
-
-            nv = None
-            if w.H % 64 == 0:
-                nv = (torch.empty((w.S, w.H // 2), dtype=torch.uint8, device=device),
-                      torch.empty((w.S, w.H // 16), dtype=torch.uint8, device=device),
-                      torch.empty((w.S,), dtype=torch.float32, device=device))
-
-            e5 = torch.empty((w.S, w.H // 2 * 3), dtype=torch.uint8, device=device) if w.H % 32 == 0 else None
-
-            def var_ops():
-                ops = {d: (lambda c=c, rx=rx, rs=rs: api.moe_dispatch(x, L.token_slot, c, recv_x=rx, recv_scale=rs,
-                                                                     d_status=L.status))
-                       for d, (c, rx, rs) in bufs.items()}
-                if nv is not None:
-                    ops["nvfp4"] = lambda: api.moe_dispatch_nvfp4(x, L.token_slot, recv_x=nv[0], block_scale=nv[1],
-                                                                  row_scale=nv[2], d_status=L.status)
-                if e5 is not None:
-                    ops["e5m6"] = lambda: api.moe_dispatch(x, L.token_slot, api.MOE_DTYPE_E5M6, recv_x=e5,
-                                                           d_status=L.status)
-                return ops
-            vt = isolated_op_times(var_ops, flush, device)
-            peak_v, _ = measured_peak()
-            variants = {}
-            for d, us in vt.items():
-                abv = algorithmic_bytes(Workload(**{**w.__dict__, "dtype": d}))["dispatch"]
-                variants[d] = {"us": us, "frac": abv / (us * 1e-6) / 1e9 / peak_v if us else None,
-                               "algorithmic_bytes": abv}
-            del bufs, nv, e5
+            variants = dispatch_variant_times(api, w, x, L, flush, device)
 
         aligned = None
         if not args.no_backward:
@@ -660,11 +683,14 @@ def run_ours(args, rank, world, device):
             # GEMM's operand); y_a doubles as that buffer
             ch_out = torch.empty((rows_a, w.H), dtype=torch.uint8, device=device)
             ch_sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+            ch_ws = torch.zeros(api.moe_quant_fp8_channel_workspace_bytes(w.E, w.H), dtype=torch.uint8,
+                                device=device)
 
             def al_ops():
                 ops = {
                     "quant_fp8_channel": lambda: api.moe_quant_fp8_channel(
-                        y_a, La.expert_offset, La.expert_count, out=ch_out, scale=ch_sc, d_status=La.status),
+                        y_a, La.expert_offset, La.expert_count, out=ch_out, scale=ch_sc, workspace=ch_ws,
+                        d_status=La.status),
                     "swiglu_fp8_mn_major": lambda: api.moe_swiglu_quant(
                         h_a, api.MOE_DTYPE_FP8_E4M3, slot_token=La.slot_token, scale_layout=api.MOE_SCALE_MN_MAJOR,
                         out=sw_out, out_scale=sw_sc),

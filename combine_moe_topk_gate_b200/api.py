@@ -77,7 +77,9 @@ def _load() -> ctypes.CDLL:
     L.moe_dispatch_nvfp4.restype = I
     L.moe_selftest_bounded_wait.argtypes = [P, P]
     L.moe_selftest_bounded_wait.restype = I
-    L.moe_quant_fp8_channel.argtypes = [P, I, I, I, P, P, I, P, P, P, P]
+    L.moe_quant_fp8_channel.argtypes = [P, I, I, I, P, P, I, P, P, P, SZ, P, P]
+    L.moe_quant_fp8_channel_workspace_bytes.argtypes = [I, I]
+    L.moe_quant_fp8_channel_workspace_bytes.restype = SZ
     L.moe_quant_fp8_channel.restype = I
     L.moe_swiglu_quant.argtypes = [P, I, I, P, I, I, P, P, P]
     L.moe_swiglu_quant.restype = I
@@ -478,11 +480,20 @@ def moe_selftest_bounded_wait(d_status: torch.Tensor, stream=None) -> None:
             _stream(stream, d_status.device))
 
 
+def moe_quant_fp8_channel_workspace_bytes(num_experts: int, hidden: int) -> int:
+    return int(_lib.moe_quant_fp8_channel_workspace_bytes(num_experts, hidden))
+
+
 def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, expert_count: torch.Tensor, *,
-                          transpose: bool = False, out=None, scale=None, d_status=None, stream=None):
+                          transpose: bool = False, out=None, scale=None, workspace="new", d_status=None,
+                          stream=None):
     """Per-(expert, channel) FP8 of the receive rows ``recv`` (bf16 [S, H]) over
     each expert's landed rows; returns ``(codes uint8 [S, H] or [H, S], scale
-    fp32 [E, H])``."""
+    fp32 [E, H])``.  ``workspace``: a uint8 device tensor of
+    ``moe_quant_fp8_channel_workspace_bytes(E, H)`` bytes, zero before its
+    first use and left zero by every call (keep one per stream); ``"new"``
+    (default) allocates a zeroed one for this call; None takes the path
+    without scratch."""
     _need(recv, "recv", torch.bfloat16)
     S, H = recv.shape
     _need(expert_count, "expert_count", torch.int32)
@@ -495,10 +506,21 @@ def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, exper
         scale = torch.empty((E, H), dtype=torch.float32, device=recv.device)
     _need(out, "out", torch.uint8, shape)
     _need(scale, "scale", torch.float32, (E, H))
+    ws_bytes = moe_quant_fp8_channel_workspace_bytes(E, H)
+    if isinstance(workspace, str):
+        if workspace != "new":
+            raise ValueError(f"workspace must be a tensor, None or 'new', not {workspace!r}")
+        # zeroed in the order of the stream the kernel runs on
+        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream(recv.device)):
+            workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=recv.device)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        if workspace.numel() < ws_bytes:
+            raise ValueError(f"workspace holds {workspace.numel()} bytes, {ws_bytes} needed")
     _launch(_lib.moe_quant_fp8_channel, "moe_quant_fp8_channel",
-            (recv, expert_offset, expert_count, out, scale, _status(d_status)), _ptr(recv), S, H, E,
-            _ptr(expert_offset), _ptr(expert_count), int(transpose), _ptr(out), _ptr(scale), _ptr(d_status),
-            _stream(stream, recv.device))
+            (recv, expert_offset, expert_count, out, scale, workspace, _status(d_status)), _ptr(recv), S, H, E,
+            _ptr(expert_offset), _ptr(expert_count), int(transpose), _ptr(out), _ptr(scale), _ptr(workspace),
+            workspace.numel() if workspace is not None else 0, _ptr(d_status), _stream(stream, recv.device))
     return out, scale
 
 

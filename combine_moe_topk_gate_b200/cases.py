@@ -79,9 +79,10 @@ def build(op: str, workload: str, rows: int | None, inter: int, device):
         recv = torch.randn(La.num_rows, w.H, generator=g).to(torch.bfloat16).to(device)
         out = torch.empty((La.num_rows, w.H), dtype=torch.uint8, device=device)
         sc = torch.empty((w.E, w.H), dtype=torch.float32, device=device)
+        ws = torch.zeros(api.moe_quant_fp8_channel_workspace_bytes(w.E, w.H), dtype=torch.uint8, device=device)
         landed = int((La.slot_token >= 0).sum().item())
         return (lambda: api.moe_quant_fp8_channel(recv, La.expert_offset, La.expert_count, out=out, scale=sc,
-                                                  d_status=La.status)), landed * w.H * 3 + 4 * w.E * w.H
+                                                  workspace=ws, d_status=La.status)), landed * w.H * 3 + 4 * w.E * w.H
     raise SystemExit(f"unknown op {op}")
 
 

@@ -232,21 +232,29 @@ moe_status_t moe_selftest_bounded_wait(int32_t* d_status, moe_stream_t stream) {
   return from_cuda(moe::launch_bounded_wait_selftest(d_status, as_stream(stream)));
 }
 
+size_t moe_quant_fp8_channel_workspace_bytes(int num_experts, int hidden) {
+  if (num_experts < 1 || num_experts > MOE_MAX_EXPERTS || hidden < 128 || hidden % 128 != 0) return 0;
+  return moe::quant_fp8_channel_workspace_bytes(num_experts, hidden);
+}
+
 moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,
                                    const int32_t* expert_offset, const int32_t* expert_count,
-                                   int transpose, void* out, float* scale, int32_t* d_status,
-                                   moe_stream_t stream) {
+                                   int transpose, void* out, float* scale, void* workspace,
+                                   size_t workspace_bytes, int32_t* d_status, moe_stream_t stream) {
   if (num_rows < 0 || hidden < 1 || num_experts < 1) return MOE_ERR_INVALID_ARG;
   if (hidden % 128 != 0 || (transpose != 0 && transpose != 1)) return MOE_ERR_INVALID_ARG;
   if (num_experts > MOE_MAX_EXPERTS) return MOE_ERR_UNSUPPORTED;
   if (!expert_offset || !expert_count || !scale || (num_rows > 0 && (!recv || !out)))
     return MOE_ERR_INVALID_ARG;
   if (!aligned(recv, 16) || !aligned(out, 16) || !aligned(scale, 4) || !aligned(expert_offset, 4) ||
-      !aligned(expert_count, 4) || !aligned(d_status, 4))
+      !aligned(expert_count, 4) || !aligned(d_status, 4) || !aligned(workspace, 16))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace &&
+      workspace_bytes < moe::quant_fp8_channel_workspace_bytes(num_experts, hidden))
     return MOE_ERR_INVALID_ARG;
   return from_cuda(moe::launch_quant_fp8_channel(recv, num_rows, hidden, num_experts, expert_offset,
                                                  expert_count, transpose != 0, out, scale, d_status,
-                                                 as_stream(stream)));
+                                                 workspace, as_stream(stream)));
 }
 
 moe_status_t moe_swiglu_quant(const void* h, int num_rows, int inter, const int32_t* slot_token,

@@ -58,10 +58,11 @@ cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int3
                                   long long num_rows, int scale_layout, void* recv_x,
                                   void* block_scale, float* row_scale, int32_t* d_status,
                                   cudaStream_t stream);
+size_t quant_fp8_channel_workspace_bytes(int E, int H);
 cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, int E,
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,
-                                     cudaStream_t stream);
+                                     void* workspace, cudaStream_t stream);
 cudaError_t launch_bounded_wait_selftest(int32_t* d_status, cudaStream_t stream);
 cudaError_t launch_swiglu_quant(const void* h, long long num_rows, int I, const int32_t* slot_token,
                                 int dtype, int scale_layout, void* out, void* out_scale,

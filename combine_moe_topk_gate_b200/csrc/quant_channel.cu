@@ -28,6 +28,8 @@
 // through distributed shared memory between two hardware cluster barriers,
 // and each CTA writes the codes of its own rows.  A max is exact in any
 // order, so every Q gives the same bits.
+#include <algorithm>
+
 #include "moe_device.cuh"
 #include "moe_launch.h"
 
@@ -39,6 +41,8 @@ constexpr int kWarpsPerCta = kThreads / 32;
 constexpr int kMinSlabLog2 = 7;                 // 128 channels: 256-byte row pieces
 constexpr long long kResidentCtas = 148 * 4;     // CTAs one wave holds (4 per SM)
 constexpr long long kWaveBytes = 96ll << 20;     // rows a wave may keep in L2 between its passes
+constexpr int kPartRows = 256;                  // rows per task of the queue kernel (a multiple of 32)
+constexpr int kMaxParts = 64;                   // parts per (expert, slab): fewer than the grid's CTAs
 
 // L2 eviction policies: pass 1 marks the slab's lines evict-last so that pass
 // 2 finds them in L2 despite the stream of other CTAs' loads and stores;
@@ -67,45 +71,17 @@ __device__ __forceinline__ void st_hint_v2(void* ptr, uint2 v, uint64_t pol) {
                "l"(pol));
 }
 
-template <bool TRANSPOSE, bool CLUSTER, int LSW>
-__global__ void __launch_bounds__(kThreads)
-    quant_fp8_channel_kernel(const uint16_t* __restrict__ x, long long S, int H, int E,
-                             const int32_t* __restrict__ expert_offset,
-                             const int32_t* __restrict__ expert_count, uint8_t* __restrict__ out,
-                             float* __restrict__ scale, int32_t* d_status) {
-  constexpr int SW = 1 << LSW;      // channels per slab
-  constexpr int LPR = SW / 8;       // lanes per row (8 channels, 16 bytes each)
-  constexpr int RPW = 32 / LPR;     // rows per warp instruction
-  constexpr int STEP = kWarpsPerCta * RPW;  // rows per CTA instruction
-  __shared__ float part[kWarpsPerCta][SW];
-  __shared__ float inv_s[SW];
-  __shared__ float cta_amax[CLUSTER ? SW : 1];  // this CTA's share, read by the cluster
-  __shared__ uint8_t tile[TRANSPOSE ? SW : 1][33];  // transposed: 32 rows per channel (+1: banks)
+// Pass 1 of a slab over rows [rb, r1): the per-channel amax of this CTA's
+// rows, returned on thread c for channel c < SW (0 on the others).  Lanes
+// reduce packed bf16 pairs (|x| and max are exact in bf16, so the result is
+// the fp32 amax), eight loads in flight per lane; part[] is left for the
+// caller to reuse after its next __syncthreads.
+template <int LSW>
+__device__ __forceinline__ float slab_amax(const uint16_t* __restrict__ col, int H, long long rb,
+                                           long long r1, uint64_t keep, float (*part)[1 << LSW]) {
+  constexpr int SW = 1 << LSW, LPR = SW / 8, RPW = 32 / LPR, STEP = kWarpsPerCta * RPW;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // cluster: x = slab * Q + rank, the Q CTAs of a cluster share (expert, slab)
-  const int Q = CLUSTER ? static_cast<int>(gridDim.x / (H / SW)) : 1;
-  const int q = CLUSTER ? static_cast<int>(cluster_rank()) : 0;
-  const int slab = CLUSTER ? static_cast<int>(blockIdx.x) / Q : static_cast<int>(blockIdx.x);
-  const int e = blockIdx.y;
-  const int sub = lane % LPR, rr = lane / LPR;  // channel group and row of the lane
-  const int cl = sub * 8;                       // the lane's first channel inside the slab
-  const int c0 = slab * SW + cl;
-  pdl_wait();
-  pdl_trigger();
-  const long long r0 = expert_offset[e];
-  const long long n = expert_count[e];
-  if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert (the
-    if (tid == 0 && slab == 0) report_bad_index(d_status);  // whole cluster returns:
-    return;                                                   // e is the same for all)
-  }
-  const long long share = CLUSTER ? ((n + Q - 1) / Q + 31) / 32 * 32 : n;  // rows per CTA
-  const long long rb = r0 + q * share < r0 + n ? r0 + q * share : r0 + n;  // this CTA's rows
-  const long long r1 = rb + share < r0 + n ? rb + share : r0 + n;
-  const uint16_t* col = x + c0;
-  const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
-
-  // pass 1: amax of the lane's 8 channels over its rows, on packed bf16
-  // pairs (|x| and max are exact in bf16, so the result is the fp32 amax)
+  const int rr = lane / LPR, cl = (lane % LPR) * 8;
   __nv_bfloat162 m2[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) m2[j] = __floats2bfloat162_rn(0.0f, 0.0f);
@@ -114,17 +90,15 @@ __global__ void __launch_bounds__(kThreads)
 #pragma unroll
     for (int j = 0; j < 4; ++j) m2[j] = __hmax2(m2[j], __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w[j])));
   };
-  {
-    long long s = rb + warp * RPW + rr;
-    for (; s + 7 * STEP < r1; s += 8 * STEP) {
-      uint4 v[8];
+  long long s = rb + warp * RPW + rr;
+  for (; s + 7 * STEP < r1; s += 8 * STEP) {
+    uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = ld_hint(col + static_cast<size_t>(s + u * STEP) * H, keep);
+    for (int u = 0; u < 8; ++u) v[u] = ld_hint(col + static_cast<size_t>(s + u * STEP) * H, keep);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) fold(v[u]);
-    }
-    for (; s < r1; s += STEP) fold(ld_hint(col + static_cast<size_t>(s) * H, keep));
+    for (int u = 0; u < 8; ++u) fold(v[u]);
   }
+  for (; s < r1; s += STEP) fold(ld_hint(col + static_cast<size_t>(s) * H, keep));
   // lanes of a warp holding the same channels differ in their row bits
 #pragma unroll
   for (int off = LPR; off < 32; off <<= 1) {
@@ -142,30 +116,27 @@ __global__ void __launch_bounds__(kThreads)
     }
   }
   __syncthreads();
-  {
-    const int c = tid;  // channel of this thread, c < SW
-    float a = 0.0f;
-    if (c < SW) {
-      a = part[0][c];
+  float a = 0.0f;
+  if (tid < SW) {
+    a = part[0][tid];
 #pragma unroll
-      for (int w = 1; w < kWarpsPerCta; ++w) a = fmaxf(a, part[w][c]);
-    }
-    if constexpr (CLUSTER) {
-      if (c < SW) cta_amax[c] = a;
-      cluster_arrive();  // every CTA's share published ...
-      cluster_wait();
-      if (c < SW) {
-        a = 0.0f;
-        for (int r = 0; r < Q; ++r) a = fmaxf(a, ld_peer_shared_f32(&cta_amax[c], static_cast<uint32_t>(r)));
-      }
-      cluster_arrive();  // ... and read; the matching wait comes before the exit
-    }
-    if (c < SW) {
-      inv_s[c] = __fdiv_rn(448.0f, a);
-      if (q == 0) scale[static_cast<size_t>(e) * H + slab * SW + c] = __fdiv_rn(a, 448.0f);
-    }
+    for (int w = 1; w < kWarpsPerCta; ++w) a = fmaxf(a, part[w][tid]);
   }
-  __syncthreads();
+  return a;
+}
+
+// Pass 2 of a slab over rows [rb, r1): codes x * inv_s[c] of every channel,
+// row-major (8 bytes per lane and row) or transposed through a shared-memory
+// tile of 32 rows (each warp store then covers 32 consecutive rows of one
+// channel).  x * inv of finite bf16 is never NaN, so the encoder without NaN
+// handling gives the same codes.  inv_s must be visible to the whole CTA.
+template <bool TRANSPOSE, int LSW>
+__device__ __forceinline__ void slab_codes(const uint16_t* __restrict__ col, uint8_t* __restrict__ out,
+                                           long long S, int H, int slab, long long rb, long long r1,
+                                           const float* inv_s, uint64_t done, uint8_t (*tile)[33]) {
+  constexpr int SW = 1 << LSW, LPR = SW / 8, RPW = 32 / LPR, STEP = kWarpsPerCta * RPW;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rr = lane / LPR, cl = (lane % LPR) * 8, c0 = slab * SW + cl;
   float inv[8];
   bool finite = true;  // every 448/amax of the lane finite: products keep zero signs
 #pragma unroll
@@ -173,9 +144,6 @@ __global__ void __launch_bounds__(kThreads)
     inv[i] = inv_s[cl + i];
     finite = finite && inv[i] <= 3.402823466e38f;
   }
-
-  // pass 2: codes of one row's 8 channels (x * inv of finite bf16 is never
-  // NaN, so the encoder without NaN handling gives the same codes)
   auto codes_of_v = [&](uint4 v) -> uint2 {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     float p[8];
@@ -229,14 +197,247 @@ __global__ void __launch_bounds__(kThreads)
       __syncthreads();
     }
   }
+}
+
+// Cluster version (no workspace): one CTA, or a cluster of Q CTAs, per
+// (expert, slab); the Q CTAs combine their amax through distributed shared
+// memory between two hardware cluster barriers.
+template <bool TRANSPOSE, bool CLUSTER, int LSW>
+__global__ void __launch_bounds__(kThreads)
+    quant_fp8_channel_kernel(const uint16_t* __restrict__ x, long long S, int H, int E,
+                             const int32_t* __restrict__ expert_offset,
+                             const int32_t* __restrict__ expert_count, uint8_t* __restrict__ out,
+                             float* __restrict__ scale, int32_t* d_status) {
+  constexpr int SW = 1 << LSW;
+  __shared__ float part[kWarpsPerCta][SW];
+  __shared__ float inv_s[SW];
+  __shared__ float cta_amax[CLUSTER ? SW : 1];  // this CTA's share, read by the cluster
+  __shared__ uint8_t tile[TRANSPOSE ? SW : 1][33];  // transposed: 32 rows per channel (+1: banks)
+  const int tid = threadIdx.x;
+  // cluster: x = slab * Q + rank, the Q CTAs of a cluster share (expert, slab)
+  const int Q = CLUSTER ? static_cast<int>(gridDim.x / (H / SW)) : 1;
+  const int q = CLUSTER ? static_cast<int>(cluster_rank()) : 0;
+  const int slab = CLUSTER ? static_cast<int>(blockIdx.x) / Q : static_cast<int>(blockIdx.x);
+  const int e = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
+  const long long r0 = expert_offset[e];
+  const long long n = expert_count[e];
+  if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert (the
+    if (tid == 0 && slab == 0) report_bad_index(d_status);  // whole cluster returns:
+    return;                                                   // e is the same for all)
+  }
+  const long long share = CLUSTER ? ((n + Q - 1) / Q + 31) / 32 * 32 : n;  // rows per CTA
+  const long long rb = r0 + q * share < r0 + n ? r0 + q * share : r0 + n;  // this CTA's rows
+  const long long r1 = rb + share < r0 + n ? rb + share : r0 + n;
+  const uint16_t* col = x + slab * SW;
+  const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
+
+  float a = slab_amax<LSW>(col + ((tid & 31) % (SW / 8)) * 8, H, rb, r1, keep, part);
+  if constexpr (CLUSTER) {
+    if (tid < SW) cta_amax[tid] = a;
+    cluster_arrive();  // every CTA's share published ...
+    cluster_wait();
+    if (tid < SW) {
+      a = 0.0f;
+      for (int r = 0; r < Q; ++r) a = fmaxf(a, ld_peer_shared_f32(&cta_amax[tid], static_cast<uint32_t>(r)));
+    }
+    cluster_arrive();  // ... and read; the matching wait comes before the exit
+  }
+  if (tid < SW) {
+    inv_s[tid] = __fdiv_rn(448.0f, a);
+    if (q == 0) scale[static_cast<size_t>(e) * H + slab * SW + tid] = __fdiv_rn(a, 448.0f);
+  }
+  __syncthreads();
+  slab_codes<TRANSPOSE, LSW>(col + ((tid & 31) % (SW / 8)) * 8, out, S, H, slab, rb, r1, inv_s, done, tile);
   if constexpr (CLUSTER) cluster_wait();  // no CTA leaves while a peer may still read its share
+}
+
+// ---------------------------------------------------------------- task queue
+// Workspace (32-bit words, all zero between calls): [0] next task, [1] CTAs
+// finished, then two counters per (expert, 128-channel slab) -- parts that
+// published their amax, parts that have read the combined one -- then the
+// combined amax of every (expert, channel) as fp32 bits (a max of
+// non-negative floats is the max of their bit patterns).
+constexpr int kWsHeaderWords = 64;
+
+__host__ __device__ inline long long ws_counter_base() { return kWsHeaderWords; }
+__host__ __device__ inline long long ws_amax_base(int E, int H) {
+  return kWsHeaderWords + 2ll * E * (H >> kMinSlabLog2);
+}
+
+// parts an expert of n rows is cut into (a bad count: one part, which only reports it)
+__device__ __forceinline__ int parts_of(long long n) {
+  if (n <= kPartRows) return 1;
+  const long long p = (n + kPartRows - 1) / kPartRows;
+  return p < kMaxParts ? static_cast<int>(p) : kMaxParts;
+}
+
+// Persistent CTAs take tasks (expert e, slab, part p) from a counter in the
+// workspace, in the order e, slab, p, so the parts of one (expert, slab) run
+// side by side and its rows are read twice within a short time (the second
+// time from L2).  A part publishes its amax with atomic max, counts itself
+// in, and waits (bounded) until every part of its (expert, slab) has done the
+// same; the parts were taken before any later task, and pass 1 waits on
+// nothing, so the wait ends as long as the grid has more CTAs than an
+// expert has parts.  The last part to read the combined amax zeroes the
+// scratch of its (expert, slab); the last CTA to finish zeroes the queue.
+template <bool TRANSPOSE, int LSW>
+__global__ void __launch_bounds__(kThreads)
+    quant_fp8_channel_queue_kernel(const uint16_t* __restrict__ x, long long S, int H, int E,
+                                   const int32_t* __restrict__ expert_offset,
+                                   const int32_t* __restrict__ expert_count, uint8_t* __restrict__ out,
+                                   float* __restrict__ scale, int32_t* d_status, uint32_t* ws) {
+  constexpr int SW = 1 << LSW;
+  __shared__ float part[kWarpsPerCta][SW];
+  __shared__ float inv_s[SW];
+  __shared__ uint8_t tile[TRANSPOSE ? SW : 1][33];
+  __shared__ int first_task[MOE_MAX_EXPERTS + 1];  // tasks of experts < e
+  __shared__ int scan[kThreads];
+  __shared__ int s_task, s_last;
+  const int tid = threadIdx.x;
+  const int slabs = H >> LSW;
+  pdl_wait();
+  pdl_trigger();
+
+  // first_task[e] = slabs * sum over e' < e of parts_of(n_e'): thread i sums
+  // the experts of its contiguous run, then a block scan of the run totals
+  {
+    const int per = (E + kThreads - 1) / kThreads;
+    const int e0 = tid * per, e1 = e0 + per < E ? e0 + per : E;
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) sum += parts_of(expert_count[e]) * slabs;
+    scan[tid] = sum;
+    __syncthreads();
+    for (int off = 1; off < kThreads; off <<= 1) {
+      const int v = tid >= off ? scan[tid - off] : 0;
+      __syncthreads();
+      scan[tid] += v;
+      __syncthreads();
+    }
+    int run = scan[tid] - sum;  // exclusive prefix of this thread's run
+    for (int e = e0; e < e1; ++e) {
+      first_task[e] = run;
+      run += parts_of(expert_count[e]) * slabs;
+    }
+    if (tid == kThreads - 1) first_task[E] = scan[kThreads - 1];
+    __syncthreads();
+  }
+  const int total = first_task[E];
+  const uint64_t keep = l2_policy_evict_last(), done = l2_policy_evict_first();
+  uint32_t* const counters = ws + ws_counter_base();
+  uint32_t* const amax_ws = ws + ws_amax_base(E, H);
+
+  if (tid == 0) s_task = static_cast<int>(atomicAdd(&ws[0], 1u));
+  __syncthreads();
+  for (;;) {
+    const int t = s_task;
+    __syncthreads();  // s_task may be overwritten from here on
+    if (t >= total) break;
+    // the expert whose tasks hold t: the last e with first_task[e] <= t
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (first_task[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    const int e = lo;
+    const long long r0 = expert_offset[e];
+    const long long n = expert_count[e];
+    const int P = parts_of(n);
+    const int j = t - first_task[e];
+    const int slab = j / P, p = j - slab * P;
+    if (r0 < 0 || n < 0 || r0 + n > S) {  // a corrupted layout: skip the expert
+      if (tid == 0) {
+        if (j == 0) report_bad_index(d_status);
+        s_task = static_cast<int>(atomicAdd(&ws[0], 1u));
+      }
+      __syncthreads();
+      continue;
+    }
+    const long long share = P == 1 ? n : ((n + P - 1) / P + 31) / 32 * 32;
+    const long long rb = r0 + p * share < r0 + n ? r0 + p * share : r0 + n;
+    const long long r1 = rb + share < r0 + n ? rb + share : r0 + n;
+    const uint16_t* col = x + slab * SW + ((tid & 31) % (SW / 8)) * 8;
+
+    float a = slab_amax<LSW>(col, H, rb, r1, keep, part);
+    if (P > 1) {
+      uint32_t* const unit_amax = amax_ws + static_cast<size_t>(e) * H + slab * SW;
+      uint32_t* const cnt = counters + 2 * (static_cast<size_t>(e) * (H >> kMinSlabLog2) + slab);
+      if (tid < SW) atomicMax(&unit_amax[tid], __float_as_uint(a));
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        atomicAdd(&cnt[0], 1u);
+        const unsigned long long t0 = globaltimer_ns();
+        while (atomicAdd(&cnt[0], 0u) < static_cast<uint32_t>(P)) {
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            report_timeout(d_status);
+            break;
+          }
+          __nanosleep(64);
+        }
+        __threadfence();
+      }
+      __syncthreads();
+      if (tid < SW) a = __uint_as_float(atomicAdd(&unit_amax[tid], 0u));
+      __syncthreads();  // every thread holds the combined amax
+      if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(&cnt[1], 1u) == static_cast<uint32_t>(P - 1);
+      }
+      __syncthreads();
+      if (s_last) {  // every part has read it: leave the scratch zeroed
+        if (tid < SW) unit_amax[tid] = 0u;
+        if (tid == 0) {
+          cnt[0] = 0u;
+          cnt[1] = 0u;
+        }
+      }
+    }
+    // this task waits on nothing from here on: take the next one now, so that
+    // the counter's round trip overlaps pass 2 (a CTA never waits while it
+    // holds a task it has not started)
+    uint32_t next = 0;
+    if (tid == 0) next = atomicAdd(&ws[0], 1u);
+    if (tid < SW) {
+      inv_s[tid] = __fdiv_rn(448.0f, a);
+      if (p == 0) scale[static_cast<size_t>(e) * H + slab * SW + tid] = __fdiv_rn(a, 448.0f);
+    }
+    __syncthreads();
+    slab_codes<TRANSPOSE, LSW>(col, out, S, H, slab, rb, r1, inv_s, done, tile);
+    if (tid == 0) s_task = static_cast<int>(next);
+    __syncthreads();  // the next task is known; inv_s and part are free again
+  }
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(&ws[1], 1u) == gridDim.x - 1) {  // the last CTA: every task is taken
+      ws[0] = 0u;
+      ws[1] = 0u;
+    }
+  }
 }
 
 template <bool TRANSPOSE, int LSW>
 cudaError_t launch_channel(bool cluster, int Q, const uint16_t* xs, long long num_rows, int H, int E,
                            const int32_t* expert_offset, const int32_t* expert_count, uint8_t* o,
-                           float* scale, int32_t* d_status, cudaStream_t stream) {
+                           float* scale, int32_t* d_status, uint32_t* ws, cudaStream_t stream) {
   const int slabs = H >> LSW;
+  if (ws) {
+    auto* kernel = quant_fp8_channel_queue_kernel<TRANSPOSE, LSW>;
+    int dev = 0, sms = 0, per_sm = 0;
+    cudaError_t err;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return err;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0)) != cudaSuccess)
+      return err;
+    // no more CTAs than tasks can exist; never fewer than an expert's parts + 1
+    const long long tasks = ((num_rows + kPartRows - 1) / kPartRows + E) * slabs;
+    long long grid = static_cast<long long>(sms) * (per_sm > 0 ? per_sm : 1);
+    if (grid > tasks) grid = tasks;
+    if (grid < kMaxParts + 1 && tasks > grid) grid = kMaxParts + 1;
+    return launch_pdl(kernel, static_cast<unsigned>(grid), kThreads, 0, stream, xs, num_rows, H, E,
+                      expert_offset, expert_count, o, scale, d_status, ws);
+  }
   if (cluster)
     return launch_pdl_cluster(quant_fp8_channel_kernel<TRANSPOSE, true, LSW>, dim3(slabs * Q, E), kThreads, 0,
                               stream, Q, xs, num_rows, H, E, expert_offset, expert_count, o, scale, d_status);
@@ -247,45 +448,55 @@ cudaError_t launch_channel(bool cluster, int Q, const uint16_t* xs, long long nu
 template <bool TRANSPOSE>
 cudaError_t launch_channel_sw(int lsw, bool cluster, int Q, const uint16_t* xs, long long num_rows, int H,
                               int E, const int32_t* expert_offset, const int32_t* expert_count, uint8_t* o,
-                              float* scale, int32_t* d_status, cudaStream_t stream) {
+                              float* scale, int32_t* d_status, uint32_t* ws, cudaStream_t stream) {
   switch (lsw) {
     case 8: return launch_channel<TRANSPOSE, 8>(cluster, Q, xs, num_rows, H, E, expert_offset, expert_count, o,
-                                                scale, d_status, stream);
-    case 7: return launch_channel<TRANSPOSE, 7>(cluster, Q, xs, num_rows, H, E, expert_offset, expert_count, o,
-                                                scale, d_status, stream);
-    case 6: return launch_channel<TRANSPOSE, 6>(cluster, Q, xs, num_rows, H, E, expert_offset, expert_count, o,
-                                                scale, d_status, stream);
-    default: return launch_channel<TRANSPOSE, 5>(cluster, Q, xs, num_rows, H, E, expert_offset, expert_count, o,
-                                                 scale, d_status, stream);
+                                                scale, d_status, ws, stream);
+    default: return launch_channel<TRANSPOSE, 7>(cluster, Q, xs, num_rows, H, E, expert_offset, expert_count, o,
+                                                 scale, d_status, ws, stream);
   }
 }
 
 }  // namespace
 
+size_t quant_fp8_channel_workspace_bytes(int E, int H) {
+  return 4 * static_cast<size_t>(ws_amax_base(E, H) + static_cast<long long>(E) * H);
+}
+
 cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, int E,
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,
-                                     cudaStream_t stream) {
+                                     void* workspace, cudaStream_t stream) {
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* o = static_cast<uint8_t*>(out);
-  // CTAs per (expert, slab): about 512 rows each on average, at most 8 (the
-  // portable cluster size); 1 keeps the plain launch
   const long long avg_rows = E > 0 ? num_rows / E : 0;
-  const int Q = avg_rows >= 4096 ? 8 : avg_rows >= 2048 ? 4 : avg_rows >= 1024 ? 2 : 1;
+  // The task queue (workspace) where the cluster path would give every
+  // (expert, slab) one CTA although the average expert already fills a part:
+  // there a hot expert's lone CTAs are the critical path (Zipf-skewed shape:
+  // 297 against 369 us).  Below that the hardware's own scheduling of the
+  // small (expert, slab) CTAs is faster than the persistent loop (prefill
+  // shape: 128 against 144 us; decode: 27 against 41 us), and from 1024 rows
+  // on the clusters already spread every expert (Mixtral shape: 103 against
+  // 108 us).
+  uint32_t* ws = (avg_rows >= kPartRows && avg_rows < 1024) ? static_cast<uint32_t*>(workspace) : nullptr;
+  // Without it: CTAs per (expert, slab) from the average rows, about 512 rows
+  // each, at most 8 (the portable cluster size); 1 keeps the plain launch.
+  const int Q = ws ? 1 : avg_rows >= 4096 ? 8 : avg_rows >= 2048 ? 4 : avg_rows >= 1024 ? 2 : 1;
   // Slab width: the rows one wave of resident CTAs holds between its two
   // passes should fit in L2, or the second pass re-reads DRAM; a narrower
   // slab gives smaller CTAs and more waves, and spreads a hot expert over
   // more CTAs.  Measured on B200 (256 / 128 / 64 / 32 channels): 256 is best
   // up to the 4096-token prefill shape, 128 on the Zipf-skewed and the
-  // Mixtral shapes, narrower never (the per-CTA overhead wins).
-  const long long share = (avg_rows + Q - 1) / Q;
+  // Mixtral shapes, narrower never (the per-CTA overhead wins).  With the
+  // workspace a task holds at most kPartRows rows of its slab.
+  const long long share = ws ? std::min<long long>(avg_rows, kPartRows) : (avg_rows + Q - 1) / Q;
   int lsw = (H % 256 == 0) ? 8 : 7;
   if (lsw > kMinSlabLog2 && kResidentCtas * share * (2ll << lsw) > kWaveBytes) --lsw;
   if (transpose)
     return launch_channel_sw<true>(lsw, Q > 1, Q, xs, num_rows, H, E, expert_offset, expert_count, o, scale,
-                                   d_status, stream);
+                                   d_status, ws, stream);
   return launch_channel_sw<false>(lsw, Q > 1, Q, xs, num_rows, H, E, expert_offset, expert_count, o, scale,
-                                  d_status, stream);
+                                  d_status, ws, stream);
 }
 
 }  // namespace moe

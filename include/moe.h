@@ -406,13 +406,33 @@ moe_status_t moe_dispatch_nvfp4(const void* x, int num_tokens, int hidden, int k
  *   transpose      0: out e4m3 [S, H] row-major; 1: out e4m3 [H, S]
  *                  (channel-major, the K-major operand).
  *   scale          fp32 [E, H] out (0 for an expert with no rows).
+ *   workspace      device scratch of at least
+ *                  moe_quant_fp8_channel_workspace_bytes(E, H) bytes,
+ *                  16-byte aligned, all zero before the first call; every
+ *                  call leaves it zero again, so one zeroing serves all
+ *                  later calls in stream order (one workspace per stream:
+ *                  calls running at the same time need their own).  It is
+ *                  used when the average expert holds 256 to 1023 of the S
+ *                  rows: each expert's rows are then cut into parts of at
+ *                  most 256 rows (64 parts at most) and a persistent grid
+ *                  takes (expert, channel slab, part) tasks from a counter
+ *                  in it, so a hot expert spreads over many CTAs, whose
+ *                  parts combine their amax through it.  Otherwise, and when
+ *                  NULL: one CTA, or a cluster of up to 8, per (expert,
+ *                  slab), sized from the average rows per expert (no
+ *                  scratch).  Both give the same bits.  A wait that outlasts
+ *                  1 s sets MOE_ERR_TIMEOUT.
  *   Padding rows (outside every expert's landed range) are not written.
  *   H % 128 == 0, 1 <= E <= MOE_MAX_EXPERTS.
  */
 moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,
                                    const int32_t* expert_offset, const int32_t* expert_count,
-                                   int transpose, void* out, float* scale, int32_t* d_status,
-                                   moe_stream_t stream);
+                                   int transpose, void* out, float* scale, void* workspace,
+                                   size_t workspace_bytes, int32_t* d_status, moe_stream_t stream);
+
+/* Bytes of moe_quant_fp8_channel's workspace for E experts of H channels
+ * (0 when E or H is outside that call's limits). */
+size_t moe_quant_fp8_channel_workspace_bytes(int num_experts, int hidden);
 
 /*
  * moe_swiglu_quant -- SwiGLU between an expert's two GEMMs, fused with the

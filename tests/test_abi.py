@@ -245,8 +245,15 @@ def test_e5m6_sizes_and_validation(api):
 def test_quant_fp8_channel_rejects_bad_arguments(api):
     L = api.lib()
 
-    def call(S=64, H=256, E=4, tr=0, recv=_P(), out=_P(), sc=_P(), off=_P(), cnt=_P()):
-        return L.moe_quant_fp8_channel(recv, S, H, E, off, cnt, tr, out, sc, None, None)
+    def call(S=64, H=256, E=4, tr=0, recv=_P(), out=_P(), sc=_P(), off=_P(), cnt=_P(), ws=None, wsb=0):
+        return L.moe_quant_fp8_channel(recv, S, H, E, off, cnt, tr, out, sc, ws, wsb, None, None)
+    need = api.moe_quant_fp8_channel_workspace_bytes(4, 256)
+    # header, two counters per (expert, 128-channel slab), one amax per (expert, channel)
+    assert need == 4 * (64 + 2 * 4 * 2 + 4 * 256)
+    assert api.moe_quant_fp8_channel_workspace_bytes(0, 256) == 0
+    assert api.moe_quant_fp8_channel_workspace_bytes(4, 192) == 0
+    assert call(ws=_P(), wsb=need - 4) == api.MOE_ERR_INVALID_ARG   # short workspace
+    assert call(ws=_P(0x1008), wsb=need) == api.MOE_ERR_INVALID_ARG  # not 16-byte aligned
     assert call(H=192) == api.MOE_ERR_INVALID_ARG           # H % 128
     assert call(E=0) == api.MOE_ERR_INVALID_ARG
     assert call(E=2000) == api.MOE_ERR_UNSUPPORTED
