@@ -99,20 +99,26 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
       for (int i = 0; i < 4; ++i) sword |= (__shfl_sync(kFullMask, byte, 8 * i) & 0xffu) << (8 * i);
     } else {
-      inv = __fdiv_rn(448.0f, amax);
-      scale = __fdiv_rn(amax, 448.0f);
+      // the block's 448 / amax and amax / 448 from one division per lane:
+      // even lanes take the first, odd lanes the second
+      const bool odd = lane & 1;
+      const float qd = __fdiv_rn(odd ? amax : 448.0f, odd ? 448.0f : amax);
+      inv = __shfl_sync(kFullMask, qd, lane & ~7);
+      scale = __shfl_sync(kFullMask, qd, (lane & ~7) | 1);
+    }
+    // a finite factor keeps the sign of a zero by itself; an infinite one (an
+    // all-zero or tiny block) needs the select
+    float p[16];
+    if (UE8M0 || inv <= 3.402823466e38f) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) p[i] = __fmul_rn(f[i], inv);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) p[i] = f[i] != 0.0f ? __fmul_rn(f[i], inv) : f[i];  // zero keeps its sign
     }
     uint32_t q[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float p[4];
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const float xv = f[4 * i + v];
-        p[v] = (UE8M0 || xv != 0.0f) ? __fmul_rn(xv, inv) : xv;  // zero keeps its sign
-      }
-      q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
-    }
+    for (int i = 0; i < 4; ++i) q[i] = e4m3x2(p[4 * i], p[4 * i + 1]) | (e4m3x2(p[4 * i + 2], p[4 * i + 3]) << 16);
     const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
     for (int j = 0; j < k; ++j) {
       const int slot = __shfl_sync(kFullMask, my_slot, j);
