@@ -83,9 +83,18 @@ __global__ void __launch_bounds__(kWarps * 32)
       f[2 * i] = bf16_lo(w[i]);
       f[2 * i + 1] = bf16_hi(w[i]);
     }
+    // A warp whose values are all finite (the usual case) takes the encoder
+    // without NaN fix-ups: no input NaN, and no inf * 0 in the scaling.  The
+    // maximum with NaN propagation doubles as the block amax there.
     float amax = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    for (int i = 0; i < 16; ++i) amax = max_abs_nan(amax, f[i]);
+    const bool special = __any_sync(kFullMask, !(amax <= 3.402823466e38f));
+    if (special) {  // warp-uniform: the amax ignores NaN, as the definition does
+      amax = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    }
     amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
     amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 2));
     amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 4));
@@ -94,7 +103,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     if constexpr (UE8M0) {
       int e = amax > 0.0f ? ceil_log2_pos(__fdiv_rn(amax, 448.0f)) : -127;
       e = e < -127 ? -127 : (e > 127 ? 127 : e);
-      inv = __int_as_float((127 - e) << 23);  // 2^-e; e <= 120 for bf16 input
+      // 2^-e exactly: a normal float for e <= 126 (every finite bf16 block:
+      // e <= 120), the subnormal 2^-127 for an infinite amax (e = 127)
+      inv = e < 127 ? __int_as_float((127 - e) << 23) : __int_as_float(0x00400000);
       const uint32_t byte = static_cast<uint32_t>(e + 127);
 #pragma unroll
       for (int i = 0; i < 4; ++i) sword |= (__shfl_sync(kFullMask, byte, 8 * i) & 0xffu) << (8 * i);
@@ -117,8 +128,14 @@ __global__ void __launch_bounds__(kWarps * 32)
       for (int i = 0; i < 16; ++i) p[i] = f[i] != 0.0f ? __fmul_rn(f[i], inv) : f[i];  // zero keeps its sign
     }
     uint32_t q[4];
+    if (special) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = e4m3x2(p[4 * i], p[4 * i + 1]) | (e4m3x2(p[4 * i + 2], p[4 * i + 3]) << 16);
+      for (int i = 0; i < 4; ++i) q[i] = e4m3x2(p[4 * i], p[4 * i + 1]) | (e4m3x2(p[4 * i + 2], p[4 * i + 3]) << 16);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = e4m3x2_nonan(p[4 * i], p[4 * i + 1]) | (e4m3x2_nonan(p[4 * i + 2], p[4 * i + 3]) << 16);
+    }
     const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
     for (int j = 0; j < k; ++j) {
       const int slot = __shfl_sync(kFullMask, my_slot, j);
@@ -201,35 +218,44 @@ __global__ void __launch_bounds__(kWarps * 32)
     f[2 * i] = bf16_lo(w[i]);
     f[2 * i + 1] = bf16_hi(w[i]);
   }
+  // all-finite warps take the encoder without NaN fix-ups (as in the FP8
+  // kernel; the scaling by a finite power of two makes no NaN)
   float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  for (int i = 0; i < 16; ++i) amax = max_abs_nan(amax, f[i]);
+  const bool special = __any_sync(kFullMask, !(amax <= 3.402823466e38f));
+  if (special) {  // warp-uniform: the amax ignores NaN, as the definition does
+    amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  }
   amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, 1));
   int e = amax > 0.0f ? floor_log2_pos(amax) - 8 : -127;
   e = e < -127 ? -127 : (e > 127 ? 127 : e);
-  const float down = __int_as_float((127 - e) << 23);  // 2^-e; e <= 119 for bf16 input
+  // 2^-e, e in [-127, 127]: a finite power of two, so every product keeps a
+  // zero's sign and scales exactly (short of underflow)
+  const float down = __int_as_float((127 - e) << 23);
   uint32_t q[4];
+  {
+    float p[16];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float p[4];
+    for (int i = 0; i < 16; ++i) p[i] = __fmul_rn(f[i], down);
+    if (special) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float v = f[4 * i + u];
-      p[u] = (v == 0.0f) ? v : __fmul_rn(v, down);  // exact scaling by a power of two
+      for (int i = 0; i < 4; ++i) q[i] = e4m3x2(p[4 * i], p[4 * i + 1]) | (e4m3x2(p[4 * i + 2], p[4 * i + 3]) << 16);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        q[i] = e4m3x2_nonan(p[4 * i], p[4 * i + 1]) | (e4m3x2_nonan(p[4 * i + 2], p[4 * i + 3]) << 16);
     }
-    q[i] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
   }
   const uint4 qv = make_uint4(q[0], q[1], q[2], q[3]);
-  // the warp's 16 scale bytes (block i sits in lane 2i)
+  // the warp's 16 scale bytes (block j from lane 2j) as 4 words, word i =
+  // blocks 4i..4i+3 gathered on lane 8i in two shuffles
   const uint32_t my_byte = static_cast<uint32_t>(e + 127);
-  uint32_t sw[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    sw[i] = 0;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) sw[i] |= (__shfl_sync(kFullMask, my_byte, 2 * (4 * i + u)) & 0xffu) << (8 * u);
-  }
-  const bool whole16 = (H % 512) == 0;  // 16-byte aligned, full 16 scale bytes per warp
+  uint32_t word = my_byte | (__shfl_down_sync(kFullMask, my_byte, 2) << 8);
+  word |= __shfl_down_sync(kFullMask, word, 4) << 16;
+  const bool whole16 = (H % 512) == 0;  // full 16 scale bytes per warp
   for (int j = 0; j < k; ++j) {
     const int slot = __shfl_sync(kFullMask, my_slot, j);
     if (slot == -1) continue;
@@ -240,19 +266,17 @@ __global__ void __launch_bounds__(kWarps * 32)
     if (active) st_stream_v4(recv_x + static_cast<size_t>(slot) * H + c0, qv);
     if constexpr (SL == MOE_SCALE_ROW_MAJOR) {
       uint8_t* srow = recv_e8m0 + static_cast<size_t>(slot) * nblk;
-      if (whole16) {
-        if (lane == 0) st_v4(srow + s * 16, make_uint4(sw[0], sw[1], sw[2], sw[3]));
+      if (whole16) {  // nblk % 16 == 0: the 4 words are 4-byte aligned
+        if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(srow + s * 16 + (lane >> 1)) = word;
       } else if (active && (lane & 1) == 0) {
         srow[c0 >> 5] = static_cast<uint8_t>(my_byte);
       }
     } else if constexpr (SL == MOE_SCALE_MMA_TILED) {
       // blocks 4i..4i+3 are 4 consecutive bytes of one atom (nblk % 4 == 0):
-      // lane i < 4 stores word i of the warp's 16 blocks
-      const int b0 = s * 16 + 4 * lane;
-      if (lane < 4 && b0 < nblk) {
-        const uint32_t word = lane == 0 ? sw[0] : lane == 1 ? sw[1] : lane == 2 ? sw[2] : sw[3];
+      // lane 8i stores word i of the warp's 16 blocks
+      const int b0 = s * 16 + (lane >> 1);
+      if ((lane & 7) == 0 && b0 < nblk)
         st_keep_b32(recv_e8m0 + scale_at<SL>(slot, b0, nblk, ld), word, l2_evict_last_policy());
-      }
     } else {
       if (active && (lane & 1) == 0)
         st_keep_b8(recv_e8m0 + scale_at<SL>(slot, c0 >> 5, nblk, ld), my_byte, l2_evict_last_policy());
@@ -312,22 +336,41 @@ __global__ void __launch_bounds__(kTokenThreads)
   if (!copy_ok) return;
   mbar_wait(bar, 0);  // the phase has completed: returns at once (and is bounded regardless)
 
-  float amax = 0.0f;
+  // the row amax with NaN propagation; a row whose values are all finite
+  // (the usual case) takes the encoder without NaN fix-ups
+  auto row_amax = [&](bool nan_max) {
+    float m = 0.0f;
 #pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int vi = i * kTokenThreads + tid;
-    if (vi < nvec) {
-      const uint4 v = ld_shared_v4(row + vi * 16);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = i * kTokenThreads + tid;
+      if (vi < nvec) {
+        const uint4 v = ld_shared_v4(row + vi * 16);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w4[u])), fabsf(bf16_hi(w4[u]))));
+        for (int u = 0; u < 4; ++u) {
+          if (nan_max) {
+            m = max_abs_nan(max_abs_nan(m, bf16_lo(w4[u])), bf16_hi(w4[u]));
+          } else {
+            m = fmaxf(m, fmaxf(fabsf(bf16_lo(w4[u])), fabsf(bf16_hi(w4[u]))));
+          }
+        }
+      }
     }
-  }
+    return m;
+  };
+  float amax = row_amax(true);
+  const bool special = !(amax <= 3.402823466e38f);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
   if (lane == 0) warp_max[warp] = amax;
-  __syncthreads();
+  const bool any_special = __syncthreads_or(special);
+  if (any_special) {  // CTA-uniform: the amax ignores NaN, as the definition does
+    amax = row_amax(false);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
+    if (lane == 0) warp_max[warp] = amax;  // nobody has read the first values yet
+    __syncthreads();
+  }
   amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
   const float inv = __fdiv_rn(448.0f, amax);
   const float scale = __fdiv_rn(amax, 448.0f);
@@ -341,14 +384,27 @@ __global__ void __launch_bounds__(kTokenThreads)
       const uint4 v = ld_shared_v4(row + vi * 16);
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
       float p[8];
+      if (finite) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float lo = bf16_lo(w4[u]), hi = bf16_hi(w4[u]);
-        p[2 * u] = (finite || lo != 0.0f) ? __fmul_rn(lo, inv) : lo;
-        p[2 * u + 1] = (finite || hi != 0.0f) ? __fmul_rn(hi, inv) : hi;
+        for (int u = 0; u < 4; ++u) {
+          p[2 * u] = __fmul_rn(bf16_lo(w4[u]), inv);
+          p[2 * u + 1] = __fmul_rn(bf16_hi(w4[u]), inv);
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float lo = bf16_lo(w4[u]), hi = bf16_hi(w4[u]);
+          p[2 * u] = lo != 0.0f ? __fmul_rn(lo, inv) : lo;
+          p[2 * u + 1] = hi != 0.0f ? __fmul_rn(hi, inv) : hi;
+        }
       }
-      q[i].x = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
-      q[i].y = e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16);
+      if (any_special) {
+        q[i].x = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+        q[i].y = e4m3x2(p[4], p[5]) | (e4m3x2(p[6], p[7]) << 16);
+      } else {
+        q[i].x = e4m3x2_nonan(p[0], p[1]) | (e4m3x2_nonan(p[2], p[3]) << 16);
+        q[i].y = e4m3x2_nonan(p[4], p[5]) | (e4m3x2_nonan(p[6], p[7]) << 16);
+      }
     }
   }
   for (int j = 0; j < k; ++j) {

@@ -595,9 +595,13 @@ static int oracle_dispatch_variant(const uint16_t* x, int N, int H, int k,
                 int e = -127;
                 if (amax > 0.0f) {
                     float qt = amax / 448.0f;
-                    int fe;
-                    double fr = frexp((double)qt, &fe);     /* qt = fr * 2^fe, fr in [0.5, 1) */
-                    e = (fr == 0.5) ? fe - 1 : fe;
+                    if (isinf(qt)) {
+                        e = 127;   /* ceil(log2(+inf)) is +inf: clamped to the largest exponent */
+                    } else {
+                        int fe;
+                        double fr = frexp((double)qt, &fe);     /* qt = fr * 2^fe, fr in [0.5, 1) */
+                        e = (fr == 0.5) ? fe - 1 : fe;
+                    }
                 }
                 if (e < -127) e = -127;
                 if (e > 127) e = 127;

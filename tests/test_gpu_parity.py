@@ -152,9 +152,17 @@ def test_bad_slots_in_dispatch_and_combine():
     assert np.array_equal(bf16_bits(out), ref_out)
 
 
+def _same_codes(got, ref):
+    """e4m3 codes equal, NaN codes (0x7f / 0xff) by class: the sign of a NaN
+    made by inf * 0 is the host's or the GPU's default, not the definition's."""
+    nan = lambda c: (c & 0x7F) == 0x7F
+    return bool(np.all((got == ref) | (nan(got) & nan(ref))))
+
+
 def test_fp8_special_blocks():
     """All-zero, negative-zero, tiny-amax (448/amax overflows fp32), subnormal,
-    near-max and mixed-magnitude blocks."""
+    near-max and mixed-magnitude blocks; blocks holding an infinity or a NaN
+    (the kernels' path with NaN fix-ups)."""
     from combine_moe_topk_gate_b200 import api
     H = 128 * 8
     rows = []
@@ -168,14 +176,21 @@ def test_fp8_special_blocks():
     mx = np.full(H, 3.38e38, np.float32); mx[1::2] *= -1; rows.append(mx)
     mixed = r.normal(size=H).astype(np.float32) * np.exp2(r.integers(-30, 30, H)).astype(np.float32); rows.append(mixed)
     ties = np.tile(np.array([448, 1, 0.5, 0.25, 3.0 / 64, 13.0 / 1024], np.float32), H // 6 + 1)[:H]; rows.append(ties)
+    for special in (np.inf, -np.inf, np.nan):
+        row = r.normal(size=H).astype(np.float32)
+        row[5] = special                    # one block with it, the others finite
+        rows.append(row)
+    row = r.normal(size=H).astype(np.float32); row[128:256] = np.nan; rows.append(row)   # an all-NaN block
     xf = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
     N, k = xf.shape[0], 3
     slots = np.arange(N * k, dtype=np.int32).reshape(N, k)
-    recv, scale = api.moe_dispatch(xf.cuda(), torch.from_numpy(slots).cuda(), api.MOE_DTYPE_FP8_E4M3)
-    torch.cuda.synchronize()
-    ref_recv, ref_scale, _ = O.dispatch(bf16_bits(xf), slots, O.DT_FP8_E4M3)
-    assert np.array_equal(recv.cpu().numpy(), ref_recv)
-    assert np.array_equal(scale.cpu().numpy().view(np.uint32), ref_scale.view(np.uint32))
+    for dt in (O.DT_FP8_E4M3, O.DT_FP8_UE8M0):
+        recv, scale = api.moe_dispatch(xf.cuda(), torch.from_numpy(slots).cuda(), dt)
+        torch.cuda.synchronize()
+        ref_recv, ref_scale, _ = O.dispatch(bf16_bits(xf), slots, dt)
+        assert _same_codes(recv.cpu().numpy(), ref_recv)
+        assert np.array_equal(np.ascontiguousarray(scale.cpu().numpy()).view(np.uint8).reshape(-1),
+                              np.ascontiguousarray(ref_scale).view(np.uint8).reshape(-1))
 
 
 def test_gate_ties_and_equal_logits():

@@ -1080,6 +1080,30 @@ def test_ue8m0_is_smallest_power_of_two_not_below_quotient():
     assert np.array_equal(recv, O.e4m3_encode_array(scaled))
 
 
+def test_ue8m0_block_with_an_infinity():
+    """A block whose amax is infinite: ceil(log2(inf / 448)) is +inf, clamped to
+    127 like any exponent beyond the byte (scale byte 254); the factor 2^-127
+    takes every finite value of the block to a zero of its sign and the
+    infinities to +-448; the other blocks of the row are untouched by it."""
+    H = 256
+    x = np.zeros((1, H), np.float32)
+    x[0, :128] = np.linspace(-3.0, 3.0, 128)
+    x[0, 5], x[0, 9] = np.inf, -np.inf
+    x[0, 128:] = np.linspace(-1.0, 1.0, 128)
+    xb = _bf16(x)
+    recv, sc, st = O.dispatch(xb, np.zeros((1, 1), np.int32), O.DT_FP8_UE8M0)
+    assert st == 0
+    assert sc[0, 0] == 254
+    codes = recv[0, :128]
+    assert codes[5] == 0x7E and codes[9] == 0xFE                     # +-448
+    finite = np.ones(128, bool); finite[[5, 9]] = False
+    sign = np.signbit(x[0, :128]).astype(np.uint8) << 7
+    assert np.array_equal(codes[finite], sign[finite])                # zeros keep their sign
+    q = (np.float32(1.0) / np.float32(448)).astype(np.float32)
+    e = int(np.ceil(np.log2(np.float64(np.float32(1.0) * q))))        # amax 1.0: the second block as usual
+    assert sc[0, 1] == e + 127
+
+
 def test_pack4_layout_is_word_transpose():
     rng = np.random.default_rng(5)
     N, k, H = 33, 2, 768                                  # 6 blocks: two words, the second half full
