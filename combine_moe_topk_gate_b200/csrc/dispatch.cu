@@ -575,6 +575,30 @@ __device__ __forceinline__ uint32_t e5m6_code(float f) {
   return sign | (__float_as_uint(t) - 0x4B400000u);
 }
 
+// The same codes for two bf16 values at once (w: low half first) when both
+// magnitudes lie in [2^-14, 65024], the range where the code is the bf16
+// exponent rebiased (127 -> 15) with the 7-bit fraction rounded to 6 bits
+// (ties to even) and no saturation: on the 16-bit halves, r = |h| - (112 << 7)
+// and the code is (r + bit 1 of r) >> 1.  No half carries into the other.
+// Returns the 24-bit pair (low value's code in bits 0..11).
+__device__ __forceinline__ uint32_t e5m6_pair_normal(uint32_t w) {
+  const uint32_t r = (w & 0x7fff7fffu) - 0x38003800u;
+  const uint32_t c = (r + ((r >> 1) & 0x00010001u)) >> 1;
+  const uint32_t lo = (c & 0x7ffu) | ((w >> 4) & 0x800u);
+  const uint32_t hi = ((c >> 16) & 0x7ffu) | ((w >> 20) & 0x800u);
+  return lo | (hi << 12);
+}
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // E5M6 dispatch: lane owns 16 channels (two 16-byte loads) -> 16 codes ->
 // 24 bytes (two codes per 3 bytes, little endian).  The warp's 768 bytes are
 // staged in shared memory and leave as 16-byte streaming stores covering 512
@@ -615,8 +639,22 @@ __global__ void __launch_bounds__(kWarps * 32)
   const uint4 a = av[u], b = bv[u];
   const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
   uint32_t p[8];  // 24-bit pairs
+  // the lane's 16 magnitudes all in [2^-14, 65024] (no zero, subnormal,
+  // saturating value, infinity or NaN): the two-at-a-time codes
+  uint32_t hmax = 0u, hmin = 0xffffffffu;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = e5m6_code(bf16_lo(w[i])) | (e5m6_code(bf16_hi(w[i])) << 12);
+  for (int i = 0; i < 8; ++i) {
+    hmax = max_u16x2(hmax, w[i] & 0x7fff7fffu);
+    hmin = min_u16x2(hmin, w[i] & 0x7fff7fffu);
+  }
+  const uint32_t top = max(hmax & 0xffffu, hmax >> 16), bottom = min(hmin & 0xffffu, hmin >> 16);
+  if (top <= 0x477Eu && bottom >= 0x3880u) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = e5m6_pair_normal(w[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) p[i] = e5m6_code(bf16_lo(w[i])) | (e5m6_code(bf16_hi(w[i])) << 12);
+  }
   if (u > 0) __syncwarp();  // every lane has read the previous segment's stage
   stage[warp][3 * lane] = make_uint2(p[0] | (p[1] << 24), (p[1] >> 8) | (p[2] << 16));
   stage[warp][3 * lane + 1] = make_uint2((p[2] >> 16) | (p[3] << 8), p[4] | (p[5] << 24));
