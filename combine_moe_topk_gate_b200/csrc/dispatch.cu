@@ -420,26 +420,28 @@ __global__ void __launch_bounds__(kTokenThreads)
   }
 }
 
-// NVFP4: one 128-thread CTA per token.  One thread copies the token's row
-// into shared memory with a 1-D bulk copy (no tensor map, no multicast) that
-// completes on an mbarrier; the CTA then works from shared memory, so the row
-// does not occupy registers and about 15 tokens fit per SM.  Each thread owns
-// the 16-channel blocks tid, tid + 128, ... (BPT of them): block maxima, the
+// NVFP4: one CTA of THREADS threads per token (128, or 64 for rows of up to
+// 4096 channels).  One thread copies the token's row into shared memory with
+// a 1-D bulk copy (no tensor map, no multicast) that completes on an
+// mbarrier; the CTA then works from shared memory, so the row does not
+// occupy registers and many tokens are in flight per SM.  Each thread owns
+// the 16-channel blocks tid, tid + THREADS, ... (BPT of them): block maxima, the
 // CTA-wide row amax (row scale g = amax / 2688, inv = 2688 / amax), then per
 // block sb = e4m3((amax_b / 6) * inv), r = inv / value(sb), codes e2m1(x * r).
 // Four neighbouring threads hold four consecutive blocks, so their scale
 // bytes leave as one 32-bit word (H % 64 == 0).  The copy's wait is bounded
 // (MOE_ERR_TIMEOUT).
 constexpr int kNvThreads = 128;
+constexpr int kNvThreadsShort = 64;  // rows of up to 4096 channels
 
-template <int BPT, int SL>
-__global__ void __launch_bounds__(kNvThreads)
+template <int BPT, int SL, int THREADS>
+__global__ void __launch_bounds__(THREADS)
     dispatch_nvfp4_kernel(const uint16_t* __restrict__ x, int N, int H, int k,
                           const int32_t* __restrict__ token_slot, long long S,
                           uint8_t* __restrict__ recv_x, uint8_t* __restrict__ block_scale,
                           float* __restrict__ row_scale, long long ld, int32_t* d_status) {
   extern __shared__ __align__(128) unsigned char smem[];  // mbarrier at 0, the row from 128
-  __shared__ float warp_max[kNvThreads / 32];
+  __shared__ float warp_max[THREADS / 32];
   __shared__ int slots[MOE_MAX_TOPK];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t = blockIdx.x;
@@ -482,7 +484,7 @@ __global__ void __launch_bounds__(kNvThreads)
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < BPT; ++i) {
-    const int b = tid + i * kNvThreads;
+    const int b = tid + i * THREADS;
     bmax[i] = 0.0f;
     if (b < nb) {
       const uint4 va = ld_shared_v4(row + b * 32), vb = ld_shared_v4(row + b * 32 + 16);
@@ -496,14 +498,16 @@ __global__ void __launch_bounds__(kNvThreads)
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(kFullMask, amax, o));
   if (lane == 0) warp_max[warp] = amax;
   __syncthreads();
-  amax = fmaxf(fmaxf(warp_max[0], warp_max[1]), fmaxf(warp_max[2], warp_max[3]));
+  amax = warp_max[0];
+#pragma unroll
+  for (int w = 1; w < THREADS / 32; ++w) amax = fmaxf(amax, warp_max[w]);
   const float g = __fdiv_rn(amax, 2688.0f);
   const float inv = __fdiv_rn(2688.0f, amax);
   uint2 q[BPT];
   uint32_t sword[BPT];
 #pragma unroll
   for (int i = 0; i < BPT; ++i) {
-    const int b = tid + i * kNvThreads;
+    const int b = tid + i * THREADS;
     const float sbf = __fmul_rn(__fdiv_rn(bmax[i], 6.0f), inv);
     const uint32_t sb = bmax[i] > 0.0f ? (e4m3x2(sbf, 0.0f) & 0xffu) : 0u;
     q[i] = make_uint2(0, 0);
@@ -542,7 +546,7 @@ __global__ void __launch_bounds__(kNvThreads)
     uint8_t* dst = recv_x + static_cast<size_t>(slot) * row_bytes;
 #pragma unroll
     for (int i = 0; i < BPT; ++i) {
-      const int b = tid + i * kNvThreads;
+      const int b = tid + i * THREADS;
       if (b < nb) {
         *reinterpret_cast<uint2*>(dst + static_cast<size_t>(b) * 8) = q[i];
         if constexpr (SL == MOE_SCALE_MN_MAJOR) {
@@ -859,14 +863,14 @@ cudaError_t launch_dispatch(const void* x, int N, int H, int k, const int32_t* t
   }
 }
 
-template <int BPT, int SL>
+template <int BPT, int SL, int THREADS>
 cudaError_t launch_nvfp4_bpt(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                              long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
                              float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
   const size_t smem = 128 + static_cast<size_t>(H) * 2;  // H <= 16384: at most 32 KB + 128
-  cudaError_t err = prefer_shared(dispatch_nvfp4_kernel<BPT, SL>);
+  cudaError_t err = prefer_shared(dispatch_nvfp4_kernel<BPT, SL, THREADS>);
   if (err != cudaSuccess) return err;
-  return launch_pdl(dispatch_nvfp4_kernel<BPT, SL>, N, kNvThreads, smem, stream, x, N, H, k,
+  return launch_pdl(dispatch_nvfp4_kernel<BPT, SL, THREADS>, N, THREADS, smem, stream, x, N, H, k,
                     token_slot, num_rows, recv_x, block_scale, row_scale, ld, d_status);
 }
 
@@ -874,18 +878,25 @@ template <int SL>
 cudaError_t launch_nvfp4(const uint16_t* x, int N, int H, int k, const int32_t* token_slot,
                          long long num_rows, uint8_t* recv_x, uint8_t* block_scale,
                          float* row_scale, long long ld, int32_t* d_status, cudaStream_t stream) {
+  // rows of up to 4096 channels: 64-thread CTAs, so twice as many tokens'
+  // rows are in flight per SM (a short row is little work for a CTA)
+  if (H <= 4096) {
+    const int bpt = (H / 16 + kNvThreadsShort - 1) / kNvThreadsShort;  // <= 4
+    if (bpt <= 1)
+      return launch_nvfp4_bpt<1, SL, kNvThreadsShort>(x, N, H, k, token_slot, num_rows, recv_x, block_scale,
+                                                      row_scale, ld, d_status, stream);
+    if (bpt <= 2)
+      return launch_nvfp4_bpt<2, SL, kNvThreadsShort>(x, N, H, k, token_slot, num_rows, recv_x, block_scale,
+                                                      row_scale, ld, d_status, stream);
+    return launch_nvfp4_bpt<4, SL, kNvThreadsShort>(x, N, H, k, token_slot, num_rows, recv_x, block_scale,
+                                                    row_scale, ld, d_status, stream);
+  }
   const int bpt = (H / 16 + kNvThreads - 1) / kNvThreads;  // blocks per thread, <= 8
-  if (bpt <= 1)
-    return launch_nvfp4_bpt<1, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
-                                   d_status, stream);
-  if (bpt <= 2)
-    return launch_nvfp4_bpt<2, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
-                                   d_status, stream);
   if (bpt <= 4)
-    return launch_nvfp4_bpt<4, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
-                                   d_status, stream);
-  return launch_nvfp4_bpt<8, SL>(x, N, H, k, token_slot, num_rows, recv_x, block_scale, row_scale, ld,
-                                 d_status, stream);
+    return launch_nvfp4_bpt<4, SL, kNvThreads>(x, N, H, k, token_slot, num_rows, recv_x, block_scale,
+                                               row_scale, ld, d_status, stream);
+  return launch_nvfp4_bpt<8, SL, kNvThreads>(x, N, H, k, token_slot, num_rows, recv_x, block_scale,
+                                             row_scale, ld, d_status, stream);
 }
 
 cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int32_t* token_slot,
