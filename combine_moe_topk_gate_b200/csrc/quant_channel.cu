@@ -28,6 +28,13 @@
 // through distributed shared memory between two hardware cluster barriers,
 // and each CTA writes the codes of its own rows.  A max is exact in any
 // order, so every Q gives the same bits.
+//
+// With a caller's workspace and experts of a few hundred rows on average
+// (where one CTA per (expert, slab) leaves a hot expert's lone CTAs on the
+// critical path), a persistent grid takes (expert, slab, part) tasks from a
+// counter instead: each expert is cut into parts of at most kPartRows rows,
+// and the parts of one (expert, slab) combine their amax through the
+// workspace (see quant_fp8_channel_queue_kernel).
 #include <algorithm>
 
 #include "moe_device.cuh"
