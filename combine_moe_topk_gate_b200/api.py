@@ -80,6 +80,8 @@ def _load() -> ctypes.CDLL:
     L.moe_quant_fp8_channel.argtypes = [P, I, I, I, P, P, I, P, P, P, SZ, P, P]
     L.moe_quant_fp8_channel_workspace_bytes.argtypes = [I, I]
     L.moe_quant_fp8_channel_workspace_bytes.restype = SZ
+    L.moe_quant_fp8_channel_takes_workspace.argtypes = [I, I]
+    L.moe_quant_fp8_channel_takes_workspace.restype = I
     L.moe_quant_fp8_channel.restype = I
     L.moe_swiglu_quant.argtypes = [P, I, I, P, I, I, P, P, P]
     L.moe_swiglu_quant.restype = I
@@ -484,6 +486,10 @@ def moe_quant_fp8_channel_workspace_bytes(num_experts: int, hidden: int) -> int:
     return int(_lib.moe_quant_fp8_channel_workspace_bytes(num_experts, hidden))
 
 
+def moe_quant_fp8_channel_takes_workspace(num_rows: int, num_experts: int) -> bool:
+    return bool(_lib.moe_quant_fp8_channel_takes_workspace(num_rows, num_experts))
+
+
 def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, expert_count: torch.Tensor, *,
                           transpose: bool = False, out=None, scale=None, workspace="new", d_status=None,
                           stream=None):
@@ -492,8 +498,9 @@ def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, exper
     fp32 [E, H])``.  ``workspace``: a uint8 device tensor of
     ``moe_quant_fp8_channel_workspace_bytes(E, H)`` bytes, zero before its
     first use and left zero by every call (keep one per stream); ``"new"``
-    (default) allocates a zeroed one for this call; None takes the path
-    without scratch."""
+    (default) allocates a zeroed one for this call when the call uses one
+    (``moe_quant_fp8_channel_takes_workspace``); None takes the path without
+    scratch."""
     _need(recv, "recv", torch.bfloat16)
     S, H = recv.shape
     _need(expert_count, "expert_count", torch.int32)
@@ -510,9 +517,12 @@ def moe_quant_fp8_channel(recv: torch.Tensor, expert_offset: torch.Tensor, exper
     if isinstance(workspace, str):
         if workspace != "new":
             raise ValueError(f"workspace must be a tensor, None or 'new', not {workspace!r}")
-        # zeroed in the order of the stream the kernel runs on
-        with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream(recv.device)):
-            workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=recv.device)
+        if moe_quant_fp8_channel_takes_workspace(S, E):
+            # zeroed in the order of the stream the kernel runs on
+            with torch.cuda.stream(stream if stream is not None else torch.cuda.current_stream(recv.device)):
+                workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=recv.device)
+        else:
+            workspace = None
     if workspace is not None:
         _need(workspace, "workspace", torch.uint8)
         if workspace.numel() < ws_bytes:

@@ -23,7 +23,7 @@ cudaStream_t as_stream(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
 
 extern "C" {
 
-int moe_abi_version(void) { return 7; }
+int moe_abi_version(void) { return 8; }
 
 const char* moe_status_string(moe_status_t s) {
   switch (s) {
@@ -235,6 +235,11 @@ moe_status_t moe_selftest_bounded_wait(int32_t* d_status, moe_stream_t stream) {
 size_t moe_quant_fp8_channel_workspace_bytes(int num_experts, int hidden) {
   if (num_experts < 1 || num_experts > MOE_MAX_EXPERTS || hidden < 128 || hidden % 128 != 0) return 0;
   return moe::quant_fp8_channel_workspace_bytes(num_experts, hidden);
+}
+
+int moe_quant_fp8_channel_takes_workspace(int num_rows, int num_experts) {
+  if (num_rows < 0 || num_experts < 1 || num_experts > MOE_MAX_EXPERTS) return 0;
+  return moe::quant_fp8_channel_takes_workspace(num_rows, num_experts) ? 1 : 0;
 }
 
 moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, int num_experts,

@@ -59,6 +59,7 @@ cudaError_t launch_dispatch_nvfp4(const void* x, int N, int H, int k, const int3
                                   void* block_scale, float* row_scale, int32_t* d_status,
                                   cudaStream_t stream);
 size_t quant_fp8_channel_workspace_bytes(int E, int H);
+bool quant_fp8_channel_takes_workspace(long long num_rows, int E);
 cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, int E,
                                      const int32_t* expert_offset, const int32_t* expert_count,
                                      bool transpose, void* out, float* scale, int32_t* d_status,

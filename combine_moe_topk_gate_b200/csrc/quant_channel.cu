@@ -466,6 +466,19 @@ cudaError_t launch_channel_sw(int lsw, bool cluster, int Q, const uint16_t* xs, 
 
 }  // namespace
 
+// The task queue (workspace) where the cluster path would give every
+// (expert, slab) one CTA although the average expert already fills a part:
+// there a hot expert's lone CTAs are the critical path (Zipf-skewed shape:
+// 297 against 369 us).  Below that the hardware's own scheduling of the
+// small (expert, slab) CTAs is faster than the persistent loop (prefill
+// shape: 128 against 144 us; decode: 27 against 41 us), and from 1024 rows
+// on the clusters already spread every expert (Mixtral shape: 103 against
+// 108 us).
+bool quant_fp8_channel_takes_workspace(long long num_rows, int E) {
+  const long long avg_rows = E > 0 ? num_rows / E : 0;
+  return avg_rows >= kPartRows && avg_rows < 1024;
+}
+
 size_t quant_fp8_channel_workspace_bytes(int E, int H) {
   return 4 * static_cast<size_t>(ws_amax_base(E, H) + static_cast<long long>(E) * H);
 }
@@ -477,15 +490,7 @@ cudaError_t launch_quant_fp8_channel(const void* x, long long num_rows, int H, i
   const uint16_t* xs = static_cast<const uint16_t*>(x);
   uint8_t* o = static_cast<uint8_t*>(out);
   const long long avg_rows = E > 0 ? num_rows / E : 0;
-  // The task queue (workspace) where the cluster path would give every
-  // (expert, slab) one CTA although the average expert already fills a part:
-  // there a hot expert's lone CTAs are the critical path (Zipf-skewed shape:
-  // 297 against 369 us).  Below that the hardware's own scheduling of the
-  // small (expert, slab) CTAs is faster than the persistent loop (prefill
-  // shape: 128 against 144 us; decode: 27 against 41 us), and from 1024 rows
-  // on the clusters already spread every expert (Mixtral shape: 103 against
-  // 108 us).
-  uint32_t* ws = (avg_rows >= kPartRows && avg_rows < 1024) ? static_cast<uint32_t*>(workspace) : nullptr;
+  uint32_t* ws = quant_fp8_channel_takes_workspace(num_rows, E) ? static_cast<uint32_t*>(workspace) : nullptr;
   // Without it: CTAs per (expert, slab) from the average rows, about 512 rows
   // each, at most 8 (the portable cluster size); 1 keeps the plain launch.
   const int Q = ws ? 1 : avg_rows >= 4096 ? 8 : avg_rows >= 2048 ? 4 : avg_rows >= 1024 ? 2 : 1;

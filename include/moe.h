@@ -434,6 +434,12 @@ moe_status_t moe_quant_fp8_channel(const void* recv, int num_rows, int hidden, i
  * (0 when E or H is outside that call's limits). */
 size_t moe_quant_fp8_channel_workspace_bytes(int num_experts, int hidden);
 
+/* 1 when moe_quant_fp8_channel over num_rows receive rows and E experts
+ * uses a workspace it is given (the average expert holds 256 to 1023 rows),
+ * 0 when it ignores it (or the sizes are outside its limits): a caller may
+ * then pass NULL and allocate nothing. */
+int moe_quant_fp8_channel_takes_workspace(int num_rows, int num_experts);
+
 /*
  * moe_swiglu_quant -- SwiGLU between an expert's two GEMMs, fused with the
  * quantisation the second GEMM reads.  [TK] list: SwiGLU combined with the

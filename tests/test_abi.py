@@ -251,6 +251,13 @@ def test_quant_fp8_channel_rejects_bad_arguments(api):
     # header, two counters per (expert, 128-channel slab), one amax per (expert, channel)
     assert need == 4 * (64 + 2 * 4 * 2 + 4 * 256)
     assert api.moe_quant_fp8_channel_workspace_bytes(0, 256) == 0
+    # used where the average expert holds 256 to 1023 rows
+    assert api.moe_quant_fp8_channel_takes_workspace(78336, 256)          # Zipf-skewed, aligned
+    assert not api.moe_quant_fp8_channel_takes_workspace(48640, 256)      # prefill, aligned
+    assert not api.moe_quant_fp8_channel_takes_workspace(33280, 8)        # Mixtral shape: clusters
+    assert api.moe_quant_fp8_channel_takes_workspace(2048, 8) and not api.moe_quant_fp8_channel_takes_workspace(2047, 8)
+    assert not api.moe_quant_fp8_channel_takes_workspace(8192, 8) and api.moe_quant_fp8_channel_takes_workspace(8191, 8)
+    assert not api.moe_quant_fp8_channel_takes_workspace(-1, 8) and not api.moe_quant_fp8_channel_takes_workspace(100, 0)
     assert api.moe_quant_fp8_channel_workspace_bytes(4, 192) == 0
     assert call(ws=_P(), wsb=need - 4) == api.MOE_ERR_INVALID_ARG   # short workspace
     assert call(ws=_P(0x1008), wsb=need) == api.MOE_ERR_INVALID_ARG  # not 16-byte aligned
