@@ -79,6 +79,7 @@ MUTANTS = {
                                     "if (transpose) out[(size_t)c * H + s] = q;"),
     "ue8m0_floor_instead_of_ceil": ("e = (fr == 0.5) ? fe - 1 : fe;", "e = fe - 1;"),
     "ue8m0_ceil_misses_powers_of_two": ("e = (fr == 0.5) ? fe - 1 : fe;", "e = fe;"),
+    "ue8m0_infinite_quotient_exponent_zero": ("e = 127;   /* ceil(log2(+inf)) is +inf", "e = 0;   /* ceil(log2(+inf)) is +inf"),
     "pack4_words_row_major": ("return (int64_t)(b / 4) * 4 * round_up64(num_rows, 4) + s * 4 + b % 4;",
                               "return s * 4 * (int64_t)((B + 3) / 4) + (int64_t)(b / 4) * 4 + b % 4;"),
     "combine_no_zero_skip_for_masked": ("if (s == -1) continue;\n                if (s < -1 || s >= S) { status = ORC_ERR_BAD_INDEX; continue; }\n                float v",
